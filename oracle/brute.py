@@ -1,0 +1,158 @@
+"""ORACLE -- test infrastructure only.
+
+Brute force in pure Python (sets, dicts, exact rationals) for inputs of a few
+dozen tokens.  It restates the same definitions as oracle.c in a different
+form -- token sets per expert instead of pair loops, a dict of rows per rank
+instead of a sorted row array -- so that the two pin each other.
+"""
+from __future__ import annotations
+
+import math
+import struct
+from fractions import Fraction
+
+
+def token_sets(ids_l, E):
+    """A_e = set of tokens that selected expert e (the Ochiai operands on the
+    Cobalt page, "Key Observation")."""
+    A = [set() for _ in range(E)]
+    for t, d in enumerate(ids_l):
+        for e in d:
+            A[int(e)].add(t)
+    return A
+
+
+def coact(ids, E):
+    """C[l][i][j] = |A_i & A_j| at layer l."""
+    out = []
+    for ids_l in ids:
+        A = token_sets(ids_l, E)
+        out.append([[len(A[i] & A[j]) for j in range(E)] for i in range(E)])
+    return out
+
+
+def f32(x: float) -> float:
+    return struct.unpack("<f", struct.pack("<f", x))[0]
+
+
+def ochiai(ids, E):
+    """|A & B| / sqrt(|A| |B|), 0 for an empty operand; fp64 then fp32."""
+    out = []
+    for ids_l in ids:
+        A = token_sets(ids_l, E)
+        S = []
+        for i in range(E):
+            row = []
+            for j in range(E):
+                den = len(A[i]) * len(A[j])
+                row.append(f32(len(A[i] & A[j]) / math.sqrt(den)) if den else 0.0)
+            S.append(row)
+        out.append(S)
+    return out
+
+
+def trans(ids, E):
+    """M[l][i][j] = |A_i^l & A_j^{l+1}|."""
+    out = []
+    for l in range(len(ids) - 1):
+        A = token_sets(ids[l], E)
+        B = token_sets(ids[l + 1], E)
+        out.append([[len(A[i] & B[j]) for j in range(E)] for i in range(E)])
+    return out
+
+
+def plan(ids_l, E, G, rpn, e2r, src_rank=None):
+    """Rows per destination rank, each rank's list ordered by (source, token)."""
+    T = len(ids_l)
+    src = [int(src_rank[t]) if src_rank is not None else t // (T // G) for t in range(T)]
+    per_dst = {r: [] for r in range(G)}
+    dest = []
+    for t, d in enumerate(ids_l):
+        ranks = {int(e2r[int(e)]) for e in d}
+        dest.append(ranks)
+        for r in ranks:
+            per_dst[r].append((src[t], t))
+    rows = []
+    for r in range(G):
+        for s, t in sorted(per_dst[r]):
+            rows.append((r, s, t))
+    where = {(t, r): i for i, (r, s, t) in enumerate(rows)}
+    row_of = [[where[(t, int(e2r[int(e)]))] for e in d] for t, d in enumerate(ids_l)]
+    row_jmask = [sum(1 << j for j, e in enumerate(ids_l[t]) if int(e2r[int(e)]) == r) for (r, s, t) in rows]
+    counts = [[0] * G for _ in range(G)]
+    for r, s, t in rows:
+        counts[s][r] += 1
+    offsets = []
+    run = 0
+    for r in range(G):
+        for s in range(G):
+            offsets.append(run)
+            run += counts[s][r]
+    offsets.append(run)
+    local = sum(1 for t, d in enumerate(ids_l) for e in d if int(e2r[int(e)]) == src[t])
+    V = sum(len({int(e2r[int(e)]) // rpn for e in d} - {src[t] // rpn}) for t, d in enumerate(ids_l))
+    remote = sum(1 for (r, s, t) in rows if r != s)
+    return dict(row_token=[t for (r, s, t) in rows], row_jmask=row_jmask, row_of=row_of,
+                counts=counts, offsets=offsets, dest=dest,
+                R=len(rows), R_remote=remote, local=local, V=V)
+
+
+def combine_exact(Y, idx, w):
+    """Exact rational sum_j w[t][j] * Y[idx[t][j]][c] (Y, w given as Python floats)."""
+    out = []
+    for t in range(len(idx)):
+        row = []
+        for c in range(len(Y[0])):
+            acc = Fraction(0)
+            for j in range(len(idx[t])):
+                acc += Fraction(float(w[t][j])) * Fraction(float(Y[idx[t][j]][c]))
+            row.append(acc)
+        out.append(row)
+    return out
+
+
+def shuffle_targets(ids_l, G, rank_score):
+    tg = []
+    for d in ids_l:
+        scores = [sum(int(rank_score[int(e)][r]) for e in d) for r in range(G)]
+        best = max(scores)
+        tg.append(scores.index(best))
+    return tg
+
+
+def place_correlated(C, G, rpn):
+    """Restatement of the greedy grouping with Python lists and Fraction-free
+    fp64 (same summation order as the specification: insertion order)."""
+    E = len(C)
+
+    def s64(i, j):
+        den = float(C[i][i]) * float(C[j][j])
+        return C[i][j] / math.sqrt(den) if den > 0 else 0.0
+
+    def groups(pool, m):
+        size = len(pool) // m
+        left = sorted(pool)
+        res = []
+        for _ in range(m):
+            seed = max(left, key=lambda e: (C[e][e], -e))
+            grp = [seed]
+            left.remove(seed)
+            while len(grp) < size:
+                def score(e):
+                    s = 0.0
+                    for g in grp:
+                        s += s64(e, g)
+                    return s
+                best = max(left, key=lambda e: (score(e), -e))
+                grp.append(best)
+                left.remove(best)
+            res.append(grp)
+        return res
+
+    nodes = G // rpn
+    e2r = [0] * E
+    for q, ng in enumerate(groups(list(range(E)), nodes)):
+        for u, rg in enumerate(groups(ng, rpn)):
+            for e in rg:
+                e2r[e] = q * rpn + u
+    return e2r

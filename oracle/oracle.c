@@ -1,0 +1,414 @@
+/*
+ * ORACLE -- test infrastructure only.
+ *
+ * A plain, slow, single-threaded CPU statement of what the co-activation and
+ * deduplicated-dispatch hot path computes, written from the pages' prose and
+ * formulas.  Its only users are the tests, the smoke check of the build entry
+ * and the CPU-baseline leg of the benchmark.  The product library never loads,
+ * links or calls it, and it shares no code with the product's CUDA sources.
+ *
+ * Pages cited (by title and section):
+ *   [EC]  "Expert Coupling in MoE Pretraining: Reducing All-to-All Overhead
+ *          with Correlated Placement and Token Shuffling", abstract.
+ *   [EPS] "Expert Parallelism > Expert Placement Strategies", the uniform
+ *          placement listing and its printed example; "Capacity-Aware Placement".
+ *   [CB]  "Cobalt: Leveraging Expert Co-activation for Efficient Distributed MoE
+ *          Training", "Key Observation (Expert Co-activation)" (Ochiai formula)
+ *          and "Problem Formulation" (cross-node cost V).
+ *   [CE]  "Training Communication-Efficient Mixture-of-Experts Language Models
+ *          with Layer Re-Configuration", footnote 3 (the dispatcher carries
+ *          hidden states and routed probabilities; combine is the inverse).
+ *
+ * Precision: counts and plans are integers.  Ochiai is fp64 rounded once to
+ * fp32.  The combine is evaluated in fp64 (the pages fix no precision for it).
+ * Compile with -O2 -ffp-contract=off.
+ *
+ * Parity pins for every function live in the CPU tests; the correlated
+ * placement's grouping quality is "parity unpinned" beyond its stated greedy
+ * steps and the planted-cluster case.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_ERR_ARG 1
+#define ORC_ERR_DATA 2
+
+/* A token's D_t is a set of k distinct expert ids in [0, E) ([EC]: "each
+ * token is routed to k of these experts").  Returns 1 when valid. */
+static int token_valid(const int32_t *d, int k, int E)
+{
+    for (int a = 0; a < k; ++a) {
+        if (d[a] < 0 || d[a] >= E) return 0;
+        for (int b = 0; b < a; ++b)
+            if (d[a] == d[b]) return 0;
+    }
+    return 1;
+}
+
+/* Co-activation counts, Ochiai similarity and cross-layer transitions.
+ *
+ * C_l[i][j] = |{t : i in D_t^l and j in D_t^l}|  ([EC]: pairs of experts
+ *   "selected together" by a token; [CB] Problem/Stage 1: the number of tokens
+ *   selecting both experts i and j).  C_l[i][i] = n_i, the expert's load.
+ * S_l[i][j] = |A_i & A_j| / sqrt(|A_i| |A_j|) = C_ij / sqrt(C_ii C_jj)
+ *   ([CB] "Key Observation": Ochiai over the token sets of two experts);
+ *   0 where C_ii C_jj = 0; fp64, then rounded to fp32.
+ * M_l[i][j] = |{t : i in D_t^l and j in D_t^{l+1}}|  ([EC]: the experts a
+ *   token selects at one layer predict those it selects at the next).
+ *
+ * ids int32 [L][T][k]; coact uint32 [L][E][E]; ochiai float [L][E][E];
+ * trans uint32 [L-1][E][E].  Any output may be NULL. */
+int orc_coact(const int32_t *ids, int L, int T, int k, int E,
+              uint32_t *coact, float *ochiai, uint32_t *trans)
+{
+    if (L < 1 || T < 0 || k < 1 || E < 1 || k > E) return ORC_ERR_ARG;
+    for (int l = 0; l < L; ++l)
+        for (int t = 0; t < T; ++t)
+            if (!token_valid(ids + ((size_t)l * T + t) * k, k, E)) return ORC_ERR_DATA;
+
+    const size_t EE = (size_t)E * E;
+    uint32_t *C = NULL;
+    if (coact || ochiai) {
+        C = coact ? coact : (uint32_t *)malloc(sizeof(uint32_t) * EE * L);
+        if (!C) return ORC_ERR_ARG;
+        memset(C, 0, sizeof(uint32_t) * EE * L);
+        for (int l = 0; l < L; ++l) {
+            uint32_t *Cl = C + EE * l;
+            for (int t = 0; t < T; ++t) {
+                const int32_t *d = ids + ((size_t)l * T + t) * k;
+                /* every ordered pair (a, b) of the token's picks, a == b included */
+                for (int a = 0; a < k; ++a)
+                    for (int b = 0; b < k; ++b)
+                        Cl[(size_t)d[a] * E + d[b]] += 1;
+            }
+        }
+    }
+    if (ochiai) {
+        for (int l = 0; l < L; ++l) {
+            const uint32_t *Cl = C + EE * l;
+            for (int i = 0; i < E; ++i)
+                for (int j = 0; j < E; ++j) {
+                    double den = (double)Cl[(size_t)i * E + i] * (double)Cl[(size_t)j * E + j];
+                    double s = 0.0;
+                    if (den > 0.0) s = (double)Cl[(size_t)i * E + j] / sqrt(den);
+                    ochiai[EE * l + (size_t)i * E + j] = (float)s;
+                }
+        }
+    }
+    if (C && C != coact) free(C);
+    if (trans && L > 1) {
+        memset(trans, 0, sizeof(uint32_t) * EE * (L - 1));
+        for (int l = 0; l + 1 < L; ++l) {
+            uint32_t *Ml = trans + EE * l;
+            for (int t = 0; t < T; ++t) {
+                const int32_t *a = ids + ((size_t)l * T + t) * k;
+                const int32_t *b = ids + ((size_t)(l + 1) * T + t) * k;
+                for (int x = 0; x < k; ++x)
+                    for (int y = 0; y < k; ++y)
+                        Ml[(size_t)a[x] * E + b[y]] += 1;
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* Uniform placement ([EPS], uniform listing): device = expert_id // (E/G),
+ * defined only when G divides E. */
+int orc_place_uniform(int E, int G, int32_t *expert_to_rank)
+{
+    if (E < 1 || G < 1 || E % G != 0) return ORC_ERR_ARG;
+    int per = E / G;
+    for (int e = 0; e < E; ++e) expert_to_rank[e] = e / per;
+    return ORC_OK;
+}
+
+/* Capacity-aware placement ([EPS] "Capacity-Aware Placement"): experts in
+ * descending order of load (equal loads: lower id first, a stable sort), each
+ * onto the device with the least load so far (ties: the lowest device index).
+ * Loads are summed in fp64 here. */
+static const double *g_sort_load;
+static int cmp_load_desc(const void *pa, const void *pb)
+{
+    int a = *(const int *)pa, b = *(const int *)pb;
+    if (g_sort_load[a] > g_sort_load[b]) return -1;
+    if (g_sort_load[a] < g_sort_load[b]) return 1;
+    return a < b ? -1 : (a > b);
+}
+
+int orc_place_capacity(const double *load, int E, int G, int32_t *expert_to_rank, double *device_load)
+{
+    if (E < 1 || G < 1) return ORC_ERR_ARG;
+    int *order = (int *)malloc(sizeof(int) * E);
+    if (!order) return ORC_ERR_ARG;
+    for (int e = 0; e < E; ++e) order[e] = e;
+    g_sort_load = load;
+    qsort(order, E, sizeof(int), cmp_load_desc);
+    for (int g = 0; g < G; ++g) device_load[g] = 0.0;
+    for (int i = 0; i < E; ++i) {
+        int e = order[i], best = 0;
+        for (int g = 1; g < G; ++g)
+            if (device_load[g] < device_load[best]) best = g;
+        expert_to_rank[e] = best;
+        device_load[best] += load[e];
+    }
+    free(order);
+    return ORC_OK;
+}
+
+/* Ochiai in fp64 without the fp32 rounding, for the placement greedy. */
+static double ochiai64(const uint32_t *C, int E, int i, int j)
+{
+    double den = (double)C[(size_t)i * E + i] * (double)C[(size_t)j * E + j];
+    if (den > 0.0) return (double)C[(size_t)i * E + j] / sqrt(den);
+    return 0.0;
+}
+
+/* Split the experts listed in pool[0..n) (ascending ids) into m groups of
+ * n/m, one group at a time: seed with the unassigned expert of largest load
+ * C_ee, then repeatedly add the unassigned expert whose summed fp64 Ochiai to
+ * the group's members (summed in insertion order) is largest; ties go to the
+ * lowest expert id.  group_of[pool index] receives the group number. */
+static void greedy_groups(const uint32_t *C, int E, const int *pool, int n, int m, int *group_of)
+{
+    int size = n / m;
+    int *taken = (int *)calloc(n, sizeof(int));
+    int *members = (int *)malloc(sizeof(int) * size);
+    for (int g = 0; g < m; ++g) {
+        int best = -1;
+        for (int x = 0; x < n; ++x) {
+            if (taken[x]) continue;
+            if (best < 0 || C[(size_t)pool[x] * E + pool[x]] > C[(size_t)pool[best] * E + pool[best]])
+                best = x;
+        }
+        taken[best] = 1;
+        group_of[best] = g;
+        members[0] = pool[best];
+        for (int cnt = 1; cnt < size; ++cnt) {
+            int pick = -1;
+            double pick_score = 0.0;
+            for (int x = 0; x < n; ++x) {
+                if (taken[x]) continue;
+                double s = 0.0;
+                for (int q = 0; q < cnt; ++q) s += ochiai64(C, E, pool[x], members[q]);
+                if (pick < 0 || s > pick_score) { pick = x; pick_score = s; }
+            }
+            taken[pick] = 1;
+            group_of[pick] = g;
+            members[cnt] = pool[pick];
+        }
+    }
+    free(members);
+    free(taken);
+}
+
+/* Correlated placement ([EC]: experts often selected together go on the same
+ * GPU).  The pages give the goal, not an algorithm; this is the greedy reading:
+ * with more than one node, first group the experts into G/rpn node groups of
+ * E/(G/rpn), then each node's experts into rpn rank groups of E/G; node group
+ * q and its rank group u map to rank q*rpn + u.  coact is one layer's
+ * uint32 [E][E] count matrix. */
+int orc_place_correlated(const uint32_t *coact, int E, int G, int rpn, int32_t *expert_to_rank)
+{
+    if (E < 1 || G < 1 || rpn < 1 || G % rpn != 0 || E % G != 0) return ORC_ERR_ARG;
+    int nodes = G / rpn;
+    int *all = (int *)malloc(sizeof(int) * E);
+    int *node_of = (int *)malloc(sizeof(int) * E);
+    int *pool = (int *)malloc(sizeof(int) * E);
+    int *grp = (int *)malloc(sizeof(int) * E);
+    for (int e = 0; e < E; ++e) all[e] = e;
+    greedy_groups(coact, E, all, E, nodes, node_of);
+    for (int q = 0; q < nodes; ++q) {
+        int n = 0;
+        for (int e = 0; e < E; ++e)
+            if (node_of[e] == q) pool[n++] = e;
+        greedy_groups(coact, E, pool, n, rpn, grp);
+        for (int x = 0; x < n; ++x) expert_to_rank[pool[x]] = q * rpn + grp[x];
+    }
+    free(all); free(node_of); free(pool); free(grp);
+    return ORC_OK;
+}
+
+/* One dispatched row: token t sent to rank dst, from source rank src. */
+typedef struct { int32_t dst, src, t; } orc_row;
+
+static int cmp_row(const void *pa, const void *pb)
+{
+    const orc_row *a = (const orc_row *)pa, *b = (const orc_row *)pb;
+    if (a->dst != b->dst) return a->dst < b->dst ? -1 : 1;
+    if (a->src != b->src) return a->src < b->src ? -1 : 1;
+    return a->t < b->t ? -1 : (a->t > b->t);
+}
+
+/* Deduplicated dispatch plan ([EC]: a dispatcher that sends each token to
+ * each GPU once; [CB] "Problem Formulation": V counts each remote node a token
+ * must reach once, given node-level deduplication).
+ *
+ * p(e) = expert_to_rank[e]; s_t = src_rank[t], or t / (T/G) when src_rank is
+ * NULL; N(r) = r / rpn.  Rows are the pairs (t, r) with r in {p(e) : e in D_t},
+ * ordered by (r, s_t, t).  Outputs:
+ *   dest_mask[t]      bit r set when the token has a row for rank r (G <= 64)
+ *   counts[s][r]      rows from source rank s to rank r
+ *   offsets[r*G + s]  first row of the (r, s) segment; offsets[G*G] = R
+ *   row_token[i], row_jmask[i] (bit j set when p(e_tj) is the row's rank)
+ *   row_of[t][j]      the row that carries (t, e_tj)
+ *   summary[5] = { R, R_remote (rows with r != s_t),
+ *                  local = #{(t,j) : p(e_tj) = s_t},
+ *                  V = sum_t |{N(p(e)) : e in D_t} \ {N(s_t)}|,  T*k }
+ * row_token / row_jmask must hold T*k entries. */
+int orc_plan(const int32_t *ids, int T, int k, int E, int G, int rpn,
+             const int32_t *expert_to_rank, const int32_t *src_rank,
+             uint64_t *dest_mask, int32_t *counts, int32_t *offsets,
+             int32_t *row_token, uint8_t *row_jmask, int32_t *row_of, int64_t *summary)
+{
+    if (T < 0 || k < 1 || k > 8 || E < 1 || k > E || G < 1 || G > 64 || rpn < 1 || G % rpn != 0)
+        return ORC_ERR_ARG;
+    if (!src_rank && (T % G != 0)) return ORC_ERR_ARG;
+    for (int e = 0; e < E; ++e)
+        if (expert_to_rank[e] < 0 || expert_to_rank[e] >= G) return ORC_ERR_DATA;
+    for (int t = 0; t < T; ++t) {
+        if (!token_valid(ids + (size_t)t * k, k, E)) return ORC_ERR_DATA;
+        if (src_rank && (src_rank[t] < 0 || src_rank[t] >= G)) return ORC_ERR_DATA;
+    }
+    int nodes = G / rpn;
+    orc_row *rows = (orc_row *)malloc(sizeof(orc_row) * ((size_t)T * k + 1));
+    if (!rows) return ORC_ERR_ARG;
+    size_t R = 0;
+    int64_t local = 0, V = 0;
+    for (int t = 0; t < T; ++t) {
+        const int32_t *d = ids + (size_t)t * k;
+        int s = src_rank ? src_rank[t] : t / (T / G);
+        int want[64] = {0}, node_hit[64] = {0};
+        for (int j = 0; j < k; ++j) {
+            int r = expert_to_rank[d[j]];
+            want[r] = 1;
+            node_hit[r / rpn] = 1;
+            if (r == s) local += 1;
+        }
+        uint64_t m = 0;
+        for (int r = 0; r < G; ++r)
+            if (want[r]) {
+                m |= (uint64_t)1 << r;
+                rows[R].dst = r; rows[R].src = s; rows[R].t = t;
+                ++R;
+            }
+        dest_mask[t] = m;
+        for (int q = 0; q < nodes; ++q)
+            if (node_hit[q] && q != s / rpn) V += 1;
+    }
+    qsort(rows, R, sizeof(orc_row), cmp_row);
+    memset(counts, 0, sizeof(int32_t) * G * G);
+    int64_t remote = 0;
+    for (size_t i = 0; i < R; ++i) {
+        int t = rows[i].t, r = rows[i].dst;
+        const int32_t *d = ids + (size_t)t * k;
+        uint8_t jm = 0;
+        for (int j = 0; j < k; ++j)
+            if (expert_to_rank[d[j]] == r) {
+                jm |= (uint8_t)(1u << j);
+                row_of[(size_t)t * k + j] = (int32_t)i;
+            }
+        row_token[i] = t;
+        row_jmask[i] = jm;
+        counts[rows[i].src * G + r] += 1;
+        if (r != rows[i].src) remote += 1;
+    }
+    int32_t run = 0;
+    for (int r = 0; r < G; ++r)
+        for (int s = 0; s < G; ++s) {
+            offsets[r * G + s] = run;
+            run += counts[s * G + r];
+        }
+    offsets[G * G] = run;
+    summary[0] = (int64_t)R;
+    summary[1] = remote;
+    summary[2] = local;
+    summary[3] = V;
+    summary[4] = (int64_t)T * k;
+    free(rows);
+    return ORC_OK;
+}
+
+/* Row permute into the rank-major send buffer: send[i] = x[row_token[i]]. */
+int orc_permute(const void *x, int elem_bytes, int T, int d, const int32_t *row_token, int64_t R, void *send)
+{
+    size_t rowB = (size_t)elem_bytes * d;
+    for (int64_t i = 0; i < R; ++i) {
+        if (row_token[i] < 0 || row_token[i] >= T) return ORC_ERR_DATA;
+        memcpy((char *)send + rowB * i, (const char *)x + rowB * row_token[i], rowB);
+    }
+    return ORC_OK;
+}
+
+static double load_elem(const void *Y, int y_is_bf16, size_t i)
+{
+    if (y_is_bf16) {
+        uint32_t u = (uint32_t)((const uint16_t *)Y)[i] << 16;
+        float f;
+        memcpy(&f, &u, 4);
+        return (double)f;
+    }
+    return (double)((const float *)Y)[i];
+}
+
+/* Weighted combine, the inverse of dispatch ([EC]: dispatch tokens to their
+ * experts "and then combine the results"; [CE] footnote 3: the hidden-state
+ * combine): out[t][c] = sum_j w[t][j] * Y[idx[t][j]][c], summed in fp64 in j
+ * order. */
+int orc_combine(const void *Y, int y_is_bf16, int64_t R_max, int d, const int32_t *idx,
+                const float *w, int T, int k, double *out)
+{
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j)
+            if (idx[(size_t)t * k + j] < 0 || idx[(size_t)t * k + j] >= R_max) return ORC_ERR_DATA;
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int j = 0; j < k; ++j) {
+                size_t row = (size_t)idx[(size_t)t * k + j];
+                acc += (double)w[(size_t)t * k + j] * load_elem(Y, y_is_bf16, row * d + c);
+            }
+            out[(size_t)t * d + c] = acc;
+        }
+    return ORC_OK;
+}
+
+/* Rank scores for token shuffling ([EC]: move each token to the GPU
+ * predicted to hold its next-layer experts):
+ * rank_score[e][r] = sum over e' with p_{l+1}(e') = r of M_l[e][e']. */
+int orc_rank_score(const uint32_t *trans, const int32_t *next_expert_to_rank, int E, int G, uint32_t *rank_score)
+{
+    for (int e = 0; e < E; ++e)
+        if (next_expert_to_rank[e] < 0 || next_expert_to_rank[e] >= G) return ORC_ERR_DATA;
+    for (int e = 0; e < E; ++e) {
+        for (int r = 0; r < G; ++r) {
+            uint64_t s = 0;
+            for (int f = 0; f < E; ++f)
+                if (next_expert_to_rank[f] == r) s += trans[(size_t)e * E + f];
+            if (s > 0xFFFFFFFFull) return ORC_ERR_DATA;
+            rank_score[(size_t)e * G + r] = (uint32_t)s;
+        }
+    }
+    return ORC_OK;
+}
+
+/* Shuffle target: target[t] = argmax_r sum_j rank_score[e_tj][r], the lowest
+ * r among equal scores. */
+int orc_shuffle_targets(const int32_t *ids, int T, int k, int E, int G, const uint32_t *rank_score, int32_t *target)
+{
+    for (int t = 0; t < T; ++t) {
+        const int32_t *d = ids + (size_t)t * k;
+        if (!token_valid(d, k, E)) return ORC_ERR_DATA;
+        int best = 0;
+        uint64_t best_s = 0;
+        for (int r = 0; r < G; ++r) {
+            uint64_t s = 0;
+            for (int j = 0; j < k; ++j) s += rank_score[(size_t)d[j] * G + r];
+            if (r == 0 || s > best_s) { best = r; best_s = s; }
+        }
+        target[t] = best;
+    }
+    return ORC_OK;
+}
