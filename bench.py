@@ -1,0 +1,479 @@
+"""Benchmark of the co-activation / deduplicated-dispatch hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--placement correlated|uniform] [--no-shuffle]
+                    [--out-dtype f32|bf16] [--impl reference]
+
+A step is one pass of the whole path over one batch: co-activation counts,
+Ochiai and transitions for every layer, then per layer the dispatch plan, the
+row permute, identity experts, the weighted combine and the shuffle targets
+for the next layer.  The default workload is large EP64 (T=131072, E=256, k=8,
+G=64 in 8 nodes, d=7168 bf16, 4 layers), the largest workload with hidden
+states; its inputs (x = 1.88 GB) exceed the 126 MB L2, so no flush is needed
+between steps.  With N GPUs each rank runs its own batch (seed + rank): weak
+scaling, no collective on the data path.
+
+value = dispatch+combine algorithmic bytes of the step / device time of the
+whole step (max over ranks), in GB/s.  Algorithmic bytes are the minimum HBM
+traffic: permute reads each token row once and writes R rows; combine reads
+the U distinct rows and writes T output rows (U = R for identity experts).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import platform
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dedup dispatch+combine GB/s (frac of HBM peak); co-activation tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="large_ep64")
+    ap.add_argument("--placement", default="correlated", choices=["correlated", "uniform"])
+    ap.add_argument("--no-shuffle", action="store_true")
+    ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle time for the CPU baseline")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None, period_ms=100):
+        self.uuid = uuid
+        self.period = period_ms
+        self.proc = None
+
+    def __enter__(self):
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", str(self.period)]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.tmp.flush()
+
+    def summary(self):
+        try:
+            with open(self.tmp.name) as f:
+                rows = [r.strip().split(", ") for r in f if r.strip()]
+        finally:
+            os.unlink(self.tmp.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ reference arm / CPU baseline
+
+def oracle_pass(w, ids, ids_cal, gates, x, placement, shuffle):
+    """One pass of the path through the CPU oracle on a token sample.
+    Returns (seconds, algorithmic dispatch+combine bytes)."""
+    import oracle as orc
+    from synth import bf16_bits_to_f32
+    L, T, k = ids.shape
+    t0 = time.perf_counter()
+    orc.coact(ids, w.E)
+    cal = orc.coact(ids_cal, w.E)
+    if placement == "correlated":
+        e2r = [orc.place_correlated(cal["coact"][l], w.G, w.rpn) for l in range(L)]
+    else:
+        e2r = [orc.place_uniform(w.E, w.G) for _ in range(L)]
+    rs = [orc.rank_score(cal["trans"][l], e2r[l + 1], w.G) for l in range(L - 1)] if shuffle else []
+    src = None
+    rowB = w.d * w.elem_bytes
+    nbytes = 0
+    for l in range(L):
+        p = orc.plan(ids[l], w.E, w.G, w.rpn, e2r[l], src_rank=src)
+        send = orc.permute(x, p["row_token"])
+        Y = bf16_bits_to_f32(send) if w.dtype == "bf16" else send
+        orc.combine(Y, p["row_of"], gates[l], y_is_bf16=False)
+        R = p["R"]
+        nbytes += T * rowB + R * rowB + 4 * T * k + R * rowB + T * w.d * 4 + 8 * T * k
+        if shuffle and l + 1 < L:
+            src = orc.shuffle_targets(ids[l], w.E, w.G, rs[l])
+    return time.perf_counter() - t0, nbytes
+
+
+def cpu_sample(w, T_s, seed):
+    from synth import make_routing, make_gates, make_hidden
+    ids = make_routing(w, seed=seed, T=T_s)
+    cal = make_routing(w, seed=seed + 1, T=T_s)
+    gates = make_gates(w, seed=seed, T=T_s)
+    x = make_hidden(w, seed=seed, T=T_s)
+    return ids, cal, gates, x
+
+
+def sized_sample(w, target_s, shuffle):
+    """Choose a token count (a multiple of G) whose oracle pass takes about target_s."""
+    T_probe = max(w.G, (1024 // w.G) * w.G)
+    ids, cal, gates, x = cpu_sample(w, T_probe, w.seed)
+    sec, _ = oracle_pass(w, ids, cal, gates, x, "correlated", shuffle)
+    T_s = int(T_probe * target_s / max(sec, 1e-6))
+    T_s = max(w.G, min(w.T, (T_s // w.G) * w.G))
+    return T_s
+
+
+def cpu_baseline(w, placement, shuffle, target_s):
+    T_s = sized_sample(w, target_s, shuffle)
+    ids, cal, gates, x = cpu_sample(w, T_s, w.seed)
+    sec, nbytes = oracle_pass(w, ids, cal, gates, x, placement, shuffle)
+    model = platform.processor() or platform.machine()
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"value": nbytes / sec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "%d of %d tokens of %s, all %d layers (stats, calibration, placement, plan, permute, "
+                      "fp64 combine, shuffle), single-threaded C oracle on 1 of %d host cores (%s); %.1f s"
+                      % (T_s, w.T, w.name, w.L, os.cpu_count() or 0, model, sec)}
+
+
+def run_reference(a, w):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    shuffle = not a.no_shuffle
+    # each step: a bounded sample, so that warmup + steps end within a few minutes
+    per_step = max(0.5, min(10.0, 150.0 / max(1, a.steps + a.warmup)))
+    T_s = sized_sample(w, per_step, shuffle)
+    ids, cal, gates, x = cpu_sample(w, T_s, w.seed)
+    for _ in range(a.warmup):
+        oracle_pass(w, ids, cal, gates, x, a.placement, shuffle)
+    secs, nb = [], 0
+    for _ in range(a.steps):
+        s, nb = oracle_pass(w, ids, cal, gates, x, a.placement, shuffle)
+        secs.append(s)
+    tot = sum(secs)
+    value = nb * a.steps / tot / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * tot / a.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "tokens_per_step": T_s, "T": w.T, "E": w.E, "k": w.k, "G": w.G,
+                       "rpn": w.rpn, "d": w.d, "L": w.L, "placement": a.placement, "shuffle": shuffle},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": "%d of %d tokens per step, single-threaded C oracle" % (T_s, w.T)},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ native arm
+
+def traffic_record(kernel_name):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    source is unchanged since the capture (else None)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel_name)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "co_activation_placement_b200", "csrc", rec["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if h == rec["source_sha256_16"] else None
+
+
+def main():
+    a = parse()
+    from synth import WORKLOADS
+    w = WORKLOADS[a.workload]
+    if a.impl == "reference":
+        run_reference(a, w)
+        return
+    import torch
+    import co_activation_placement_b200 as cap
+    from co_activation_placement_b200 import pipeline
+    from synth import make_routing, make_gates, make_hidden
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        pg = dist
+    seed = w.seed + 1000 * rank
+    shuffle = (not a.no_shuffle) and w.L > 1
+    out_dtype = torch.float32 if a.out_dtype == "f32" else torch.bfloat16
+    if w.d == 0:
+        raise SystemExit("workload %s has no hidden states; it is measured as the co-activation sweep" % w.name)
+
+    ids = make_routing(w, seed=seed)
+    ids_cal = make_routing(w, seed=seed + 1)
+    gates = make_gates(w, seed=seed)
+    x = make_hidden(w, seed=seed)
+    hp = pipeline.prepare(w.E, w.G, w.rpn, ids, gates, x, w.dtype, ids_cal, placement=a.placement,
+                          shuffle=shuffle, out_dtype=out_dtype, device=device, timers=True)
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    for _ in range(a.warmup):
+        hp.step()
+    torch.cuda.synchronize()
+    if int(hp.err.item()) != 0:
+        raise SystemExit("device data error %d" % int(hp.err.item()))
+    summaries = hp.summaries()
+    sb = hp.step_bytes(summaries)
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+    barrier()
+    torch.cuda.synchronize()
+    hp.reset_events()
+    n0 = cap.launch_count()
+    with ClockSampler(uuid) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        stop = torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(a.steps):
+            hp.step()
+        stop.record()
+        torch.cuda.synchronize()
+    n1 = cap.launch_count()
+    barrier()
+    per_kernel = hp.kernel_times_ms()
+    hp.reset_events()
+    ms_total = start.elapsed_time(stop)
+    ms_step = ms_total / a.steps
+    if pg is not None:
+        t = torch.tensor([ms_step], device=device, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_step = float(t.item())
+    clocks = clk.summary()
+
+    hbm, hbm_kind = peaks()
+    value = world * sb.dispatch_combine / (ms_step * 1e-3) / 1e9
+    kern = {}
+    bytes_of = {"stats": sb.stats, "plan": sb.plan, "permute": sb.permute, "combine": sb.combine,
+                "shuffle": sb.shuffle}
+    launches_of = {"stats": 1, "plan": w.L, "permute": w.L, "combine": w.L, "shuffle": (w.L - 1) if shuffle else 0}
+    for name, tot_ms in per_kernel.items():
+        ms = tot_ms / a.steps                         # per step
+        gbs = bytes_of[name] / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
+        kern[name] = {"ms_per_step": ms, "launches_per_step": launches_of[name], "gbs": gbs,
+                      "frac_of_hbm": gbs / hbm}
+    dom = max(kern, key=lambda n: kern[n]["ms_per_step"])
+    nl = launches_of[dom]
+    per_launch_ms = kern[dom]["ms_per_step"] / nl
+    traffic = traffic_record(dom)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["gbs"], "peak": hbm, "unit": "GB/s",
+                "frac": kern[dom]["gbs"] / hbm, "peak_kind": hbm_kind,
+                "algorithmic_bytes_per_launch": bytes_of[dom] // nl, "ms_per_launch": per_launch_ms,
+                "traffic": traffic}
+
+    # co-activation tokens/s on this step and on the statistics sweep
+    stats_ms = kern["stats"]["ms_per_step"]
+    coact_tps = world * w.L * w.T / (stats_ms * 1e-3)
+    sweep = None
+    if not a.no_sweep:
+        sweep = run_sweep(cap, pipeline, device, seed, a.steps, a.warmup, hbm, pg)
+
+    e2e = None
+    if not a.no_e2e:
+        e2e = run_e2e(hp, ids, gates, x, w, a, device, sb, pg, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(w, a.placement, shuffle, a.cpu_seconds)
+
+    if rank == 0:
+        R = [int(s[0]) for s in summaries]
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "G": w.G, "rpn": w.rpn, "d": w.d,
+                       "L": w.L, "x_dtype": w.dtype, "out_dtype": a.out_dtype, "placement": a.placement,
+                       "shuffle": shuffle, "parallelism": "replicas (weak scaling, one batch per GPU)",
+                       "l2": "inputs larger than L2 (x %.2f GB per GPU; no flush)" % (x.nbytes / 1e9)},
+            "frac_of_hbm_peak": value / hbm,
+            "roofline": roofline,
+            "kernels": kern,
+            "coact_tokens_per_s": coact_tps,
+            "coact_sweep": sweep,
+            "rows": {"R": R, "T_k": w.T * w.k, "dedup_removed": [1 - r / (w.T * w.k) for r in R],
+                     "R_remote": [int(s[1]) for s in summaries],
+                     "local_share": [int(s[2]) / (w.T * w.k) for s in summaries],
+                     "V": [int(s[3]) for s in summaries]},
+            "clocks": clocks,
+            "e2e": e2e,
+            "gpu_launches": int(n1 - n0),
+            "gpu_launches_per_step": (n1 - n0) / a.steps,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
+    """Co-activation statistics on the 1M-token, 8-layer sweep: tokens/s and
+    the fraction of HBM the statistics kernels reach on their input bytes."""
+    import torch
+    from synth import WORKLOADS, make_routing
+    w = WORKLOADS["stats_sweep"]
+    ids = make_routing(w, seed=seed)
+    hp = pipeline.HotPath(E=w.E, G=1, rpn=1, ids=torch.from_numpy(ids).to(device), gates=None, x=None,
+                          e2r=[], rank_scores=[], rows=False)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for _ in range(warmup):
+        hp.step()
+    torch.cuda.synchronize()
+    tot = 0.0
+    n = max(steps, 10)
+    for _ in range(n):
+        flush.zero_()                                 # ids (268 MB) exceed L2; flush anyway
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        hp.step()
+        e.record()
+        torch.cuda.synchronize()
+        tot += s.elapsed_time(e)
+    ms = tot / n
+    if pg is not None:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    nbytes = hp.step_bytes(None).stats
+    world = pg.get_world_size() if pg is not None else 1
+    return {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "L": w.L, "ms": ms,
+            "tokens_per_s": world * w.L * w.T / (ms * 1e-3),
+            "increments_per_s": world * (w.L * w.T * w.k * (w.k + 1) // 2 + (w.L - 1) * w.T * w.k * w.k) / (ms * 1e-3),
+            "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
+            "algorithmic_bytes": nbytes, "err": int(hp.err.item())}
+
+
+def run_e2e(hp, ids, gates, x, w, a, device, sb, pg, world):
+    """The same metric through the public API with host buffers: every step
+    copies its inputs from pinned host memory and reads its results back."""
+    import torch
+    from co_activation_placement_b200.pipeline import bf16_from_bits
+    ids_h = torch.from_numpy(ids).pin_memory()
+    gates_h = torch.from_numpy(gates).pin_memory()
+    x_h = (bf16_from_bits(x) if w.dtype == "bf16" else torch.from_numpy(x)).pin_memory()
+    out_h = torch.empty(hp.outs[-1].shape, dtype=hp.outs[-1].dtype).pin_memory()
+    st_h = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in hp.stats.items() if v is not None}
+    sum_h = torch.empty((w.L, 5), dtype=torch.int64).pin_memory()
+    hp.timers = False
+
+    def one():
+        hp.ids.copy_(ids_h, non_blocking=True)
+        hp.gates.copy_(gates_h, non_blocking=True)
+        hp.x.copy_(x_h, non_blocking=True)
+        hp.step()
+        out_h.copy_(hp.outs[-1], non_blocking=True)
+        for k_, v in st_h.items():
+            v.copy_(hp.stats[k_], non_blocking=True)
+        sum_h.copy_(torch.stack([p.summary for p in hp.plans]), non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    n = max(3, min(a.steps, 10))
+    if pg is not None:
+        pg.barrier()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(n):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / n
+    if pg is not None:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    hp.timers = True
+    h2d = ids_h.numel() * 4 + gates_h.numel() * 4 + x_h.numel() * x_h.element_size()
+    d2h = out_h.numel() * out_h.element_size() + sum(v.numel() * v.element_size() for v in st_h.values()) + sum_h.numel() * 8
+    return {"value": world * sb.dispatch_combine / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+            "steps": n, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+if __name__ == "__main__":
+    main()

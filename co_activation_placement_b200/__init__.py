@@ -1,0 +1,323 @@
+"""Co-activation statistics and deduplicated expert-parallel dispatch on B200.
+
+Python binding of libmoecoact.so (C ABI in include/moe_coact.h).  Every
+function here only marshals torch tensors into pointers and sizes and enqueues
+the library's sm_100a kernels on torch's current CUDA stream; no step of the
+path is computed in Python or by torch.  If the shared library is missing the
+import of any entry point raises: there is no fallback.
+
+Entry points (names follow the C ABI without the ``moe_`` prefix):
+  coact_stats, plan_dispatch, permute, combine, rank_score, shuffle_targets,
+  place_uniform, place_capacity, place_correlated, launch_count.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoecoact.so")
+
+MOE_OK, MOE_ERR_ARG, MOE_ERR_DATA, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_UNSUPPORTED = range(6)
+DERR_ID_RANGE, DERR_ID_REPEAT, DERR_RANK_RANGE, DERR_ROW_RANGE = 1, 2, 3, 4
+MOE_F32, MOE_BF16 = 0, 1
+
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = lib().moe_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__("%s: %s (status %d)" % (fn, msg, status))
+        self.status = status
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [("dest_mask", ctypes.c_void_p), ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
+                ("row_token", ctypes.c_void_p), ("row_jmask", ctypes.c_void_p), ("row_of", ctypes.c_void_p),
+                ("summary", ctypes.c_void_p)]
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoecoact.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libmoecoact.so is not built (run python -m co_activation_placement_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        sigs = {
+            "moe_status_string": ([i], ctypes.c_char_p),
+            "moe_launch_count": ([], ctypes.c_uint64),
+            "moe_coact_stats_workspace": ([i, i, i, i, i], sz),
+            "moe_coact_stats": ([P, i, i, i, i, P, P, P, P, P, sz, P], i),
+            "moe_plan_dispatch_workspace": ([i, i, i, i], sz),
+            "moe_plan_dispatch": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
+            "moe_permute": ([P, i, i, i, i, P, i64, P, P, P], i),
+            "moe_combine": ([P, i, i64, i, P, P, i, i, P, i, P, P], i),
+            "moe_rank_score": ([P, P, i, i, P, P, P], i),
+            "moe_shuffle_targets": ([P, i, i, i, i, P, P, P, P], i),
+            "moe_place_uniform": ([i, i, P], i),
+            "moe_place_capacity": ([P, i, i, P, P], i),
+            "moe_place_correlated": ([P, i, i, i, P], i),
+        }
+        for name, (args, res) in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def launch_count() -> int:
+    return int(lib().moe_launch_count())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _check(fn: str, st: int):
+    if st != MOE_OK:
+        raise MoeError(fn, st)
+
+
+def _dev(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError("%s must have %d dims" % (name, ndim))
+    return t
+
+
+class Workspace:
+    """A growable device byte buffer, 256-byte aligned (torch allocations are)."""
+
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.buf = torch.empty(0, dtype=torch.uint8, device=self.device)
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+_ws = {}
+
+
+def _workspace(device, slot: str) -> Workspace:
+    key = (str(torch.device(device)), slot)
+    if key not in _ws:
+        _ws[key] = Workspace(device)
+    return _ws[key]
+
+
+def new_err(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+# ---------------------------------------------------------------- statistics
+
+def coact_stats_workspace(L: int, T: int, k: int, E: int, with_trans: bool = True) -> int:
+    return int(lib().moe_coact_stats_workspace(L, T, k, E, int(bool(with_trans))))
+
+
+def coact_stats(ids: torch.Tensor, E: int, coact=None, ochiai=None, trans=None, err=None,
+                want=("coact", "ochiai", "trans"), ws: Optional[torch.Tensor] = None):
+    """ids int32 [L][T][k] -> dict(coact uint32 [L][E][E], ochiai f32 [L][E][E], trans uint32 [L-1][E][E], err)."""
+    _dev(ids, torch.int32, "ids", 3)
+    L, T, k = ids.shape
+    dev = ids.device
+    if coact is None and "coact" in want:
+        coact = torch.empty((L, E, E), dtype=torch.uint32, device=dev)
+    if ochiai is None and "ochiai" in want:
+        ochiai = torch.empty((L, E, E), dtype=torch.float32, device=dev)
+    if trans is None and "trans" in want and L > 1:
+        trans = torch.empty((L - 1, E, E), dtype=torch.uint32, device=dev)
+    err = new_err(dev) if err is None else err
+    need = coact_stats_workspace(L, T, k, E, trans is not None)
+    if ws is None:
+        ws = _workspace(dev, "stats").get(need)
+    st = lib().moe_coact_stats(_ptr(ids), L, T, k, E, _ptr(coact), _ptr(ochiai), _ptr(trans), _ptr(err),
+                               _ptr(ws), ws.numel(), _stream(ids))
+    _check("moe_coact_stats", st)
+    return dict(coact=coact, ochiai=ochiai, trans=trans, err=err)
+
+
+# ---------------------------------------------------------------- dispatch plan
+
+@dataclass
+class Plan:
+    dest_mask: torch.Tensor   # uint64 [T]
+    counts: torch.Tensor      # int32 [G][G]
+    offsets: torch.Tensor     # int32 [G*G+1]
+    row_token: torch.Tensor   # int32 [T*k]
+    row_jmask: torch.Tensor   # uint8 [T*k]
+    row_of: torch.Tensor      # int32 [T][k]
+    summary: torch.Tensor     # int64 [5]
+    err: torch.Tensor         # int32 [1]
+    T: int
+    k: int
+    G: int
+
+    @property
+    def R_max(self) -> int:
+        return self.T * self.k
+
+    @staticmethod
+    def empty(T: int, k: int, G: int, device) -> "Plan":
+        n = max(T * k, 1)
+        return Plan(dest_mask=torch.empty(max(T, 1), dtype=torch.uint64, device=device),
+                    counts=torch.empty((G, G), dtype=torch.int32, device=device),
+                    offsets=torch.empty(G * G + 1, dtype=torch.int32, device=device),
+                    row_token=torch.empty(n, dtype=torch.int32, device=device),
+                    row_jmask=torch.empty(n, dtype=torch.uint8, device=device),
+                    row_of=torch.empty((max(T, 1), k), dtype=torch.int32, device=device),
+                    summary=torch.empty(5, dtype=torch.int64, device=device),
+                    err=new_err(device), T=T, k=k, G=G)
+
+    def c_struct(self) -> _Plan:
+        return _Plan(self.dest_mask.data_ptr(), self.counts.data_ptr(), self.offsets.data_ptr(),
+                     self.row_token.data_ptr(), self.row_jmask.data_ptr(), self.row_of.data_ptr(),
+                     self.summary.data_ptr())
+
+
+def plan_dispatch_workspace(T: int, k: int, G: int, with_src_rank: bool) -> int:
+    return int(lib().moe_plan_dispatch_workspace(T, k, G, int(bool(with_src_rank))))
+
+
+def plan_dispatch(ids: torch.Tensor, E: int, G: int, rpn: int, expert_to_rank: torch.Tensor,
+                  src_rank: Optional[torch.Tensor] = None, plan: Optional[Plan] = None,
+                  ws: Optional[torch.Tensor] = None) -> Plan:
+    """ids int32 [T][k] (one layer) -> Plan (device tensors; row arrays sized T*k)."""
+    _dev(ids, torch.int32, "ids", 2)
+    _dev(expert_to_rank, torch.int32, "expert_to_rank", 1)
+    if src_rank is not None:
+        _dev(src_rank, torch.int32, "src_rank", 1)
+    T, k = ids.shape
+    dev = ids.device
+    if plan is None:
+        plan = Plan.empty(T, k, G, dev)
+    need = plan_dispatch_workspace(T, k, G, src_rank is not None)
+    if ws is None:
+        ws = _workspace(dev, "plan").get(need)
+    cs = plan.c_struct()
+    st = lib().moe_plan_dispatch(_ptr(ids), T, k, E, G, rpn, _ptr(expert_to_rank), _ptr(src_rank),
+                                 ctypes.byref(cs), _ptr(plan.err), _ptr(ws), ws.numel(), _stream(ids))
+    _check("moe_plan_dispatch", st)
+    return plan
+
+
+# ---------------------------------------------------------------- rows
+
+def _dtype_code(dt) -> int:
+    if dt == torch.float32:
+        return MOE_F32
+    if dt == torch.bfloat16:
+        return MOE_BF16
+    raise ValueError("dtype must be float32 or bfloat16")
+
+
+def permute(x: torch.Tensor, row_of: torch.Tensor, R_max: int, send: Optional[torch.Tensor] = None,
+            err: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """send[row_of[t][j]] = x[t]; send is [R_max][d] (rows >= R untouched)."""
+    if x.dim() != 2:
+        raise ValueError("x must be [T][d]")
+    _dev(x, x.dtype, "x")
+    _dev(row_of, torch.int32, "row_of", 2)
+    T, d = x.shape
+    k = row_of.shape[1]
+    if send is None:
+        send = torch.empty((max(R_max, 1), d), dtype=x.dtype, device=x.device)
+    err = new_err(x.device) if err is None else err
+    st = lib().moe_permute(_ptr(x), _dtype_code(x.dtype), T, d, k, _ptr(row_of), R_max, _ptr(send), _ptr(err),
+                           _stream(x))
+    _check("moe_permute", st)
+    return send
+
+
+def combine(Y: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, out_dtype=torch.float32,
+            out: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out[t] = sum_j w[t][j] * Y[idx[t][j]] (fp32 FMA accumulation; out fp32 or bf16)."""
+    _dev(Y, Y.dtype, "Y", 2)
+    _dev(idx, torch.int32, "idx", 2)
+    _dev(w, torch.float32, "w", 2)
+    T, k = idx.shape
+    R_max, d = Y.shape
+    if out is None:
+        out = torch.empty((T, d), dtype=out_dtype, device=Y.device)
+    err = new_err(Y.device) if err is None else err
+    st = lib().moe_combine(_ptr(Y), _dtype_code(Y.dtype), R_max, d, _ptr(idx), _ptr(w), T, k, _ptr(out),
+                           _dtype_code(out.dtype), _ptr(err), _stream(Y))
+    _check("moe_combine", st)
+    return out
+
+
+# ---------------------------------------------------------------- token shuffle
+
+def rank_score(trans_l: torch.Tensor, next_expert_to_rank: torch.Tensor, G: int,
+               out: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _dev(trans_l, torch.uint32, "trans_l", 2)
+    _dev(next_expert_to_rank, torch.int32, "next_expert_to_rank", 1)
+    E = trans_l.shape[0]
+    if out is None:
+        out = torch.empty((E, G), dtype=torch.uint32, device=trans_l.device)
+    err = new_err(trans_l.device) if err is None else err
+    st = lib().moe_rank_score(_ptr(trans_l), _ptr(next_expert_to_rank), E, G, _ptr(out), _ptr(err), _stream(trans_l))
+    _check("moe_rank_score", st)
+    return out
+
+
+def shuffle_targets(ids: torch.Tensor, E: int, G: int, rank_score_tab: torch.Tensor,
+                    target: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _dev(ids, torch.int32, "ids", 2)
+    _dev(rank_score_tab, torch.uint32, "rank_score", 2)
+    T, k = ids.shape
+    if target is None:
+        target = torch.empty(max(T, 1), dtype=torch.int32, device=ids.device)
+    err = new_err(ids.device) if err is None else err
+    st = lib().moe_shuffle_targets(_ptr(ids), T, k, E, G, _ptr(rank_score_tab), _ptr(target), _ptr(err), _stream(ids))
+    _check("moe_shuffle_targets", st)
+    return target
+
+
+# ---------------------------------------------------------------- placement (host)
+
+def _np_ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def place_uniform(E: int, G: int) -> np.ndarray:
+    out = np.empty(E, np.int32)
+    _check("moe_place_uniform", lib().moe_place_uniform(E, G, _np_ptr(out)))
+    return out
+
+
+def place_capacity(load, G: int):
+    load = np.ascontiguousarray(load, dtype=np.float64)
+    out = np.empty(load.size, np.int32)
+    dev = np.empty(G, np.float64)
+    _check("moe_place_capacity", lib().moe_place_capacity(_np_ptr(load), load.size, G, _np_ptr(out), _np_ptr(dev)))
+    return out, dev
+
+
+def place_correlated(coact_l, G: int, rpn: int) -> np.ndarray:
+    c = np.ascontiguousarray(coact_l, dtype=np.uint32)
+    E = c.shape[0]
+    out = np.empty(E, np.int32)
+    _check("moe_place_correlated", lib().moe_place_correlated(_np_ptr(c), E, G, rpn, _np_ptr(out)))
+    return out

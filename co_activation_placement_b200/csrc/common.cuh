@@ -1,0 +1,44 @@
+// Shared helpers of the libmoecoact CUDA sources (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "moe_coact.h"
+
+namespace moe {
+
+// Count of kernels launched by this library (for benchmark accounting).
+void note_launches(uint64_t n);
+
+// Record the first device-side data error: the word keeps its first non-zero
+// value.  Never traps.
+__device__ __forceinline__ void record_error(int32_t *err, int32_t code)
+{
+    if (err) atomicCAS(err, 0, code);
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory on the current
+// device (needed once per kernel and device; cheap to repeat).
+template <typename F>
+inline cudaError_t allow_smem(F *kernel, size_t bytes)
+{
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(reinterpret_cast<const void *>(kernel),
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+inline moe_status launch_status()
+{
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Number of SMs of the current device (cached per device ordinal).
+int sm_count();
+
+}  // namespace moe

@@ -1,0 +1,114 @@
+// Expert placement on the host (run once per re-layout, not per step).
+//
+// Uniform: "Expert Parallelism > Expert Placement Strategies", the uniform
+// listing (device = expert_id // (E/G)).  Capacity-aware: same page,
+// "Capacity-Aware Placement" (largest expected load first, onto the least
+// loaded device).  Correlated: "Expert Coupling in MoE Pretraining", abstract
+// (experts often selected together share a GPU) -- the page gives the goal;
+// this is a greedy equal-size grouping by fp64 Ochiai, node level first when
+// ranks span several nodes ("Cobalt": a token crosses to a remote node once,
+// so co-activated experts should share nodes as well as ranks).
+//
+// The greedy keeps, for every unassigned expert, its running sum of Ochiai to
+// the current group's members; each new member adds its column once, so the
+// sum is accumulated in the order members joined (O(E^2) per level).
+#include <cmath>
+#include <cstdint>
+#include <vector>
+
+#include "moe_coact.h"
+
+namespace {
+
+double ochiai64(const uint32_t *C, int E, int i, int j)
+{
+    const double den = (double)C[(size_t)i * E + i] * (double)C[(size_t)j * E + j];
+    if (den > 0.0) return (double)C[(size_t)i * E + j] / std::sqrt(den);
+    return 0.0;
+}
+
+// Split `pool` (ascending expert ids) into m groups of pool.size()/m.
+std::vector<int> greedy_split(const uint32_t *C, int E, const std::vector<int> &pool, int m)
+{
+    const int n = (int)pool.size();
+    const int size = n / m;
+    std::vector<int> group(n, -1);
+    std::vector<double> score(n);
+    for (int g = 0; g < m; ++g) {
+        int seed = -1;
+        for (int x = 0; x < n; ++x) {
+            if (group[x] >= 0) continue;
+            if (seed < 0 || C[(size_t)pool[x] * E + pool[x]] > C[(size_t)pool[seed] * E + pool[seed]]) seed = x;
+        }
+        group[seed] = g;
+        for (int x = 0; x < n; ++x) score[x] = 0.0;
+        int last = seed;
+        for (int cnt = 1; cnt < size; ++cnt) {
+            int pick = -1;
+            for (int x = 0; x < n; ++x) {
+                if (group[x] >= 0) continue;
+                score[x] += ochiai64(C, E, pool[x], pool[last]);
+                if (pick < 0 || score[x] > score[pick]) pick = x;
+            }
+            group[pick] = g;
+            last = pick;
+        }
+    }
+    return group;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_place_uniform(int E, int G, int32_t *expert_to_rank)
+{
+    if (E < 1 || G < 1 || E % G != 0 || !expert_to_rank) return MOE_ERR_ARG;
+    const int per = E / G;
+    for (int e = 0; e < E; ++e) expert_to_rank[e] = e / per;
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_place_capacity(const double *load, int E, int G, int32_t *expert_to_rank, double *rank_load)
+{
+    if (E < 1 || G < 1 || !load || !expert_to_rank) return MOE_ERR_ARG;
+    std::vector<int> order(E);
+    for (int e = 0; e < E; ++e) order[e] = e;
+    // stable insertion by descending load (lower id first among equals)
+    for (int i = 1; i < E; ++i) {
+        const int e = order[i];
+        int j = i;
+        while (j > 0 && load[order[j - 1]] < load[e]) {
+            order[j] = order[j - 1];
+            --j;
+        }
+        order[j] = e;
+    }
+    std::vector<double> dev(G, 0.0);
+    for (int i = 0; i < E; ++i) {
+        const int e = order[i];
+        int best = 0;
+        for (int g = 1; g < G; ++g)
+            if (dev[g] < dev[best]) best = g;
+        expert_to_rank[e] = best;
+        dev[best] += load[e];
+    }
+    if (rank_load)
+        for (int g = 0; g < G; ++g) rank_load[g] = dev[g];
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_place_correlated(const uint32_t *coact, int E, int G, int rpn, int32_t *expert_to_rank)
+{
+    if (E < 1 || G < 1 || rpn < 1 || G % rpn != 0 || E % G != 0 || !coact || !expert_to_rank) return MOE_ERR_ARG;
+    const int nodes = G / rpn;
+    std::vector<int> all(E);
+    for (int e = 0; e < E; ++e) all[e] = e;
+    const std::vector<int> node_of = greedy_split(coact, E, all, nodes);
+    for (int q = 0; q < nodes; ++q) {
+        std::vector<int> pool;
+        for (int e = 0; e < E; ++e)
+            if (node_of[e] == q) pool.push_back(e);
+        const std::vector<int> grp = greedy_split(coact, E, pool, rpn);
+        for (size_t x = 0; x < pool.size(); ++x) expert_to_rank[pool[x]] = q * rpn + grp[x];
+    }
+    return MOE_OK;
+}

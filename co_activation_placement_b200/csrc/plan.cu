@@ -1,0 +1,488 @@
+// Deduplicated, rank-major dispatch plan.
+//
+// "Expert Coupling in MoE Pretraining", abstract: a dispatcher that sends each
+// token to each GPU once.  "Cobalt", "Problem Formulation": the cross-node
+// cost V = sum_t |{N(r_t^e) : e in D_t} \ {N(s_t)}| under node-level
+// deduplication; here r_t^e = p(e) (one replica per expert).
+//
+// Rows are the pairs (t, r), r in m_t = {p(e) : e in D_t}, ordered by
+// (r, s_t, t).  The order is produced without sorting keys:
+//   1. (only when source ranks are given) a stable counting sort of the tokens
+//      by s_t -> perm; with contiguous shards perm is the identity;
+//   2. the token sequence in perm order is cut into chunks of kChunk tokens
+//      that never straddle a source shard.  Each chunk's block computes m_t
+//      (bitmask of destination ranks), the summary terms and its per-rank row
+//      counts; the last block to finish scans the counts over chunks (column
+//      per rank), which yields every chunk's first row per rank, the rank
+//      segment offsets and counts[s][r] (chunks of one shard are adjacent);
+//   3. each chunk's block ranks its rows per destination with warp ballots
+//      (stable in perm order) and writes row_token, row_jmask and row_of.
+// All arithmetic is integer; the result is unique and does not depend on
+// scheduling.  No kernel waits on another block.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kChunk = 256;   // tokens per block, one per thread
+constexpr int kWarps = kChunk / 32;
+
+struct PlanWsHeader {
+    unsigned int done_count;      // blocks finished in plan_count
+    unsigned int done_src;        // blocks finished in plan_src_count
+    unsigned int pad[2];
+    unsigned long long acc[4];    // R, R_remote, local, V
+};
+
+struct PlanWs {
+    PlanWsHeader *hdr;
+    int32_t *soff;       // [G+1] first perm position of each source shard
+    int32_t *scnt;       // [G]   tokens per source shard
+    int32_t *cpre;       // [G+1] first chunk of each shard; cpre[G] = active chunks
+    int32_t *perm;       // [T]
+    int32_t *sblk;       // [Bs][G]
+    int32_t *sblk_pref;  // [Bs+1][G]
+    int32_t *blk;        // [Bc][G]
+    int32_t *blk_pref;   // [Bc+1][G]
+};
+
+inline int src_blocks(int T) { return (T + kChunk - 1) / kChunk; }
+inline int chunk_blocks(int T, int G, bool with_src)
+{
+    if (with_src) return (T + kChunk - 1) / kChunk + G;
+    const int shard = T / G;
+    return G * std::max(1, (shard + kChunk - 1) / kChunk);
+}
+
+size_t carve(void *ws, int T, int G, bool with_src, PlanWs *out)
+{
+    char *p = static_cast<char *>(ws);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *q = p ? p + off : nullptr;
+        off = round_up(off + bytes, 256);
+        return q;
+    };
+    PlanWs w{};
+    w.hdr = reinterpret_cast<PlanWsHeader *>(take(sizeof(PlanWsHeader)));
+    w.soff = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (G + 1)));
+    w.scnt = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * G));
+    w.cpre = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (G + 1)));
+    const int Bs = src_blocks(T), Bc = chunk_blocks(T, G, with_src);
+    if (with_src) {
+        w.perm = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * std::max(T, 1)));
+        w.sblk = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * Bs * G));
+        w.sblk_pref = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (Bs + 1) * G));
+    }
+    w.blk = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)Bc * G));
+    w.blk_pref = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)(Bc + 1) * G));
+    if (out) *out = w;
+    return off;
+}
+
+template <int K>
+__device__ __forceinline__ void load_token(const int32_t *__restrict__ p, int (&v)[K])
+{
+#pragma unroll
+    for (int q = 0; q < K; ++q) v[q] = __ldg(p + q);
+}
+
+template <int K>
+__device__ __forceinline__ int token_error(const int (&v)[K], int E)
+{
+    int bad_range = 0, bad_rep = 0;
+#pragma unroll
+    for (int a = 0; a < K; ++a) {
+        bad_range |= (unsigned)v[a] >= (unsigned)E;
+#pragma unroll
+        for (int b = 0; b < a; ++b) bad_rep |= v[a] == v[b];
+    }
+    return bad_range ? MOE_DERR_ID_RANGE : (bad_rep ? MOE_DERR_ID_REPEAT : 0);
+}
+
+__device__ __forceinline__ int clamp_rank(int r, int G, int32_t *err)
+{
+    if ((unsigned)r >= (unsigned)G) {
+        record_error(err, MOE_DERR_RANK_RANGE);
+        return 0;
+    }
+    return r;
+}
+
+// Last block: exclusive scan of a [B][G] column table (rows b, column d) into
+// pref[b][d] and tot[d] (shared).  Called by all threads of one block.
+__device__ void scan_columns(const int32_t *tab, int32_t *pref, int B, int G, int32_t *tot_sh, int32_t *seg_sh)
+{
+    const int nseg = blockDim.x / G;   // >= 1 since G <= 64 < blockDim
+    const int d = threadIdx.x % G, q = threadIdx.x / G;
+    const int per = (B + nseg - 1) / nseg;
+    const int b0 = min(B, q * per), b1 = min(B, b0 + per);
+    if (q < nseg) {
+        int s = 0;
+        for (int b = b0; b < b1; ++b) s += __ldcg(tab + (size_t)b * G + d);
+        seg_sh[q * G + d] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        int run = 0;
+        for (int qq = 0; qq < nseg; ++qq) {
+            int v = seg_sh[qq * G + threadIdx.x];
+            seg_sh[qq * G + threadIdx.x] = run;
+            run += v;
+        }
+        tot_sh[threadIdx.x] = run;
+    }
+    __syncthreads();
+    if (q < nseg) {
+        int run = seg_sh[q * G + d];
+        for (int b = b0; b < b1; ++b) {
+            pref[(size_t)b * G + d] = run;
+            run += __ldcg(tab + (size_t)b * G + d);
+        }
+    }
+    if (threadIdx.x < G) pref[(size_t)B * G + threadIdx.x] = tot_sh[threadIdx.x];
+    __syncthreads();
+}
+
+// ---- step 1: stable counting sort of tokens by source rank ---------------
+
+__global__ void __launch_bounds__(kChunk)
+plan_src_count_kernel(const int32_t *__restrict__ src_rank, int T, int G, PlanWs w, int32_t *err)
+{
+    __shared__ int32_t hist[64];
+    __shared__ int32_t tot[64];
+    __shared__ int32_t seg[kChunk];
+    __shared__ bool last;
+    if (threadIdx.x < G) hist[threadIdx.x] = 0;
+    __syncthreads();
+    const int t = blockIdx.x * kChunk + threadIdx.x;
+    if (t < T) {
+        const int s = clamp_rank(__ldg(src_rank + t), G, err);
+        atomicAdd(&hist[s], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x < G) w.sblk[(size_t)blockIdx.x * G + threadIdx.x] = hist[threadIdx.x];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(&w.hdr->done_src, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    scan_columns(w.sblk, w.sblk_pref, gridDim.x, G, tot, seg);
+    if (threadIdx.x == 0) {
+        int run = 0, ch = 0;
+        for (int s = 0; s < G; ++s) {
+            w.soff[s] = run;
+            w.scnt[s] = tot[s];
+            w.cpre[s] = ch;
+            run += tot[s];
+            ch += (tot[s] + kChunk - 1) / kChunk;
+        }
+        w.soff[G] = run;
+        w.cpre[G] = ch;
+        w.hdr->done_src = 0;
+    }
+}
+
+__global__ void __launch_bounds__(kChunk)
+plan_src_scatter_kernel(const int32_t *__restrict__ src_rank, int T, int G, PlanWs w)
+{
+    __shared__ int32_t wcnt[kWarps][64];
+    __shared__ int32_t wbase[kWarps][64];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kWarps * 64; i += kChunk) (&wcnt[0][0])[i] = 0;
+    __syncthreads();
+    const int t = blockIdx.x * kChunk + threadIdx.x;
+    const bool act = t < T;
+    int s = act ? __ldg(src_rank + t) : G;       // inactive lanes get key G
+    if (act && (unsigned)s >= (unsigned)G) s = 0; // same clamp as the count kernel
+    const unsigned peers = __match_any_sync(0xffffffffu, s);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (act && rank == 0) wcnt[wid][s] = __popc(peers);
+    __syncthreads();
+    if (threadIdx.x < G) {
+        int run = 0;
+        for (int q = 0; q < kWarps; ++q) {
+            wbase[q][threadIdx.x] = run;
+            run += wcnt[q][threadIdx.x];
+        }
+    }
+    __syncthreads();
+    if (act) {
+        const int pos = __ldcg(w.soff + s) + __ldcg(w.sblk_pref + (size_t)blockIdx.x * G + s) + wbase[wid][s] + rank;
+        w.perm[pos] = t;
+    }
+}
+
+// ---- step 2: destination sets, summary terms, per-chunk row counts ---------
+
+struct ChunkRange {
+    int s, p0, p1;   // source shard, perm positions [p0, p1)
+    bool active;
+};
+
+__device__ __forceinline__ ChunkRange chunk_range(int b, int T, int G, bool with_src, const PlanWs &w)
+{
+    ChunkRange c;
+    if (with_src) {
+        const int nact = __ldcg(w.cpre + G);
+        if (b >= nact) { c.active = false; c.s = 0; c.p0 = c.p1 = 0; return c; }
+        int s = 0;
+        while (s + 1 < G && __ldcg(w.cpre + s + 1) <= b) ++s;
+        const int base = __ldcg(w.soff + s), n = __ldcg(w.scnt + s);
+        c.s = s;
+        c.p0 = base + (b - __ldcg(w.cpre + s)) * kChunk;
+        c.p1 = min(base + n, c.p0 + kChunk);
+        c.active = true;
+    } else {
+        const int shard = T / G;
+        const int nch = max(1, (shard + kChunk - 1) / kChunk);
+        c.s = b / nch;
+        c.p0 = c.s * shard + (b % nch) * kChunk;
+        c.p1 = min((c.s + 1) * shard, c.p0 + kChunk);
+        c.active = true;
+    }
+    return c;
+}
+
+template <int K>
+__global__ void __launch_bounds__(kChunk)
+plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
+                  const int32_t *__restrict__ e2r_g, bool with_src, PlanWs w, moe_plan P, int32_t *err)
+{
+    extern __shared__ int32_t e2r[];           // [E]
+    __shared__ int32_t cnt[64];
+    __shared__ int32_t tot[64];
+    __shared__ int32_t seg[kChunk];
+    __shared__ unsigned long long red[4][kWarps];
+    __shared__ bool last;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    for (int e = threadIdx.x; e < E; e += kChunk) e2r[e] = clamp_rank(__ldg(e2r_g + e), G, err);
+    if (threadIdx.x < 64) cnt[threadIdx.x] = 0;
+    __syncthreads();
+
+    const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, w);
+    unsigned long long my[4] = {0, 0, 0, 0};
+    const int p = c.p0 + threadIdx.x;
+    if (c.active && p < c.p1) {
+        const int t = with_src ? __ldcg(w.perm + p) : p;
+        int v[K];
+        load_token<K>(ids + (size_t)t * K, v);
+        const int bad = token_error<K>(v, E);
+        unsigned long long m = 0, nodes = 0;
+        if (bad) {
+            record_error(err, bad);
+        } else {
+            int local = 0;
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                const int r = e2r[v[j]];
+                m |= 1ull << r;
+                nodes |= 1ull << (r / rpn);
+                local += r == c.s;
+            }
+            my[0] = __popcll(m);
+            my[1] = __popcll(m & ~(1ull << c.s));
+            my[2] = local;
+            my[3] = __popcll(nodes & ~(1ull << (c.s / rpn)));
+            for (unsigned long long q = m; q; q &= q - 1) atomicAdd(&cnt[__ffsll((long long)q) - 1], 1);
+        }
+        P.dest_mask[t] = m;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        unsigned long long x = my[i];
+        for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0) red[i][wid] = x;
+    }
+    __syncthreads();
+    if (threadIdx.x < 4) {
+        unsigned long long x = 0;
+        for (int q = 0; q < kWarps; ++q) x += red[threadIdx.x][q];
+        if (x) atomicAdd(&w.hdr->acc[threadIdx.x], x);
+    }
+    if (threadIdx.x < G) w.blk[(size_t)blockIdx.x * G + threadIdx.x] = cnt[threadIdx.x];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(&w.hdr->done_count, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+
+    // the last block: scan chunk counts, then offsets, counts and summary
+    const int B = with_src ? __ldcg(w.cpre + G) : gridDim.x;
+    scan_columns(w.blk, w.blk_pref, B, G, tot, seg);
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int d = 0; d < G; ++d) { seg[d] = run; run += tot[d]; }   // seg[d] = first row of rank d
+        P.offsets[G * G] = run;
+    }
+    __syncthreads();
+    const int nshard = G;
+    for (int i = threadIdx.x; i < G * G; i += kChunk) {
+        const int d = i / G, s = i % G;   // offsets in (d, s) order
+        int b0, b1;
+        if (with_src) { b0 = __ldcg(w.cpre + s); b1 = __ldcg(w.cpre + s + 1); }
+        else { const int nch = B / nshard; b0 = s * nch; b1 = b0 + nch; }
+        const int a0 = __ldcg(w.blk_pref + (size_t)b0 * G + d);
+        const int a1 = __ldcg(w.blk_pref + (size_t)b1 * G + d);
+        P.offsets[d * G + s] = seg[d] + a0;
+        P.counts[s * G + d] = a1 - a0;
+    }
+    if (threadIdx.x < 4) P.summary[threadIdx.x] = (int64_t)atomicAdd(&w.hdr->acc[threadIdx.x], 0ull);
+    if (threadIdx.x == 4) P.summary[4] = (int64_t)T * K;
+    if (threadIdx.x == 0) w.hdr->done_count = 0;
+}
+
+// ---- step 3: stable per-destination ranks and row writes -----------------
+
+template <int K>
+__global__ void __launch_bounds__(kChunk)
+plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
+                    const int32_t *__restrict__ e2r_g, bool with_src, PlanWs w, moe_plan P)
+{
+    extern __shared__ int32_t e2r[];           // [E]
+    __shared__ int32_t base[64];               // first row of this chunk per rank
+    __shared__ int32_t wcnt[kWarps][64];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, w);
+    if (!c.active) return;
+    for (int e = threadIdx.x; e < E; e += kChunk) {
+        const int r = __ldg(e2r_g + e);
+        e2r[e] = (unsigned)r >= (unsigned)G ? 0 : r;
+    }
+    for (int i = threadIdx.x; i < kWarps * 64; i += kChunk) (&wcnt[0][0])[i] = 0;
+    if (threadIdx.x < G)
+        base[threadIdx.x] = __ldcg(P.offsets + threadIdx.x * G) + __ldcg(w.blk_pref + (size_t)blockIdx.x * G + threadIdx.x);
+    __syncthreads();
+
+    const int p = c.p0 + threadIdx.x;
+    const bool act = p < c.p1;
+    int t = 0, v[K], r[K];
+    unsigned long long m = 0;
+    if (act) {
+        t = with_src ? __ldcg(w.perm + p) : p;
+        load_token<K>(ids + (size_t)t * K, v);
+        if (token_error<K>(v, E) == 0) {
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                r[j] = e2r[v[j]];
+                m |= 1ull << r[j];
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < K; ++j) P.row_of[(size_t)t * K + j] = -1;
+        }
+    }
+    const unsigned lt = (1u << lane) - 1u;
+    unsigned lo = __reduce_or_sync(0xffffffffu, (unsigned)m);
+    unsigned hi = __reduce_or_sync(0xffffffffu, (unsigned)(m >> 32));
+    unsigned long long wor = ((unsigned long long)hi << 32) | lo;
+    for (unsigned long long q = wor; q; q &= q - 1) {
+        const int d = __ffsll((long long)q) - 1;
+        const unsigned bal = __ballot_sync(0xffffffffu, (m >> d) & 1ull);
+        if (lane == 0) wcnt[wid][d] = __popc(bal);
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        int run = 0;
+        for (int q = 0; q < kWarps; ++q) {
+            const int x = wcnt[q][threadIdx.x];
+            wcnt[q][threadIdx.x] = run;
+            run += x;
+        }
+    }
+    __syncthreads();
+    for (unsigned long long q = wor; q; q &= q - 1) {
+        const int d = __ffsll((long long)q) - 1;
+        const unsigned bal = __ballot_sync(0xffffffffu, (m >> d) & 1ull);
+        if ((m >> d) & 1ull) {
+            const int pos = base[d] + wcnt[wid][d] + __popc(bal & lt);
+            unsigned jm = 0;
+#pragma unroll
+            for (int j = 0; j < K; ++j)
+                if (r[j] == d) {
+                    jm |= 1u << j;
+                    P.row_of[(size_t)t * K + j] = pos;
+                }
+            P.row_token[pos] = t;
+            P.row_jmask[pos] = (uint8_t)jm;
+        }
+    }
+}
+
+template <int K>
+moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const int32_t *e2r,
+                       const int32_t *src_rank, const moe_plan &P, int32_t *err, const PlanWs &w,
+                       cudaStream_t s)
+{
+    const bool with_src = src_rank != nullptr;
+    const size_t smem = sizeof(int32_t) * (size_t)E;
+    int launched = 0;
+    if (with_src) {
+        const int Bs = src_blocks(T);
+        plan_src_count_kernel<<<Bs, kChunk, 0, s>>>(src_rank, T, G, w, err);
+        plan_src_scatter_kernel<<<Bs, kChunk, 0, s>>>(src_rank, T, G, w);
+        launched += 2;
+    }
+    const int Bc = chunk_blocks(T, G, with_src);
+    if (allow_smem(plan_count_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    if (allow_smem(plan_scatter_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    plan_count_kernel<K><<<Bc, kChunk, smem, s>>>(ids, T, E, G, rpn, e2r, with_src, w, P, err);
+    plan_scatter_kernel<K><<<Bc, kChunk, smem, s>>>(ids, T, E, G, e2r, with_src, w, P);
+    launched += 2;
+    moe_status st = launch_status();
+    if (st == MOE_OK) note_launches(launched);
+    return st;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" size_t moe_plan_dispatch_workspace(int T, int k, int G, int with_src_rank)
+{
+    (void)k;
+    if (T < 0 || G < 1 || G > 64) return 0;
+    return carve(nullptr, T, G, with_src_rank != 0, nullptr) + 256;
+}
+
+extern "C" moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                                        const int32_t *expert_to_rank, const int32_t *src_rank,
+                                        const moe_plan *plan, int32_t *err,
+                                        void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    if (T < 0 || k < 1 || k > 8 || E < k || G < 1 || G > 64 || rpn < 1 || G % rpn != 0) return MOE_ERR_ARG;
+    if ((long long)T * k >= (1ll << 31)) return MOE_ERR_ARG;
+    if (E > 12 * 1024) return MOE_ERR_UNSUPPORTED;
+    if (!plan || !err || !expert_to_rank) return MOE_ERR_ARG;
+    if (!plan->counts || !plan->offsets || !plan->summary) return MOE_ERR_ARG;
+    if (T > 0 && (!ids || !plan->dest_mask || !plan->row_token || !plan->row_jmask || !plan->row_of))
+        return MOE_ERR_ARG;
+    if (!src_rank && T % G != 0) return MOE_ERR_ARG;
+    if (T == 0) {
+        if (cudaMemsetAsync(plan->counts, 0, sizeof(int32_t) * G * G, stream) != cudaSuccess ||
+            cudaMemsetAsync(plan->offsets, 0, sizeof(int32_t) * (G * G + 1), stream) != cudaSuccess ||
+            cudaMemsetAsync(plan->summary, 0, sizeof(int64_t) * 5, stream) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    PlanWs w;
+    const size_t need = carve(ws, T, G, src_rank != nullptr, &w);
+    if (!ws || !aligned256(ws) || ws_bytes < need) return MOE_ERR_WORKSPACE;
+    if (cudaMemsetAsync(w.hdr, 0, sizeof(PlanWsHeader), stream) != cudaSuccess) return MOE_ERR_CUDA;
+    switch (k) {
+    case 1: return launch_plan<1>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
+    case 2: return launch_plan<2>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
+    case 3: return launch_plan<3>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
+    case 4: return launch_plan<4>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
+    case 5: return launch_plan<5>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
+    case 6: return launch_plan<6>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
+    case 7: return launch_plan<7>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
+    case 8: return launch_plan<8>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
+    }
+    return MOE_ERR_ARG;
+}

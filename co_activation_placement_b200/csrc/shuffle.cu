@@ -1,0 +1,139 @@
+// Token shuffling targets.
+//
+// "Expert Coupling in MoE Pretraining", abstract: under sequence parallelism
+// each token moves, during the reduce-scatter after attention, to the GPU
+// predicted to hold its next-layer experts.  The prediction used here: a token
+// that picks e at layer l picks an expert on rank r at layer l+1 as often as
+// the transition counts M_l say,
+//   rank_score[e][r] = sum_{e' : p_{l+1}(e') = r} M_l[e][e'],
+//   target_t = argmax_r sum_j rank_score[e_tj][r]   (lowest r on ties).
+//
+// moe_rank_score: one block per expert row e, a shared uint64 accumulator per
+// rank (integer atomics: order-free).  moe_shuffle_targets: the E x G table
+// sits in shared memory; one warp per token, each lane owns ranks lane and
+// lane+32 (conflict-free: a row of the table is read contiguously), uint64
+// sums, and a warp argmax with (score desc, rank asc).
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+
+__global__ void __launch_bounds__(kThreads)
+rank_score_kernel(const uint32_t *__restrict__ trans, const int32_t *__restrict__ e2r, int E, int G,
+                  uint32_t *__restrict__ rs, int32_t *err)
+{
+    __shared__ unsigned long long acc[64];
+    const int e = blockIdx.x;
+    if (threadIdx.x < G) acc[threadIdx.x] = 0;
+    __syncthreads();
+    for (int f = threadIdx.x; f < E; f += kThreads) {
+        const int r = __ldg(e2r + f);
+        if ((unsigned)r >= (unsigned)G) {
+            record_error(err, MOE_DERR_RANK_RANGE);
+            continue;
+        }
+        const uint32_t v = __ldg(trans + (size_t)e * E + f);
+        if (v) atomicAdd(&acc[r], (unsigned long long)v);
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const unsigned long long v = acc[threadIdx.x];
+        rs[(size_t)e * G + threadIdx.x] = v > 0xffffffffull ? 0xffffffffu : (uint32_t)v;
+    }
+}
+
+template <int K>
+__global__ void __launch_bounds__(kThreads)
+shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, const uint32_t *__restrict__ rs_g,
+                       int32_t *__restrict__ target, int32_t *err)
+{
+    extern __shared__ uint32_t tab[];   // [E][G]
+    for (int i = threadIdx.x; i < E * G; i += kThreads) tab[i] = __ldg(rs_g + i);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * (kThreads / 32);
+    for (int t = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t < T; t += nwarps) {
+        const int mine = lane < K ? __ldg(ids + (size_t)t * K + lane) : 0;
+        const bool bad = __any_sync(0xffffffffu, lane < K && (unsigned)mine >= (unsigned)E);
+        if (bad) {
+            if (lane == 0) {
+                record_error(err, MOE_DERR_ID_RANGE);
+                target[t] = 0;
+            }
+            continue;
+        }
+        unsigned long long a0 = 0, a1 = 0;
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            const int e = __shfl_sync(0xffffffffu, mine, j);
+            const uint32_t *row = tab + (size_t)e * G;
+            if (lane < G) a0 += row[lane];
+            if (lane + 32 < G) a1 += row[lane + 32];
+        }
+        // candidate key: score + 1 for a real rank, 0 for none
+        unsigned long long best = lane < G ? a0 + 1 : 0;
+        int bi = lane;
+        if (lane + 32 < G && a1 + 1 > best) { best = a1 + 1; bi = lane + 32; }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+        }
+        if (lane == 0) target[t] = bi;
+    }
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" moe_status moe_rank_score(const uint32_t *trans_l, const int32_t *next_expert_to_rank,
+                                     int E, int G, uint32_t *rank_score, int32_t *err, cudaStream_t stream)
+{
+    if (E < 1 || G < 1 || G > 64 || !trans_l || !next_expert_to_rank || !rank_score || !err) return MOE_ERR_ARG;
+    rank_score_kernel<<<E, kThreads, 0, stream>>>(trans_l, next_expert_to_rank, E, G, rank_score, err);
+    moe_status st = launch_status();
+    if (st == MOE_OK) note_launches(1);
+    return st;
+}
+
+template <int K>
+static moe_status launch_shuffle(const int32_t *ids, int T, int E, int G, const uint32_t *rs, int32_t *target,
+                                 int32_t *err, cudaStream_t s)
+{
+    const size_t smem = sizeof(uint32_t) * (size_t)E * G;
+    if (allow_smem(shuffle_targets_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    const long long need = ((long long)T + (kThreads / 32) - 1) / (kThreads / 32);
+    const int grid = (int)std::max<long long>(1, std::min<long long>(need, (long long)sm_count() * 3));
+    shuffle_targets_kernel<K><<<grid, kThreads, smem, s>>>(ids, T, E, G, rs, target, err);
+    return launch_status();
+}
+
+extern "C" moe_status moe_shuffle_targets(const int32_t *ids, int T, int k, int E, int G,
+                                          const uint32_t *rank_score, int32_t *target,
+                                          int32_t *err, cudaStream_t stream)
+{
+    if (T < 0 || k < 1 || k > 8 || E < k || G < 1 || G > 64 || !err) return MOE_ERR_ARG;
+    if ((long long)E * G > 16384) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!ids || !rank_score || !target) return MOE_ERR_ARG;
+    moe_status st = MOE_ERR_ARG;
+    switch (k) {
+    case 1: st = launch_shuffle<1>(ids, T, E, G, rank_score, target, err, stream); break;
+    case 2: st = launch_shuffle<2>(ids, T, E, G, rank_score, target, err, stream); break;
+    case 3: st = launch_shuffle<3>(ids, T, E, G, rank_score, target, err, stream); break;
+    case 4: st = launch_shuffle<4>(ids, T, E, G, rank_score, target, err, stream); break;
+    case 5: st = launch_shuffle<5>(ids, T, E, G, rank_score, target, err, stream); break;
+    case 6: st = launch_shuffle<6>(ids, T, E, G, rank_score, target, err, stream); break;
+    case 7: st = launch_shuffle<7>(ids, T, E, G, rank_score, target, err, stream); break;
+    case 8: st = launch_shuffle<8>(ids, T, E, G, rank_score, target, err, stream); break;
+    }
+    if (st == MOE_OK) note_launches(1);
+    return st;
+}

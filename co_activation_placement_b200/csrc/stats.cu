@@ -1,0 +1,387 @@
+// Co-activation counts, Ochiai similarity and cross-layer transition counts.
+//
+// Definitions ("Expert Coupling in MoE Pretraining", abstract: pairs of
+// experts selected together, and next-layer experts predicted by this layer's;
+// "Cobalt", "Key Observation": Ochiai over the experts' token sets):
+//   C_l[i][j] = |{t : i, j in D_t^l}|,   S_l = C_ij / sqrt(C_ii C_jj),
+//   M_l[i][j] = |{t : i in D_t^l, j in D_t^{l+1}}|.
+//
+// Design (sm_100a).  The work is a histogram: k(k+1)/2 counter increments per
+// token and layer for C (upper triangle incl. diagonal) and k^2 per token and
+// layer pair for M.  Each thread block owns one "group" -- (C of layer l, a band
+// of triangle rows) or (M of layer pair l, a band of rows) -- small enough to
+// live as uint32 counters in shared memory (<= 64 KB, three blocks per SM), and
+// one contiguous token slice.  Threads take one token at a time, load its k ids
+// with vector loads, sort them with a compare-exchange network (C only) and
+// issue shared-memory atomic adds for the pairs whose row falls in the band.
+// Blocks are numbered slice-major, so the blocks that read the same token
+// slice of a layer (C of l, M of l-1 and M of l) run in the same wave and
+// share it through L2.  Each block writes its counters once, coalesced, to a
+// partial buffer; a second kernel sums the partials of each cell (integer, so
+// the result does not depend on order), mirrors the triangle and evaluates
+// Ochiai in fp64 with IEEE-rounded multiply, square root and divide.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kHistThreads = 512;
+constexpr int kMaxBands = 64;
+constexpr int kBudgetCells = 16384;      // 64 KB of uint32 counters per block
+constexpr int kTargetBlocks = 148 * 3;   // one wave at three blocks per SM
+constexpr int kMinSliceTokens = 2048;
+constexpr int kReduceThreads = 256;
+
+struct StatsGeom {
+    int L, T, k, E;
+    int Jc, Jt;          // groups: Jc = L*nbc (0 if no C wanted), Jt = (L-1)*nbt
+    int nbc, nbt, S;
+    int rows_t;          // rows per M band
+    int max_cells;
+    long long c_layer;   // partial words per C layer  = S * E(E+1)/2
+    long long t_layer;   // partial words per M layer  = S * E*E
+    long long c_total;   // Jc ? L * c_layer : 0
+    int band_c[kMaxBands + 1];
+};
+
+__host__ __device__ inline long long tri_start(int i, int E)
+{
+    return (long long)i * E - (long long)i * (i - 1) / 2;
+}
+
+bool make_geom(int L, int T, int k, int E, bool want_c, bool want_t, StatsGeom &g)
+{
+    g = StatsGeom{};
+    g.L = L; g.T = T; g.k = k; g.E = E;
+    const long long tri_all = tri_start(E, E);
+    // C bands: equal shares of the triangle, each within the counter budget
+    int nbc = 0;
+    if (want_c) {
+        nbc = (int)((tri_all + kBudgetCells - 1) / kBudgetCells);
+        for (;; ++nbc) {
+            if (nbc > kMaxBands) return false;
+            g.band_c[0] = 0;
+            bool ok = true;
+            int r = 0;
+            for (int b = 1; b <= nbc; ++b) {
+                long long want = tri_all * b / nbc;
+                while (r < E && tri_start(r, E) < want) ++r;
+                g.band_c[b] = (b == nbc) ? E : r;
+                long long cells = tri_start(g.band_c[b], E) - tri_start(g.band_c[b - 1], E);
+                if (cells > kBudgetCells || g.band_c[b] <= g.band_c[b - 1]) ok = false;
+            }
+            if (ok) break;
+        }
+    }
+    // M bands: equal row counts; at least enough to fit the budget, and about
+    // as many as makes a band's k^2/nbt increments per token match a C band's
+    // k(k+1)/2/nbc, so that blocks of both kinds take similar time.
+    int nbt = 0;
+    if (want_t && L > 1) {
+        int rows_fit = std::max(1, kBudgetCells / E);
+        int nbt_min = (E + rows_fit - 1) / rows_fit;
+        int want = want_c ? (int)((double)nbc * 2.0 * k / (k + 1) + 0.5) : 1;
+        nbt = std::min(E, std::max(nbt_min, want));
+        g.rows_t = (E + nbt - 1) / nbt;
+        nbt = (E + g.rows_t - 1) / g.rows_t;
+        if (g.rows_t * E > kBudgetCells) return false;
+    }
+    g.nbc = nbc;
+    g.nbt = nbt;
+    g.Jc = want_c ? L * nbc : 0;
+    g.Jt = (want_t && L > 1) ? (L - 1) * nbt : 0;
+    int J = g.Jc + g.Jt;
+    if (J == 0) return false;
+    int S = (kTargetBlocks + J / 2) / J;
+    S = std::max(1, std::min(S, std::max(1, T / kMinSliceTokens)));
+    g.S = S;
+    int mc = 0;
+    for (int b = 0; b < nbc; ++b)
+        mc = std::max(mc, (int)(tri_start(g.band_c[b + 1], E) - tri_start(g.band_c[b], E)));
+    if (nbt) mc = std::max(mc, g.rows_t * E);
+    g.max_cells = mc;
+    g.c_layer = (long long)S * tri_all;
+    g.t_layer = (long long)S * E * E;
+    g.c_total = g.Jc ? (long long)L * g.c_layer : 0;
+    return true;
+}
+
+long long partial_words(const StatsGeom &g)
+{
+    return g.c_total + (g.Jt ? (long long)(g.L - 1) * g.t_layer : 0);
+}
+
+// Load token t's K ids; VEC selects 16- or 8-byte vector loads (the host checks
+// the base alignment).
+template <int K, bool VEC>
+__device__ __forceinline__ void load_ids(const int32_t *__restrict__ p, int (&v)[K])
+{
+    if constexpr (VEC && K % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < K / 4; ++q) {
+            int4 a = __ldg(reinterpret_cast<const int4 *>(p) + q);
+            v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+        }
+    } else if constexpr (VEC && K % 2 == 0) {
+#pragma unroll
+        for (int q = 0; q < K / 2; ++q) {
+            int2 a = __ldg(reinterpret_cast<const int2 *>(p) + q);
+            v[2 * q] = a.x; v[2 * q + 1] = a.y;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < K; ++q) v[q] = __ldg(p + q);
+    }
+}
+
+template <int K>
+__device__ __forceinline__ void sort_ids(int (&v)[K])
+{
+#pragma unroll
+    for (int i = 0; i < K; ++i)
+#pragma unroll
+        for (int j = 0; j + 1 < K - i; ++j) {
+            int a = v[j], b = v[j + 1];
+            v[j] = min(a, b);
+            v[j + 1] = max(a, b);
+        }
+}
+
+// 0 when the K ids are distinct and in [0, E), else the device error code.
+template <int K>
+__device__ __forceinline__ int check_ids(const int (&v)[K], int E)
+{
+    int bad_range = 0, bad_rep = 0;
+#pragma unroll
+    for (int a = 0; a < K; ++a) {
+        bad_range |= (unsigned)v[a] >= (unsigned)E;
+#pragma unroll
+        for (int b = 0; b < a; ++b) bad_rep |= v[a] == v[b];
+    }
+    return bad_range ? MOE_DERR_ID_RANGE : (bad_rep ? MOE_DERR_ID_REPEAT : 0);
+}
+
+template <int K, bool VEC>
+__global__ void __launch_bounds__(kHistThreads)
+stats_hist_kernel(const int32_t *__restrict__ ids, StatsGeom G, uint32_t *__restrict__ part, int32_t *err)
+{
+    extern __shared__ uint32_t hist[];
+    const int J = G.Jc + G.Jt;
+    const int slice = blockIdx.x / J;
+    const int grp = blockIdx.x % J;
+    const int T = G.T, E = G.E;
+    const int t0 = (int)((long long)T * slice / G.S);
+    const int t1 = (int)((long long)T * (slice + 1) / G.S);
+    const bool is_c = grp < G.Jc;
+    int l, r0, r1, cells;
+    long long out;
+    if (is_c) {
+        l = grp / G.nbc;
+        const int band = grp % G.nbc;
+        r0 = G.band_c[band];
+        r1 = G.band_c[band + 1];
+        cells = (int)(tri_start(r1, E) - tri_start(r0, E));
+        out = (long long)l * G.c_layer + (long long)G.S * tri_start(r0, E) + (long long)slice * cells;
+    } else {
+        const int q = grp - G.Jc;
+        l = q / G.nbt;
+        const int band = q % G.nbt;
+        r0 = band * G.rows_t;
+        r1 = min(E, r0 + G.rows_t);
+        cells = (r1 - r0) * E;
+        out = G.c_total + (long long)l * G.t_layer + (long long)G.S * r0 * E + (long long)slice * cells;
+    }
+    for (int c = threadIdx.x; c < cells; c += blockDim.x) hist[c] = 0u;
+    __syncthreads();
+
+    const int32_t *lay = ids + (size_t)l * T * K;
+    if (is_c) {
+        const int base0 = (int)tri_start(r0, E);
+        for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+            int v[K];
+            load_ids<K, VEC>(lay + (size_t)t * K, v);
+            sort_ids<K>(v);
+            int bad = ((unsigned)v[0] >= (unsigned)E || (unsigned)v[K - 1] >= (unsigned)E) ? MOE_DERR_ID_RANGE : 0;
+#pragma unroll
+            for (int a = 0; a + 1 < K; ++a)
+                if (!bad && v[a] == v[a + 1]) bad = MOE_DERR_ID_REPEAT;
+            if (bad) {
+                record_error(err, bad);
+                continue;
+            }
+#pragma unroll
+            for (int a = 0; a < K; ++a) {
+                const int i = v[a];
+                if (i >= r0 && i < r1) {
+                    const int row = (int)tri_start(i, E) - base0 - i;
+#pragma unroll
+                    for (int b = a; b < K; ++b) atomicAdd(&hist[row + v[b]], 1u);
+                }
+            }
+        }
+    } else {
+        const int32_t *nxt = lay + (size_t)T * K;
+        for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+            int a[K], c[K];
+            load_ids<K, VEC>(lay + (size_t)t * K, a);
+            load_ids<K, VEC>(nxt + (size_t)t * K, c);
+            int bad = check_ids<K>(a, E);
+            if (!bad) bad = check_ids<K>(c, E);
+            if (bad) {
+                record_error(err, bad);
+                continue;
+            }
+#pragma unroll
+            for (int x = 0; x < K; ++x) {
+                const int i = a[x];
+                if (i >= r0 && i < r1) {
+                    const int row = (i - r0) * E;
+#pragma unroll
+                    for (int y = 0; y < K; ++y) atomicAdd(&hist[row + c[y]], 1u);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    uint32_t *dst = part + out;
+    for (int c = threadIdx.x; c < cells; c += blockDim.x) dst[c] = hist[c];
+}
+
+__device__ __forceinline__ uint32_t c_cell_sum(const StatsGeom &G, const uint32_t *__restrict__ part, int l, int a, int b)
+{
+    // (a, b) with a <= b: find a's band, then sum the slices
+    int band = 0;
+    while (a >= G.band_c[band + 1]) ++band;
+    const int r0 = G.band_c[band];
+    const long long cells = tri_start(G.band_c[band + 1], G.E) - tri_start(r0, G.E);
+    const long long base = (long long)l * G.c_layer + (long long)G.S * tri_start(r0, G.E)
+                           + (tri_start(a, G.E) - tri_start(r0, G.E)) + (b - a);
+    uint32_t s = 0;
+    for (int q = 0; q < G.S; ++q) s += __ldg(part + base + (long long)q * cells);
+    return s;
+}
+
+// blockIdx.y selects the matrix: [0, L) C of layer y, [L, 2L-1) M of layer y-L.
+__global__ void __launch_bounds__(kReduceThreads)
+stats_reduce_kernel(StatsGeom G, const uint32_t *__restrict__ part, uint32_t *coact, float *ochiai, uint32_t *trans)
+{
+    extern __shared__ uint32_t diag[];
+    const int E = G.E;
+    const int m = blockIdx.y;
+    const long long EE = (long long)E * E;
+    if (m < G.L) {
+        if (!G.Jc) return;
+        const int l = m;
+        if (ochiai) {
+            for (int e = threadIdx.x; e < E; e += blockDim.x) diag[e] = c_cell_sum(G, part, l, e, e);
+            __syncthreads();
+        }
+        for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < EE; c += (long long)gridDim.x * blockDim.x) {
+            const int i = (int)(c / E), j = (int)(c % E);
+            const uint32_t v = c_cell_sum(G, part, l, min(i, j), max(i, j));
+            if (coact) coact[(long long)l * EE + c] = v;
+            if (ochiai) {
+                const double den = __dmul_rn((double)diag[i], (double)diag[j]);
+                const double s = den > 0.0 ? __ddiv_rn((double)v, __dsqrt_rn(den)) : 0.0;
+                ochiai[(long long)l * EE + c] = __double2float_rn(s);
+            }
+        }
+    } else {
+        if (!G.Jt || !trans) return;
+        const int l = m - G.L;
+        for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < EE; c += (long long)gridDim.x * blockDim.x) {
+            const int i = (int)(c / E), j = (int)(c % E);
+            const int band = i / G.rows_t;
+            const int r0 = band * G.rows_t;
+            const int r1 = min(E, r0 + G.rows_t);
+            const long long cells = (long long)(r1 - r0) * E;
+            const long long base = G.c_total + (long long)l * G.t_layer + (long long)G.S * r0 * E
+                                   + (long long)(i - r0) * E + j;
+            uint32_t s = 0;
+            for (int q = 0; q < G.S; ++q) s += __ldg(part + base + (long long)q * cells);
+            trans[(long long)l * EE + c] = s;
+        }
+    }
+}
+
+template <int K>
+moe_status launch_hist(const int32_t *ids, const StatsGeom &g, uint32_t *part, int32_t *err, cudaStream_t s)
+{
+    const size_t smem = (size_t)g.max_cells * sizeof(uint32_t);
+    const int blocks = (g.Jc + g.Jt) * g.S;
+    const bool vec = (K % 4 == 0) ? aligned16(ids) : ((K % 2 == 0) ? ((reinterpret_cast<uintptr_t>(ids) & 7u) == 0) : false);
+    if (vec) {
+        if (allow_smem(stats_hist_kernel<K, true>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+        stats_hist_kernel<K, true><<<blocks, kHistThreads, smem, s>>>(ids, g, part, err);
+    } else {
+        if (allow_smem(stats_hist_kernel<K, false>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+        stats_hist_kernel<K, false><<<blocks, kHistThreads, smem, s>>>(ids, g, part, err);
+    }
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" size_t moe_coact_stats_workspace(int L, int T, int k, int E, int with_trans)
+{
+    if (L < 1 || T < 0 || k < 1 || k > 8 || E < k || E > 1024) return 0;
+    // the largest of the geometries a call may choose (with or without C)
+    long long words = 0;
+    StatsGeom g;
+    if (make_geom(L, T, k, E, true, with_trans != 0, g)) words = std::max(words, partial_words(g));
+    if (with_trans && L > 1 && make_geom(L, T, k, E, false, true, g)) words = std::max(words, partial_words(g));
+    if (words == 0) return 0;
+    return round_up((size_t)words * sizeof(uint32_t), 256) + 256;
+}
+
+extern "C" moe_status moe_coact_stats(const int32_t *ids, int L, int T, int k, int E,
+                                      uint32_t *coact, float *ochiai, uint32_t *trans,
+                                      int32_t *err, void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    if (L < 1 || T < 0 || k < 1 || k > 8 || E < k || E > 1024) return MOE_ERR_ARG;
+    if ((long long)L * T * k >= (1ll << 31)) return MOE_ERR_ARG;
+    if (!err || (T > 0 && !ids)) return MOE_ERR_ARG;
+    if (L == 1) trans = nullptr;
+    const bool want_c = coact || ochiai;
+    const bool want_t = trans != nullptr;
+    if (!want_c && !want_t) return MOE_OK;
+    const size_t EE = (size_t)E * E;
+    if (T == 0) {
+        if (coact && cudaMemsetAsync(coact, 0, sizeof(uint32_t) * EE * L, stream) != cudaSuccess) return MOE_ERR_CUDA;
+        if (ochiai && cudaMemsetAsync(ochiai, 0, sizeof(float) * EE * L, stream) != cudaSuccess) return MOE_ERR_CUDA;
+        if (trans && cudaMemsetAsync(trans, 0, sizeof(uint32_t) * EE * (L - 1), stream) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    StatsGeom g;
+    if (!make_geom(L, T, k, E, want_c, want_t, g)) return MOE_ERR_UNSUPPORTED;
+    const size_t need = (size_t)partial_words(g) * sizeof(uint32_t);
+    if (!ws || !aligned256(ws) || ws_bytes < need) return MOE_ERR_WORKSPACE;
+    uint32_t *part = static_cast<uint32_t *>(ws);
+    moe_status st = MOE_ERR_ARG;
+    switch (k) {
+    case 1: st = launch_hist<1>(ids, g, part, err, stream); break;
+    case 2: st = launch_hist<2>(ids, g, part, err, stream); break;
+    case 3: st = launch_hist<3>(ids, g, part, err, stream); break;
+    case 4: st = launch_hist<4>(ids, g, part, err, stream); break;
+    case 5: st = launch_hist<5>(ids, g, part, err, stream); break;
+    case 6: st = launch_hist<6>(ids, g, part, err, stream); break;
+    case 7: st = launch_hist<7>(ids, g, part, err, stream); break;
+    case 8: st = launch_hist<8>(ids, g, part, err, stream); break;
+    }
+    if (st != MOE_OK) return st;
+    note_launches(1);
+    const int mats = L + (want_t ? L - 1 : 0);
+    const long long per_block = (long long)kReduceThreads * 4;
+    int bx = (int)std::min<long long>(((long long)EE + per_block - 1) / per_block, 1024);
+    dim3 grid(bx, mats);
+    const size_t smem = (size_t)E * sizeof(uint32_t);
+    stats_reduce_kernel<<<grid, kReduceThreads, smem, stream>>>(g, part, coact, ochiai, trans);
+    st = launch_status();
+    if (st == MOE_OK) note_launches(1);
+    return st;
+}

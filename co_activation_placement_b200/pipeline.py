@@ -1,0 +1,197 @@
+"""One step of the hot path over a batch, on preallocated device buffers.
+
+A step is, for a batch of top-k routing decisions over L MoE layers:
+
+  1. co-activation counts, Ochiai and cross-layer transitions for all layers
+     (moe_coact_stats);
+  2. per layer l: the deduplicated dispatch plan under that layer's placement,
+     with source ranks = the previous layer's shuffle targets when token
+     shuffling is on (moe_plan_dispatch); the row permute of the hidden states
+     into the rank-major send buffer (moe_permute); identity experts (the
+     expert output of a row is the row); the weighted combine back to token
+     order (moe_combine); and, before layer l+1, the shuffle targets from
+     layer l's picks (moe_shuffle_targets).
+
+Every step is a library call on torch's current stream; this module only
+allocates buffers and sequences the calls.  Placements and rank-score tables
+are inputs: they are computed from a calibration batch (a re-layout happens
+every so many training steps, not every step).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+import co_activation_placement_b200 as cap
+
+
+def bf16_from_bits(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+
+@dataclass
+class StepBytes:
+    """Algorithmic HBM bytes of one step (minimum traffic of each kernel)."""
+    permute: int = 0
+    combine: int = 0
+    plan: int = 0
+    stats: int = 0
+    shuffle: int = 0
+
+    @property
+    def dispatch_combine(self) -> int:
+        return self.permute + self.combine
+
+
+@dataclass
+class HotPath:
+    E: int
+    G: int
+    rpn: int
+    ids: torch.Tensor                  # int32 [L][T][k]
+    gates: Optional[torch.Tensor]      # f32 [L][T][k]
+    x: Optional[torch.Tensor]          # [T][d] f32 or bf16
+    e2r: List[torch.Tensor]            # int32 [E] per layer
+    rank_scores: List[torch.Tensor]    # uint32 [E][G] per layer pair (empty: no shuffle)
+    out_dtype: torch.dtype = torch.bfloat16
+    rows: bool = True                  # run plan/permute/combine (False: statistics only)
+    timers: bool = False               # record CUDA events around each library call
+    # buffers
+    stats: dict = field(default_factory=dict)
+    plans: List[cap.Plan] = field(default_factory=list)
+    send: Optional[torch.Tensor] = None
+    outs: List[torch.Tensor] = field(default_factory=list)
+    targets: List[torch.Tensor] = field(default_factory=list)
+    err: Optional[torch.Tensor] = None
+    events: list = field(default_factory=list)
+
+    def __post_init__(self):
+        L, T, k = self.ids.shape
+        dev = self.ids.device
+        E = self.E
+        self.L, self.T, self.k = L, T, k
+        self.err = cap.new_err(dev)
+        self.stats = dict(coact=torch.empty((L, E, E), dtype=torch.uint32, device=dev),
+                          ochiai=torch.empty((L, E, E), dtype=torch.float32, device=dev),
+                          trans=torch.empty((max(L - 1, 1), E, E), dtype=torch.uint32, device=dev) if L > 1 else None)
+        self.stats_ws = torch.empty(max(cap.coact_stats_workspace(L, T, k, E, L > 1), 1), dtype=torch.uint8, device=dev)
+        if not self.rows:
+            return
+        self.shuffle = len(self.rank_scores) > 0
+        self.plans = [cap.Plan.empty(T, k, self.G, dev) for _ in range(L)]
+        self.plan_ws = torch.empty(max(cap.plan_dispatch_workspace(T, k, self.G, True), 1), dtype=torch.uint8, device=dev)
+        d = self.x.shape[1]
+        self.send = torch.empty((T * k, d), dtype=self.x.dtype, device=dev)
+        self.outs = [torch.empty((T, d), dtype=self.out_dtype, device=dev) for _ in range(L)]
+        self.targets = [torch.empty(T, dtype=torch.int32, device=dev) for _ in range(max(L - 1, 0))] if self.shuffle else []
+
+    # ------------------------------------------------------------------ step
+    def _mark(self, name):
+        if self.timers:
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record()
+            self.events.append((name, ev))
+
+    def reset_events(self):
+        self.events = []
+
+    def step(self):
+        self._mark("start")
+        cap.coact_stats(self.ids, self.E, coact=self.stats["coact"], ochiai=self.stats["ochiai"],
+                        trans=self.stats["trans"], err=self.err, ws=self.stats_ws)
+        self._mark("stats")
+        if not self.rows:
+            return
+        for l in range(self.L):
+            src = self.targets[l - 1] if (self.shuffle and l > 0) else None
+            p = cap.plan_dispatch(self.ids[l], self.E, self.G, self.rpn, self.e2r[l], src_rank=src,
+                                  plan=self.plans[l], ws=self.plan_ws)
+            self._mark("plan")
+            cap.permute(self.x, p.row_of, p.R_max, send=self.send, err=self.err)
+            self._mark("permute")
+            cap.combine(self.send, p.row_of, self.gates[l], out=self.outs[l], err=self.err)
+            self._mark("combine")
+            if self.shuffle and l + 1 < self.L:
+                cap.shuffle_targets(self.ids[l], self.E, self.G, self.rank_scores[l],
+                                    target=self.targets[l], err=self.err)
+                self._mark("shuffle")
+
+    def kernel_times_ms(self):
+        """Device time (ms) of each kind of call, summed over all steps run
+        since reset_events() (call after synchronising)."""
+        out = {}
+        for (a, ea), (b, eb) in zip(self.events, self.events[1:]):
+            if b != "start":
+                out[b] = out.get(b, 0.0) + ea.elapsed_time(eb)
+        return out
+
+    # ------------------------------------------------------------------ bytes
+    def step_bytes(self, summaries: np.ndarray) -> StepBytes:
+        """summaries int64 [L][5] as read back from the plans."""
+        L, T, k, E = self.L, self.T, self.k, self.E
+        b = StepBytes()
+        b.stats = L * T * k * 4 + (2 * L + max(L - 1, 0)) * E * E * 4
+        if not self.rows:
+            return b
+        d = self.x.shape[1]
+        rowB = d * self.x.element_size()
+        outB = d * torch.tensor([], dtype=self.out_dtype).element_size()
+        for l in range(L):
+            R = int(summaries[l][0])
+            src_b = 4 * T if (self.shuffle and l > 0) else 0
+            b.plan += T * k * 4 + E * 4 + src_b + 8 * T + 5 * R + 4 * T * k + 8 * self.G * self.G
+            b.permute += T * rowB + R * rowB + 4 * T * k
+            b.combine += R * rowB + T * outB + 8 * T * k
+            if self.shuffle and l + 1 < L:
+                b.shuffle += T * k * 4 + E * self.G * 4 + 4 * T
+        return b
+
+    def summaries(self) -> np.ndarray:
+        return torch.stack([p.summary for p in self.plans]).cpu().numpy()
+
+
+def calibrate(ids_cal: torch.Tensor, E: int, G: int, rpn: int, placement: str, shuffle: bool):
+    """Placements and rank-score tables from a calibration batch (int32
+    [L][T][k] on the device): its statistics come from moe_coact_stats, the
+    placement from the host greedy, the tables from moe_rank_score.
+    Returns (list of e2r int32 [E] device tensors, list of rank_score uint32
+    [E][G] device tensors, host coact of the calibration batch)."""
+    L = ids_cal.shape[0]
+    st = cap.coact_stats(ids_cal, E, want=("coact", "trans"))
+    torch.cuda.current_stream(ids_cal.device).synchronize()
+    if int(st["err"].item()):
+        raise ValueError("calibration batch has invalid ids (device code %d)" % int(st["err"].item()))
+    coact_h = st["coact"].cpu().numpy()
+    if placement == "uniform":
+        e2r_h = [cap.place_uniform(E, G) for _ in range(L)]
+    elif placement == "correlated":
+        e2r_h = [cap.place_correlated(coact_h[l], G, rpn) for l in range(L)]
+    else:
+        raise ValueError("placement must be uniform or correlated")
+    e2r = [torch.from_numpy(a).to(ids_cal.device) for a in e2r_h]
+    rs = []
+    if shuffle:
+        for l in range(L - 1):
+            rs.append(cap.rank_score(st["trans"][l], e2r[l + 1], G))
+    return e2r, rs, coact_h
+
+
+def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarray], x: Optional[np.ndarray],
+            x_dtype: str, ids_cal: np.ndarray, placement: str = "correlated", shuffle: bool = True,
+            out_dtype=torch.bfloat16, device="cuda", rows: bool = True, timers: bool = False) -> HotPath:
+    """Upload a batch (host numpy arrays; x as float32 or bf16 bit patterns)
+    and its calibration batch, calibrate, and return the step's HotPath."""
+    dev = torch.device(device)
+    ids_d = torch.from_numpy(np.ascontiguousarray(ids, dtype=np.int32)).to(dev)
+    cal_d = torch.from_numpy(np.ascontiguousarray(ids_cal, dtype=np.int32)).to(dev)
+    e2r, rs, _ = calibrate(cal_d, E, G, rpn, placement, shuffle and ids.shape[0] > 1) if rows else ([], [], None)
+    gates_d = torch.from_numpy(np.ascontiguousarray(gates, dtype=np.float32)).to(dev) if rows else None
+    if rows:
+        x_d = (bf16_from_bits(x) if x_dtype == "bf16" else torch.from_numpy(np.ascontiguousarray(x, np.float32))).to(dev)
+    else:
+        x_d = None
+    return HotPath(E=E, G=G, rpn=rpn, ids=ids_d, gates=gates_d, x=x_d, e2r=e2r, rank_scores=rs,
+                   out_dtype=out_dtype, rows=rows, timers=timers)

@@ -1,0 +1,236 @@
+/*
+ * moe_coact.h -- C ABI of libmoecoact.so: expert co-activation statistics and
+ * deduplicated, rank-major expert-parallel dispatch and combine on one B200.
+ *
+ * What the library computes is defined on these pages (cited by title and
+ * section):
+ *   [EC]  "Expert Coupling in MoE Pretraining: Reducing All-to-All Overhead
+ *          with Correlated Placement and Token Shuffling", abstract.
+ *   [EPS] "Expert Parallelism > Expert Placement Strategies": the uniform
+ *          placement listing; "Capacity-Aware Placement".
+ *   [CB]  "Cobalt: Leveraging Expert Co-activation for Efficient Distributed
+ *          MoE Training": "Key Observation (Expert Co-activation)" (Ochiai),
+ *          "Problem Formulation" (cross-node cost V, node-level deduplication).
+ *   [CE]  "Training Communication-Efficient Mixture-of-Experts Language Models
+ *          with Layer Re-Configuration", footnote 3 (hidden states and routed
+ *          probabilities are dispatched; combine is the inverse exchange).
+ *
+ * Notation: T tokens, E experts, k experts per token (k <= 8), L layers,
+ * G expert-parallel ranks (G <= 64), rpn ranks per node, d hidden size.
+ * D_t^l is the set of k distinct experts token t selects at layer l;
+ * p(e) = expert_to_rank[e]; s_t is token t's source rank; N(r) = r / rpn.
+ * EP ranks and nodes are logical partitions of one GPU's memory: "rank r's
+ * receive buffer" is a segment of one device buffer.
+ *
+ * Conventions for every call:
+ *  - Pointers marked "device" are device memory owned by the caller; "host"
+ *    pointers are host memory owned by the caller.  The library never
+ *    allocates or frees memory.
+ *  - Device work is enqueued asynchronously on `stream`.  Argument errors are
+ *    detected on the host before anything is enqueued and returned as
+ *    MOE_ERR_ARG / MOE_ERR_WORKSPACE / MOE_ERR_UNSUPPORTED; nothing is
+ *    enqueued then.  A CUDA launch failure returns MOE_ERR_CUDA.
+ *  - Errors in the data (an expert id outside [0, E), a repeated id within a
+ *    token, a rank outside [0, G), a row index outside the buffer) are found by
+ *    the kernels, which skip the offending item and record a code in the
+ *    caller's device word `err` (int32).  The first code recorded is kept
+ *    (later ones do not overwrite a non-zero word) and no call clears it: the
+ *    caller zeroes `err` and reads it after synchronising.  When it is
+ *    non-zero the outputs of that call are unspecified.  Kernels never trap.
+ *  - Calls keep no state between invocations except the global launch
+ *    counter below.  Workspace ("ws") is caller-provided device memory of at
+ *    least the size the matching *_workspace query returns, 256-byte aligned.
+ */
+#ifndef MOE_COACT_H
+#define MOE_COACT_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_ARG = 1,          /* invalid size, null pointer or misalignment   */
+    MOE_ERR_DATA = 2,         /* host-visible data error (host placement calls) */
+    MOE_ERR_WORKSPACE = 3,    /* ws too small or misaligned                   */
+    MOE_ERR_CUDA = 4,         /* a CUDA runtime call failed                   */
+    MOE_ERR_UNSUPPORTED = 5   /* shape outside what the kernels implement     */
+} moe_status;
+
+/* Codes written to the device error word. */
+#define MOE_DERR_ID_RANGE   1   /* expert id outside [0, E)             */
+#define MOE_DERR_ID_REPEAT  2   /* an expert id repeated within a token */
+#define MOE_DERR_RANK_RANGE 3   /* expert_to_rank or src_rank outside [0, G) */
+#define MOE_DERR_ROW_RANGE  4   /* a row index outside the row buffer   */
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+const char *moe_status_string(moe_status s);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all streams), for benchmark accounting.  Thread-safe. */
+uint64_t moe_launch_count(void);
+
+/* ------------------------------------------------------------------------
+ * Co-activation statistics  ([EC]; [CB] "Key Observation")
+ *
+ *   coact[l][i][j]  = |{t : i in D_t^l and j in D_t^l}|   (C_ii = load n_i)
+ *   ochiai[l][i][j] = C_ij / sqrt(C_ii * C_jj), evaluated in fp64 with IEEE
+ *                     division and square root, rounded once to fp32; 0 when
+ *                     C_ii * C_jj = 0
+ *   trans[l][i][j]  = |{t : i in D_t^l and j in D_t^{l+1}}|, l < L-1
+ *
+ * ids     device int32 [L][T][k], row-major (token t's k picks contiguous)
+ * coact   device uint32 [L][E][E] or NULL
+ * ochiai  device float  [L][E][E] or NULL
+ * trans   device uint32 [L-1][E][E] or NULL (ignored when L == 1)
+ * err     device int32 [1]
+ * ws      device workspace, moe_coact_stats_workspace(L, T, k, E, trans != NULL) bytes
+ * Limits: 1 <= k <= 8, k <= E <= 1024, T >= 0, L >= 1, L*T*k < 2^31.
+ * Data errors: MOE_DERR_ID_RANGE, MOE_DERR_ID_REPEAT.
+ * ---------------------------------------------------------------------- */
+size_t moe_coact_stats_workspace(int L, int T, int k, int E, int with_trans);
+moe_status moe_coact_stats(const int32_t *ids, int L, int T, int k, int E,
+                           uint32_t *coact, float *ochiai, uint32_t *trans,
+                           int32_t *err, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Deduplicated dispatch plan  ([EC]: "sends each token to each GPU once";
+ * [CB] "Problem Formulation": V with node-level deduplication, r_t^e = p(e))
+ *
+ * Rows are the pairs (t, r) with r in m_t = {p(e) : e in D_t}, i.e. one row
+ * per token and destination rank however many of its experts live there.
+ * Row order is (r, s_t, t) ascending: destination-major ("rank-major"), so
+ * rank r's rows are the contiguous segment [offsets[r*G], offsets[r*G+G]),
+ * split by source rank.
+ *
+ * All members are device pointers supplied by the caller:
+ *   dest_mask [T]        uint64, bit r set iff r in m_t
+ *   counts    [G][G]     int32, counts[s][r] = rows from source s to rank r
+ *   offsets   [G*G+1]    int32, offsets[r*G+s] = first row of (r, s);
+ *                        offsets[G*G] = R
+ *   row_token [T*k]      int32, token of row i (entries [0, R) written)
+ *   row_jmask [T*k]      uint8, bit j set iff p(e_tj) is row i's rank
+ *   row_of    [T][k]     int32, the row that carries (t, e_tj)
+ *   summary   [5]        int64: R, R_remote (rows with r != s_t),
+ *                        local = #{(t,j) : p(e_tj) = s_t},
+ *                        V = sum_t |{N(r) : r in m_t} \ {N(s_t)}|, T*k
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    uint64_t *dest_mask;
+    int32_t *counts;
+    int32_t *offsets;
+    int32_t *row_token;
+    uint8_t *row_jmask;
+    int32_t *row_of;
+    int64_t *summary;
+} moe_plan;
+
+/* ids            device int32 [T][k] (one layer)
+ * expert_to_rank device int32 [E], values in [0, G)
+ * src_rank       device int32 [T] or NULL; NULL means contiguous shards
+ *                s_t = t / (T/G) and then requires G | T
+ * Limits: 1 <= k <= 8, k <= E, 1 <= G <= 64, rpn >= 1, G % rpn == 0, T >= 0,
+ * T*k < 2^31.  Data errors: MOE_DERR_ID_RANGE, MOE_DERR_ID_REPEAT,
+ * MOE_DERR_RANK_RANGE. */
+size_t moe_plan_dispatch_workspace(int T, int k, int G, int with_src_rank);
+moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                             const int32_t *expert_to_rank, const int32_t *src_rank,
+                             const moe_plan *plan, int32_t *err,
+                             void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Row permute into the rank-major send buffer  ([EC]; [CE] footnote 3)
+ *   send[row_of[t][j]][:] = x[t][:]   for every t, j
+ * which equals send[i] = x[row_token[i]] for every row i < R.  Each token's
+ * row is read from x once and written to each of its distinct rows.
+ *
+ * x        device [T][d] elements of `dtype` (16-byte aligned)
+ * row_of   device int32 [T][k] (from moe_plan_dispatch)
+ * send     device [R_max][d] of `dtype` (16-byte aligned); rows >= R untouched
+ * Requires d * sizeof(dtype) to be a multiple of 16 bytes.
+ * Data errors: MOE_DERR_ROW_RANGE (row_of outside [0, R_max)).
+ * ---------------------------------------------------------------------- */
+moe_status moe_permute(const void *x, moe_dtype dtype, int T, int d, int k,
+                       const int32_t *row_of, int64_t R_max, void *send,
+                       int32_t *err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Weighted combine, the inverse of dispatch  ([EC]: "then combine the
+ * results"; [CE] footnote 3)
+ *   out[t][:] = sum_j w[t][j] * Y[idx[t][j]][:]
+ * accumulated in fp32 with fused multiply-adds.  When several j of a token
+ * name the same row (several of its experts on one rank), that row is read
+ * once and its weights are first summed in j order; the distinct rows are
+ * then accumulated in order of first appearance.  Worst-case error against
+ * the exact sum is below (2k-1) * 2^-24 * sum_j |w_tj * Y_idx_tj|.
+ * Output is fp32, or rounded to bf16 (nearest even) for out_dtype MOE_BF16.
+ *
+ * Y    device [R_max][d] of y_dtype (16-byte aligned)
+ * idx  device int32 [T][k] row indices into Y (e.g. row_of)
+ * w    device float [T][k]
+ * out  device [T][d] of out_dtype (16-byte aligned)
+ * Requires d * sizeof(y_dtype) to be a multiple of 16 bytes.
+ * Data errors: MOE_DERR_ROW_RANGE (that term is skipped).
+ * ---------------------------------------------------------------------- */
+moe_status moe_combine(const void *Y, moe_dtype y_dtype, int64_t R_max, int d,
+                       const int32_t *idx, const float *w, int T, int k,
+                       void *out, moe_dtype out_dtype, int32_t *err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Token shuffling  ([EC]: move each token to the GPU predicted to hold its
+ * next-layer experts)
+ *
+ * moe_rank_score: rank_score[e][r] = sum over e' with p_{l+1}(e') = r of
+ *   trans_l[e][e'] -- how often a token that picks e at layer l picks an
+ *   expert hosted on rank r at layer l+1.
+ *   trans_l device uint32 [E][E]; next_expert_to_rank device int32 [E];
+ *   rank_score device uint32 [E][G].  Data errors: MOE_DERR_RANK_RANGE.
+ *
+ * moe_shuffle_targets: target[t] = argmax_r sum_j rank_score[e_tj][r]
+ *   (sums in uint64; the lowest r among equal scores).
+ *   ids device int32 [T][k]; rank_score device uint32 [E][G], E*G <= 16384;
+ *   target device int32 [T].  Data errors: MOE_DERR_ID_RANGE.
+ * ---------------------------------------------------------------------- */
+moe_status moe_rank_score(const uint32_t *trans_l, const int32_t *next_expert_to_rank,
+                          int E, int G, uint32_t *rank_score, int32_t *err, cudaStream_t stream);
+moe_status moe_shuffle_targets(const int32_t *ids, int T, int k, int E, int G,
+                               const uint32_t *rank_score, int32_t *target,
+                               int32_t *err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Placement (host, synchronous)
+ *
+ * moe_place_uniform ([EPS] uniform listing): expert_to_rank[e] = e / (E/G);
+ *   MOE_ERR_ARG unless G divides E.
+ *
+ * moe_place_capacity ([EPS] "Capacity-Aware Placement"): experts in
+ *   descending load (equal loads: lower id first) each go to the rank with the
+ *   least load so far (ties: lowest rank); loads summed in fp64.
+ *   load host double [E]; rank_load host double [G] (out, may be NULL).
+ *
+ * moe_place_correlated ([EC]: experts often selected together share a GPU).
+ *   The pages state the goal only; this is a greedy equal-size grouping.
+ *   With nodes = G/rpn > 1, experts are first split into `nodes` groups of
+ *   E/nodes, then each node's experts into rpn groups of E/G.  A group is
+ *   seeded with the unassigned expert of largest C_ee and grown by the
+ *   unassigned expert whose fp64 Ochiai summed over the group's members (in
+ *   the order they joined) is largest; ties go to the lowest id.  Node group
+ *   q, rank group u -> rank q*rpn + u.
+ *   coact host uint32 [E][E] (one layer); requires G | E and rpn | G.
+ *
+ * expert_to_rank host int32 [E] (out) for all three.
+ * ---------------------------------------------------------------------- */
+moe_status moe_place_uniform(int E, int G, int32_t *expert_to_rank);
+moe_status moe_place_capacity(const double *load, int E, int G, int32_t *expert_to_rank, double *rank_load);
+moe_status moe_place_correlated(const uint32_t *coact, int E, int G, int rpn, int32_t *expert_to_rank);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_COACT_H */

@@ -1,0 +1,120 @@
+"""The C ABI without a GPU: the library builds and loads, exports every entry
+point that include/*.h declares, the host placement entry points agree with
+the oracle exactly, and argument checks fail before any device work."""
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+from conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def cap():
+    from co_activation_placement_b200 import build
+    build.build()
+    import co_activation_placement_b200 as cap
+    cap.lib()
+    return cap
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(moe_[a-z_0-9]+)\s*\(", src):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for want in ["moe_coact_stats", "moe_plan_dispatch", "moe_permute", "moe_combine",
+                 "moe_shuffle_targets", "moe_rank_score", "moe_place_uniform", "moe_place_correlated"]:
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(cap):
+    lib = ctypes.CDLL(cap.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings(cap):
+    assert cap.lib().moe_status_string(0) == b"ok"
+    assert cap.lib().moe_status_string(3).startswith(b"workspace")
+
+
+@pytest.mark.parametrize("E,G", [(64, 8), (8, 4), (256, 64), (12, 12), (5, 1)])
+def test_place_uniform_matches_oracle(cap, orc, E, G):
+    assert (cap.place_uniform(E, G) == orc.place_uniform(E, G)).all()
+
+
+def test_place_uniform_rejects_uneven(cap):
+    with pytest.raises(cap.MoeError) as ei:
+        cap.place_uniform(10, 4)
+    assert ei.value.status == cap.MOE_ERR_ARG
+
+
+def test_place_capacity_matches_oracle(cap, orc):
+    rng = np.random.default_rng(0)
+    for E, G in [(64, 8), (256, 64), (13, 4)]:
+        load = rng.random(E) * rng.integers(1, 100, E)
+        load[3] = load[5]                    # a tie: lower id first
+        a, da = cap.place_capacity(load, G)
+        b, db = orc.place_capacity(load, G)
+        assert (a == b).all() and (da == db).all()
+
+
+def test_place_correlated_matches_oracle(cap, orc):
+    from synth import WORKLOADS, make_routing
+    for name in ["tiny", "one_node", "ep32"]:
+        w = WORKLOADS[name]
+        ids = make_routing(w, seed=1, T=min(w.T, 20000))
+        C = orc.coact(ids[:1], w.E, want=("coact",))["coact"][0]
+        for G, rpn in [(w.G, w.rpn), (w.G, 1), (w.G, w.G)]:
+            if G % rpn:
+                continue
+            assert (cap.place_correlated(C, G, rpn) == orc.place_correlated(C, G, rpn)).all()
+
+
+def test_place_correlated_large_matches_oracle(cap, orc):
+    rng = np.random.default_rng(1)
+    E = 256
+    C = rng.integers(0, 1000, (E, E)).astype(np.uint32)
+    C = np.triu(C, 1)
+    C = C + C.T
+    np.fill_diagonal(C, 5000 + rng.integers(0, 3, E))
+    C = C.astype(np.uint32)
+    assert (cap.place_correlated(C, 64, 8) == orc.place_correlated(C, 64, 8)).all()
+
+
+def test_workspace_queries(cap):
+    assert cap.coact_stats_workspace(8, 1 << 20, 8, 128) > 0
+    assert cap.coact_stats_workspace(1, 10, 9, 128) == 0          # k > 8
+    assert cap.plan_dispatch_workspace(131072, 8, 64, True) > cap.plan_dispatch_workspace(131072, 8, 64, False)
+    assert cap.plan_dispatch_workspace(16, 2, 65, False) == 0     # G > 64
+
+
+def test_argument_errors_return_before_device_work(cap):
+    L = cap.lib()
+    P = ctypes.c_void_p
+    fake = P(256)   # never dereferenced: each call below fails its host checks first
+    # k out of range
+    assert L.moe_coact_stats(fake, 1, 10, 9, 16, fake, None, None, fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
+    # workspace too small
+    assert L.moe_coact_stats(fake, 2, 4096, 2, 8, fake, None, None, fake, fake, 16, None) == cap.MOE_ERR_WORKSPACE
+    # G > 64, rpn not dividing G, T not a multiple of G without src_rank
+    pl = cap._Plan(256, 256, 256, 256, 256, 256, 256)
+    assert L.moe_plan_dispatch(fake, 64, 2, 8, 65, 1, fake, None, ctypes.byref(pl), fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
+    assert L.moe_plan_dispatch(fake, 64, 2, 8, 8, 3, fake, None, ctypes.byref(pl), fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
+    assert L.moe_plan_dispatch(fake, 63, 2, 8, 8, 8, fake, None, ctypes.byref(pl), fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
+    # misaligned rows / unsupported row size / bad dtype
+    assert L.moe_permute(P(264), cap.MOE_BF16, 4, 8, 2, fake, 8, fake, fake, None) == cap.MOE_ERR_ARG
+    assert L.moe_permute(fake, cap.MOE_BF16, 4, 7, 2, fake, 8, fake, fake, None) == cap.MOE_ERR_UNSUPPORTED
+    assert L.moe_combine(fake, 7, 8, 8, fake, fake, 4, 2, fake, 0, fake, None) == cap.MOE_ERR_ARG
+    assert L.moe_shuffle_targets(fake, 4, 2, 1024, 64, fake, fake, fake, None) == cap.MOE_ERR_UNSUPPORTED

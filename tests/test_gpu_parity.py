@@ -1,0 +1,353 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bit-exact: counts, Ochiai (fp64 math, one rounding on both sides), plans,
+permuted rows, rank scores, shuffle targets.  Combine: within the bound that
+follows from the arithmetic -- fp32 weight folding and FMA accumulation give
+|out - exact| <= (2k-1) 2^-24 sum_j |w_j y_j| (fp32 output; <= 1e-6 relative
+for k <= 8), plus half a bf16 ulp for bf16 output.  Full-size cases run the
+pipeline exactly as bench.py times it."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from synth import WORKLOADS, make_routing, make_gates, make_hidden, bf16_bits_to_f32
+
+pytestmark = pytest.mark.gpu
+
+U24 = 2.0 ** -24
+
+
+@pytest.fixture(scope="module")
+def cap():
+    from co_activation_placement_b200 import build
+    build.build()
+    import co_activation_placement_b200 as cap
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    cap.lib()
+    return cap
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def clustered_ids(rng, L, T, E, k, hot=0.7):
+    """k distinct ids per token; most tokens draw from a small hot set."""
+    out = np.empty((L, T, k), np.int32)
+    hotset = rng.permutation(E)[: min(E, k + 2)]
+    for l in range(L):
+        u = rng.random(T) < hot
+        pick_all = np.argsort(rng.random((T, E)), axis=1)[:, :k]
+        pick_hot = hotset[np.argsort(rng.random((T, hotset.size)), axis=1)[:, :k]]
+        out[l] = np.where(u[:, None], pick_hot, pick_all)
+    return out
+
+
+def combine_bound(Yf, idx, w, k, out_bf16, ref):
+    mag = np.einsum("tj,tjc->tc", np.abs(w.astype(np.float64)), np.abs(Yf[idx].astype(np.float64)))
+    b = (2 * k - 1) * U24 * mag * 1.0001 + 1e-30
+    if out_bf16:
+        b = b + 2.0 ** -8 * (np.abs(ref) + b)
+    return b
+
+
+# --------------------------------------------------------------- statistics
+
+STATS_SHAPES = [  # L, T, k, E
+    (1, 1, 1, 4), (2, 1000, 2, 8), (3, 4097, 3, 16), (2, 300, 8, 8), (2, 5000, 6, 64),
+    (2, 3333, 8, 128), (3, 2500, 8, 256), (2, 777, 5, 1000), (1, 12345, 4, 32),
+]
+
+
+@pytest.mark.parametrize("shape", STATS_SHAPES)
+def test_stats_small(cap, shape):
+    L, T, k, E = shape
+    rng = np.random.default_rng(sum(shape))
+    ids = clustered_ids(rng, L, T, E, k)
+    g = cap.coact_stats(dev(ids), E)
+    o = orc.coact(ids, E)
+    assert int(host(g["err"])[0]) == 0
+    assert (host(g["coact"]) == o["coact"]).all()
+    assert (host(g["ochiai"]).view(np.uint32) == o["ochiai"].view(np.uint32)).all()
+    if L > 1:
+        assert (host(g["trans"]) == o["trans"]).all()
+
+
+def test_stats_partial_outputs(cap):
+    rng = np.random.default_rng(3)
+    ids = clustered_ids(rng, 3, 2000, 4, 64)
+    o = orc.coact(ids, 64)
+    g = cap.coact_stats(dev(ids), 64, want=("trans",))
+    assert g["coact"] is None and (host(g["trans"]) == o["trans"]).all()
+    g = cap.coact_stats(dev(ids), 64, want=("ochiai",))
+    assert (host(g["ochiai"]).view(np.uint32) == o["ochiai"].view(np.uint32)).all()
+
+
+@pytest.mark.parametrize("name", ["tiny", "one_node", "ep32", "large_ep64", "stats_sweep"])
+def test_stats_workloads_full_size(cap, name):
+    w = WORKLOADS[name]
+    ids = make_routing(w)
+    g = cap.coact_stats(dev(ids), w.E)
+    o = orc.coact(ids, w.E)
+    assert int(host(g["err"])[0]) == 0
+    assert (host(g["coact"]) == o["coact"]).all()
+    assert (host(g["ochiai"]).view(np.uint32) == o["ochiai"].view(np.uint32)).all()
+    assert (host(g["trans"]) == o["trans"]).all()
+
+
+# --------------------------------------------------------------- plan
+
+PLAN_SHAPES = [  # T, k, E, G, rpn, src mode
+    (64, 1, 4, 4, 2, None), (1000, 2, 8, 4, 2, None), (4096, 2, 8, 4, 2, "rand"),
+    (5000, 3, 12, 4, 1, "rand"), (777, 8, 64, 64, 8, "rand"), (1024, 8, 256, 64, 8, None),
+    (2048, 6, 64, 32, 8, "skew"), (300, 4, 16, 1, 1, None), (999, 5, 40, 8, 4, "one"),
+    (65536, 8, 64, 8, 8, "empty"),
+]
+
+
+def make_src(rng, mode, T, G):
+    if mode is None:
+        return None
+    if mode == "rand":
+        return rng.integers(0, G, T).astype(np.int32)
+    if mode == "skew":
+        return np.minimum(rng.geometric(0.3, T) - 1, G - 1).astype(np.int32)
+    if mode == "one":
+        return np.full(T, G - 1, np.int32)
+    if mode == "empty":   # every other shard empty
+        return (2 * rng.integers(0, G // 2, T)).astype(np.int32)
+    raise ValueError(mode)
+
+
+def check_plan(p, o, T, k):
+    R = o["R"]
+    assert int(host(p.err)[0]) == 0
+    assert host(p.summary).tolist() == o["summary"].tolist()
+    assert (host(p.dest_mask)[:T] == o["dest_mask"]).all()
+    assert (host(p.counts) == o["counts"]).all()
+    assert (host(p.offsets) == o["offsets"]).all()
+    assert (host(p.row_token)[:R] == o["row_token"]).all()
+    assert (host(p.row_jmask)[:R] == o["row_jmask"]).all()
+    assert (host(p.row_of)[:T] == o["row_of"]).all()
+
+
+@pytest.mark.parametrize("shape", PLAN_SHAPES)
+def test_plan_small(cap, shape):
+    T, k, E, G, rpn, mode = shape
+    rng = np.random.default_rng(T + k + E + G)
+    ids = clustered_ids(rng, 1, T, E, k)[0]
+    e2r = rng.permutation(orc.place_uniform(E, G)).astype(np.int32)
+    src = make_src(rng, mode, T, G)
+    p = cap.plan_dispatch(dev(ids), E, G, rpn, dev(e2r), src_rank=None if src is None else dev(src))
+    check_plan(p, orc.plan(ids, E, G, rpn, e2r, src_rank=src), T, k)
+
+
+def test_plan_reuses_workspace_and_buffers(cap):
+    # the same Plan and workspace reused across calls of different sizes
+    rng = np.random.default_rng(5)
+    p = None
+    for T, src in [(4096, True), (2048, False), (4096, False), (1000, True)]:
+        ids = clustered_ids(rng, 1, T, 16, 3)[0]
+        e2r = orc.place_uniform(16, 8)
+        s = rng.integers(0, 8, T).astype(np.int32) if src else None
+        if not src and T % 8:
+            continue
+        p = cap.plan_dispatch(dev(ids), 16, 8, 4, dev(e2r), src_rank=None if s is None else dev(s))
+        check_plan(p, orc.plan(ids, 16, 8, 4, e2r, src_rank=s), T, 3)
+
+
+# --------------------------------------------------------------- rows
+
+@pytest.mark.parametrize("dtype,d,k", [("f32", 128, 2), ("bf16", 2048, 2), ("bf16", 96, 8), ("f32", 36, 5),
+                                       ("bf16", 7168, 8)])
+@pytest.mark.parametrize("out_bf16", [False, True])
+def test_permute_combine_small(cap, dtype, d, k, out_bf16):
+    rng = np.random.default_rng(d + k)
+    T, E, G = 1111 if d < 7168 else 300, 32, 8
+    ids = clustered_ids(rng, 1, T, E, k)[0]
+    e2r = rng.permutation(orc.place_uniform(E, G)).astype(np.int32)
+    src = rng.integers(0, G, T).astype(np.int32)
+    xf = rng.standard_normal((T, d)).astype(np.float32)
+    if dtype == "bf16":
+        from synth import f32_to_bf16_bits
+        xh = f32_to_bf16_bits(xf)
+        xd = dev(xh.view(np.int16)).view(torch.bfloat16)
+        xf = bf16_bits_to_f32(xh)
+    else:
+        xh, xd = xf, dev(xf)
+    p = cap.plan_dispatch(dev(ids), E, G, 4, dev(e2r), src_rank=dev(src))
+    o = orc.plan(ids, E, G, 4, e2r, src_rank=src)
+    send = cap.permute(xd, p.row_of, p.R_max, err=p.err)
+    R = o["R"]
+    got = host(send.view(torch.int16) if dtype == "bf16" else send)[:R]
+    want = orc.permute(xh, o["row_token"])
+    assert (got.view(want.dtype) == want).all()
+    # combine with identity experts (Y = send) and with a random Y
+    z = rng.standard_normal((T, k)).astype(np.float32)
+    wts = (np.exp(z) / np.exp(z).sum(1, keepdims=True)).astype(np.float32)
+    out = cap.combine(send, p.row_of, dev(wts), out_dtype=torch.bfloat16 if out_bf16 else torch.float32, err=p.err)
+    outf = host(out.float())
+    Yf = orc.permute(xf, o["row_token"])
+    ref = orc.combine(Yf, o["row_of"], wts, y_is_bf16=False)
+    assert (np.abs(outf - ref) <= combine_bound(Yf, o["row_of"], wts, k, out_bf16, ref)).all()
+    if out_bf16 and dtype == "bf16":
+        assert (host(out.view(torch.int16)).view(np.uint16) == xh).all()   # identity round trip is exact
+    idx = rng.integers(0, R, (T, k)).astype(np.int32)
+    idx[:, -1] = idx[:, 0]                                                # repeated rows fold their weights
+    out2 = cap.combine(send, dev(idx), dev(wts), out_dtype=torch.float32, err=p.err)
+    ref2 = orc.combine(Yf, idx, wts, y_is_bf16=False)
+    assert (np.abs(host(out2) - ref2) <= combine_bound(Yf, idx, wts, k, False, ref2)).all()
+    assert int(host(p.err)[0]) == 0
+
+
+# --------------------------------------------------------------- shuffle
+
+@pytest.mark.parametrize("T,k,E,G", [(1000, 2, 8, 4), (4097, 8, 256, 64), (3000, 6, 64, 32), (500, 1, 16, 1)])
+def test_shuffle_small(cap, T, k, E, G):
+    rng = np.random.default_rng(T + G)
+    ids = clustered_ids(rng, 2, T, E, k)
+    st = orc.coact(ids, E)
+    e2r = rng.permutation(orc.place_uniform(E, G)).astype(np.int32)
+    rs = cap.rank_score(dev(st["trans"][0]), dev(e2r), G)
+    rs_o = orc.rank_score(st["trans"][0], e2r, G)
+    assert (host(rs) == rs_o).all()
+    tg = cap.shuffle_targets(dev(ids[0]), E, G, rs)
+    assert (host(tg)[:T] == orc.shuffle_targets(ids[0], E, G, rs_o)).all()
+    # ties: an all-zero table sends every token to rank 0
+    z = cap.shuffle_targets(dev(ids[0]), E, G, dev(np.zeros((E, G), np.uint32)))
+    assert (host(z)[:T] == 0).all()
+
+
+# --------------------------------------------------------------- full pipeline
+
+ROW_WORKLOADS = ["tiny", "one_node", "ep32", "large_ep64"]
+
+
+@pytest.mark.parametrize("name", ROW_WORKLOADS)
+@pytest.mark.parametrize("placement,shuffle", [("correlated", True), ("uniform", False)])
+def test_pipeline_full_size(cap, name, placement, shuffle):
+    from co_activation_placement_b200 import pipeline
+    w = WORKLOADS[name]
+    if name in ("ep32", "large_ep64") and placement == "uniform":
+        pytest.skip("uniform placement at this size is covered by the plan checks of the correlated run")
+    ids = make_routing(w)
+    ids_cal = make_routing(w, seed=w.seed + 1)
+    gates = make_gates(w)
+    x = make_hidden(w)
+    hp = pipeline.prepare(w.E, w.G, w.rpn, ids, gates, x, w.dtype, ids_cal, placement=placement,
+                          shuffle=shuffle, out_dtype=torch.float32)
+    hp.step()
+    torch.cuda.synchronize()
+    assert int(host(hp.err)[0]) == 0
+    # statistics
+    o = orc.coact(ids, w.E)
+    assert (host(hp.stats["coact"]) == o["coact"]).all()
+    assert (host(hp.stats["ochiai"]).view(np.uint32) == o["ochiai"].view(np.uint32)).all()
+    assert (host(hp.stats["trans"]) == o["trans"]).all()
+    # calibration: placement and rank scores from the oracle's own statistics
+    oc = orc.coact(ids_cal, w.E)
+    e2r_o = [orc.place_correlated(oc["coact"][l], w.G, w.rpn) if placement == "correlated"
+             else orc.place_uniform(w.E, w.G) for l in range(w.L)]
+    for l in range(w.L):
+        assert (host(hp.e2r[l]) == e2r_o[l]).all()
+    rs_o = [orc.rank_score(oc["trans"][l], e2r_o[l + 1], w.G) for l in range(w.L - 1)] if shuffle else []
+    for a, b in zip(hp.rank_scores, rs_o):
+        assert (host(a) == b).all()
+    xf = bf16_bits_to_f32(x) if w.dtype == "bf16" else x
+    rng = np.random.default_rng(0)
+    src = None
+    for l in range(w.L):
+        op = orc.plan(ids[l], w.E, w.G, w.rpn, e2r_o[l], src_rank=src)
+        check_plan(hp.plans[l], op, w.T, w.k)
+        R = op["R"]
+        # rows: sampled against the oracle's permute
+        rows = np.unique(np.concatenate([rng.integers(0, R, 4096), [0, R - 1]]))
+        sub = host(hp.send[torch.from_numpy(rows).cuda()].view(torch.int16 if w.dtype == "bf16" else torch.float32))
+        want = orc.permute(x, op["row_token"][rows])
+        assert (sub.view(want.dtype) == want).all()
+        # combine: sampled tokens against the oracle's fp64 combine
+        toks = np.unique(np.concatenate([rng.integers(0, w.T, 1024), [0, w.T - 1]]))
+        idx = op["row_of"][toks]
+        need, inv = np.unique(idx, return_inverse=True)
+        Ysub = orc.permute(xf, op["row_token"][need])
+        ref = orc.combine(Ysub, inv.reshape(idx.shape).astype(np.int32), gates[l][toks], y_is_bf16=False)
+        got = host(hp.outs[l][torch.from_numpy(toks).cuda()])
+        bound = combine_bound(Ysub, inv.reshape(idx.shape), gates[l][toks], w.k, False, ref)
+        assert (np.abs(got - ref) <= bound).all()
+        rel = np.abs(got - ref) / np.maximum(np.abs(ref), 1e-30)
+        assert np.median(rel) < 1e-6
+        # any size: identity experts give out = x * sum_j w  (every token)
+        if l == w.L - 1:
+            outf = host(hp.outs[l])
+            np.testing.assert_allclose(outf, xf * gates[l].sum(-1, dtype=np.float64)[:, None], rtol=1e-6, atol=1e-30)
+        if shuffle and l + 1 < w.L:
+            tg = orc.shuffle_targets(ids[l], w.E, w.G, rs_o[l])
+            assert (host(hp.targets[l]) == tg).all()
+            src = tg
+    # determinism: a second step reproduces every output bit for bit
+    first = [host(p.row_of).copy() for p in hp.plans] + [host(hp.outs[-1]).copy()]
+    hp.step()
+    again = [host(p.row_of) for p in hp.plans] + [host(hp.outs[-1])]
+    for a, b in zip(first, again):
+        assert (a.view(np.uint8) == b.view(np.uint8)).all()
+
+
+# --------------------------------------------------------------- edge cases / errors
+
+def test_empty_batch(cap):
+    ids = torch.empty((2, 0, 2), dtype=torch.int32, device="cuda")
+    g = cap.coact_stats(ids, 8)
+    assert (host(g["coact"]) == 0).all() and (host(g["trans"]) == 0).all() and (host(g["ochiai"]) == 0).all()
+    p = cap.plan_dispatch(ids[0], 8, 4, 2, dev(orc.place_uniform(8, 4)))
+    assert (host(p.summary) == 0).all() and (host(p.offsets) == 0).all() and (host(p.counts) == 0).all()
+
+
+def test_data_errors_are_reported_not_trapped(cap):
+    E, G = 16, 4
+    good = np.array([[[0, 1], [2, 3], [4, 5], [6, 7]]], np.int32)
+    for bad_val, code in [(16, cap.DERR_ID_RANGE), (-3, cap.DERR_ID_RANGE)]:
+        ids = good.copy(); ids[0, 2, 1] = bad_val
+        assert int(host(cap.coact_stats(dev(ids), E)["err"])[0]) == code
+        p = cap.plan_dispatch(dev(ids[0]), E, G, 2, dev(orc.place_uniform(E, G)))
+        assert int(host(p.err)[0]) == code
+    ids = good.copy(); ids[0, 1] = [3, 3]
+    assert int(host(cap.coact_stats(dev(ids), E)["err"])[0]) == cap.DERR_ID_REPEAT
+    assert int(host(cap.plan_dispatch(dev(ids[0]), E, G, 2, dev(orc.place_uniform(E, G))).err)[0]) == cap.DERR_ID_REPEAT
+    e2r = orc.place_uniform(E, G); e2r[5] = 9
+    assert int(host(cap.plan_dispatch(dev(good[0]), E, G, 2, dev(e2r)).err)[0]) == cap.DERR_RANK_RANGE
+    src = np.array([0, 1, 7, 2], np.int32)
+    assert int(host(cap.plan_dispatch(dev(good[0]), E, G, 2, dev(orc.place_uniform(E, G)), src_rank=dev(src)).err)[0]) \
+        == cap.DERR_RANK_RANGE
+    x = torch.zeros((4, 8), dtype=torch.float32, device="cuda")
+    row_of = dev(np.array([[0, 1], [2, 3], [4, 99], [6, 7]], np.int32))
+    err = cap.new_err("cuda")
+    cap.permute(x, row_of, 8, err=err)
+    assert int(host(err)[0]) == cap.DERR_ROW_RANGE
+    err = cap.new_err("cuda")
+    cap.combine(torch.zeros((8, 8), device="cuda"), row_of, dev(np.ones((4, 2), np.float32)), err=err)
+    assert int(host(err)[0]) == cap.DERR_ROW_RANGE
+    err = cap.new_err("cuda")
+    cap.shuffle_targets(dev(np.array([[0, 20]], np.int32)), E, G, dev(np.zeros((E, G), np.uint32)), err=err)
+    assert int(host(err)[0]) == cap.DERR_ID_RANGE
+    # the context is still usable after every reported error
+    assert int(host(cap.coact_stats(dev(good), E)["err"])[0]) == 0
+
+
+def test_argument_errors_enqueue_nothing(cap):
+    x = torch.zeros((4, 7), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cap.MoeError) as ei:
+        cap.permute(x, dev(np.zeros((4, 2), np.int32)), 8)
+    assert ei.value.status == cap.MOE_ERR_UNSUPPORTED
+    with pytest.raises(cap.MoeError) as ei:
+        cap.plan_dispatch(dev(np.zeros((10, 2), np.int32)), 8, 4, 2, dev(orc.place_uniform(8, 4)))
+    assert ei.value.status == cap.MOE_ERR_ARG     # 4 does not divide 10 without src_rank
+    before = cap.launch_count()
+    with pytest.raises(cap.MoeError):
+        cap.coact_stats(dev(np.zeros((1, 4, 9), np.int32)), 16)
+    assert cap.launch_count() == before
