@@ -62,8 +62,30 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--sweep-only", action="store_true", help="only the co-activation statistics sweep")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle time for the CPU baseline")
     return ap.parse_args()
+
+
+def rank_seed(w, rank):
+    """Each rank draws its own batch (weak scaling); the cluster layout (the
+    stand-in for the trained router) is the workload's, shared by all ranks."""
+    return w.seed + 1000 * rank
+
+
+def reduce_max(x, pg, device):
+    """Max over ranks of a per-rank time (the only collective in the bench)."""
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(world, bytes_per_rank, ms_step):
+    """Whole-job GB/s: all ranks' bytes over the slowest rank's step time."""
+    return world * bytes_per_rank / (ms_step * 1e-3) / 1e9
 
 
 def dist_env():
@@ -270,7 +292,15 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
         pg = dist
-    seed = w.seed + 1000 * rank
+    seed = rank_seed(w, rank)
+    if a.sweep_only:
+        hbm, _ = peaks()
+        sweep = run_sweep(cap, pipeline, device, seed, a.steps, a.warmup, hbm, pg)
+        if rank == 0:
+            print(json.dumps({"coact_sweep": sweep}), flush=True)
+        if pg is not None:
+            pg.destroy_process_group()
+        return
     shuffle = (not a.no_shuffle) and w.L > 1
     out_dtype = torch.float32 if a.out_dtype == "f32" else torch.bfloat16
     if w.d == 0:
@@ -318,14 +348,11 @@ def main():
     hp.reset_events()
     ms_total = start.elapsed_time(stop)
     ms_step = ms_total / a.steps
-    if pg is not None:
-        t = torch.tensor([ms_step], device=device, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = reduce_max(ms_step, pg, device)
     clocks = clk.summary()
 
     hbm, hbm_kind = peaks()
-    value = world * sb.dispatch_combine / (ms_step * 1e-3) / 1e9
+    value = weak_value(world, sb.dispatch_combine, ms_step)
     kern = {}
     bytes_of = {"stats": sb.stats, "plan": sb.plan, "permute": sb.permute, "combine": sb.combine,
                 "shuffle": sb.shuffle}
@@ -413,11 +440,7 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
         e.record()
         torch.cuda.synchronize()
         tot += s.elapsed_time(e)
-    ms = tot / n
-    if pg is not None:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(tot / n, pg, device)
     nbytes = hp.step_bytes(None).stats
     world = pg.get_world_size() if pg is not None else 1
     return {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "L": w.L, "ms": ms,
@@ -463,15 +486,11 @@ def run_e2e(hp, ids, gates, x, w, a, device, sb, pg, world):
         one()
     e.record()
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / n
-    if pg is not None:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(s.elapsed_time(e) / n, pg, device)
     hp.timers = True
     h2d = ids_h.numel() * 4 + gates_h.numel() * 4 + x_h.numel() * x_h.element_size()
     d2h = out_h.numel() * out_h.element_size() + sum(v.numel() * v.element_size() for v in st_h.values()) + sum_h.numel() * 8
-    return {"value": world * sb.dispatch_combine / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+    return {"value": weak_value(world, sb.dispatch_combine, ms), "unit": "GB/s", "ms_per_step": ms,
             "steps": n, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 

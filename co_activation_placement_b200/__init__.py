@@ -24,7 +24,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoecoact.so")
 
 MOE_OK, MOE_ERR_ARG, MOE_ERR_DATA, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_UNSUPPORTED = range(6)
-DERR_ID_RANGE, DERR_ID_REPEAT, DERR_RANK_RANGE, DERR_ROW_RANGE = 1, 2, 3, 4
+DERR_ID_RANGE, DERR_ID_REPEAT, DERR_RANK_RANGE, DERR_ROW_RANGE, DERR_TIMEOUT = 1, 2, 3, 4, 5
 MOE_F32, MOE_BF16 = 0, 1
 
 _lib = None

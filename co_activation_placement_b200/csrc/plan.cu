@@ -26,7 +26,7 @@
 namespace moe {
 namespace {
 
-constexpr int kChunk = 256;   // tokens per block, one per thread
+constexpr int kChunk = 1024;  // tokens per block, one per thread
 constexpr int kWarps = kChunk / 32;
 
 struct PlanWsHeader {
@@ -119,9 +119,16 @@ __device__ void scan_columns(const int32_t *tab, int32_t *pref, int B, int G, in
     const int d = threadIdx.x % G, q = threadIdx.x / G;
     const int per = (B + nseg - 1) / nseg;
     const int b0 = min(B, q * per), b1 = min(B, b0 + per);
+    constexpr int kBatch = 8;          // independent L2 loads in flight per thread
     if (q < nseg) {
         int s = 0;
-        for (int b = b0; b < b1; ++b) s += __ldcg(tab + (size_t)b * G + d);
+        for (int b = b0; b < b1; b += kBatch) {
+            int v[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) v[i] = b + i < b1 ? __ldcg(tab + (size_t)(b + i) * G + d) : 0;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) s += v[i];
+        }
         seg_sh[q * G + d] = s;
     }
     __syncthreads();
@@ -137,9 +144,16 @@ __device__ void scan_columns(const int32_t *tab, int32_t *pref, int B, int G, in
     __syncthreads();
     if (q < nseg) {
         int run = seg_sh[q * G + d];
-        for (int b = b0; b < b1; ++b) {
-            pref[(size_t)b * G + d] = run;
-            run += __ldcg(tab + (size_t)b * G + d);
+        for (int b = b0; b < b1; b += kBatch) {
+            int v[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) v[i] = b + i < b1 ? __ldcg(tab + (size_t)(b + i) * G + d) : 0;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                if (b + i < b1) {
+                    pref[(size_t)(b + i) * G + d] = run;
+                    run += v[i];
+                }
         }
     }
     if (threadIdx.x < G) pref[(size_t)B * G + threadIdx.x] = tot_sh[threadIdx.x];

@@ -5,14 +5,19 @@
 // "Training Communication-Efficient MoE ...", footnote 3: the dispatcher moves
 // hidden states (and routed probabilities), the combine is the inverse.
 //
-// Both kernels are HBM streams with 16-byte vectors; nothing here is a dense
-// contraction.  Both are token-major: one warp owns one token at a time.
-//  - permute reads the token's row of x once and writes it to each of its
-//    distinct send rows (row_of[t][j], duplicates skipped), so HBM traffic is
-//    T_active*rowB read + R*rowB written -- the minimum.
-//  - combine reads each distinct row a token names once, sums the weights of
-//    repeated rows in j order, and accumulates the distinct rows with fp32
-//    FMAs in order of first appearance; traffic is U*rowB + T*rowB_out.
+// Both kernels are HBM streams of 32-byte vectors (the 256-bit
+// ld/st.global.v8 forms; 16-byte vectors when a row or pointer is not 32-byte
+// aligned); nothing here is a dense contraction.  Both are token-major: one
+// warp owns one token at a time.
+//  - permute reads the token's row of x once (4 vectors per lane in flight)
+//    and writes it to each of its distinct send rows (row_of[t][j], duplicates
+//    skipped), so HBM traffic is T_active*rowB read + R*rowB written -- the
+//    minimum.  (A variant staging rows in shared memory with bulk async copies
+//    measured 2% slower on B200 for 4-14 KB rows and was dropped.)
+//  - combine folds the weights of repeated rows in j order (lane-parallel
+//    across the token's k picks), compacts the distinct rows, loads them all
+//    before accumulating with fp32 FMAs in order of first appearance; traffic
+//    is U*rowB + T*rowB_out.
 // Loads and stores use the streaming (evict-first) cache hint: every byte is
 // touched once.  Grids are persistent: a multiple of the SM count.
 #include <algorithm>
@@ -26,9 +31,6 @@ namespace {
 
 constexpr int kRowThreads = 256;
 constexpr int kRowBlocksPerSM = 8;
-
-__device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
-__device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v) { __stcs(p, v); }
 
 // Warp-uniform per-token row list: dst[j] and a bitmask of the j that are the
 // first occurrence of a valid row.  Returns false (after recording the error)
@@ -55,124 +57,195 @@ __device__ __forceinline__ bool token_rows(const int32_t *__restrict__ idx, int 
     return ok;
 }
 
-template <int K, int U>
+template <int K, int U, int VB>
 __global__ void __launch_bounds__(kRowThreads)
-permute_kernel(const uint4 *__restrict__ x, int nvec, int T, const int32_t *__restrict__ row_of,
-               long long R_max, uint4 *__restrict__ send, int32_t *err)
+permute_kernel(const char *__restrict__ x, int nvec, int T, const int32_t *__restrict__ row_of,
+               long long R_max, char *__restrict__ send, int32_t *err);
+
+// One vector of VB bytes (16 or 32) as 32-bit words, moved with streaming
+// (evict-first) loads and stores; 32-byte vectors use the 256-bit forms.
+template <int VB> struct Vw { uint32_t w[VB / 4]; };
+
+template <int VB>
+__device__ __forceinline__ Vw<VB> ld_vec(const void *p)
+{
+    Vw<VB> v;
+    if constexpr (VB == 16) {
+        const uint4 a = __ldcs(static_cast<const uint4 *>(p));
+        v.w[0] = a.x; v.w[1] = a.y; v.w[2] = a.z; v.w[3] = a.w;
+    } else {
+        asm volatile("ld.global.cs.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]),
+                       "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+                     : "l"(p));
+    }
+    return v;
+}
+
+template <int NW>
+__device__ __forceinline__ void st_words(void *p, const uint32_t (&w)[NW])
+{
+    // NW words at p: 8-word (32 B) pieces first, then 4, then 2
+    static_assert(NW % 2 == 0, "even word count");
+    uint32_t *q = static_cast<uint32_t *>(p);
+    int o = 0;
+#pragma unroll
+    for (; o + 8 <= NW; o += 8)
+        asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                     ::"l"(q + o), "r"(w[o]), "r"(w[o + 1]), "r"(w[o + 2]), "r"(w[o + 3]),
+                       "r"(w[o + 4]), "r"(w[o + 5]), "r"(w[o + 6]), "r"(w[o + 7])
+                     : "memory");
+#pragma unroll
+    for (; o + 4 <= NW; o += 4) __stcs(reinterpret_cast<uint4 *>(q + o), make_uint4(w[o], w[o + 1], w[o + 2], w[o + 3]));
+#pragma unroll
+    for (; o + 2 <= NW; o += 2) __stcs(reinterpret_cast<uint2 *>(q + o), make_uint2(w[o], w[o + 1]));
+}
+
+// Permute with VB-byte vectors: a warp reads a token's row once, U vectors
+// per lane in flight, and writes them to each of the token's distinct rows.
+template <int K, int U, int VB>
+__global__ void __launch_bounds__(kRowThreads)
+permute_kernel(const char *__restrict__ x, int nvec, int T, const int32_t *__restrict__ row_of,
+               long long R_max, char *__restrict__ send, int32_t *err)
 {
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (kRowThreads / 32);
+    const size_t rowB = (size_t)nvec * VB;
     for (int t = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); t < T; t += nwarps) {
         int dst[K];
         unsigned keep;
         token_rows<K>(row_of, t, R_max, dst, keep, err);
-        const uint4 *src = x + (size_t)t * nvec;
+        const char *src = x + (size_t)t * rowB;
         for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
-            uint4 buf[U];
+            Vw<VB> buf[U];
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                if (v0 + 32 * u < nvec) buf[u] = ld_stream(src + v0 + 32 * u);
+                if (v0 + 32 * u < nvec) buf[u] = ld_vec<VB>(src + (size_t)(v0 + 32 * u) * VB);
 #pragma unroll
             for (int j = 0; j < K; ++j) {
                 if (!((keep >> j) & 1u)) continue;
-                uint4 *o = send + (size_t)dst[j] * nvec;
+                char *o = send + (size_t)dst[j] * rowB;
 #pragma unroll
                 for (int u = 0; u < U; ++u)
-                    if (v0 + 32 * u < nvec) st_stream(o + v0 + 32 * u, buf[u]);
+                    if (v0 + 32 * u < nvec) st_words<VB / 4>(o + (size_t)(v0 + 32 * u) * VB, buf[u].w);
             }
         }
     }
 }
 
-// Element access for one 16-byte vector of Y.
-template <typename YT> struct Vec;
-template <> struct Vec<float> {
-    static constexpr int N = 4;
-    __device__ static __forceinline__ float get(const uint4 &v, int e)
-    {
-        const unsigned w = e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
-        return __uint_as_float(w);
-    }
+// Element e of a vector of Y.
+template <typename YT> struct Elem;
+template <> struct Elem<float> {
+    static constexpr int BYTES = 4;
+    template <int NW> __device__ static __forceinline__ float get(const uint32_t (&w)[NW], int e) { return __uint_as_float(w[e]); }
 };
-template <> struct Vec<__nv_bfloat16> {
-    static constexpr int N = 8;
-    __device__ static __forceinline__ float get(const uint4 &v, int e)
+template <> struct Elem<__nv_bfloat16> {
+    static constexpr int BYTES = 2;
+    template <int NW> __device__ static __forceinline__ float get(const uint32_t (&w)[NW], int e)
     {
-        const unsigned w = (e >> 1) == 0 ? v.x : (e >> 1) == 1 ? v.y : (e >> 1) == 2 ? v.z : v.w;
-        return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+        const uint32_t x = w[e >> 1];
+        return __uint_as_float((e & 1) ? (x & 0xffff0000u) : (x << 16));
     }
 };
 
-template <int N, bool OUT_BF16>
-__device__ __forceinline__ void store_out(void *out, size_t elem, const float (&a)[N])
+// A token's distinct rows, compacted: lane j < K holds pick j's row and
+// weight; a pick that repeats an earlier pick's row adds its weight to that
+// earlier lane (in j order) and drops out.  Returns the number of distinct
+// valid rows U; the q-th of them (in order of first appearance) is
+// (shfl(row, src[q]), shfl(W, src[q])).
+template <int K>
+__device__ __forceinline__ int token_distinct(const int32_t *__restrict__ idx, const float *__restrict__ w, int t,
+                                              long long R_max, int &row, float &W, int (&src)[K], int32_t *err)
 {
-    if constexpr (!OUT_BF16) {
-        float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + elem);
+    const int lane = threadIdx.x & 31;
+    row = lane < K ? __ldg(idx + (size_t)t * K + lane) : -1;
+    const float wl = lane < K ? __ldg(w + (size_t)t * K + lane) : 0.f;
+    const bool valid = lane < K && row >= 0 && (long long)row < R_max;
+    if (__any_sync(0xffffffffu, lane < K && !valid) && lane == 0) record_error(err, MOE_DERR_ROW_RANGE);
+    bool first = valid;
+    W = wl;
 #pragma unroll
-        for (int q = 0; q < N / 4; ++q) __stcs(o + q, make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]));
-    } else {
-        unsigned w[N / 2];
-#pragma unroll
-        for (int q = 0; q < N / 2; ++q) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * q], a[2 * q + 1]);
-            w[q] = *reinterpret_cast<unsigned *>(&h);
-        }
-        __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(out) + elem;
-        if constexpr (N == 8) __stcs(reinterpret_cast<uint4 *>(ob), make_uint4(w[0], w[1], w[2], w[3]));
-        else __stcs(reinterpret_cast<uint2 *>(ob), make_uint2(w[0], w[1]));
+    for (int j = 0; j < K; ++j) {
+        const int rj = __shfl_sync(0xffffffffu, row, j);
+        const float wj = __shfl_sync(0xffffffffu, wl, j);
+        if (j < lane && rj == row) first = false;
+        if (j > lane && rj == row) W = __fadd_rn(W, wj);
     }
+    unsigned m = __ballot_sync(0xffffffffu, first);
+    const int U = __popc(m);
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+        src[q] = m ? __ffs(m) - 1 : 0;
+        m &= m - 1;
+    }
+    return U;
 }
 
-template <int K, int U, typename YT, bool OUT_BF16>
+// Vectors are VB bytes of Y (N elements).  Distinct rows are read in chunks
+// of CH rows; U vectors per lane are in flight per row.
+template <int K, int CH, int U, typename YT, bool OUT_BF16, int VB>
 __global__ void __launch_bounds__(kRowThreads)
-combine_kernel(const uint4 *__restrict__ Y, int nvec, long long R_max, const int32_t *__restrict__ idx,
+combine_kernel(const char *__restrict__ Y, int nvec, long long R_max, const int32_t *__restrict__ idx,
                const float *__restrict__ w, int T, void *__restrict__ out, int32_t *err)
 {
-    constexpr int N = Vec<YT>::N;
+    constexpr int N = VB / Elem<YT>::BYTES;
+    constexpr int OW = OUT_BF16 ? N / 2 : N;          // output words per vector
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (kRowThreads / 32);
+    const size_t rowB = (size_t)nvec * VB;
     for (int t = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); t < T; t += nwarps) {
-        int row[K];
-        unsigned keep;
-        token_rows<K>(idx, t, R_max, row, keep, err);
-        const float wm = lane < K ? __ldg(w + (size_t)t * K + lane) : 0.f;
-        float W[K];
+        int row, src[K];
+        float Wl;
+        const int Ut = token_distinct<K>(idx, w, t, R_max, row, Wl, src, err);
+        int rc[K];
+        float Wc[K];
 #pragma unroll
-        for (int j = 0; j < K; ++j) W[j] = 0.f;
-        // fold the weights of repeated rows onto their first occurrence, in j order
-#pragma unroll
-        for (int j = 0; j < K; ++j) {
-            const float wj = __shfl_sync(0xffffffffu, wm, j);
-            bool placed = false;
-#pragma unroll
-            for (int q = 0; q < j; ++q) {
-                const bool hit = !placed && ((keep >> q) & 1u) && row[q] == row[j];
-                if (hit) W[q] = __fadd_rn(W[q], wj);
-                placed |= hit;
-            }
-            if ((keep >> j) & 1u) W[j] = wj;
+        for (int q = 0; q < K; ++q) {
+            rc[q] = __shfl_sync(0xffffffffu, row, src[q]);
+            Wc[q] = __shfl_sync(0xffffffffu, Wl, src[q]);
         }
+        char *ob = static_cast<char *>(out) + (size_t)t * nvec * (OW * 4);
         for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
-            uint4 y[U][K];
+            float acc[U][N];
 #pragma unroll
             for (int u = 0; u < U; ++u)
 #pragma unroll
-                for (int j = 0; j < K; ++j)
-                    if (((keep >> j) & 1u) && v0 + 32 * u < nvec)
-                        y[u][j] = ld_stream(Y + (size_t)row[j] * nvec + v0 + 32 * u);
+                for (int e = 0; e < N; ++e) acc[u][e] = 0.f;
+#pragma unroll
+            for (int c0 = 0; c0 < K; c0 += CH) {
+                if (c0 >= Ut) break;
+                Vw<VB> y[CH][U];
+#pragma unroll
+                for (int c = 0; c < CH; ++c)
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+                        if (c0 + c < K && c0 + c < Ut && v0 + 32 * u < nvec)
+                            y[c][u] = ld_vec<VB>(Y + (size_t)rc[c0 + c] * rowB + (size_t)(v0 + 32 * u) * VB);
+#pragma unroll
+                for (int c = 0; c < CH; ++c) {
+                    if (c0 + c >= K || c0 + c >= Ut) break;
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+#pragma unroll
+                        for (int e = 0; e < N; ++e)
+                            acc[u][e] = __fmaf_rn(Wc[c0 + c], Elem<YT>::get(y[c][u].w, e), acc[u][e]);
+                }
+            }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (v0 + 32 * u >= nvec) break;
-                float acc[N];
+                uint32_t o[OW];
+                if constexpr (OUT_BF16) {
 #pragma unroll
-                for (int e = 0; e < N; ++e) acc[e] = 0.f;
+                    for (int q = 0; q < OW; ++q) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(acc[u][2 * q], acc[u][2 * q + 1]);
+                        o[q] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                } else {
 #pragma unroll
-                for (int j = 0; j < K; ++j) {
-                    if (!((keep >> j) & 1u)) continue;
-#pragma unroll
-                    for (int e = 0; e < N; ++e) acc[e] = __fmaf_rn(W[j], Vec<YT>::get(y[u][j], e), acc[e]);
+                    for (int q = 0; q < OW; ++q) o[q] = __float_as_uint(acc[u][q]);
                 }
-                store_out<N, OUT_BF16>(out, ((size_t)t * nvec + v0 + 32 * u) * N, acc);
+                st_words<OW>(ob + (size_t)(v0 + 32 * u) * (OW * 4), o);
             }
         }
     }
@@ -186,40 +259,64 @@ int row_grid(long long T)
 }
 
 template <int K>
-moe_status launch_permute(const void *x, int nvec, int T, const int32_t *row_of, long long R_max, void *send,
+moe_status launch_permute(const void *x, size_t rowB, int T, const int32_t *row_of, long long R_max, void *send,
                           int32_t *err, cudaStream_t s)
 {
-    permute_kernel<K, 4><<<row_grid(T), kRowThreads, 0, s>>>(static_cast<const uint4 *>(x), nvec, T, row_of, R_max,
-                                                             static_cast<uint4 *>(send), err);
+    const char *xb = static_cast<const char *>(x);
+    char *sb = static_cast<char *>(send);
+    if (rowB % 32 == 0 && (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (reinterpret_cast<uintptr_t>(send) & 31u) == 0)
+        permute_kernel<K, 4, 32><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 32), T, row_of, R_max, sb, err);
+    else
+        permute_kernel<K, 4, 16><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 16), T, row_of, R_max, sb, err);
     return launch_status();
 }
 
+// Combine tuning, measured on B200 at d = 7168 bf16, k = 8: one vector per
+// lane in flight per distinct row, all distinct rows loaded before the FMAs
+// (chunk = k), 32-byte vectors.
+constexpr int kCombineU = 1;
+constexpr int kCombineChunk = 8;
+
+template <int K, typename YT, int VB>
+moe_status launch_combine_vb(const void *Y, int nvec, long long R_max, const int32_t *idx, const float *w, int T,
+                             void *out, bool out_bf16, int32_t *err, cudaStream_t s)
+{
+    constexpr int U = kCombineU;
+    constexpr int CH = K < kCombineChunk ? K : kCombineChunk;
+    const char *y = static_cast<const char *>(Y);
+    if (out_bf16)
+        combine_kernel<K, CH, U, YT, true, VB><<<row_grid(T), kRowThreads, 0, s>>>(y, nvec, R_max, idx, w, T, out, err);
+    else
+        combine_kernel<K, CH, U, YT, false, VB><<<row_grid(T), kRowThreads, 0, s>>>(y, nvec, R_max, idx, w, T, out, err);
+    return launch_status();
+}
+
+// 32-byte vectors when Y and out are 32-byte aligned and rows split evenly
+// into them (out rows are at least as long as Y rows), else 16-byte vectors.
 template <int K, typename YT>
-moe_status launch_combine(const void *Y, int nvec, long long R_max, const int32_t *idx, const float *w, int T,
+moe_status launch_combine(const void *Y, size_t rowB, long long R_max, const int32_t *idx, const float *w, int T,
                           void *out, bool out_bf16, int32_t *err, cudaStream_t s)
 {
-    constexpr int U = K <= 4 ? 2 : 1;
-    const uint4 *y = static_cast<const uint4 *>(Y);
-    if (out_bf16)
-        combine_kernel<K, U, YT, true><<<row_grid(T), kRowThreads, 0, s>>>(y, nvec, R_max, idx, w, T, out, err);
-    else
-        combine_kernel<K, U, YT, false><<<row_grid(T), kRowThreads, 0, s>>>(y, nvec, R_max, idx, w, T, out, err);
-    return launch_status();
+    const bool v32 = rowB % 32 == 0 && (reinterpret_cast<uintptr_t>(Y) & 31u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(out) & 31u) == 0 &&
+                     (out_bf16 ? (sizeof(YT) == 2 || rowB % 64 == 0) : true);
+    if (v32) return launch_combine_vb<K, YT, 32>(Y, (int)(rowB / 32), R_max, idx, w, T, out, out_bf16, err, s);
+    return launch_combine_vb<K, YT, 16>(Y, (int)(rowB / 16), R_max, idx, w, T, out, out_bf16, err, s);
 }
 
 template <typename YT>
-moe_status dispatch_combine_k(int k, const void *Y, int nvec, long long R_max, const int32_t *idx, const float *w,
+moe_status dispatch_combine_k(int k, const void *Y, size_t rowB, long long R_max, const int32_t *idx, const float *w,
                               int T, void *out, bool out_bf16, int32_t *err, cudaStream_t s)
 {
     switch (k) {
-    case 1: return launch_combine<1, YT>(Y, nvec, R_max, idx, w, T, out, out_bf16, err, s);
-    case 2: return launch_combine<2, YT>(Y, nvec, R_max, idx, w, T, out, out_bf16, err, s);
-    case 3: return launch_combine<3, YT>(Y, nvec, R_max, idx, w, T, out, out_bf16, err, s);
-    case 4: return launch_combine<4, YT>(Y, nvec, R_max, idx, w, T, out, out_bf16, err, s);
-    case 5: return launch_combine<5, YT>(Y, nvec, R_max, idx, w, T, out, out_bf16, err, s);
-    case 6: return launch_combine<6, YT>(Y, nvec, R_max, idx, w, T, out, out_bf16, err, s);
-    case 7: return launch_combine<7, YT>(Y, nvec, R_max, idx, w, T, out, out_bf16, err, s);
-    case 8: return launch_combine<8, YT>(Y, nvec, R_max, idx, w, T, out, out_bf16, err, s);
+    case 1: return launch_combine<1, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 2: return launch_combine<2, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 3: return launch_combine<3, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 4: return launch_combine<4, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 5: return launch_combine<5, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 6: return launch_combine<6, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 7: return launch_combine<7, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 8: return launch_combine<8, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
     }
     return MOE_ERR_ARG;
 }
@@ -241,17 +338,16 @@ extern "C" moe_status moe_permute(const void *x, moe_dtype dtype, int T, int d, 
     if (!x || !row_of || !send || !aligned16(x) || !aligned16(send)) return MOE_ERR_ARG;
     const size_t rowB = eb * (size_t)d;
     if (rowB % 16) return MOE_ERR_UNSUPPORTED;
-    const int nvec = (int)(rowB / 16);
     moe_status st = MOE_ERR_ARG;
     switch (k) {
-    case 1: st = launch_permute<1>(x, nvec, T, row_of, R_max, send, err, stream); break;
-    case 2: st = launch_permute<2>(x, nvec, T, row_of, R_max, send, err, stream); break;
-    case 3: st = launch_permute<3>(x, nvec, T, row_of, R_max, send, err, stream); break;
-    case 4: st = launch_permute<4>(x, nvec, T, row_of, R_max, send, err, stream); break;
-    case 5: st = launch_permute<5>(x, nvec, T, row_of, R_max, send, err, stream); break;
-    case 6: st = launch_permute<6>(x, nvec, T, row_of, R_max, send, err, stream); break;
-    case 7: st = launch_permute<7>(x, nvec, T, row_of, R_max, send, err, stream); break;
-    case 8: st = launch_permute<8>(x, nvec, T, row_of, R_max, send, err, stream); break;
+    case 1: st = launch_permute<1>(x, rowB, T, row_of, R_max, send, err, stream); break;
+    case 2: st = launch_permute<2>(x, rowB, T, row_of, R_max, send, err, stream); break;
+    case 3: st = launch_permute<3>(x, rowB, T, row_of, R_max, send, err, stream); break;
+    case 4: st = launch_permute<4>(x, rowB, T, row_of, R_max, send, err, stream); break;
+    case 5: st = launch_permute<5>(x, rowB, T, row_of, R_max, send, err, stream); break;
+    case 6: st = launch_permute<6>(x, rowB, T, row_of, R_max, send, err, stream); break;
+    case 7: st = launch_permute<7>(x, rowB, T, row_of, R_max, send, err, stream); break;
+    case 8: st = launch_permute<8>(x, rowB, T, row_of, R_max, send, err, stream); break;
     }
     if (st == MOE_OK) note_launches(1);
     return st;
@@ -267,11 +363,10 @@ extern "C" moe_status moe_combine(const void *Y, moe_dtype y_dtype, int64_t R_ma
     if (!Y || !idx || !w || !out || !aligned16(Y) || !aligned16(out)) return MOE_ERR_ARG;
     const size_t rowB = eb * (size_t)d;
     if (rowB % 16) return MOE_ERR_UNSUPPORTED;
-    const int nvec = (int)(rowB / 16);
     const bool ob = out_dtype == MOE_BF16;
     moe_status st = y_dtype == MOE_BF16
-                        ? dispatch_combine_k<__nv_bfloat16>(k, Y, nvec, R_max, idx, w, T, out, ob, err, stream)
-                        : dispatch_combine_k<float>(k, Y, nvec, R_max, idx, w, T, out, ob, err, stream);
+                        ? dispatch_combine_k<__nv_bfloat16>(k, Y, rowB, R_max, idx, w, T, out, ob, err, stream)
+                        : dispatch_combine_k<float>(k, Y, rowB, R_max, idx, w, T, out, ob, err, stream);
     if (st == MOE_OK) note_launches(1);
     return st;
 }

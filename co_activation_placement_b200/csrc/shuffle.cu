@@ -21,6 +21,7 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kShuffleThreads = 512;
 
 __global__ void __launch_bounds__(kThreads)
 rank_score_kernel(const uint32_t *__restrict__ trans, const int32_t *__restrict__ e2r, int E, int G,
@@ -47,16 +48,16 @@ rank_score_kernel(const uint32_t *__restrict__ trans, const int32_t *__restrict_
 }
 
 template <int K>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kShuffleThreads)
 shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, const uint32_t *__restrict__ rs_g,
                        int32_t *__restrict__ target, int32_t *err)
 {
     extern __shared__ uint32_t tab[];   // [E][G]
-    for (int i = threadIdx.x; i < E * G; i += kThreads) tab[i] = __ldg(rs_g + i);
+    for (int i = threadIdx.x; i < E * G; i += kShuffleThreads) tab[i] = __ldg(rs_g + i);
     __syncthreads();
     const int lane = threadIdx.x & 31;
-    const int nwarps = gridDim.x * (kThreads / 32);
-    for (int t = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t < T; t += nwarps) {
+    const int nwarps = gridDim.x * (kShuffleThreads / 32);
+    for (int t = blockIdx.x * (kShuffleThreads / 32) + (threadIdx.x >> 5); t < T; t += nwarps) {
         const int mine = lane < K ? __ldg(ids + (size_t)t * K + lane) : 0;
         const bool bad = __any_sync(0xffffffffu, lane < K && (unsigned)mine >= (unsigned)E);
         if (bad) {
@@ -109,9 +110,10 @@ static moe_status launch_shuffle(const int32_t *ids, int T, int E, int G, const 
 {
     const size_t smem = sizeof(uint32_t) * (size_t)E * G;
     if (allow_smem(shuffle_targets_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
-    const long long need = ((long long)T + (kThreads / 32) - 1) / (kThreads / 32);
-    const int grid = (int)std::max<long long>(1, std::min<long long>(need, (long long)sm_count() * 3));
-    shuffle_targets_kernel<K><<<grid, kThreads, smem, s>>>(ids, T, E, G, rs, target, err);
+    // one block per SM at most: every block first copies the whole table
+    const long long need = ((long long)T + (kShuffleThreads / 32) - 1) / (kShuffleThreads / 32);
+    const int grid = (int)std::max<long long>(1, std::min<long long>(need, (long long)sm_count()));
+    shuffle_targets_kernel<K><<<grid, kShuffleThreads, smem, s>>>(ids, T, E, G, rs, target, err);
     return launch_status();
 }
 

@@ -10,16 +10,20 @@
 // token and layer for C (upper triangle incl. diagonal) and k^2 per token and
 // layer pair for M.  Each thread block owns one "group" -- (C of layer l, a band
 // of triangle rows) or (M of layer pair l, a band of rows) -- small enough to
-// live as uint32 counters in shared memory (<= 64 KB, three blocks per SM), and
-// one contiguous token slice.  Threads take one token at a time, load its k ids
-// with vector loads, sort them with a compare-exchange network (C only) and
-// issue shared-memory atomic adds for the pairs whose row falls in the band.
-// Blocks are numbered slice-major, so the blocks that read the same token
-// slice of a layer (C of l, M of l-1 and M of l) run in the same wave and
-// share it through L2.  Each block writes its counters once, coalesced, to a
-// partial buffer; a second kernel sums the partials of each cell (integer, so
-// the result does not depend on order), mirrors the triangle and evaluates
-// Ochiai in fp64 with IEEE-rounded multiply, square root and divide.
+// live as uint32 counters in shared memory (about 64 KB, three blocks per SM),
+// and one contiguous token slice; M blocks take q times shorter slices than C
+// blocks so that both kinds do about the same number of increments.  Threads
+// take one token at a time, load its k ids with vector loads, sort them with a
+// compare-exchange network (C only) and issue shared-memory atomic adds.  M rows
+// are padded to an odd stride, so that tokens incrementing the same column
+// (a popular next-layer expert) in different rows hit different banks.  Only C
+// blocks check ids for repeats (M blocks keep the range check that guards the
+// histogram) unless C is not computed.  Blocks are numbered slice-major, so the
+// blocks reading the same token slice run in the same wave and share it
+// through L2.  Each block writes its counters once, coalesced, to a partial
+// buffer; a second kernel sums the partials of each cell (integer, so the
+// result does not depend on order), mirrors the triangle and evaluates Ochiai
+// in fp64 with IEEE-rounded multiply, square root and divide.
 #include <algorithm>
 
 #include "common.cuh"
@@ -29,7 +33,8 @@ namespace {
 
 constexpr int kHistThreads = 512;
 constexpr int kMaxBands = 64;
-constexpr int kBudgetCells = 16384;      // 64 KB of uint32 counters per block
+constexpr int kBudgetCells = 16384;      // C: 64 KB of uint32 counters per block
+constexpr int kBudgetWords = 16640;      // M: the same plus row padding
 constexpr int kTargetBlocks = 148 * 3;   // one wave at three blocks per SM
 constexpr int kMinSliceTokens = 2048;
 constexpr int kReduceThreads = 256;
@@ -37,11 +42,13 @@ constexpr int kReduceThreads = 256;
 struct StatsGeom {
     int L, T, k, E;
     int Jc, Jt;          // groups: Jc = L*nbc (0 if no C wanted), Jt = (L-1)*nbt
-    int nbc, nbt, S;
+    int nbc, nbt;        // bands of C (triangle rows) and of M (rows)
+    int S, q;            // C slices S; M sub-slices S*q
     int rows_t;          // rows per M band
-    int max_cells;
+    int tstride;         // shared-memory row stride of an M band (odd)
+    int max_words;       // shared memory words per block
     long long c_layer;   // partial words per C layer  = S * E(E+1)/2
-    long long t_layer;   // partial words per M layer  = S * E*E
+    long long t_layer;   // partial words per M layer  = S*q * E*E
     long long c_total;   // Jc ? L * c_layer : 0
     int band_c[kMaxBands + 1];
 };
@@ -75,35 +82,34 @@ bool make_geom(int L, int T, int k, int E, bool want_c, bool want_t, StatsGeom &
             if (ok) break;
         }
     }
-    // M bands: equal row counts; at least enough to fit the budget, and about
-    // as many as makes a band's k^2/nbt increments per token match a C band's
-    // k(k+1)/2/nbc, so that blocks of both kinds take similar time.
+    // M bands: as few as fit the budget with rows padded to an odd stride
     int nbt = 0;
+    g.tstride = E | 1;
     if (want_t && L > 1) {
-        int rows_fit = std::max(1, kBudgetCells / E);
-        int nbt_min = (E + rows_fit - 1) / rows_fit;
-        int want = want_c ? (int)((double)nbc * 2.0 * k / (k + 1) + 0.5) : 1;
-        nbt = std::min(E, std::max(nbt_min, want));
+        const int rows_fit = std::max(1, kBudgetWords / g.tstride);
+        nbt = (E + rows_fit - 1) / rows_fit;
         g.rows_t = (E + nbt - 1) / nbt;
         nbt = (E + g.rows_t - 1) / g.rows_t;
-        if (g.rows_t * E > kBudgetCells) return false;
+        if (nbt > kMaxBands) return false;
     }
     g.nbc = nbc;
     g.nbt = nbt;
     g.Jc = want_c ? L * nbc : 0;
     g.Jt = (want_t && L > 1) ? (L - 1) * nbt : 0;
-    int J = g.Jc + g.Jt;
-    if (J == 0) return false;
-    int S = (kTargetBlocks + J / 2) / J;
+    if (g.Jc + g.Jt == 0) return false;
+    // an M block does k^2/nbt increments per token, a C block about k(k+1)/2/nbc
+    g.q = (g.Jc && g.Jt) ? std::max(1, (int)(2.0 * k * nbc / ((k + 1.0) * nbt) + 0.5)) : 1;
+    const int per_slice = g.Jc + g.Jt * g.q;
+    int S = (kTargetBlocks + per_slice / 2) / per_slice;
     S = std::max(1, std::min(S, std::max(1, T / kMinSliceTokens)));
     g.S = S;
-    int mc = 0;
+    int mw = 0;
     for (int b = 0; b < nbc; ++b)
-        mc = std::max(mc, (int)(tri_start(g.band_c[b + 1], E) - tri_start(g.band_c[b], E)));
-    if (nbt) mc = std::max(mc, g.rows_t * E);
-    g.max_cells = mc;
+        mw = std::max(mw, (int)(tri_start(g.band_c[b + 1], E) - tri_start(g.band_c[b], E)));
+    if (nbt) mw = std::max(mw, g.rows_t * g.tstride);
+    g.max_words = mw;
     g.c_layer = (long long)S * tri_all;
-    g.t_layer = (long long)S * E * E;
+    g.t_layer = (long long)S * g.q * E * E;
     g.c_total = g.Jc ? (long long)L * g.c_layer : 0;
     return true;
 }
@@ -136,17 +142,31 @@ __device__ __forceinline__ void load_ids(const int32_t *__restrict__ p, int (&v)
     }
 }
 
+__device__ __forceinline__ void cmpx(int &a, int &b)
+{
+    const int lo = min(a, b), hi = max(a, b);
+    a = lo;
+    b = hi;
+}
+
+// Ascending sort of K ids: Batcher's 19-comparator network for K = 8, a
+// bubble network otherwise.
 template <int K>
 __device__ __forceinline__ void sort_ids(int (&v)[K])
 {
+    if constexpr (K == 8) {
+        cmpx(v[0], v[1]); cmpx(v[2], v[3]); cmpx(v[4], v[5]); cmpx(v[6], v[7]);
+        cmpx(v[0], v[2]); cmpx(v[1], v[3]); cmpx(v[4], v[6]); cmpx(v[5], v[7]);
+        cmpx(v[1], v[2]); cmpx(v[5], v[6]);
+        cmpx(v[0], v[4]); cmpx(v[1], v[5]); cmpx(v[2], v[6]); cmpx(v[3], v[7]);
+        cmpx(v[2], v[4]); cmpx(v[3], v[5]);
+        cmpx(v[1], v[2]); cmpx(v[3], v[4]); cmpx(v[5], v[6]);
+    } else {
 #pragma unroll
-    for (int i = 0; i < K; ++i)
+        for (int i = 0; i < K; ++i)
 #pragma unroll
-        for (int j = 0; j + 1 < K - i; ++j) {
-            int a = v[j], b = v[j + 1];
-            v[j] = min(a, b);
-            v[j + 1] = max(a, b);
-        }
+            for (int j = 0; j + 1 < K - i; ++j) cmpx(v[j], v[j + 1]);
+    }
 }
 
 // 0 when the K ids are distinct and in [0, E), else the device error code.
@@ -163,37 +183,52 @@ __device__ __forceinline__ int check_ids(const int (&v)[K], int E)
     return bad_range ? MOE_DERR_ID_RANGE : (bad_rep ? MOE_DERR_ID_REPEAT : 0);
 }
 
+template <int K>
+__device__ __forceinline__ bool ids_in_range(const int (&v)[K], int E)
+{
+    bool ok = true;
+#pragma unroll
+    for (int a = 0; a < K; ++a) ok &= (unsigned)v[a] < (unsigned)E;
+    return ok;
+}
+
 template <int K, bool VEC>
 __global__ void __launch_bounds__(kHistThreads)
 stats_hist_kernel(const int32_t *__restrict__ ids, StatsGeom G, uint32_t *__restrict__ part, int32_t *err)
 {
     extern __shared__ uint32_t hist[];
-    const int J = G.Jc + G.Jt;
-    const int slice = blockIdx.x / J;
-    const int grp = blockIdx.x % J;
+    const int per_slice = G.Jc + G.Jt * G.q;
+    const int slice = blockIdx.x / per_slice;
+    const int r = blockIdx.x % per_slice;
     const int T = G.T, E = G.E;
-    const int t0 = (int)((long long)T * slice / G.S);
-    const int t1 = (int)((long long)T * (slice + 1) / G.S);
-    const bool is_c = grp < G.Jc;
-    int l, r0, r1, cells;
+    const bool is_c = r < G.Jc;
+    int l, r0, r1, cells, t0, t1;
     long long out;
     if (is_c) {
-        l = grp / G.nbc;
-        const int band = grp % G.nbc;
+        l = r / G.nbc;
+        const int band = r % G.nbc;
         r0 = G.band_c[band];
         r1 = G.band_c[band + 1];
         cells = (int)(tri_start(r1, E) - tri_start(r0, E));
         out = (long long)l * G.c_layer + (long long)G.S * tri_start(r0, E) + (long long)slice * cells;
+        t0 = (int)((long long)T * slice / G.S);
+        t1 = (int)((long long)T * (slice + 1) / G.S);
     } else {
-        const int q = grp - G.Jc;
-        l = q / G.nbt;
-        const int band = q % G.nbt;
+        const int rr = r - G.Jc;
+        const int grp = rr / G.q;
+        const int sub = slice * G.q + rr % G.q;
+        const int nsub = G.S * G.q;
+        l = grp / G.nbt;
+        const int band = grp % G.nbt;
         r0 = band * G.rows_t;
         r1 = min(E, r0 + G.rows_t);
         cells = (r1 - r0) * E;
-        out = G.c_total + (long long)l * G.t_layer + (long long)G.S * r0 * E + (long long)slice * cells;
+        out = G.c_total + (long long)l * G.t_layer + (long long)nsub * r0 * E + (long long)sub * cells;
+        t0 = (int)((long long)T * sub / nsub);
+        t1 = (int)((long long)T * (sub + 1) / nsub);
     }
-    for (int c = threadIdx.x; c < cells; c += blockDim.x) hist[c] = 0u;
+    const int words = is_c ? cells : (r1 - r0) * G.tstride;
+    for (int c = threadIdx.x; c < words; c += blockDim.x) hist[c] = 0u;
     __syncthreads();
 
     const int32_t *lay = ids + (size_t)l * T * K;
@@ -223,21 +258,28 @@ stats_hist_kernel(const int32_t *__restrict__ ids, StatsGeom G, uint32_t *__rest
         }
     } else {
         const int32_t *nxt = lay + (size_t)T * K;
+        const bool full_check = G.Jc == 0;   // C blocks report repeats when they run
+        const int stride = G.tstride;
         for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
             int a[K], c[K];
             load_ids<K, VEC>(lay + (size_t)t * K, a);
             load_ids<K, VEC>(nxt + (size_t)t * K, c);
-            int bad = check_ids<K>(a, E);
-            if (!bad) bad = check_ids<K>(c, E);
-            if (bad) {
-                record_error(err, bad);
+            if (full_check) {
+                int bad = check_ids<K>(a, E);
+                if (!bad) bad = check_ids<K>(c, E);
+                if (bad) {
+                    record_error(err, bad);
+                    continue;
+                }
+            } else if (!ids_in_range<K>(a, E) || !ids_in_range<K>(c, E)) {
+                record_error(err, MOE_DERR_ID_RANGE);
                 continue;
             }
 #pragma unroll
             for (int x = 0; x < K; ++x) {
                 const int i = a[x];
                 if (i >= r0 && i < r1) {
-                    const int row = (i - r0) * E;
+                    const int row = (i - r0) * stride;
 #pragma unroll
                     for (int y = 0; y < K; ++y) atomicAdd(&hist[row + c[y]], 1u);
                 }
@@ -246,7 +288,27 @@ stats_hist_kernel(const int32_t *__restrict__ ids, StatsGeom G, uint32_t *__rest
     }
     __syncthreads();
     uint32_t *dst = part + out;
-    for (int c = threadIdx.x; c < cells; c += blockDim.x) dst[c] = hist[c];
+    if (is_c) {
+        for (int c = threadIdx.x; c < cells; c += blockDim.x) dst[c] = hist[c];
+    } else {
+        for (int c = threadIdx.x; c < cells; c += blockDim.x) dst[c] = hist[(c / E) * G.tstride + c % E];
+    }
+}
+
+// Sum of n partial words at base, base + stride, ... (8 loads in flight).
+__device__ __forceinline__ uint32_t sum_strided(const uint32_t *__restrict__ part, long long base, long long stride, int n)
+{
+    uint32_t s = 0;
+    int q = 0;
+    for (; q + 8 <= n; q += 8) {
+        uint32_t v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __ldg(part + base + (long long)(q + i) * stride);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s += v[i];
+    }
+    for (; q < n; ++q) s += __ldg(part + base + (long long)q * stride);
+    return s;
 }
 
 __device__ __forceinline__ uint32_t c_cell_sum(const StatsGeom &G, const uint32_t *__restrict__ part, int l, int a, int b)
@@ -258,12 +320,11 @@ __device__ __forceinline__ uint32_t c_cell_sum(const StatsGeom &G, const uint32_
     const long long cells = tri_start(G.band_c[band + 1], G.E) - tri_start(r0, G.E);
     const long long base = (long long)l * G.c_layer + (long long)G.S * tri_start(r0, G.E)
                            + (tri_start(a, G.E) - tri_start(r0, G.E)) + (b - a);
-    uint32_t s = 0;
-    for (int q = 0; q < G.S; ++q) s += __ldg(part + base + (long long)q * cells);
-    return s;
+    return sum_strided(part, base, cells, G.S);
 }
 
 // blockIdx.y selects the matrix: [0, L) C of layer y, [L, 2L-1) M of layer y-L.
+// One output cell per thread.
 __global__ void __launch_bounds__(kReduceThreads)
 stats_reduce_kernel(StatsGeom G, const uint32_t *__restrict__ part, uint32_t *coact, float *ochiai, uint32_t *trans)
 {
@@ -271,6 +332,7 @@ stats_reduce_kernel(StatsGeom G, const uint32_t *__restrict__ part, uint32_t *co
     const int E = G.E;
     const int m = blockIdx.y;
     const long long EE = (long long)E * E;
+    const long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (m < G.L) {
         if (!G.Jc) return;
         const int l = m;
@@ -278,7 +340,7 @@ stats_reduce_kernel(StatsGeom G, const uint32_t *__restrict__ part, uint32_t *co
             for (int e = threadIdx.x; e < E; e += blockDim.x) diag[e] = c_cell_sum(G, part, l, e, e);
             __syncthreads();
         }
-        for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < EE; c += (long long)gridDim.x * blockDim.x) {
+        if (c < EE) {
             const int i = (int)(c / E), j = (int)(c % E);
             const uint32_t v = c_cell_sum(G, part, l, min(i, j), max(i, j));
             if (coact) coact[(long long)l * EE + c] = v;
@@ -289,28 +351,25 @@ stats_reduce_kernel(StatsGeom G, const uint32_t *__restrict__ part, uint32_t *co
             }
         }
     } else {
-        if (!G.Jt || !trans) return;
+        if (!G.Jt || !trans || c >= EE) return;
         const int l = m - G.L;
-        for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < EE; c += (long long)gridDim.x * blockDim.x) {
-            const int i = (int)(c / E), j = (int)(c % E);
-            const int band = i / G.rows_t;
-            const int r0 = band * G.rows_t;
-            const int r1 = min(E, r0 + G.rows_t);
-            const long long cells = (long long)(r1 - r0) * E;
-            const long long base = G.c_total + (long long)l * G.t_layer + (long long)G.S * r0 * E
-                                   + (long long)(i - r0) * E + j;
-            uint32_t s = 0;
-            for (int q = 0; q < G.S; ++q) s += __ldg(part + base + (long long)q * cells);
-            trans[(long long)l * EE + c] = s;
-        }
+        const int i = (int)(c / E), j = (int)(c % E);
+        const int band = i / G.rows_t;
+        const int r0 = band * G.rows_t;
+        const int r1 = min(E, r0 + G.rows_t);
+        const long long cells = (long long)(r1 - r0) * E;
+        const int nsub = G.S * G.q;
+        const long long base = G.c_total + (long long)l * G.t_layer + (long long)nsub * r0 * E
+                               + (long long)(i - r0) * E + j;
+        trans[(long long)l * EE + c] = sum_strided(part, base, cells, nsub);
     }
 }
 
 template <int K>
 moe_status launch_hist(const int32_t *ids, const StatsGeom &g, uint32_t *part, int32_t *err, cudaStream_t s)
 {
-    const size_t smem = (size_t)g.max_cells * sizeof(uint32_t);
-    const int blocks = (g.Jc + g.Jt) * g.S;
+    const size_t smem = (size_t)g.max_words * sizeof(uint32_t);
+    const int blocks = (g.Jc + g.Jt * g.q) * g.S;
     const bool vec = (K % 4 == 0) ? aligned16(ids) : ((K % 2 == 0) ? ((reinterpret_cast<uintptr_t>(ids) & 7u) == 0) : false);
     if (vec) {
         if (allow_smem(stats_hist_kernel<K, true>, smem) != cudaSuccess) return MOE_ERR_CUDA;
@@ -376,8 +435,7 @@ extern "C" moe_status moe_coact_stats(const int32_t *ids, int L, int T, int k, i
     if (st != MOE_OK) return st;
     note_launches(1);
     const int mats = L + (want_t ? L - 1 : 0);
-    const long long per_block = (long long)kReduceThreads * 4;
-    int bx = (int)std::min<long long>(((long long)EE + per_block - 1) / per_block, 1024);
+    const int bx = (int)(((long long)EE + kReduceThreads - 1) / kReduceThreads);
     dim3 grid(bx, mats);
     const size_t smem = (size_t)E * sizeof(uint32_t);
     stats_reduce_kernel<<<grid, kReduceThreads, smem, stream>>>(g, part, coact, ochiai, trans);

@@ -66,6 +66,8 @@ typedef enum {
 #define MOE_DERR_ID_REPEAT  2   /* an expert id repeated within a token */
 #define MOE_DERR_RANK_RANGE 3   /* expert_to_rank or src_rank outside [0, G) */
 #define MOE_DERR_ROW_RANGE  4   /* a row index outside the row buffer   */
+#define MOE_DERR_TIMEOUT    5   /* a bounded wait on an asynchronous copy ran out
+                                   (the kernel stopped early; outputs incomplete) */
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 

@@ -15,9 +15,12 @@ Recipe (draw order is part of the definition, so both sides of a test see the
 same bits):
 
 * ``numpy.random.Generator(PCG64)`` streams seeded with ``SeedSequence``:
-  ``[seed, 0]`` draws the per-layer cluster layout, ``[seed, 0, 1 + b]`` the
-  routing of token block b (65536 tokens per block), ``[seed, 1]`` the gate
-  logits and ``[seed, 2, b]`` hidden-state row block b (4096 rows per block);
+  ``[layout_seed, 0]`` draws the per-layer cluster layout -- the stand-in for
+  the trained router, shared by every batch of one workload, so it defaults to
+  the workload's seed -- ``[seed, 0, 1 + b]`` the routing of token block b
+  (65536 tokens per block), ``[seed, 1]`` the gate logits and ``[seed, 2, b]``
+  hidden-state row block b (4096 rows per block).  A calibration batch is the
+  same workload with another token seed;
 * per layer l a random permutation pi_l of the E expert ids, cut into
   ``n_clusters`` clusters of ``cluster_size`` (so clusters are never runs of
   contiguous ids);
@@ -199,19 +202,22 @@ def _parallel(fn, nblocks):
         return list(ex.map(fn, range(nblocks)))
 
 
-def make_routing(w: Workload, seed: Optional[int] = None, T: Optional[int] = None) -> np.ndarray:
+def make_routing(w: Workload, seed: Optional[int] = None, T: Optional[int] = None,
+                 layout_seed: Optional[int] = None) -> np.ndarray:
     """Top-k expert ids, int32 [L][T][k], k distinct ids per token and layer.
 
     Tokens are drawn in blocks of TOKENS_PER_BLOCK, each from its own
-    generator, so the result does not depend on the thread count.
+    generator, so the result does not depend on the thread count.  The
+    cluster layout comes from ``layout_seed`` (default: the workload's seed).
     """
     seed = w.seed if seed is None else seed
+    layout_seed = w.seed if layout_seed is None else layout_seed
     T = w.T if T is None else T
     if w.n_clusters * w.cluster_size > w.E:
         raise ValueError("clusters do not fit in E")
     if w.k > w.E:
         raise ValueError("k > E")
-    layout = _layout(w, seed)
+    layout = _layout(w, layout_seed)
     nb = max(1, -(-T // TOKENS_PER_BLOCK))
     parts = _parallel(lambda b: _routing_block(
         w, seed, b, min(T, (b + 1) * TOKENS_PER_BLOCK) - b * TOKENS_PER_BLOCK, layout), nb)

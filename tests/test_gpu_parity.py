@@ -81,7 +81,7 @@ def test_stats_small(cap, shape):
 
 def test_stats_partial_outputs(cap):
     rng = np.random.default_rng(3)
-    ids = clustered_ids(rng, 3, 2000, 4, 64)
+    ids = clustered_ids(rng, 3, 2000, 64, 4)
     o = orc.coact(ids, 64)
     g = cap.coact_stats(dev(ids), 64, want=("trans",))
     assert g["coact"] is None and (host(g["trans"]) == o["trans"]).all()
@@ -266,11 +266,14 @@ def test_pipeline_full_size(cap, name, placement, shuffle):
         op = orc.plan(ids[l], w.E, w.G, w.rpn, e2r_o[l], src_rank=src)
         check_plan(hp.plans[l], op, w.T, w.k)
         R = op["R"]
-        # rows: sampled against the oracle's permute
-        rows = np.unique(np.concatenate([rng.integers(0, R, 4096), [0, R - 1]]))
-        sub = host(hp.send[torch.from_numpy(rows).cuda()].view(torch.int16 if w.dtype == "bf16" else torch.float32))
-        want = orc.permute(x, op["row_token"][rows])
-        assert (sub.view(want.dtype) == want).all()
+        # rows: the step reuses one send buffer for every layer (as a training
+        # step would), so after the step it holds the last layer's rows; each
+        # earlier layer's rows are checked through its combine output below
+        if l == w.L - 1:
+            rows = np.unique(np.concatenate([rng.integers(0, R, 4096), [0, R - 1]]))
+            sub = host(hp.send[torch.from_numpy(rows).cuda()].view(torch.int16 if w.dtype == "bf16" else torch.float32))
+            want = orc.permute(x, op["row_token"][rows])
+            assert (sub.view(want.dtype) == want).all()
         # combine: sampled tokens against the oracle's fp64 combine
         toks = np.unique(np.concatenate([rng.integers(0, w.T, 1024), [0, w.T - 1]]))
         idx = op["row_of"][toks]
