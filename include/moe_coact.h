@@ -146,6 +146,33 @@ moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E, int G, int
                              void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Dispatch plan without caller-provided workspace.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory -- code running inside another framework's allocator or
+ * memory-pool hook (a cudaMalloc there would re-enter the allocator),
+ * processes that reserve their whole device-memory budget at start-up, and
+ * latency-critical loops that cannot accept cudaMalloc's possible implicit
+ * device synchronisation.
+ *
+ * Same arguments, outputs and errors as moe_plan_dispatch, without ws and
+ * ws_bytes.  The scratch is a statically reserved device array of
+ * MOE_PLAN_STATIC_SCRATCH_BYTES held by every GPU that loads the library until
+ * the process exits.  Calls whose moe_plan_dispatch_workspace(T, k, G,
+ * src_rank != NULL) exceeds it return MOE_ERR_WORKSPACE and enqueue nothing
+ * (4 MiB covers, for example, T = 786432 tokens at G = 64 with source ranks).
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine).  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, which also loads the library's kernels on that
+ * device); make that first call before any stream capture.  All calls on a
+ * device share the array and each clears the part that must start at zero:
+ * calls whose kernels overlap on the GPU (unordered streams) race on it.
+ * ---------------------------------------------------------------------- */
+#define MOE_PLAN_STATIC_SCRATCH_BYTES (4u << 20)
+moe_status moe_plan_dispatch_static(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                                    const int32_t *expert_to_rank, const int32_t *src_rank,
+                                    const moe_plan *plan, int32_t *err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Row permute into the rank-major send buffer  ([EC]; [CE] footnote 3)
  *   send[row_of[t][j]][:] = x[t][:]   for every t, j
  * which equals send[i] = x[row_token[i]] for every row i < R.  Each token's
