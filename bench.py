@@ -38,6 +38,7 @@ if ROOT not in sys.path:
 
 METRIC = "dedup dispatch+combine GB/s (frac of HBM peak); co-activation tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+SM_MAX_MHZ = 1965.0            # B200 clocks.max.sm
 
 
 def peaks():
@@ -60,6 +61,11 @@ def parse():
     ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of one CUDA graph")
+    ap.add_argument("--replicas", type=int, default=0, metavar="EXTRA",
+                    help="replicate experts (EXTRA more per rank) and assign tasks to the fewest remote nodes")
+    ap.add_argument("--prereduce", action="store_true",
+                    help="receiver-side pre-reduced combine with stand-in experts (gates dispatched with rows)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--sweep-only", action="store_true", help="only the co-activation statistics sweep")
@@ -254,9 +260,12 @@ def run_reference(a, w):
 
 # ------------------------------------------------------------------ native arm
 
-def traffic_record(kernel_name):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel's
-    source is unchanged since the capture (else None)."""
+def traffic_record(kernel_name, algorithmic_bytes_per_launch):
+    """DRAM bytes per launch for the dominant kernel, from the committed ncu
+    capture (profiles/traffic.json): the capture's DRAM bytes over its
+    algorithmic bytes, scaled to this launch's algorithmic bytes (both kernels
+    stream, so traffic grows in proportion).  None when the kernel's source
+    changed since the capture."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -267,7 +276,9 @@ def traffic_record(kernel_name):
         return None
     src = os.path.join(ROOT, "co_activation_placement_b200", "csrc", rec["source"])
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["bytes_per_launch"] if h == rec["source_sha256_16"] else None
+    if h != rec["source_sha256_16"]:
+        return None
+    return int(rec["traffic_over_algorithmic"] * algorithmic_bytes_per_launch)
 
 
 def main():
@@ -280,7 +291,7 @@ def main():
     import torch
     import co_activation_placement_b200 as cap
     from co_activation_placement_b200 import pipeline
-    from synth import make_routing, make_gates, make_hidden
+    from synth import make_routing, make_gates, make_hidden, make_expert_scales
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -311,7 +322,9 @@ def main():
     gates = make_gates(w, seed=seed)
     x = make_hidden(w, seed=seed)
     hp = pipeline.prepare(w.E, w.G, w.rpn, ids, gates, x, w.dtype, ids_cal, placement=a.placement,
-                          shuffle=shuffle, out_dtype=out_dtype, device=device, timers=True)
+                          shuffle=shuffle, out_dtype=out_dtype, device=device, timers=True,
+                          scales=make_expert_scales(w, seed=seed) if a.prereduce else None,
+                          replica_extra=a.replicas)
 
     def barrier():
         if pg is not None:
@@ -330,22 +343,41 @@ def main():
         uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
     except Exception:
         pass
+    # the timed steps: captured once into a CUDA graph (launch gaps between
+    # the small kernels vanish), or launched eagerly with --no-graph
+    graph = None
+    graph_note = None
+    if not a.no_graph:
+        try:
+            n0 = cap.launch_count()
+            graph = hp.capture(a.steps)
+            n_launch = cap.launch_count() - n0      # kernels inside the replayed graph
+        except Exception as ex:                    # capture unsupported here: time eagerly
+            graph, graph_note = None, "graph capture failed: %s" % str(ex).splitlines()[0][:120]
+            torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    hp.reset_events()
-    n0 = cap.launch_count()
+    if graph is None:
+        hp.reset_events()
+        n0 = cap.launch_count()
     with ClockSampler(uuid) as clk:
         start = torch.cuda.Event(enable_timing=True)
         stop = torch.cuda.Event(enable_timing=True)
         start.record()
-        for _ in range(a.steps):
-            hp.step()
+        if graph is not None:
+            graph.replay()
+        else:
+            for _ in range(a.steps):
+                hp.step()
         stop.record()
         torch.cuda.synchronize()
-    n1 = cap.launch_count()
+    if graph is None:
+        n_launch = cap.launch_count() - n0
     barrier()
     per_kernel = hp.kernel_times_ms()
     hp.reset_events()
+    if int(hp.err.item()) != 0:
+        raise SystemExit("device data error %d in the timed steps" % int(hp.err.item()))
     ms_total = start.elapsed_time(stop)
     ms_step = ms_total / a.steps
     ms_step = reduce_max(ms_step, pg, device)
@@ -355,8 +387,9 @@ def main():
     value = weak_value(world, sb.dispatch_combine, ms_step)
     kern = {}
     bytes_of = {"stats": sb.stats, "plan": sb.plan, "permute": sb.permute, "combine": sb.combine,
-                "shuffle": sb.shuffle}
-    launches_of = {"stats": 1, "plan": w.L, "permute": w.L, "combine": w.L, "shuffle": (w.L - 1) if shuffle else 0}
+                "shuffle": sb.shuffle, "gates": sb.gates, "reduce": sb.reduce}
+    launches_of = {"stats": 1, "plan": w.L, "permute": w.L, "combine": w.L, "shuffle": (w.L - 1) if shuffle else 0,
+                   "gates": w.L, "reduce": w.L}
     for name, tot_ms in per_kernel.items():
         ms = tot_ms / a.steps                         # per step
         gbs = bytes_of[name] / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
@@ -365,7 +398,7 @@ def main():
     dom = max(kern, key=lambda n: kern[n]["ms_per_step"])
     nl = launches_of[dom]
     per_launch_ms = kern[dom]["ms_per_step"] / nl
-    traffic = traffic_record(dom)
+    traffic = traffic_record(dom, bytes_of[dom] // nl)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["gbs"], "peak": hbm, "unit": "GB/s",
                 "frac": kern[dom]["gbs"] / hbm, "peak_kind": hbm_kind,
                 "algorithmic_bytes_per_launch": bytes_of[dom] // nl, "ms_per_launch": per_launch_ms,
@@ -394,6 +427,9 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "G": w.G, "rpn": w.rpn, "d": w.d,
                        "L": w.L, "x_dtype": w.dtype, "out_dtype": a.out_dtype, "placement": a.placement,
+                       "combine": "receiver-side pre-reduced (stand-in experts)" if a.prereduce
+                                  else "source-side weighted (identity experts)",
+                       "replicas_per_rank": a.replicas,
                        "shuffle": shuffle, "parallelism": "replicas (weak scaling, one batch per GPU)",
                        "l2": "inputs larger than L2 (x %.2f GB per GPU; no flush)" % (x.nbytes / 1e9)},
             "frac_of_hbm_peak": value / hbm,
@@ -407,8 +443,10 @@ def main():
                      "V": [int(s[3]) for s in summaries]},
             "clocks": clocks,
             "e2e": e2e,
-            "gpu_launches": int(n1 - n0),
-            "gpu_launches_per_step": (n1 - n0) / a.steps,
+            "gpu_launches": int(n_launch),
+            "gpu_launches_per_step": n_launch / a.steps,
+            "timing": "one CUDA graph of the %d steps" % a.steps if graph is not None else
+                      ("eager launches" + ("; " + graph_note if graph_note else "")),
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -443,55 +481,99 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
     ms = reduce_max(tot / n, pg, device)
     nbytes = hp.step_bytes(None).stats
     world = pg.get_world_size() if pg is not None else 1
+    incs = (w.L * w.T * w.k * (w.k + 1) // 2 + (w.L - 1) * w.T * w.k * w.k) / (ms * 1e-3)
+    # the unit that bounds this kernel: shared memory serves 32 4-byte accesses
+    # per clock per SM, so at most 32 counter increments per clock per SM
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    peak_inc = 32.0 * sms * SM_MAX_MHZ * 1e6
     return {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "L": w.L, "ms": ms,
             "tokens_per_s": world * w.L * w.T / (ms * 1e-3),
-            "increments_per_s": world * (w.L * w.T * w.k * (w.k + 1) // 2 + (w.L - 1) * w.T * w.k * w.k) / (ms * 1e-3),
+            "increments_per_s": world * incs,
             "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
+            "atomic_roofline": {"bound": "shared-memory atomics", "achieved": incs, "unit": "increments/s",
+                                "peak": peak_inc, "frac": incs / peak_inc,
+                                "peak_note": "32 per clock per SM x %d SMs x %.0f MHz" % (sms, SM_MAX_MHZ)},
             "algorithmic_bytes": nbytes, "err": int(hp.err.item())}
 
 
 def run_e2e(hp, ids, gates, x, w, a, device, sb, pg, world):
     """The same metric through the public API with host buffers: every step
-    copies its inputs from pinned host memory and reads its results back."""
+    copies its inputs from pinned host memory and reads its results back
+    (statistics, plan summaries, shuffle targets and the last layer's combine
+    output).  Steps are pipelined: inputs and the big output are double
+    buffered, so step i+1's host-to-device copy and step i-1's device-to-host
+    copy run on their own streams while step i computes."""
     import torch
     from co_activation_placement_b200.pipeline import bf16_from_bits
     ids_h = torch.from_numpy(ids).pin_memory()
     gates_h = torch.from_numpy(gates).pin_memory()
     x_h = (bf16_from_bits(x) if w.dtype == "bf16" else torch.from_numpy(x)).pin_memory()
     out_h = torch.empty(hp.outs[-1].shape, dtype=hp.outs[-1].dtype).pin_memory()
-    st_h = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in hp.stats.items() if v is not None}
+    small = {k: v for k, v in hp.stats.items() if v is not None}
+    small_h = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in small.items()}
     sum_h = torch.empty((w.L, 5), dtype=torch.int64).pin_memory()
+    tgt_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in hp.targets]
+    sets = [dict(ids=hp.ids, gates=hp.gates, x=hp.x, out=hp.outs[-1]),
+            dict(ids=torch.empty_like(hp.ids), gates=torch.empty_like(hp.gates), x=torch.empty_like(hp.x),
+                 out=torch.empty_like(hp.outs[-1]))]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    ready, done, read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for e in done + read:
+        e.record(comp)
     hp.timers = False
 
-    def one():
-        hp.ids.copy_(ids_h, non_blocking=True)
-        hp.gates.copy_(gates_h, non_blocking=True)
-        hp.x.copy_(x_h, non_blocking=True)
-        hp.step()
-        out_h.copy_(hp.outs[-1], non_blocking=True)
-        for k_, v in st_h.items():
-            v.copy_(hp.stats[k_], non_blocking=True)
-        sum_h.copy_(torch.stack([p.summary for p in hp.plans]), non_blocking=True)
+    def upload(j):
+        s_in.wait_event(done[j])                  # the step that last read set j is over
+        with torch.cuda.stream(s_in):
+            sets[j]["ids"].copy_(ids_h, non_blocking=True)
+            sets[j]["gates"].copy_(gates_h, non_blocking=True)
+            sets[j]["x"].copy_(x_h, non_blocking=True)
+        ready[j].record(s_in)
 
-    for _ in range(2):
-        one()
+    def run(n, t0=None):
+        if t0 is not None:
+            t0.record(s_in)                       # before the first upload
+        upload(0)
+        for i in range(n):
+            j = i % 2
+            if i + 1 < n:
+                upload(1 - j)
+            comp.wait_event(ready[j])
+            comp.wait_event(read[j])              # set j's output was read back
+            hp.ids, hp.gates, hp.x, hp.outs[-1] = sets[j]["ids"], sets[j]["gates"], sets[j]["x"], sets[j]["out"]
+            hp.step()
+            for k_, v in small.items():           # small results, in stream order
+                small_h[k_].copy_(v, non_blocking=True)
+            sum_h.copy_(torch.stack([p.summary for p in hp.plans]), non_blocking=True)
+            for th, td in zip(tgt_h, hp.targets):
+                th.copy_(td, non_blocking=True)
+            done[j].record(comp)
+            s_out.wait_event(done[j])
+            with torch.cuda.stream(s_out):
+                out_h.copy_(sets[j]["out"], non_blocking=True)
+            read[j].record(s_out)
+
+    run(2)
     torch.cuda.synchronize()
-    n = max(3, min(a.steps, 10))
+    n = max(4, min(a.steps, 12))
     if pg is not None:
         pg.barrier()
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(n):
-        one()
-    e.record()
+    run(n, t0=s)
+    e.record(s_out)
     torch.cuda.synchronize()
     ms = reduce_max(s.elapsed_time(e) / n, pg, device)
+    hp.ids, hp.gates, hp.x, hp.outs[-1] = sets[0]["ids"], sets[0]["gates"], sets[0]["x"], sets[0]["out"]
     hp.timers = True
     h2d = ids_h.numel() * 4 + gates_h.numel() * 4 + x_h.numel() * x_h.element_size()
-    d2h = out_h.numel() * out_h.element_size() + sum(v.numel() * v.element_size() for v in st_h.values()) + sum_h.numel() * 8
+    d2h = (out_h.numel() * out_h.element_size() + sum(v.numel() * v.element_size() for v in small_h.values())
+           + sum_h.numel() * 8 + sum(t.numel() * 4 for t in tgt_h))
     return {"value": weak_value(world, sb.dispatch_combine, ms), "unit": "GB/s", "ms_per_step": ms,
-            "steps": n, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+            "steps": n, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "pipelined": "inputs and output double buffered; copies overlap compute across steps"}
 
 
 if __name__ == "__main__":

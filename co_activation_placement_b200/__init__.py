@@ -8,6 +8,8 @@ import of any entry point raises: there is no fallback.
 
 Entry points (names follow the C ABI without the ``moe_`` prefix):
   coact_stats, plan_dispatch, permute, combine, rank_score, shuffle_targets,
+  dispatch_gates, expert_reduce, combine_rows,
+  place_replicas, assign_replicas, plan_dispatch_ranks,
   place_uniform, place_capacity, place_correlated, launch_count.
 """
 from __future__ import annotations
@@ -60,11 +62,17 @@ def lib() -> ctypes.CDLL:
             "moe_plan_dispatch": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
             "moe_permute": ([P, i, i, i, i, P, i64, P, P, P], i),
             "moe_combine": ([P, i, i64, i, P, P, i, i, P, i, P, P], i),
+            "moe_dispatch_gates": ([P, P, i, i, P, P, P, i64, P, P, P, P], i),
+            "moe_expert_reduce": ([P, i, i64, i, P, P, P, i, P, i, P, i, P, P], i),
+            "moe_combine_rows": ([P, i, i64, i, P, i, i, P, i, P, P], i),
             "moe_rank_score": ([P, P, i, i, P, P, P], i),
             "moe_shuffle_targets": ([P, i, i, i, i, P, P, P, P], i),
             "moe_place_uniform": ([i, i, P], i),
             "moe_place_capacity": ([P, i, i, P, P], i),
             "moe_place_correlated": ([P, i, i, i, P], i),
+            "moe_place_replicas": ([P, i, i, i, P, i, P, P], i),
+            "moe_assign_replicas": ([P, i, i, i, i, i, P, P, P, P, P, P, P], i),
+            "moe_plan_dispatch_ranks": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
         }
         for name, (args, res) in sigs.items():
             f = getattr(L, name)
@@ -222,6 +230,47 @@ def plan_dispatch(ids: torch.Tensor, E: int, G: int, rpn: int, expert_to_rank: t
     return plan
 
 
+def plan_dispatch_ranks(ids: torch.Tensor, E: int, G: int, rpn: int, pick_rank: torch.Tensor,
+                        src_rank: Optional[torch.Tensor] = None, plan: Optional[Plan] = None,
+                        ws: Optional[torch.Tensor] = None) -> Plan:
+    """The dispatch plan with the serving rank of every pick given (replicated experts)."""
+    _dev(ids, torch.int32, "ids", 2)
+    _dev(pick_rank, torch.int32, "pick_rank", 2)
+    if src_rank is not None:
+        _dev(src_rank, torch.int32, "src_rank", 1)
+    T, k = ids.shape
+    dev = ids.device
+    if plan is None:
+        plan = Plan.empty(T, k, G, dev)
+    need = plan_dispatch_workspace(T, k, G, src_rank is not None)
+    if ws is None:
+        ws = _workspace(dev, "plan").get(need)
+    cs = plan.c_struct()
+    st = lib().moe_plan_dispatch_ranks(_ptr(ids), T, k, E, G, rpn, _ptr(pick_rank), _ptr(src_rank),
+                                       ctypes.byref(cs), _ptr(plan.err), _ptr(ws), ws.numel(), _stream(ids))
+    _check("moe_plan_dispatch_ranks", st)
+    return plan
+
+
+def assign_replicas(ids: torch.Tensor, E: int, G: int, rpn: int, replica_rank: torch.Tensor, n_rep: torch.Tensor,
+                    src_rank: Optional[torch.Tensor] = None, pick_rank: Optional[torch.Tensor] = None,
+                    n_remote: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None):
+    """(pick_rank int32 [T][k], n_remote int32 [T]): fewest remote nodes per token over the replicas."""
+    _dev(ids, torch.int32, "ids", 2)
+    _dev(replica_rank, torch.int32, "replica_rank", 2)
+    _dev(n_rep, torch.int32, "n_rep", 1)
+    T, k = ids.shape
+    if pick_rank is None:
+        pick_rank = torch.empty((max(T, 1), k), dtype=torch.int32, device=ids.device)
+    if n_remote is None:
+        n_remote = torch.empty(max(T, 1), dtype=torch.int32, device=ids.device)
+    err = new_err(ids.device) if err is None else err
+    st = lib().moe_assign_replicas(_ptr(ids), T, k, E, G, rpn, _ptr(replica_rank), _ptr(n_rep), _ptr(src_rank),
+                                   _ptr(pick_rank), _ptr(n_remote), _ptr(err), _stream(ids))
+    _check("moe_assign_replicas", st)
+    return pick_rank, n_remote
+
+
 # ---------------------------------------------------------------- rows
 
 def _dtype_code(dt) -> int:
@@ -264,6 +313,62 @@ def combine(Y: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, out_dtype=torch
     st = lib().moe_combine(_ptr(Y), _dtype_code(Y.dtype), R_max, d, _ptr(idx), _ptr(w), T, k, _ptr(out),
                            _dtype_code(out.dtype), _ptr(err), _stream(Y))
     _check("moe_combine", st)
+    return out
+
+
+# ---------------------------------------------------------------- receiver-side pre-reduced combine
+
+def dispatch_gates(ids: torch.Tensor, w: torch.Tensor, plan: Plan, send_e: Optional[torch.Tensor] = None,
+                   send_w: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None):
+    """(send_e int32 [R_max][k], send_w f32 [R_max][k]) for the plan's rows (rows >= R untouched)."""
+    _dev(ids, torch.int32, "ids", 2)
+    _dev(w, torch.float32, "w", 2)
+    T, k = ids.shape
+    R_max = plan.R_max
+    if send_e is None:
+        send_e = torch.empty((max(R_max, 1), k), dtype=torch.int32, device=ids.device)
+    if send_w is None:
+        send_w = torch.empty((max(R_max, 1), k), dtype=torch.float32, device=ids.device)
+    err = plan.err if err is None else err
+    st = lib().moe_dispatch_gates(_ptr(ids), _ptr(w), T, k, _ptr(plan.row_token), _ptr(plan.row_jmask),
+                                  _ptr(plan.summary), R_max, _ptr(send_e), _ptr(send_w), _ptr(err), _stream(ids))
+    _check("moe_dispatch_gates", st)
+    return send_e, send_w
+
+
+def expert_reduce(send: torch.Tensor, summary: torch.Tensor, send_e: torch.Tensor, send_w: torch.Tensor,
+                  scale: torch.Tensor, y_dtype=None, y: Optional[torch.Tensor] = None,
+                  err: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y[i] = sum_j send_w[i][j] * scale[send_e[i][j]] * send[i] for the rows i < summary[0]."""
+    _dev(send, send.dtype, "send", 2)
+    _dev(send_e, torch.int32, "send_e", 2)
+    _dev(send_w, torch.float32, "send_w", 2)
+    _dev(scale, torch.float32, "scale", 1)
+    R_max, d = send.shape
+    k = send_e.shape[1]
+    if y is None:
+        y = torch.empty((R_max, d), dtype=y_dtype or send.dtype, device=send.device)
+    err = new_err(send.device) if err is None else err
+    st = lib().moe_expert_reduce(_ptr(send), _dtype_code(send.dtype), R_max, d, _ptr(summary), _ptr(send_e),
+                                 _ptr(send_w), k, _ptr(scale), scale.numel(), _ptr(y), _dtype_code(y.dtype),
+                                 _ptr(err), _stream(send))
+    _check("moe_expert_reduce", st)
+    return y
+
+
+def combine_rows(Y: torch.Tensor, row_of: torch.Tensor, out_dtype=torch.float32, out: Optional[torch.Tensor] = None,
+                 err: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out[t] = sum of the distinct rows {row_of[t][j]} of Y, each once."""
+    _dev(Y, Y.dtype, "Y", 2)
+    _dev(row_of, torch.int32, "row_of", 2)
+    T, k = row_of.shape
+    R_max, d = Y.shape
+    if out is None:
+        out = torch.empty((T, d), dtype=out_dtype, device=Y.device)
+    err = new_err(Y.device) if err is None else err
+    st = lib().moe_combine_rows(_ptr(Y), _dtype_code(Y.dtype), R_max, d, _ptr(row_of), T, k, _ptr(out),
+                                _dtype_code(out.dtype), _ptr(err), _stream(Y))
+    _check("moe_combine_rows", st)
     return out
 
 
@@ -321,3 +426,15 @@ def place_correlated(coact_l, G: int, rpn: int) -> np.ndarray:
     out = np.empty(E, np.int32)
     _check("moe_place_correlated", lib().moe_place_correlated(_np_ptr(c), E, G, rpn, _np_ptr(out)))
     return out
+
+
+def place_replicas(coact_l, G: int, rpn: int, expert_to_rank, extra: int):
+    """(replica_rank int32 [E][1 + G/rpn], n_rep int32 [E]) on the host."""
+    c = np.ascontiguousarray(coact_l, dtype=np.uint32)
+    E = c.shape[0]
+    e2r = np.ascontiguousarray(expert_to_rank, dtype=np.int32)
+    rr = np.empty((E, 1 + G // rpn), np.int32)
+    nr = np.empty(E, np.int32)
+    _check("moe_place_replicas", lib().moe_place_replicas(_np_ptr(c), E, G, rpn, _np_ptr(e2r), extra,
+                                                          _np_ptr(rr), _np_ptr(nr)))
+    return rr, nr

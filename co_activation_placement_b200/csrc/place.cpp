@@ -12,6 +12,7 @@
 // The greedy keeps, for every unassigned expert, its running sum of Ochiai to
 // the current group's members; each new member adds its column once, so the
 // sum is accumulated in the order members joined (O(E^2) per level).
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <vector>
@@ -109,6 +110,51 @@ extern "C" moe_status moe_place_correlated(const uint32_t *coact, int E, int G, 
             if (node_of[e] == q) pool.push_back(e);
         const std::vector<int> grp = greedy_split(coact, E, pool, rpn);
         for (size_t x = 0; x < pool.size(); ++x) expert_to_rank[pool[x]] = q * rpn + grp[x];
+    }
+    return MOE_OK;
+}
+
+// Replica layout ("Cobalt", "Problem Formulation": every expert on at least one
+// rank, at most (1+rho)E/G experts per rank; "Two-Stage Expert Layout
+// Planner": co-activated experts share nodes).  Greedy, from a placement with
+// one replica per expert: every rank gets room for `extra` more experts; the
+// candidate replicas (e, node q), e not already on q, are taken in decreasing
+// order of score(e, q) = sum of C[e][e'] over the experts e' placed on q (ties:
+// lower e, then lower q); a candidate whose node has no room left is skipped
+// for good (room only shrinks), the others go on the rank of q with the most
+// room (ties: lowest rank).  Candidates scoring 0 are never added.
+extern "C" moe_status moe_place_replicas(const uint32_t *coact, int E, int G, int rpn, const int32_t *expert_to_rank,
+                                         int extra, int32_t *replica_rank, int32_t *n_rep)
+{
+    if (E < 1 || G < 1 || rpn < 1 || G % rpn != 0 || extra < 0 || !coact || !expert_to_rank || !replica_rank || !n_rep)
+        return MOE_ERR_ARG;
+    const int nodes = G / rpn, max_rep = 1 + nodes;
+    for (int e = 0; e < E; ++e)
+        if (expert_to_rank[e] < 0 || expert_to_rank[e] >= G) return MOE_ERR_DATA;
+    std::vector<uint64_t> score((size_t)E * nodes, 0);
+    for (int e = 0; e < E; ++e)
+        for (int f = 0; f < E; ++f)
+            if (f != e) score[(size_t)e * nodes + expert_to_rank[f] / rpn] += coact[(size_t)e * E + f];
+    struct Cand { uint64_t s; int e, q; };
+    std::vector<Cand> cands;
+    for (int e = 0; e < E; ++e) {
+        for (int q = 0; q < max_rep; ++q) replica_rank[(size_t)e * max_rep + q] = -1;
+        replica_rank[(size_t)e * max_rep] = expert_to_rank[e];
+        n_rep[e] = 1;
+        for (int q = 0; q < nodes; ++q)
+            if (q != expert_to_rank[e] / rpn && score[(size_t)e * nodes + q] > 0)
+                cands.push_back({score[(size_t)e * nodes + q], e, q});
+    }
+    std::stable_sort(cands.begin(), cands.end(), [](const Cand &a, const Cand &b) { return a.s > b.s; });
+    std::vector<int> room(G, extra);
+    for (const Cand &c : cands) {
+        int br = -1;
+        for (int r = c.q * rpn; r < (c.q + 1) * rpn; ++r)
+            if (room[r] > 0 && (br < 0 || room[r] > room[br])) br = r;
+        if (br < 0) continue;
+        room[br] -= 1;
+        replica_rank[(size_t)c.e * max_rep + n_rep[c.e]] = br;
+        n_rep[c.e] += 1;
     }
     return MOE_OK;
 }

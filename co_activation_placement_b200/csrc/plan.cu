@@ -15,8 +15,12 @@
 //      counts; the last block to finish scans the counts over chunks (column
 //      per rank), which yields every chunk's first row per rank, the rank
 //      segment offsets and counts[s][r] (chunks of one shard are adjacent);
-//   3. each chunk's block ranks its rows per destination with warp ballots
-//      (stable in perm order) and writes row_token, row_jmask and row_of.
+//   3. each chunk's block ranks its rows per destination, stable in perm
+//      order: a warp transposes its 32 x G destination bit matrix with five
+//      shuffle stages, so lane d holds the ballot of rank d; a row's rank in
+//      the warp is a popcount of that word below the lane, and warps are
+//      ordered by a prefix over the block.  It writes row_token, row_jmask and
+//      row_of.
 // All arithmetic is integer; the result is unique and does not depend on
 // scheduling.  No kernel waits on another block.
 #include <algorithm>
@@ -109,6 +113,21 @@ __device__ __forceinline__ int clamp_rank(int r, int G, int32_t *err)
         return 0;
     }
     return r;
+}
+
+// Transpose the warp's 32 x 32 bit matrix (lane r holds row r): afterwards
+// lane c holds column c, i.e. bit r of lane c's result = bit c of lane r's
+// input -- the ballot of bit c, for all 32 c at once (five butterfly stages).
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane)
+{
+    constexpr uint32_t kMask[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+    for (int st = 0; st < 5; ++st) {
+        const int j = 16 >> st;
+        const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+        x = (lane & j) ? ((x & ~kMask[st]) | ((y & ~kMask[st]) >> j)) : ((x & kMask[st]) | ((y & kMask[st]) << j));
+    }
+    return x;
 }
 
 // Last block: exclusive scan of a [B][G] column table (rows b, column d) into
@@ -237,18 +256,37 @@ struct ChunkRange {
     bool active;
 };
 
-__device__ __forceinline__ ChunkRange chunk_range(int b, int T, int G, bool with_src, const PlanWs &w)
+// Shard table of the source-sorted order, staged in shared memory once per
+// block (G + 1 entries each) so that locating a chunk costs no global loads.
+struct ShardTable {
+    int32_t soff[65], scnt[64], cpre[65];
+};
+
+__device__ __forceinline__ void load_shards(ShardTable &sh, int G, bool with_src, const PlanWs &w)
+{
+    if (!with_src) return;
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) {
+        sh.soff[i] = __ldcg(w.soff + i);
+        sh.cpre[i] = __ldcg(w.cpre + i);
+        if (i < G) sh.scnt[i] = __ldcg(w.scnt + i);
+    }
+}
+
+// Chunk b of the token sequence (call after load_shards and a barrier).
+__device__ __forceinline__ ChunkRange chunk_range(int b, int T, int G, bool with_src, const ShardTable &sh)
 {
     ChunkRange c;
     if (with_src) {
-        const int nact = __ldcg(w.cpre + G);
-        if (b >= nact) { c.active = false; c.s = 0; c.p0 = c.p1 = 0; return c; }
-        int s = 0;
-        while (s + 1 < G && __ldcg(w.cpre + s + 1) <= b) ++s;
-        const int base = __ldcg(w.soff + s), n = __ldcg(w.scnt + s);
+        if (b >= sh.cpre[G]) { c.active = false; c.s = 0; c.p0 = c.p1 = 0; return c; }
+        int lo = 0, hi = G - 1;   // last shard s with cpre[s] <= b
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sh.cpre[mid] <= b) lo = mid; else hi = mid - 1;
+        }
+        const int s = lo;
         c.s = s;
-        c.p0 = base + (b - __ldcg(w.cpre + s)) * kChunk;
-        c.p1 = min(base + n, c.p0 + kChunk);
+        c.p0 = sh.soff[s] + (b - sh.cpre[s]) * kChunk;
+        c.p1 = min(sh.soff[s] + sh.scnt[s], c.p0 + kChunk);
         c.active = true;
     } else {
         const int shard = T / G;
@@ -261,38 +299,67 @@ __device__ __forceinline__ ChunkRange chunk_range(int b, int T, int G, bool with
     return c;
 }
 
-template <int K>
+// Serving rank of each of a token's K picks: p(e) from the placement, or,
+// with PICKS, the per-(token, pick) ranks of a replica assignment.  Returns a
+// device error code (0 when the ranks are usable).
+template <int K, bool PICKS>
+__device__ __forceinline__ int serving_ranks(const int (&v)[K], const int32_t *e2r_sh,
+                                             const int32_t *__restrict__ picks, int t, int G, int (&r)[K])
+{
+    int bad = 0;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        if constexpr (PICKS) {
+            r[j] = __ldg(picks + (size_t)t * K + j);
+            if ((unsigned)r[j] >= (unsigned)G) {
+                bad = MOE_DERR_RANK_RANGE;
+                r[j] = 0;
+            }
+        } else {
+            r[j] = e2r_sh[v[j]];
+        }
+    }
+    return bad;
+}
+
+template <int K, bool PICKS>
 __global__ void __launch_bounds__(kChunk)
 plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
-                  const int32_t *__restrict__ e2r_g, bool with_src, PlanWs w, moe_plan P, int32_t *err)
+                  const int32_t *__restrict__ e2r_g, const int32_t *__restrict__ picks, bool with_src, PlanWs w,
+                  moe_plan P, int32_t *err)
 {
-    extern __shared__ int32_t e2r[];           // [E]
+    extern __shared__ int32_t e2r[];           // [E] (unused with PICKS)
     __shared__ int32_t cnt[64];
     __shared__ int32_t tot[64];
     __shared__ int32_t seg[kChunk];
     __shared__ unsigned long long red[4][kWarps];
+    __shared__ ShardTable sh;
     __shared__ bool last;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    for (int e = threadIdx.x; e < E; e += kChunk) e2r[e] = clamp_rank(__ldg(e2r_g + e), G, err);
+    if (!PICKS)
+        for (int e = threadIdx.x; e < E; e += kChunk) e2r[e] = clamp_rank(__ldg(e2r_g + e), G, err);
     if (threadIdx.x < 64) cnt[threadIdx.x] = 0;
+    load_shards(sh, G, with_src, w);
     __syncthreads();
 
-    const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, w);
+    const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, sh);
     unsigned long long my[4] = {0, 0, 0, 0};
     const int p = c.p0 + threadIdx.x;
+    unsigned long long m = 0;
     if (c.active && p < c.p1) {
         const int t = with_src ? __ldcg(w.perm + p) : p;
-        int v[K];
+        int v[K], rk[K];
         load_token<K>(ids + (size_t)t * K, v);
-        const int bad = token_error<K>(v, E);
-        unsigned long long m = 0, nodes = 0;
+        int bad = token_error<K>(v, E);
+        if (!bad) bad = serving_ranks<K, PICKS>(v, e2r, picks, t, G, rk);
+        unsigned long long nodes = 0;
         if (bad) {
             record_error(err, bad);
         } else {
             int local = 0;
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-                const int r = e2r[v[j]];
+                const int r = rk[j];
                 m |= 1ull << r;
                 nodes |= 1ull << (r / rpn);
                 local += r == c.s;
@@ -301,9 +368,14 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
             my[1] = __popcll(m & ~(1ull << c.s));
             my[2] = local;
             my[3] = __popcll(nodes & ~(1ull << (c.s / rpn)));
-            for (unsigned long long q = m; q; q &= q - 1) atomicAdd(&cnt[__ffsll((long long)q) - 1], 1);
         }
         P.dest_mask[t] = m;
+    }
+    {   // rows per rank: lane d counts column d (and d+32) of the warp's destination bits
+        const uint32_t clo = warp_transpose32((uint32_t)m, lane);
+        const uint32_t chi = warp_transpose32((uint32_t)(m >> 32), lane);
+        if (lane < G && clo) atomicAdd(&cnt[lane], __popc(clo));
+        if (lane + 32 < G && chi) atomicAdd(&cnt[lane + 32], __popc(chi));
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -326,7 +398,7 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
     __threadfence();
 
     // the last block: scan chunk counts, then offsets, counts and summary
-    const int B = with_src ? __ldcg(w.cpre + G) : gridDim.x;
+    const int B = with_src ? sh.cpre[G] : gridDim.x;
     scan_columns(w.blk, w.blk_pref, B, G, tot, seg);
     if (threadIdx.x == 0) {
         int run = 0;
@@ -338,7 +410,7 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
     for (int i = threadIdx.x; i < G * G; i += kChunk) {
         const int d = i / G, s = i % G;   // offsets in (d, s) order
         int b0, b1;
-        if (with_src) { b0 = __ldcg(w.cpre + s); b1 = __ldcg(w.cpre + s + 1); }
+        if (with_src) { b0 = sh.cpre[s]; b1 = sh.cpre[s + 1]; }
         else { const int nch = B / nshard; b0 = s * nch; b1 = b0 + nch; }
         const int a0 = __ldcg(w.blk_pref + (size_t)b0 * G + d);
         const int a1 = __ldcg(w.blk_pref + (size_t)b1 * G + d);
@@ -352,22 +424,27 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
 
 // ---- step 3: stable per-destination ranks and row writes -----------------
 
-template <int K>
+template <int K, bool PICKS>
 __global__ void __launch_bounds__(kChunk)
 plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
-                    const int32_t *__restrict__ e2r_g, bool with_src, PlanWs w, moe_plan P)
+                    const int32_t *__restrict__ e2r_g, const int32_t *__restrict__ picks, bool with_src, PlanWs w,
+                    moe_plan P)
 {
     extern __shared__ int32_t e2r[];           // [E]
     __shared__ int32_t base[64];               // first row of this chunk per rank
-    __shared__ int32_t wcnt[kWarps][64];
+    __shared__ int32_t wcnt[kWarps][64];       // rows per (warp, rank), then their exclusive prefix
+    __shared__ uint32_t colw[kWarps][64];      // lanes of the warp with a row for the rank
+    __shared__ ShardTable sh;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, w);
+    load_shards(sh, G, with_src, w);
+    __syncthreads();
+    const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, sh);
     if (!c.active) return;
-    for (int e = threadIdx.x; e < E; e += kChunk) {
-        const int r = __ldg(e2r_g + e);
-        e2r[e] = (unsigned)r >= (unsigned)G ? 0 : r;
-    }
-    for (int i = threadIdx.x; i < kWarps * 64; i += kChunk) (&wcnt[0][0])[i] = 0;
+    if (!PICKS)
+        for (int e = threadIdx.x; e < E; e += kChunk) {
+            const int r = __ldg(e2r_g + e);
+            e2r[e] = (unsigned)r >= (unsigned)G ? 0 : r;
+        }
     if (threadIdx.x < G)
         base[threadIdx.x] = __ldcg(P.offsets + threadIdx.x * G) + __ldcg(w.blk_pref + (size_t)blockIdx.x * G + threadIdx.x);
     __syncthreads();
@@ -379,25 +456,24 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
     if (act) {
         t = with_src ? __ldcg(w.perm + p) : p;
         load_token<K>(ids + (size_t)t * K, v);
-        if (token_error<K>(v, E) == 0) {
+        if (token_error<K>(v, E) == 0 && serving_ranks<K, PICKS>(v, e2r, picks, t, G, r) == 0) {
 #pragma unroll
-            for (int j = 0; j < K; ++j) {
-                r[j] = e2r[v[j]];
-                m |= 1ull << r[j];
-            }
+            for (int j = 0; j < K; ++j) m |= 1ull << r[j];
         } else {
 #pragma unroll
             for (int j = 0; j < K; ++j) P.row_of[(size_t)t * K + j] = -1;
         }
     }
-    const unsigned lt = (1u << lane) - 1u;
-    unsigned lo = __reduce_or_sync(0xffffffffu, (unsigned)m);
-    unsigned hi = __reduce_or_sync(0xffffffffu, (unsigned)(m >> 32));
-    unsigned long long wor = ((unsigned long long)hi << 32) | lo;
-    for (unsigned long long q = wor; q; q &= q - 1) {
-        const int d = __ffsll((long long)q) - 1;
-        const unsigned bal = __ballot_sync(0xffffffffu, (m >> d) & 1ull);
-        if (lane == 0) wcnt[wid][d] = __popc(bal);
+    // column d of the warp's 32 x G destination bit matrix: which lanes send to rank d
+    const uint32_t clo = warp_transpose32((uint32_t)m, lane);
+    const uint32_t chi = warp_transpose32((uint32_t)(m >> 32), lane);
+    if (lane < G) {
+        colw[wid][lane] = clo;
+        wcnt[wid][lane] = __popc(clo);
+    }
+    if (lane + 32 < G) {
+        colw[wid][lane + 32] = chi;
+        wcnt[wid][lane + 32] = __popc(chi);
     }
     __syncthreads();
     if (threadIdx.x < G) {
@@ -409,31 +485,30 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
         }
     }
     __syncthreads();
-    for (unsigned long long q = wor; q; q &= q - 1) {
+    // each lane writes its own rows: rank within the warp = earlier lanes with that rank
+    const unsigned lt = (1u << lane) - 1u;
+    for (unsigned long long q = m; q; q &= q - 1) {
         const int d = __ffsll((long long)q) - 1;
-        const unsigned bal = __ballot_sync(0xffffffffu, (m >> d) & 1ull);
-        if ((m >> d) & 1ull) {
-            const int pos = base[d] + wcnt[wid][d] + __popc(bal & lt);
-            unsigned jm = 0;
+        const int pos = base[d] + wcnt[wid][d] + __popc(colw[wid][d] & lt);
+        unsigned jm = 0;
 #pragma unroll
-            for (int j = 0; j < K; ++j)
-                if (r[j] == d) {
-                    jm |= 1u << j;
-                    P.row_of[(size_t)t * K + j] = pos;
-                }
-            P.row_token[pos] = t;
-            P.row_jmask[pos] = (uint8_t)jm;
-        }
+        for (int j = 0; j < K; ++j)
+            if (r[j] == d) {
+                jm |= 1u << j;
+                P.row_of[(size_t)t * K + j] = pos;
+            }
+        P.row_token[pos] = t;
+        P.row_jmask[pos] = (uint8_t)jm;
     }
 }
 
-template <int K>
-moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const int32_t *e2r,
+template <int K, bool PICKS>
+moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const int32_t *e2r, const int32_t *picks,
                        const int32_t *src_rank, const moe_plan &P, int32_t *err, const PlanWs &w,
                        cudaStream_t s)
 {
     const bool with_src = src_rank != nullptr;
-    const size_t smem = sizeof(int32_t) * (size_t)E;
+    const size_t smem = PICKS ? 0 : sizeof(int32_t) * (size_t)E;
     int launched = 0;
     if (with_src) {
         const int Bs = src_blocks(T);
@@ -442,10 +517,10 @@ moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const i
         launched += 2;
     }
     const int Bc = chunk_blocks(T, G, with_src);
-    if (allow_smem(plan_count_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
-    if (allow_smem(plan_scatter_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
-    plan_count_kernel<K><<<Bc, kChunk, smem, s>>>(ids, T, E, G, rpn, e2r, with_src, w, P, err);
-    plan_scatter_kernel<K><<<Bc, kChunk, smem, s>>>(ids, T, E, G, e2r, with_src, w, P);
+    if (allow_smem(plan_count_kernel<K, PICKS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    if (allow_smem(plan_scatter_kernel<K, PICKS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    plan_count_kernel<K, PICKS><<<Bc, kChunk, smem, s>>>(ids, T, E, G, rpn, e2r, picks, with_src, w, P, err);
+    plan_scatter_kernel<K, PICKS><<<Bc, kChunk, smem, s>>>(ids, T, E, G, e2r, picks, with_src, w, P);
     launched += 2;
     moe_status st = launch_status();
     if (st == MOE_OK) note_launches(launched);
@@ -464,15 +539,16 @@ extern "C" size_t moe_plan_dispatch_workspace(int T, int k, int G, int with_src_
     return carve(nullptr, T, G, with_src_rank != 0, nullptr) + 256;
 }
 
-extern "C" moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E, int G, int rpn,
-                                        const int32_t *expert_to_rank, const int32_t *src_rank,
-                                        const moe_plan *plan, int32_t *err,
-                                        void *ws, size_t ws_bytes, cudaStream_t stream)
+namespace {
+
+moe_status plan_entry(const int32_t *ids, int T, int k, int E, int G, int rpn, const int32_t *expert_to_rank,
+                      const int32_t *pick_rank, const int32_t *src_rank, const moe_plan *plan, int32_t *err,
+                      void *ws, size_t ws_bytes, cudaStream_t stream)
 {
     if (T < 0 || k < 1 || k > 8 || E < k || G < 1 || G > 64 || rpn < 1 || G % rpn != 0) return MOE_ERR_ARG;
     if ((long long)T * k >= (1ll << 31)) return MOE_ERR_ARG;
     if (E > 12 * 1024) return MOE_ERR_UNSUPPORTED;
-    if (!plan || !err || !expert_to_rank) return MOE_ERR_ARG;
+    if (!plan || !err || (!expert_to_rank && !pick_rank)) return MOE_ERR_ARG;
     if (!plan->counts || !plan->offsets || !plan->summary) return MOE_ERR_ARG;
     if (T > 0 && (!ids || !plan->dest_mask || !plan->row_token || !plan->row_jmask || !plan->row_of))
         return MOE_ERR_ARG;
@@ -488,15 +564,42 @@ extern "C" moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E,
     const size_t need = carve(ws, T, G, src_rank != nullptr, &w);
     if (!ws || !aligned256(ws) || ws_bytes < need) return MOE_ERR_WORKSPACE;
     if (cudaMemsetAsync(w.hdr, 0, sizeof(PlanWsHeader), stream) != cudaSuccess) return MOE_ERR_CUDA;
+    const int32_t *e2r = expert_to_rank;
+    const int32_t *pk = pick_rank;
+#define MOE_PLAN_CASE(KK)                                                                                  \
+    case KK:                                                                                               \
+        return pk ? launch_plan<KK, true>(ids, T, E, G, rpn, e2r, pk, src_rank, *plan, err, w, stream)   \
+                  : launch_plan<KK, false>(ids, T, E, G, rpn, e2r, pk, src_rank, *plan, err, w, stream);
     switch (k) {
-    case 1: return launch_plan<1>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
-    case 2: return launch_plan<2>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
-    case 3: return launch_plan<3>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
-    case 4: return launch_plan<4>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
-    case 5: return launch_plan<5>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
-    case 6: return launch_plan<6>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
-    case 7: return launch_plan<7>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
-    case 8: return launch_plan<8>(ids, T, E, G, rpn, expert_to_rank, src_rank, *plan, err, w, stream);
+        MOE_PLAN_CASE(1)
+        MOE_PLAN_CASE(2)
+        MOE_PLAN_CASE(3)
+        MOE_PLAN_CASE(4)
+        MOE_PLAN_CASE(5)
+        MOE_PLAN_CASE(6)
+        MOE_PLAN_CASE(7)
+        MOE_PLAN_CASE(8)
     }
+#undef MOE_PLAN_CASE
     return MOE_ERR_ARG;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                                        const int32_t *expert_to_rank, const int32_t *src_rank,
+                                        const moe_plan *plan, int32_t *err,
+                                        void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!expert_to_rank) return MOE_ERR_ARG;
+    return plan_entry(ids, T, k, E, G, rpn, expert_to_rank, nullptr, src_rank, plan, err, ws, ws_bytes, stream);
+}
+
+extern "C" moe_status moe_plan_dispatch_ranks(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                                              const int32_t *pick_rank, const int32_t *src_rank,
+                                              const moe_plan *plan, int32_t *err,
+                                              void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!pick_rank) return MOE_ERR_ARG;
+    return plan_entry(ids, T, k, E, G, rpn, nullptr, pick_rank, src_rank, plan, err, ws, ws_bytes, stream);
 }

@@ -30,7 +30,7 @@ namespace moe {
 namespace {
 
 constexpr int kRowThreads = 256;
-constexpr int kRowBlocksPerSM = 8;
+constexpr int kRowBlocksPerSM = 16;   // two waves of resident blocks: measured best for permute and combine
 
 // Warp-uniform per-token row list: dst[j] and a bitmask of the j that are the
 // first occurrence of a valid row.  Returns false (after recording the error)
@@ -153,13 +153,14 @@ template <> struct Elem<__nv_bfloat16> {
 // earlier lane (in j order) and drops out.  Returns the number of distinct
 // valid rows U; the q-th of them (in order of first appearance) is
 // (shfl(row, src[q]), shfl(W, src[q])).
-template <int K>
+template <int K, bool UNIT>
 __device__ __forceinline__ int token_distinct(const int32_t *__restrict__ idx, const float *__restrict__ w, int t,
                                               long long R_max, int &row, float &W, int (&src)[K], int32_t *err)
 {
     const int lane = threadIdx.x & 31;
     row = lane < K ? __ldg(idx + (size_t)t * K + lane) : -1;
-    const float wl = lane < K ? __ldg(w + (size_t)t * K + lane) : 0.f;
+    // UNIT: every distinct row counts once with weight 1 (repeats add nothing)
+    const float wl = UNIT ? 1.f : (lane < K ? __ldg(w + (size_t)t * K + lane) : 0.f);
     const bool valid = lane < K && row >= 0 && (long long)row < R_max;
     if (__any_sync(0xffffffffu, lane < K && !valid) && lane == 0) record_error(err, MOE_DERR_ROW_RANGE);
     bool first = valid;
@@ -169,7 +170,7 @@ __device__ __forceinline__ int token_distinct(const int32_t *__restrict__ idx, c
         const int rj = __shfl_sync(0xffffffffu, row, j);
         const float wj = __shfl_sync(0xffffffffu, wl, j);
         if (j < lane && rj == row) first = false;
-        if (j > lane && rj == row) W = __fadd_rn(W, wj);
+        if (!UNIT && j > lane && rj == row) W = __fadd_rn(W, wj);
     }
     unsigned m = __ballot_sync(0xffffffffu, first);
     const int U = __popc(m);
@@ -183,7 +184,7 @@ __device__ __forceinline__ int token_distinct(const int32_t *__restrict__ idx, c
 
 // Vectors are VB bytes of Y (N elements).  Distinct rows are read in chunks
 // of CH rows; U vectors per lane are in flight per row.
-template <int K, int CH, int U, typename YT, bool OUT_BF16, int VB>
+template <int K, int CH, int U, typename YT, bool OUT_BF16, int VB, bool UNIT>
 __global__ void __launch_bounds__(kRowThreads)
 combine_kernel(const char *__restrict__ Y, int nvec, long long R_max, const int32_t *__restrict__ idx,
                const float *__restrict__ w, int T, void *__restrict__ out, int32_t *err)
@@ -196,7 +197,7 @@ combine_kernel(const char *__restrict__ Y, int nvec, long long R_max, const int3
     for (int t = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); t < T; t += nwarps) {
         int row, src[K];
         float Wl;
-        const int Ut = token_distinct<K>(idx, w, t, R_max, row, Wl, src, err);
+        const int Ut = token_distinct<K, UNIT>(idx, w, t, R_max, row, Wl, src, err);
         int rc[K];
         float Wc[K];
 #pragma unroll
@@ -251,6 +252,99 @@ combine_kernel(const char *__restrict__ Y, int nvec, long long R_max, const int3
     }
 }
 
+// Gate dispatch: row i (< R, read from the plan's summary on the device)
+// carries (e_tj, w_tj) for the picks j of its token whose expert lives on the
+// row's rank, (-1, 0) for the others.
+__global__ void __launch_bounds__(kRowThreads)
+dispatch_gates_kernel(const int32_t *__restrict__ ids, const float *__restrict__ w, int T, int k,
+                      const int32_t *__restrict__ row_token, const uint8_t *__restrict__ row_jmask,
+                      const int64_t *__restrict__ summary, long long R_max, int32_t *__restrict__ send_e,
+                      float *__restrict__ send_w, int32_t *err)
+{
+    long long R = *summary;
+    if (R > R_max) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) record_error(err, MOE_DERR_ROW_RANGE);
+        R = R_max;
+    }
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < R; i += (long long)gridDim.x * blockDim.x) {
+        const int t = __ldg(row_token + i);
+        const unsigned jm = __ldg(row_jmask + i);
+        const bool ok = (unsigned)t < (unsigned)T;
+        if (!ok) record_error(err, MOE_DERR_ROW_RANGE);
+        for (int j = 0; j < k; ++j) {
+            const bool on = ok && ((jm >> j) & 1u);
+            send_e[i * k + j] = on ? __ldg(ids + (size_t)t * k + j) : -1;
+            send_w[i * k + j] = on ? __ldg(w + (size_t)t * k + j) : 0.f;
+        }
+    }
+}
+
+// Receiver-side pre-reduction with stand-in experts (expert e maps a row x
+// to scale[e] * x): y[i] = sum_j send_w[i][j] * scale[e_ij] * send[i] over the
+// row's experts, one warp per row.  g_j = send_w * scale is rounded to fp32
+// once, then the row is accumulated with fp32 FMAs in j order.
+template <int K, typename YT, bool OUT_BF16, int VB>
+__global__ void __launch_bounds__(kRowThreads)
+expert_reduce_kernel(const char *__restrict__ send, int nvec, const int64_t *__restrict__ summary, long long R_max,
+                     const int32_t *__restrict__ send_e, const float *__restrict__ send_w,
+                     const float *__restrict__ scale, int E, void *__restrict__ y, int32_t *err)
+{
+    constexpr int N = VB / Elem<YT>::BYTES;
+    constexpr int OW = OUT_BF16 ? N / 2 : N;
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * (kRowThreads / 32);
+    long long R = *summary;
+    if (R > R_max) R = R_max;
+    const size_t rowB = (size_t)nvec * VB;
+    for (long long i = (long long)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); i < R; i += nwarps) {
+        const int el = lane < K ? __ldg(send_e + i * K + lane) : -1;
+        const bool bad = __any_sync(0xffffffffu, el >= E);
+        if (bad && lane == 0) record_error(err, MOE_DERR_ID_RANGE);
+        const float gl = (el >= 0 && el < E) ? __fmul_rn(__ldg(send_w + i * K + lane), __ldg(scale + el)) : 0.f;
+        float g[K];
+        bool on[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            g[j] = __shfl_sync(0xffffffffu, gl, j);
+            on[j] = __shfl_sync(0xffffffffu, el, j) >= 0 && !bad;
+        }
+        const char *src = send + (size_t)i * rowB;
+        char *dst = static_cast<char *>(y) + (size_t)i * nvec * (OW * 4);
+        constexpr int U = 4;   // vectors per lane in flight
+        for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
+            Vw<VB> x[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (v0 + 32 * u < nvec) x[u] = ld_vec<VB>(src + (size_t)(v0 + 32 * u) * VB);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (v0 + 32 * u >= nvec) break;
+                float acc[N];
+#pragma unroll
+                for (int e = 0; e < N; ++e) acc[e] = 0.f;
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    if (!on[j]) continue;
+#pragma unroll
+                    for (int e = 0; e < N; ++e) acc[e] = __fmaf_rn(g[j], Elem<YT>::get(x[u].w, e), acc[e]);
+                }
+                uint32_t o[OW];
+                if constexpr (OUT_BF16) {
+#pragma unroll
+                    for (int q = 0; q < OW; ++q) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+                        o[q] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < OW; ++q) o[q] = __float_as_uint(acc[q]);
+                }
+                st_words<OW>(dst + (size_t)(v0 + 32 * u) * (OW * 4), o);
+            }
+        }
+    }
+}
+
 int row_grid(long long T)
 {
     const long long want = (long long)sm_count() * kRowBlocksPerSM;
@@ -277,7 +371,7 @@ moe_status launch_permute(const void *x, size_t rowB, int T, const int32_t *row_
 constexpr int kCombineU = 1;
 constexpr int kCombineChunk = 8;
 
-template <int K, typename YT, int VB>
+template <int K, typename YT, int VB, bool UNIT>
 moe_status launch_combine_vb(const void *Y, int nvec, long long R_max, const int32_t *idx, const float *w, int T,
                              void *out, bool out_bf16, int32_t *err, cudaStream_t s)
 {
@@ -285,38 +379,38 @@ moe_status launch_combine_vb(const void *Y, int nvec, long long R_max, const int
     constexpr int CH = K < kCombineChunk ? K : kCombineChunk;
     const char *y = static_cast<const char *>(Y);
     if (out_bf16)
-        combine_kernel<K, CH, U, YT, true, VB><<<row_grid(T), kRowThreads, 0, s>>>(y, nvec, R_max, idx, w, T, out, err);
+        combine_kernel<K, CH, U, YT, true, VB, UNIT><<<row_grid(T), kRowThreads, 0, s>>>(y, nvec, R_max, idx, w, T, out, err);
     else
-        combine_kernel<K, CH, U, YT, false, VB><<<row_grid(T), kRowThreads, 0, s>>>(y, nvec, R_max, idx, w, T, out, err);
+        combine_kernel<K, CH, U, YT, false, VB, UNIT><<<row_grid(T), kRowThreads, 0, s>>>(y, nvec, R_max, idx, w, T, out, err);
     return launch_status();
 }
 
 // 32-byte vectors when Y and out are 32-byte aligned and rows split evenly
 // into them (out rows are at least as long as Y rows), else 16-byte vectors.
-template <int K, typename YT>
+template <int K, typename YT, bool UNIT>
 moe_status launch_combine(const void *Y, size_t rowB, long long R_max, const int32_t *idx, const float *w, int T,
                           void *out, bool out_bf16, int32_t *err, cudaStream_t s)
 {
     const bool v32 = rowB % 32 == 0 && (reinterpret_cast<uintptr_t>(Y) & 31u) == 0 &&
                      (reinterpret_cast<uintptr_t>(out) & 31u) == 0 &&
                      (out_bf16 ? (sizeof(YT) == 2 || rowB % 64 == 0) : true);
-    if (v32) return launch_combine_vb<K, YT, 32>(Y, (int)(rowB / 32), R_max, idx, w, T, out, out_bf16, err, s);
-    return launch_combine_vb<K, YT, 16>(Y, (int)(rowB / 16), R_max, idx, w, T, out, out_bf16, err, s);
+    if (v32) return launch_combine_vb<K, YT, 32, UNIT>(Y, (int)(rowB / 32), R_max, idx, w, T, out, out_bf16, err, s);
+    return launch_combine_vb<K, YT, 16, UNIT>(Y, (int)(rowB / 16), R_max, idx, w, T, out, out_bf16, err, s);
 }
 
-template <typename YT>
+template <typename YT, bool UNIT>
 moe_status dispatch_combine_k(int k, const void *Y, size_t rowB, long long R_max, const int32_t *idx, const float *w,
                               int T, void *out, bool out_bf16, int32_t *err, cudaStream_t s)
 {
     switch (k) {
-    case 1: return launch_combine<1, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
-    case 2: return launch_combine<2, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
-    case 3: return launch_combine<3, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
-    case 4: return launch_combine<4, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
-    case 5: return launch_combine<5, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
-    case 6: return launch_combine<6, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
-    case 7: return launch_combine<7, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
-    case 8: return launch_combine<8, YT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 1: return launch_combine<1, YT, UNIT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 2: return launch_combine<2, YT, UNIT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 3: return launch_combine<3, YT, UNIT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 4: return launch_combine<4, YT, UNIT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 5: return launch_combine<5, YT, UNIT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 6: return launch_combine<6, YT, UNIT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 7: return launch_combine<7, YT, UNIT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
+    case 8: return launch_combine<8, YT, UNIT>(Y, rowB, R_max, idx, w, T, out, out_bf16, err, s);
     }
     return MOE_ERR_ARG;
 }
@@ -365,8 +459,102 @@ extern "C" moe_status moe_combine(const void *Y, moe_dtype y_dtype, int64_t R_ma
     if (rowB % 16) return MOE_ERR_UNSUPPORTED;
     const bool ob = out_dtype == MOE_BF16;
     moe_status st = y_dtype == MOE_BF16
-                        ? dispatch_combine_k<__nv_bfloat16>(k, Y, rowB, R_max, idx, w, T, out, ob, err, stream)
-                        : dispatch_combine_k<float>(k, Y, rowB, R_max, idx, w, T, out, ob, err, stream);
+                        ? dispatch_combine_k<__nv_bfloat16, false>(k, Y, rowB, R_max, idx, w, T, out, ob, err, stream)
+                        : dispatch_combine_k<float, false>(k, Y, rowB, R_max, idx, w, T, out, ob, err, stream);
+    if (st == MOE_OK) note_launches(1);
+    return st;
+}
+
+namespace moe {
+namespace {
+
+template <int K, typename YT, bool OB>
+moe_status launch_reduce(const void *send, size_t rowB, const int64_t *summary, long long R_max, const int32_t *se,
+                         const float *sw, const float *scale, int E, void *y, int32_t *err, cudaStream_t s)
+{
+    const char *sb = static_cast<const char *>(send);
+    const bool v32 = rowB % 32 == 0 && (reinterpret_cast<uintptr_t>(send) & 31u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(y) & 31u) == 0 && (!OB || sizeof(YT) == 2 || rowB % 64 == 0);
+    if (v32)
+        expert_reduce_kernel<K, YT, OB, 32><<<row_grid(R_max), kRowThreads, 0, s>>>(sb, (int)(rowB / 32), summary, R_max,
+                                                                                   se, sw, scale, E, y, err);
+    else
+        expert_reduce_kernel<K, YT, OB, 16><<<row_grid(R_max), kRowThreads, 0, s>>>(sb, (int)(rowB / 16), summary, R_max,
+                                                                                   se, sw, scale, E, y, err);
+    return launch_status();
+}
+
+template <typename YT, bool OB>
+moe_status reduce_k(int k, const void *send, size_t rowB, const int64_t *summary, long long R_max, const int32_t *se,
+                    const float *sw, const float *scale, int E, void *y, int32_t *err, cudaStream_t s)
+{
+    switch (k) {
+    case 1: return launch_reduce<1, YT, OB>(send, rowB, summary, R_max, se, sw, scale, E, y, err, s);
+    case 2: return launch_reduce<2, YT, OB>(send, rowB, summary, R_max, se, sw, scale, E, y, err, s);
+    case 3: return launch_reduce<3, YT, OB>(send, rowB, summary, R_max, se, sw, scale, E, y, err, s);
+    case 4: return launch_reduce<4, YT, OB>(send, rowB, summary, R_max, se, sw, scale, E, y, err, s);
+    case 5: return launch_reduce<5, YT, OB>(send, rowB, summary, R_max, se, sw, scale, E, y, err, s);
+    case 6: return launch_reduce<6, YT, OB>(send, rowB, summary, R_max, se, sw, scale, E, y, err, s);
+    case 7: return launch_reduce<7, YT, OB>(send, rowB, summary, R_max, se, sw, scale, E, y, err, s);
+    case 8: return launch_reduce<8, YT, OB>(send, rowB, summary, R_max, se, sw, scale, E, y, err, s);
+    }
+    return MOE_ERR_ARG;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_dispatch_gates(const int32_t *ids, const float *w, int T, int k,
+                                         const int32_t *row_token, const uint8_t *row_jmask, const int64_t *summary,
+                                         int64_t R_max, int32_t *send_e, float *send_w, int32_t *err,
+                                         cudaStream_t stream)
+{
+    if (T < 0 || k < 1 || k > 8 || R_max < 0 || !err) return MOE_ERR_ARG;
+    if (R_max == 0) return MOE_OK;
+    if (!ids || !w || !row_token || !row_jmask || !summary || !send_e || !send_w) return MOE_ERR_ARG;
+    dispatch_gates_kernel<<<row_grid(R_max / 8 + 1), kRowThreads, 0, stream>>>(ids, w, T, k, row_token, row_jmask,
+                                                                               summary, R_max, send_e, send_w, err);
+    moe_status st = launch_status();
+    if (st == MOE_OK) note_launches(1);
+    return st;
+}
+
+extern "C" moe_status moe_expert_reduce(const void *send, moe_dtype dtype, int64_t R_max, int d,
+                                        const int64_t *summary, const int32_t *send_e, const float *send_w, int k,
+                                        const float *scale, int E, void *y, moe_dtype y_dtype, int32_t *err,
+                                        cudaStream_t stream)
+{
+    const size_t eb = dtype_bytes(dtype);
+    if (!eb || !dtype_bytes(y_dtype) || R_max < 0 || d < 1 || k < 1 || k > 8 || E < 1 || !err) return MOE_ERR_ARG;
+    if (R_max == 0) return MOE_OK;
+    if (!send || !summary || !send_e || !send_w || !scale || !y || !aligned16(send) || !aligned16(y)) return MOE_ERR_ARG;
+    const size_t rowB = eb * (size_t)d;
+    if (rowB % 16) return MOE_ERR_UNSUPPORTED;
+    const bool ob = y_dtype == MOE_BF16;
+    moe_status st;
+    if (dtype == MOE_BF16)
+        st = ob ? reduce_k<__nv_bfloat16, true>(k, send, rowB, summary, R_max, send_e, send_w, scale, E, y, err, stream)
+                : reduce_k<__nv_bfloat16, false>(k, send, rowB, summary, R_max, send_e, send_w, scale, E, y, err, stream);
+    else
+        st = ob ? reduce_k<float, true>(k, send, rowB, summary, R_max, send_e, send_w, scale, E, y, err, stream)
+                : reduce_k<float, false>(k, send, rowB, summary, R_max, send_e, send_w, scale, E, y, err, stream);
+    if (st == MOE_OK) note_launches(1);
+    return st;
+}
+
+extern "C" moe_status moe_combine_rows(const void *Y, moe_dtype y_dtype, int64_t R_max, int d, const int32_t *row_of,
+                                       int T, int k, void *out, moe_dtype out_dtype, int32_t *err, cudaStream_t stream)
+{
+    const size_t eb = dtype_bytes(y_dtype);
+    if (!eb || !dtype_bytes(out_dtype) || T < 0 || d < 1 || k < 1 || k > 8 || R_max < 0 || !err) return MOE_ERR_ARG;
+    if (T == 0) return MOE_OK;
+    if (!Y || !row_of || !out || !aligned16(Y) || !aligned16(out)) return MOE_ERR_ARG;
+    const size_t rowB = eb * (size_t)d;
+    if (rowB % 16) return MOE_ERR_UNSUPPORTED;
+    const bool ob = out_dtype == MOE_BF16;
+    moe_status st = y_dtype == MOE_BF16
+                        ? dispatch_combine_k<__nv_bfloat16, true>(k, Y, rowB, R_max, row_of, nullptr, T, out, ob, err, stream)
+                        : dispatch_combine_k<float, true>(k, Y, rowB, R_max, row_of, nullptr, T, out, ob, err, stream);
     if (st == MOE_OK) note_launches(1);
     return st;
 }

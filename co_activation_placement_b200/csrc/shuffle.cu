@@ -10,9 +10,11 @@
 //
 // moe_rank_score: one block per expert row e, a shared uint64 accumulator per
 // rank (integer atomics: order-free).  moe_shuffle_targets: the E x G table
-// sits in shared memory; one warp per token, each lane owns ranks lane and
-// lane+32 (conflict-free: a row of the table is read contiguously), uint64
-// sums, and a warp argmax with (score desc, rank asc).
+// sits in shared memory (one block per SM, so it is copied once per SM); a
+// warp loads the picks of 32 tokens at once (one per lane) and then scores
+// them one at a time, each lane owning ranks lane and lane+32 (conflict-free:
+// a row of the table is read contiguously), with uint64 sums and a warp argmax
+// on (score desc, rank asc).
 #include <algorithm>
 
 #include "common.cuh"
@@ -52,40 +54,69 @@ __global__ void __launch_bounds__(kShuffleThreads)
 shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, const uint32_t *__restrict__ rs_g,
                        int32_t *__restrict__ target, int32_t *err)
 {
-    extern __shared__ uint32_t tab[];   // [E][G]
-    for (int i = threadIdx.x; i < E * G; i += kShuffleThreads) tab[i] = __ldg(rs_g + i);
+    extern __shared__ __align__(16) uint32_t tab[];   // [E][G]
+    {   // copy the table: 16-byte vectors where the layout allows, 8 in flight per thread
+        const int n = E * G;
+        const bool vec = (n % 4 == 0) && ((reinterpret_cast<uintptr_t>(rs_g) & 15u) == 0);
+        if (vec) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(rs_g);
+            uint4 *dst = reinterpret_cast<uint4 *>(tab);
+            for (int i0 = threadIdx.x; i0 < n / 4; i0 += 8 * kShuffleThreads) {
+                uint4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (i0 + u * kShuffleThreads < n / 4) v[u] = __ldg(src + i0 + u * kShuffleThreads);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (i0 + u * kShuffleThreads < n / 4) dst[i0 + u * kShuffleThreads] = v[u];
+            }
+        } else {
+            for (int i = threadIdx.x; i < n; i += kShuffleThreads) tab[i] = __ldg(rs_g + i);
+        }
+    }
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (kShuffleThreads / 32);
-    for (int t = blockIdx.x * (kShuffleThreads / 32) + (threadIdx.x >> 5); t < T; t += nwarps) {
-        const int mine = lane < K ? __ldg(ids + (size_t)t * K + lane) : 0;
-        const bool bad = __any_sync(0xffffffffu, lane < K && (unsigned)mine >= (unsigned)E);
-        if (bad) {
-            if (lane == 0) {
-                record_error(err, MOE_DERR_ID_RANGE);
-                target[t] = 0;
-            }
-            continue;
-        }
-        unsigned long long a0 = 0, a1 = 0;
+    const int gw = blockIdx.x * (kShuffleThreads / 32) + (threadIdx.x >> 5);
+    // a warp takes 32 tokens at a time: lane l loads token t0+l's picks, then
+    // the warp scores the 32 tokens one after another
+    for (int t0 = gw * 32; t0 < T; t0 += nwarps * 32) {
+        const int tl = t0 + lane;
+        int e[K];
+        bool ok = tl < T;
 #pragma unroll
         for (int j = 0; j < K; ++j) {
-            const int e = __shfl_sync(0xffffffffu, mine, j);
-            const uint32_t *row = tab + (size_t)e * G;
-            if (lane < G) a0 += row[lane];
-            if (lane + 32 < G) a1 += row[lane + 32];
+            e[j] = tl < T ? __ldg(ids + (size_t)tl * K + j) : 0;
+            ok &= (unsigned)e[j] < (unsigned)E;
         }
-        // candidate key: score + 1 for a real rank, 0 for none
-        unsigned long long best = lane < G ? a0 + 1 : 0;
-        int bi = lane;
-        if (lane + 32 < G && a1 + 1 > best) { best = a1 + 1; bi = lane + 32; }
+        if (tl < T && !ok) record_error(err, MOE_DERR_ID_RANGE);
+        const int n = min(32, T - t0);
+        int result = 0;
+        for (int i = 0; i < n; ++i) {
+            const bool good = __shfl_sync(0xffffffffu, ok, i);
+            unsigned long long a0 = 0, a1 = 0;
 #pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+            for (int j = 0; j < K; ++j) {
+                const int ej = __shfl_sync(0xffffffffu, e[j], i);
+                if (good) {
+                    const uint32_t *row = tab + (size_t)ej * G;
+                    if (lane < G) a0 += row[lane];
+                    if (lane + 32 < G) a1 += row[lane + 32];
+                }
+            }
+            // candidate key: score + 1 for a real rank, 0 for none
+            unsigned long long best = lane < G ? a0 + 1 : 0;
+            int bi = lane;
+            if (lane + 32 < G && a1 + 1 > best) { best = a1 + 1; bi = lane + 32; }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+            }
+            if (lane == i) result = good ? bi : 0;
         }
-        if (lane == 0) target[t] = bi;
+        if (tl < T) target[tl] = result;
     }
 }
 
@@ -111,7 +142,7 @@ static moe_status launch_shuffle(const int32_t *ids, int T, int E, int G, const 
     const size_t smem = sizeof(uint32_t) * (size_t)E * G;
     if (allow_smem(shuffle_targets_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
     // one block per SM at most: every block first copies the whole table
-    const long long need = ((long long)T + (kShuffleThreads / 32) - 1) / (kShuffleThreads / 32);
+    const long long need = ((long long)T + kShuffleThreads - 1) / kShuffleThreads;
     const int grid = (int)std::max<long long>(1, std::min<long long>(need, (long long)sm_count()));
     shuffle_targets_kernel<K><<<grid, kShuffleThreads, smem, s>>>(ids, T, E, G, rs, target, err);
     return launch_status();

@@ -40,10 +40,12 @@ class StepBytes:
     plan: int = 0
     stats: int = 0
     shuffle: int = 0
+    gates: int = 0
+    reduce: int = 0
 
     @property
     def dispatch_combine(self) -> int:
-        return self.permute + self.combine
+        return self.permute + self.gates + self.reduce + self.combine
 
 
 @dataclass
@@ -59,6 +61,9 @@ class HotPath:
     out_dtype: torch.dtype = torch.bfloat16
     rows: bool = True                  # run plan/permute/combine (False: statistics only)
     timers: bool = False               # record CUDA events around each library call
+    prereduce: bool = False            # receiver-side pre-reduced combine with stand-in experts
+    scales: List[torch.Tensor] = field(default_factory=list)   # f32 [E] per layer (prereduce)
+    replicas: list = field(default_factory=list)   # per layer (replica_rank [E][1+nodes], n_rep [E]) or empty
     # buffers
     stats: dict = field(default_factory=dict)
     plans: List[cap.Plan] = field(default_factory=list)
@@ -87,11 +92,21 @@ class HotPath:
         self.send = torch.empty((T * k, d), dtype=self.x.dtype, device=dev)
         self.outs = [torch.empty((T, d), dtype=self.out_dtype, device=dev) for _ in range(L)]
         self.targets = [torch.empty(T, dtype=torch.int32, device=dev) for _ in range(max(L - 1, 0))] if self.shuffle else []
+        if self.replicas:
+            self.pick_rank = torch.empty((T, k), dtype=torch.int32, device=dev)
+            self.n_remote = torch.empty(T, dtype=torch.int32, device=dev)
+        if self.prereduce:
+            if len(self.scales) != L:
+                raise ValueError("prereduce needs one scale vector per layer")
+            self.send_e = torch.empty((T * k, k), dtype=torch.int32, device=dev)
+            self.send_w = torch.empty((T * k, k), dtype=torch.float32, device=dev)
+            self.y = torch.empty((T * k, d), dtype=self.x.dtype, device=dev)
 
     # ------------------------------------------------------------------ step
     def _mark(self, name):
         if self.timers:
-            ev = torch.cuda.Event(enable_timing=True)
+            # external: inside a captured graph this is a real event-record node
+            ev = torch.cuda.Event(enable_timing=True, external=True)
             ev.record()
             self.events.append((name, ev))
 
@@ -107,17 +122,50 @@ class HotPath:
             return
         for l in range(self.L):
             src = self.targets[l - 1] if (self.shuffle and l > 0) else None
-            p = cap.plan_dispatch(self.ids[l], self.E, self.G, self.rpn, self.e2r[l], src_rank=src,
-                                  plan=self.plans[l], ws=self.plan_ws)
+            if self.replicas:
+                # each task to a replica of its expert: fewest remote nodes per token
+                rr, nr = self.replicas[l]
+                cap.assign_replicas(self.ids[l], self.E, self.G, self.rpn, rr, nr, src_rank=src,
+                                    pick_rank=self.pick_rank, n_remote=self.n_remote, err=self.err)
+                p = cap.plan_dispatch_ranks(self.ids[l], self.E, self.G, self.rpn, self.pick_rank, src_rank=src,
+                                            plan=self.plans[l], ws=self.plan_ws)
+            else:
+                p = cap.plan_dispatch(self.ids[l], self.E, self.G, self.rpn, self.e2r[l], src_rank=src,
+                                      plan=self.plans[l], ws=self.plan_ws)
             self._mark("plan")
             cap.permute(self.x, p.row_of, p.R_max, send=self.send, err=self.err)
             self._mark("permute")
-            cap.combine(self.send, p.row_of, self.gates[l], out=self.outs[l], err=self.err)
-            self._mark("combine")
+            if self.prereduce:
+                # gates travel with the rows; the receiving rank applies its
+                # experts and returns one row per (token, rank); the source sums
+                cap.dispatch_gates(self.ids[l], self.gates[l], p, send_e=self.send_e, send_w=self.send_w,
+                                   err=self.err)
+                self._mark("gates")
+                cap.expert_reduce(self.send, p.summary, self.send_e, self.send_w, self.scales[l], y=self.y,
+                                  err=self.err)
+                self._mark("reduce")
+                cap.combine_rows(self.y, p.row_of, out=self.outs[l], err=self.err)
+                self._mark("combine")
+            else:
+                cap.combine(self.send, p.row_of, self.gates[l], out=self.outs[l], err=self.err)
+                self._mark("combine")
             if self.shuffle and l + 1 < self.L:
                 cap.shuffle_targets(self.ids[l], self.E, self.G, self.rank_scores[l],
                                     target=self.targets[l], err=self.err)
                 self._mark("shuffle")
+
+    def capture(self, n_steps: int) -> torch.cuda.CUDAGraph:
+        """Capture n_steps consecutive steps into one CUDA graph.  The library
+        allocates nothing and every buffer is preallocated, so replaying the
+        graph reruns exactly these steps.  Timing events (if on) are captured
+        as event-record nodes; read them with kernel_times_ms() after a replay."""
+        g = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize()
+        self.reset_events()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for _ in range(n_steps):
+                self.step()
+        return g
 
     def kernel_times_ms(self):
         """Device time (ms) of each kind of call, summed over all steps run
@@ -143,8 +191,16 @@ class HotPath:
             R = int(summaries[l][0])
             src_b = 4 * T if (self.shuffle and l > 0) else 0
             b.plan += T * k * 4 + E * 4 + src_b + 8 * T + 5 * R + 4 * T * k + 8 * self.G * self.G
+            if self.replicas:   # the assignment reads ids, writes pick ranks; the plan reads them back
+                b.plan += T * k * 4 + T * k * 4 + 4 * T + T * k * 4
             b.permute += T * rowB + R * rowB + 4 * T * k
-            b.combine += R * rowB + T * outB + 8 * T * k
+            if self.prereduce:
+                # gates: row_token + jmask read, (e, w) gathered and written per row slot
+                b.gates += 5 * R + 8 * T * k + 8 * R * k
+                b.reduce += R * rowB + R * rowB + 8 * R * k + 4 * self.E
+                b.combine += R * rowB + T * outB + 4 * T * k
+            else:
+                b.combine += R * rowB + T * outB + 8 * T * k
             if self.shuffle and l + 1 < L:
                 b.shuffle += T * k * 4 + E * self.G * 4 + 4 * T
         return b
@@ -153,7 +209,8 @@ class HotPath:
         return torch.stack([p.summary for p in self.plans]).cpu().numpy()
 
 
-def calibrate(ids_cal: torch.Tensor, E: int, G: int, rpn: int, placement: str, shuffle: bool):
+def calibrate(ids_cal: torch.Tensor, E: int, G: int, rpn: int, placement: str, shuffle: bool,
+              replica_extra: int = 0):
     """Placements and rank-score tables from a calibration batch (int32
     [L][T][k] on the device): its statistics come from moe_coact_stats, the
     placement from the host greedy, the tables from moe_rank_score.
@@ -176,22 +233,32 @@ def calibrate(ids_cal: torch.Tensor, E: int, G: int, rpn: int, placement: str, s
     if shuffle:
         for l in range(L - 1):
             rs.append(cap.rank_score(st["trans"][l], e2r[l + 1], G))
-    return e2r, rs, coact_h
+    reps = []
+    if replica_extra > 0:
+        for l in range(L):
+            rr, nr = cap.place_replicas(coact_h[l], G, rpn, e2r_h[l], replica_extra)
+            reps.append((torch.from_numpy(rr).to(ids_cal.device), torch.from_numpy(nr).to(ids_cal.device)))
+    return e2r, rs, coact_h, reps
 
 
 def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarray], x: Optional[np.ndarray],
             x_dtype: str, ids_cal: np.ndarray, placement: str = "correlated", shuffle: bool = True,
-            out_dtype=torch.bfloat16, device="cuda", rows: bool = True, timers: bool = False) -> HotPath:
+            out_dtype=torch.bfloat16, device="cuda", rows: bool = True, timers: bool = False,
+            scales: Optional[np.ndarray] = None, replica_extra: int = 0) -> HotPath:
     """Upload a batch (host numpy arrays; x as float32 or bf16 bit patterns)
     and its calibration batch, calibrate, and return the step's HotPath."""
     dev = torch.device(device)
     ids_d = torch.from_numpy(np.ascontiguousarray(ids, dtype=np.int32)).to(dev)
     cal_d = torch.from_numpy(np.ascontiguousarray(ids_cal, dtype=np.int32)).to(dev)
-    e2r, rs, _ = calibrate(cal_d, E, G, rpn, placement, shuffle and ids.shape[0] > 1) if rows else ([], [], None)
+    e2r, rs, _, reps = calibrate(cal_d, E, G, rpn, placement, shuffle and ids.shape[0] > 1, replica_extra) \
+        if rows else ([], [], None, [])
     gates_d = torch.from_numpy(np.ascontiguousarray(gates, dtype=np.float32)).to(dev) if rows else None
     if rows:
         x_d = (bf16_from_bits(x) if x_dtype == "bf16" else torch.from_numpy(np.ascontiguousarray(x, np.float32))).to(dev)
     else:
         x_d = None
+    scales_d = [torch.from_numpy(np.ascontiguousarray(s_, dtype=np.float32)).to(dev) for s_ in scales] \
+        if scales is not None else []
     return HotPath(E=E, G=G, rpn=rpn, ids=ids_d, gates=gates_d, x=x_d, e2r=e2r, rank_scores=rs,
-                   out_dtype=out_dtype, rows=rows, timers=timers)
+                   out_dtype=out_dtype, rows=rows, timers=timers, prereduce=scales is not None, scales=scales_d,
+                   replicas=reps)

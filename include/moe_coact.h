@@ -145,6 +145,39 @@ moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E, int G, int
                              const moe_plan *plan, int32_t *err,
                              void *ws, size_t ws_bytes, cudaStream_t stream);
 
+/* The same plan when experts have several replicas ([CB] "Problem
+ * Formulation": task (t, e) runs on a rank r_t^e holding e): pick_rank
+ * device int32 [T][k] gives the serving rank of every pick (e.g. from
+ * moe_assign_replicas), in place of p(e).  Rows, order, outputs, workspace
+ * and errors as moe_plan_dispatch; a pick rank outside [0, G) is
+ * MOE_DERR_RANK_RANGE. */
+moe_status moe_plan_dispatch_ranks(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                                   const int32_t *pick_rank, const int32_t *src_rank,
+                                   const moe_plan *plan, int32_t *err,
+                                   void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Communication-aware task assignment over replicas  ([CB] "Problem
+ * Formulation": V counts the remote nodes a token's tasks reach; the
+ * assignment "routes tokens to the fewest remote nodes possible")
+ *
+ * For every token t (source rank s = src_rank[t], or t/(T/G) when NULL; node
+ * ns = s / rpn): the smallest set S of nodes other than ns such that every
+ * pick's expert has a replica on ns or on a node of S (exact; ties: smallest
+ * S as a bit pattern); then, pick by pick in j order, among the ranks hosting
+ * the expert on ns (or, if none, on the nodes of S): rank s if it is one of
+ * them, else the lowest one an earlier pick of the token already uses (no new
+ * row), else the lowest one.  n_remote[t] = |S|, the token's share of V.
+ * replica_rank device int32 [E][1 + G/rpn] (ranks, unused slots -1) and
+ * n_rep device int32 [E], e.g. from moe_place_replicas; pick_rank device
+ * int32 [T][k] out; n_remote device int32 [T] out or NULL.
+ * Limits: G/rpn <= 8 nodes.  Data errors: MOE_DERR_ID_RANGE (invalid ids or an
+ * expert without replicas; the token's outputs are -1), MOE_DERR_RANK_RANGE.
+ * ---------------------------------------------------------------------- */
+moe_status moe_assign_replicas(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                               const int32_t *replica_rank, const int32_t *n_rep, const int32_t *src_rank,
+                               int32_t *pick_rank, int32_t *n_remote, int32_t *err, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------
  * Dispatch plan without caller-provided workspace.  The pages have no
  * counterpart: this entry point exists for callers that cannot allocate
@@ -211,6 +244,45 @@ moe_status moe_combine(const void *Y, moe_dtype y_dtype, int64_t R_max, int d,
                        void *out, moe_dtype out_dtype, int32_t *err, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Receiver-side pre-reduced combine  ([CE] footnote 3: the dispatcher moves
+ * hidden states and routed probabilities; [EC]: dispatch, then combine)
+ *
+ * With deduplicated dispatch a row reaches its rank once however many of the
+ * token's experts live there.  The receiving rank can then apply those
+ * experts, weight their outputs with the dispatched gates and return a single
+ * row per (token, rank); the source only sums its rows.
+ *
+ * moe_dispatch_gates: for each row i < R (R = summary[0], read on the device):
+ *   send_e[i][j] = e_tj and send_w[i][j] = w[t][j] for the picks j of token
+ *   t = row_token[i] with bit j of row_jmask[i] set; -1 and 0 otherwise.
+ *   ids device int32 [T][k]; w device float [T][k]; row_token, row_jmask,
+ *   summary from moe_plan_dispatch; send_e device int32 [R_max][k]; send_w
+ *   device float [R_max][k].  Data errors: MOE_DERR_ROW_RANGE.
+ *
+ * moe_expert_reduce: stand-in experts, expert e mapping a row x to scale[e]*x:
+ *   y[i] = sum_j send_w[i][j] * scale[send_e[i][j]] * send[i]  (j with
+ *   send_e >= 0), for i < R: g_j = send_w * scale rounded to fp32 once, then an
+ *   fp32 FMA chain in j order; y fp32 or rounded to bf16 (nearest even).
+ *   send device [R_max][d] of dtype; scale device float [E]; y device
+ *   [R_max][d] of y_dtype (both 16-byte aligned; rows a multiple of 16 bytes).
+ *   Data errors: MOE_DERR_ID_RANGE (send_e >= E; the row is not reduced).
+ *
+ * moe_combine_rows: out[t] = sum of the distinct rows {row_of[t][j]} of Y,
+ *   each once (weight 1), fp32 accumulation in order of first appearance;
+ *   Y device [R_max][d] of y_dtype, row_of device int32 [T][k], out device
+ *   [T][d] of out_dtype.  Data errors: MOE_DERR_ROW_RANGE.
+ * ---------------------------------------------------------------------- */
+moe_status moe_dispatch_gates(const int32_t *ids, const float *w, int T, int k,
+                              const int32_t *row_token, const uint8_t *row_jmask, const int64_t *summary,
+                              int64_t R_max, int32_t *send_e, float *send_w, int32_t *err, cudaStream_t stream);
+moe_status moe_expert_reduce(const void *send, moe_dtype dtype, int64_t R_max, int d,
+                             const int64_t *summary, const int32_t *send_e, const float *send_w, int k,
+                             const float *scale, int E, void *y, moe_dtype y_dtype, int32_t *err,
+                             cudaStream_t stream);
+moe_status moe_combine_rows(const void *Y, moe_dtype y_dtype, int64_t R_max, int d, const int32_t *row_of,
+                            int T, int k, void *out, moe_dtype out_dtype, int32_t *err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Token shuffling  ([EC]: move each token to the GPU predicted to hold its
  * next-layer experts)
  *
@@ -257,6 +329,20 @@ moe_status moe_shuffle_targets(const int32_t *ids, int T, int k, int E, int G,
 moe_status moe_place_uniform(int E, int G, int32_t *expert_to_rank);
 moe_status moe_place_capacity(const double *load, int E, int G, int32_t *expert_to_rank, double *rank_load);
 moe_status moe_place_correlated(const uint32_t *coact, int E, int G, int rpn, int32_t *expert_to_rank);
+
+/* moe_place_replicas ([CB] "Problem Formulation": every expert has at least
+ *   one replica, |P_r| <= (1+rho)E/G; "Two-Stage Expert Layout Planner":
+ *   co-activated experts share nodes).  The page states the constraints, not
+ *   an algorithm; this is a greedy.  Starting from expert_to_rank (one replica
+ *   each), every rank gets room for `extra` more experts (extra = rho*E/G);
+ *   candidate replicas (e, node q), e not on q, are taken in decreasing
+ *   score(e, q) = sum of coact[e][e'] over the experts e' placed on q (ties:
+ *   lower e, then lower q), each onto the rank of q with the most room left
+ *   (ties: lowest rank), skipping nodes without room; zero scores are not added.
+ *   replica_rank host int32 [E][1 + G/rpn] out (original rank first, then in
+ *   the order added; -1 unused), n_rep host int32 [E] out. */
+moe_status moe_place_replicas(const uint32_t *coact, int E, int G, int rpn, const int32_t *expert_to_rank,
+                              int extra, int32_t *replica_rank, int32_t *n_rep);
 
 #ifdef __cplusplus
 }

@@ -36,7 +36,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        # ORACLE_LIB points the pins at another build of oracle.c (the
+        # mutation test plants mistakes in copies and expects the pins to fail)
+        _lib = ctypes.CDLL(os.environ.get("ORACLE_LIB") or build())
         P = ctypes.c_void_p
         i = ctypes.c_int
         i64 = ctypes.c_int64
@@ -50,6 +52,12 @@ def lib():
             "orc_combine": [P, i, i64, i, P, P, i, i, P],
             "orc_rank_score": [P, P, i, i, P],
             "orc_shuffle_targets": [P, i, i, i, i, P, P],
+            "orc_dispatch_gates": [P, P, i, i, P, P, i64, P, P],
+            "orc_expert_reduce": [P, i, i64, i, P, P, i, P, i, P],
+            "orc_combine_rows": [P, i, i64, i, P, i, i, P],
+            "orc_plan_ranks": [P, i, i, i, i, i, P, P, P, P, P, P, P, P, P],
+            "orc_place_replicas": [P, i, i, i, P, i, P, P],
+            "orc_assign_replicas": [P, i, i, i, i, i, P, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(_lib, name)
@@ -113,11 +121,13 @@ def place_correlated(coact_l: np.ndarray, G: int, rpn: int) -> np.ndarray:
     return e2r
 
 
-def plan(ids_l: np.ndarray, E: int, G: int, rpn: int, expert_to_rank: np.ndarray, src_rank=None):
-    """ids_l int32 [T][k] (one layer) -> dict of plan arrays (row arrays trimmed to R)."""
+def plan(ids_l: np.ndarray, E: int, G: int, rpn: int, expert_to_rank: np.ndarray, src_rank=None, pick_rank=None):
+    """ids_l int32 [T][k] (one layer) -> dict of plan arrays (row arrays trimmed to R).
+    With pick_rank int32 [T][k] the serving rank of every pick is given (expert_to_rank ignored)."""
     ids_l = np.ascontiguousarray(ids_l, dtype=np.int32)
     T, k = ids_l.shape
-    e2r = np.ascontiguousarray(expert_to_rank, dtype=np.int32)
+    e2r = None if expert_to_rank is None else np.ascontiguousarray(expert_to_rank, dtype=np.int32)
+    pr = None if pick_rank is None else np.ascontiguousarray(pick_rank, dtype=np.int32)
     src = None if src_rank is None else np.ascontiguousarray(src_rank, dtype=np.int32)
     dm = np.empty(T, np.uint64)
     counts = np.empty((G, G), np.int32)
@@ -126,8 +136,13 @@ def plan(ids_l: np.ndarray, E: int, G: int, rpn: int, expert_to_rank: np.ndarray
     row_jmask = np.empty(max(T * k, 1), np.uint8)
     row_of = np.empty((T, k), np.int32)
     summary = np.empty(5, np.int64)
-    _check("orc_plan", lib().orc_plan(_p(ids_l), T, k, E, G, rpn, _p(e2r), _p(src), _p(dm), _p(counts),
-                                      _p(offsets), _p(row_token), _p(row_jmask), _p(row_of), _p(summary)))
+    if pr is None:
+        _check("orc_plan", lib().orc_plan(_p(ids_l), T, k, E, G, rpn, _p(e2r), _p(src), _p(dm), _p(counts),
+                                          _p(offsets), _p(row_token), _p(row_jmask), _p(row_of), _p(summary)))
+    else:
+        _check("orc_plan_ranks", lib().orc_plan_ranks(_p(ids_l), T, k, E, G, rpn, _p(pr), _p(src), _p(dm),
+                                                      _p(counts), _p(offsets), _p(row_token), _p(row_jmask),
+                                                      _p(row_of), _p(summary)))
     R = int(summary[0])
     return dict(dest_mask=dm, counts=counts, offsets=offsets, row_token=row_token[:R].copy(),
                 row_jmask=row_jmask[:R].copy(), row_of=row_of, summary=summary,
@@ -171,3 +186,66 @@ def shuffle_targets(ids_l: np.ndarray, E: int, G: int, rank_score_tab: np.ndarra
     tgt = np.empty(T, np.int32)
     _check("orc_shuffle_targets", lib().orc_shuffle_targets(_p(ids_l), T, k, E, G, _p(rs), _p(tgt)))
     return tgt
+
+
+def dispatch_gates(ids_l, w_l, row_token, row_jmask):
+    """(send_e int32 [R][k], send_w f32 [R][k]) for the plan's rows."""
+    ids_l = np.ascontiguousarray(ids_l, dtype=np.int32)
+    w_l = np.ascontiguousarray(w_l, dtype=np.float32)
+    T, k = ids_l.shape
+    rt = np.ascontiguousarray(row_token, dtype=np.int32)
+    jm = np.ascontiguousarray(row_jmask, dtype=np.uint8)
+    R = rt.size
+    se = np.empty((R, k), np.int32)
+    sw = np.empty((R, k), np.float32)
+    _check("orc_dispatch_gates", lib().orc_dispatch_gates(_p(ids_l), _p(w_l), T, k, _p(rt), _p(jm), R, _p(se), _p(sw)))
+    return se, sw
+
+
+def expert_reduce(send, send_e, send_w, scale, y_is_bf16):
+    """fp64 y [R][d]: per row, the gate-weighted sum of the stand-in experts' outputs."""
+    send = np.ascontiguousarray(send)
+    R, d = send.shape
+    se = np.ascontiguousarray(send_e, dtype=np.int32)
+    sw = np.ascontiguousarray(send_w, dtype=np.float32)
+    sc = np.ascontiguousarray(scale, dtype=np.float32)
+    y = np.empty((R, d), np.float64)
+    _check("orc_expert_reduce", lib().orc_expert_reduce(_p(send), int(bool(y_is_bf16)), R, d, _p(se), _p(sw),
+                                                        se.shape[1], _p(sc), sc.size, _p(y)))
+    return y
+
+
+def combine_rows(y, row_of, y_is_bf16=False):
+    """fp64 out [T][d]: each token's distinct pre-reduced rows summed once (y float32 or bf16 bits)."""
+    y = np.ascontiguousarray(y)
+    R, d = y.shape
+    ro = np.ascontiguousarray(row_of, dtype=np.int32)
+    T, k = ro.shape
+    out = np.empty((T, d), np.float64)
+    _check("orc_combine_rows", lib().orc_combine_rows(_p(y), int(bool(y_is_bf16)), R, d, _p(ro), T, k, _p(out)))
+    return out
+
+
+def place_replicas(coact_l, G: int, rpn: int, expert_to_rank, extra: int):
+    """(replica_rank int32 [E][1 + G/rpn], n_rep int32 [E])."""
+    c = np.ascontiguousarray(coact_l, dtype=np.uint32)
+    E = c.shape[0]
+    e2r = np.ascontiguousarray(expert_to_rank, dtype=np.int32)
+    rr = np.empty((E, 1 + G // rpn), np.int32)
+    nr = np.empty(E, np.int32)
+    _check("orc_place_replicas", lib().orc_place_replicas(_p(c), E, G, rpn, _p(e2r), extra, _p(rr), _p(nr)))
+    return rr, nr
+
+
+def assign_replicas(ids_l, E: int, G: int, rpn: int, replica_rank, n_rep, src_rank=None):
+    """(pick_rank int32 [T][k], n_remote int32 [T])."""
+    ids_l = np.ascontiguousarray(ids_l, dtype=np.int32)
+    T, k = ids_l.shape
+    rr = np.ascontiguousarray(replica_rank, dtype=np.int32)
+    nr = np.ascontiguousarray(n_rep, dtype=np.int32)
+    src = None if src_rank is None else np.ascontiguousarray(src_rank, dtype=np.int32)
+    pr = np.empty((T, k), np.int32)
+    nrem = np.empty(T, np.int32)
+    _check("orc_assign_replicas", lib().orc_assign_replicas(_p(ids_l), T, k, E, G, rpn, _p(rr), _p(nr), _p(src),
+                                                            _p(pr), _p(nrem)))
+    return pr, nrem

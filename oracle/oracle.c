@@ -258,19 +258,31 @@ static int cmp_row(const void *pa, const void *pb)
  *                  local = #{(t,j) : p(e_tj) = s_t},
  *                  V = sum_t |{N(p(e)) : e in D_t} \ {N(s_t)}|,  T*k }
  * row_token / row_jmask must hold T*k entries. */
-int orc_plan(const int32_t *ids, int T, int k, int E, int G, int rpn,
-             const int32_t *expert_to_rank, const int32_t *src_rank,
-             uint64_t *dest_mask, int32_t *counts, int32_t *offsets,
-             int32_t *row_token, uint8_t *row_jmask, int32_t *row_of, int64_t *summary)
+/* The rank serving pick j of token t: pick_rank[t][j] when given (replicated
+ * experts, see orc_assign_replicas), else p(e_tj). */
+static int serving_rank(const int32_t *ids, const int32_t *expert_to_rank, const int32_t *pick_rank,
+                        int k, int t, int j)
+{
+    return pick_rank ? pick_rank[(size_t)t * k + j] : expert_to_rank[ids[(size_t)t * k + j]];
+}
+
+static int plan_impl(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                     const int32_t *expert_to_rank, const int32_t *pick_rank, const int32_t *src_rank,
+                     uint64_t *dest_mask, int32_t *counts, int32_t *offsets,
+                     int32_t *row_token, uint8_t *row_jmask, int32_t *row_of, int64_t *summary)
 {
     if (T < 0 || k < 1 || k > 8 || E < 1 || k > E || G < 1 || G > 64 || rpn < 1 || G % rpn != 0)
         return ORC_ERR_ARG;
     if (!src_rank && (T % G != 0)) return ORC_ERR_ARG;
-    for (int e = 0; e < E; ++e)
-        if (expert_to_rank[e] < 0 || expert_to_rank[e] >= G) return ORC_ERR_DATA;
+    if (!pick_rank)
+        for (int e = 0; e < E; ++e)
+            if (expert_to_rank[e] < 0 || expert_to_rank[e] >= G) return ORC_ERR_DATA;
     for (int t = 0; t < T; ++t) {
         if (!token_valid(ids + (size_t)t * k, k, E)) return ORC_ERR_DATA;
         if (src_rank && (src_rank[t] < 0 || src_rank[t] >= G)) return ORC_ERR_DATA;
+        if (pick_rank)
+            for (int j = 0; j < k; ++j)
+                if (pick_rank[(size_t)t * k + j] < 0 || pick_rank[(size_t)t * k + j] >= G) return ORC_ERR_DATA;
     }
     int nodes = G / rpn;
     orc_row *rows = (orc_row *)malloc(sizeof(orc_row) * ((size_t)T * k + 1));
@@ -278,11 +290,10 @@ int orc_plan(const int32_t *ids, int T, int k, int E, int G, int rpn,
     size_t R = 0;
     int64_t local = 0, V = 0;
     for (int t = 0; t < T; ++t) {
-        const int32_t *d = ids + (size_t)t * k;
         int s = src_rank ? src_rank[t] : t / (T / G);
         int want[64] = {0}, node_hit[64] = {0};
         for (int j = 0; j < k; ++j) {
-            int r = expert_to_rank[d[j]];
+            int r = serving_rank(ids, expert_to_rank, pick_rank, k, t, j);
             want[r] = 1;
             node_hit[r / rpn] = 1;
             if (r == s) local += 1;
@@ -303,10 +314,9 @@ int orc_plan(const int32_t *ids, int T, int k, int E, int G, int rpn,
     int64_t remote = 0;
     for (size_t i = 0; i < R; ++i) {
         int t = rows[i].t, r = rows[i].dst;
-        const int32_t *d = ids + (size_t)t * k;
         uint8_t jm = 0;
         for (int j = 0; j < k; ++j)
-            if (expert_to_rank[d[j]] == r) {
+            if (serving_rank(ids, expert_to_rank, pick_rank, k, t, j) == r) {
                 jm |= (uint8_t)(1u << j);
                 row_of[(size_t)t * k + j] = (int32_t)i;
             }
@@ -329,6 +339,25 @@ int orc_plan(const int32_t *ids, int T, int k, int E, int G, int rpn,
     summary[4] = (int64_t)T * k;
     free(rows);
     return ORC_OK;
+}
+
+int orc_plan(const int32_t *ids, int T, int k, int E, int G, int rpn,
+             const int32_t *expert_to_rank, const int32_t *src_rank,
+             uint64_t *dest_mask, int32_t *counts, int32_t *offsets,
+             int32_t *row_token, uint8_t *row_jmask, int32_t *row_of, int64_t *summary)
+{
+    return plan_impl(ids, T, k, E, G, rpn, expert_to_rank, NULL, src_rank, dest_mask, counts, offsets,
+                     row_token, row_jmask, row_of, summary);
+}
+
+/* The same plan with the serving rank of every (token, pick) given. */
+int orc_plan_ranks(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                   const int32_t *pick_rank, const int32_t *src_rank,
+                   uint64_t *dest_mask, int32_t *counts, int32_t *offsets,
+                   int32_t *row_token, uint8_t *row_jmask, int32_t *row_of, int64_t *summary)
+{
+    return plan_impl(ids, T, k, E, G, rpn, NULL, pick_rank, src_rank, dest_mask, counts, offsets,
+                     row_token, row_jmask, row_of, summary);
 }
 
 /* Row permute into the rank-major send buffer: send[i] = x[row_token[i]]. */
@@ -409,6 +438,197 @@ int orc_shuffle_targets(const int32_t *ids, int T, int k, int E, int G, const ui
             if (r == 0 || s > best_s) { best = r; best_s = s; }
         }
         target[t] = best;
+    }
+    return ORC_OK;
+}
+
+/* ---- receiver-side pre-reduced combine (a NEXT row of the path) ----------- */
+
+/* Gate dispatch ([CE] footnote 3: the routed probabilities are dispatched with
+ * the hidden states).  Row i carries token t = row_token[i]; for each pick j
+ * of t whose expert lives on the row's rank (bit j of row_jmask[i]) the row
+ * carries (e_tj, w_tj), else (-1, 0). */
+int orc_dispatch_gates(const int32_t *ids, const float *w, int T, int k, const int32_t *row_token,
+                       const uint8_t *row_jmask, int64_t R, int32_t *send_e, float *send_w)
+{
+    for (int64_t i = 0; i < R; ++i) {
+        int t = row_token[i];
+        if (t < 0 || t >= T) return ORC_ERR_DATA;
+        for (int j = 0; j < k; ++j) {
+            int on = (row_jmask[i] >> j) & 1;
+            send_e[i * k + j] = on ? ids[(size_t)t * k + j] : -1;
+            send_w[i * k + j] = on ? w[(size_t)t * k + j] : 0.0f;
+        }
+    }
+    return ORC_OK;
+}
+
+/* The receiving rank applies each of the row's experts and sums their
+ * outputs weighted by the dispatched gates, returning one row per (token,
+ * rank) ([EC]: dispatch, then combine; here the weighting moves to the
+ * receiver).  Stand-in experts: expert e maps a row x to scale[e] * x.
+ *   y[i][c] = sum_j send_w[i][j] * scale[send_e[i][j]] * send[i][c]
+ * over the j with send_e[i][j] >= 0, in fp64. */
+int orc_expert_reduce(const void *send, int is_bf16, int64_t R, int d, const int32_t *send_e,
+                      const float *send_w, int k, const float *scale, int E, double *y)
+{
+    for (int64_t i = 0; i < R; ++i)
+        for (int j = 0; j < k; ++j)
+            if (send_e[i * k + j] >= E) return ORC_ERR_DATA;
+    for (int64_t i = 0; i < R; ++i)
+        for (int c = 0; c < d; ++c) {
+            double x = load_elem(send, is_bf16, (size_t)i * d + c), acc = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int e = send_e[i * k + j];
+                if (e >= 0) acc += (double)send_w[i * k + j] * (double)scale[e] * x;
+            }
+            y[(size_t)i * d + c] = acc;
+        }
+    return ORC_OK;
+}
+
+/* The source sums the pre-reduced rows of each token once each:
+ * out[t][c] = sum over the distinct rows r in {row_of[t][j]} of y[r][c] (fp64,
+ * y given as float32 or bf16 bits). */
+int orc_combine_rows(const void *y, int is_bf16, int64_t R_max, int d, const int32_t *row_of, int T, int k,
+                     double *out)
+{
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j)
+            if (row_of[(size_t)t * k + j] < 0 || row_of[(size_t)t * k + j] >= R_max) return ORC_ERR_DATA;
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int r = row_of[(size_t)t * k + j], seen = 0;
+                for (int q = 0; q < j; ++q) seen |= row_of[(size_t)t * k + q] == r;
+                if (!seen) acc += load_elem(y, is_bf16, (size_t)r * d + c);
+            }
+            out[(size_t)t * d + c] = acc;
+        }
+    return ORC_OK;
+}
+
+/* ---- expert replicas and communication-aware task assignment ([CB]) ------- */
+
+/* Replica layout.  [CB] "Problem Formulation": P_r is the set of experts with
+ * a replica on rank r, every expert has at least one, |P_r| <= (1+rho)E/G;
+ * "Two-Stage Expert Layout Planner" maximises co-activation within nodes.  The
+ * page gives no algorithm; this is the greedy reading: start from a placement
+ * with one replica per expert (expert_to_rank), give every rank room for
+ * `extra` more experts, and repeatedly add the replica (e, node q) of largest
+ * score(e, q) = sum over the experts e' placed on q of C[e][e'] (e not yet on
+ * q; ties: lower e, then lower q) on the rank of q with the most free room
+ * (ties: lowest rank), until no rank has room or no candidate scores above 0.
+ * Output: replica_rank[e][0..n_rep[e]) (the original rank first, then in the
+ * order added), unused slots -1; max_rep = 1 + G/rpn slots per expert. */
+int orc_place_replicas(const uint32_t *coact, int E, int G, int rpn, const int32_t *expert_to_rank, int extra,
+                       int32_t *replica_rank, int32_t *n_rep)
+{
+    if (E < 1 || G < 1 || rpn < 1 || G % rpn != 0 || extra < 0) return ORC_ERR_ARG;
+    const int nodes = G / rpn, max_rep = 1 + nodes;
+    int *room = (int *)malloc(sizeof(int) * G);
+    int *on_node = (int *)calloc((size_t)E * nodes, sizeof(int));
+    uint64_t *score = (uint64_t *)calloc((size_t)E * nodes, sizeof(uint64_t));
+    int *used = (int *)calloc((size_t)E * nodes, sizeof(int));
+    for (int r = 0; r < G; ++r) room[r] = extra;
+    for (int e = 0; e < E; ++e) {
+        if (expert_to_rank[e] < 0 || expert_to_rank[e] >= G) { free(room); free(on_node); free(score); free(used); return ORC_ERR_DATA; }
+        for (int q = 0; q < max_rep; ++q) replica_rank[(size_t)e * max_rep + q] = -1;
+        replica_rank[(size_t)e * max_rep] = expert_to_rank[e];
+        n_rep[e] = 1;
+        on_node[(size_t)e * nodes + expert_to_rank[e] / rpn] = 1;
+    }
+    for (int e = 0; e < E; ++e)
+        for (int f = 0; f < E; ++f)
+            if (f != e) score[(size_t)e * nodes + expert_to_rank[f] / rpn] += coact[(size_t)e * E + f];
+    for (;;) {
+        int be = -1, bq = -1;
+        uint64_t bs = 0;
+        for (int e = 0; e < E; ++e)
+            for (int q = 0; q < nodes; ++q) {
+                if (on_node[(size_t)e * nodes + q] || used[(size_t)e * nodes + q]) continue;
+                uint64_t sc = score[(size_t)e * nodes + q];
+                if (sc == 0) continue;
+                int has_room = 0;
+                for (int r = q * rpn; r < (q + 1) * rpn; ++r) has_room |= room[r] > 0;
+                if (!has_room) continue;
+                if (be < 0 || sc > bs) { be = e; bq = q; bs = sc; }
+            }
+        if (be < 0) break;
+        int br = -1;
+        for (int r = bq * rpn; r < (bq + 1) * rpn; ++r)
+            if (room[r] > 0 && (br < 0 || room[r] > room[br])) br = r;
+        room[br] -= 1;
+        used[(size_t)be * nodes + bq] = 1;
+        on_node[(size_t)be * nodes + bq] = 1;
+        replica_rank[(size_t)be * max_rep + n_rep[be]] = br;
+        n_rep[be] += 1;
+    }
+    free(room); free(on_node); free(score); free(used);
+    return ORC_OK;
+}
+
+/* Communication-aware task assignment ([CB]: tokens are routed "to the fewest
+ * remote nodes possible"; V counts, per token, the remote nodes its tasks
+ * reach).  For token t with source rank s (node ns = s / rpn): among all
+ * choices of one replica rank per pick, the fewest distinct nodes other than
+ * ns -- found as the smallest node set S (ties: smallest as a bit pattern)
+ * such that every pick's expert has a replica on ns or in S.  Then, pick by
+ * pick in j order, among the ranks hosting the expert on ns (or, if none, on
+ * the nodes of S): rank s if it is one of them; else the lowest of them that
+ * an earlier pick of the token already uses (no new row); else the lowest of
+ * them.  Requires G/rpn <= 8.
+ * pick_rank [T][k] out; n_remote [T] out (|S|, may be NULL). */
+int orc_assign_replicas(const int32_t *ids, int T, int k, int E, int G, int rpn, const int32_t *replica_rank,
+                        const int32_t *n_rep, const int32_t *src_rank, int32_t *pick_rank, int32_t *n_remote)
+{
+    if (T < 0 || k < 1 || k > 8 || G < 1 || rpn < 1 || G % rpn != 0 || G / rpn > 8) return ORC_ERR_ARG;
+    if (!src_rank && T % G != 0) return ORC_ERR_ARG;
+    const int nodes = G / rpn, max_rep = 1 + nodes;
+    for (int t = 0; t < T; ++t) {
+        const int32_t *d = ids + (size_t)t * k;
+        if (!token_valid(d, k, E)) return ORC_ERR_DATA;
+        const int s = src_rank ? src_rank[t] : t / (T / G);
+        if (s < 0 || s >= G) return ORC_ERR_DATA;
+        const int ns = s / rpn;
+        int best_size = nodes + 1, best_set = 0;
+        for (int set = 0; set < (1 << nodes); ++set) {
+            if ((set >> ns) & 1) continue;
+            int ok = 1;
+            for (int j = 0; j < k && ok; ++j) {
+                int covered = 0;
+                for (int q = 0; q < n_rep[d[j]]; ++q) {
+                    int node = replica_rank[(size_t)d[j] * max_rep + q] / rpn;
+                    if (node == ns || ((set >> node) & 1)) covered = 1;
+                }
+                ok = covered;
+            }
+            if (!ok) continue;
+            int size = 0;
+            for (int q = 0; q < nodes; ++q) size += (set >> q) & 1;
+            if (size < best_size) { best_size = size; best_set = set; }
+        }
+        if (best_size > nodes) return ORC_ERR_DATA;   /* an expert without replicas */
+        for (int j = 0; j < k; ++j) {
+            int any_ns = 0;
+            for (int q = 0; q < n_rep[d[j]]; ++q)
+                if (replica_rank[(size_t)d[j] * max_rep + q] / rpn == ns) any_ns = 1;
+            int pick = -1, used_pick = -1, low = -1;
+            for (int q = 0; q < n_rep[d[j]]; ++q) {
+                int r = replica_rank[(size_t)d[j] * max_rep + q];
+                int allowed = any_ns ? (r / rpn == ns) : ((best_set >> (r / rpn)) & 1);
+                if (!allowed) continue;
+                if (r == s) pick = r;
+                int used = 0;
+                for (int q2 = 0; q2 < j; ++q2) used |= pick_rank[(size_t)t * k + q2] == r;
+                if (used && (used_pick < 0 || r < used_pick)) used_pick = r;
+                if (low < 0 || r < low) low = r;
+            }
+            if (pick < 0) pick = used_pick >= 0 ? used_pick : low;
+            pick_rank[(size_t)t * k + j] = pick;
+        }
+        if (n_remote) n_remote[t] = best_size;
     }
     return ORC_OK;
 }

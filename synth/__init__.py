@@ -10,6 +10,7 @@ from .workloads import (  # noqa: F401
     make_routing,
     make_gates,
     make_hidden,
+    make_expert_scales,
     bf16_bits_to_f32,
     f32_to_bf16_bits,
 )

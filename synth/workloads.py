@@ -35,6 +35,9 @@ same bits):
   are exhausted, uniform over all not yet chosen experts (rejection sampling,
   which is exactly uniform over the remaining set);
 * gate weights: softmax over the k chosen experts of N(0,1) logits, fp32;
+* stand-in experts (for the receiver-side pre-reduced combine): expert e of
+  layer l scales its input row by a factor drawn uniformly from [0.5, 1.5]
+  (fp32, stream ``[seed, 3]``);
 * hidden states: N(0,1) fp32, rounded to bf16 (round to nearest even) where
   the workload is bf16.
 """
@@ -48,6 +51,7 @@ import numpy as np
 STREAM_ROUTING = 0
 STREAM_GATES = 1
 STREAM_HIDDEN = 2
+STREAM_EXPERTS = 3
 
 
 @dataclass(frozen=True)
@@ -269,3 +273,10 @@ def make_hidden(w: Workload, seed: Optional[int] = None, T: Optional[int] = None
 
     _parallel(fill, max(1, -(-T // rows_per_block)))
     return out
+
+
+def make_expert_scales(w: Workload, seed: Optional[int] = None) -> np.ndarray:
+    """Per-expert scale factors of the stand-in experts, fp32 [L][E] in [0.5, 1.5)."""
+    seed = w.seed if seed is None else seed
+    rng = _rng(seed, STREAM_EXPERTS)
+    return (0.5 + rng.random((w.L, w.E))).astype(np.float32)

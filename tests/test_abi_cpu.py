@@ -118,3 +118,16 @@ def test_argument_errors_return_before_device_work(cap):
     assert L.moe_permute(fake, cap.MOE_BF16, 4, 7, 2, fake, 8, fake, fake, None) == cap.MOE_ERR_UNSUPPORTED
     assert L.moe_combine(fake, 7, 8, 8, fake, fake, 4, 2, fake, 0, fake, None) == cap.MOE_ERR_ARG
     assert L.moe_shuffle_targets(fake, 4, 2, 1024, 64, fake, fake, fake, None) == cap.MOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("E,G,rpn,extra", [(16, 8, 2, 1), (64, 8, 8, 2), (64, 32, 8, 1), (256, 64, 8, 1), (24, 6, 1, 3)])
+def test_place_replicas_matches_oracle(cap, orc, E, G, rpn, extra):
+    rng = np.random.default_rng(E + G + extra)
+    C = rng.integers(0, 200, (E, E)) * (rng.random((E, E)) < 0.3)
+    C = np.triu(C, 1)
+    C = (C + C.T + np.diag(rng.integers(100, 300, E))).astype(np.uint32)
+    C[3, 5] = C[5, 3] = C[3, 7] = C[7, 3] = 777                  # equal scores: ties by (e, node)
+    e2r = orc.place_correlated(C, G, rpn)
+    a = cap.place_replicas(C, G, rpn, e2r, extra)
+    b = orc.place_replicas(C, G, rpn, e2r, extra)
+    assert (a[0] == b[0]).all() and (a[1] == b[1]).all()

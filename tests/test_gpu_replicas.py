@@ -1,0 +1,93 @@
+"""Parity of the replica assignment and of the plan over per-pick serving
+ranks with the oracle ("Cobalt ...", "Problem Formulation": tasks run on a
+replica of their expert; the assignment reaches the fewest remote nodes).
+Integers throughout: bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from synth import WORKLOADS, make_routing
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cap():
+    from co_activation_placement_b200 import build
+    build.build()
+    import co_activation_placement_b200 as cap
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    cap.lib()
+    return cap
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def check_plan(p, o, T):
+    R = o["R"]
+    assert int(host(p.err)[0]) == 0
+    assert host(p.summary).tolist() == o["summary"].tolist()
+    assert (host(p.counts) == o["counts"]).all() and (host(p.offsets) == o["offsets"]).all()
+    assert (host(p.row_token)[:R] == o["row_token"]).all()
+    assert (host(p.row_jmask)[:R] == o["row_jmask"]).all()
+    assert (host(p.row_of)[:T] == o["row_of"]).all()
+
+
+@pytest.mark.parametrize("name,extra,with_src", [("one_node", 2, False), ("ep32", 1, True), ("ep32", 2, False),
+                                                 ("large_ep64", 1, True), ("large_ep64", 2, False)])
+def test_replica_assignment_and_plan(cap, name, extra, with_src):
+    w = WORKLOADS[name]
+    ids = make_routing(w)[0]
+    cal = make_routing(w, seed=1)[0]
+    C = orc.coact(cal[None], w.E, want=("coact",))["coact"][0]
+    e2r = orc.place_correlated(C, w.G, w.rpn)
+    rr, nr = cap.place_replicas(C, w.G, w.rpn, e2r, extra)
+    rr_o, nr_o = orc.place_replicas(C, w.G, w.rpn, e2r, extra)
+    assert (rr == rr_o).all() and (nr == nr_o).all()
+    rng = np.random.default_rng(7)
+    src = rng.integers(0, w.G, w.T).astype(np.int32) if with_src else None
+    pr, nrem = cap.assign_replicas(dev(ids), w.E, w.G, w.rpn, dev(rr), dev(nr),
+                                   src_rank=None if src is None else dev(src))
+    pr_o, nrem_o = orc.assign_replicas(ids, w.E, w.G, w.rpn, rr_o, nr_o, src_rank=src)
+    assert (host(pr)[: w.T] == pr_o).all() and (host(nrem)[: w.T] == nrem_o).all()
+    p = cap.plan_dispatch_ranks(dev(ids), w.E, w.G, w.rpn, pr, src_rank=None if src is None else dev(src))
+    o = orc.plan(ids, w.E, w.G, w.rpn, None, src_rank=src, pick_rank=pr_o)
+    check_plan(p, o, w.T)
+    assert o["V"] == int(nrem_o.sum())
+    # replicas never add remote nodes compared with the single placement
+    base = orc.plan(ids, w.E, w.G, w.rpn, e2r, src_rank=src)
+    assert o["V"] <= base["V"]
+
+
+def test_replica_assignment_small_and_errors(cap):
+    rng = np.random.default_rng(3)
+    T, E, k, G, rpn = 999, 16, 3, 8, 2
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    C = orc.coact(ids[None], E, want=("coact",))["coact"][0]
+    e2r = orc.place_correlated(C, G, rpn)
+    rr, nr = orc.place_replicas(C, G, rpn, e2r, 2)
+    src = rng.integers(0, G, T).astype(np.int32)
+    pr, nrem = cap.assign_replicas(dev(ids), E, G, rpn, dev(rr), dev(nr), src_rank=dev(src))
+    pr_o, nrem_o = orc.assign_replicas(ids, E, G, rpn, rr, nr, src_rank=src)
+    assert (host(pr)[:T] == pr_o).all() and (host(nrem)[:T] == nrem_o).all()
+    # an out-of-range id is reported and its token gets -1
+    bad = ids.copy()
+    bad[5, 1] = E + 3
+    err = cap.new_err("cuda")
+    pr2, nrem2 = cap.assign_replicas(dev(bad), E, G, rpn, dev(rr), dev(nr), src_rank=dev(src), err=err)
+    assert int(host(err)[0]) == cap.DERR_ID_RANGE and (host(pr2)[5] == -1).all()
+    # pick ranks out of range are reported by the plan
+    prb = host(pr).copy()
+    prb[7, 0] = G
+    p = cap.plan_dispatch_ranks(dev(ids), E, G, rpn, dev(prb[:T]), src_rank=dev(src))
+    assert int(host(p.err)[0]) == cap.DERR_RANK_RANGE
+    with pytest.raises(cap.MoeError):
+        cap.assign_replicas(dev(ids), E, 16, 1, dev(rr), dev(nr), src_rank=dev(src))   # 16 nodes > 8

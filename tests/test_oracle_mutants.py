@@ -1,0 +1,74 @@
+"""Mutation test of the oracle's pins.
+
+Each mutant plants one plausible mistake in a copy of oracle/oracle.c (a
+dropped term, a swapped index, a wrong tie-break, a transposed operand), built
+in a temporary directory; the pin suites are then run against it and must
+fail.  A mutant that survives means some part of the oracle is not pinned."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+from conftest import ROOT
+
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+PINS = ["tests/test_oracle_pins.py", "tests/test_oracle_brute.py", "tests/test_oracle_prereduce.py",
+        "tests/test_oracle_replicas.py"]
+
+MUTANTS = {
+    "counts_drop_diagonal": ("                for (int a = 0; a < k; ++a)\n                    for (int b = 0; b < k; ++b)\n"
+                             "                        Cl[(size_t)d[a] * E + d[b]] += 1;",
+                             "                for (int a = 0; a < k; ++a)\n                    for (int b = 0; b < k; ++b)\n"
+                             "                        if (a != b) Cl[(size_t)d[a] * E + d[b]] += 1;"),
+    "ochiai_sum_not_product": ("double den = (double)Cl[(size_t)i * E + i] * (double)Cl[(size_t)j * E + j];",
+                               "double den = (double)Cl[(size_t)i * E + i] + (double)Cl[(size_t)j * E + j];"),
+    "transitions_transposed": ("Ml[(size_t)a[x] * E + b[y]] += 1;", "Ml[(size_t)b[y] * E + a[x]] += 1;"),
+    "uniform_off_by_one": ("for (int e = 0; e < E; ++e) expert_to_rank[e] = e / per;",
+                           "for (int e = 0; e < E; ++e) expert_to_rank[e] = ((e + 1) / per) % G;"),
+    "rows_source_major": ("    if (a->dst != b->dst) return a->dst < b->dst ? -1 : 1;\n"
+                          "    if (a->src != b->src) return a->src < b->src ? -1 : 1;",
+                          "    if (a->src != b->src) return a->src < b->src ? -1 : 1;\n"
+                          "    if (a->dst != b->dst) return a->dst < b->dst ? -1 : 1;"),
+    "V_counts_source_node": ("if (node_hit[q] && q != s / rpn) V += 1;", "if (node_hit[q]) V += 1;"),
+    "local_counts_remote": ("if (r == s) local += 1;", "if (r != s) local += 1;"),
+    "jmask_reversed": ("jm |= (uint8_t)(1u << j);", "jm |= (uint8_t)(1u << (k - 1 - j));"),
+    "combine_drops_last_pick": ("            for (int j = 0; j < k; ++j) {\n                size_t row",
+                                "            for (int j = 0; j < k - 1; ++j) {\n                size_t row"),
+    "shuffle_ties_highest_rank": ("if (r == 0 || s > best_s) { best = r; best_s = s; }",
+                                  "if (r == 0 || s >= best_s) { best = r; best_s = s; }"),
+    "correlated_seed_lowest_load": ("C[(size_t)pool[x] * E + pool[x]] > C[(size_t)pool[best] * E + pool[best]]",
+                                    "C[(size_t)pool[x] * E + pool[x]] < C[(size_t)pool[best] * E + pool[best]]"),
+    "rank_score_transposed": ("if (next_expert_to_rank[f] == r) s += trans[(size_t)e * E + f];",
+                              "if (next_expert_to_rank[f] == r) s += trans[(size_t)f * E + e];"),
+    "capacity_ties_highest_device": ("if (device_load[g] < device_load[best]) best = g;",
+                                     "if (device_load[g] <= device_load[best]) best = g;"),
+    "reduce_ignores_scale": ("acc += (double)send_w[i * k + j] * (double)scale[e] * x;",
+                             "acc += (double)send_w[i * k + j] * x;"),
+    "row_sum_counts_repeats": ("if (!seen) acc += load_elem(y, is_bf16, (size_t)r * d + c);",
+                               "acc += load_elem(y, is_bf16, (size_t)r * d + c);"),
+    "replica_pick_ignores_source_node": ("int allowed = any_ns ? (r / rpn == ns) : ((best_set >> (r / rpn)) & 1);",
+                                         "int allowed = ((best_set >> (r / rpn)) & 1) || r / rpn == ns;"),
+    "replica_pick_ignores_used_ranks": ("if (pick < 0) pick = used_pick >= 0 ? used_pick : low;",
+                                        "if (pick < 0) pick = low;"),
+    "replica_set_ties_largest": ("if (size < best_size) { best_size = size; best_set = set; }",
+                                 "if (size <= best_size) { best_size = size; best_set = set; }"),
+    "replica_room_ties_highest_rank": ("if (room[r] > 0 && (br < 0 || room[r] > room[br])) br = r;",
+                                       "if (room[r] > 0 && (br < 0 || room[r] >= room[br])) br = r;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation site not found exactly once"
+    mutant = tmp_path / "oracle_mutant.c"
+    mutant.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mutant.so"
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-std=c11", "-fPIC", "-shared", str(mutant),
+                           "-o", str(lib), "-lm"])
+    env = dict(os.environ, ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider"] + PINS,
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, "mutant %s survived the pins:\n%s" % (name, r.stdout[-2000:])

@@ -383,3 +383,14 @@ def test_rank_score_definition(orc):
     onehot = np.zeros((E, G), np.int64)
     onehot[np.arange(E), e2r] = 1
     assert (rs == M.astype(np.int64) @ onehot).all()
+
+
+def test_capacity_placement_hand_example(orc):
+    # loads 5, 4, 3, 2 on 2 devices, largest first onto the least-loaded device
+    # (equal loads: the lower device): 5 -> d0 ; 4 -> d1 ; 3 -> d1 (4 < 5) ;
+    # 2 -> d0 (5 < 7)  =>  device loads 7, 7
+    e2r, dev = orc.place_capacity(np.array([2.0, 5.0, 3.0, 4.0]), 2)
+    assert e2r.tolist() == [0, 0, 1, 1] and dev.tolist() == [7.0, 7.0]
+    # all loads equal: experts in id order, each onto the lowest least-loaded device
+    e2r, _ = orc.place_capacity(np.ones(6), 3)
+    assert e2r.tolist() == [0, 1, 2, 0, 1, 2]
