@@ -114,9 +114,11 @@ class HotPath:
         self.events = []
 
     def step(self):
+        nv = torch.cuda.nvtx.range   # one NVTX range per library call (Nsight timelines)
         self._mark("start")
-        cap.coact_stats(self.ids, self.E, coact=self.stats["coact"], ochiai=self.stats["ochiai"],
-                        trans=self.stats["trans"], err=self.err, ws=self.stats_ws)
+        with nv("moe_coact_stats"):
+            cap.coact_stats(self.ids, self.E, coact=self.stats["coact"], ochiai=self.stats["ochiai"],
+                            trans=self.stats["trans"], err=self.err, ws=self.stats_ws)
         self._mark("stats")
         if not self.rows:
             return
@@ -125,33 +127,42 @@ class HotPath:
             if self.replicas:
                 # each task to a replica of its expert: fewest remote nodes per token
                 rr, nr = self.replicas[l]
-                cap.assign_replicas(self.ids[l], self.E, self.G, self.rpn, rr, nr, src_rank=src,
-                                    pick_rank=self.pick_rank, n_remote=self.n_remote, err=self.err)
-                p = cap.plan_dispatch_ranks(self.ids[l], self.E, self.G, self.rpn, self.pick_rank, src_rank=src,
-                                            plan=self.plans[l], ws=self.plan_ws)
+                with nv("moe_assign_replicas"):
+                    cap.assign_replicas(self.ids[l], self.E, self.G, self.rpn, rr, nr, src_rank=src,
+                                        pick_rank=self.pick_rank, n_remote=self.n_remote, err=self.err)
+                with nv("moe_plan_dispatch_ranks"):
+                    p = cap.plan_dispatch_ranks(self.ids[l], self.E, self.G, self.rpn, self.pick_rank,
+                                                src_rank=src, plan=self.plans[l], ws=self.plan_ws)
             else:
-                p = cap.plan_dispatch(self.ids[l], self.E, self.G, self.rpn, self.e2r[l], src_rank=src,
-                                      plan=self.plans[l], ws=self.plan_ws)
+                with nv("moe_plan_dispatch"):
+                    p = cap.plan_dispatch(self.ids[l], self.E, self.G, self.rpn, self.e2r[l], src_rank=src,
+                                          plan=self.plans[l], ws=self.plan_ws)
             self._mark("plan")
-            cap.permute(self.x, p.row_of, p.R_max, send=self.send, err=self.err)
+            with nv("moe_permute"):
+                cap.permute(self.x, p.row_of, p.R_max, send=self.send, err=self.err)
             self._mark("permute")
             if self.prereduce:
                 # gates travel with the rows; the receiving rank applies its
                 # experts and returns one row per (token, rank); the source sums
-                cap.dispatch_gates(self.ids[l], self.gates[l], p, send_e=self.send_e, send_w=self.send_w,
-                                   err=self.err)
+                with nv("moe_dispatch_gates"):
+                    cap.dispatch_gates(self.ids[l], self.gates[l], p, send_e=self.send_e, send_w=self.send_w,
+                                       err=self.err)
                 self._mark("gates")
-                cap.expert_reduce(self.send, p.summary, self.send_e, self.send_w, self.scales[l], y=self.y,
-                                  err=self.err)
+                with nv("moe_expert_reduce"):
+                    cap.expert_reduce(self.send, p.summary, self.send_e, self.send_w, self.scales[l], y=self.y,
+                                      err=self.err)
                 self._mark("reduce")
-                cap.combine_rows(self.y, p.row_of, out=self.outs[l], err=self.err)
+                with nv("moe_combine_rows"):
+                    cap.combine_rows(self.y, p.row_of, out=self.outs[l], err=self.err)
                 self._mark("combine")
             else:
-                cap.combine(self.send, p.row_of, self.gates[l], out=self.outs[l], err=self.err)
+                with nv("moe_combine"):
+                    cap.combine(self.send, p.row_of, self.gates[l], out=self.outs[l], err=self.err)
                 self._mark("combine")
             if self.shuffle and l + 1 < self.L:
-                cap.shuffle_targets(self.ids[l], self.E, self.G, self.rank_scores[l],
-                                    target=self.targets[l], err=self.err)
+                with nv("moe_shuffle_targets"):
+                    cap.shuffle_targets(self.ids[l], self.E, self.G, self.rank_scores[l],
+                                        target=self.targets[l], err=self.err)
                 self._mark("shuffle")
 
     def capture(self, n_steps: int) -> torch.cuda.CUDAGraph:
@@ -262,3 +273,35 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
     return HotPath(E=E, G=G, rpn=rpn, ids=ids_d, gates=gates_d, x=x_d, e2r=e2r, rank_scores=rs,
                    out_dtype=out_dtype, rows=rows, timers=timers, prereduce=scales is not None, scales=scales_d,
                    replicas=reps)
+
+
+def save_layout(path: str, expert_to_rank, rank_scores=(), replicas=(), stats=None):
+    """Write a placement (and what was derived with it) to one .npz file: the
+    expert-to-rank map per layer, rank-score tables per layer pair, replica
+    tables per layer and, optionally, the statistics they came from.  Accepts
+    numpy arrays or tensors (device tensors are copied to the host)."""
+    def h(a):
+        return a.detach().cpu().numpy() if isinstance(a, torch.Tensor) else np.asarray(a)
+    arrays = {"expert_to_rank": np.stack([h(a) for a in expert_to_rank]).astype(np.int32)}
+    if len(rank_scores):
+        arrays["rank_score"] = np.stack([h(a) for a in rank_scores]).astype(np.uint32)
+    if len(replicas):
+        arrays["replica_rank"] = np.stack([h(r) for r, _ in replicas]).astype(np.int32)
+        arrays["n_rep"] = np.stack([h(n) for _, n in replicas]).astype(np.int32)
+    for k_, v in (stats or {}).items():
+        if v is not None:
+            arrays["stats_" + k_] = h(v)
+    np.savez(path, **arrays)
+
+
+def load_layout(path: str, device=None) -> dict:
+    """Read save_layout's file: lists per layer (tensors on `device` when
+    given, else numpy arrays) under the same names, statistics under 'stats'."""
+    with np.load(path) as z:
+        d = {k_: z[k_] for k_ in z.files}
+    conv = (lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)) if device is not None else (lambda a: a)
+    out = {"expert_to_rank": [conv(a) for a in d["expert_to_rank"]],
+           "rank_score": [conv(a) for a in d.get("rank_score", [])],
+           "replicas": [(conv(r), conv(n)) for r, n in zip(d.get("replica_rank", []), d.get("n_rep", []))],
+           "stats": {k_[6:]: d[k_] for k_ in d if k_.startswith("stats_")}}
+    return out
