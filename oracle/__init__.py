@@ -52,6 +52,7 @@ def lib():
             "orc_combine": [P, i, i64, i, P, P, i, i, P],
             "orc_rank_score": [P, P, i, i, P],
             "orc_shuffle_targets": [P, i, i, i, i, P, P],
+            "orc_shuffle_balanced": [P, i, i, i, i, P, i, P],
             "orc_dispatch_gates": [P, P, i, i, P, P, i64, P, P],
             "orc_expert_reduce": [P, i, i64, i, P, P, i, P, i, P],
             "orc_combine_rows": [P, i, i64, i, P, i, i, P],
@@ -185,6 +186,17 @@ def shuffle_targets(ids_l: np.ndarray, E: int, G: int, rank_score_tab: np.ndarra
     rs = np.ascontiguousarray(rank_score_tab, dtype=np.uint32)
     tgt = np.empty(T, np.int32)
     _check("orc_shuffle_targets", lib().orc_shuffle_targets(_p(ids_l), T, k, E, G, _p(rs), _p(tgt)))
+    return tgt
+
+
+def shuffle_balanced(ids_l: np.ndarray, E: int, G: int, rank_score_tab: np.ndarray, capacity: int) -> np.ndarray:
+    """Shuffle targets with at most `capacity` tokens per rank: pairs (t, r)
+    accepted greedily in the order score desc, t asc, r asc."""
+    ids_l = np.ascontiguousarray(ids_l, dtype=np.int32)
+    T, k = ids_l.shape
+    rs = np.ascontiguousarray(rank_score_tab, dtype=np.uint32)
+    tgt = np.empty(T, np.int32)
+    _check("orc_shuffle_balanced", lib().orc_shuffle_balanced(_p(ids_l), T, k, E, G, _p(rs), int(capacity), _p(tgt)))
     return tgt
 
 

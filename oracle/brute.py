@@ -120,6 +120,53 @@ def shuffle_targets(ids_l, G, rank_score):
     return tg
 
 
+def shuffle_balanced_da(ids_l, G, rank_score, capacity):
+    """Capacity-balanced shuffle by token-proposing deferred acceptance
+    (Gale-Shapley): each free token proposes to its next rank in the order
+    score desc, rank asc; a rank keeps its `capacity` best proposers in the
+    order score desc, token asc and rejects the rest.  Preferences that come
+    from one common ordering of the (t, r) pairs have exactly one stable
+    assignment, so this must agree with the greedy over that ordering."""
+    T = len(ids_l)
+    S = [[sum(int(rank_score[int(e)][r]) for e in d) for r in range(G)] for d in ids_l]
+    pref = [sorted(range(G), key=lambda r: (-S[t][r], r)) for t in range(T)]
+    nxt = [0] * T
+    held = [[] for _ in range(G)]
+    free = list(range(T))
+    while free:
+        t = free.pop()
+        r = pref[t][nxt[t]]
+        nxt[t] += 1
+        held[r].append(t)
+        if len(held[r]) > capacity:
+            held[r].sort(key=lambda u: (-S[u][r], u))
+            free.append(held[r].pop())
+    tgt = [None] * T
+    for r in range(G):
+        for t in held[r]:
+            tgt[t] = r
+    return tgt
+
+
+def blocking_pairs(ids_l, G, rank_score, capacity, tgt):
+    """(t, r) pairs that would both rather be matched to each other: t ranks r
+    above its own rank (score desc, rank asc) and r has room or holds a token
+    it ranks below t (score desc, token asc)."""
+    T = len(ids_l)
+    S = [[sum(int(rank_score[int(e)][r]) for e in d) for r in range(G)] for d in ids_l]
+    held = [[t for t in range(T) if tgt[t] == r] for r in range(G)]
+    out = []
+    for t in range(T):
+        mine = (-S[t][tgt[t]], tgt[t])
+        for r in range(G):
+            if (-S[t][r], r) >= mine:
+                continue
+            worst = max(held[r], key=lambda u: (-S[u][r], u)) if held[r] else None
+            if len(held[r]) < capacity or (-S[worst][r], worst) > (-S[t][r], t):
+                out.append((t, r))
+    return out
+
+
 def place_correlated(C, G, rpn):
     """Restatement of the greedy grouping with Python lists and Fraction-free
     fp64 (same summation order as the specification: insertion order)."""

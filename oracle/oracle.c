@@ -442,6 +442,59 @@ int orc_shuffle_targets(const int32_t *ids, int T, int k, int E, int G, const ui
     return ORC_OK;
 }
 
+/* Capacity-balanced shuffle target.  [EC] moves each token to the GPU
+ * predicted to hold its next-layer experts during the reduce-scatter that
+ * follows attention; a reduce-scatter hands every rank an equal shard, so here
+ * every rank receives at most `capacity` tokens (exactly T/G when T =
+ * G*capacity).  Reading taken: score S_t(r) = sum_j rank_score[e_tj][r] as in
+ * the unconstrained target; all (t, r) pairs are taken in the order S desc,
+ * then t asc, then r asc, and a pair is accepted when t has no rank yet and r
+ * holds fewer than `capacity` tokens.  With capacity >= T this is the
+ * unconstrained argmax. */
+typedef struct { uint64_t s; int32_t t, r; } orc_pair;
+
+static int cmp_pair(const void *pa, const void *pb)
+{
+    const orc_pair *a = (const orc_pair *)pa, *b = (const orc_pair *)pb;
+    if (a->s != b->s) return a->s > b->s ? -1 : 1;
+    if (a->t != b->t) return a->t < b->t ? -1 : 1;
+    if (a->r != b->r) return a->r < b->r ? -1 : 1;
+    return 0;
+}
+
+int orc_shuffle_balanced(const int32_t *ids, int T, int k, int E, int G, const uint32_t *rank_score,
+                         int capacity, int32_t *target)
+{
+    if (T < 0 || k < 1 || G < 1 || capacity < 0 || (int64_t)G * capacity < T) return ORC_ERR_ARG;
+    for (int t = 0; t < T; ++t)
+        if (!token_valid(ids + (size_t)t * k, k, E)) return ORC_ERR_DATA;
+    size_t n = (size_t)T * G;
+    orc_pair *pairs = (orc_pair *)malloc((n ? n : 1) * sizeof(orc_pair));
+    int32_t *held = (int32_t *)calloc((size_t)G, sizeof(int32_t));
+    if (!pairs || !held) { free(pairs); free(held); return ORC_ERR_ARG; }
+    for (int t = 0; t < T; ++t) {
+        const int32_t *d = ids + (size_t)t * k;
+        for (int r = 0; r < G; ++r) {
+            uint64_t s = 0;
+            for (int j = 0; j < k; ++j) s += rank_score[(size_t)d[j] * G + r];
+            orc_pair *p = &pairs[(size_t)t * G + r];
+            p->s = s; p->t = t; p->r = r;
+        }
+        target[t] = -1;
+    }
+    qsort(pairs, n, sizeof(orc_pair), cmp_pair);
+    for (size_t i = 0; i < n; ++i) {
+        const orc_pair *p = &pairs[i];
+        if (target[p->t] < 0 && held[p->r] < capacity) {
+            target[p->t] = p->r;
+            held[p->r] += 1;
+        }
+    }
+    free(pairs);
+    free(held);
+    return ORC_OK;
+}
+
 /* ---- receiver-side pre-reduced combine (a NEXT row of the path) ----------- */
 
 /* Gate dispatch ([CE] footnote 3: the routed probabilities are dispatched with

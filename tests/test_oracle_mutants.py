@@ -14,7 +14,7 @@ from conftest import ROOT
 
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_pins.py", "tests/test_oracle_brute.py", "tests/test_oracle_prereduce.py",
-        "tests/test_oracle_replicas.py"]
+        "tests/test_oracle_replicas.py", "tests/test_oracle_shuffle_balanced.py"]
 
 MUTANTS = {
     "counts_drop_diagonal": ("                for (int a = 0; a < k; ++a)\n                    for (int b = 0; b < k; ++b)\n"
@@ -55,6 +55,14 @@ MUTANTS = {
                                  "if (size <= best_size) { best_size = size; best_set = set; }"),
     "replica_room_ties_highest_rank": ("if (room[r] > 0 && (br < 0 || room[r] > room[br])) br = r;",
                                        "if (room[r] > 0 && (br < 0 || room[r] >= room[br])) br = r;"),
+    "balanced_ties_highest_token": ("if (a->t != b->t) return a->t < b->t ? -1 : 1;",
+                                    "if (a->t != b->t) return a->t > b->t ? -1 : 1;"),
+    "balanced_ties_highest_rank": ("if (a->r != b->r) return a->r < b->r ? -1 : 1;",
+                                   "if (a->r != b->r) return a->r > b->r ? -1 : 1;"),
+    "balanced_capacity_off_by_one": ("if (target[p->t] < 0 && held[p->r] < capacity) {",
+                                     "if (target[p->t] < 0 && held[p->r] <= capacity) {"),
+    "balanced_score_ascending": ("if (a->s != b->s) return a->s > b->s ? -1 : 1;",
+                                 "if (a->s != b->s) return a->s < b->s ? -1 : 1;"),
 }
 
 
