@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--workload", default="large_ep64")
     ap.add_argument("--placement", default="correlated", choices=["correlated", "uniform"])
     ap.add_argument("--no-shuffle", action="store_true")
+    ap.add_argument("--balanced-shuffle", action="store_true",
+                    help="cap every rank's shard at T/G tokens (capacity-balanced shuffle targets)")
     ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -163,7 +165,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ reference arm / CPU baseline
 
-def oracle_pass(w, ids, ids_cal, gates, x, placement, shuffle):
+def oracle_pass(w, ids, ids_cal, gates, x, placement, shuffle, balanced=False):
     """One pass of the path through the CPU oracle on a token sample.
     Returns (seconds, algorithmic dispatch+combine bytes)."""
     import oracle as orc
@@ -188,7 +190,8 @@ def oracle_pass(w, ids, ids_cal, gates, x, placement, shuffle):
         R = p["R"]
         nbytes += T * rowB + R * rowB + 4 * T * k + R * rowB + T * w.d * 4 + 8 * T * k
         if shuffle and l + 1 < L:
-            src = orc.shuffle_targets(ids[l], w.E, w.G, rs[l])
+            src = orc.shuffle_balanced(ids[l], w.E, w.G, rs[l], T // w.G) if balanced else \
+                orc.shuffle_targets(ids[l], w.E, w.G, rs[l])
     return time.perf_counter() - t0, nbytes
 
 
@@ -201,20 +204,20 @@ def cpu_sample(w, T_s, seed):
     return ids, cal, gates, x
 
 
-def sized_sample(w, target_s, shuffle):
+def sized_sample(w, target_s, shuffle, balanced=False):
     """Choose a token count (a multiple of G) whose oracle pass takes about target_s."""
     T_probe = max(w.G, (1024 // w.G) * w.G)
     ids, cal, gates, x = cpu_sample(w, T_probe, w.seed)
-    sec, _ = oracle_pass(w, ids, cal, gates, x, "correlated", shuffle)
+    sec, _ = oracle_pass(w, ids, cal, gates, x, "correlated", shuffle, balanced)
     T_s = int(T_probe * target_s / max(sec, 1e-6))
     T_s = max(w.G, min(w.T, (T_s // w.G) * w.G))
     return T_s
 
 
-def cpu_baseline(w, placement, shuffle, target_s):
-    T_s = sized_sample(w, target_s, shuffle)
+def cpu_baseline(w, placement, shuffle, target_s, balanced=False):
+    T_s = sized_sample(w, target_s, shuffle, balanced)
     ids, cal, gates, x = cpu_sample(w, T_s, w.seed)
-    sec, nbytes = oracle_pass(w, ids, cal, gates, x, placement, shuffle)
+    sec, nbytes = oracle_pass(w, ids, cal, gates, x, placement, shuffle, balanced)
     model = platform.processor() or platform.machine()
     try:
         with open("/proc/cpuinfo") as f:
@@ -235,15 +238,16 @@ def run_reference(a, w):
     if rank != 0:
         return
     shuffle = not a.no_shuffle
+    bal = shuffle and a.balanced_shuffle
     # each step: a bounded sample, so that warmup + steps end within a few minutes
     per_step = max(0.5, min(10.0, 150.0 / max(1, a.steps + a.warmup)))
-    T_s = sized_sample(w, per_step, shuffle)
+    T_s = sized_sample(w, per_step, shuffle, bal)
     ids, cal, gates, x = cpu_sample(w, T_s, w.seed)
     for _ in range(a.warmup):
-        oracle_pass(w, ids, cal, gates, x, a.placement, shuffle)
+        oracle_pass(w, ids, cal, gates, x, a.placement, shuffle, bal)
     secs, nb = [], 0
     for _ in range(a.steps):
-        s, nb = oracle_pass(w, ids, cal, gates, x, a.placement, shuffle)
+        s, nb = oracle_pass(w, ids, cal, gates, x, a.placement, shuffle, bal)
         secs.append(s)
     tot = sum(secs)
     value = nb * a.steps / tot / 1e9
@@ -251,7 +255,8 @@ def run_reference(a, w):
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * tot / a.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "tokens_per_step": T_s, "T": w.T, "E": w.E, "k": w.k, "G": w.G,
-                       "rpn": w.rpn, "d": w.d, "L": w.L, "placement": a.placement, "shuffle": shuffle},
+                       "rpn": w.rpn, "d": w.d, "L": w.L, "placement": a.placement,
+                       "shuffle": ("balanced" if bal else True) if shuffle else False},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": "%d of %d tokens per step, single-threaded C oracle" % (T_s, w.T)},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -313,6 +318,7 @@ def main():
             pg.destroy_process_group()
         return
     shuffle = (not a.no_shuffle) and w.L > 1
+    balanced = shuffle and a.balanced_shuffle
     out_dtype = torch.float32 if a.out_dtype == "f32" else torch.bfloat16
     if w.d == 0:
         raise SystemExit("workload %s has no hidden states; it is measured as the co-activation sweep" % w.name)
@@ -324,7 +330,7 @@ def main():
     hp = pipeline.prepare(w.E, w.G, w.rpn, ids, gates, x, w.dtype, ids_cal, placement=a.placement,
                           shuffle=shuffle, out_dtype=out_dtype, device=device, timers=True,
                           scales=make_expert_scales(w, seed=seed) if a.prereduce else None,
-                          replica_extra=a.replicas)
+                          replica_extra=a.replicas, shuffle_capacity=w.T // w.G if balanced else 0)
 
     def barrier():
         if pg is not None:
@@ -417,7 +423,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu = cpu_baseline(w, a.placement, shuffle, a.cpu_seconds)
+        cpu = cpu_baseline(w, a.placement, shuffle, a.cpu_seconds, balanced)
 
     if rank == 0:
         R = [int(s[0]) for s in summaries]
@@ -430,7 +436,8 @@ def main():
                        "combine": "receiver-side pre-reduced (stand-in experts)" if a.prereduce
                                   else "source-side weighted (identity experts)",
                        "replicas_per_rank": a.replicas,
-                       "shuffle": shuffle, "parallelism": "replicas (weak scaling, one batch per GPU)",
+                       "shuffle": ("balanced (T/G tokens per rank)" if balanced else True) if shuffle else False,
+                       "parallelism": "replicas (weak scaling, one batch per GPU)",
                        "l2": "inputs larger than L2 (x %.2f GB per GPU; no flush)" % (x.nbytes / 1e9)},
             "frac_of_hbm_peak": value / hbm,
             "roofline": roofline,
@@ -442,6 +449,11 @@ def main():
                      "local_share": [int(s[2]) / (w.T * w.k) for s in summaries],
                      "V": [int(s[3]) for s in summaries]},
             "clocks": clocks,
+            "balanced_shuffle": {
+                "rounds": hp.shuffle_info[:, 0].tolist(), "proposals": hp.shuffle_info[:, 1].tolist(),
+                "phase_us": {n: (hp.shuffle_info[:, 2 + i].double() / 1e3).tolist()
+                              for i, n in enumerate(["propose", "gather", "select", "barrier_wait"])}}
+            if balanced else None,
             "e2e": e2e,
             "gpu_launches": int(n_launch),
             "gpu_launches_per_step": n_launch / a.steps,

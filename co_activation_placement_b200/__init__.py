@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
             "moe_combine_rows": ([P, i, i64, i, P, i, i, P, i, P, P], i),
             "moe_rank_score": ([P, P, i, i, P, P, P], i),
             "moe_shuffle_targets": ([P, i, i, i, i, P, P, P, P], i),
+            "moe_shuffle_balanced_workspace": ([i, i, i], sz),
+            "moe_shuffle_balanced": ([P, i, i, i, i, P, i, P, P, P, sz, P, P], i),
             "moe_place_uniform": ([i, i, P], i),
             "moe_place_capacity": ([P, i, i, P, P], i),
             "moe_place_correlated": ([P, i, i, i, P], i),
@@ -397,6 +399,34 @@ def shuffle_targets(ids: torch.Tensor, E: int, G: int, rank_score_tab: torch.Ten
     err = new_err(ids.device) if err is None else err
     st = lib().moe_shuffle_targets(_ptr(ids), T, k, E, G, _ptr(rank_score_tab), _ptr(target), _ptr(err), _stream(ids))
     _check("moe_shuffle_targets", st)
+    return target
+
+
+def shuffle_balanced_workspace(T: int, G: int, capacity: int) -> int:
+    return int(lib().moe_shuffle_balanced_workspace(T, G, capacity))
+
+
+def shuffle_balanced(ids: torch.Tensor, E: int, G: int, rank_score_tab: torch.Tensor, capacity: int,
+                     target: Optional[torch.Tensor] = None, info: Optional[torch.Tensor] = None,
+                     err: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Shuffle targets with at most `capacity` tokens per rank (the unique
+    stable assignment under score desc, token asc, rank asc).  `info`, when
+    given (device int64 [6]), receives the rounds taken, the proposals made
+    and the nanoseconds spent proposing, gathering, selecting (slowest block)
+    and waiting at barriers."""
+    _dev(ids, torch.int32, "ids", 2)
+    _dev(rank_score_tab, torch.uint32, "rank_score", 2)
+    T, k = ids.shape
+    if target is None:
+        target = torch.empty(max(T, 1), dtype=torch.int32, device=ids.device)
+    err = new_err(ids.device) if err is None else err
+    need = shuffle_balanced_workspace(T, G, capacity)
+    if ws is None:
+        ws = _workspace(ids.device, "shuffle").get(need)
+    st = lib().moe_shuffle_balanced(_ptr(ids), T, k, E, G, _ptr(rank_score_tab), int(capacity), _ptr(target),
+                                    _ptr(info) if info is not None else None, _ptr(ws), ws.numel(), _ptr(err),
+                                    _stream(ids))
+    _check("moe_shuffle_balanced", st)
     return target
 
 

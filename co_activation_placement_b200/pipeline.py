@@ -10,7 +10,8 @@ A step is, for a batch of top-k routing decisions over L MoE layers:
      into the rank-major send buffer (moe_permute); identity experts (the
      expert output of a row is the row); the weighted combine back to token
      order (moe_combine); and, before layer l+1, the shuffle targets from
-     layer l's picks (moe_shuffle_targets).
+     layer l's picks (moe_shuffle_targets, or moe_shuffle_balanced when every
+     rank's shard is capped).
 
 Every step is a library call on torch's current stream; this module only
 allocates buffers and sequences the calls.  Placements and rank-score tables
@@ -64,6 +65,7 @@ class HotPath:
     prereduce: bool = False            # receiver-side pre-reduced combine with stand-in experts
     scales: List[torch.Tensor] = field(default_factory=list)   # f32 [E] per layer (prereduce)
     replicas: list = field(default_factory=list)   # per layer (replica_rank [E][1+nodes], n_rep [E]) or empty
+    shuffle_capacity: int = 0          # > 0: at most this many tokens per rank (moe_shuffle_balanced)
     # buffers
     stats: dict = field(default_factory=dict)
     plans: List[cap.Plan] = field(default_factory=list)
@@ -92,6 +94,11 @@ class HotPath:
         self.send = torch.empty((T * k, d), dtype=self.x.dtype, device=dev)
         self.outs = [torch.empty((T, d), dtype=self.out_dtype, device=dev) for _ in range(L)]
         self.targets = [torch.empty(T, dtype=torch.int32, device=dev) for _ in range(max(L - 1, 0))] if self.shuffle else []
+        if self.shuffle and self.shuffle_capacity > 0:
+            self.shuffle_ws = torch.empty(max(cap.shuffle_balanced_workspace(T, self.G, self.shuffle_capacity), 1),
+                                          dtype=torch.uint8, device=dev)
+            # rounds and proposals of each balanced shuffle
+            self.shuffle_info = torch.zeros((max(L - 1, 1), 6), dtype=torch.int64, device=dev)
         if self.replicas:
             self.pick_rank = torch.empty((T, k), dtype=torch.int32, device=dev)
             self.n_remote = torch.empty(T, dtype=torch.int32, device=dev)
@@ -160,9 +167,15 @@ class HotPath:
                     cap.combine(self.send, p.row_of, self.gates[l], out=self.outs[l], err=self.err)
                 self._mark("combine")
             if self.shuffle and l + 1 < self.L:
-                with nv("moe_shuffle_targets"):
-                    cap.shuffle_targets(self.ids[l], self.E, self.G, self.rank_scores[l],
-                                        target=self.targets[l], err=self.err)
+                if self.shuffle_capacity > 0:
+                    with nv("moe_shuffle_balanced"):
+                        cap.shuffle_balanced(self.ids[l], self.E, self.G, self.rank_scores[l], self.shuffle_capacity,
+                                             target=self.targets[l], info=self.shuffle_info[l], err=self.err,
+                                             ws=self.shuffle_ws)
+                else:
+                    with nv("moe_shuffle_targets"):
+                        cap.shuffle_targets(self.ids[l], self.E, self.G, self.rank_scores[l],
+                                            target=self.targets[l], err=self.err)
                 self._mark("shuffle")
 
     def capture(self, n_steps: int) -> torch.cuda.CUDAGraph:
@@ -255,7 +268,7 @@ def calibrate(ids_cal: torch.Tensor, E: int, G: int, rpn: int, placement: str, s
 def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarray], x: Optional[np.ndarray],
             x_dtype: str, ids_cal: np.ndarray, placement: str = "correlated", shuffle: bool = True,
             out_dtype=torch.bfloat16, device="cuda", rows: bool = True, timers: bool = False,
-            scales: Optional[np.ndarray] = None, replica_extra: int = 0) -> HotPath:
+            scales: Optional[np.ndarray] = None, replica_extra: int = 0, shuffle_capacity: int = 0) -> HotPath:
     """Upload a batch (host numpy arrays; x as float32 or bf16 bit patterns)
     and its calibration batch, calibrate, and return the step's HotPath."""
     dev = torch.device(device)
@@ -272,7 +285,7 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
         if scales is not None else []
     return HotPath(E=E, G=G, rpn=rpn, ids=ids_d, gates=gates_d, x=x_d, e2r=e2r, rank_scores=rs,
                    out_dtype=out_dtype, rows=rows, timers=timers, prereduce=scales is not None, scales=scales_d,
-                   replicas=reps)
+                   replicas=reps, shuffle_capacity=shuffle_capacity)
 
 
 def save_layout(path: str, expert_to_rank, rank_scores=(), replicas=(), stats=None):

@@ -304,6 +304,32 @@ moe_status moe_shuffle_targets(const int32_t *ids, int T, int k, int E, int G,
                                int32_t *err, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * moe_shuffle_balanced ([EC] abstract: the shuffle happens in the
+ *   reduce-scatter after attention, and a reduce-scatter hands every rank an
+ *   equal shard).  Shuffle targets with at most `capacity` tokens per rank:
+ *   with S_t(r) = sum_j rank_score[e_tj][r] (uint64), the result is that of
+ *   taking all (t, r) pairs in the order S desc, t asc, r asc and accepting a
+ *   pair when t has no rank yet and r holds fewer than `capacity` tokens --
+ *   the unique stable assignment of tokens to ranks under these orders.  With
+ *   capacity >= T it equals moe_shuffle_targets.  Computed by deferred
+ *   acceptance in one cooperative kernel (one block per SM).
+ *   ids device int32 [T][k]; rank_score device uint32 [E][G], E*G <= 16384,
+ *   G <= 64, T < 2^27; requires G*capacity >= T (MOE_ERR_ARG otherwise);
+ *   target device int32 [T] (out); info device int64 [6] (out, may be NULL):
+ *   rounds taken, proposals made, then nanoseconds spent proposing (block
+ *   0), gathering a rank's proposals and selecting (the slowest block's
+ *   totals) and waiting at grid barriers (block 0).  ws: moe_shuffle_balanced_workspace(T, G,
+ *   capacity) bytes, 256-byte aligned.  Data errors: MOE_DERR_ID_RANGE (the
+ *   token's picks then score 0); MOE_DERR_TIMEOUT if a grid barrier waited
+ *   more than 2 s (the kernel then returns with target incomplete).
+ * ---------------------------------------------------------------------- */
+size_t moe_shuffle_balanced_workspace(int T, int G, int capacity);
+moe_status moe_shuffle_balanced(const int32_t *ids, int T, int k, int E, int G,
+                                const uint32_t *rank_score, int capacity, int32_t *target,
+                                long long *info, void *ws, size_t ws_bytes, int32_t *err,
+                                cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Placement (host, synchronous)
  *
  * moe_place_uniform ([EPS] uniform listing): expert_to_rank[e] = e / (E/G);

@@ -118,6 +118,12 @@ def test_argument_errors_return_before_device_work(cap):
     assert L.moe_permute(fake, cap.MOE_BF16, 4, 7, 2, fake, 8, fake, fake, None) == cap.MOE_ERR_UNSUPPORTED
     assert L.moe_combine(fake, 7, 8, 8, fake, fake, 4, 2, fake, 0, fake, None) == cap.MOE_ERR_ARG
     assert L.moe_shuffle_targets(fake, 4, 2, 1024, 64, fake, fake, fake, None) == cap.MOE_ERR_UNSUPPORTED
+    # balanced shuffle: shards that cannot hold T, a table too large, a short workspace
+    assert L.moe_shuffle_balanced(fake, 9, 1, 4, 4, fake, 2, fake, None, fake, 1 << 30, fake, None) == cap.MOE_ERR_ARG
+    assert L.moe_shuffle_balanced(fake, 64, 2, 1024, 64, fake, 1, fake, None, fake, 1 << 30, fake, None) \
+        == cap.MOE_ERR_UNSUPPORTED
+    assert L.moe_shuffle_balanced(fake, 64, 2, 8, 4, fake, 16, fake, None, fake, 64, fake, None) == cap.MOE_ERR_WORKSPACE
+    assert cap.shuffle_balanced_workspace(1000, 8, 125) < cap.shuffle_balanced_workspace(1000, 8, 1000)
 
 
 @pytest.mark.parametrize("E,G,rpn,extra", [(16, 8, 2, 1), (64, 8, 8, 2), (64, 32, 8, 1), (256, 64, 8, 1), (24, 6, 1, 3)])

@@ -96,3 +96,19 @@ def test_fuzz_path(cap, seed):
         tg = cap.shuffle_targets(dev(ids[0]), E, G, dev(rs))
         assert (host(tg)[:T] == orc.shuffle_targets(ids[0], E, G, rs)).all()
     assert int(host(p.err)[0]) == 0
+
+
+@pytest.mark.parametrize("E", [6144, 8192, 12288])
+def test_plan_many_experts(cap, E):
+    # the placement table fills most of the plan kernels' shared memory
+    rng = np.random.default_rng(E)
+    T, k, G, rpn = 2048, 8, 64, 8
+    ids = np.argsort(rng.random((T, 64)), axis=1)[:, :k].astype(np.int32) * (E // 64) + rng.integers(0, E // 64, (T, 1))
+    ids = ids.astype(np.int32)
+    e2r = rng.permutation(orc.place_uniform(E, G)).astype(np.int32)
+    src = rng.integers(0, G, T).astype(np.int32)
+    p = cap.plan_dispatch(dev(ids), E, G, rpn, dev(e2r), src_rank=dev(src))
+    op = orc.plan(ids, E, G, rpn, e2r, src_rank=src)
+    assert int(host(p.err)[0]) == 0
+    assert host(p.summary).tolist() == op["summary"].tolist()
+    assert (host(p.row_of)[:T] == op["row_of"]).all()

@@ -74,7 +74,7 @@ def test_reference_arm_rank_nonzero_does_nothing(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
 
     class A:
-        steps, warmup, gpus, placement, no_shuffle = 1, 0, 2, "correlated", False
+        steps, warmup, gpus, placement, no_shuffle, balanced_shuffle = 1, 0, 2, "correlated", False, False
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
         bench.run_reference(A(), WORKLOADS["tiny"])
@@ -89,7 +89,7 @@ def test_reference_arm_prints_contract_line(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "1")
 
     class A:
-        steps, warmup, gpus, placement, no_shuffle = 1, 0, 1, "correlated", False
+        steps, warmup, gpus, placement, no_shuffle, balanced_shuffle = 1, 0, 1, "correlated", False, False
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
         bench.run_reference(A(), WORKLOADS["tiny"])
