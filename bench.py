@@ -50,6 +50,15 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def tensor_peak():
+    """Dense bf16 TFLOP/s for a kernel timed alone: the measured burst figure."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -68,6 +77,8 @@ def parse():
                     help="replicate experts (EXTRA more per rank) and assign tasks to the fewest remote nodes")
     ap.add_argument("--prereduce", action="store_true",
                     help="receiver-side pre-reduced combine with stand-in experts (gates dispatched with rows)")
+    ap.add_argument("--coact-method", default="auto", choices=["auto", "histogram", "tensor"],
+                    help="how the co-activation statistics count: per call, shared-memory histograms, tensor cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--sweep-only", action="store_true", help="only the co-activation statistics sweep")
@@ -309,6 +320,7 @@ def main():
                                 device_id=device)
         pg = dist
     seed = rank_seed(w, rank)
+    cap.coact_stats_method({"auto": 0, "histogram": 1, "tensor": 2}[a.coact_method])
     if a.sweep_only:
         hbm, _ = peaks()
         sweep = run_sweep(cap, pipeline, device, seed, a.steps, a.warmup, hbm, pg)
@@ -498,7 +510,17 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
     # per clock per SM, so at most 32 counter increments per clock per SM
     sms = torch.cuda.get_device_properties(device).multi_processor_count
     peak_inc = 32.0 * sms * SM_MAX_MHZ * 1e6
-    return {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "L": w.L, "ms": ms,
+    path = cap.coact_stats_path(w.L, w.T, w.k, w.E, True)
+    tensor = None
+    if path == "tensor":
+        # C_l = X_l X_l^T and M_l = X_l X_{l+1}^T: 2 E^2 T int8 operations each
+        ops = 2.0 * w.E * w.E * w.T * (2 * w.L - 1) / (ms * 1e-3)
+        bf16, kind = tensor_peak()
+        tensor = {"bound": "tensor", "achieved": ops / 1e12, "unit": "TOP/s (int8)", "peak": 2 * bf16,
+                  "frac": ops / 1e12 / (2 * bf16),
+                  "peak_note": "%s bf16 dense %.1f TFLOP/s x 2 (nominal int8 / bf16 ratio 4.5 / 2.25)" % (kind, bf16)}
+    return {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "L": w.L, "ms": ms, "method": path,
+            "tensor_roofline": tensor,
             "tokens_per_s": world * w.L * w.T / (ms * 1e-3),
             "increments_per_s": world * incs,
             "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,

@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
             "moe_status_string": ([i], ctypes.c_char_p),
             "moe_launch_count": ([], ctypes.c_uint64),
             "moe_coact_stats_workspace": ([i, i, i, i, i], sz),
+            "moe_coact_stats_method": ([i], i),
+            "moe_coact_stats_path": ([i, i, i, i, i], i),
             "moe_coact_stats": ([P, i, i, i, i, P, P, P, P, P, sz, P], i),
             "moe_plan_dispatch_workspace": ([i, i, i, i], sz),
             "moe_plan_dispatch": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
@@ -141,6 +143,20 @@ def new_err(device) -> torch.Tensor:
 
 
 # ---------------------------------------------------------------- statistics
+
+def coact_stats_method(method: int) -> int:
+    """0 = choose per call, 1 = shared-memory histograms, 2 = tensor cores
+    where the shape allows; returns the previous setting (process-wide)."""
+    prev = int(lib().moe_coact_stats_method(int(method)))
+    if prev < 0:
+        raise ValueError("method must be 0, 1 or 2")
+    return prev
+
+
+def coact_stats_path(L: int, T: int, k: int, E: int, with_trans: bool = True) -> str:
+    """'tensor' or 'histogram': the method moe_coact_stats would use now."""
+    return {1: "histogram", 2: "tensor"}.get(int(lib().moe_coact_stats_path(L, T, k, E, int(bool(with_trans)))), "none")
+
 
 def coact_stats_workspace(L: int, T: int, k: int, E: int, with_trans: bool = True) -> int:
     return int(lib().moe_coact_stats_workspace(L, T, k, E, int(bool(with_trans))))

@@ -25,8 +25,10 @@
 // result does not depend on order), mirrors the triangle and evaluates Ochiai
 // in fp64 with IEEE-rounded multiply, square root and divide.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
+#include "stats_mma.cuh"
 
 namespace moe {
 namespace {
@@ -386,14 +388,41 @@ moe_status launch_hist(const int32_t *ids, const StatsGeom &g, uint32_t *part, i
 
 using namespace moe;
 
+namespace {
+// 0: default (the histograms: on B200 they measured as fast as or faster than
+// the tensor-core contraction for E <= 256, k = 8, where building the one-hot
+// operand tiles costs about what the counter increments do); 1: histograms;
+// 2: tensor cores where the shape allows
+std::atomic<int> g_coact_method{0};
+}  // namespace
+
+extern "C" int moe_coact_stats_method(int method)
+{
+    if (method < 0 || method > 2) return -1;
+    return g_coact_method.exchange(method);
+}
+
+extern "C" int moe_coact_stats_path(int L, int T, int k, int E, int with_trans)
+{
+    if (L < 1 || T < 1 || k < 1 || k > 8 || E < k || E > 1024) return 0;
+    const int method = g_coact_method.load();
+    MmaGeom mg;
+    if (method == 2 && make_mma_geom(L, T, k, E, true, with_trans != 0, mg)) return 2;
+    return 1;
+}
+
 extern "C" size_t moe_coact_stats_workspace(int L, int T, int k, int E, int with_trans)
 {
     if (L < 1 || T < 0 || k < 1 || k > 8 || E < k || E > 1024) return 0;
-    // the largest of the geometries a call may choose (with or without C)
+    // the largest of the geometries a call may choose (with or without C, either method)
     long long words = 0;
     StatsGeom g;
     if (make_geom(L, T, k, E, true, with_trans != 0, g)) words = std::max(words, partial_words(g));
     if (with_trans && L > 1 && make_geom(L, T, k, E, false, true, g)) words = std::max(words, partial_words(g));
+    MmaGeom mg;
+    if (make_mma_geom(L, T, k, E, true, with_trans != 0, mg)) words = std::max(words, (long long)mma_partial_words(mg));
+    if (with_trans && L > 1 && make_mma_geom(L, T, k, E, false, true, mg))
+        words = std::max(words, (long long)mma_partial_words(mg));
     if (words == 0) return 0;
     return round_up((size_t)words * sizeof(uint32_t), 256) + 256;
 }
@@ -415,6 +444,13 @@ extern "C" moe_status moe_coact_stats(const int32_t *ids, int L, int T, int k, i
         if (ochiai && cudaMemsetAsync(ochiai, 0, sizeof(float) * EE * L, stream) != cudaSuccess) return MOE_ERR_CUDA;
         if (trans && cudaMemsetAsync(trans, 0, sizeof(uint32_t) * EE * (L - 1), stream) != cudaSuccess) return MOE_ERR_CUDA;
         return MOE_OK;
+    }
+    const int method = g_coact_method.load();
+    MmaGeom mg;
+    if (method == 2 && aligned16(ids) && make_mma_geom(L, T, k, E, want_c, want_t, mg)) {
+        const size_t need = mma_partial_words(mg) * sizeof(uint32_t);
+        if (!ws || !aligned256(ws) || ws_bytes < need) return MOE_ERR_WORKSPACE;
+        return coact_mma(ids, mg, static_cast<uint32_t *>(ws), coact, ochiai, trans, err, stream);
     }
     StatsGeom g;
     if (!make_geom(L, T, k, E, want_c, want_t, g)) return MOE_ERR_UNSUPPORTED;
