@@ -504,6 +504,19 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
         tot += s.elapsed_time(e)
     ms = reduce_max(tot / n, pg, device)
     nbytes = hp.step_bytes(None).stats
+    # what the placements do on this batch: local share and V per token at
+    # each rank count (8 ranks per node), placements from a calibration batch
+    effect = {}
+    ids_cal = torch.from_numpy(make_routing(w, seed=seed + 1)).to(device)
+    for G in w.sweep_G:
+        row = {}
+        for placement in ("uniform", "correlated"):
+            sm = pipeline.placement_effect(hp.ids, ids_cal, w.E, G, w.rpn, placement)
+            row[placement] = {"local_share": [round(int(r[2]) / int(r[4]), 5) for r in sm],
+                              "V_per_token": [round(int(r[3]) / w.T, 4) for r in sm],
+                              "rows_removed": [round(1 - int(r[0]) / int(r[4]), 4) for r in sm]}
+        effect["G=%d" % G] = row
+    del ids_cal
     world = pg.get_world_size() if pg is not None else 1
     incs = (w.L * w.T * w.k * (w.k + 1) // 2 + (w.L - 1) * w.T * w.k * w.k) / (ms * 1e-3)
     # the unit that bounds this kernel: shared memory serves 32 4-byte accesses
@@ -527,7 +540,8 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
             "atomic_roofline": {"bound": "shared-memory atomics", "achieved": incs, "unit": "increments/s",
                                 "peak": peak_inc, "frac": incs / peak_inc,
                                 "peak_note": "32 per clock per SM x %d SMs x %.0f MHz" % (sms, SM_MAX_MHZ)},
-            "algorithmic_bytes": nbytes, "err": int(hp.err.item())}
+            "algorithmic_bytes": nbytes, "err": int(hp.err.item()),
+            "placement_effect": effect}
 
 
 def run_e2e(hp, ids, gates, x, w, a, device, sb, pg, world):

@@ -288,6 +288,26 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
                    replicas=reps, shuffle_capacity=shuffle_capacity)
 
 
+def placement_effect(ids: torch.Tensor, ids_cal: torch.Tensor, E: int, G: int, rpn: int,
+                     placement: str = "correlated") -> np.ndarray:
+    """What a placement does to a batch without hidden states: the placement
+    is computed from the calibration batch (as calibrate() does), then every
+    layer's dispatch plan of the evaluation batch (contiguous shards of T/G
+    tokens) is built on the device.  Returns int64 [L][5]: R, R_remote, local,
+    V, T*k per layer (local share = local / (T*k), V per token = V / T)."""
+    e2r, _, _, _ = calibrate(ids_cal, E, G, rpn, placement, False)
+    L, T, k = ids.shape
+    ws = torch.empty(max(cap.plan_dispatch_workspace(T, k, G, False), 1), dtype=torch.uint8, device=ids.device)
+    plan = cap.Plan.empty(T, k, G, ids.device)
+    out = []
+    for l in range(L):
+        p = cap.plan_dispatch(ids[l], E, G, rpn, e2r[l], plan=plan, ws=ws)
+        out.append(p.summary.cpu().numpy().copy())
+        if int(p.err.item()):
+            raise ValueError("device data error %d" % int(p.err.item()))
+    return np.stack(out)
+
+
 def save_layout(path: str, expert_to_rank, rank_scores=(), replicas=(), stats=None):
     """Write a placement (and what was derived with it) to one .npz file: the
     expert-to-rank map per layer, rank-score tables per layer pair, replica

@@ -354,3 +354,17 @@ def test_argument_errors_enqueue_nothing(cap):
     with pytest.raises(cap.MoeError):
         cap.coact_stats(dev(np.zeros((1, 4, 9), np.int32)), 16)
     assert cap.launch_count() == before
+
+
+@pytest.mark.parametrize("G", [8, 32, 64])
+def test_sweep_placement_effect_full_size(cap, G):
+    """Local share and V of the statistics sweep's batch (1M tokens) under the
+    correlated placement of its calibration batch, layer 0, against the oracle."""
+    from co_activation_placement_b200 import pipeline
+    w = WORKLOADS["stats_sweep"]
+    ids = make_routing(w, seed=w.seed)[:1]
+    cal = make_routing(w, seed=w.seed + 1)[:1]
+    got = pipeline.placement_effect(dev(ids), dev(cal), w.E, G, w.rpn, "correlated")
+    e2r = orc.place_correlated(orc.coact(cal, w.E, want=("coact",))["coact"][0], G, w.rpn)
+    want = orc.plan(ids[0], w.E, G, w.rpn, e2r)["summary"]
+    assert got[0].tolist() == want.tolist()
