@@ -65,7 +65,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="large_ep64")
-    ap.add_argument("--placement", default="correlated", choices=["correlated", "uniform"])
+    ap.add_argument("--placement", default="correlated", choices=["correlated", "uniform", "capacity"])
     ap.add_argument("--no-shuffle", action="store_true")
     ap.add_argument("--balanced-shuffle", action="store_true",
                     help="cap every rank's shard at T/G tokens (capacity-balanced shuffle targets)")
@@ -187,6 +187,8 @@ def oracle_pass(w, ids, ids_cal, gates, x, placement, shuffle, balanced=False):
     cal = orc.coact(ids_cal, w.E)
     if placement == "correlated":
         e2r = [orc.place_correlated(cal["coact"][l], w.G, w.rpn) for l in range(L)]
+    elif placement == "capacity":
+        e2r = [orc.place_capacity(np.diag(cal["coact"][l]).astype(np.float64), w.G)[0] for l in range(L)]
     else:
         e2r = [orc.place_uniform(w.E, w.G) for _ in range(L)]
     rs = [orc.rank_score(cal["trans"][l], e2r[l + 1], w.G) for l in range(L - 1)] if shuffle else []
@@ -504,17 +506,21 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
         tot += s.elapsed_time(e)
     ms = reduce_max(tot / n, pg, device)
     nbytes = hp.step_bytes(None).stats
-    # what the placements do on this batch: local share and V per token at
-    # each rank count (8 ranks per node), placements from a calibration batch
+    # what the placements do on this batch: local share, V per token and rank
+    # load balance at each rank count (8 ranks per node), placements from a
+    # calibration batch
     effect = {}
     ids_cal = torch.from_numpy(make_routing(w, seed=seed + 1)).to(device)
     for G in w.sweep_G:
         row = {}
-        for placement in ("uniform", "correlated"):
-            sm = pipeline.placement_effect(hp.ids, ids_cal, w.E, G, w.rpn, placement)
+        for placement in ("uniform", "correlated", "capacity"):
+            sm, rl = pipeline.placement_effect(hp.ids, ids_cal, w.E, G, w.rpn, placement, loads=True)
             row[placement] = {"local_share": [round(int(r[2]) / int(r[4]), 5) for r in sm],
                               "V_per_token": [round(int(r[3]) / w.T, 4) for r in sm],
-                              "rows_removed": [round(1 - int(r[0]) / int(r[4]), 4) for r in sm]}
+                              "rows_removed": [round(1 - int(r[0]) / int(r[4]), 4) for r in sm],
+                              # per-rank load: token-expert assignments served
+                              "load_max_over_mean": [round(float(x.max() / x.mean()), 4) for x in rl],
+                              "load_cv": [round(float(x.std() / x.mean()), 4) for x in rl]}
         effect["G=%d" % G] = row
     del ids_cal
     world = pg.get_world_size() if pg is not None else 1

@@ -250,8 +250,11 @@ def calibrate(ids_cal: torch.Tensor, E: int, G: int, rpn: int, placement: str, s
         e2r_h = [cap.place_uniform(E, G) for _ in range(L)]
     elif placement == "correlated":
         e2r_h = [cap.place_correlated(coact_h[l], G, rpn) for l in range(L)]
+    elif placement == "capacity":
+        # first-fit decreasing on the calibration loads n_e = C_ee
+        e2r_h = [cap.place_capacity(np.diag(coact_h[l]).astype(np.float64), G)[0] for l in range(L)]
     else:
-        raise ValueError("placement must be uniform or correlated")
+        raise ValueError("placement must be uniform, correlated or capacity")
     e2r = [torch.from_numpy(a).to(ids_cal.device) for a in e2r_h]
     rs = []
     if shuffle:
@@ -289,12 +292,15 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
 
 
 def placement_effect(ids: torch.Tensor, ids_cal: torch.Tensor, E: int, G: int, rpn: int,
-                     placement: str = "correlated") -> np.ndarray:
+                     placement: str = "correlated", loads: bool = False):
     """What a placement does to a batch without hidden states: the placement
     is computed from the calibration batch (as calibrate() does), then every
     layer's dispatch plan of the evaluation batch (contiguous shards of T/G
     tokens) is built on the device.  Returns int64 [L][5]: R, R_remote, local,
-    V, T*k per layer (local share = local / (T*k), V per token = V / T)."""
+    V, T*k per layer (local share = local / (T*k), V per token = V / T).
+    With loads=True also returns float64 [L][G]: the token-expert
+    assignments each rank serves in the evaluation batch (sum of n_e = C_ee
+    over its experts)."""
     e2r, _, _, _ = calibrate(ids_cal, E, G, rpn, placement, False)
     L, T, k = ids.shape
     ws = torch.empty(max(cap.plan_dispatch_workspace(T, k, G, False), 1), dtype=torch.uint8, device=ids.device)
@@ -305,7 +311,13 @@ def placement_effect(ids: torch.Tensor, ids_cal: torch.Tensor, E: int, G: int, r
         out.append(p.summary.cpu().numpy().copy())
         if int(p.err.item()):
             raise ValueError("device data error %d" % int(p.err.item()))
-    return np.stack(out)
+    if not loads:
+        return np.stack(out)
+    n = cap.coact_stats(ids, E, want=("coact",))["coact"].cpu().numpy()
+    rank_load = np.zeros((L, G))
+    for l in range(L):
+        np.add.at(rank_load[l], e2r[l].cpu().numpy(), np.diag(n[l]).astype(np.float64))
+    return np.stack(out), rank_load
 
 
 def save_layout(path: str, expert_to_rank, rank_scores=(), replicas=(), stats=None):

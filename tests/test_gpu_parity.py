@@ -368,3 +368,25 @@ def test_sweep_placement_effect_full_size(cap, G):
     e2r = orc.place_correlated(orc.coact(cal, w.E, want=("coact",))["coact"][0], G, w.rpn)
     want = orc.plan(ids[0], w.E, G, w.rpn, e2r)["summary"]
     assert got[0].tolist() == want.tolist()
+
+
+@pytest.mark.parametrize("name", ["one_node", "ep32"])
+def test_pipeline_capacity_placement(cap, name):
+    """The step under the capacity-aware placement (first-fit decreasing on the
+    calibration loads): placements and plans against the oracle."""
+    from co_activation_placement_b200 import pipeline
+    w = WORKLOADS[name]
+    ids = make_routing(w)
+    ids_cal = make_routing(w, seed=w.seed + 1)
+    hp = pipeline.prepare(w.E, w.G, w.rpn, ids, make_gates(w), make_hidden(w), w.dtype, ids_cal,
+                          placement="capacity", shuffle=False, out_dtype=torch.float32)
+    hp.step()
+    torch.cuda.synchronize()
+    assert int(host(hp.err)[0]) == 0
+    oc = orc.coact(ids_cal, w.E, want=("coact",))["coact"]
+    for l in range(w.L):
+        e2r = orc.place_capacity(np.diag(oc[l]).astype(np.float64), w.G)[0]
+        assert (host(hp.e2r[l]) == e2r).all()
+        op = orc.plan(ids[l], w.E, w.G, w.rpn, e2r)
+        assert host(hp.plans[l].summary).tolist() == op["summary"].tolist()
+        assert (host(hp.plans[l].row_of)[: w.T] == op["row_of"]).all()
