@@ -11,10 +11,12 @@
 // moe_rank_score: one block per expert row e, a shared uint64 accumulator per
 // rank (integer atomics: order-free).  moe_shuffle_targets: the E x G table
 // sits in shared memory (one block per SM, so it is copied once per SM); a
-// warp loads the picks of 32 tokens at once (one per lane) and then scores
-// them one at a time, each lane owning ranks lane and lane+32 (conflict-free:
-// a row of the table is read contiguously), with uint64 sums and a warp argmax
-// on (score desc, rank asc).
+// warp stages the picks of 32 tokens in shared memory and then scores them one
+// at a time, every lane reading the token's picks with broadcast loads and
+// owning ranks lane and lane+32 (conflict-free: a row of the table is read
+// contiguously), with uint64 sums.  The argmax on (score desc, rank asc) is a
+// maximum of the packed key (score << 6) | (63 - rank): one redux.sync when the
+// warp's sums fit 26 bits, five 64-bit shuffles otherwise.
 #include <algorithm>
 
 #include "common.cuh"
@@ -54,7 +56,8 @@ __global__ void __launch_bounds__(kShuffleThreads)
 shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, const uint32_t *__restrict__ rs_g,
                        int32_t *__restrict__ target, int32_t *err)
 {
-    extern __shared__ __align__(16) uint32_t tab[];   // [E][G]
+    extern __shared__ __align__(16) uint32_t tab[];   // [E][G], then each warp's 32 tokens' picks
+    int *picks_all = reinterpret_cast<int *>(tab + ((E * G + 3) & ~3));
     {   // copy the table: 16-byte vectors where the layout allows, 8 in flight per thread
         const int n = E * G;
         const bool vec = (n % 4 == 0) && ((reinterpret_cast<uintptr_t>(rs_g) & 15u) == 0);
@@ -75,48 +78,66 @@ shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, con
         }
     }
     __syncthreads();
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int KP = (K + 3) & ~3;                  // picks per token in shared memory, padded to int4
+    int *picks = picks_all + warp * 32 * KP;
     const int nwarps = gridDim.x * (kShuffleThreads / 32);
-    const int gw = blockIdx.x * (kShuffleThreads / 32) + (threadIdx.x >> 5);
-    // a warp takes 32 tokens at a time: lane l loads token t0+l's picks, then
-    // the warp scores the 32 tokens one after another
+    const int gw = blockIdx.x * (kShuffleThreads / 32) + warp;
+    // a warp takes 32 tokens at a time: lane l loads token t0+l's picks into
+    // shared memory, then the warp scores the 32 tokens one after another,
+    // every lane reading the token's picks with broadcast loads
     for (int t0 = gw * 32; t0 < T; t0 += nwarps * 32) {
         const int tl = t0 + lane;
-        int e[K];
         bool ok = tl < T;
+        {
+            int e[KP];
 #pragma unroll
-        for (int j = 0; j < K; ++j) {
-            e[j] = tl < T ? __ldg(ids + (size_t)tl * K + j) : 0;
-            ok &= (unsigned)e[j] < (unsigned)E;
+            for (int j = 0; j < KP; ++j) {
+                e[j] = (j < K && tl < T) ? __ldg(ids + (size_t)tl * K + j) : 0;
+                if (j < K && (unsigned)e[j] >= (unsigned)E) { ok = false; }
+            }
+            if (tl < T && !ok) record_error(err, MOE_DERR_ID_RANGE);
+#pragma unroll
+            for (int j = 0; j < KP; ++j) picks[lane * KP + j] = (ok && j < K) ? e[j] : -1;
         }
-        if (tl < T && !ok) record_error(err, MOE_DERR_ID_RANGE);
+        __syncwarp();
         const int n = min(32, T - t0);
         int result = 0;
         for (int i = 0; i < n; ++i) {
-            const bool good = __shfl_sync(0xffffffffu, ok, i);
+            int e[KP];
+#pragma unroll
+            for (int q = 0; q < KP / 4; ++q) {
+                const int4 v = reinterpret_cast<const int4 *>(picks + i * KP)[q];
+                e[4 * q] = v.x; e[4 * q + 1] = v.y; e[4 * q + 2] = v.z; e[4 * q + 3] = v.w;
+            }
             unsigned long long a0 = 0, a1 = 0;
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-                const int ej = __shfl_sync(0xffffffffu, e[j], i);
-                if (good) {
-                    const uint32_t *row = tab + (size_t)ej * G;
+                if (e[j] >= 0) {
+                    const uint32_t *row = tab + (size_t)e[j] * G;
                     if (lane < G) a0 += row[lane];
                     if (lane + 32 < G) a1 += row[lane + 32];
                 }
             }
-            // candidate key: score + 1 for a real rank, 0 for none
-            unsigned long long best = lane < G ? a0 + 1 : 0;
-            int bi = lane;
-            if (lane + 32 < G && a1 + 1 > best) { best = a1 + 1; bi = lane + 32; }
+            // packed key (score << 6) | (63 - rank): the maximum is the best
+            // rank, the lowest rank among equal scores
+            int bi;
+            if (__all_sync(0xffffffffu, (a0 | a1) < (1ull << 26))) {
+                uint32_t key = lane < G ? (((uint32_t)a0 << 6) | (uint32_t)(63 - lane)) : 0u;
+                if (lane + 32 < G) key = max(key, ((uint32_t)a1 << 6) | (uint32_t)(31 - lane));
+                key = __reduce_max_sync(0xffffffffu, key);
+                bi = 63 - (int)(key & 63u);
+            } else {
+                unsigned long long best = lane < G ? (a0 << 6) | (unsigned long long)(63 - lane) : 0ull;
+                if (lane + 32 < G) best = max(best, (a1 << 6) | (unsigned long long)(31 - lane));
 #pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+                for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+                bi = 63 - (int)(best & 63u);
             }
-            if (lane == i) result = good ? bi : 0;
+            if (lane == i) result = e[0] >= 0 ? bi : 0;
         }
         if (tl < T) target[tl] = result;
+        __syncwarp();
     }
 }
 
@@ -139,7 +160,8 @@ template <int K>
 static moe_status launch_shuffle(const int32_t *ids, int T, int E, int G, const uint32_t *rs, int32_t *target,
                                  int32_t *err, cudaStream_t s)
 {
-    const size_t smem = sizeof(uint32_t) * (size_t)E * G;
+    constexpr int KP = (K + 3) & ~3;
+    const size_t smem = sizeof(uint32_t) * (size_t)((E * G + 3) & ~3) + sizeof(int) * (kShuffleThreads / 32) * 32 * KP;
     if (allow_smem(shuffle_targets_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
     // one block per SM at most: every block first copies the whole table
     const long long need = ((long long)T + kShuffleThreads - 1) / kShuffleThreads;

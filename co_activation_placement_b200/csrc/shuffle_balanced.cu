@@ -170,6 +170,9 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
     __shared__ int cnt_s[64], base_s[64], tot_s[64], hn_s[64], hsel_s[64];
     __shared__ unsigned int hist_s[256];
     __shared__ int kept_s, digit_s, need_s, gather_s, bin_s;
+    constexpr int KP = (K + 3) & ~3;                  // picks per staged token, padded to int4
+    __shared__ __align__(16) int picks_s[kBalWarps][32 * KP];
+    __shared__ int tok_s[kBalWarps][32];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = a.G, E = a.E, Cc = a.Cc;
@@ -227,38 +230,60 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
                 if ((unsigned)e[j] >= (unsigned)E) { ok = false; e[j] = 0; }
             }
             if (mine && !ok) record_error(a.err, MOE_DERR_ID_RANGE);
+            // stage the warp's tokens and picks (-1: a token with an invalid
+            // pick, which then scores 0 everywhere) for broadcast reads
+            int *pk = picks_s[warp];
+            if (lane < per) {
+                tok_s[warp][lane] = t;
+#pragma unroll
+                for (int j = 0; j < KP; ++j) pk[lane * KP + j] = (j < K && ok) ? e[j] : -1;
+            }
+            __syncwarp();
             const int n = min(per, nF - i0);
             int my_r = 0;
             unsigned long long my_key = 0;
             for (int q = 0; q < n; ++q) {
-                const int tq = __shfl_sync(0xffffffffu, t, q);
-                const bool good = __shfl_sync(0xffffffffu, ok, q);
-                unsigned long long s0 = 0, s1 = 0;
+                const int tq = tok_s[warp][q];
+                int ev[KP];
 #pragma unroll
-                for (int j = 0; j < K; ++j) {
-                    const int ej = __shfl_sync(0xffffffffu, e[j], q);
-                    if (good) {
-                        const uint32_t *row = tab + (size_t)ej * G;
+                for (int c4 = 0; c4 < KP / 4; ++c4) {
+                    const int4 v = reinterpret_cast<const int4 *>(pk + q * KP)[c4];
+                    ev[4 * c4] = v.x; ev[4 * c4 + 1] = v.y; ev[4 * c4 + 2] = v.z; ev[4 * c4 + 3] = v.w;
+                }
+                const bool good = ev[0] >= 0;
+                unsigned long long s0 = 0, s1 = 0;
+                if (good) {
+#pragma unroll
+                    for (int j = 0; j < K; ++j) {
+                        const uint32_t *row = tab + (size_t)ev[j] * G;
                         if (lane < G) s0 += row[lane];
                         if (lane + 32 < G) s1 += row[lane + 32];
                     }
                 }
                 // one packed value per rank: (S + 1) << 6 | (63 - r), or 0 for a
                 // rank that would reject the token (its key <= theta_r); the
-                // warp maximum is the best acceptable rank (equal S: lower r)
+                // warp maximum is the best acceptable rank (equal S: lower r):
+                // one redux.sync when every S fits 25 bits, else 64-bit shuffles
                 const unsigned long long low = kTokMask - (unsigned long long)tq;
-                unsigned long long best = 0;
-                if (lane < G && ((s0 << kKeyShift) | low) > theta_s[lane])
-                    best = ((s0 + 1) << 6) | (unsigned long long)(63 - lane);
-                if (lane + 32 < G && ((s1 << kKeyShift) | low) > theta_s[lane + 32])
-                    best = max(best, ((s1 + 1) << 6) | (unsigned long long)(31 - lane));
+                const bool ok0 = lane < G && ((s0 << kKeyShift) | low) > theta_s[lane];
+                const bool ok1 = lane + 32 < G && ((s1 << kKeyShift) | low) > theta_s[lane + 32];
+                unsigned long long best;
+                if (__all_sync(0xffffffffu, (s0 | s1) < (1ull << 25))) {
+                    uint32_t v = ok0 ? (((uint32_t)s0 + 1u) << 6) | (uint32_t)(63 - lane) : 0u;
+                    if (ok1) v = max(v, (((uint32_t)s1 + 1u) << 6) | (uint32_t)(31 - lane));
+                    best = __reduce_max_sync(0xffffffffu, v);
+                } else {
+                    best = ok0 ? ((s0 + 1) << 6) | (unsigned long long)(63 - lane) : 0ull;
+                    if (ok1) best = max(best, ((s1 + 1) << 6) | (unsigned long long)(31 - lane));
 #pragma unroll
-                for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+                    for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+                }
                 if (lane == q) {
                     my_r = 63 - (int)(best & 63u);
                     my_key = best ? (((best >> 6) - 1) << kKeyShift) | low : 0ull;
                 }
             }
+            __syncwarp();
             if (mine) {
                 if (my_key == 0) {            // no rank can take it: impossible while T <= G*capacity
                     record_error(a.err, MOE_DERR_RANK_RANGE);
