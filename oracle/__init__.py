@@ -53,6 +53,7 @@ def lib():
             "orc_rank_score": [P, P, i, i, P],
             "orc_shuffle_targets": [P, i, i, i, i, P, P],
             "orc_shuffle_balanced": [P, i, i, i, i, P, i, P],
+            "orc_coact_ema": [P, i, i, ctypes.c_double, P, P, P],
             "orc_dispatch_gates": [P, P, i, i, P, P, i64, P, P],
             "orc_expert_reduce": [P, i, i64, i, P, P, i, P, i, P],
             "orc_combine_rows": [P, i, i64, i, P, i, i, P],
@@ -198,6 +199,18 @@ def shuffle_balanced(ids_l: np.ndarray, E: int, G: int, rank_score_tab: np.ndarr
     tgt = np.empty(T, np.int32)
     _check("orc_shuffle_balanced", lib().orc_shuffle_balanced(_p(ids_l), T, k, E, G, _p(rs), int(capacity), _p(tgt)))
     return tgt
+
+
+def coact_ema(coact, alpha: float, ema_in=None):
+    """(ema fp64 [L][E][E], ochiai f32 [L][E][E]) after one batch's counts."""
+    c = np.ascontiguousarray(coact, dtype=np.uint32)
+    L, E, _ = c.shape
+    out = np.empty(c.shape, np.float64)
+    och = np.empty(c.shape, np.float32)
+    ein = None if ema_in is None else np.ascontiguousarray(ema_in, dtype=np.float64)
+    _check("orc_coact_ema", lib().orc_coact_ema(_p(c), L, E, float(alpha), _p(ein) if ein is not None else None,
+                                                _p(out), _p(och)))
+    return out, och
 
 
 def dispatch_gates(ids_l, w_l, row_token, row_jmask):

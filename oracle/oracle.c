@@ -495,6 +495,41 @@ int orc_shuffle_balanced(const int32_t *ids, int T, int k, int E, int G, const u
     return ORC_OK;
 }
 
+/* Exponential moving averages of the co-activation counts ("Cobalt", "Key
+ * Observation": the planner keeps an EMA of the tokens selecting both experts
+ * i and j, and of each expert's load, and evaluates Ochiai on them).  Per cell,
+ * in fp64: ema_out = alpha * C + (1 - alpha) * ema_in, or C when ema_in is
+ * NULL (the first batch); the load EMA is the diagonal.  Ochiai on the
+ * averages: ema_ij / sqrt(ema_ii * ema_jj), rounded once to fp32, 0 when the
+ * product is 0. */
+int orc_coact_ema(const uint32_t *coact, int L, int E, double alpha, const double *ema_in, double *ema_out,
+                  float *ochiai)
+{
+    if (L < 1 || E < 1 || !(alpha >= 0.0 && alpha <= 1.0)) return ORC_ERR_ARG;
+    size_t EE = (size_t)E * E;
+    for (size_t c = 0; c < (size_t)L * EE; ++c) {
+        double x = (double)coact[c];
+        if (ema_in) {
+            double a = alpha * x;
+            double b = (1.0 - alpha) * ema_in[c];
+            ema_out[c] = a + b;
+        } else {
+            ema_out[c] = x;
+        }
+    }
+    if (ochiai) {
+        for (int l = 0; l < L; ++l) {
+            const double *m = ema_out + (size_t)l * EE;
+            for (int i = 0; i < E; ++i)
+                for (int j = 0; j < E; ++j) {
+                    double den = m[(size_t)i * E + i] * m[(size_t)j * E + j];
+                    ochiai[(size_t)l * EE + (size_t)i * E + j] = den > 0.0 ? (float)(m[(size_t)i * E + j] / sqrt(den)) : 0.0f;
+                }
+        }
+    }
+    return ORC_OK;
+}
+
 /* ---- receiver-side pre-reduced combine (a NEXT row of the path) ----------- */
 
 /* Gate dispatch ([CE] footnote 3: the routed probabilities are dispatched with

@@ -14,7 +14,7 @@ from conftest import ROOT
 
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_pins.py", "tests/test_oracle_brute.py", "tests/test_oracle_prereduce.py",
-        "tests/test_oracle_replicas.py", "tests/test_oracle_shuffle_balanced.py"]
+        "tests/test_oracle_replicas.py", "tests/test_oracle_shuffle_balanced.py", "tests/test_oracle_ema.py"]
 
 MUTANTS = {
     "counts_drop_diagonal": ("                for (int a = 0; a < k; ++a)\n                    for (int b = 0; b < k; ++b)\n"
@@ -63,6 +63,9 @@ MUTANTS = {
                                      "if (target[p->t] < 0 && held[p->r] <= capacity) {"),
     "balanced_score_ascending": ("if (a->s != b->s) return a->s > b->s ? -1 : 1;",
                                  "if (a->s != b->s) return a->s < b->s ? -1 : 1;"),
+    "ema_weights_swapped": ("double a = alpha * x;\n            double b = (1.0 - alpha) * ema_in[c];",
+                            "double a = (1.0 - alpha) * x;\n            double b = alpha * ema_in[c];"),
+    "ema_first_batch_zero": ("            ema_out[c] = x;\n        }", "            ema_out[c] = 0.0 * x;\n        }"),
 }
 
 
