@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
             "moe_coact_stats_workspace": ([i, i, i, i, i], sz),
             "moe_coact_stats_method": ([i], i),
             "moe_coact_stats_path": ([i, i, i, i, i], i),
+            "moe_coact_ema": ([P, i, i, ctypes.c_double, P, P, P, P], i),
             "moe_coact_stats": ([P, i, i, i, i, P, P, P, P, P, sz, P], i),
             "moe_plan_dispatch_workspace": ([i, i, i, i], sz),
             "moe_plan_dispatch": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
@@ -182,6 +183,22 @@ def coact_stats(ids: torch.Tensor, E: int, coact=None, ochiai=None, trans=None, 
                                _ptr(ws), ws.numel(), _stream(ids))
     _check("moe_coact_stats", st)
     return dict(coact=coact, ochiai=ochiai, trans=trans, err=err)
+
+
+def coact_ema(coact: torch.Tensor, alpha: float, ema_in: Optional[torch.Tensor] = None,
+              ema_out: Optional[torch.Tensor] = None, ochiai: Optional[torch.Tensor] = None, want_ochiai: bool = True):
+    """EMA of co-activation counts (float64 [L][E][E], out of place) and
+    Ochiai on it.  ema_in None: the first batch.  Returns (ema_out, ochiai)."""
+    _dev(coact, torch.uint32, "coact", 3)
+    L, E, _ = coact.shape
+    if ema_out is None:
+        ema_out = torch.empty((L, E, E), dtype=torch.float64, device=coact.device)
+    if ochiai is None and want_ochiai:
+        ochiai = torch.empty((L, E, E), dtype=torch.float32, device=coact.device)
+    st = lib().moe_coact_ema(_ptr(coact), L, E, float(alpha), _ptr(ema_in), _ptr(ema_out), _ptr(ochiai),
+                             _stream(coact))
+    _check("moe_coact_ema", st)
+    return ema_out, ochiai
 
 
 # ---------------------------------------------------------------- dispatch plan

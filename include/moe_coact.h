@@ -192,6 +192,22 @@ moe_status moe_assign_replicas(const int32_t *ids, int T, int k, int E, int G, i
                                int32_t *pick_rank, int32_t *n_remote, int32_t *err, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * moe_coact_ema ([CB] "Key Observation": Ochiai on exponential moving averages
+ *   of the co-selection counts and loads).  Per cell, in fp64 with IEEE
+ *   rounding and no fused multiply-add:
+ *     ema_out[l][i][j] = alpha * coact[l][i][j] + (1 - alpha) * ema_in[l][i][j]
+ *   (ema_out = coact when ema_in is NULL: the first batch); the diagonal is the
+ *   load EMA; ochiai[l][i][j] = ema_ij / sqrt(ema_ii * ema_jj) rounded once to
+ *   fp32, 0 when the product is 0.
+ *   coact device uint32 [L][E][E] (moe_coact_stats's output); ema_in device
+ *   double [L][E][E] or NULL; ema_out device double [L][E][E], not ema_in
+ *   (out of place; alternate two buffers); ochiai device float [L][E][E] or
+ *   NULL.  MOE_ERR_ARG for alpha outside [0, 1], ema_in == ema_out, E > 4096.
+ * ---------------------------------------------------------------------- */
+moe_status moe_coact_ema(const uint32_t *coact, int L, int E, double alpha, const double *ema_in,
+                         double *ema_out, float *ochiai, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Dispatch plan without caller-provided workspace.  The pages have no
  * counterpart: this entry point exists for callers that cannot allocate
  * device memory -- code running inside another framework's allocator or

@@ -124,6 +124,9 @@ def test_argument_errors_return_before_device_work(cap):
         == cap.MOE_ERR_UNSUPPORTED
     assert L.moe_shuffle_balanced(fake, 64, 2, 8, 4, fake, 16, fake, None, fake, 64, fake, None) == cap.MOE_ERR_WORKSPACE
     assert cap.shuffle_balanced_workspace(1000, 8, 125) < cap.shuffle_balanced_workspace(1000, 8, 1000)
+    # EMA: alpha outside [0, 1], in place
+    assert L.moe_coact_ema(fake, 1, 4, ctypes.c_double(1.5), None, fake, None, None) == cap.MOE_ERR_ARG
+    assert L.moe_coact_ema(fake, 1, 4, ctypes.c_double(0.5), fake, fake, None, None) == cap.MOE_ERR_ARG
 
 
 @pytest.mark.parametrize("E,G,rpn,extra", [(16, 8, 2, 1), (64, 8, 8, 2), (64, 32, 8, 1), (256, 64, 8, 1), (24, 6, 1, 3)])
