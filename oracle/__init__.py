@@ -47,6 +47,7 @@ def lib():
             "orc_place_uniform": [i, i, P],
             "orc_place_capacity": [P, i, i, P, P],
             "orc_place_correlated": [P, i, i, i, P],
+            "orc_place_correlated_capped": [P, i, i, i, ctypes.c_double, P],
             "orc_plan": [P, i, i, i, i, i, P, P, P, P, P, P, P, P, P],
             "orc_permute": [P, i, i, i, P, i64, P],
             "orc_combine": [P, i, i64, i, P, P, i, i, P],
@@ -120,6 +121,15 @@ def place_correlated(coact_l: np.ndarray, G: int, rpn: int) -> np.ndarray:
     E = c.shape[0]
     e2r = np.empty(E, np.int32)
     _check("orc_place_correlated", lib().orc_place_correlated(_p(c), E, G, rpn, _p(e2r)))
+    return e2r
+
+
+def place_correlated_capped(coact_l: np.ndarray, G: int, rpn: int, eps: float) -> np.ndarray:
+    """Correlated placement with load tolerance eps (eps < 0: none)."""
+    c = np.ascontiguousarray(coact_l, dtype=np.uint32)
+    E = c.shape[0]
+    e2r = np.empty(E, np.int32)
+    _check("orc_place_correlated_capped", lib().orc_place_correlated_capped(_p(c), E, G, rpn, float(eps), _p(e2r)))
     return e2r
 
 

@@ -167,22 +167,26 @@ def blocking_pairs(ids_l, G, rank_score, capacity, tgt):
     return out
 
 
-def place_correlated(C, G, rpn):
+def place_correlated(C, G, rpn, eps=-1.0):
     """Restatement of the greedy grouping with Python lists and Fraction-free
-    fp64 (same summation order as the specification: insertion order)."""
+    fp64 (same summation order as the specification: insertion order); with
+    eps >= 0 a group only admits experts that keep its load within the cap,
+    else the lightest expert left."""
     E = len(C)
+    W = float(sum(int(C[e][e]) for e in range(E)))
 
     def s64(i, j):
         den = float(C[i][i]) * float(C[j][j])
         return C[i][j] / math.sqrt(den) if den > 0 else 0.0
 
-    def groups(pool, m):
+    def groups(pool, m, cap):
         size = len(pool) // m
         left = sorted(pool)
         res = []
         for _ in range(m):
             seed = max(left, key=lambda e: (C[e][e], -e))
             grp = [seed]
+            load = int(C[seed][seed])
             left.remove(seed)
             while len(grp) < size:
                 def score(e):
@@ -190,16 +194,23 @@ def place_correlated(C, G, rpn):
                     for g in grp:
                         s += s64(e, g)
                     return s
-                best = max(left, key=lambda e: (score(e), -e))
+                fits = [e for e in left if cap < 0 or float(load + int(C[e][e])) <= cap]
+                if fits:
+                    best = max(fits, key=lambda e: (score(e), -e))
+                else:
+                    best = min(left, key=lambda e: (int(C[e][e]), e))
                 grp.append(best)
+                load += int(C[best][best])
                 left.remove(best)
             res.append(grp)
         return res
 
     nodes = G // rpn
+    cap_node = (1 + eps) * W / nodes if eps >= 0 else -1.0
+    cap_rank = (1 + eps) * W / G if eps >= 0 else -1.0
     e2r = [0] * E
-    for q, ng in enumerate(groups(list(range(E)), nodes)):
-        for u, rg in enumerate(groups(ng, rpn)):
+    for q, ng in enumerate(groups(list(range(E)), nodes, cap_node)):
+        for u, rg in enumerate(groups(ng, rpn, cap_rank)):
             for e in rg:
                 e2r[e] = q * rpn + u
     return e2r

@@ -171,7 +171,15 @@ static double ochiai64(const uint32_t *C, int E, int i, int j)
  * C_ee, then repeatedly add the unassigned expert whose summed fp64 Ochiai to
  * the group's members (summed in insertion order) is largest; ties go to the
  * lowest expert id.  group_of[pool index] receives the group number. */
-static void greedy_groups(const uint32_t *C, int E, const int *pool, int n, int m, int *group_of)
+/* Greedy equal-size grouping of pool[0..n) into m groups.  A group is seeded
+ * with the unassigned expert of largest load n_e = C_ee and grown by the
+ * unassigned expert whose Ochiai summed over the group's members (in joining
+ * order) is largest; ties go to the lowest id.  With cap >= 0 (the load
+ * tolerance of "Cobalt", "Problem Formulation"), only experts whose load keeps
+ * the group's load n_e summed at most cap are candidates; when none is, the
+ * lightest unassigned expert joins (ties: lowest id), so every group still
+ * gets its n/m experts. */
+static void greedy_groups(const uint32_t *C, int E, const int *pool, int n, int m, int *group_of, double cap)
 {
     int size = n / m;
     int *taken = (int *)calloc(n, sizeof(int));
@@ -186,18 +194,29 @@ static void greedy_groups(const uint32_t *C, int E, const int *pool, int n, int 
         taken[best] = 1;
         group_of[best] = g;
         members[0] = pool[best];
+        uint64_t load = C[(size_t)pool[best] * E + pool[best]];
         for (int cnt = 1; cnt < size; ++cnt) {
             int pick = -1;
             double pick_score = 0.0;
             for (int x = 0; x < n; ++x) {
                 if (taken[x]) continue;
+                uint64_t nx = C[(size_t)pool[x] * E + pool[x]];
+                if (cap >= 0.0 && (double)(load + nx) > cap) continue;
                 double s = 0.0;
                 for (int q = 0; q < cnt; ++q) s += ochiai64(C, E, pool[x], members[q]);
                 if (pick < 0 || s > pick_score) { pick = x; pick_score = s; }
             }
+            if (pick < 0) {   /* nothing fits: the lightest */
+                for (int x = 0; x < n; ++x) {
+                    if (taken[x]) continue;
+                    if (pick < 0 || C[(size_t)pool[x] * E + pool[x]] < C[(size_t)pool[pick] * E + pool[pick]])
+                        pick = x;
+                }
+            }
             taken[pick] = 1;
             group_of[pick] = g;
             members[cnt] = pool[pick];
+            load += C[(size_t)pool[pick] * E + pool[pick]];
         }
     }
     free(members);
@@ -209,26 +228,37 @@ static void greedy_groups(const uint32_t *C, int E, const int *pool, int n, int 
  * with more than one node, first group the experts into G/rpn node groups of
  * E/(G/rpn), then each node's experts into rpn rank groups of E/G; node group
  * q and its rank group u map to rank q*rpn + u.  coact is one layer's
- * uint32 [E][E] count matrix. */
-int orc_place_correlated(const uint32_t *coact, int E, int G, int rpn, int32_t *expert_to_rank)
+ * uint32 [E][E] count matrix.  With eps >= 0 every node group's load is kept
+ * to at most (1+eps) W / (G/rpn) and every rank group's to (1+eps) W / G
+ * where possible, W the total load; eps < 0: no load limit. */
+int orc_place_correlated_capped(const uint32_t *coact, int E, int G, int rpn, double eps, int32_t *expert_to_rank)
 {
     if (E < 1 || G < 1 || rpn < 1 || G % rpn != 0 || E % G != 0) return ORC_ERR_ARG;
     int nodes = G / rpn;
+    double W = 0.0;
+    for (int e = 0; e < E; ++e) W += (double)coact[(size_t)e * E + e];
+    double cap_node = eps >= 0.0 ? (1.0 + eps) * W / nodes : -1.0;
+    double cap_rank = eps >= 0.0 ? (1.0 + eps) * W / G : -1.0;
     int *all = (int *)malloc(sizeof(int) * E);
     int *node_of = (int *)malloc(sizeof(int) * E);
     int *pool = (int *)malloc(sizeof(int) * E);
     int *grp = (int *)malloc(sizeof(int) * E);
     for (int e = 0; e < E; ++e) all[e] = e;
-    greedy_groups(coact, E, all, E, nodes, node_of);
+    greedy_groups(coact, E, all, E, nodes, node_of, cap_node);
     for (int q = 0; q < nodes; ++q) {
         int n = 0;
         for (int e = 0; e < E; ++e)
             if (node_of[e] == q) pool[n++] = e;
-        greedy_groups(coact, E, pool, n, rpn, grp);
+        greedy_groups(coact, E, pool, n, rpn, grp, cap_rank);
         for (int x = 0; x < n; ++x) expert_to_rank[pool[x]] = q * rpn + grp[x];
     }
     free(all); free(node_of); free(pool); free(grp);
     return ORC_OK;
+}
+
+int orc_place_correlated(const uint32_t *coact, int E, int G, int rpn, int32_t *expert_to_rank)
+{
+    return orc_place_correlated_capped(coact, E, G, rpn, -1.0, expert_to_rank);
 }
 
 /* One dispatched row: token t sent to rank dst, from source rank src. */

@@ -14,7 +14,7 @@ from conftest import ROOT
 
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_pins.py", "tests/test_oracle_brute.py", "tests/test_oracle_prereduce.py",
-        "tests/test_oracle_replicas.py", "tests/test_oracle_shuffle_balanced.py", "tests/test_oracle_ema.py"]
+        "tests/test_oracle_replicas.py", "tests/test_oracle_shuffle_balanced.py", "tests/test_oracle_ema.py", "tests/test_oracle_capped.py"]
 
 MUTANTS = {
     "counts_drop_diagonal": ("                for (int a = 0; a < k; ++a)\n                    for (int b = 0; b < k; ++b)\n"
@@ -66,6 +66,9 @@ MUTANTS = {
     "ema_weights_swapped": ("double a = alpha * x;\n            double b = (1.0 - alpha) * ema_in[c];",
                             "double a = (1.0 - alpha) * x;\n            double b = alpha * ema_in[c];"),
     "ema_first_batch_zero": ("            ema_out[c] = x;\n        }", "            ema_out[c] = 0.0 * x;\n        }"),
+    "capped_forced_pick_heaviest": ("if (pick < 0 || C[(size_t)pool[x] * E + pool[x]] < C[(size_t)pool[pick] * E + pool[pick]])",
+                                    "if (pick < 0 || C[(size_t)pool[x] * E + pool[x]] > C[(size_t)pool[pick] * E + pool[pick]])"),
+    "capped_cap_ignored": ("if (cap >= 0.0 && (double)(load + nx) > cap) continue;", "(void)nx;"),
 }
 
 
