@@ -65,7 +65,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="large_ep64")
-    ap.add_argument("--placement", default="correlated", choices=["correlated", "uniform", "capacity"])
+    ap.add_argument("--placement", default="correlated", choices=["correlated", "uniform", "capacity", "capped"],
+                    help="capped: correlated with every rank's load within 1.1 x the average")
     ap.add_argument("--no-shuffle", action="store_true")
     ap.add_argument("--balanced-shuffle", action="store_true",
                     help="cap every rank's shard at T/G tokens (capacity-balanced shuffle targets)")
@@ -189,6 +190,8 @@ def oracle_pass(w, ids, ids_cal, gates, x, placement, shuffle, balanced=False):
         e2r = [orc.place_correlated(cal["coact"][l], w.G, w.rpn) for l in range(L)]
     elif placement == "capacity":
         e2r = [orc.place_capacity(np.diag(cal["coact"][l]).astype(np.float64), w.G)[0] for l in range(L)]
+    elif placement == "capped":
+        e2r = [orc.place_correlated_capped(cal["coact"][l], w.G, w.rpn, 0.1) for l in range(L)]
     else:
         e2r = [orc.place_uniform(w.E, w.G) for _ in range(L)]
     rs = [orc.rank_score(cal["trans"][l], e2r[l + 1], w.G) for l in range(L - 1)] if shuffle else []
@@ -513,7 +516,7 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
     ids_cal = torch.from_numpy(make_routing(w, seed=seed + 1)).to(device)
     for G in w.sweep_G:
         row = {}
-        for placement in ("uniform", "correlated", "capacity"):
+        for placement in ("uniform", "correlated", "capped", "capacity"):
             sm, rl = pipeline.placement_effect(hp.ids, ids_cal, w.E, G, w.rpn, placement, loads=True)
             row[placement] = {"local_share": [round(int(r[2]) / int(r[4]), 5) for r in sm],
                               "V_per_token": [round(int(r[3]) / w.T, 4) for r in sm],

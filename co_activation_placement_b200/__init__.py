@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "moe_place_uniform": ([i, i, P], i),
             "moe_place_capacity": ([P, i, i, P, P], i),
             "moe_place_correlated": ([P, i, i, i, P], i),
+            "moe_place_correlated_capped": ([P, i, i, i, ctypes.c_double, P], i),
             "moe_place_replicas": ([P, i, i, i, P, i, P, P], i),
             "moe_assign_replicas": ([P, i, i, i, i, i, P, P, P, P, P, P, P], i),
             "moe_plan_dispatch_ranks": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
@@ -488,6 +489,16 @@ def place_correlated(coact_l, G: int, rpn: int) -> np.ndarray:
     E = c.shape[0]
     out = np.empty(E, np.int32)
     _check("moe_place_correlated", lib().moe_place_correlated(_np_ptr(c), E, G, rpn, _np_ptr(out)))
+    return out
+
+
+def place_correlated_capped(coact_l: np.ndarray, G: int, rpn: int, eps: float) -> np.ndarray:
+    """Correlated placement with load tolerance eps (eps < 0: none)."""
+    c = np.ascontiguousarray(coact_l, dtype=np.uint32)
+    E = c.shape[0]
+    out = np.empty(E, np.int32)
+    _check("moe_place_correlated_capped", lib().moe_place_correlated_capped(_np_ptr(c), E, G, rpn, float(eps),
+                                                                           _np_ptr(out)))
     return out
 
 

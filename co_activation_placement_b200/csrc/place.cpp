@@ -28,20 +28,25 @@ double ochiai64(const uint32_t *C, int E, int i, int j)
     return 0.0;
 }
 
-// Split `pool` (ascending expert ids) into m groups of pool.size()/m.
-std::vector<int> greedy_split(const uint32_t *C, int E, const std::vector<int> &pool, int m)
+// Split `pool` (ascending expert ids) into m groups of pool.size()/m.  With
+// cap >= 0 a group only admits experts that keep its load (sum of C_ee) at
+// most cap; when none does, the lightest unassigned expert joins (ties: lowest
+// id).  Running Ochiai sums per candidate, in the members' joining order.
+std::vector<int> greedy_split(const uint32_t *C, int E, const std::vector<int> &pool, int m, double cap)
 {
     const int n = (int)pool.size();
     const int size = n / m;
     std::vector<int> group(n, -1);
     std::vector<double> score(n);
+    auto load_of = [&](int x) { return (uint64_t)C[(size_t)pool[x] * E + pool[x]]; };
     for (int g = 0; g < m; ++g) {
         int seed = -1;
         for (int x = 0; x < n; ++x) {
             if (group[x] >= 0) continue;
-            if (seed < 0 || C[(size_t)pool[x] * E + pool[x]] > C[(size_t)pool[seed] * E + pool[seed]]) seed = x;
+            if (seed < 0 || load_of(x) > load_of(seed)) seed = x;
         }
         group[seed] = g;
+        uint64_t load = load_of(seed);
         for (int x = 0; x < n; ++x) score[x] = 0.0;
         int last = seed;
         for (int cnt = 1; cnt < size; ++cnt) {
@@ -49,13 +54,39 @@ std::vector<int> greedy_split(const uint32_t *C, int E, const std::vector<int> &
             for (int x = 0; x < n; ++x) {
                 if (group[x] >= 0) continue;
                 score[x] += ochiai64(C, E, pool[x], pool[last]);
+                if (cap >= 0.0 && (double)(load + load_of(x)) > cap) continue;
                 if (pick < 0 || score[x] > score[pick]) pick = x;
             }
+            if (pick < 0)
+                for (int x = 0; x < n; ++x)
+                    if (group[x] < 0 && (pick < 0 || load_of(x) < load_of(pick))) pick = x;
             group[pick] = g;
+            load += load_of(pick);
             last = pick;
         }
     }
     return group;
+}
+
+moe_status place_correlated(const uint32_t *coact, int E, int G, int rpn, double eps, int32_t *expert_to_rank)
+{
+    if (E < 1 || G < 1 || rpn < 1 || G % rpn != 0 || E % G != 0 || !coact || !expert_to_rank) return MOE_ERR_ARG;
+    const int nodes = G / rpn;
+    double W = 0.0;
+    for (int e = 0; e < E; ++e) W += (double)coact[(size_t)e * E + e];
+    const double cap_node = eps >= 0.0 ? (1.0 + eps) * W / nodes : -1.0;
+    const double cap_rank = eps >= 0.0 ? (1.0 + eps) * W / G : -1.0;
+    std::vector<int> all(E);
+    for (int e = 0; e < E; ++e) all[e] = e;
+    const std::vector<int> node_of = greedy_split(coact, E, all, nodes, cap_node);
+    for (int q = 0; q < nodes; ++q) {
+        std::vector<int> pool;
+        for (int e = 0; e < E; ++e)
+            if (node_of[e] == q) pool.push_back(e);
+        const std::vector<int> grp = greedy_split(coact, E, pool, rpn, cap_rank);
+        for (size_t x = 0; x < pool.size(); ++x) expert_to_rank[pool[x]] = q * rpn + grp[x];
+    }
+    return MOE_OK;
 }
 
 }  // namespace
@@ -99,19 +130,13 @@ extern "C" moe_status moe_place_capacity(const double *load, int E, int G, int32
 
 extern "C" moe_status moe_place_correlated(const uint32_t *coact, int E, int G, int rpn, int32_t *expert_to_rank)
 {
-    if (E < 1 || G < 1 || rpn < 1 || G % rpn != 0 || E % G != 0 || !coact || !expert_to_rank) return MOE_ERR_ARG;
-    const int nodes = G / rpn;
-    std::vector<int> all(E);
-    for (int e = 0; e < E; ++e) all[e] = e;
-    const std::vector<int> node_of = greedy_split(coact, E, all, nodes);
-    for (int q = 0; q < nodes; ++q) {
-        std::vector<int> pool;
-        for (int e = 0; e < E; ++e)
-            if (node_of[e] == q) pool.push_back(e);
-        const std::vector<int> grp = greedy_split(coact, E, pool, rpn);
-        for (size_t x = 0; x < pool.size(); ++x) expert_to_rank[pool[x]] = q * rpn + grp[x];
-    }
-    return MOE_OK;
+    return place_correlated(coact, E, G, rpn, -1.0, expert_to_rank);
+}
+
+extern "C" moe_status moe_place_correlated_capped(const uint32_t *coact, int E, int G, int rpn, double eps,
+                                                  int32_t *expert_to_rank)
+{
+    return place_correlated(coact, E, G, rpn, eps, expert_to_rank);
 }
 
 // Replica layout ("Cobalt", "Problem Formulation": every expert on at least one

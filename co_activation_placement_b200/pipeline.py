@@ -234,7 +234,7 @@ class HotPath:
 
 
 def calibrate(ids_cal: torch.Tensor, E: int, G: int, rpn: int, placement: str, shuffle: bool,
-              replica_extra: int = 0):
+              replica_extra: int = 0, load_tolerance: float = 0.1):
     """Placements and rank-score tables from a calibration batch (int32
     [L][T][k] on the device): its statistics come from moe_coact_stats, the
     placement from the host greedy, the tables from moe_rank_score.
@@ -250,11 +250,14 @@ def calibrate(ids_cal: torch.Tensor, E: int, G: int, rpn: int, placement: str, s
         e2r_h = [cap.place_uniform(E, G) for _ in range(L)]
     elif placement == "correlated":
         e2r_h = [cap.place_correlated(coact_h[l], G, rpn) for l in range(L)]
+    elif placement == "capped":
+        # correlated grouping with every rank's load within (1 + tolerance) x the average
+        e2r_h = [cap.place_correlated_capped(coact_h[l], G, rpn, load_tolerance) for l in range(L)]
     elif placement == "capacity":
         # first-fit decreasing on the calibration loads n_e = C_ee
         e2r_h = [cap.place_capacity(np.diag(coact_h[l]).astype(np.float64), G)[0] for l in range(L)]
     else:
-        raise ValueError("placement must be uniform, correlated or capacity")
+        raise ValueError("placement must be uniform, correlated, capped or capacity")
     e2r = [torch.from_numpy(a).to(ids_cal.device) for a in e2r_h]
     rs = []
     if shuffle:

@@ -385,6 +385,16 @@ moe_status moe_place_uniform(int E, int G, int32_t *expert_to_rank);
 moe_status moe_place_capacity(const double *load, int E, int G, int32_t *expert_to_rank, double *rank_load);
 moe_status moe_place_correlated(const uint32_t *coact, int E, int G, int rpn, int32_t *expert_to_rank);
 
+/* moe_place_correlated_capped ([CB] "Problem Formulation": a load tolerance on
+ *   every rank).  The correlated greedy above, where a node group only admits
+ *   experts that keep its load (sum of C_ee) at most (1+eps) W / (G/rpn) and a
+ *   rank group at most (1+eps) W / G, W = sum_e C_ee; when no unassigned
+ *   expert fits, the lightest one joins (ties: lowest id), so a group exceeds
+ *   its cap by less than one expert's load.  eps < 0: no cap (equals
+ *   moe_place_correlated). */
+moe_status moe_place_correlated_capped(const uint32_t *coact, int E, int G, int rpn, double eps,
+                                       int32_t *expert_to_rank);
+
 /* moe_place_replicas ([CB] "Problem Formulation": every expert has at least
  *   one replica, |P_r| <= (1+rho)E/G; "Two-Stage Expert Layout Planner":
  *   co-activated experts share nodes).  The page states the constraints, not

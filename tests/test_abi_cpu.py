@@ -140,3 +140,18 @@ def test_place_replicas_matches_oracle(cap, orc, E, G, rpn, extra):
     a = cap.place_replicas(C, G, rpn, e2r, extra)
     b = orc.place_replicas(C, G, rpn, e2r, extra)
     assert (a[0] == b[0]).all() and (a[1] == b[1]).all()
+
+
+@pytest.mark.parametrize("eps", [-1.0, 0.0, 0.1, 0.5])
+def test_place_correlated_capped_matches_oracle(cap, orc, eps):
+    from synth import WORKLOADS, make_routing
+    for name in ["one_node", "ep32"]:
+        w = WORKLOADS[name]
+        ids = make_routing(w, seed=1, T=min(w.T, 20000))
+        C = orc.coact(ids[:1], w.E, want=("coact",))["coact"][0]
+        assert (cap.place_correlated_capped(C, w.G, w.rpn, eps) == orc.place_correlated_capped(C, w.G, w.rpn, eps)).all()
+    rng = np.random.default_rng(3)
+    C = rng.integers(0, 1000, (256, 256)).astype(np.uint32)
+    C = np.triu(C, 1)
+    C = (C + C.T + np.diag(rng.integers(1000, 90000, 256))).astype(np.uint32)
+    assert (cap.place_correlated_capped(C, 64, 8, eps) == orc.place_correlated_capped(C, 64, 8, eps)).all()

@@ -370,22 +370,25 @@ def test_sweep_placement_effect_full_size(cap, G):
     assert got[0].tolist() == want.tolist()
 
 
+@pytest.mark.parametrize("placement", ["capacity", "capped"])
 @pytest.mark.parametrize("name", ["one_node", "ep32"])
-def test_pipeline_capacity_placement(cap, name):
+def test_pipeline_capacity_placement(cap, name, placement):
     """The step under the capacity-aware placement (first-fit decreasing on the
-    calibration loads): placements and plans against the oracle."""
+    calibration loads) and under the correlated placement with a 10% load
+    tolerance: placements and plans against the oracle."""
     from co_activation_placement_b200 import pipeline
     w = WORKLOADS[name]
     ids = make_routing(w)
     ids_cal = make_routing(w, seed=w.seed + 1)
     hp = pipeline.prepare(w.E, w.G, w.rpn, ids, make_gates(w), make_hidden(w), w.dtype, ids_cal,
-                          placement="capacity", shuffle=False, out_dtype=torch.float32)
+                          placement=placement, shuffle=False, out_dtype=torch.float32)
     hp.step()
     torch.cuda.synchronize()
     assert int(host(hp.err)[0]) == 0
     oc = orc.coact(ids_cal, w.E, want=("coact",))["coact"]
     for l in range(w.L):
-        e2r = orc.place_capacity(np.diag(oc[l]).astype(np.float64), w.G)[0]
+        e2r = orc.place_capacity(np.diag(oc[l]).astype(np.float64), w.G)[0] if placement == "capacity" \
+            else orc.place_correlated_capped(oc[l], w.G, w.rpn, 0.1)
         assert (host(hp.e2r[l]) == e2r).all()
         op = orc.plan(ids[l], w.E, w.G, w.rpn, e2r)
         assert host(hp.plans[l].summary).tolist() == op["summary"].tolist()
