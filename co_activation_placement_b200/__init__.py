@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
             "moe_coact_stats_method": ([i], i),
             "moe_coact_stats_path": ([i, i, i, i, i], i),
             "moe_coact_ema": ([P, i, i, ctypes.c_double, P, P, P, P], i),
+            "moe_selftest_workspace": ([], sz),
+            "moe_selftest_wait_timeout": ([i, P, P, sz, P], i),
             "moe_coact_stats": ([P, i, i, i, i, P, P, P, P, P, sz, P], i),
             "moe_plan_dispatch_workspace": ([i, i, i, i], sz),
             "moe_plan_dispatch": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
@@ -200,6 +202,18 @@ def coact_ema(coact: torch.Tensor, alpha: float, ema_in: Optional[torch.Tensor] 
                              _stream(coact))
     _check("moe_coact_ema", st)
     return ema_out, ochiai
+
+
+def selftest_wait_timeout(kind: int, device="cuda") -> torch.Tensor:
+    """Make one kind of bounded device wait run out on purpose (0: a grid
+    barrier one block never reaches; 1: an mbarrier phase nothing completes);
+    returns the error word (device int32 [1]), MOE_DERR_TIMEOUT when the wait
+    gave up as designed."""
+    err = new_err(device)
+    ws = torch.empty(max(int(lib().moe_selftest_workspace()), 1), dtype=torch.uint8, device=device)
+    _check("moe_selftest_wait_timeout", lib().moe_selftest_wait_timeout(int(kind), _ptr(err), _ptr(ws), ws.numel(),
+                                                                        _stream(err)))
+    return err
 
 
 # ---------------------------------------------------------------- dispatch plan

@@ -37,6 +37,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "waits.cuh"
 
 namespace moe {
 namespace {
@@ -45,15 +46,12 @@ constexpr int kBalThreads = 512;
 constexpr int kBalWarps = kBalThreads / 32;
 constexpr int kKeyShift = 28;
 constexpr unsigned long long kTokMask = (1ull << kKeyShift) - 1;
-constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr int kScratchKeys = 4096;          // boundary-bin scratch of the selection (32 KB)
 
 struct BalHeader {            // cleared before every launch
-    unsigned int bar_count;
-    unsigned int bar_gen;
-    unsigned int abort;
+    GridBarrier bar;
     int nfree[2];             // free tokens for the round of that parity
-    int pad;
+    int pad[2];
     long long proposals;
     int cnt[2][64];           // proposals per rank, round parity
     unsigned long long theta[64];   // weakest holder's key of a full rank; 0 while it has room
@@ -95,59 +93,6 @@ struct BalArgs {
     int32_t *err;
 };
 
-__device__ __forceinline__ unsigned long long globaltimer()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ unsigned int ld_acquire(const unsigned int *p)
-{
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release(unsigned int *p, unsigned int v)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Grid-wide barrier with a bounded wait.  Returns false (in every thread of
-// the block) when the wait ran out or another block aborted.
-__device__ bool grid_sync(BalHeader *h, int32_t *err)
-{
-    __shared__ int ok_s;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int ok = 1;
-        const unsigned int gen = ld_acquire(&h->bar_gen);
-        __threadfence();
-        if (atomicAdd(&h->bar_count, 1u) + 1 == gridDim.x) {
-            atomicExch(&h->bar_count, 0u);
-            __threadfence();
-            st_release(&h->bar_gen, gen + 1);
-        } else {
-            const unsigned long long t0 = globaltimer();
-            while (ld_acquire(&h->bar_gen) == gen) {
-                if (ld_acquire(&h->abort)) { ok = 0; break; }
-                if (globaltimer() - t0 > kWaitNs) {
-                    record_error(err, MOE_DERR_TIMEOUT);
-                    atomicExch(&h->abort, 1u);
-                    ok = 0;
-                    break;
-                }
-                __nanosleep(64);
-            }
-        }
-        __threadfence();
-        ok_s = ok;
-    }
-    __syncthreads();
-    return ok_s != 0;
-}
-
 __device__ __forceinline__ unsigned long long block_min(unsigned long long v, unsigned long long *red)
 {
 #pragma unroll
@@ -188,10 +133,10 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
     // time in each phase (info[2..5]): proposing and waiting at barriers as
     // block 0 sees them, gathering and selecting as the slowest block's total
     const bool clk = a.info && tid == 0;
-    unsigned long long t_a = 0, t_b = 0, t_c = 0, t_w = 0, t_mark = clk ? globaltimer() : 0;
+    unsigned long long t_a = 0, t_b = 0, t_c = 0, t_w = 0, t_mark = clk ? gtimer_ns() : 0;
     auto lap = [&](unsigned long long &acc) {
         if (clk) {
-            const unsigned long long now = globaltimer();
+            const unsigned long long now = gtimer_ns();
             acc += now - t_mark;
             t_mark = now;
         }
@@ -287,7 +232,7 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
             if (mine) {
                 if (my_key == 0) {            // no rank can take it: impossible while T <= G*capacity
                     record_error(a.err, MOE_DERR_RANK_RANGE);
-                    atomicExch(&h->abort, 1u);
+                    atomicExch(&h->bar.abort, 1u);
                     my_r = 0;
                 }
                 __stcg(a.prop_r + i, my_r);
@@ -298,7 +243,7 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
         __syncthreads();
         if (tid < G && cnt_s[tid]) atomicAdd(&h->cnt[p][tid], cnt_s[tid]);
         lap(t_a);
-        if (!grid_sync(h, a.err)) return;
+        if (!grid_barrier(&h->bar, a.err)) return;
         lap(t_w);
 
         // proposals per rank and their exclusive prefix (a rank's segment of
@@ -524,7 +469,7 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
             if (tid == 0) {
                 if (kept_s != Cc) {           // impossible: keys are distinct
                     record_error(a.err, MOE_DERR_ROW_RANGE);
-                    atomicExch(&h->abort, 1u);
+                    atomicExch(&h->bar.abort, 1u);
                 }
                 hn_s[r] = Cc;
                 hsel_s[r] = sel ^ 1;
@@ -534,7 +479,7 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
             __syncthreads();
         }
         lap(t_c);
-        if (!grid_sync(h, a.err) || __ldcg(&h->abort)) return;
+        if (!grid_barrier(&h->bar, a.err) || __ldcg(&h->bar.abort)) return;
         lap(t_w);
         if (__ldcg(&h->nfree[pn]) == 0) break;
         if (rd + 1 >= round_limit) {           // cannot happen: each round is a new rank for every free token

@@ -33,6 +33,7 @@
 
 #include "common.cuh"
 #include "stats_mma.cuh"
+#include "waits.cuh"
 
 namespace moe {
 namespace {
@@ -42,44 +43,7 @@ constexpr int kMmaWarp = kBuildThreads / 32;   // warp 8 issues the MMAs
 constexpr int kMmaThreads = kBuildThreads + 32;
 constexpr int kTok = 128;                 // tokens per stage
 constexpr int kStages = 3;
-constexpr unsigned long long kMmaWaitNs = 2000000000ull;
 constexpr int kMmaReduceThreads = 256;
-
-__device__ __forceinline__ unsigned long long mma_now()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-// true once the phase with the given parity has completed; false after 2 s
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
-{
-    const uint32_t a = smem_u32(bar);
-    const unsigned long long t0 = mma_now();
-    for (;;) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(a), "r"(parity)
-            : "memory");
-        if (done) return true;
-        if (mma_now() - t0 > kMmaWaitNs) return false;
-    }
-}
 
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle
 // layout: rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte
@@ -109,15 +73,10 @@ __device__ __forceinline__ void mma_u8(uint32_t tmem_d, uint64_t da, uint64_t db
         : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 __device__ __forceinline__ void mma_commit(uint64_t *bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 ::"r"(smem_u32(bar)) : "memory");
+                 ::"r"(smem_addr(bar)) : "memory");
 }
 
 // Token t's K ids: 16-byte loads when K % 4 == 0, 8-byte when K % 2 == 0
@@ -210,7 +169,7 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
     }
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(&tmem_base_s)), "r"((uint32_t)G.cols) : "memory");
+                     ::"r"(smem_addr(&tmem_base_s)), "r"((uint32_t)G.cols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -294,7 +253,7 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
         // ---- MMA warp: per full stage, one lane issues K / 32 x M tiles MMAs
         // into each accumulator and commits them to the stage's empty barrier
         const uint32_t idesc = (2u << 4) | ((uint32_t)(E >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-        const uint32_t base = smem_u32(sm);
+        const uint32_t base = smem_addr(sm);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages, n = c / kStages;
             if (!mbar_wait(&full_bar[s], n & 1)) { ok = false; break; }

@@ -409,6 +409,18 @@ moe_status moe_place_correlated_capped(const uint32_t *coact, int E, int G, int 
 moe_status moe_place_replicas(const uint32_t *coact, int E, int G, int rpn, const int32_t *expert_to_rank,
                               int extra, int32_t *replica_rank, int32_t *n_rep);
 
+/* ------------------------------------------------------------------------
+ * moe_selftest_wait_timeout (no counterpart on the pages: a test of the error
+ *   path of the bounded device waits).  kind 0: a cooperative launch of 4
+ *   blocks meets at a grid barrier that block 1 never reaches; kind 1: one
+ *   block waits on an mbarrier phase that nothing completes.  Either way the
+ *   waits give up after about 2 s, err receives MOE_DERR_TIMEOUT and the
+ *   kernel returns; nothing faults and the context stays usable.  ws:
+ *   moe_selftest_workspace() bytes, 256-byte aligned (kind 0 only).
+ * ---------------------------------------------------------------------- */
+size_t moe_selftest_workspace(void);
+moe_status moe_selftest_wait_timeout(int kind, int32_t *err, void *ws, size_t ws_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
