@@ -38,8 +38,13 @@
  *    caller zeroes `err` and reads it after synchronising.  When it is
  *    non-zero the outputs of that call are unspecified.  Kernels never trap.
  *  - Calls keep no state between invocations except the global launch
- *    counter below.  Workspace ("ws") is caller-provided device memory of at
- *    least the size the matching *_workspace query returns, 256-byte aligned.
+ *    counter, the statistics method setting (moe_coact_stats_method) and the
+ *    static scratch of moe_plan_dispatch_static.  Workspace ("ws") is
+ *    caller-provided device memory of at least the size the matching
+ *    *_workspace query returns, 256-byte aligned.
+ *  - The only kernels that wait on other blocks or on the tensor cores
+ *    (moe_shuffle_balanced, the tensor-core method of moe_coact_stats) give
+ *    every wait a 2 s limit and then report MOE_DERR_TIMEOUT in `err`.
  */
 #ifndef MOE_COACT_H
 #define MOE_COACT_H
