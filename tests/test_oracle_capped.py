@@ -1,6 +1,6 @@
 """Pins for the load-capped correlated placement ("Cobalt", "Problem
 Formulation": every rank's load within a tolerance of the average; the
-grouping itself is this build's greedy).  eps < 0 and a huge eps reduce to the
+grouping itself is a greedy of our own reading).  eps < 0 and a huge eps reduce to the
 plain correlated greedy; a hand-worked case; the pure-Python restatement; a
 group overshoots its cap by less than one expert's load."""
 import numpy as np
