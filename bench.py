@@ -74,6 +74,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of one CUDA graph")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="run plans, shuffle targets and statistics in line instead of on a second stream")
     ap.add_argument("--replicas", type=int, default=0, metavar="EXTRA",
                     help="replicate experts (EXTRA more per rank) and assign tasks to the fewest remote nodes")
     ap.add_argument("--prereduce", action="store_true",
@@ -347,7 +349,8 @@ def main():
     hp = pipeline.prepare(w.E, w.G, w.rpn, ids, gates, x, w.dtype, ids_cal, placement=a.placement,
                           shuffle=shuffle, out_dtype=out_dtype, device=device, timers=True,
                           scales=make_expert_scales(w, seed=seed) if a.prereduce else None,
-                          replica_extra=a.replicas, shuffle_capacity=w.T // w.G if balanced else 0)
+                          replica_extra=a.replicas, shuffle_capacity=w.T // w.G if balanced else 0,
+                          overlap=not a.no_overlap)
 
     def barrier():
         if pg is not None:
@@ -453,6 +456,8 @@ def main():
                        "combine": "receiver-side pre-reduced (stand-in experts)" if a.prereduce
                                   else "source-side weighted (identity experts)",
                        "replicas_per_rank": a.replicas,
+                       "overlap": "plans, shuffle targets and statistics on a second stream"
+                                  if not a.no_overlap else "none",
                        "shuffle": ("balanced (T/G tokens per rank)" if balanced else True) if shuffle else False,
                        "parallelism": "replicas (weak scaling, one batch per GPU)",
                        "l2": "inputs larger than L2 (x %.2f GB per GPU; no flush)" % (x.nbytes / 1e9)},
@@ -474,6 +479,10 @@ def main():
             "e2e": e2e,
             "gpu_launches": int(n_launch),
             "gpu_launches_per_step": n_launch / a.steps,
+            "kernel_times": "CUDA events around each library call on its stream; plans, shuffle targets and "
+                            "statistics run on a second stream beside the row traffic, so their times include "
+                            "waiting for SM slots and the kernel times add up to more than the step"
+                            if not a.no_overlap else "CUDA events around each library call",
             "timing": "one CUDA graph of the %d steps" % a.steps if graph is not None else
                       ("eager launches" + ("; " + graph_note if graph_note else "")),
             "cpu_baseline": cpu,

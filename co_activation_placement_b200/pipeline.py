@@ -66,6 +66,7 @@ class HotPath:
     scales: List[torch.Tensor] = field(default_factory=list)   # f32 [E] per layer (prereduce)
     replicas: list = field(default_factory=list)   # per layer (replica_rank [E][1+nodes], n_rep [E]) or empty
     shuffle_capacity: int = 0          # > 0: at most this many tokens per rank (moe_shuffle_balanced)
+    overlap: bool = True               # control work on a second stream beside the row traffic
     # buffers
     stats: dict = field(default_factory=dict)
     plans: List[cap.Plan] = field(default_factory=list)
@@ -99,6 +100,11 @@ class HotPath:
                                           dtype=torch.uint8, device=dev)
             # rounds and proposals of each balanced shuffle
             self.shuffle_info = torch.zeros((max(L - 1, 1), 6), dtype=torch.int64, device=dev)
+        if self.overlap:
+            self.side = torch.cuda.Stream(device=dev)
+            self.fork_ev = torch.cuda.Event()
+            self.join_ev = torch.cuda.Event()
+            self.plan_ev = [torch.cuda.Event() for _ in range(L)]
         if self.replicas:
             self.pick_rank = torch.empty((T, k), dtype=torch.int32, device=dev)
             self.n_remote = torch.empty(T, dtype=torch.int32, device=dev)
@@ -110,73 +116,105 @@ class HotPath:
             self.y = torch.empty((T * k, d), dtype=self.x.dtype, device=dev)
 
     # ------------------------------------------------------------------ step
-    def _mark(self, name):
-        if self.timers:
-            # external: inside a captured graph this is a real event-record node
-            ev = torch.cuda.Event(enable_timing=True, external=True)
-            ev.record()
-            self.events.append((name, ev))
+    def _call(self, name, fn):
+        """Run one library call on torch's current stream inside an NVTX range
+        (visible in Nsight timelines), bracketed by timing events when timers
+        are on (external events: inside a captured graph they are real
+        event-record nodes)."""
+        with torch.cuda.nvtx.range("moe_" + name):
+            if self.timers:
+                a = torch.cuda.Event(enable_timing=True, external=True)
+                a.record()
+            out = fn()
+            if self.timers:
+                b = torch.cuda.Event(enable_timing=True, external=True)
+                b.record()
+                self.events.append((name, a, b))
+        return out
 
     def reset_events(self):
         self.events = []
 
-    def step(self):
-        nv = torch.cuda.nvtx.range   # one NVTX range per library call (Nsight timelines)
-        self._mark("start")
-        with nv("moe_coact_stats"):
-            cap.coact_stats(self.ids, self.E, coact=self.stats["coact"], ochiai=self.stats["ochiai"],
-                            trans=self.stats["trans"], err=self.err, ws=self.stats_ws)
-        self._mark("stats")
-        if not self.rows:
+    # the parts of a step
+    def _stats(self):
+        self._call("stats", lambda: cap.coact_stats(self.ids, self.E, coact=self.stats["coact"],
+                                                     ochiai=self.stats["ochiai"], trans=self.stats["trans"],
+                                                     err=self.err, ws=self.stats_ws))
+
+    def _plan(self, l):
+        src = self.targets[l - 1] if (self.shuffle and l > 0) else None
+        if self.replicas:
+            # each task to a replica of its expert: fewest remote nodes per token
+            rr, nr = self.replicas[l]
+
+            def go():
+                cap.assign_replicas(self.ids[l], self.E, self.G, self.rpn, rr, nr, src_rank=src,
+                                    pick_rank=self.pick_rank, n_remote=self.n_remote, err=self.err)
+                cap.plan_dispatch_ranks(self.ids[l], self.E, self.G, self.rpn, self.pick_rank, src_rank=src,
+                                        plan=self.plans[l], ws=self.plan_ws)
+            self._call("plan", go)
+        else:
+            self._call("plan", lambda: cap.plan_dispatch(self.ids[l], self.E, self.G, self.rpn, self.e2r[l],
+                                                         src_rank=src, plan=self.plans[l], ws=self.plan_ws))
+
+    def _rows(self, l):
+        p = self.plans[l]
+        self._call("permute", lambda: cap.permute(self.x, p.row_of, p.R_max, send=self.send, err=self.err))
+        if self.prereduce:
+            # gates travel with the rows; the receiving rank applies its
+            # experts and returns one row per (token, rank); the source sums
+            self._call("gates", lambda: cap.dispatch_gates(self.ids[l], self.gates[l], p, send_e=self.send_e,
+                                                           send_w=self.send_w, err=self.err))
+            self._call("reduce", lambda: cap.expert_reduce(self.send, p.summary, self.send_e, self.send_w,
+                                                           self.scales[l], y=self.y, err=self.err))
+            self._call("combine", lambda: cap.combine_rows(self.y, p.row_of, out=self.outs[l], err=self.err))
+        else:
+            self._call("combine", lambda: cap.combine(self.send, p.row_of, self.gates[l], out=self.outs[l],
+                                                      err=self.err))
+
+    def _shuffle(self, l):
+        if not (self.shuffle and l + 1 < self.L):
             return
+        if self.shuffle_capacity > 0:
+            self._call("shuffle", lambda: cap.shuffle_balanced(self.ids[l], self.E, self.G, self.rank_scores[l],
+                                                               self.shuffle_capacity, target=self.targets[l],
+                                                               info=self.shuffle_info[l], err=self.err,
+                                                               ws=self.shuffle_ws))
+        else:
+            self._call("shuffle", lambda: cap.shuffle_targets(self.ids[l], self.E, self.G, self.rank_scores[l],
+                                                              target=self.targets[l], err=self.err))
+
+    def step(self):
+        """One step.  With overlap, the control work -- plans, shuffle targets
+        and statistics, which read only routing ids and tables -- runs on a
+        second stream that starts when everything before the step is done and
+        keeps ahead of the row traffic; the permute and combine of layer l wait
+        only for layer l's plan."""
+        if not self.rows:
+            self._stats()
+            return
+        if not self.overlap:
+            self._stats()
+            for l in range(self.L):
+                self._plan(l)
+                self._rows(l)
+                self._shuffle(l)
+            return
+        main = torch.cuda.current_stream(self.ids.device)
+        self.fork_ev.record(main)
+        self.side.wait_event(self.fork_ev)
+        with torch.cuda.stream(self.side):
+            for l in range(self.L):
+                self._plan(l)
+                self.plan_ev[l].record(self.side)
+                if l == 0:
+                    self._stats()
+                self._shuffle(l)
+            self.join_ev.record(self.side)
         for l in range(self.L):
-            src = self.targets[l - 1] if (self.shuffle and l > 0) else None
-            if self.replicas:
-                # each task to a replica of its expert: fewest remote nodes per token
-                rr, nr = self.replicas[l]
-                with nv("moe_assign_replicas"):
-                    cap.assign_replicas(self.ids[l], self.E, self.G, self.rpn, rr, nr, src_rank=src,
-                                        pick_rank=self.pick_rank, n_remote=self.n_remote, err=self.err)
-                with nv("moe_plan_dispatch_ranks"):
-                    p = cap.plan_dispatch_ranks(self.ids[l], self.E, self.G, self.rpn, self.pick_rank,
-                                                src_rank=src, plan=self.plans[l], ws=self.plan_ws)
-            else:
-                with nv("moe_plan_dispatch"):
-                    p = cap.plan_dispatch(self.ids[l], self.E, self.G, self.rpn, self.e2r[l], src_rank=src,
-                                          plan=self.plans[l], ws=self.plan_ws)
-            self._mark("plan")
-            with nv("moe_permute"):
-                cap.permute(self.x, p.row_of, p.R_max, send=self.send, err=self.err)
-            self._mark("permute")
-            if self.prereduce:
-                # gates travel with the rows; the receiving rank applies its
-                # experts and returns one row per (token, rank); the source sums
-                with nv("moe_dispatch_gates"):
-                    cap.dispatch_gates(self.ids[l], self.gates[l], p, send_e=self.send_e, send_w=self.send_w,
-                                       err=self.err)
-                self._mark("gates")
-                with nv("moe_expert_reduce"):
-                    cap.expert_reduce(self.send, p.summary, self.send_e, self.send_w, self.scales[l], y=self.y,
-                                      err=self.err)
-                self._mark("reduce")
-                with nv("moe_combine_rows"):
-                    cap.combine_rows(self.y, p.row_of, out=self.outs[l], err=self.err)
-                self._mark("combine")
-            else:
-                with nv("moe_combine"):
-                    cap.combine(self.send, p.row_of, self.gates[l], out=self.outs[l], err=self.err)
-                self._mark("combine")
-            if self.shuffle and l + 1 < self.L:
-                if self.shuffle_capacity > 0:
-                    with nv("moe_shuffle_balanced"):
-                        cap.shuffle_balanced(self.ids[l], self.E, self.G, self.rank_scores[l], self.shuffle_capacity,
-                                             target=self.targets[l], info=self.shuffle_info[l], err=self.err,
-                                             ws=self.shuffle_ws)
-                else:
-                    with nv("moe_shuffle_targets"):
-                        cap.shuffle_targets(self.ids[l], self.E, self.G, self.rank_scores[l],
-                                            target=self.targets[l], err=self.err)
-                self._mark("shuffle")
+            main.wait_event(self.plan_ev[l])
+            self._rows(l)
+        main.wait_event(self.join_ev)
 
     def capture(self, n_steps: int) -> torch.cuda.CUDAGraph:
         """Capture n_steps consecutive steps into one CUDA graph.  The library
@@ -193,11 +231,12 @@ class HotPath:
 
     def kernel_times_ms(self):
         """Device time (ms) of each kind of call, summed over all steps run
-        since reset_events() (call after synchronising)."""
+        since reset_events() (call after synchronising).  With overlap the
+        control calls run beside the row traffic, so the times add up to more
+        than the step."""
         out = {}
-        for (a, ea), (b, eb) in zip(self.events, self.events[1:]):
-            if b != "start":
-                out[b] = out.get(b, 0.0) + ea.elapsed_time(eb)
+        for name, a, b in self.events:
+            out[name] = out.get(name, 0.0) + a.elapsed_time(b)
         return out
 
     # ------------------------------------------------------------------ bytes
@@ -274,7 +313,8 @@ def calibrate(ids_cal: torch.Tensor, E: int, G: int, rpn: int, placement: str, s
 def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarray], x: Optional[np.ndarray],
             x_dtype: str, ids_cal: np.ndarray, placement: str = "correlated", shuffle: bool = True,
             out_dtype=torch.bfloat16, device="cuda", rows: bool = True, timers: bool = False,
-            scales: Optional[np.ndarray] = None, replica_extra: int = 0, shuffle_capacity: int = 0) -> HotPath:
+            scales: Optional[np.ndarray] = None, replica_extra: int = 0, shuffle_capacity: int = 0,
+            overlap: bool = True) -> HotPath:
     """Upload a batch (host numpy arrays; x as float32 or bf16 bit patterns)
     and its calibration batch, calibrate, and return the step's HotPath."""
     dev = torch.device(device)
@@ -291,7 +331,7 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
         if scales is not None else []
     return HotPath(E=E, G=G, rpn=rpn, ids=ids_d, gates=gates_d, x=x_d, e2r=e2r, rank_scores=rs,
                    out_dtype=out_dtype, rows=rows, timers=timers, prereduce=scales is not None, scales=scales_d,
-                   replicas=reps, shuffle_capacity=shuffle_capacity)
+                   replicas=reps, shuffle_capacity=shuffle_capacity, overlap=overlap)
 
 
 def placement_effect(ids: torch.Tensor, ids_cal: torch.Tensor, E: int, G: int, rpn: int,

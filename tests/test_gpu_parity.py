@@ -393,3 +393,31 @@ def test_pipeline_capacity_placement(cap, name, placement):
         op = orc.plan(ids[l], w.E, w.G, w.rpn, e2r)
         assert host(hp.plans[l].summary).tolist() == op["summary"].tolist()
         assert (host(hp.plans[l].row_of)[: w.T] == op["row_of"]).all()
+
+
+@pytest.mark.parametrize("name", ["ep32", "large_ep64"])
+def test_overlapped_step_equals_serial_step(cap, name):
+    """The step with the control work on a second stream produces every
+    output bit for bit as the step run in line, also when replayed from a
+    CUDA graph."""
+    from co_activation_placement_b200 import pipeline
+    w = WORKLOADS[name]
+    ids = make_routing(w)
+    ids_cal = make_routing(w, seed=w.seed + 1)
+    gates, x = make_gates(w), make_hidden(w)
+    outs = {}
+    for overlap in (False, True):
+        hp = pipeline.prepare(w.E, w.G, w.rpn, ids, gates, x, w.dtype, ids_cal, out_dtype=torch.float32,
+                              overlap=overlap)
+        hp.step()
+        g = hp.capture(2)
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(host(hp.err)[0]) == 0
+        outs[overlap] = ([host(p.row_of).copy() for p in hp.plans] + [host(p.summary).copy() for p in hp.plans]
+                         + [host(t).copy() for t in hp.targets] + [host(hp.stats["coact"]).copy()]
+                         + [host(o).copy() for o in hp.outs])
+        del g, hp
+        torch.cuda.empty_cache()
+    for a, b in zip(outs[False], outs[True]):
+        assert (a.view(np.uint8) == b.view(np.uint8)).all()
