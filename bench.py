@@ -457,7 +457,7 @@ def main():
                                   else "source-side weighted (identity experts)",
                        "replicas_per_rank": a.replicas,
                        "overlap": "plans, shuffle targets and statistics on a second stream"
-                                  if not a.no_overlap else "none",
+                                  if hp.overlap else "none",
                        "shuffle": ("balanced (T/G tokens per rank)" if balanced else True) if shuffle else False,
                        "parallelism": "replicas (weak scaling, one batch per GPU)",
                        "l2": "inputs larger than L2 (x %.2f GB per GPU; no flush)" % (x.nbytes / 1e9)},
@@ -482,7 +482,7 @@ def main():
             "kernel_times": "CUDA events around each library call on its stream; plans, shuffle targets and "
                             "statistics run on a second stream beside the row traffic, so their times include "
                             "waiting for SM slots and the kernel times add up to more than the step"
-                            if not a.no_overlap else "CUDA events around each library call",
+                            if hp.overlap else "CUDA events around each library call",
             "timing": "one CUDA graph of the %d steps" % a.steps if graph is not None else
                       ("eager launches" + ("; " + graph_note if graph_note else "")),
             "cpu_baseline": cpu,

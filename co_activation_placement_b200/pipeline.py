@@ -100,6 +100,10 @@ class HotPath:
                                           dtype=torch.uint8, device=dev)
             # rounds and proposals of each balanced shuffle
             self.shuffle_info = torch.zeros((max(L - 1, 1), 6), dtype=torch.int64, device=dev)
+        if self.shuffle and self.shuffle_capacity > 0:
+            # the balanced shuffle is one cooperative launch over every SM:
+            # beside the row kernels it would slow them and itself
+            self.overlap = False
         if self.overlap:
             self.side = torch.cuda.Stream(device=dev)
             self.fork_ev = torch.cuda.Event()
