@@ -432,7 +432,9 @@ def main():
 
     # co-activation tokens/s on this step and on the statistics sweep
     stats_ms = kern["stats"]["ms_per_step"]
-    coact_tps = world * w.L * w.T / (stats_ms * 1e-3)
+    # in line only: with the overlap the statistics share the SMs with the
+    # row kernels and their event time is not their own (the sweep times them alone)
+    coact_tps = None if hp.overlap else world * w.L * w.T / (stats_ms * 1e-3)
     sweep = None
     if not a.no_sweep:
         sweep = run_sweep(cap, pipeline, device, seed, a.steps, a.warmup, hbm, pg)
@@ -465,6 +467,8 @@ def main():
             "roofline": roofline,
             "kernels": kern,
             "coact_tokens_per_s": coact_tps,
+            "coact_tokens_per_s_source": "the statistics sweep (coact_sweep.tokens_per_s) times the statistics alone"
+                                         if hp.overlap else "this step's statistics call",
             "coact_sweep": sweep,
             "rows": {"R": R, "T_k": w.T * w.k, "dedup_removed": [1 - r / (w.T * w.k) for r in R],
                      "R_remote": [int(s[1]) for s in summaries],
