@@ -1,13 +1,17 @@
 """Benchmark of the co-activation / deduplicated-dispatch hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--placement correlated|uniform] [--no-shuffle]
+                    [--placement correlated|uniform|capacity|capped] [--no-shuffle]
+                    [--balanced-shuffle] [--prereduce] [--replicas N]
+                    [--coact-method auto|histogram|tensor] [--no-overlap] [--no-graph]
                     [--out-dtype f32|bf16] [--impl reference]
 
 A step is one pass of the whole path over one batch: co-activation counts,
 Ochiai and transitions for every layer, then per layer the dispatch plan, the
 row permute, identity experts, the weighted combine and the shuffle targets
-for the next layer.  The default workload is large EP64 (T=131072, E=256, k=8,
+for the next layer.  Plans, shuffle targets and statistics run on a second
+stream beside the row traffic (--no-overlap: in line); the timed steps are
+replayed from one CUDA graph (--no-graph: eager launches).  The default workload is large EP64 (T=131072, E=256, k=8,
 G=64 in 8 nodes, d=7168 bf16, 4 layers), the largest workload with hidden
 states; its inputs (x = 1.88 GB) exceed the 126 MB L2, so no flush is needed
 between steps.  With N GPUs each rank runs its own batch (seed + rank): weak
