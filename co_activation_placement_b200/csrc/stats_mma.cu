@@ -154,7 +154,13 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
     const int tile = rows * kTok;                      // bytes per X tile
     // stage s: tile A at s * per_stage, tile B right after it (M products)
     const int per_stage = has_m ? 2 * tile : tile;
-    const uint32_t m_off = has_c ? (uint32_t)(G.mt * E) : 0u;   // TMEM column of the M accumulator
+    // C_l and M_l in one MMA: tile B (X_{l+1}) follows tile A (X_l), so the
+    // 2*rows rows from tile A on are one N = 2*rows operand [X_l; X_{l+1}]
+    // (single 128-row tile, rows <= 128); D's columns [0, rows) are C_l's,
+    // [rows, 2 rows) M_l's
+    const bool stacked = has_c && has_m && G.mt == 1;
+    // TMEM column of the M accumulator
+    const uint32_t m_off = stacked ? (uint32_t)rows : (has_c ? (uint32_t)(G.mt * E) : 0u);
 
     // zero the tiles once; later stages only set and clear their own ones
     for (int i = tid * 16; i < kStages * per_stage; i += kMmaThreads * 16)
@@ -253,6 +259,7 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
         // ---- MMA warp: per full stage, one lane issues K / 32 x M tiles MMAs
         // into each accumulator and commits them to the stage's empty barrier
         const uint32_t idesc = (2u << 4) | ((uint32_t)(E >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+        const uint32_t idesc2 = (2u << 4) | ((uint32_t)((2 * rows) >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
         const uint32_t base = smem_addr(sm);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages, n = c / kStages;
@@ -269,8 +276,12 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
                     const uint64_t dB = smem_desc_sw128(b0 + koff);
                     for (int mi = 0; mi < G.mt; ++mi) {
                         const uint64_t da = smem_desc_sw128(a0 + koff + (uint32_t)(mi * 128 * 128));
-                        if (has_c) mma_u8(tmem + (uint32_t)(mi * E), da, dA, idesc, acc);
-                        if (has_m) mma_u8(tmem + m_off + (uint32_t)(mi * E), da, dB, idesc, acc);
+                        if (stacked) {
+                            mma_u8(tmem, da, dA, idesc2, acc);
+                        } else {
+                            if (has_c) mma_u8(tmem + (uint32_t)(mi * E), da, dA, idesc, acc);
+                            if (has_m) mma_u8(tmem + m_off + (uint32_t)(mi * E), da, dB, idesc, acc);
+                        }
                     }
                 }
                 mma_commit(&empty_bar[s]);
@@ -399,7 +410,9 @@ bool make_mma_geom(int L, int T, int k, int E, bool want_c, bool want_t, MmaGeom
     // C_l and M_l share layer l's tile when both accumulators fit tensor memory
     g.paired = g.nc > 0 && nm > 0 && 2 * g.mt * E <= 512;
     g.J = g.paired ? L : g.P;
-    const int acc_cols = (g.paired ? 2 : 1) * g.mt * E;
+    // paired implies one 128-row tile (2 * mt * E <= 512); its C and M share one
+    // N = 2 * rows accumulator
+    const int acc_cols = g.paired ? 2 * g.rows : g.mt * E;
     int cols = 32;
     while (cols < acc_cols) cols <<= 1;
     g.cols = cols;
