@@ -62,6 +62,7 @@ def combine_bound(Yf, idx, w, k, out_bf16, ref):
 STATS_SHAPES = [  # L, T, k, E
     (1, 1, 1, 4), (2, 1000, 2, 8), (3, 4097, 3, 16), (2, 300, 8, 8), (2, 5000, 6, 64),
     (2, 3333, 8, 128), (3, 2500, 8, 256), (2, 777, 5, 1000), (1, 12345, 4, 32),
+    (2, 1500, 8, 1024),                                   # the largest E the call accepts
 ]
 
 
@@ -108,6 +109,8 @@ PLAN_SHAPES = [  # T, k, E, G, rpn, src mode
     (5000, 3, 12, 4, 1, "rand"), (777, 8, 64, 64, 8, "rand"), (1024, 8, 256, 64, 8, None),
     (2048, 6, 64, 32, 8, "skew"), (300, 4, 16, 1, 1, None), (999, 5, 40, 8, 4, "one"),
     (65536, 8, 64, 8, 8, "empty"),
+    (3000, 8, 128, 64, 1, "rand"),                        # 64 nodes of one rank: every bit of the node mask
+    (2048, 4, 64, 64, 64, None),                          # 64 ranks on one node: V = 0
 ]
 
 
