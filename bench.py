@@ -84,6 +84,8 @@ def parse():
                     help="replicate experts (EXTRA more per rank) and assign tasks to the fewest remote nodes")
     ap.add_argument("--prereduce", action="store_true",
                     help="receiver-side pre-reduced combine with stand-in experts (gates dispatched with rows)")
+    ap.add_argument("--seed", type=int, default=None,
+                    help="seed of the evaluation batch (calibration: seed + 1); the cluster layout stays the workload's")
     ap.add_argument("--coact-method", default="auto", choices=["auto", "histogram", "tensor"],
                     help="how the co-activation statistics count: per call, shared-memory histograms, tensor cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -93,10 +95,10 @@ def parse():
     return ap.parse_args()
 
 
-def rank_seed(w, rank):
+def rank_seed(base, rank):
     """Each rank draws its own batch (weak scaling); the cluster layout (the
     stand-in for the trained router) is the workload's, shared by all ranks."""
-    return w.seed + 1000 * rank
+    return base + 1000 * rank
 
 
 def reduce_max(x, pg, device):
@@ -226,19 +228,21 @@ def cpu_sample(w, T_s, seed):
     return ids, cal, gates, x
 
 
-def sized_sample(w, target_s, shuffle, balanced=False):
+def sized_sample(w, target_s, shuffle, balanced=False, base_seed=None):
     """Choose a token count (a multiple of G) whose oracle pass takes about target_s."""
+    base_seed = w.seed if base_seed is None else base_seed
     T_probe = max(w.G, (1024 // w.G) * w.G)
-    ids, cal, gates, x = cpu_sample(w, T_probe, w.seed)
+    ids, cal, gates, x = cpu_sample(w, T_probe, base_seed)
     sec, _ = oracle_pass(w, ids, cal, gates, x, "correlated", shuffle, balanced)
     T_s = int(T_probe * target_s / max(sec, 1e-6))
     T_s = max(w.G, min(w.T, (T_s // w.G) * w.G))
     return T_s
 
 
-def cpu_baseline(w, placement, shuffle, target_s, balanced=False):
-    T_s = sized_sample(w, target_s, shuffle, balanced)
-    ids, cal, gates, x = cpu_sample(w, T_s, w.seed)
+def cpu_baseline(w, placement, shuffle, target_s, balanced=False, base_seed=None):
+    base_seed = w.seed if base_seed is None else base_seed
+    T_s = sized_sample(w, target_s, shuffle, balanced, base_seed)
+    ids, cal, gates, x = cpu_sample(w, T_s, base_seed)
     sec, nbytes = oracle_pass(w, ids, cal, gates, x, placement, shuffle, balanced)
     model = platform.processor() or platform.machine()
     try:
@@ -263,8 +267,9 @@ def run_reference(a, w):
     bal = shuffle and a.balanced_shuffle
     # each step: a bounded sample, so that warmup + steps end within a few minutes
     per_step = max(0.5, min(10.0, 150.0 / max(1, a.steps + a.warmup)))
-    T_s = sized_sample(w, per_step, shuffle, bal)
-    ids, cal, gates, x = cpu_sample(w, T_s, w.seed)
+    base_seed = a.seed if getattr(a, "seed", None) is not None else w.seed
+    T_s = sized_sample(w, per_step, shuffle, bal, base_seed)
+    ids, cal, gates, x = cpu_sample(w, T_s, base_seed)
     for _ in range(a.warmup):
         oracle_pass(w, ids, cal, gates, x, a.placement, shuffle, bal)
     secs, nb = [], 0
@@ -330,7 +335,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
         pg = dist
-    seed = rank_seed(w, rank)
+    seed = rank_seed(a.seed if a.seed is not None else w.seed, rank)
     cap.coact_stats_method({"auto": 0, "histogram": 1, "tensor": 2}[a.coact_method])
     if a.sweep_only:
         hbm, _ = peaks()
@@ -449,7 +454,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu = cpu_baseline(w, a.placement, shuffle, a.cpu_seconds, balanced)
+        cpu = cpu_baseline(w, a.placement, shuffle, a.cpu_seconds, balanced, seed)
 
     if rank == 0:
         R = [int(s[0]) for s in summaries]
@@ -457,7 +462,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "G": w.G, "rpn": w.rpn, "d": w.d,
+            "config": {"workload": w.name, "seed": seed, "T": w.T, "E": w.E, "k": w.k, "G": w.G, "rpn": w.rpn, "d": w.d,
                        "L": w.L, "x_dtype": w.dtype, "out_dtype": a.out_dtype, "placement": a.placement,
                        "combine": "receiver-side pre-reduced (stand-in experts)" if a.prereduce
                                   else "source-side weighted (identity experts)",

@@ -28,7 +28,7 @@ def _worker(rank, world, port, q):
         from synth import WORKLOADS, make_routing
         import oracle as orc
         w = WORKLOADS["tiny"]
-        seed = bench.rank_seed(w, rank)
+        seed = bench.rank_seed(w.seed, rank)
         ids = make_routing(w, seed=seed, T=1024)
         st = orc.coact(ids, w.E)
         ms = [3.0, 5.0, 4.0][rank]
