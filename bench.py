@@ -11,9 +11,9 @@ Ochiai and transitions for every layer, then per layer the dispatch plan, the
 row permute, identity experts, the weighted combine and the shuffle targets
 for the next layer.  Plans, shuffle targets and statistics run on a second
 stream beside the row traffic (--no-overlap: in line); the timed steps are
-replayed from one CUDA graph (--no-graph: eager launches).  The default workload is large EP64 (T=131072, E=256, k=8,
-G=64 in 8 nodes, d=7168 bf16, 4 layers), the largest workload with hidden
-states; its inputs (x = 1.88 GB) exceed the 126 MB L2, so no flush is needed
+replayed from one CUDA graph (--no-graph: eager launches).  The default
+workload is large EP64 (T=131072, E=256, k=8, G=64 in 8 nodes, d=7168 bf16,
+4 layers), the largest workload with hidden states; its inputs (x = 1.88 GB) exceed the 126 MB L2, so no flush is needed
 between steps.  With N GPUs each rank runs its own batch (seed + rank): weak
 scaling, no collective on the data path.
 
@@ -379,9 +379,12 @@ def main():
     except Exception:
         pass
     # the timed steps: captured once into a CUDA graph (launch gaps between
-    # the small kernels vanish), or launched eagerly with --no-graph
+    # the small kernels vanish), or launched eagerly with --no-graph.  The
+    # timed graph carries no per-call timing events; a second graph with them
+    # is replayed afterwards for the per-kernel breakdown.
     graph = None
     graph_note = None
+    hp.timers = False
     if not a.no_graph:
         try:
             n0 = cap.launch_count()
@@ -393,7 +396,6 @@ def main():
     barrier()
     torch.cuda.synchronize()
     if graph is None:
-        hp.reset_events()
         n0 = cap.launch_count()
     with ClockSampler(uuid) as clk:
         start = torch.cuda.Event(enable_timing=True)
@@ -409,6 +411,20 @@ def main():
     if graph is None:
         n_launch = cap.launch_count() - n0
     barrier()
+    # per-kernel device times: the same steps again, with events around every call
+    graphed = graph is not None
+    hp.timers = True
+    hp.reset_events()
+    if graphed:
+        del graph
+        timed = hp.capture(a.steps)
+        timed.replay()
+        torch.cuda.synchronize()
+        del timed
+    else:
+        for _ in range(a.steps):
+            hp.step()
+        torch.cuda.synchronize()
     per_kernel = hp.kernel_times_ms()
     hp.reset_events()
     if int(hp.err.item()) != 0:
@@ -496,7 +512,8 @@ def main():
                             "statistics run on a second stream beside the row traffic, so their times include "
                             "waiting for SM slots and the kernel times add up to more than the step"
                             if hp.overlap else "CUDA events around each library call",
-            "timing": "one CUDA graph of the %d steps" % a.steps if graph is not None else
+            "timing": "one CUDA graph of the %d steps, without per-call events (a second graph with "
+                      "them gives the kernel breakdown)" % a.steps if graphed else
                       ("eager launches" + ("; " + graph_note if graph_note else "")),
             "cpu_baseline": cpu,
         }
