@@ -211,9 +211,8 @@ class HotPath:
             for l in range(self.L):
                 self._plan(l)
                 self.plan_ev[l].record(self.side)
-                if l == 0:
-                    self._stats()
                 self._shuffle(l)
+            self._stats()                       # nothing in the step waits for the statistics
             self.join_ev.record(self.side)
         for l in range(self.L):
             main.wait_event(self.plan_ev[l])
