@@ -13,8 +13,10 @@ for the next layer.  Plans, shuffle targets and statistics run on a second
 stream beside the row traffic (--no-overlap: in line); the timed steps are
 replayed from one CUDA graph (--no-graph: eager launches).  The default
 workload is large EP64 (T=131072, E=256, k=8, G=64 in 8 nodes, d=7168 bf16,
-4 layers), the largest workload with hidden states; its inputs (x = 1.88 GB) exceed the 126 MB L2, so no flush is needed
-between steps.  With N GPUs each rank runs its own batch (seed + rank): weak
+4 layers), the largest workload with hidden states; its inputs (x = 1.88 GB)
+exceed the 126 MB L2, so no flush is needed between steps.  Workloads whose
+inputs fit in L2 (one node, tiny) time each step on its own after a write of
+twice the L2 size.  With N GPUs each rank runs its own batch (seed + rank): weak
 scaling, no collective on the data path.
 
 value = dispatch+combine algorithmic bytes of the step / device time of the
@@ -382,14 +384,20 @@ def main():
     # the small kernels vanish), or launched eagerly with --no-graph.  The
     # timed graph carries no per-call timing events; a second graph with them
     # is replayed afterwards for the per-kernel breakdown.
+    # inputs that fit in L2 would stay cached from one step to the next: then
+    # every step is timed on its own, after a write of twice the L2 size
+    l2_bytes = int(getattr(torch.cuda.get_device_properties(device), "L2_cache_size", 0) or (126 << 20))
+    in_bytes = x.nbytes + ids.nbytes + gates.nbytes
+    flush = None if in_bytes > l2_bytes else torch.empty(2 * l2_bytes, dtype=torch.uint8, device=device)
+    per_graph = a.steps if flush is None else 1      # steps recorded in one graph
     graph = None
     graph_note = None
     hp.timers = False
     if not a.no_graph:
         try:
             n0 = cap.launch_count()
-            graph = hp.capture(a.steps)
-            n_launch = cap.launch_count() - n0      # kernels inside the replayed graph
+            graph = hp.capture(per_graph)
+            n_launch = (cap.launch_count() - n0) * (a.steps // per_graph)   # kernels the replays run
         except Exception as ex:                    # capture unsupported here: time eagerly
             graph, graph_note = None, "graph capture failed: %s" % str(ex).splitlines()[0][:120]
             torch.cuda.synchronize()
@@ -397,39 +405,62 @@ def main():
     torch.cuda.synchronize()
     if graph is None:
         n0 = cap.launch_count()
-    with ClockSampler(uuid) as clk:
-        start = torch.cuda.Event(enable_timing=True)
-        stop = torch.cuda.Event(enable_timing=True)
-        start.record()
+
+    def run(n):
         if graph is not None:
             graph.replay()
         else:
-            for _ in range(a.steps):
+            for _ in range(n):
                 hp.step()
-        stop.record()
-        torch.cuda.synchronize()
+
+    with ClockSampler(uuid) as clk:
+        if flush is None:
+            start = torch.cuda.Event(enable_timing=True)
+            stop = torch.cuda.Event(enable_timing=True)
+            start.record()
+            run(a.steps)
+            stop.record()
+            torch.cuda.synchronize()
+            ms_total = start.elapsed_time(stop)
+        else:
+            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(a.steps)]
+            for s0, s1 in pairs:
+                flush.zero_()
+                s0.record()
+                run(1)
+                s1.record()
+            torch.cuda.synchronize()
+            ms_total = sum(s0.elapsed_time(s1) for s0, s1 in pairs)
     if graph is None:
         n_launch = cap.launch_count() - n0
     barrier()
-    # per-kernel device times: the same steps again, with events around every call
+    # per-kernel device times: the same steps again, with events around every
+    # call (a replayed graph re-records its events: they hold its last replay)
     graphed = graph is not None
     hp.timers = True
     hp.reset_events()
     if graphed:
         del graph
-        timed = hp.capture(a.steps)
-        timed.replay()
+        timed = hp.capture(per_graph)
+        for _ in range(a.steps // per_graph):
+            if flush is not None:
+                flush.zero_()
+            timed.replay()
         torch.cuda.synchronize()
         del timed
+        ev_steps = per_graph
     else:
         for _ in range(a.steps):
+            if flush is not None:
+                flush.zero_()
             hp.step()
         torch.cuda.synchronize()
+        ev_steps = a.steps
     per_kernel = hp.kernel_times_ms()
     hp.reset_events()
     if int(hp.err.item()) != 0:
         raise SystemExit("device data error %d in the timed steps" % int(hp.err.item()))
-    ms_total = start.elapsed_time(stop)
     ms_step = ms_total / a.steps
     ms_step = reduce_max(ms_step, pg, device)
     clocks = clk.summary()
@@ -442,11 +473,15 @@ def main():
     launches_of = {"stats": 1, "plan": w.L, "permute": w.L, "combine": w.L, "shuffle": (w.L - 1) if shuffle else 0,
                    "gates": w.L, "reduce": w.L}
     for name, tot_ms in per_kernel.items():
-        ms = tot_ms / a.steps                         # per step
+        ms = tot_ms / ev_steps                        # per step
         gbs = bytes_of[name] / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
         kern[name] = {"ms_per_step": ms, "launches_per_step": launches_of[name], "gbs": gbs,
                       "frac_of_hbm": gbs / hbm}
-    dom = max(kern, key=lambda n: kern[n]["ms_per_step"])
+    # with the overlap the control calls' event times include waiting for SM
+    # slots beside the row traffic: the dominant kernel is taken among the
+    # calls on the main stream, whose chain is the step
+    side_calls = ("stats", "plan", "shuffle") if hp.overlap else ()
+    dom = max((n for n in kern if n not in side_calls), key=lambda n: kern[n]["ms_per_step"])
     nl = launches_of[dom]
     per_launch_ms = kern[dom]["ms_per_step"] / nl
     traffic = traffic_record(dom, bytes_of[dom] // nl)
@@ -487,7 +522,10 @@ def main():
                                   if hp.overlap else "none",
                        "shuffle": ("balanced (T/G tokens per rank)" if balanced else True) if shuffle else False,
                        "parallelism": "replicas (weak scaling, one batch per GPU)",
-                       "l2": "inputs larger than L2 (x %.2f GB per GPU; no flush)" % (x.nbytes / 1e9)},
+                       "l2": ("inputs larger than L2 (%.2f GB per GPU; no flush)" % (in_bytes / 1e9))
+                             if flush is None else
+                             ("inputs within L2 (%.3f GB per GPU): L2 flushed (%d MB write) before every "
+                              "step, steps timed one by one" % (in_bytes / 1e9, flush.nbytes >> 20))},
             "frac_of_hbm_peak": value / hbm,
             "roofline": roofline,
             "kernels": kern,
@@ -512,9 +550,10 @@ def main():
                             "statistics run on a second stream beside the row traffic, so their times include "
                             "waiting for SM slots and the kernel times add up to more than the step"
                             if hp.overlap else "CUDA events around each library call",
-            "timing": "one CUDA graph of the %d steps, without per-call events (a second graph with "
-                      "them gives the kernel breakdown)" % a.steps if graphed else
-                      ("eager launches" + ("; " + graph_note if graph_note else "")),
+            "timing": ("one CUDA graph of the %d steps" % a.steps if flush is None else
+                       "one CUDA graph of one step, replayed %d times between L2 flushes" % a.steps)
+                      + ", without per-call events (a second graph with them gives the kernel breakdown)"
+                      if graphed else ("eager launches" + ("; " + graph_note if graph_note else "")),
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
