@@ -81,6 +81,10 @@ def lib() -> ctypes.CDLL:
             "moe_place_replicas": ([P, i, i, i, P, i, P, P], i),
             "moe_assign_replicas": ([P, i, i, i, i, i, P, P, P, P, P, P, P], i),
             "moe_plan_dispatch_ranks": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
+            "moe_ep_routes": ([P, P, i, i, i, P, P, P], i),
+            "moe_ep_permute": ([P, i, i, i, i, P, i64, P, i, i, P, i64, P, P], i),
+            "moe_ep_combine": ([P, i, i64, i, P, i, i, i64, P, P, i, i, P, i, P, P], i),
+            "moe_ep_scatter_rows": ([P, i64, i64, P, i, i, P, i64, P, P], i),
         }
         for name, (args, res) in sigs.items():
             f = getattr(L, name)
@@ -420,6 +424,73 @@ def combine_rows(Y: torch.Tensor, row_of: torch.Tensor, out_dtype=torch.float32,
                                 _dtype_code(out.dtype), _ptr(err), _stream(Y))
     _check("moe_combine_rows", st)
     return out
+
+
+# ---------------------------------------------------------------- several devices
+
+def ep_route_len(G: int, W: int) -> int:
+    """Entries (int64) of a route table for G ranks over W devices."""
+    return 2 * G * (G // W) + 2
+
+
+def ep_routes(counts_all: torch.Tensor, offsets: torch.Tensor, G: int, W: int, me: int,
+              route: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """route int64 [2*G*(G/W) + 2]: where this device's rows land in the receiving devices' buffers."""
+    _dev(counts_all, torch.int32, "counts_all", 2)
+    _dev(offsets, torch.int32, "offsets", 1)
+    if route is None:
+        route = torch.empty(ep_route_len(G, W), dtype=torch.int64, device=counts_all.device)
+    err = new_err(counts_all.device) if err is None else err
+    st = lib().moe_ep_routes(_ptr(counts_all), _ptr(offsets), G, W, me, _ptr(route), _ptr(err), _stream(counts_all))
+    _check("moe_ep_routes", st)
+    return route
+
+
+def ep_permute(x: torch.Tensor, row_of: torch.Tensor, R_max: int, route: torch.Tensor, G: int, W: int,
+               recv_base: torch.Tensor, recv_cap: int, err: Optional[torch.Tensor] = None):
+    """Store every local row x[t] into its receiving device's buffer (recv_base: int64 [W] addresses)."""
+    _dev(x, x.dtype, "x", 2)
+    _dev(row_of, torch.int32, "row_of", 2)
+    _dev(route, torch.int64, "route", 1)
+    _dev(recv_base, torch.int64, "recv_base", 1)
+    T, d = x.shape
+    k = row_of.shape[1]
+    err = new_err(x.device) if err is None else err
+    st = lib().moe_ep_permute(_ptr(x), _dtype_code(x.dtype), T, d, k, _ptr(row_of), R_max, _ptr(route), G, W,
+                              _ptr(recv_base), recv_cap, _ptr(err), _stream(x))
+    _check("moe_ep_permute", st)
+
+
+def ep_combine(y_base: torch.Tensor, y_dtype, y_cap: int, d: int, route: torch.Tensor, G: int, W: int,
+               R_max: int, idx: torch.Tensor, w: Optional[torch.Tensor], out: torch.Tensor,
+               err: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out[t] = sum_j w[t][j] * Y[idx[t][j]] (w None: distinct rows once), rows read from the devices' buffers."""
+    _dev(y_base, torch.int64, "y_base", 1)
+    _dev(route, torch.int64, "route", 1)
+    _dev(idx, torch.int32, "idx", 2)
+    if w is not None:
+        _dev(w, torch.float32, "w", 2)
+    _dev(out, out.dtype, "out", 2)
+    T, k = idx.shape
+    err = new_err(out.device) if err is None else err
+    st = lib().moe_ep_combine(_ptr(y_base), _dtype_code(y_dtype), y_cap, d, _ptr(route), G, W, R_max, _ptr(idx),
+                              _ptr(w), T, k, _ptr(out), _dtype_code(out.dtype), _ptr(err), _stream(out))
+    _check("moe_ep_combine", st)
+    return out
+
+
+def ep_scatter_rows(src: torch.Tensor, route: torch.Tensor, G: int, W: int, dst_base: torch.Tensor, dst_cap: int,
+                    err: Optional[torch.Tensor] = None):
+    """Per-row records src [R_max][...] (4-byte elements) stored to the receiving devices' buffers."""
+    _dev(src, src.dtype, "src")
+    _dev(route, torch.int64, "route", 1)
+    _dev(dst_base, torch.int64, "dst_base", 1)
+    R_max = src.shape[0]
+    row_bytes = src[0].numel() * src.element_size() if R_max else 4
+    err = new_err(src.device) if err is None else err
+    st = lib().moe_ep_scatter_rows(_ptr(src), row_bytes, R_max, _ptr(route), G, W, _ptr(dst_base), dst_cap,
+                                   _ptr(err), _stream(src))
+    _check("moe_ep_scatter_rows", st)
 
 
 # ---------------------------------------------------------------- token shuffle

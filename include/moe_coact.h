@@ -20,7 +20,8 @@
  * D_t^l is the set of k distinct experts token t selects at layer l;
  * p(e) = expert_to_rank[e]; s_t is token t's source rank; N(r) = r / rpn.
  * EP ranks and nodes are logical partitions of one GPU's memory: "rank r's
- * receive buffer" is a segment of one device buffer.
+ * receive buffer" is a segment of one device buffer (the moe_ep_* calls
+ * spread the ranks over several devices instead).
  *
  * Conventions for every call:
  *  - Pointers marked "device" are device memory owned by the caller; "host"
@@ -315,6 +316,78 @@ moe_status moe_expert_reduce(const void *send, moe_dtype dtype, int64_t R_max, i
                              cudaStream_t stream);
 moe_status moe_combine_rows(const void *Y, moe_dtype y_dtype, int64_t R_max, int d, const int32_t *row_of,
                             int T, int k, void *out, moe_dtype out_dtype, int32_t *err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Expert parallelism over several devices  ([EC]: each token is sent to each
+ * GPU once and the results combined; [CE] footnote 3: hidden states and
+ * routed probabilities are dispatched, the combine is the inverse exchange)
+ *
+ * The G ranks are spread over W devices, Gl = G/W consecutive ranks per
+ * device: device h hosts ranks h*Gl .. h*Gl+Gl-1.  Each device plans its own
+ * tokens with moe_plan_dispatch, every token's source rank in the device's
+ * range (src_rank given).  Device h's receive buffer then holds the rows
+ * addressed to its ranks in the order the one-device plan over all tokens
+ * gives them -- destination rank, then source rank, then token -- i.e.
+ * exactly rows [off(h*Gl, 0), off(h*Gl+Gl, 0)) of that plan's send buffer,
+ * off(r, s) being its offsets[r*G+s].  Rows are stored to and loaded from
+ * the other devices' buffers through peer pointers (plain loads and stores
+ * over NVLink).  Synchronising the devices between the phases (all stores of
+ * every device done before any receiver reads; all combines done before the
+ * next dispatch overwrites a buffer) is the caller's, e.g. a small NCCL
+ * all-reduce on the same stream.
+ *
+ * moe_ep_routes: counts_all device int32 [G][G], row s = the counts row of
+ *   source rank s as planned by the device hosting s (gathered from all
+ *   devices); offsets device int32 [G*G+1] of this device's plan; me = this
+ *   device's index in [0, W).  Writes route device int64 [2*G*Gl + 2]:
+ *   route[0] = rows this device receives; route[1+i], i <= P = G*Gl: the
+ *   local row where segment i starts (segment i = destination rank i/Gl,
+ *   source rank me*Gl + i%Gl; route[1+P] = this device's R); route[P+2+i]:
+ *   the shift from a local row of segment i to its row in the receiving
+ *   device's buffer.  Data errors: MOE_DERR_ROW_RANGE if a gathered count is
+ *   negative or this device's row of counts_all disagrees with its plan.
+ *
+ * moe_ep_permute: recv[h][q][:] = x[t][:] for every local row (t, r) of this
+ *   device's plan, h = r/Gl and q its row in h's buffer (from route); each
+ *   token's row of x is read once.  x device [T][d] of dtype (16-byte
+ *   aligned); row_of device int32 [T][k] of the local plan; recv_base device
+ *   array of W addresses (this device's own buffer at index me; every buffer
+ *   32-byte aligned, recv_cap rows of d elements).  Data errors:
+ *   MOE_DERR_ROW_RANGE (a row outside the plan, a target row outside
+ *   [0, recv_cap) or a misaligned or null base: that store is skipped).
+ *
+ * moe_ep_combine: the combine of moe_combine (w given) or of
+ *   moe_combine_rows (w NULL: each distinct row once, weight 1) for this
+ *   device's T tokens, with Y's row for a local row read from its receiving
+ *   device's buffer: y_base device array of W addresses (32-byte aligned,
+ *   y_cap rows of d elements of y_dtype each, in the receive-buffer order);
+ *   idx device int32 [T][k] local rows (row_of), R_max the local row bound;
+ *   out device [T][d] of out_dtype.  Results equal those of moe_combine /
+ *   moe_combine_rows on the one-device send buffer bit for bit.  Data errors:
+ *   MOE_DERR_ROW_RANGE (the term is skipped).
+ *
+ * moe_ep_scatter_rows: a record of row_bytes bytes per local row (e.g. the
+ *   gates of moe_dispatch_gates: k int32 or k floats) stored to the receiving
+ *   devices the same way: dst[h][q] = src[x] for the local rows x < R (R from
+ *   route).  src device [R_max][row_bytes] (4-byte aligned); dst_base device
+ *   array of W addresses (32-byte aligned, dst_cap records each); row_bytes a
+ *   multiple of 4, at most 1024.
+ *
+ * Limits: 1 <= G <= 64, W | G, 0 <= me < W, 1 <= k <= 8, d*sizeof(dtype) a
+ * multiple of 16 bytes.
+ * ---------------------------------------------------------------------- */
+moe_status moe_ep_routes(const int32_t *counts_all, const int32_t *offsets, int G, int W, int me,
+                         int64_t *route, int32_t *err, cudaStream_t stream);
+moe_status moe_ep_permute(const void *x, moe_dtype dtype, int T, int d, int k, const int32_t *row_of,
+                          int64_t R_max, const int64_t *route, int G, int W, void *const *recv_base,
+                          int64_t recv_cap, int32_t *err, cudaStream_t stream);
+moe_status moe_ep_combine(void *const *y_base, moe_dtype y_dtype, int64_t y_cap, int d,
+                          const int64_t *route, int G, int W, int64_t R_max, const int32_t *idx,
+                          const float *w, int T, int k, void *out, moe_dtype out_dtype, int32_t *err,
+                          cudaStream_t stream);
+moe_status moe_ep_scatter_rows(const void *src, int64_t row_bytes, int64_t R_max, const int64_t *route,
+                               int G, int W, void *const *dst_base, int64_t dst_cap, int32_t *err,
+                               cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Token shuffling  ([EC]: move each token to the GPU predicted to hold its

@@ -127,6 +127,21 @@ def test_argument_errors_return_before_device_work(cap):
     # EMA: alpha outside [0, 1], in place
     assert L.moe_coact_ema(fake, 1, 4, ctypes.c_double(1.5), None, fake, None, None) == cap.MOE_ERR_ARG
     assert L.moe_coact_ema(fake, 1, 4, ctypes.c_double(0.5), fake, fake, None, None) == cap.MOE_ERR_ARG
+    # several devices: W not dividing G, me outside [0, W), G > 64, misaligned x, odd row sizes, records
+    assert L.moe_ep_routes(fake, fake, 8, 3, 0, fake, fake, None) == cap.MOE_ERR_ARG
+    assert L.moe_ep_routes(fake, fake, 8, 4, 4, fake, fake, None) == cap.MOE_ERR_ARG
+    assert L.moe_ep_routes(fake, fake, 128, 2, 0, fake, fake, None) == cap.MOE_ERR_ARG
+    assert L.moe_ep_permute(P(264), cap.MOE_BF16, 4, 8, 2, fake, 8, fake, 8, 2, fake, 8, fake, None) == cap.MOE_ERR_ARG
+    assert L.moe_ep_permute(fake, cap.MOE_BF16, 4, 7, 2, fake, 8, fake, 8, 2, fake, 8, fake, None) \
+        == cap.MOE_ERR_UNSUPPORTED
+    assert L.moe_ep_permute(fake, cap.MOE_F32, 4, 8, 9, fake, 8, fake, 8, 2, fake, 8, fake, None) == cap.MOE_ERR_ARG
+    assert L.moe_ep_combine(fake, cap.MOE_F32, 8, 8, fake, 8, 3, 8, fake, fake, 4, 2, fake, 0, fake, None) \
+        == cap.MOE_ERR_ARG
+    assert L.moe_ep_combine(fake, cap.MOE_F32, 8, 8, fake, 8, 2, 8, fake, fake, 4, 2, P(260), 0, fake, None) \
+        == cap.MOE_ERR_ARG
+    assert L.moe_ep_scatter_rows(fake, 6, 8, fake, 8, 2, fake, 8, fake, None) == cap.MOE_ERR_ARG
+    assert L.moe_ep_scatter_rows(P(258), 8, 8, fake, 8, 2, fake, 8, fake, None) == cap.MOE_ERR_ARG
+    assert cap.ep_route_len(64, 8) == 2 * 64 * 8 + 2
 
 
 @pytest.mark.parametrize("E,G,rpn,extra", [(16, 8, 2, 1), (64, 8, 8, 2), (64, 32, 8, 1), (256, 64, 8, 1), (24, 6, 1, 3)])
