@@ -4,7 +4,7 @@
                     [--placement correlated|uniform|capacity|capped] [--no-shuffle]
                     [--balanced-shuffle] [--prereduce] [--replicas N]
                     [--coact-method auto|histogram|tensor] [--no-overlap] [--no-graph]
-                    [--out-dtype f32|bf16] [--impl reference]
+                    [--out-dtype f32|bf16] [--ep-emulate W] [--impl reference]
 
 A step is one pass of the whole path over one batch: co-activation counts,
 Ochiai and transitions for every layer, then per layer the dispatch plan, the
@@ -90,6 +90,8 @@ def parse():
                     help="seed of the evaluation batch (calibration: seed + 1); the cluster layout stays the workload's")
     ap.add_argument("--coact-method", default="auto", choices=["auto", "histogram", "tensor"],
                     help="how the co-activation statistics count: per call, shared-memory histograms, tensor cores")
+    ap.add_argument("--ep-emulate", type=int, default=0, metavar="W",
+                    help="also time the several-device path with W virtual devices on this GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--sweep-only", action="store_true", help="only the co-activation statistics sweep")
@@ -499,6 +501,10 @@ def main():
     if not a.no_sweep:
         sweep = run_sweep(cap, pipeline, device, seed, a.steps, a.warmup, hbm, pg)
 
+    ep_emu = None
+    if a.ep_emulate > 0 and not a.prereduce and a.replicas == 0:
+        ep_emu = run_ep_emulated(hp, w, a.ep_emulate, a.steps, a.warmup, hbm, sb, pg)
+
     e2e = None
     if not a.no_e2e:
         e2e = run_e2e(hp, ids, gates, x, w, a, device, sb, pg, world)
@@ -544,6 +550,7 @@ def main():
                               for i, n in enumerate(["propose", "gather", "select", "barrier_wait"])}}
             if balanced else None,
             "e2e": e2e,
+            "ep_emulated": ep_emu,
             "gpu_launches": int(n_launch),
             "gpu_launches_per_step": n_launch / a.steps,
             "kernel_times": "CUDA events around each library call on its stream; plans, shuffle targets and "
@@ -629,6 +636,58 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
                                 "peak_note": "32 per clock per SM x %d SMs x %.0f MHz" % (sms, SM_MAX_MHZ)},
             "algorithmic_bytes": nbytes, "err": int(hp.err.item()),
             "placement_effect": effect}
+
+
+def run_ep_emulated(hp, w, W, steps, warmup, hbm, sb, pg):
+    """The several-device path (moe_ep_routes / moe_ep_permute / moe_ep_combine)
+    with W virtual devices on this GPU, each with its own receive buffer and
+    T/W tokens, over all layers with identity experts; one CUDA graph of the
+    steps.  The bytes are the step's dispatch+combine bytes: R does not depend
+    on which rank a token starts from."""
+    import torch
+    import co_activation_placement_b200 as cap
+    from co_activation_placement_b200.ep import EPEmulation
+    if w.G % W or w.T % W:
+        return {"devices": W, "skipped": "W must divide G and T"}
+    Gl = w.G // W
+    rows = 0
+    for l in range(w.L):                      # receive capacity from the contiguous-source plans
+        p = cap.plan_dispatch(hp.ids[l], w.E, w.G, w.rpn, hp.e2r[l])
+        off = p.offsets.cpu().numpy().astype(np.int64)
+        rows = max(rows, max(int(off[(h + 1) * Gl * w.G] - off[h * Gl * w.G]) for h in range(W)))
+        del p
+    emu = EPEmulation(W, w.E, w.G, w.rpn, w.T, w.k, w.d, hp.x.dtype, hp.x.device, rows, out_dtype=hp.out_dtype)
+
+    def step():
+        for l in range(w.L):
+            emu.step(hp.ids[l], hp.x, hp.gates[l], hp.e2r[l])
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if any(emu.errors()):
+        raise SystemExit("device data error in the several-device path: %s" % emu.errors())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        for _ in range(steps):
+            step()
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    del g
+    nbytes = sb.permute + sb.combine
+    return {"devices": W, "ranks_per_device": Gl, "tokens_per_device": w.T // W, "recv_rows_max": rows,
+            "ms_per_step": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
+            "errors": emu.errors(),
+            "note": "W virtual devices on this GPU, each with its own receive buffer, launched one after another; "
+                    "rows move through the peer-addressed kernels within this GPU's memory; per layer and "
+                    "device: plan, routes, permute, combine (the counts gathered with one device-side copy)"}
 
 
 def run_e2e(hp, ids, gates, x, w, a, device, sb, pg, world):
