@@ -4,7 +4,7 @@
                     [--placement correlated|uniform|capacity|capped] [--no-shuffle]
                     [--balanced-shuffle] [--prereduce] [--replicas N]
                     [--coact-method auto|histogram|tensor] [--no-overlap] [--no-graph]
-                    [--out-dtype f32|bf16] [--ep-emulate W] [--impl reference]
+                    [--out-dtype f32|bf16] [--ep] [--ep-emulate W] [--impl reference]
 
 A step is one pass of the whole path over one batch: co-activation counts,
 Ochiai and transitions for every layer, then per layer the dispatch plan, the
@@ -90,6 +90,9 @@ def parse():
                     help="seed of the evaluation batch (calibration: seed + 1); the cluster layout stays the workload's")
     ap.add_argument("--coact-method", default="auto", choices=["auto", "histogram", "tensor"],
                     help="how the co-activation statistics count: per call, shared-memory histograms, tensor cores")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism over the job's GPUs: the G ranks spread over the N processes "
+                         "(rows stored to and loaded from the other GPUs' buffers)")
     ap.add_argument("--ep-emulate", type=int, default=0, metavar="W",
                     help="also time the several-device path with W virtual devices on this GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -341,6 +344,9 @@ def main():
         pg = dist
     seed = rank_seed(a.seed if a.seed is not None else w.seed, rank)
     cap.coact_stats_method({"auto": 0, "histogram": 1, "tensor": 2}[a.coact_method])
+    if a.ep:
+        run_ep(a, w, rank, world, device, seed)
+        return
     if a.sweep_only:
         hbm, _ = peaks()
         sweep = run_sweep(cap, pipeline, device, seed, a.steps, a.warmup, hbm, pg)
@@ -636,6 +642,112 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
                                 "peak_note": "32 per clock per SM x %d SMs x %.0f MHz" % (sms, SM_MAX_MHZ)},
             "algorithmic_bytes": nbytes, "err": int(hp.err.item()),
             "placement_effect": effect}
+
+
+def run_ep(a, w, rank, world, device, seed):
+    """--ep: one process per GPU, the workload's G ranks spread over the N
+    GPUs (G/N each), every GPU with its own batch of T tokens (weak scaling:
+    N*T tokens over the G ranks).  A step: the statistics of all GPUs' tokens
+    (local counts, one all-reduce) and, per layer, the plan of this GPU's
+    tokens, the counts all-gather, the route table, the rows stored into the
+    receiving GPUs' buffers, identity experts and the combine loading them
+    back (EPGroup).  The placement comes from one calibration batch that every
+    GPU draws alike.  Timed eagerly with CUDA events, max over the GPUs."""
+    import datetime
+    import socket
+    import torch
+    import torch.distributed as dist
+    import co_activation_placement_b200 as cap
+    from co_activation_placement_b200 import pipeline
+    from co_activation_placement_b200.ep import EPGroup
+    from synth import make_routing, make_gates, make_hidden
+    if not dist.is_initialized():                 # one GPU: a one-process group
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % port, rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120), device_id=device)
+    if w.G % world or w.d == 0:
+        raise SystemExit("--ep needs hidden states and N dividing G")
+    base = a.seed if a.seed is not None else w.seed
+    ids = torch.from_numpy(make_routing(w, seed=seed)).to(device)
+    gates = torch.from_numpy(make_gates(w, seed=seed)).to(device)
+    xh = make_hidden(w, seed=seed)
+    x = (torch.from_numpy(xh.view(np.int16)).to(device).view(torch.bfloat16) if w.dtype == "bf16"
+         else torch.from_numpy(xh).to(device))
+    cal = torch.from_numpy(make_routing(w, seed=base + 1)).to(device)
+    e2r = pipeline.calibrate(cal, w.E, w.G, w.rpn, a.placement, False)[0]
+    Gl = w.G // world
+    # receive capacity and row counts: every layer planned once, counts gathered
+    from co_activation_placement_b200.ep import EPShard, gather_counts
+    sh = EPShard(world, rank, w.E, w.G, w.rpn, w.T, w.k, w.d, x.dtype, device)
+    need, R = 0, []
+    for l in range(w.L):
+        sh.plan_layer(ids[l], e2r[l])
+        gather_counts(sh.counts_all, sh.my_counts())
+        c = sh.counts_all.cpu().numpy().astype(np.int64)
+        need = max(need, int(c[:, rank * Gl:(rank + 1) * Gl].sum()))
+        R.append(int(sh.plan.summary[0].item()))
+    del sh
+    t = torch.tensor([need], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    recv_cap = int(t.item()) + 64
+    out_dtype = torch.float32 if a.out_dtype == "f32" else torch.bfloat16
+    grp = EPGroup(w.E, w.G, w.rpn, w.T, w.k, w.d, x.dtype, device, recv_cap, out_dtype=out_dtype)
+
+    def step():
+        grp.stats(ids, w.E)
+        for l in range(w.L):
+            grp.step(ids[l], x, gates[l], e2r[l])
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(grp.shard.err.item()):
+        raise SystemExit("device data error %d" % int(grp.shard.err.item()))
+    dist.barrier()
+    torch.cuda.synchronize()
+    n0 = cap.launch_count()
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+    with ClockSampler(uuid) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(a.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    n_launch = cap.launch_count() - n0
+    dist.barrier()
+    ms = reduce_max(e0.elapsed_time(e1) / a.steps, dist, device)
+    rowB = w.d * x.element_size()
+    ob = w.d * (4 if a.out_dtype == "f32" else 2)
+    mine = sum(w.T * rowB + r * rowB + 4 * w.T * w.k + r * rowB + w.T * ob + 8 * w.T * w.k for r in R)
+    tb = torch.tensor([float(mine)], dtype=torch.float64, device=device)
+    dist.all_reduce(tb)
+    hbm, hbm_kind = peaks()
+    value = float(tb.item()) / (ms * 1e-3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "seed": seed, "T_per_gpu": w.T, "E": w.E, "k": w.k, "G": w.G, "rpn": w.rpn,
+                       "d": w.d, "L": w.L, "x_dtype": w.dtype, "out_dtype": a.out_dtype, "placement": a.placement,
+                       "parallelism": "expert parallel over %d GPU(s), %d ranks each" % (world, Gl),
+                       "recv_rows_capacity": recv_cap,
+                       "l2": "inputs larger than L2" if x.nbytes > (126 << 20) else "inputs within L2 (no flush)"},
+            "frac_of_hbm_peak": value / hbm if world == 1 else None,
+            "roofline": None,
+            "roofline_note": "per-kernel events are not taken in this mode; the one-GPU path reports the kernels",
+            "clocks": clk.summary(), "gpu_launches": int(n_launch), "e2e": None, "cpu_baseline": None,
+            "timing": "eager launches between two CUDA events, max over the GPUs",
+        }), flush=True)
+    del grp
+    dist.destroy_process_group()
 
 
 def run_ep_emulated(hp, w, W, steps, warmup, hbm, sb, pg):

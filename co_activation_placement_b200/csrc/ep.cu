@@ -285,7 +285,10 @@ moe_status launch_ep_permute(const void *x, size_t rowB, int T, const int32_t *r
 {
     const char *xb = static_cast<const char *>(x);
     if (rowB % 32 == 0 && (reinterpret_cast<uintptr_t>(x) & 31u) == 0)
-        ep_permute_kernel<K, 8, 32><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 32), T, row_of, R_max, rt, err);
+        if (T >= kDeepPermuteTokens)
+            ep_permute_kernel<K, 8, 32><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 32), T, row_of, R_max, rt, err);
+        else
+            ep_permute_kernel<K, 4, 32><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 32), T, row_of, R_max, rt, err);
     else
         ep_permute_kernel<K, 4, 16><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 16), T, row_of, R_max, rt, err);
     return launch_status();

@@ -9,8 +9,8 @@
 // ld/st.global.v8 forms; 16-byte vectors when a row or pointer is not 32-byte
 // aligned); nothing here is a dense contraction.  Both are token-major: one
 // warp owns one token at a time.
-//  - permute reads the token's row of x once (8 32-byte vectors per lane in
-//    flight: measured 0.6% faster than 4 and 1.5% faster than 2 on 14 KB rows)
+//  - permute reads the token's row of x once (8 or 4 32-byte vectors per lane
+//    in flight, by launch size: kDeepPermuteTokens)
 //    and writes it to each of its distinct send rows (row_of[t][j], duplicates
 //    skipped), so HBM traffic is T_active*rowB read + R*rowB written -- the
 //    minimum.  (A variant staging rows in shared memory with bulk async copies
@@ -228,7 +228,10 @@ moe_status launch_permute(const void *x, size_t rowB, int T, const int32_t *row_
     const char *xb = static_cast<const char *>(x);
     char *sb = static_cast<char *>(send);
     if (rowB % 32 == 0 && (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (reinterpret_cast<uintptr_t>(send) & 31u) == 0)
-        permute_kernel<K, 8, 32><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 32), T, row_of, R_max, sb, err);
+        if (T >= kDeepPermuteTokens)
+            permute_kernel<K, 8, 32><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 32), T, row_of, R_max, sb, err);
+        else
+            permute_kernel<K, 4, 32><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 32), T, row_of, R_max, sb, err);
     else
         permute_kernel<K, 4, 16><<<row_grid(T), kRowThreads, 0, s>>>(xb, (int)(rowB / 16), T, row_of, R_max, sb, err);
     return launch_status();

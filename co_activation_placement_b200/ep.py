@@ -228,11 +228,20 @@ class EPGroup:
     def stats(self, ids: torch.Tensor, E: int):
         """Counts, Ochiai and transitions of all devices' tokens: local counts,
         one all-reduce, Ochiai from the sums."""
-        st = cap.coact_stats(ids, E, want=("coact", "trans"))
-        allreduce_counts(*[c for c in (st["coact"], st["trans"]) if c is not None], group=self.group)
         L = ids.shape[0]
-        ema = torch.empty((L, E, E), dtype=torch.float64, device=ids.device)
-        st["ochiai"] = cap.coact_ema(st["coact"], 1.0, ema_out=ema)[1]
+        key = (L, E, str(ids.device))
+        if getattr(self, "_stats_key", None) != key:
+            dev = ids.device
+            self._stats_key = key
+            self._st = dict(coact=torch.empty((L, E, E), dtype=torch.uint32, device=dev),
+                            trans=torch.empty((L - 1, E, E), dtype=torch.uint32, device=dev) if L > 1 else None,
+                            ochiai=torch.empty((L, E, E), dtype=torch.float32, device=dev),
+                            ema=torch.empty((L, E, E), dtype=torch.float64, device=dev), err=cap.new_err(dev))
+        b = self._st
+        st = cap.coact_stats(ids, E, coact=b["coact"], trans=b["trans"], err=b["err"], want=("coact", "trans"))
+        allreduce_counts(*[c for c in (st["coact"], st["trans"]) if c is not None], group=self.group)
+        cap.coact_ema(st["coact"], 1.0, ema_out=b["ema"], ochiai=b["ochiai"])
+        st["ochiai"] = b["ochiai"]
         return st
 
     def step(self, ids: torch.Tensor, x: torch.Tensor, gates: torch.Tensor, expert_to_rank: torch.Tensor):

@@ -272,3 +272,53 @@ def test_ep_group_one_process(cap):
                        capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
     assert "ep_group ok rank=0" in r.stdout
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_ep_fuzz(cap, seed):
+    """Seeded random shapes: G in 1..64, W any divisor of G, tokens a ragged
+    multiple of G, k 1..8, f32 or bf16 rows of 16..544 bytes, uniform or
+    permuted placement, with and without pre-reduction."""
+    from co_activation_placement_b200.ep import EPEmulation
+    rng = np.random.default_rng(5000 + seed)
+    G = int(rng.choice([1, 2, 3, 4, 6, 8, 12, 16, 32, 64]))
+    W = int(rng.choice([w_ for w_ in range(1, G + 1) if G % w_ == 0]))
+    rpn = int(rng.choice([r for r in range(1, G + 1) if G % r == 0]))
+    E = G * int(rng.integers(1, max(2, 256 // G) + 1))
+    k = int(rng.integers(1, min(8, E) + 1))
+    T = G * int(rng.integers(1, max(2, 3000 // G)))
+    bf16 = bool(rng.integers(0, 2))
+    d = int(rng.choice([8, 16, 40, 64, 136]))
+    if (d * (2 if bf16 else 4)) % 16:
+        d += 8 - d % 8
+    prereduce = bool(rng.integers(0, 2))
+    ids, w, xf, xh, xd, scale, e2r = _setup(6000 + seed, T, E, k, G, d, bf16)
+    if rng.integers(0, 2):
+        e2r = orc.place_uniform(E, G)
+    o = orc.plan(ids, E, G, rpn, e2r)
+    off = o["offsets"].astype(np.int64)
+    Gl = G // W
+    rows = [int(off[(h + 1) * Gl * G] - off[h * Gl * G]) for h in range(W)]
+    dt = torch.bfloat16 if bf16 else torch.float32
+    emu = EPEmulation(W, E, G, rpn, T, k, d, dt, "cuda", max(max(rows), 1), prereduce=prereduce, scale=dev(scale))
+    outs = emu.step(dev(ids), xd, dev(w), dev(e2r))
+    assert emu.errors() == [0] * W, (G, W, rpn, E, k, T, d, bf16, prereduce)
+    send = orc.permute(xh, o["row_token"])
+    for h in range(W):
+        got = host(emu.recv[h].view(torch.int16) if bf16 else emu.recv[h])[: rows[h]]
+        assert (got.view(send.dtype) == send[off[h * Gl * G]: off[h * Gl * G] + rows[h]]).all()
+    p = cap.plan_dispatch(dev(ids), E, G, rpn, dev(e2r))
+    one = cap.permute(xd, p.row_of, p.R_max, err=p.err)
+    if prereduce:
+        se, sw = cap.dispatch_gates(dev(ids), dev(w), p)
+        y1 = cap.expert_reduce(one, p.summary, se, sw, dev(scale), y_dtype=dt, err=p.err)
+        out1 = cap.combine_rows(y1, p.row_of, err=p.err)
+    else:
+        out1 = cap.combine(one, p.row_of, dev(w), err=p.err)
+    got = np.concatenate([host(t) for t in outs])
+    assert (host(out1).view(np.uint32) == got.view(np.uint32)).all()
+    if not prereduce:
+        Yf = orc.permute(xf, o["row_token"])
+        ref = orc.combine(Yf, o["row_of"], w, y_is_bf16=False)
+        assert (np.abs(got - ref) <= combine_bound(Yf, o["row_of"], w, k)).all()
+    assert int(host(p.err)[0]) == 0
