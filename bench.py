@@ -313,8 +313,9 @@ def traffic_record(kernel_name, algorithmic_bytes_per_launch):
         rec = json.load(f).get(kernel_name)
     if not rec:
         return None
-    src = os.path.join(ROOT, "co_activation_placement_b200", "csrc", rec["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    names = rec["source"].split("+")              # the kernel's file and the headers it is built from
+    blob = b"".join(open(os.path.join(ROOT, "co_activation_placement_b200", "csrc", n), "rb").read() for n in names)
+    h = hashlib.sha256(blob).hexdigest()[:16]
     if h != rec["source_sha256_16"]:
         return None
     return int(rec["traffic_over_algorithmic"] * algorithmic_bytes_per_launch)
