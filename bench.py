@@ -371,6 +371,7 @@ def main():
                           scales=make_expert_scales(w, seed=seed) if a.prereduce else None,
                           replica_extra=a.replicas, shuffle_capacity=w.T // w.G if balanced else 0,
                           overlap=not a.no_overlap)
+    place = time_placement(cap, ids_cal, w, a.placement, device)
 
     def barrier():
         if pg is not None:
@@ -557,6 +558,7 @@ def main():
                               for i, n in enumerate(["propose", "gather", "select", "barrier_wait"])}}
             if balanced else None,
             "e2e": e2e,
+            "placement_host": place,
             "ep_emulated": ep_emu,
             "gpu_launches": int(n_launch),
             "gpu_launches_per_step": n_launch / a.steps,
@@ -643,6 +645,32 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
                                 "peak_note": "32 per clock per SM x %d SMs x %.0f MHz" % (sms, SM_MAX_MHZ)},
             "algorithmic_bytes": nbytes, "err": int(hp.err.item()),
             "placement_effect": effect}
+
+
+def time_placement(cap, ids_cal, w, placement, device):
+    """Host time of the placement from the calibration batch's counts (the
+    step that runs once per re-layout, on one CPU thread): per layer, and the
+    counts' device-to-host read beside it."""
+    import torch
+    cal = torch.from_numpy(ids_cal).to(device)
+    st = cap.coact_stats(cal, w.E, want=("coact",))
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    coact = st["coact"].cpu().numpy()
+    t1 = time.perf_counter()
+    for l in range(w.L):
+        c = coact[l]
+        if placement == "uniform":
+            cap.place_uniform(w.E, w.G)
+        elif placement == "correlated":
+            cap.place_correlated(c, w.G, w.rpn)
+        elif placement == "capped":
+            cap.place_correlated_capped(c, w.G, w.rpn, 0.1)
+        else:
+            cap.place_capacity(np.diag(c).astype(np.float64), w.G)
+    t2 = time.perf_counter()
+    return {"kind": placement, "ms_per_layer": (t2 - t1) * 1e3 / w.L, "counts_readback_ms": (t1 - t0) * 1e3,
+            "threads": 1, "E": w.E, "G": w.G}
 
 
 def run_ep(a, w, rank, world, device, seed):
