@@ -10,13 +10,17 @@
 //
 // moe_rank_score: one block per expert row e, a shared uint64 accumulator per
 // rank (integer atomics: order-free).  moe_shuffle_targets: the E x G table
-// sits in shared memory (one block per SM, so it is copied once per SM); a
-// warp stages the picks of 32 tokens in shared memory and then scores them one
-// at a time, every lane reading the token's picks with broadcast loads and
-// owning ranks lane and lane+32 (conflict-free: a row of the table is read
-// contiguously), with uint64 sums.  The argmax on (score desc, rank asc) is a
-// maximum of the packed key (score << 6) | (63 - rank): one redux.sync when the
-// warp's sums fit 26 bits, five 64-bit shuffles otherwise.
+// sits in shared memory (one block per SM, so it is copied once per SM), with
+// one extra row of zeros that the picks of an invalid token point to; a warp
+// stages the picks of 32 tokens in shared memory and then scores them one at a
+// time, every lane reading the token's picks with broadcast loads.  The argmax
+// on (score desc, rank asc) is a maximum of the packed key
+// (score << 6) | (63 - rank).  When G is even and k times the largest table
+// entry stays below 2^26 (checked once per block while copying), lane l owns
+// ranks 2l and 2l+1, reads both with one 8-byte load per pick, sums in 32 bits
+// and takes the maximum with one redux.sync: about 45 instructions per token.
+// Otherwise lane l owns ranks l and l+32 with uint64 sums, and the maximum is
+// one redux.sync when the warp's sums fit 26 bits, five 64-bit shuffles if not.
 #include <algorithm>
 
 #include "common.cuh"
@@ -56,11 +60,16 @@ __global__ void __launch_bounds__(kShuffleThreads)
 shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, const uint32_t *__restrict__ rs_g,
                        int32_t *__restrict__ target, int32_t *err)
 {
-    extern __shared__ __align__(16) uint32_t tab[];   // [E][G], then each warp's 32 tokens' picks
-    int *picks_all = reinterpret_cast<int *>(tab + ((E * G + 3) & ~3));
+    extern __shared__ __align__(16) uint32_t tab[];   // [E+1][G] (row E zeros), then each warp's picks
+    __shared__ uint32_t tab_max;
+    int *picks_all = reinterpret_cast<int *>(tab + (((E + 1) * G + 3) & ~3));
+    if (threadIdx.x == 0) tab_max = 0;
+    for (int i = threadIdx.x; i < G; i += kShuffleThreads) tab[E * G + i] = 0u;
+    __syncthreads();
     {   // copy the table: 16-byte vectors where the layout allows, 8 in flight per thread
         const int n = E * G;
         const bool vec = (n % 4 == 0) && ((reinterpret_cast<uintptr_t>(rs_g) & 15u) == 0);
+        uint32_t mx = 0;
         if (vec) {
             const uint4 *src = reinterpret_cast<const uint4 *>(rs_g);
             uint4 *dst = reinterpret_cast<uint4 *>(tab);
@@ -71,13 +80,24 @@ shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, con
                     if (i0 + u * kShuffleThreads < n / 4) v[u] = __ldg(src + i0 + u * kShuffleThreads);
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
-                    if (i0 + u * kShuffleThreads < n / 4) dst[i0 + u * kShuffleThreads] = v[u];
+                    if (i0 + u * kShuffleThreads < n / 4) {
+                        dst[i0 + u * kShuffleThreads] = v[u];
+                        mx = max(max(mx, max(v[u].x, v[u].y)), max(v[u].z, v[u].w));
+                    }
             }
         } else {
-            for (int i = threadIdx.x; i < n; i += kShuffleThreads) tab[i] = __ldg(rs_g + i);
+            for (int i = threadIdx.x; i < n; i += kShuffleThreads) {
+                const uint32_t v = __ldg(rs_g + i);
+                tab[i] = v;
+                mx = max(mx, v);
+            }
         }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if ((threadIdx.x & 31) == 0) atomicMax(&tab_max, mx);
     }
     __syncthreads();
+    // sums of K entries fit 26 bits: 32-bit sums and one redux per token
+    const bool narrow = (G % 2 == 0) && (unsigned long long)tab_max * K < (1ull << 26);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     constexpr int KP = (K + 3) & ~3;                  // picks per token in shared memory, padded to int4
     int *picks = picks_all + warp * 32 * KP;
@@ -97,12 +117,40 @@ shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, con
                 if (j < K && (unsigned)e[j] >= (unsigned)E) { ok = false; }
             }
             if (tl < T && !ok) record_error(err, MOE_DERR_ID_RANGE);
+            // an invalid token (or a padding pick) points to the zero row: score 0 everywhere, rank 0
 #pragma unroll
-            for (int j = 0; j < KP; ++j) picks[lane * KP + j] = (ok && j < K) ? e[j] : -1;
+            for (int j = 0; j < KP; ++j) picks[lane * KP + j] = (ok && j < K) ? e[j] : E;
         }
         __syncwarp();
         const int n = min(32, T - t0);
         int result = 0;
+        if (narrow) {
+            const bool mine = 2 * lane < G;
+            const uint32_t k0 = (uint32_t)(63 - 2 * lane), k1 = (uint32_t)(62 - 2 * lane);
+            for (int i = 0; i < n; ++i) {
+                int e[KP];
+#pragma unroll
+                for (int q = 0; q < KP / 4; ++q) {
+                    const int4 v = reinterpret_cast<const int4 *>(picks + i * KP)[q];
+                    e[4 * q] = v.x; e[4 * q + 1] = v.y; e[4 * q + 2] = v.z; e[4 * q + 3] = v.w;
+                }
+                uint32_t s0 = 0, s1 = 0;
+                if (mine) {
+#pragma unroll
+                    for (int j = 0; j < K; ++j) {
+                        const uint2 v = reinterpret_cast<const uint2 *>(tab + (size_t)e[j] * G)[lane];
+                        s0 += v.x;
+                        s1 += v.y;
+                    }
+                }
+                const uint32_t key = mine ? max((s0 << 6) | k0, (s1 << 6) | k1) : 0u;
+                const int bi = 63 - (int)(__reduce_max_sync(0xffffffffu, key) & 63u);
+                if (lane == i) result = bi;
+            }
+            if (tl < T) target[tl] = result;
+            __syncwarp();
+            continue;
+        }
         for (int i = 0; i < n; ++i) {
             int e[KP];
 #pragma unroll
@@ -113,11 +161,9 @@ shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, con
             unsigned long long a0 = 0, a1 = 0;
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-                if (e[j] >= 0) {
-                    const uint32_t *row = tab + (size_t)e[j] * G;
-                    if (lane < G) a0 += row[lane];
-                    if (lane + 32 < G) a1 += row[lane + 32];
-                }
+                const uint32_t *row = tab + (size_t)e[j] * G;
+                if (lane < G) a0 += row[lane];
+                if (lane + 32 < G) a1 += row[lane + 32];
             }
             // packed key (score << 6) | (63 - rank): the maximum is the best
             // rank, the lowest rank among equal scores
@@ -134,7 +180,7 @@ shuffle_targets_kernel(const int32_t *__restrict__ ids, int T, int E, int G, con
                 for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
                 bi = 63 - (int)(best & 63u);
             }
-            if (lane == i) result = e[0] >= 0 ? bi : 0;
+            if (lane == i) result = bi;
         }
         if (tl < T) target[tl] = result;
         __syncwarp();
@@ -161,7 +207,7 @@ static moe_status launch_shuffle(const int32_t *ids, int T, int E, int G, const 
                                  int32_t *err, cudaStream_t s)
 {
     constexpr int KP = (K + 3) & ~3;
-    const size_t smem = sizeof(uint32_t) * (size_t)((E * G + 3) & ~3) + sizeof(int) * (kShuffleThreads / 32) * 32 * KP;
+    const size_t smem = sizeof(uint32_t) * (size_t)(((E + 1) * G + 3) & ~3) + sizeof(int) * (kShuffleThreads / 32) * 32 * KP;
     if (allow_smem(shuffle_targets_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
     // one block per SM at most: every block first copies the whole table
     const long long need = ((long long)T + kShuffleThreads - 1) / kShuffleThreads;

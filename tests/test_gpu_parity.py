@@ -227,6 +227,33 @@ def test_shuffle_small(cap, T, k, E, G):
     assert (host(z)[:T] == 0).all()
 
 
+@pytest.mark.parametrize("G", [1, 2, 3, 5, 32, 63, 64])
+@pytest.mark.parametrize("scale", ["small", "edge_narrow", "edge_wide", "huge"])
+def test_shuffle_table_ranges(cap, G, scale):
+    """Both scoring paths: 32-bit sums with one redux when G is even and k
+    times the table maximum stays below 2^26, 64-bit sums otherwise (odd G,
+    the boundary either side, entries up to 2^32 - 1); ties go to the lowest
+    rank; an invalid token scores 0 everywhere (rank 0, error recorded)."""
+    T, k, E = 3000, 8, 16 * max(1, 64 // max(G, 1))
+    rng = np.random.default_rng(G * 7 + len(scale))
+    ids = clustered_ids(rng, 1, T, E, k)[0]
+    top = {"small": 1000, "edge_narrow": ((1 << 26) - 1) // k, "edge_wide": ((1 << 26) - 1) // k + 1,
+           "huge": (1 << 32) - 1}[scale]
+    tab = rng.integers(0, top + 1, (E, G), dtype=np.int64)
+    tab[rng.integers(0, E), rng.integers(0, G)] = top                  # the maximum is reached
+    tab[:, G // 2:] = tab[:, :1] if G > 1 and scale == "small" else tab[:, G // 2:]   # many equal scores
+    tab = tab.astype(np.uint32)
+    ids[5, 3] = E + 7                                                   # one invalid token
+    err = cap.new_err("cuda")
+    tg = host(cap.shuffle_targets(dev(ids), E, G, dev(tab), err=err))[:T]
+    ids_ok = ids.copy()
+    ids_ok[5] = np.arange(k)                                            # the oracle scores valid tokens only
+    want = orc.shuffle_targets(ids_ok, E, G, tab)
+    want[5] = 0
+    assert (tg == want).all()
+    assert int(host(err)[0]) == cap.DERR_ID_RANGE
+
+
 # --------------------------------------------------------------- full pipeline
 
 ROW_WORKLOADS = ["tiny", "one_node", "ep32", "large_ep64"]
