@@ -18,7 +18,8 @@
 // (score << 6) | (63 - rank).  When G is even and k times the largest table
 // entry stays below 2^26 (checked once per block while copying), lane l owns
 // ranks 2l and 2l+1, reads both with one 8-byte load per pick, sums in 32 bits
-// and takes the maximum with one redux.sync: about 45 instructions per token.
+// and takes the maximum with one redux.sync: 57 warp instructions per token
+// against 170 for the general path (ncu counts on 131072 tokens, G = 64).
 // Otherwise lane l owns ranks l and l+32 with uint64 sums, and the maximum is
 // one redux.sync when the warp's sums fit 26 bits, five 64-bit shuffles if not.
 #include <algorithm>
