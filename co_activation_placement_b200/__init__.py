@@ -123,6 +123,12 @@ def _dev(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None):
     return t
 
 
+def _need(cond: bool, what: str):
+    """Shape agreement between the tensors of one call (checked before anything is enqueued)."""
+    if not cond:
+        raise ValueError(what)
+
+
 class Workspace:
     """A growable device byte buffer, 256-byte aligned (torch allocations are)."""
 
@@ -344,8 +350,11 @@ def permute(x: torch.Tensor, row_of: torch.Tensor, R_max: int, send: Optional[to
     _dev(row_of, torch.int32, "row_of", 2)
     T, d = x.shape
     k = row_of.shape[1]
+    _need(row_of.shape[0] >= T, "row_of needs a row per token of x")
     if send is None:
         send = torch.empty((max(R_max, 1), d), dtype=x.dtype, device=x.device)
+    _need(send.dim() == 2 and send.shape[0] >= R_max and send.shape[1] == d and send.dtype == x.dtype
+          and send.is_contiguous(), "send must be a contiguous [R_max][d] tensor of x's dtype")
     err = new_err(x.device) if err is None else err
     st = lib().moe_permute(_ptr(x), _dtype_code(x.dtype), T, d, k, _ptr(row_of), R_max, _ptr(send), _ptr(err),
                            _stream(x))
@@ -361,8 +370,11 @@ def combine(Y: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, out_dtype=torch
     _dev(w, torch.float32, "w", 2)
     T, k = idx.shape
     R_max, d = Y.shape
+    _need(w.shape[0] >= T and w.shape[1] == k, "w needs a weight per (token, pick) of idx")
     if out is None:
         out = torch.empty((T, d), dtype=out_dtype, device=Y.device)
+    _need(out.dim() == 2 and out.shape[0] >= T and out.shape[1] == d and out.is_contiguous(),
+          "out must be a contiguous [T][d] tensor")
     err = new_err(Y.device) if err is None else err
     st = lib().moe_combine(_ptr(Y), _dtype_code(Y.dtype), R_max, d, _ptr(idx), _ptr(w), T, k, _ptr(out),
                            _dtype_code(out.dtype), _ptr(err), _stream(Y))
@@ -379,6 +391,7 @@ def dispatch_gates(ids: torch.Tensor, w: torch.Tensor, plan: Plan, send_e: Optio
     _dev(w, torch.float32, "w", 2)
     T, k = ids.shape
     R_max = plan.R_max
+    _need(w.shape[0] >= T and w.shape[1] == k, "w needs a weight per (token, pick) of ids")
     if send_e is None:
         send_e = torch.empty((max(R_max, 1), k), dtype=torch.int32, device=ids.device)
     if send_w is None:
@@ -400,8 +413,12 @@ def expert_reduce(send: torch.Tensor, summary: torch.Tensor, send_e: torch.Tenso
     _dev(scale, torch.float32, "scale", 1)
     R_max, d = send.shape
     k = send_e.shape[1]
+    _need(send_e.shape[0] >= R_max and tuple(send_w.shape) == tuple(send_e.shape),
+          "send_e and send_w need k entries per row of send")
     if y is None:
         y = torch.empty((R_max, d), dtype=y_dtype or send.dtype, device=send.device)
+    _need(y.dim() == 2 and y.shape[0] >= R_max and y.shape[1] == d and y.is_contiguous(),
+          "y must be a contiguous [R_max][d] tensor")
     err = new_err(send.device) if err is None else err
     st = lib().moe_expert_reduce(_ptr(send), _dtype_code(send.dtype), R_max, d, _ptr(summary), _ptr(send_e),
                                  _ptr(send_w), k, _ptr(scale), scale.numel(), _ptr(y), _dtype_code(y.dtype),
@@ -419,6 +436,8 @@ def combine_rows(Y: torch.Tensor, row_of: torch.Tensor, out_dtype=torch.float32,
     R_max, d = Y.shape
     if out is None:
         out = torch.empty((T, d), dtype=out_dtype, device=Y.device)
+    _need(out.dim() == 2 and out.shape[0] >= T and out.shape[1] == d and out.is_contiguous(),
+          "out must be a contiguous [T][d] tensor")
     err = new_err(Y.device) if err is None else err
     st = lib().moe_combine_rows(_ptr(Y), _dtype_code(Y.dtype), R_max, d, _ptr(row_of), T, k, _ptr(out),
                                 _dtype_code(out.dtype), _ptr(err), _stream(Y))
@@ -455,6 +474,8 @@ def ep_permute(x: torch.Tensor, row_of: torch.Tensor, R_max: int, route: torch.T
     _dev(recv_base, torch.int64, "recv_base", 1)
     T, d = x.shape
     k = row_of.shape[1]
+    _need(row_of.shape[0] >= T, "row_of needs a row per token of x")
+    _need(recv_base.numel() == W, "recv_base needs one address per device")
     err = new_err(x.device) if err is None else err
     st = lib().moe_ep_permute(_ptr(x), _dtype_code(x.dtype), T, d, k, _ptr(row_of), R_max, _ptr(route), G, W,
                               _ptr(recv_base), recv_cap, _ptr(err), _stream(x))
@@ -472,6 +493,9 @@ def ep_combine(y_base: torch.Tensor, y_dtype, y_cap: int, d: int, route: torch.T
         _dev(w, torch.float32, "w", 2)
     _dev(out, out.dtype, "out", 2)
     T, k = idx.shape
+    _need(w is None or (w.shape[0] >= T and w.shape[1] == k), "w needs a weight per (token, pick) of idx")
+    _need(out.shape[0] >= T and out.shape[1] == d, "out must be a [T][d] tensor")
+    _need(y_base.numel() == W, "y_base needs one address per device")
     err = new_err(out.device) if err is None else err
     st = lib().moe_ep_combine(_ptr(y_base), _dtype_code(y_dtype), y_cap, d, _ptr(route), G, W, R_max, _ptr(idx),
                               _ptr(w), T, k, _ptr(out), _dtype_code(out.dtype), _ptr(err), _stream(out))
@@ -487,6 +511,7 @@ def ep_scatter_rows(src: torch.Tensor, route: torch.Tensor, G: int, W: int, dst_
     _dev(dst_base, torch.int64, "dst_base", 1)
     R_max = src.shape[0]
     row_bytes = src[0].numel() * src.element_size() if R_max else 4
+    _need(dst_base.numel() == W, "dst_base needs one address per device")
     err = new_err(src.device) if err is None else err
     st = lib().moe_ep_scatter_rows(_ptr(src), row_bytes, R_max, _ptr(route), G, W, _ptr(dst_base), dst_cap,
                                    _ptr(err), _stream(src))
