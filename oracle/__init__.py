@@ -61,6 +61,7 @@ def lib():
             "orc_plan_ranks": [P, i, i, i, i, i, P, P, P, P, P, P, P, P, P],
             "orc_place_replicas": [P, i, i, i, P, i, P, P],
             "orc_assign_replicas": [P, i, i, i, i, i, P, P, P, P, P],
+            "orc_ep_routes": [P, P, i, i, i, P],
         }
         for name, args in sig.items():
             f = getattr(_lib, name)
@@ -284,3 +285,13 @@ def assign_replicas(ids_l, E: int, G: int, rpn: int, replica_rank, n_rep, src_ra
     _check("orc_assign_replicas", lib().orc_assign_replicas(_p(ids_l), T, k, E, G, rpn, _p(rr), _p(nr), _p(src),
                                                             _p(pr), _p(nrem)))
     return pr, nrem
+
+
+def ep_routes(counts_all, offsets, G: int, W: int, me: int) -> np.ndarray:
+    """int64 [2*G*(G/W) + 2]: device me's route table (rows received, its
+    segments' first local rows, its R, the shifts to the receiving buffers)."""
+    c = np.ascontiguousarray(counts_all, dtype=np.int32)
+    o = np.ascontiguousarray(offsets, dtype=np.int32)
+    route = np.empty(2 * G * (G // W) + 2, np.int64)
+    _check("orc_ep_routes", lib().orc_ep_routes(_p(c), _p(o), G, W, me, _p(route)))
+    return route

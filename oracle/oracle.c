@@ -750,3 +750,43 @@ int orc_assign_replicas(const int32_t *ids, int T, int k, int E, int G, int rpn,
     }
     return ORC_OK;
 }
+
+/* Expert parallelism over W devices ([EC] abstract: each token is sent to each
+ * GPU once; reading taken: device h hosts ranks h*Gl .. h*Gl+Gl-1, Gl = G/W,
+ * and its receive buffer holds its ranks' rows in the one-device order --
+ * destination rank, source rank, token).  From every source rank's row counts
+ * counts_all[s][r] and device me's own plan offsets (its tokens only), the
+ * route of each of me's segments (r, s), s among me's ranks:
+ *   route[0]       rows device me receives,
+ *   route[1+i]     first local row of segment i = r*Gl + (s - me*Gl),
+ *   route[1+P]     me's row count R (P = G*Gl segments),
+ *   route[P+2+i]   row of the segment's first row in device r/Gl's buffer
+ *                  minus its local row.
+ * Written as the definition: the one-device offsets are the running sum of
+ * the counts in (r, s) order; a device's buffer starts at the offset of its
+ * first rank. */
+int orc_ep_routes(const int32_t *counts_all, const int32_t *offsets, int G, int W, int me, int64_t *route)
+{
+    if (G < 1 || G > 64 || W < 1 || G % W || me < 0 || me >= W) return ORC_ERR_ARG;
+    const int Gl = G / W, P = G * Gl;
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(G * G + 1));
+    if (!off) return ORC_ERR_ARG;
+    int64_t run = 0;
+    for (int r = 0; r < G; ++r)
+        for (int s = 0; s < G; ++s) {
+            off[r * G + s] = run;
+            run += counts_all[s * G + r];
+        }
+    off[G * G] = run;
+    route[0] = off[(me + 1) * Gl * G] - off[me * Gl * G];
+    for (int i = 0; i < P; ++i) {
+        const int r = i / Gl, s = me * Gl + i % Gl;
+        const int64_t first_local = offsets[r * G + s];
+        const int64_t first_global = off[r * G + s] - off[(r / Gl) * Gl * G];
+        route[1 + i] = first_local;
+        route[P + 2 + i] = first_global - first_local;
+    }
+    route[1 + P] = offsets[G * G];
+    free(off);
+    return ORC_OK;
+}

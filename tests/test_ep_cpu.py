@@ -36,31 +36,54 @@ def _local_plan(ids, E, G, rpn, e2r, W, h):
     return orc.plan(ids[h * Tl:(h + 1) * Tl], E, G, rpn, e2r, src_rank=src)
 
 
+def test_routes_hand_worked():
+    """G = 2 ranks on W = 2 devices.  Source rank 0 sends 3 rows to rank 0 and
+    1 to rank 1; source rank 1 sends 2 and 4.  One-device order (r, s): rank
+    0's buffer is rows 0-2 from s 0 then 3-4 from s 1 (5 rows); rank 1's is
+    row 0 from s 0 then rows 1-4 from s 1.  Device 0's own plan has local
+    rows 0-2 for rank 0 and row 3 for rank 1: rows 0-2 stay in place, row 3
+    becomes row 0 of device 1."""
+    counts_all = np.array([[3, 1], [2, 4]], np.int32)
+    local0 = np.array([0, 3, 3, 4, 4], np.int32)           # offsets (r, s): (0,0) (0,1) (1,0) (1,1), R
+    assert orc.ep_routes(counts_all, local0, 2, 2, 0).tolist() == [5, 0, 3, 4, 0, -3]
+    local1 = np.array([0, 0, 2, 2, 6], np.int32)           # device 1 plans source rank 1 only
+    # segments (r=0, s=1) at local row 0 -> device 0 row 3; (r=1, s=1) at local row 2 -> device 1 row 1
+    assert orc.ep_routes(counts_all, local1, 2, 2, 1).tolist() == [5, 0, 2, 6, 3, -1]
+
+
 @pytest.mark.parametrize("T,E,k,G,rpn,W", [(512, 16, 2, 4, 2, 2), (1536, 64, 6, 32, 8, 4), (960, 24, 5, 12, 4, 3),
                                             (1024, 64, 3, 64, 8, 64), (640, 32, 4, 8, 8, 1)])
 def test_route_definition(T, E, k, G, rpn, W):
+    """The oracle's route tables move every local row of every device onto the
+    one-device plan's row for the same token and rank, each row once."""
     ids = _ids(T + W, T, E, k)
     e2r = np.random.default_rng(G).permutation(np.arange(E, dtype=np.int32) // (E // G)).astype(np.int32)
     o = orc.plan(ids, E, G, rpn, e2r)
     off_g = o["offsets"].astype(np.int64)
     Gl, Tl = G // W, T // W
+    P = G * Gl
+    plans = [_local_plan(ids, E, G, rpn, e2r, W, h) for h in range(W)]
+    counts_all = np.concatenate([plans[h]["counts"][h * Gl:(h + 1) * Gl] for h in range(W)])
+    assert (counts_all == o["counts"]).all()
     seen = np.zeros(o["R"], bool)
-    for h in range(W):
-        lo = _local_plan(ids, E, G, rpn, e2r, W, h)
-        off_l = lo["offsets"].astype(np.int64)
+    for h, lo in enumerate(plans):
+        route = orc.ep_routes(counts_all, lo["offsets"], G, W, h)
+        assert route[0] == off_g[(h + 1) * Gl * G] - off_g[h * Gl * G]
+        assert route[1 + P] == lo["R"]
+        start = route[1:P + 2]
         for x in range(lo["R"]):
-            seg = int(np.searchsorted(off_l, x, side="right")) - 1     # (r, s) = divmod(seg, G)
-            r, s = divmod(seg, G)
-            assert h * Gl <= s < (h + 1) * Gl                            # only this device's sources
-            q = x + off_g[r * G + s] - off_g[(r // Gl) * Gl * G] - off_l[seg]
-            g = off_g[(r // Gl) * Gl * G] + q                            # the one-device row
-            assert off_g[r * G + s] <= g < off_g[r * G + s + 1]
+            i = int(np.searchsorted(start, x, side="right")) - 1      # the segment holding local row x
+            r, s = i // Gl, h * Gl + i % Gl
+            q = x + route[P + 2 + i]                                    # its row in device r/Gl's buffer
+            g = off_g[(r // Gl) * Gl * G] + q                           # the one-device row
+            assert 0 <= q and off_g[r * G + s] <= g < off_g[r * G + s + 1]
             assert o["row_token"][g] == h * Tl + lo["row_token"][x]
+            assert (o["row_jmask"][g] == lo["row_jmask"][x])
             assert not seen[g]
             seen[g] = True
-        rows_h = off_g[(h + 1) * Gl * G] - off_g[h * Gl * G]
-        assert rows_h == sum(int(c) for c in o["counts"][:, h * Gl:(h + 1) * Gl].ravel())
-    assert seen.all()                                                    # every row arrives exactly once
+        if W == 1:
+            assert (route[P + 2:] == 0).all()                          # one device: the routes are the identity
+    assert seen.all()                                                   # every row arrives exactly once
 
 
 def _free_port():

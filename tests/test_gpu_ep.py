@@ -6,8 +6,8 @@ oracle's one-device plan over all tokens (contiguous source ranks):
   - device h's receive buffer holds that plan's send rows
     [offsets[h*Gl*G], offsets[(h+1)*Gl*G]) bit for bit, and so do the
     dispatched gate records;
-  - the route table equals the one recomputed here from the oracle's
-    per-device plans and its one-device offsets;
+  - the route table equals the oracle's (orc.ep_routes on the device's
+    oracle plan and the gathered counts);
   - the combined outputs lie within the combine's rounding bound of the
     oracle's fp64 combine, and equal the one-device CUDA combine bit for bit
     (same fp32 operations in the same order).
@@ -68,26 +68,15 @@ def combine_bound(Yf, idx, w, k):
 
 
 def expected_routes(ids, E, G, rpn, e2r, W, o_global):
-    """The route tables from the definition: per device, its oracle plan's
-    segment starts and the shift to the one-device row minus the device's
-    first row."""
-    T, k = ids.shape
+    """The oracle's route tables: per device, from its own oracle plan and the
+    gathered counts (the one-device plan's counts)."""
+    T = ids.shape[0]
     Gl, Tl = G // W, T // W
-    off_g = o_global["offsets"].astype(np.int64)
-    P = G * Gl
     out = []
     for h in range(W):
         src = (h * Gl + np.arange(Tl) // (Tl // Gl)).astype(np.int32)
         o = orc.plan(ids[h * Tl:(h + 1) * Tl], E, G, rpn, e2r, src_rank=src)
-        off_l = o["offsets"].astype(np.int64)
-        r = np.empty(2 * P + 2, np.int64)
-        r[0] = off_g[(h + 1) * Gl * G] - off_g[h * Gl * G]
-        for i in range(P):
-            rr, s = i // Gl, h * Gl + i % Gl
-            r[1 + i] = off_l[rr * G + s]
-            r[P + 2 + i] = off_g[rr * G + s] - off_g[(rr // Gl) * Gl * G] - off_l[rr * G + s]
-        r[1 + P] = off_l[G * G]
-        out.append(r)
+        out.append(orc.ep_routes(o_global["counts"], o["offsets"], G, W, h))
     return out
 
 

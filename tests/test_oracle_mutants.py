@@ -14,7 +14,8 @@ from conftest import ROOT
 
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_pins.py", "tests/test_oracle_brute.py", "tests/test_oracle_prereduce.py",
-        "tests/test_oracle_replicas.py", "tests/test_oracle_shuffle_balanced.py", "tests/test_oracle_ema.py", "tests/test_oracle_capped.py"]
+        "tests/test_oracle_replicas.py", "tests/test_oracle_shuffle_balanced.py", "tests/test_oracle_ema.py", "tests/test_oracle_capped.py",
+        "tests/test_ep_cpu.py::test_routes_hand_worked", "tests/test_ep_cpu.py::test_route_definition"]
 
 MUTANTS = {
     "counts_drop_diagonal": ("                for (int a = 0; a < k; ++a)\n                    for (int b = 0; b < k; ++b)\n"
@@ -69,6 +70,9 @@ MUTANTS = {
     "capped_forced_pick_heaviest": ("if (pick < 0 || C[(size_t)pool[x] * E + pool[x]] < C[(size_t)pool[pick] * E + pool[pick]])",
                                     "if (pick < 0 || C[(size_t)pool[x] * E + pool[x]] > C[(size_t)pool[pick] * E + pool[pick]])"),
     "capped_cap_ignored": ("if (cap >= 0.0 && (double)(load + nx) > cap) continue;", "(void)nx;"),
+    "ep_routes_counts_transposed": ("run += counts_all[s * G + r];", "run += counts_all[r * G + s];"),
+    "ep_routes_sender_base": ("const int64_t first_global = off[r * G + s] - off[(r / Gl) * Gl * G];",
+                              "const int64_t first_global = off[r * G + s] - off[me * Gl * G];"),
 }
 
 
