@@ -71,8 +71,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="large_ep64")
-    ap.add_argument("--placement", default="correlated", choices=["correlated", "uniform", "capacity", "capped"],
-                    help="capped: correlated with every rank's load within 1.1 x the average")
+    ap.add_argument("--placement", default=None, choices=["correlated", "uniform", "capacity", "capped"],
+                    help="default: uniform for the tiny workload (its stated placement), correlated otherwise; "
+                         "capped: correlated with every rank's load within 1.1 x the average")
     ap.add_argument("--no-shuffle", action="store_true")
     ap.add_argument("--balanced-shuffle", action="store_true",
                     help="cap every rank's shard at T/G tokens (capacity-balanced shuffle targets)")
@@ -325,6 +326,8 @@ def main():
     a = parse()
     from synth import WORKLOADS
     w = WORKLOADS[a.workload]
+    if a.placement is None:
+        a.placement = "uniform" if w.name == "tiny" else "correlated"
     if a.impl == "reference":
         run_reference(a, w)
         return
