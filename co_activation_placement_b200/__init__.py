@@ -7,10 +7,13 @@ path is computed in Python or by torch.  If the shared library is missing the
 import of any entry point raises: there is no fallback.
 
 Entry points (names follow the C ABI without the ``moe_`` prefix):
-  coact_stats, plan_dispatch, permute, combine, rank_score, shuffle_targets,
+  coact_stats, coact_stats_method, coact_stats_path, coact_ema,
+  plan_dispatch, permute, combine, rank_score, shuffle_targets, shuffle_balanced,
   dispatch_gates, expert_reduce, combine_rows,
   place_replicas, assign_replicas, plan_dispatch_ranks,
-  place_uniform, place_capacity, place_correlated, launch_count.
+  ep_routes, ep_permute, ep_combine, ep_scatter_rows (ranks over several devices),
+  place_uniform, place_capacity, place_correlated, place_correlated_capped,
+  selftest_wait_timeout, launch_count.
 """
 from __future__ import annotations
 
