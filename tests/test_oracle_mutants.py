@@ -15,7 +15,8 @@ from conftest import ROOT
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_pins.py", "tests/test_oracle_brute.py", "tests/test_oracle_prereduce.py",
         "tests/test_oracle_replicas.py", "tests/test_oracle_shuffle_balanced.py", "tests/test_oracle_ema.py", "tests/test_oracle_capped.py",
-        "tests/test_ep_cpu.py::test_routes_hand_worked", "tests/test_ep_cpu.py::test_route_definition"]
+        "tests/test_ep_cpu.py::test_routes_hand_worked", "tests/test_ep_cpu.py::test_route_definition",
+        "tests/test_oracle_property.py"]
 
 MUTANTS = {
     "counts_drop_diagonal": ("                for (int a = 0; a < k; ++a)\n                    for (int b = 0; b < k; ++b)\n"
