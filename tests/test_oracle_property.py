@@ -88,3 +88,35 @@ def test_routes_cover_the_one_device_rows(orc, shape):
             seen[g] += 1
         assert route[0] == sum(int(o["counts"][s_, r_]) for s_ in range(G) for r_ in range(h * Gl, (h + 1) * Gl))
     assert (seen == 1).all()
+
+
+@SETTINGS
+@given(shapes(), st.integers(0, 3))
+def test_balanced_shuffle_matches_deferred_acceptance(orc, shape, slack):
+    """The greedy over one pair order (the oracle) and token-proposing
+    deferred acceptance (the brute force) reach the same, stable assignment
+    for any capacity that can hold all tokens."""
+    T, E, k, G, rpn, W, _, seed = shape
+    rng = np.random.default_rng(seed)
+    ids = _routing(rng, 1, T, E, k)[0]
+    rs = rng.integers(0, 4, (E, G)).astype(np.uint32)          # small scores: many ties
+    capacity = -(-T // G) + slack
+    got = orc.shuffle_balanced(ids, E, G, rs, capacity).tolist()
+    assert got == brute.shuffle_balanced_da(ids.tolist(), G, rs.tolist(), capacity)
+    assert brute.blocking_pairs(ids.tolist(), G, rs.tolist(), capacity, got) == []
+    assert max(np.bincount(np.array(got), minlength=G)) <= capacity
+
+
+@SETTINGS
+@given(st.sampled_from([(4, 2, 1), (8, 4, 2), (12, 6, 3), (16, 8, 4), (12, 4, 4), (16, 4, 1)]),
+       st.integers(0, 2 ** 31), st.sampled_from([-1.0, 0.0, 0.1, 0.5]))
+def test_correlated_placement_matches_brute(orc, egr, seed, eps):
+    """The greedy grouping (with and without a load tolerance) equals its
+    pure-Python restatement on random symmetric co-activation counts."""
+    E, G, rpn = egr
+    rng = np.random.default_rng(seed)
+    ids = _routing(rng, 1, 200, E, min(4, E))
+    C = orc.coact(ids, E)["coact"][0]
+    want = brute.place_correlated(C.tolist(), G, rpn, eps)
+    got = orc.place_correlated_capped(C, G, rpn, eps) if eps >= 0 else orc.place_correlated(C, G, rpn)
+    assert got.tolist() == list(want)
