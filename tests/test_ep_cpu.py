@@ -146,3 +146,46 @@ def test_ep_collectives_gloo(world):
     assert all(r[1] for r in res), "summed statistics differ from the whole batch's"
     assert all(r[2] for r in res), "Ochiai on the summed counts differs"
     assert all(r[3] for r in res), "gathered counts differ from the one-device plan's"
+
+
+def _lost_rank_worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    from co_activation_placement_b200 import ep
+    flag = torch.zeros(1, dtype=torch.int32)
+    ep.meet(flag)                                   # everyone present once
+    if rank == world - 1:
+        q.put((rank, "left"))                       # this rank stops taking part: it never meets again
+        q.close()
+        q.join_thread()                             # the message is out before the process ends
+        os._exit(0)
+    try:
+        ep.meet(flag)
+        q.put((rank, "met"))
+    except Exception as ex:                          # the others learn of it from the meeting itself
+        q.put((rank, "error: " + type(ex).__name__))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_meet_reports_a_lost_rank(world):
+    """A rank that stops taking part between steps (host-side failure, no GPU
+    involved): the other ranks' next meeting ends with an error instead of
+    waiting for ever (the process group's timeout or the closed connection)."""
+    import time
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_lost_rank_worker, args=(r, world, port, q)) for r in range(world)]
+    t0 = time.time()
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+    assert res[world - 1] == "left"
+    assert all(res[r].startswith("error") for r in range(world - 1)), res
+    assert time.time() - t0 < 100
