@@ -170,3 +170,26 @@ def test_place_correlated_capped_matches_oracle(cap, orc, eps):
     C = np.triu(C, 1)
     C = (C + C.T + np.diag(rng.integers(1000, 90000, 256))).astype(np.uint32)
     assert (cap.place_correlated_capped(C, 64, 8, eps) == orc.place_correlated_capped(C, 64, 8, eps)).all()
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/moe_coact.h is a C header: a C99 translation unit that includes
+    it and names its types and entry points compiles with warnings as errors."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if not gcc or not os.path.isdir(cuda_inc):
+        pytest.skip("gcc or the CUDA headers are not installed")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "moe_coact.h"\n'
+                   "int use(void) {\n"
+                   "    moe_plan p = {0};\n"
+                   "    moe_status (*f)(const int32_t *, int, int, int, int, uint32_t *, float *, uint32_t *,\n"
+                   "                    int32_t *, void *, size_t, cudaStream_t) = moe_coact_stats;\n"
+                   "    return (int)(p.counts == 0) + (f != 0) + (int)moe_launch_count();\n"
+                   "}\n")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        "-I", cuda_inc, "-c", str(src), "-o", str(tmp_path / "use_header.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
