@@ -193,3 +193,36 @@ def test_header_is_plain_c(tmp_path):
                         "-I", cuda_inc, "-c", str(src), "-o", str(tmp_path / "use_header.o")],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_c_program_links_and_calls_the_library(cap, tmp_path):
+    """A plain C program linked against libmoecoact.so calls a host entry
+    point through the C ABI alone (no Python): the uniform placement of 64
+    experts on 8 ranks, the pages' worked example (rank d holds 8d..8d+7)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if not gcc or not os.path.isdir(cuda_inc):
+        pytest.skip("gcc or the CUDA headers are not installed")
+    libdir = os.path.dirname(cap.LIB_PATH)
+    src = tmp_path / "place.c"
+    src.write_text('#include <stdio.h>\n#include "moe_coact.h"\n'
+                   "int main(void) {\n"
+                   "    int32_t e2r[64];\n"
+                   "    if (moe_place_uniform(64, 8, e2r) != MOE_OK) return 1;\n"
+                   "    if (moe_place_uniform(63, 8, e2r) != MOE_ERR_ARG) return 2;\n"
+                   "    for (int e = 0; e < 64; ++e) printf(\"%d \", e2r[e]);\n"
+                   "    printf(\"\\n%s\\n\", moe_status_string(MOE_ERR_ARG));\n"
+                   "    return 0;\n"
+                   "}\n")
+    exe = tmp_path / "place"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc,
+                        str(src), "-o", str(exe), "-L", libdir, "-l:libmoecoact.so", "-Wl,-rpath," + libdir],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr
+    ranks = [int(v) for v in run.stdout.split("\n")[0].split()]
+    assert ranks == [e // 8 for e in range(64)]
+    assert run.stdout.split("\n")[1].strip() != ""
