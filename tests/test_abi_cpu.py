@@ -226,3 +226,32 @@ def test_c_program_links_and_calls_the_library(cap, tmp_path):
     ranks = [int(v) for v in run.stdout.split("\n")[0].split()]
     assert ranks == [e // 8 for e in range(64)]
     assert run.stdout.split("\n")[1].strip() != ""
+
+
+def test_host_placements_match_oracle_on_random_inputs(cap, orc):
+    """The library's host placements (C++) against the oracle on 120 seeded
+    random shapes and co-activation matrices: uniform, capacity-aware,
+    correlated, capped, and replica layouts, bit for bit."""
+    rng = np.random.default_rng(2024)
+    for _ in range(120):
+        G = int(rng.choice([1, 2, 4, 6, 8, 16]))
+        rpn = int(rng.choice([r for r in range(1, G + 1) if G % r == 0]))
+        E = G * int(rng.integers(1, 6))
+        k = int(rng.integers(1, min(E, 6) + 1))
+        T = int(rng.integers(1, 300))
+        hot = rng.permutation(E)[: min(E, k + 2)]
+        ids = np.where((rng.random(T) < 0.6)[:, None],
+                       hot[np.argsort(rng.random((T, hot.size)), axis=1)[:, :k]],
+                       np.argsort(rng.random((T, E)), axis=1)[:, :k]).astype(np.int32)[None]
+        C = orc.coact(ids, E)["coact"][0]
+        assert (cap.place_uniform(E, G) == orc.place_uniform(E, G)).all()
+        load = np.diag(C).astype(np.float64)
+        assert (cap.place_capacity(load, G)[0] == orc.place_capacity(load, G)[0]).all()
+        assert (cap.place_correlated(C, G, rpn) == orc.place_correlated(C, G, rpn)).all()
+        eps = float(rng.choice([0.0, 0.05, 0.2]))
+        assert (cap.place_correlated_capped(C, G, rpn, eps) == orc.place_correlated_capped(C, G, rpn, eps)).all()
+        e2r = orc.place_correlated(C, G, rpn)
+        extra = int(rng.integers(0, 3))
+        got = cap.place_replicas(C, G, rpn, e2r, extra)
+        want = orc.place_replicas(C, G, rpn, e2r, extra)
+        assert (got[0] == want[0]).all() and (got[1] == want[1]).all()
