@@ -529,7 +529,8 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "dtype_note": "the combine accumulates in fp32; rows (x_dtype) are moved bit for bit; counts and plans are integer",
             "config": {"workload": w.name, "seed": seed, "T": w.T, "E": w.E, "k": w.k, "G": w.G, "rpn": w.rpn, "d": w.d,
                        "L": w.L, "x_dtype": w.dtype, "out_dtype": a.out_dtype, "placement": a.placement,
                        "combine": "receiver-side pre-reduced (stand-in experts)" if a.prereduce
@@ -766,7 +767,8 @@ def run_ep(a, w, rank, world, device, seed):
         print(json.dumps({
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "dtype_note": "the combine accumulates in fp32; rows (x_dtype) are moved bit for bit; counts and plans are integer",
             "config": {"workload": w.name, "seed": seed, "T_per_gpu": w.T, "E": w.E, "k": w.k, "G": w.G, "rpn": w.rpn,
                        "d": w.d, "L": w.L, "x_dtype": w.dtype, "out_dtype": a.out_dtype, "placement": a.placement,
                        "parallelism": "expert parallel over %d GPU(s), %d ranks each" % (world, Gl),
