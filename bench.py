@@ -85,6 +85,8 @@ def parse():
                     help="run plans, shuffle targets and statistics in line instead of on a second stream")
     ap.add_argument("--replicas", type=int, default=0, metavar="EXTRA",
                     help="replicate experts (EXTRA more per rank) and assign tasks to the fewest remote nodes")
+    ap.add_argument("--replica-eps", type=float, default=None, metavar="EPS",
+                    help="with --replicas: cap every rank's tasks at (1 + EPS) T k / G in the assignment")
     ap.add_argument("--prereduce", action="store_true",
                     help="receiver-side pre-reduced combine with stand-in experts (gates dispatched with rows)")
     ap.add_argument("--seed", type=int, default=None,
@@ -373,7 +375,7 @@ def main():
                           shuffle=shuffle, out_dtype=out_dtype, device=device, timers=True,
                           scales=make_expert_scales(w, seed=seed) if a.prereduce else None,
                           replica_extra=a.replicas, shuffle_capacity=w.T // w.G if balanced else 0,
-                          overlap=not a.no_overlap)
+                          overlap=not a.no_overlap, replica_eps=a.replica_eps)
     place = time_placement(cap, ids_cal, w, a.placement, device)
 
     def barrier():
@@ -536,6 +538,7 @@ def main():
                        "combine": "receiver-side pre-reduced (stand-in experts)" if a.prereduce
                                   else "source-side weighted (identity experts)",
                        "replicas_per_rank": a.replicas,
+                       "replica_eps": a.replica_eps if a.replicas else None,
                        "overlap": "plans, shuffle targets and statistics on a second stream"
                                   if hp.overlap else "none",
                        "shuffle": ("balanced (T/G tokens per rank)" if balanced else True) if shuffle else False,
@@ -555,6 +558,7 @@ def main():
                      "R_remote": [int(s[1]) for s in summaries],
                      "local_share": [int(s[2]) / (w.T * w.k) for s in summaries],
                      "V": [int(s[3]) for s in summaries]},
+            "replica_load": replica_load(hp, w),
             "clocks": clocks,
             "balanced_shuffle": {
                 "rounds": hp.shuffle_info[:, 0].tolist(), "proposals": hp.shuffle_info[:, 1].tolist(),
@@ -651,6 +655,16 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
             "placement_effect": effect}
 
 
+def replica_load(hp, w):
+    """Per-rank task loads the capped replica assignment returned (one row
+    per layer): busiest rank over the mean, next to V in "rows"."""
+    if not hp.replicas or hp.replica_eps is None:
+        return None
+    ld = hp.rank_load.cpu().double()
+    return {"eps": hp.replica_eps, "max_over_mean": [float(r.max() / r.mean()) for r in ld],
+            "max": [int(r.max()) for r in ld], "mean": [float(r.mean()) for r in ld]}
+
+
 def time_placement(cap, ids_cal, w, placement, device):
     """Host time of the placement from the calibration batch's counts (the
     step that runs once per re-layout, on one CPU thread): per layer, and the
@@ -714,11 +728,12 @@ def run_ep(a, w, rank, world, device, seed):
     # receive capacity and row counts: every layer planned once, counts gathered
     from co_activation_placement_b200.ep import EPShard, gather_counts
     sh = EPShard(world, rank, w.E, w.G, w.rpn, w.T, w.k, w.d, x.dtype, device)
-    need, R = 0, []
+    need, R, counts = 0, [], []
     for l in range(w.L):
         sh.plan_layer(ids[l], e2r[l])
         gather_counts(sh.counts_all, sh.my_counts())
         c = sh.counts_all.cpu().numpy().astype(np.int64)
+        counts.append(c.astype(np.int32))
         need = max(need, int(c[:, rank * Gl:(rank + 1) * Gl].sum()))
         R.append(int(sh.plan.summary[0].item()))
     del sh
@@ -778,10 +793,36 @@ def run_ep(a, w, rank, world, device, seed):
             "roofline": None,
             "roofline_note": "per-kernel events are not taken in this mode; the one-GPU path reports the kernels",
             "clocks": clk.summary(), "gpu_launches": int(n_launch), "e2e": None, "cpu_baseline": None,
+            "cross_device": exchange_record(cap, counts, w.G, world, w.d * x.element_size(), ms),
             "timing": "eager launches between two CUDA events, max over the GPUs",
         }), flush=True)
     del grp
     dist.destroy_process_group()
+
+
+NVLINK_GBS = 770.0   # measured peer copy per direction per GPU on this machine (the profiling recipe's figure)
+
+
+def exchange_record(cap, counts_layers, G, W, rowB, ms_step):
+    """Rows and bytes that cross devices in the exchange with the G ranks on W
+    devices (moe_ep_exchange_rows on each layer's gathered counts), and the
+    NVLink floor they set: per layer the busiest device sends or receives
+    max(sent_h, received_h) rows in the dispatch and again in the combine, at
+    NVLINK_GBS per direction."""
+    rows, busiest = [], []
+    for c in counts_layers:
+        sent, recv = cap.ep_exchange_rows(c, G, W)
+        rows.append(int(sent.sum()))
+        busiest.append(int(max(sent.max(), recv.max())))
+    floor_ms = sum(2.0 * b * rowB / (NVLINK_GBS * 1e9) * 1e3 for b in busiest)
+    busiest_bytes = sum(2 * b * rowB for b in busiest)
+    return {"devices": W, "rows_crossing_per_layer": rows, "bytes_each_way_per_step": sum(rows) * rowB,
+            "busiest_device_rows_per_layer": busiest,
+            "nvlink": {"bound": "nvlink", "peak": NVLINK_GBS, "unit": "GB/s",
+                       "peak_kind": "measured peer copy per direction (pool figure)",
+                       "busiest_device_bytes_per_step": busiest_bytes, "floor_ms_per_step": floor_ms,
+                       "achieved": busiest_bytes / (ms_step * 1e-3) / 1e9 if ms_step > 0 else None,
+                       "frac": floor_ms / ms_step if ms_step > 0 else None}}
 
 
 def run_ep_emulated(hp, w, W, steps, warmup, hbm, sb, pg):
@@ -827,8 +868,15 @@ def run_ep_emulated(hp, w, W, steps, warmup, hbm, sb, pg):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
     del g
+    counts = []
+    for l in range(w.L):                      # each layer's gathered counts, for the exchange record
+        emu.step(hp.ids[l], hp.x, hp.gates[l], hp.e2r[l])
+        counts.append(emu.shards[0].counts_all.cpu().numpy())
     nbytes = sb.permute + sb.combine
     return {"devices": W, "ranks_per_device": Gl, "tokens_per_device": w.T // W, "recv_rows_max": rows,
+            "exchange": exchange_record(cap, counts, w.G, W, w.d * hp.x.element_size(), ms),
+            "exchange_note": "the rows that would cross NVLink with the W devices on W GPUs; here they move "
+                             "within one GPU's memory, so the nvlink frac is the floor over the measured step",
             "ms_per_step": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
             "errors": emu.errors(),
             "note": "W virtual devices on this GPU, each with its own receive buffer, launched one after another; "

@@ -10,9 +10,9 @@ Entry points (names follow the C ABI without the ``moe_`` prefix):
   coact_stats, coact_stats_method, coact_stats_path, coact_ema,
   plan_dispatch, permute, combine, rank_score, shuffle_targets, shuffle_balanced,
   dispatch_gates, expert_reduce, combine_rows,
-  place_replicas, assign_replicas, plan_dispatch_ranks,
-  ep_routes, ep_permute, ep_combine, ep_scatter_rows (ranks over several devices),
-  place_uniform, place_capacity, place_correlated, place_correlated_capped,
+  place_replicas, assign_replicas, assign_replicas_capped, plan_dispatch_ranks,
+  ep_routes, ep_permute, ep_combine, ep_scatter_rows, ep_exchange_rows (ranks over several devices),
+  place_uniform, place_capacity, place_correlated, place_correlated_capped, rank_loads,
   selftest_wait_timeout, launch_count.
 """
 from __future__ import annotations
@@ -83,6 +83,10 @@ def lib() -> ctypes.CDLL:
             "moe_place_correlated_capped": ([P, i, i, i, ctypes.c_double, P], i),
             "moe_place_replicas": ([P, i, i, i, P, i, P, P], i),
             "moe_assign_replicas": ([P, i, i, i, i, i, P, P, P, P, P, P, P], i),
+            "moe_assign_replicas_capped_workspace": ([i], sz),
+            "moe_assign_replicas_capped": ([P, i, i, i, i, i, P, P, P, ctypes.c_double, P, P, P, P, P, sz, P], i),
+            "moe_rank_loads": ([P, i, i, P, P], i),
+            "moe_ep_exchange_rows": ([P, i, i, P, P], i),
             "moe_plan_dispatch_ranks": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
             "moe_ep_routes": ([P, P, i, i, i, P, P, P], i),
             "moe_ep_permute": ([P, i, i, i, i, P, i64, P, i, i, P, i64, P, P], i),
@@ -332,6 +336,40 @@ def assign_replicas(ids: torch.Tensor, E: int, G: int, rpn: int, replica_rank: t
                                    _ptr(pick_rank), _ptr(n_remote), _ptr(err), _stream(ids))
     _check("moe_assign_replicas", st)
     return pick_rank, n_remote
+
+
+def assign_replicas_capped_workspace(G: int) -> int:
+    return int(lib().moe_assign_replicas_capped_workspace(G))
+
+
+def assign_replicas_capped(ids: torch.Tensor, E: int, G: int, rpn: int, replica_rank: torch.Tensor,
+                           n_rep: torch.Tensor, eps: float, src_rank: Optional[torch.Tensor] = None,
+                           pick_rank: Optional[torch.Tensor] = None, n_remote: Optional[torch.Tensor] = None,
+                           rank_load: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None,
+                           ws: Optional[torch.Tensor] = None):
+    """(pick_rank int32 [T][k], n_remote int32 [T], rank_load int64 [G]): the
+    fewest-remote-nodes assignment with each rank's tasks capped at
+    floor((1 + eps) T k / G), tokens taken in id order."""
+    _dev(ids, torch.int32, "ids", 2)
+    _dev(replica_rank, torch.int32, "replica_rank", 2)
+    _dev(n_rep, torch.int32, "n_rep", 1)
+    T, k = ids.shape
+    dev = ids.device
+    if pick_rank is None:
+        pick_rank = torch.empty((max(T, 1), k), dtype=torch.int32, device=dev)
+    if n_remote is None:
+        n_remote = torch.empty(max(T, 1), dtype=torch.int32, device=dev)
+    if rank_load is None:
+        rank_load = torch.empty(G, dtype=torch.int64, device=dev)
+    err = new_err(dev) if err is None else err
+    need = int(lib().moe_assign_replicas_capped_workspace(G))
+    if ws is None:
+        ws = _workspace(dev, "capped").get(need)
+    st = lib().moe_assign_replicas_capped(_ptr(ids), T, k, E, G, rpn, _ptr(replica_rank), _ptr(n_rep),
+                                          _ptr(src_rank), float(eps), _ptr(pick_rank), _ptr(n_remote),
+                                          _ptr(rank_load), _ptr(err), _ptr(ws), ws.numel(), _stream(ids))
+    _check("moe_assign_replicas_capped", st)
+    return pick_rank, n_remote, rank_load
 
 
 # ---------------------------------------------------------------- rows
@@ -595,6 +633,27 @@ def place_capacity(load, G: int):
     dev = np.empty(G, np.float64)
     _check("moe_place_capacity", lib().moe_place_capacity(_np_ptr(load), load.size, G, _np_ptr(out), _np_ptr(dev)))
     return out, dev
+
+
+def ep_exchange_rows(counts_all, G: int, W: int):
+    """(sent int64 [W], received int64 [W]): rows that cross devices when the
+    G ranks are spread over W devices, from host counts int32 [G][G]."""
+    c = np.ascontiguousarray(counts_all, dtype=np.int32)
+    sent = np.empty(W, np.int64)
+    recv = np.empty(W, np.int64)
+    _check("moe_ep_exchange_rows", lib().moe_ep_exchange_rows(_np_ptr(c), G, W, _np_ptr(sent), _np_ptr(recv)))
+    return sent, recv
+
+
+def rank_loads(coact_l, expert_to_rank, G: int) -> np.ndarray:
+    """int64 [G]: tasks each rank serves under a one-replica placement (the
+    sum of n_e = C_ee over its experts), from host arrays."""
+    c = np.ascontiguousarray(coact_l, dtype=np.uint32)
+    E = c.shape[0]
+    e2r = np.ascontiguousarray(expert_to_rank, dtype=np.int32)
+    out = np.empty(G, np.int64)
+    _check("moe_rank_loads", lib().moe_rank_loads(_np_ptr(c), E, G, _np_ptr(e2r), _np_ptr(out)))
+    return out
 
 
 def place_correlated(coact_l, G: int, rpn: int) -> np.ndarray:

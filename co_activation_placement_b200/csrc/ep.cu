@@ -436,3 +436,25 @@ extern "C" moe_status moe_ep_scatter_rows(const void *src, int64_t row_bytes, in
     if (st == MOE_OK) note_launches(1);
     return st;
 }
+
+// Rows that cross devices in the exchange: sent[h] = rows from device h's
+// source ranks to other devices' ranks, received[h] = rows to device h's
+// ranks from other devices' sources; each such row crosses once in the
+// dispatch and once back in the combine.
+extern "C" moe_status moe_ep_exchange_rows(const int32_t *counts_all, int G, int W, long long *sent,
+                                           long long *received)
+{
+    if (!counts_all || !sent || !received || G < 1 || G > 64 || W < 1 || G % W) return MOE_ERR_ARG;
+    const int Gl = G / W;
+    for (int h = 0; h < W; ++h) sent[h] = received[h] = 0;
+    for (int s = 0; s < G; ++s)
+        for (int r = 0; r < G; ++r) {
+            const int32_t c = counts_all[(size_t)s * G + r];
+            if (c < 0) return MOE_ERR_ARG;
+            if (s / Gl != r / Gl) {
+                sent[s / Gl] += c;
+                received[r / Gl] += c;
+            }
+        }
+    return MOE_OK;
+}

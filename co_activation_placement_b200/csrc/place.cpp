@@ -183,3 +183,17 @@ extern "C" moe_status moe_place_replicas(const uint32_t *coact, int E, int G, in
     }
     return MOE_OK;
 }
+
+// Tasks each rank serves under a one-replica placement: the sum of n_e = C_ee
+// over the experts it holds ("Expert Placement Strategies", "Capacity-Aware
+// Placement": a device's load is its experts' loads together).
+extern "C" moe_status moe_rank_loads(const uint32_t *coact, int E, int G, const int32_t *expert_to_rank,
+                                     long long *rank_load)
+{
+    if (!coact || !expert_to_rank || !rank_load || E < 1 || G < 1) return MOE_ERR_ARG;
+    for (int e = 0; e < E; ++e)
+        if (expert_to_rank[e] < 0 || expert_to_rank[e] >= G) return MOE_ERR_ARG;
+    for (int r = 0; r < G; ++r) rank_load[r] = 0;
+    for (int e = 0; e < E; ++e) rank_load[expert_to_rank[e]] += coact[(size_t)e * E + e];
+    return MOE_OK;
+}

@@ -198,8 +198,12 @@ class EPGroup:
                  out_dtype=torch.float32, prereduce: bool = False, scale: Optional[torch.Tensor] = None, group=None):
         import os
         import torch.distributed as dist
-        # the kernels use plain peer loads and stores: no multicast object is wanted
-        os.environ.setdefault("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1")
+        # the kernels use plain peer loads and stores, never multicast: a rank
+        # that leaves while its memory is bound to an NVLink multicast object
+        # can fault the other ranks' GPUs, so no multicast object is ever made
+        if os.environ.get("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1") != "1":
+            raise ValueError("EPGroup needs TORCH_SYMM_MEM_DISABLE_MULTICAST=1 (no multicast objects)")
+        os.environ["TORCH_SYMM_MEM_DISABLE_MULTICAST"] = "1"
         import torch.distributed._symmetric_memory as symm_mem
         self.group = group if group is not None else dist.group.WORLD
         W, me = dist.get_world_size(self.group), dist.get_rank(self.group)

@@ -66,6 +66,7 @@ class HotPath:
     scales: List[torch.Tensor] = field(default_factory=list)   # f32 [E] per layer (prereduce)
     replicas: list = field(default_factory=list)   # per layer (replica_rank [E][1+nodes], n_rep [E]) or empty
     shuffle_capacity: int = 0          # > 0: at most this many tokens per rank (moe_shuffle_balanced)
+    replica_eps: Optional[float] = None   # load tolerance of the replica assignment (None: no cap)
     overlap: bool = True               # control work on a second stream beside the row traffic
     # buffers
     stats: dict = field(default_factory=dict)
@@ -112,6 +113,12 @@ class HotPath:
         if self.replicas:
             self.pick_rank = torch.empty((T, k), dtype=torch.int32, device=dev)
             self.n_remote = torch.empty(T, dtype=torch.int32, device=dev)
+            if self.replica_eps is not None:
+                # the capped assignment is one cooperative launch over every SM
+                self.overlap = False
+                self.rank_load = torch.zeros((L, self.G), dtype=torch.int64, device=dev)
+                self.capped_ws = torch.empty(cap.assign_replicas_capped_workspace(self.G), dtype=torch.uint8,
+                                             device=dev)
         if self.prereduce:
             if len(self.scales) != L:
                 raise ValueError("prereduce needs one scale vector per layer")
@@ -152,8 +159,13 @@ class HotPath:
             rr, nr = self.replicas[l]
 
             def go():
-                cap.assign_replicas(self.ids[l], self.E, self.G, self.rpn, rr, nr, src_rank=src,
-                                    pick_rank=self.pick_rank, n_remote=self.n_remote, err=self.err)
+                if self.replica_eps is not None:
+                    cap.assign_replicas_capped(self.ids[l], self.E, self.G, self.rpn, rr, nr, self.replica_eps,
+                                               src_rank=src, pick_rank=self.pick_rank, n_remote=self.n_remote,
+                                               rank_load=self.rank_load[l], err=self.err, ws=self.capped_ws)
+                else:
+                    cap.assign_replicas(self.ids[l], self.E, self.G, self.rpn, rr, nr, src_rank=src,
+                                        pick_rank=self.pick_rank, n_remote=self.n_remote, err=self.err)
                 cap.plan_dispatch_ranks(self.ids[l], self.E, self.G, self.rpn, self.pick_rank, src_rank=src,
                                         plan=self.plans[l], ws=self.plan_ws)
             self._call("plan", go)
@@ -317,7 +329,7 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
             x_dtype: str, ids_cal: np.ndarray, placement: str = "correlated", shuffle: bool = True,
             out_dtype=torch.bfloat16, device="cuda", rows: bool = True, timers: bool = False,
             scales: Optional[np.ndarray] = None, replica_extra: int = 0, shuffle_capacity: int = 0,
-            overlap: bool = True) -> HotPath:
+            overlap: bool = True, replica_eps: Optional[float] = None) -> HotPath:
     """Upload a batch (host numpy arrays; x as float32 or bf16 bit patterns)
     and its calibration batch, calibrate, and return the step's HotPath."""
     dev = torch.device(device)
@@ -334,7 +346,8 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
         if scales is not None else []
     return HotPath(E=E, G=G, rpn=rpn, ids=ids_d, gates=gates_d, x=x_d, e2r=e2r, rank_scores=rs,
                    out_dtype=out_dtype, rows=rows, timers=timers, prereduce=scales is not None, scales=scales_d,
-                   replicas=reps, shuffle_capacity=shuffle_capacity, overlap=overlap)
+                   replicas=reps, shuffle_capacity=shuffle_capacity, overlap=overlap,
+                   replica_eps=replica_eps if replica_extra > 0 else None)
 
 
 def placement_effect(ids: torch.Tensor, ids_cal: torch.Tensor, E: int, G: int, rpn: int,
@@ -360,9 +373,7 @@ def placement_effect(ids: torch.Tensor, ids_cal: torch.Tensor, E: int, G: int, r
     if not loads:
         return np.stack(out)
     n = cap.coact_stats(ids, E, want=("coact",))["coact"].cpu().numpy()
-    rank_load = np.zeros((L, G))
-    for l in range(L):
-        np.add.at(rank_load[l], e2r[l].cpu().numpy(), np.diag(n[l]).astype(np.float64))
+    rank_load = np.stack([cap.rank_loads(n[l], e2r[l].cpu().numpy(), G) for l in range(L)]).astype(np.float64)
     return np.stack(out), rank_load
 
 

@@ -198,6 +198,34 @@ moe_status moe_assign_replicas(const int32_t *ids, int T, int k, int E, int G, i
                                int32_t *pick_rank, int32_t *n_remote, int32_t *err, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Task assignment under a load tolerance  ([CB] "Problem Formulation": the
+ * tasks a rank runs, sum_e w_r^e, at most (1 + eps) K T / G, beside the
+ * fewest remote nodes per token)
+ *
+ * The page states the constraint, not how to meet it.  Reading taken: tokens
+ * in id order; before token t every rank whose task count has reached
+ * cap = floor((1 + eps) * (T k) / G) (fp64: one multiply, one divide; no cap
+ * for eps = inf) is closed to t, and t is assigned exactly as by
+ * moe_assign_replicas over the open replicas of its experts -- a pick whose
+ * expert has no open replica may use all of them (the cap gives way, never
+ * the task).  A token can take a rank past the cap by at most k - 1 tasks;
+ * eps = inf gives moe_assign_replicas's result.  The kernel reaches the same
+ * result with every token in flight at once, in at most G + 1 rounds of one
+ * cooperative launch (grid barriers with the library's 2 s bounded wait).
+ * Arguments as moe_assign_replicas, plus: eps >= 0 (else MOE_ERR_ARG);
+ * rank_load device int64 [G] out or NULL (tasks per rank after the batch);
+ * ws device, moe_assign_replicas_capped_workspace(G) bytes, 256-byte aligned,
+ * caller-owned, overwritten by each call (calls on one workspace must not
+ * overlap).  Data errors as moe_assign_replicas; an invalid token counts for
+ * no rank.
+ * ---------------------------------------------------------------------- */
+size_t moe_assign_replicas_capped_workspace(int G);
+moe_status moe_assign_replicas_capped(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                                      const int32_t *replica_rank, const int32_t *n_rep, const int32_t *src_rank,
+                                      double eps, int32_t *pick_rank, int32_t *n_remote, long long *rank_load,
+                                      int32_t *err, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * moe_coact_ema ([CB] "Key Observation": Ochiai on exponential moving averages
  *   of the co-selection counts and loads).  Per cell, in fp64 with IEEE
  *   rounding and no fused multiply-add:
@@ -389,6 +417,16 @@ moe_status moe_ep_scatter_rows(const void *src, int64_t row_bytes, int64_t R_max
                                int G, int W, void *const *dst_base, int64_t dst_cap, int32_t *err,
                                cudaStream_t stream);
 
+/* moe_ep_exchange_rows ([EC] abstract: the method's gain is the rows that no
+ *   longer cross GPUs): with the G ranks on W devices (Gl = G/W consecutive
+ *   ranks each) and counts_all host int32 [G][G] (rows from source rank s to
+ *   rank r, the gathered counts of every device's plan), sent[h] = rows whose
+ *   source is on device h and whose rank is not, received[h] = rows whose rank
+ *   is on device h and whose source is not.  Each such row crosses NVLink once
+ *   in the dispatch and once back in the combine.  sent, received host int64
+ *   [W] out.  MOE_ERR_ARG for a negative count or W not dividing G. */
+moe_status moe_ep_exchange_rows(const int32_t *counts_all, int G, int W, long long *sent, long long *received);
+
 /* ------------------------------------------------------------------------
  * Token shuffling  ([EC]: move each token to the GPU predicted to hold its
  * next-layer experts)
@@ -486,6 +524,15 @@ moe_status moe_place_correlated_capped(const uint32_t *coact, int E, int G, int 
  *   the order added; -1 unused), n_rep host int32 [E] out. */
 moe_status moe_place_replicas(const uint32_t *coact, int E, int G, int rpn, const int32_t *expert_to_rank,
                               int extra, int32_t *replica_rank, int32_t *n_rep);
+
+/* moe_rank_loads ([EPS] "Capacity-Aware Placement": a device's load is the
+ *   sum of its experts' loads).  rank_load[r] = sum of C_ee over the experts e
+ *   with expert_to_rank[e] = r: the tasks rank r serves in the batch whose
+ *   counts coact holds (only the diagonal is read).  coact host uint32 [E][E];
+ *   expert_to_rank host int32 [E]; rank_load host int64 [G] out.  MOE_ERR_ARG
+ *   for a rank outside [0, G). */
+moe_status moe_rank_loads(const uint32_t *coact, int E, int G, const int32_t *expert_to_rank,
+                          long long *rank_load);
 
 /* ------------------------------------------------------------------------
  * moe_selftest_wait_timeout (no counterpart on the pages: a test of the error

@@ -61,12 +61,17 @@ def lib():
             "orc_plan_ranks": [P, i, i, i, i, i, P, P, P, P, P, P, P, P, P],
             "orc_place_replicas": [P, i, i, i, P, i, P, P],
             "orc_assign_replicas": [P, i, i, i, i, i, P, P, P, P, P],
+            "orc_assign_replicas_capped": [P, i, i, i, i, i, P, P, P, ctypes.c_double, P, P, P],
+            "orc_rank_loads": [P, i, i, P, P],
             "orc_ep_routes": [P, P, i, i, i, P],
+            "orc_ep_exchange_rows": [P, i, i, P, P],
         }
         for name, args in sig.items():
             f = getattr(_lib, name)
             f.argtypes = args
             f.restype = ctypes.c_int
+        _lib.orc_load_cap.argtypes = [i, i, i, ctypes.c_double]
+        _lib.orc_load_cap.restype = i64
     return _lib
 
 
@@ -287,6 +292,39 @@ def assign_replicas(ids_l, E: int, G: int, rpn: int, replica_rank, n_rep, src_ra
     return pr, nrem
 
 
+def assign_replicas_capped(ids_l, E: int, G: int, rpn: int, replica_rank, n_rep, eps: float, src_rank=None):
+    """(pick_rank int32 [T][k], n_remote int32 [T], rank_load int64 [G]) under
+    the per-rank task cap floor((1 + eps) T k / G), tokens in id order."""
+    ids_l = np.ascontiguousarray(ids_l, dtype=np.int32)
+    T, k = ids_l.shape
+    rr = np.ascontiguousarray(replica_rank, dtype=np.int32)
+    nr = np.ascontiguousarray(n_rep, dtype=np.int32)
+    src = None if src_rank is None else np.ascontiguousarray(src_rank, dtype=np.int32)
+    pr = np.empty((T, k), np.int32)
+    nrem = np.empty(T, np.int32)
+    load = np.empty(G, np.int64)
+    _check("orc_assign_replicas_capped",
+           lib().orc_assign_replicas_capped(_p(ids_l), T, k, E, G, rpn, _p(rr), _p(nr), _p(src), float(eps),
+                                            _p(pr), _p(nrem), _p(load)))
+    return pr, nrem, load
+
+
+def load_cap(T: int, k: int, G: int, eps: float) -> int:
+    """floor((1 + eps) T k / G) in fp64 (the per-rank task cap)."""
+    return int(lib().orc_load_cap(T, k, G, float(eps)))
+
+
+def rank_loads(coact_l, expert_to_rank, G: int) -> np.ndarray:
+    """int64 [G]: the tasks each rank serves under a one-replica placement
+    (sum of n_e = C_ee over its experts)."""
+    c = np.ascontiguousarray(coact_l, dtype=np.uint32)
+    E = c.shape[0]
+    e2r = np.ascontiguousarray(expert_to_rank, dtype=np.int32)
+    load = np.empty(G, np.int64)
+    _check("orc_rank_loads", lib().orc_rank_loads(_p(c), E, G, _p(e2r), _p(load)))
+    return load
+
+
 def ep_routes(counts_all, offsets, G: int, W: int, me: int) -> np.ndarray:
     """int64 [2*G*(G/W) + 2]: device me's route table (rows received, its
     segments' first local rows, its R, the shifts to the receiving buffers)."""
@@ -295,3 +333,12 @@ def ep_routes(counts_all, offsets, G: int, W: int, me: int) -> np.ndarray:
     route = np.empty(2 * G * (G // W) + 2, np.int64)
     _check("orc_ep_routes", lib().orc_ep_routes(_p(c), _p(o), G, W, me, _p(route)))
     return route
+
+
+def ep_exchange_rows(counts_all, G: int, W: int):
+    """(sent int64 [W], received int64 [W]): rows crossing devices per device."""
+    c = np.ascontiguousarray(counts_all, dtype=np.int32)
+    sent = np.empty(W, np.int64)
+    recv = np.empty(W, np.int64)
+    _check("orc_ep_exchange_rows", lib().orc_ep_exchange_rows(_p(c), G, W, _p(sent), _p(recv)))
+    return sent, recv

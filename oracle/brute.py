@@ -214,3 +214,54 @@ def place_correlated(C, G, rpn, eps=-1.0):
             for e in rg:
                 e2r[e] = q * rpn + u
     return e2r
+
+
+def assign_replicas_capped(ids_l, G, rpn, replica_rank, n_rep, eps, src_rank=None):
+    """Restatement of the load-capped assignment with Python sets: tokens in
+    id order; ranks whose task count has reached floor((1 + eps) T k / G) are
+    closed to the next token; a pick uses its expert's open replicas, or all
+    of them when none is open; the remote node set is the smallest covering
+    one (ties: smallest bit pattern), found by listing every node set; picks
+    in j order prefer the source rank, then a rank the token already uses,
+    then the lowest rank, among the usable ranks on the source node or, if
+    none, on the chosen set.  Returns (picks, n_remote, loads) as lists."""
+    T, k = len(ids_l), len(ids_l[0]) if len(ids_l) else 0
+    nodes = G // rpn
+    cap = math.floor((1.0 + eps) * float(T * k) / G) if math.isfinite(eps) else math.inf
+    load = [0] * G
+    picks, nrem = [], []
+    for t in range(T):
+        s = int(src_rank[t]) if src_rank is not None else t // (T // G)
+        ns = s // rpn
+        open_r = {r for r in range(G) if load[r] < cap}
+        usable = []
+        for e in ids_l[t]:
+            reps = [int(r) for r in replica_rank[e][: n_rep[e]]]
+            opn = [r for r in reps if r in open_r]
+            usable.append(opn if opn else reps)
+        best = None
+        for bits in range(1 << nodes):
+            S = {q for q in range(nodes) if (bits >> q) & 1}
+            if ns in S:
+                continue
+            if all(any(r // rpn == ns or r // rpn in S for r in u) for u in usable):
+                key = (len(S), bits)
+                if best is None or key < best[0]:
+                    best = (key, S)
+        S = best[1]
+        mine = []
+        for u in usable:
+            home = [r for r in u if r // rpn == ns]
+            allowed = home if home else [r for r in u if r // rpn in S]
+            if s in allowed:
+                p = s
+            elif any(r in mine for r in allowed):
+                p = min(r for r in allowed if r in mine)
+            else:
+                p = min(allowed)
+            mine.append(p)
+        for p in mine:
+            load[p] += 1
+        picks.append(mine)
+        nrem.append(len(S))
+    return picks, nrem, load

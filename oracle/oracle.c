@@ -687,66 +687,166 @@ int orc_place_replicas(const uint32_t *coact, int E, int G, int rpn, const int32
     return ORC_OK;
 }
 
-/* Communication-aware task assignment ([CB]: tokens are routed "to the fewest
- * remote nodes possible"; V counts, per token, the remote nodes its tasks
- * reach).  For token t with source rank s (node ns = s / rpn): among all
- * choices of one replica rank per pick, the fewest distinct nodes other than
- * ns -- found as the smallest node set S (ties: smallest as a bit pattern)
- * such that every pick's expert has a replica on ns or in S.  Then, pick by
- * pick in j order, among the ranks hosting the expert on ns (or, if none, on
- * the nodes of S): rank s if it is one of them; else the lowest of them that
- * an earlier pick of the token already uses (no new row); else the lowest of
- * them.  Requires G/rpn <= 8.
- * pick_rank [T][k] out; n_remote [T] out (|S|, may be NULL). */
+/* Communication-aware task assignment of one token ([CB]: tokens are routed
+ * "to the fewest remote nodes possible"; V counts, per token, the remote
+ * nodes its tasks reach).  Token with picks d[0..k) and source rank s (node
+ * ns = s / rpn).  A replica of a pick's expert may serve it when its rank is
+ * open (bit r of open_ranks), or when none of that expert's replicas is open.
+ * Among all choices of one such replica per pick, the fewest distinct nodes
+ * other than ns -- found as the smallest node set S (ties: smallest as a bit
+ * pattern) such that every pick's expert has a usable replica on ns or in S.
+ * Then, pick by pick in j order, among the usable ranks hosting the expert on
+ * ns (or, if none, on the nodes of S): rank s if it is one of them; else the
+ * lowest of them that an earlier pick of the token already uses (no new row);
+ * else the lowest of them.  Writes pick_rank[0..k); returns |S|, or -1 when
+ * an expert has no replica at all. */
+static int assign_token(const int32_t *d, int k, int s, int rpn, int nodes, const int32_t *replica_rank,
+                        const int32_t *n_rep, uint64_t open_ranks, int32_t *pick_rank)
+{
+    const int max_rep = 1 + nodes, ns = s / rpn;
+    int any_open[8];
+    for (int j = 0; j < k; ++j) {
+        any_open[j] = 0;
+        for (int q = 0; q < n_rep[d[j]]; ++q)
+            if ((open_ranks >> replica_rank[(size_t)d[j] * max_rep + q]) & 1) any_open[j] = 1;
+    }
+#define USABLE(j, r) (!any_open[j] || ((open_ranks >> (r)) & 1))
+    int best_size = nodes + 1, best_set = 0;
+    for (int set = 0; set < (1 << nodes); ++set) {
+        if ((set >> ns) & 1) continue;
+        int ok = 1;
+        for (int j = 0; j < k && ok; ++j) {
+            int covered = 0;
+            for (int q = 0; q < n_rep[d[j]]; ++q) {
+                int r = replica_rank[(size_t)d[j] * max_rep + q], node = r / rpn;
+                if (USABLE(j, r) && (node == ns || ((set >> node) & 1))) covered = 1;
+            }
+            ok = covered;
+        }
+        if (!ok) continue;
+        int size = 0;
+        for (int q = 0; q < nodes; ++q) size += (set >> q) & 1;
+        if (size < best_size) { best_size = size; best_set = set; }
+    }
+    if (best_size > nodes) return -1;   /* an expert without replicas */
+    for (int j = 0; j < k; ++j) {
+        int any_ns = 0;
+        for (int q = 0; q < n_rep[d[j]]; ++q) {
+            int r = replica_rank[(size_t)d[j] * max_rep + q];
+            if (USABLE(j, r) && r / rpn == ns) any_ns = 1;
+        }
+        int pick = -1, used_pick = -1, low = -1;
+        for (int q = 0; q < n_rep[d[j]]; ++q) {
+            int r = replica_rank[(size_t)d[j] * max_rep + q];
+            if (!USABLE(j, r)) continue;
+            int allowed = any_ns ? (r / rpn == ns) : ((best_set >> (r / rpn)) & 1);
+            if (!allowed) continue;
+            if (r == s) pick = r;
+            int used = 0;
+            for (int q2 = 0; q2 < j; ++q2) used |= pick_rank[q2] == r;
+            if (used && (used_pick < 0 || r < used_pick)) used_pick = r;
+            if (low < 0 || r < low) low = r;
+        }
+        if (pick < 0) pick = used_pick >= 0 ? used_pick : low;
+        pick_rank[j] = pick;
+    }
+#undef USABLE
+    return best_size;
+}
+
+static int check_replica_table(int E, int G, int max_rep, const int32_t *replica_rank, const int32_t *n_rep)
+{
+    for (int e = 0; e < E; ++e) {
+        if (n_rep[e] < 0 || n_rep[e] > max_rep) return ORC_ERR_DATA;
+        for (int q = 0; q < n_rep[e]; ++q)
+            if (replica_rank[(size_t)e * max_rep + q] < 0 || replica_rank[(size_t)e * max_rep + q] >= G)
+                return ORC_ERR_DATA;
+    }
+    return ORC_OK;
+}
+
+/* Every rank open: the assignment of [CB]'s "fewest remote nodes possible"
+ * alone.  Requires G/rpn <= 8.  pick_rank [T][k] out; n_remote [T] out (|S|,
+ * may be NULL). */
 int orc_assign_replicas(const int32_t *ids, int T, int k, int E, int G, int rpn, const int32_t *replica_rank,
                         const int32_t *n_rep, const int32_t *src_rank, int32_t *pick_rank, int32_t *n_remote)
 {
-    if (T < 0 || k < 1 || k > 8 || G < 1 || rpn < 1 || G % rpn != 0 || G / rpn > 8) return ORC_ERR_ARG;
+    if (T < 0 || k < 1 || k > 8 || G < 1 || G > 64 || rpn < 1 || G % rpn != 0 || G / rpn > 8) return ORC_ERR_ARG;
     if (!src_rank && T % G != 0) return ORC_ERR_ARG;
-    const int nodes = G / rpn, max_rep = 1 + nodes;
+    const int nodes = G / rpn;
+    if (check_replica_table(E, G, 1 + nodes, replica_rank, n_rep) != ORC_OK) return ORC_ERR_DATA;
     for (int t = 0; t < T; ++t) {
         const int32_t *d = ids + (size_t)t * k;
         if (!token_valid(d, k, E)) return ORC_ERR_DATA;
         const int s = src_rank ? src_rank[t] : t / (T / G);
         if (s < 0 || s >= G) return ORC_ERR_DATA;
-        const int ns = s / rpn;
-        int best_size = nodes + 1, best_set = 0;
-        for (int set = 0; set < (1 << nodes); ++set) {
-            if ((set >> ns) & 1) continue;
-            int ok = 1;
-            for (int j = 0; j < k && ok; ++j) {
-                int covered = 0;
-                for (int q = 0; q < n_rep[d[j]]; ++q) {
-                    int node = replica_rank[(size_t)d[j] * max_rep + q] / rpn;
-                    if (node == ns || ((set >> node) & 1)) covered = 1;
-                }
-                ok = covered;
-            }
-            if (!ok) continue;
-            int size = 0;
-            for (int q = 0; q < nodes; ++q) size += (set >> q) & 1;
-            if (size < best_size) { best_size = size; best_set = set; }
-        }
-        if (best_size > nodes) return ORC_ERR_DATA;   /* an expert without replicas */
-        for (int j = 0; j < k; ++j) {
-            int any_ns = 0;
-            for (int q = 0; q < n_rep[d[j]]; ++q)
-                if (replica_rank[(size_t)d[j] * max_rep + q] / rpn == ns) any_ns = 1;
-            int pick = -1, used_pick = -1, low = -1;
-            for (int q = 0; q < n_rep[d[j]]; ++q) {
-                int r = replica_rank[(size_t)d[j] * max_rep + q];
-                int allowed = any_ns ? (r / rpn == ns) : ((best_set >> (r / rpn)) & 1);
-                if (!allowed) continue;
-                if (r == s) pick = r;
-                int used = 0;
-                for (int q2 = 0; q2 < j; ++q2) used |= pick_rank[(size_t)t * k + q2] == r;
-                if (used && (used_pick < 0 || r < used_pick)) used_pick = r;
-                if (low < 0 || r < low) low = r;
-            }
-            if (pick < 0) pick = used_pick >= 0 ? used_pick : low;
-            pick_rank[(size_t)t * k + j] = pick;
-        }
-        if (n_remote) n_remote[t] = best_size;
+        const int size = assign_token(d, k, s, rpn, nodes, replica_rank, n_rep, ~(uint64_t)0, pick_rank + (size_t)t * k);
+        if (size < 0) return ORC_ERR_DATA;
+        if (n_remote) n_remote[t] = size;
+    }
+    return ORC_OK;
+}
+
+/* The per-rank workload cap of [CB] "Problem Formulation": the tasks rank r
+ * runs, sum_e w_r^e, at most (1 + eps) K T / G.  cap = floor((1 + eps) * (T k)
+ * / G) in fp64 (one multiply, one divide, IEEE rounding); INT64_MAX when that
+ * is 9e18 or more (eps = inf: no cap). */
+int64_t orc_load_cap(int T, int k, int G, double eps)
+{
+    const double c = floor((1.0 + eps) * (double)((int64_t)T * k) / (double)G);
+    return c >= 9.0e18 ? INT64_MAX : (int64_t)c;
+}
+
+/* Assignment under the load tolerance eps ([CB] "Problem Formulation": the
+ * fewest remote nodes per token, and sum_e w_r^e <= (1 + eps) K T / G per
+ * rank).  The page states the constraint, not how to meet it; the reading
+ * taken: tokens in id order; before token t a rank whose load (tasks already
+ * assigned to it) has reached cap = orc_load_cap(T, k, G, eps) is closed, and
+ * t is assigned as in assign_token over the open ranks.  A pick whose expert
+ * has no open replica may use all of its replicas (the cap gives way, not the
+ * task), and a token may take a rank past the cap by at most k - 1 tasks.
+ * pick_rank [T][k] out; n_remote [T] out or NULL; rank_load [G] out or NULL
+ * (tasks per rank). */
+int orc_assign_replicas_capped(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                               const int32_t *replica_rank, const int32_t *n_rep, const int32_t *src_rank,
+                               double eps, int32_t *pick_rank, int32_t *n_remote, int64_t *rank_load)
+{
+    if (T < 0 || k < 1 || k > 8 || G < 1 || G > 64 || rpn < 1 || G % rpn != 0 || G / rpn > 8) return ORC_ERR_ARG;
+    if (!(eps >= 0.0)) return ORC_ERR_ARG;
+    if (!src_rank && T % G != 0) return ORC_ERR_ARG;
+    const int nodes = G / rpn;
+    if (check_replica_table(E, G, 1 + nodes, replica_rank, n_rep) != ORC_OK) return ORC_ERR_DATA;
+    const int64_t cap = orc_load_cap(T, k, G, eps);
+    int64_t load[64] = {0};
+    for (int t = 0; t < T; ++t) {
+        const int32_t *d = ids + (size_t)t * k;
+        if (!token_valid(d, k, E)) return ORC_ERR_DATA;
+        const int s = src_rank ? src_rank[t] : t / (T / G);
+        if (s < 0 || s >= G) return ORC_ERR_DATA;
+        uint64_t open_ranks = 0;
+        for (int r = 0; r < G; ++r)
+            if (load[r] < cap) open_ranks |= (uint64_t)1 << r;
+        const int size = assign_token(d, k, s, rpn, nodes, replica_rank, n_rep, open_ranks, pick_rank + (size_t)t * k);
+        if (size < 0) return ORC_ERR_DATA;
+        for (int j = 0; j < k; ++j) load[pick_rank[(size_t)t * k + j]] += 1;
+        if (n_remote) n_remote[t] = size;
+    }
+    if (rank_load)
+        for (int r = 0; r < G; ++r) rank_load[r] = load[r];
+    return ORC_OK;
+}
+
+/* Tasks each rank serves under a one-replica placement: load[r] = sum of n_e
+ * over the experts e with expert_to_rank[e] = r, n_e = C_ee the tokens that
+ * pick e ([EPS] "Capacity-Aware Placement": a device's load is the sum of its
+ * experts' loads).  coact [E][E] (only the diagonal is read); load [G] out. */
+int orc_rank_loads(const uint32_t *coact, int E, int G, const int32_t *expert_to_rank, int64_t *load)
+{
+    if (E < 1 || G < 1) return ORC_ERR_ARG;
+    for (int r = 0; r < G; ++r) load[r] = 0;
+    for (int e = 0; e < E; ++e) {
+        if (expert_to_rank[e] < 0 || expert_to_rank[e] >= G) return ORC_ERR_DATA;
+        load[expert_to_rank[e]] += coact[(size_t)e * E + e];
     }
     return ORC_OK;
 }
@@ -788,5 +888,24 @@ int orc_ep_routes(const int32_t *counts_all, const int32_t *offsets, int G, int 
     }
     route[1 + P] = offsets[G * G];
     free(off);
+    return ORC_OK;
+}
+
+/* Rows crossing devices in the exchange, as the definition: with the G ranks
+ * on W devices (G/W consecutive ranks each), a row from source rank s to rank
+ * r crosses when s and r are on different devices.  sent[h]: rows whose
+ * source is on device h and rank elsewhere; received[h]: the reverse. */
+int orc_ep_exchange_rows(const int32_t *counts_all, int G, int W, int64_t *sent, int64_t *received)
+{
+    if (G < 1 || G > 64 || W < 1 || G % W) return ORC_ERR_ARG;
+    const int Gl = G / W;
+    for (int h = 0; h < W; ++h) { sent[h] = 0; received[h] = 0; }
+    for (int s = 0; s < G; ++s)
+        for (int r = 0; r < G; ++r) {
+            if (counts_all[s * G + r] < 0) return ORC_ERR_DATA;
+            if (s / Gl == r / Gl) continue;
+            sent[s / Gl] += counts_all[s * G + r];
+            received[r / Gl] += counts_all[s * G + r];
+        }
     return ORC_OK;
 }

@@ -255,3 +255,4 @@ def test_host_placements_match_oracle_on_random_inputs(cap, orc):
         got = cap.place_replicas(C, G, rpn, e2r, extra)
         want = orc.place_replicas(C, G, rpn, e2r, extra)
         assert (got[0] == want[0]).all() and (got[1] == want[1]).all()
+        assert (cap.rank_loads(C, e2r, G) == orc.rank_loads(C, e2r, G)).all()

@@ -189,3 +189,33 @@ def test_meet_reports_a_lost_rank(world):
     assert res[world - 1] == "left"
     assert all(res[r].startswith("error") for r in range(world - 1)), res
     assert time.time() - t0 < 100
+
+
+@pytest.mark.parametrize("T,E,k,G,rpn,W", [(512, 16, 2, 4, 2, 2), (1536, 64, 6, 32, 8, 4), (960, 24, 5, 12, 4, 3),
+                                            (1024, 64, 3, 64, 8, 64), (640, 32, 4, 8, 8, 1)])
+def test_exchange_rows_from_route_tables(T, E, k, G, rpn, W):
+    """Rows crossing devices, counted from the route tables: device h's local
+    segments (r, s) with r on another device are the rows it sends; of the
+    rows its buffer receives (route[0]), those not from its own segments
+    came from other devices.  The oracle's definition and the library's host
+    count agree with both."""
+    import co_activation_placement_b200 as cap
+    ids = _ids(T + 7 * W, T, E, k)
+    e2r = np.random.default_rng(G + 1).permutation(np.arange(E, dtype=np.int32) // (E // G)).astype(np.int32)
+    Gl = G // W
+    P = G * Gl
+    plans = [_local_plan(ids, E, G, rpn, e2r, W, h) for h in range(W)]
+    counts_all = np.concatenate([plans[h]["counts"][h * Gl:(h + 1) * Gl] for h in range(W)])
+    sent_o, recv_o = orc.ep_exchange_rows(counts_all, G, W)
+    sent_l, recv_l = cap.ep_exchange_rows(counts_all, G, W)
+    assert sent_l.tolist() == sent_o.tolist() and recv_l.tolist() == recv_o.tolist()
+    for h, lo in enumerate(plans):
+        route = orc.ep_routes(counts_all, lo["offsets"], G, W, h)
+        start = route[1:P + 2]
+        seg = np.diff(start)                                  # rows of each local segment
+        away = np.array([(i // Gl) // Gl != h for i in range(P)])
+        assert int(seg[away].sum()) == sent_o[h]
+        assert int(route[0]) - int(seg[~away].sum()) == recv_o[h]
+    assert sent_o.sum() == recv_o.sum()
+    if W == 1:
+        assert sent_o.tolist() == [0]

@@ -264,8 +264,6 @@ ROW_WORKLOADS = ["tiny", "one_node", "ep32", "large_ep64"]
 def test_pipeline_full_size(cap, name, placement, shuffle):
     from co_activation_placement_b200 import pipeline
     w = WORKLOADS[name]
-    if name in ("ep32", "large_ep64") and placement == "uniform":
-        pytest.skip("uniform placement at this size is covered by the plan checks of the correlated run")
     ids = make_routing(w)
     ids_cal = make_routing(w, seed=w.seed + 1)
     gates = make_gates(w)

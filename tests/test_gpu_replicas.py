@@ -91,3 +91,77 @@ def test_replica_assignment_small_and_errors(cap):
     assert int(host(p.err)[0]) == cap.DERR_RANK_RANGE
     with pytest.raises(cap.MoeError):
         cap.assign_replicas(dev(ids), E, 16, 1, dev(rr), dev(nr), src_rank=dev(src))   # 16 nodes > 8
+
+
+# ------------------------------------------------- load-capped assignment
+
+@pytest.mark.parametrize("name,extra,eps,with_src", [("one_node", 2, 0.0, False), ("one_node", 2, 0.1, True),
+                                                     ("ep32", 2, 0.05, False), ("ep32", 1, 0.2, True),
+                                                     ("large_ep64", 1, 0.1, False), ("large_ep64", 2, 0.0, True),
+                                                     ("large_ep64", 2, float("inf"), False)])
+def test_capped_assignment_full_size(cap, name, extra, eps, with_src):
+    """The load-capped assignment ("Cobalt", "Problem Formulation": sum_e w_r^e
+    <= (1 + eps) K T / G) bit for bit against the oracle's token-order greedy
+    at the workloads' full sizes: picks, remote nodes per token, rank loads;
+    eps = inf equals the uncapped assignment; the plan over the picks too."""
+    w = WORKLOADS[name]
+    ids = make_routing(w)[0]
+    cal = make_routing(w, seed=1)[0]
+    C = orc.coact(cal[None], w.E, want=("coact",))["coact"][0]
+    e2r = orc.place_correlated(C, w.G, w.rpn)
+    rr, nr = orc.place_replicas(C, w.G, w.rpn, e2r, extra)
+    rng = np.random.default_rng(11)
+    src = rng.integers(0, w.G, w.T).astype(np.int32) if with_src else None
+    err = cap.new_err("cuda")
+    pr, nrem, load = cap.assign_replicas_capped(dev(ids), w.E, w.G, w.rpn, dev(rr), dev(nr), eps,
+                                                src_rank=None if src is None else dev(src), err=err)
+    pr_o, nrem_o, load_o = orc.assign_replicas_capped(ids, w.E, w.G, w.rpn, rr, nr, eps, src_rank=src)
+    assert int(host(err)[0]) == 0
+    assert (host(pr)[: w.T] == pr_o).all()
+    assert (host(nrem)[: w.T] == nrem_o).all()
+    assert host(load).tolist() == load_o.tolist()
+    if eps == float("inf"):
+        pu, nu = orc.assign_replicas(ids, w.E, w.G, w.rpn, rr, nr, src_rank=src)
+        assert (pr_o == pu).all() and (nrem_o == nu).all()
+    p = cap.plan_dispatch_ranks(dev(ids), w.E, w.G, w.rpn, pr, src_rank=None if src is None else dev(src))
+    check_plan(p, orc.plan(ids, w.E, w.G, w.rpn, None, src_rank=src, pick_rank=pr_o), w.T)
+
+
+@pytest.mark.parametrize("T,E,k,G,rpn,eps", [(999, 16, 3, 8, 2, 0.0), (5000, 32, 4, 8, 4, 0.03),
+                                             (1, 16, 3, 8, 2, 0.0), (130, 64, 8, 64, 8, 0.0),
+                                             (4096, 16, 2, 4, 1, 0.5), (777, 24, 6, 8, 1, 0.01)])
+def test_capped_assignment_shapes(cap, T, E, k, G, rpn, eps):
+    """Ragged token counts, one token, tight caps (many closing rounds), every
+    rank its own node, explicit source ranks."""
+    rng = np.random.default_rng(T + E + G)
+    hot = rng.permutation(E)[: k + 2]
+    ids = np.where((rng.random(T) < 0.8)[:, None], hot[np.argsort(rng.random((T, hot.size)), axis=1)[:, :k]],
+                   np.argsort(rng.random((T, E)), axis=1)[:, :k]).astype(np.int32)
+    C = orc.coact(ids[None], E, want=("coact",))["coact"][0]
+    e2r = orc.place_correlated(C, G, rpn)
+    rr, nr = orc.place_replicas(C, G, rpn, e2r, 2)
+    src = rng.integers(0, G, T).astype(np.int32)
+    pr, nrem, load = cap.assign_replicas_capped(dev(ids), E, G, rpn, dev(rr), dev(nr), eps, src_rank=dev(src))
+    pr_o, nrem_o, load_o = orc.assign_replicas_capped(ids, E, G, rpn, rr, nr, eps, src_rank=src)
+    assert (host(pr)[:T] == pr_o).all() and (host(nrem)[:T] == nrem_o).all()
+    assert host(load).tolist() == load_o.tolist()
+
+
+def test_capped_assignment_errors(cap):
+    rng = np.random.default_rng(4)
+    T, E, k, G, rpn = 600, 16, 3, 8, 2
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    C = orc.coact(ids[None], E, want=("coact",))["coact"][0]
+    rr, nr = orc.place_replicas(C, G, rpn, orc.place_correlated(C, G, rpn), 1)
+    bad = ids.copy()
+    bad[9, 2] = E + 1
+    err = cap.new_err("cuda")
+    pr, nrem, load = cap.assign_replicas_capped(dev(bad), E, G, rpn, dev(rr), dev(nr), 0.1, err=err)
+    assert int(host(err)[0]) == cap.DERR_ID_RANGE and (host(pr)[9] == -1).all()
+    assert int(host(load).sum()) == (T - 1) * k          # the invalid token counts for no rank
+    for eps in (-0.5, float("nan")):
+        with pytest.raises(cap.MoeError):
+            cap.assign_replicas_capped(dev(ids), E, G, rpn, dev(rr), dev(nr), eps)
+    # the context stays usable
+    pr, _, _ = cap.assign_replicas_capped(dev(ids), E, G, rpn, dev(rr), dev(nr), 0.1)
+    assert (host(pr)[:T] == orc.assign_replicas_capped(ids, E, G, rpn, rr, nr, 0.1)[0]).all()

@@ -14,8 +14,9 @@ from conftest import ROOT
 
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_pins.py", "tests/test_oracle_brute.py", "tests/test_oracle_prereduce.py",
-        "tests/test_oracle_replicas.py", "tests/test_oracle_shuffle_balanced.py", "tests/test_oracle_ema.py", "tests/test_oracle_capped.py",
+        "tests/test_oracle_replicas.py", "tests/test_oracle_replicas_capped.py", "tests/test_oracle_shuffle_balanced.py", "tests/test_oracle_ema.py", "tests/test_oracle_capped.py",
         "tests/test_ep_cpu.py::test_routes_hand_worked", "tests/test_ep_cpu.py::test_route_definition",
+        "tests/test_ep_cpu.py::test_exchange_rows_from_route_tables",
         "tests/test_oracle_property.py"]
 
 MUTANTS = {
@@ -71,6 +72,18 @@ MUTANTS = {
     "capped_forced_pick_heaviest": ("if (pick < 0 || C[(size_t)pool[x] * E + pool[x]] < C[(size_t)pool[pick] * E + pool[pick]])",
                                     "if (pick < 0 || C[(size_t)pool[x] * E + pool[x]] > C[(size_t)pool[pick] * E + pool[pick]])"),
     "capped_cap_ignored": ("if (cap >= 0.0 && (double)(load + nx) > cap) continue;", "(void)nx;"),
+    "capped_closes_late": ("if (load[r] < cap) open_ranks |= (uint64_t)1 << r;",
+                           "if (load[r] <= cap) open_ranks |= (uint64_t)1 << r;"),
+    "capped_forced_pick_closed_only": ("#define USABLE(j, r) (!any_open[j] || ((open_ranks >> (r)) & 1))",
+                                       "#define USABLE(j, r) (((open_ranks >> (r)) & 1))"),
+    "capped_cap_rounded_up": ("const double c = floor((1.0 + eps) * (double)((int64_t)T * k) / (double)G);",
+                              "const double c = ceil((1.0 + eps) * (double)((int64_t)T * k) / (double)G);"),
+    "capped_load_drops_last_pick": ("for (int j = 0; j < k; ++j) load[pick_rank[(size_t)t * k + j]] += 1;",
+                                    "for (int j = 0; j + 1 < k; ++j) load[pick_rank[(size_t)t * k + j]] += 1;"),
+    "rank_loads_off_diagonal": ("load[expert_to_rank[e]] += coact[(size_t)e * E + e];",
+                                "load[expert_to_rank[e]] += coact[(size_t)e * E + (e + 1) % E];"),
+    "exchange_counts_own_device": ("            if (s / Gl == r / Gl) continue;\n            sent[s / Gl]",
+                                   "            sent[s / Gl]"),
     "ep_routes_counts_transposed": ("run += counts_all[s * G + r];", "run += counts_all[r * G + s];"),
     "ep_routes_sender_base": ("const int64_t first_global = off[r * G + s] - off[(r / Gl) * Gl * G];",
                               "const int64_t first_global = off[r * G + s] - off[me * Gl * G];"),
