@@ -302,18 +302,21 @@ def run_reference(a, w):
 
 # ------------------------------------------------------------------ native arm
 
-def traffic_record(kernel_name, algorithmic_bytes_per_launch):
+def traffic_record(kernel_name, algorithmic_bytes_per_launch, k=None):
     """DRAM bytes per launch for the dominant kernel, from the committed ncu
     capture (profiles/traffic.json): the capture's DRAM bytes over its
     algorithmic bytes, scaled to this launch's algorithmic bytes (both kernels
-    stream, so traffic grows in proportion).  None when the kernel's source
-    changed since the capture."""
+    stream, so traffic grows in proportion).  The record of the same top-k
+    instantiation ("combine_k8") is preferred to the kernel's general one.
+    None when the kernel's source changed since the capture."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        rec = json.load(f).get(kernel_name)
+        recs = json.load(f)
+    rec = recs.get("%s_k%d" % (kernel_name, k)) if k is not None else None
+    rec = rec or recs.get(kernel_name)
     if not rec:
         return None
     names = rec["source"].split("+")              # the kernel's file and the headers it is built from
@@ -499,7 +502,7 @@ def main():
     dom = max((n for n in kern if n not in side_calls), key=lambda n: kern[n]["ms_per_step"])
     nl = launches_of[dom]
     per_launch_ms = kern[dom]["ms_per_step"] / nl
-    traffic = traffic_record(dom, bytes_of[dom] // nl)
+    traffic = traffic_record(dom, bytes_of[dom] // nl, w.k)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["gbs"], "peak": hbm, "unit": "GB/s",
                 "frac": kern[dom]["gbs"] / hbm, "peak_kind": hbm_kind,
                 "algorithmic_bytes_per_launch": bytes_of[dom] // nl, "ms_per_launch": per_launch_ms,
@@ -879,7 +882,7 @@ def run_ep_emulated(hp, w, W, steps, warmup, hbm, sb, pg):
                              "within one GPU's memory, so the nvlink frac is the floor over the measured step",
             "ms_per_step": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
             "errors": emu.errors(),
-            "note": "W virtual devices on this GPU, each with its own receive buffer, launched one after another; "
+            "note": "W virtual devices on this GPU, each with its own receive buffer and stream (a phase of the W devices runs side by side, each meeting joins the streams); "
                     "rows move through the peer-addressed kernels within this GPU's memory; per layer and "
                     "device: plan, routes, permute, combine (the counts gathered with one device-side copy)"}
 

@@ -8,7 +8,7 @@ import of any entry point raises: there is no fallback.
 
 Entry points (names follow the C ABI without the ``moe_`` prefix):
   coact_stats, coact_stats_method, coact_stats_path, coact_ema,
-  plan_dispatch, permute, combine, rank_score, shuffle_targets, shuffle_balanced,
+  plan_dispatch, plan_dispatch_method, permute, combine, rank_score, shuffle_targets, shuffle_balanced,
   dispatch_gates, expert_reduce, combine_rows,
   place_replicas, assign_replicas, assign_replicas_capped, plan_dispatch_ranks,
   ep_routes, ep_permute, ep_combine, ep_scatter_rows, ep_exchange_rows (ranks over several devices),
@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
             "moe_selftest_wait_timeout": ([i, P, P, sz, P], i),
             "moe_coact_stats": ([P, i, i, i, i, P, P, P, P, P, sz, P], i),
             "moe_plan_dispatch_workspace": ([i, i, i, i], sz),
+            "moe_plan_dispatch_method": ([i], i),
             "moe_plan_dispatch": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
             "moe_permute": ([P, i, i, i, i, P, i64, P, P, P], i),
             "moe_combine": ([P, i, i64, i, P, P, i, i, P, i, P, P], i),
@@ -269,6 +270,15 @@ class Plan:
         return _Plan(self.dest_mask.data_ptr(), self.counts.data_ptr(), self.offsets.data_ptr(),
                      self.row_token.data_ptr(), self.row_jmask.data_ptr(), self.row_of.data_ptr(),
                      self.summary.data_ptr())
+
+
+def plan_dispatch_method(method: int) -> int:
+    """0 = separate kernels (default), 1 = one cooperative launch when the
+    plan has at most 512 chunks; returns the previous setting (process-wide)."""
+    prev = int(lib().moe_plan_dispatch_method(int(method)))
+    if prev < 0:
+        raise ValueError("method must be 0 or 1")
+    return prev
 
 
 def plan_dispatch_workspace(T: int, k: int, G: int, with_src_rank: bool) -> int:

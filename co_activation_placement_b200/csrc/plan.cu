@@ -24,8 +24,10 @@
 // All arithmetic is integer; the result is unique and does not depend on
 // scheduling.  No kernel waits on another block.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
+#include "waits.cuh"
 
 namespace moe {
 namespace {
@@ -38,6 +40,7 @@ struct PlanWsHeader {
     unsigned int done_src;        // blocks finished in plan_src_count
     unsigned int pad[2];
     unsigned long long acc[4];    // R, R_remote, local, V
+    GridBarrier bar;              // the single-launch plan's grid barrier
 };
 
 struct PlanWs {
@@ -502,11 +505,309 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
     }
 }
 
+// ---- the whole plan in one cooperative launch ------------------------------
+//
+// The same three steps in one kernel, the cross-block scans replaced by grid
+// barriers: every block derives the shard table and the per-rank totals from
+// the per-chunk counts itself (a column sum over the chunks), so no single
+// block's serial tail sits on the critical path.  Blocks loop over chunks
+// when there are more chunks than co-resident blocks.  Used when the caller
+// selects it (moe_plan_dispatch_method) and the chunk count is small enough
+// for the column sums to stay cheap.
+
+constexpr int kFusedMaxChunks = 512;
+
+struct FusedArgs {
+    const int32_t *ids;
+    int T, E, G, rpn;
+    const int32_t *e2r_g, *picks, *src;
+    PlanWs w;
+    moe_plan P;
+    int32_t *err;
+    int Bs;               // source-count chunks (with source ranks)
+};
+
+// sum over rows b < B of tab[b][d] for d < G, into out[d] (shared); all
+// threads of the block; part: blockDim.x ints of shared scratch
+__device__ __forceinline__ void column_sums(const int32_t *tab, int B, int G, int32_t *out, int32_t *part)
+{
+    const int nseg = blockDim.x / G, d = threadIdx.x % G, q = threadIdx.x / G;
+    if (q < nseg) {
+        int s = 0;
+        for (int b = q; b < B; b += nseg) s += __ldcg(tab + (size_t)b * G + d);
+        part[q * G + d] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        int x = 0;
+        for (int qq = 0; qq < nseg; ++qq) x += part[qq * G + threadIdx.x];
+        out[threadIdx.x] = x;
+    }
+    __syncthreads();
+}
+
+template <int K, bool PICKS>
+__global__ void __launch_bounds__(kChunk, 1)
+plan_fused_kernel(FusedArgs a)
+{
+    extern __shared__ int32_t e2r[];           // [E] (unused with PICKS)
+    __shared__ int32_t cnt[64], base[64], tot[64], seg[64];
+    __shared__ int32_t part[kChunk];
+    __shared__ int32_t wcnt[kWarps][64];       // rows per (warp, rank), then their exclusive prefix
+    __shared__ uint32_t colw[kWarps][64];      // lanes of the warp with a row for the rank
+    __shared__ unsigned long long red[4][kWarps];
+    __shared__ ShardTable sh;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int T = a.T, E = a.E, G = a.G;
+    const bool with_src = a.src != nullptr;
+    GridBarrier *bar = &a.w.hdr->bar;
+    if (!PICKS)
+        for (int e = tid; e < E; e += kChunk) e2r[e] = clamp_rank(__ldg(a.e2r_g + e), G, a.err);
+
+    // ---- step 1 (source ranks given): counting sort of the tokens by s_t
+    if (with_src) {
+        for (int b = blockIdx.x; b < a.Bs; b += gridDim.x) {
+            if (tid < 64) cnt[tid] = 0;
+            __syncthreads();
+            const int t = b * kChunk + tid;
+            if (t < T) atomicAdd(&cnt[clamp_rank(__ldg(a.src + t), G, a.err)], 1);
+            __syncthreads();
+            if (tid < G) a.w.sblk[(size_t)b * G + tid] = cnt[tid];
+            __syncthreads();
+        }
+        if (!grid_barrier(bar, a.err)) return;
+        column_sums(a.w.sblk, a.Bs, G, tot, part);
+        if (tid == 0) {
+            int run = 0, ch = 0;
+            for (int s = 0; s < G; ++s) {
+                sh.soff[s] = run;
+                sh.scnt[s] = tot[s];
+                sh.cpre[s] = ch;
+                run += tot[s];
+                ch += (tot[s] + kChunk - 1) / kChunk;
+            }
+            sh.soff[G] = run;
+            sh.cpre[G] = ch;
+        }
+        __syncthreads();
+        for (int b = blockIdx.x; b < a.Bs; b += gridDim.x) {
+            column_sums(a.w.sblk, b, G, base, part);      // tokens of each shard in earlier chunks
+            for (int i = tid; i < kWarps * 64; i += kChunk) (&wcnt[0][0])[i] = 0;
+            __syncthreads();
+            const int t = b * kChunk + tid;
+            const bool act = t < T;
+            int s = act ? __ldg(a.src + t) : G;
+            if (act && (unsigned)s >= (unsigned)G) s = 0;
+            const unsigned peers = __match_any_sync(0xffffffffu, s);
+            const int rk = __popc(peers & ((1u << lane) - 1u));
+            if (act && rk == 0) wcnt[wid][s] = __popc(peers);
+            __syncthreads();
+            if (tid < G) {
+                int run = 0;
+                for (int q = 0; q < kWarps; ++q) {
+                    const int x = wcnt[q][tid];
+                    wcnt[q][tid] = run;
+                    run += x;
+                }
+            }
+            __syncthreads();
+            if (act) a.w.perm[sh.soff[s] + base[s] + wcnt[wid][s] + rk] = t;
+            __syncthreads();
+        }
+        if (!grid_barrier(bar, a.err)) return;
+    }
+    const int shard = with_src ? 0 : T / G;
+    const int nch = with_src ? 0 : max(1, (shard + kChunk - 1) / kChunk);
+    const int B = with_src ? sh.cpre[G] : G * nch;
+
+    // ---- step 2: destination sets, summary terms, per-chunk row counts
+    unsigned long long my[4] = {0, 0, 0, 0};
+    for (int b = blockIdx.x; b < B; b += gridDim.x) {
+        if (tid < 64) cnt[tid] = 0;
+        __syncthreads();
+        const ChunkRange c = chunk_range(b, T, G, with_src, sh);
+        const int p = c.p0 + tid;
+        unsigned long long m = 0;
+        if (p < c.p1) {
+            const int t = with_src ? __ldcg(a.w.perm + p) : p;
+            int v[K], rk[K];
+            load_token<K>(a.ids + (size_t)t * K, v);
+            int bad = token_error<K>(v, E);
+            if (!bad) bad = serving_ranks<K, PICKS>(v, e2r, a.picks, t, G, rk);
+            if (bad) {
+                record_error(a.err, bad);
+            } else {
+                unsigned long long nodes = 0;
+                int local = 0;
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    const int r = rk[j];
+                    m |= 1ull << r;
+                    nodes |= 1ull << (r / a.rpn);
+                    local += r == c.s;
+                }
+                my[0] += __popcll(m);
+                my[1] += __popcll(m & ~(1ull << c.s));
+                my[2] += local;
+                my[3] += __popcll(nodes & ~(1ull << (c.s / a.rpn)));
+            }
+            a.P.dest_mask[t] = m;
+        }
+        const uint32_t clo = warp_transpose32((uint32_t)m, lane);
+        const uint32_t chi = warp_transpose32((uint32_t)(m >> 32), lane);
+        if (lane < G && clo) atomicAdd(&cnt[lane], __popc(clo));
+        if (lane + 32 < G && chi) atomicAdd(&cnt[lane + 32], __popc(chi));
+        __syncthreads();
+        if (tid < G) a.w.blk[(size_t)b * G + tid] = cnt[tid];
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        unsigned long long x = my[i];
+        for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0) red[i][wid] = x;
+    }
+    __syncthreads();
+    if (tid < 4) {
+        unsigned long long x = 0;
+        for (int q = 0; q < kWarps; ++q) x += red[tid][q];
+        if (x) atomicAdd(&a.w.hdr->acc[tid], x);
+    }
+    if (!grid_barrier(bar, a.err)) return;
+
+    // ---- step 3: rank segments, then every chunk's rows
+    column_sums(a.w.blk, B, G, tot, part);
+    if (tid == 0) {
+        int run = 0;
+        for (int d = 0; d < G; ++d) { seg[d] = run; run += tot[d]; }
+        if (blockIdx.x == 0) a.P.offsets[G * G] = run;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        // offsets in (d, s) order and counts[s][d]: running sums over the
+        // chunks of each rank's column, read at the shards' chunk boundaries
+        if (tid < G) {
+            const int d = tid;
+            int run = 0, b = 0;
+            for (int s = 0; s < G; ++s) {
+                const int b1 = with_src ? sh.cpre[s + 1] : (s + 1) * nch;
+                const int at = run;
+                for (; b < b1; ++b) run += __ldcg(a.w.blk + (size_t)b * G + d);
+                a.P.offsets[d * G + s] = seg[d] + at;
+                a.P.counts[s * G + d] = run - at;
+            }
+        }
+        if (tid < 4) a.P.summary[tid] = (int64_t)__ldcg(&a.w.hdr->acc[tid]);
+        if (tid == 4) a.P.summary[4] = (int64_t)T * K;
+    }
+    for (int b = blockIdx.x; b < B; b += gridDim.x) {
+        column_sums(a.w.blk, b, G, base, part);       // rows of each rank in earlier chunks
+        if (tid < G) base[tid] += seg[tid];
+        const ChunkRange c = chunk_range(b, T, G, with_src, sh);
+        const int p = c.p0 + tid;
+        const bool act = p < c.p1;
+        int t = 0, v[K], r[K];
+        unsigned long long m = 0;
+        if (act) {
+            t = with_src ? __ldcg(a.w.perm + p) : p;
+            load_token<K>(a.ids + (size_t)t * K, v);
+            if (token_error<K>(v, E) == 0 && serving_ranks<K, PICKS>(v, e2r, a.picks, t, G, r) == 0) {
+#pragma unroll
+                for (int j = 0; j < K; ++j) m |= 1ull << r[j];
+            } else {
+#pragma unroll
+                for (int j = 0; j < K; ++j) a.P.row_of[(size_t)t * K + j] = -1;
+            }
+        }
+        const uint32_t clo = warp_transpose32((uint32_t)m, lane);
+        const uint32_t chi = warp_transpose32((uint32_t)(m >> 32), lane);
+        if (lane < G) {
+            colw[wid][lane] = clo;
+            wcnt[wid][lane] = __popc(clo);
+        }
+        if (lane + 32 < G) {
+            colw[wid][lane + 32] = chi;
+            wcnt[wid][lane + 32] = __popc(chi);
+        }
+        __syncthreads();
+        if (tid < G) {
+            int run = 0;
+            for (int q = 0; q < kWarps; ++q) {
+                const int x = wcnt[q][tid];
+                wcnt[q][tid] = run;
+                run += x;
+            }
+        }
+        __syncthreads();
+        const unsigned lt = (1u << lane) - 1u;
+        for (unsigned long long q = m; q; q &= q - 1) {
+            const int d = __ffsll((long long)q) - 1;
+            const int pos = base[d] + wcnt[wid][d] + __popc(colw[wid][d] & lt);
+            unsigned jm = 0;
+#pragma unroll
+            for (int j = 0; j < K; ++j)
+                if (r[j] == d) {
+                    jm |= 1u << j;
+                    a.P.row_of[(size_t)t * K + j] = pos;
+                }
+            a.P.row_token[pos] = t;
+            a.P.row_jmask[pos] = (uint8_t)jm;
+        }
+        __syncthreads();
+    }
+}
+
+// The single-launch plan when the shape allows it; MOE_ERR_UNSUPPORTED
+// otherwise (the caller then runs the separate kernels).
+template <int K, bool PICKS>
+moe_status launch_plan_fused(const int32_t *ids, int T, int E, int G, int rpn, const int32_t *e2r,
+                             const int32_t *picks, const int32_t *src_rank, const moe_plan &P, int32_t *err,
+                             const PlanWs &w, cudaStream_t s)
+{
+    const bool with_src = src_rank != nullptr;
+    const int Bs = with_src ? src_blocks(T) : 0;
+    const int Bc = chunk_blocks(T, G, with_src);
+    if (Bc > kFusedMaxChunks || Bs > kFusedMaxChunks) return MOE_ERR_UNSUPPORTED;
+    auto kern = plan_fused_kernel<K, PICKS>;
+    const size_t smem = PICKS ? 0 : sizeof(int32_t) * (size_t)E;
+    if (allow_smem(kern, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kChunk, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    if (per_sm < 1) return MOE_ERR_UNSUPPORTED;
+    FusedArgs a{};
+    a.ids = ids; a.T = T; a.E = E; a.G = G; a.rpn = rpn;
+    a.e2r_g = e2r; a.picks = picks; a.src = src_rank;
+    a.w = w; a.P = P; a.err = err; a.Bs = Bs;
+    const int grid = std::min(std::max(Bc, Bs), sm_count() * per_sm);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kChunk);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return MOE_ERR_CUDA;
+    moe_status st = launch_status();
+    if (st == MOE_OK) note_launches(1);
+    return st;
+}
+
+// 0: separate kernels (they run beside other kernels without waiting on one
+// another); 1: one cooperative launch when the chunk count allows
+std::atomic<int> g_plan_method{0};
+
 template <int K, bool PICKS>
 moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const int32_t *e2r, const int32_t *picks,
                        const int32_t *src_rank, const moe_plan &P, int32_t *err, const PlanWs &w,
                        cudaStream_t s)
 {
+    if (g_plan_method.load() == 1) {
+        const moe_status fs = launch_plan_fused<K, PICKS>(ids, T, E, G, rpn, e2r, picks, src_rank, P, err, w, s);
+        if (fs != MOE_ERR_UNSUPPORTED) return fs;
+    }
     const bool with_src = src_rank != nullptr;
     const size_t smem = PICKS ? 0 : sizeof(int32_t) * (size_t)E;
     int launched = 0;
@@ -531,6 +832,12 @@ moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const i
 }  // namespace moe
 
 using namespace moe;
+
+extern "C" int moe_plan_dispatch_method(int method)
+{
+    if (method < 0 || method > 1) return -1;
+    return g_plan_method.exchange(method);
+}
 
 extern "C" size_t moe_plan_dispatch_workspace(int T, int k, int G, int with_src_rank)
 {

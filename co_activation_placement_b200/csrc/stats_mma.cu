@@ -6,25 +6,35 @@
 // With X_l the E x T one-hot matrix (X_l[e][t] = 1 iff token t selects e at
 // layer l) these are the products
 //     C_l = X_l X_l^T,     M_l = X_l X_{l+1}^T,
-// an exact integer contraction over tokens.  Each thread block owns one
-// product and one token slice.  Per stage of 128 tokens it writes the ones of
-// its X tiles into shared memory (and clears the previous stage's ones, so a
-// tile is zeroed only once), then one thread issues tcgen05.mma kind::i8
-// (u8 x u8 -> s32, K-major operands, M = 128, N = E, K = 32 per instruction)
-// accumulating in tensor memory.  The work is split by warp: eight warps
-// write the tiles of a stage and arrive on its "full" mbarrier; a ninth warp
-// waits on it, issues the stage's MMAs and commits them to its "empty"
-// mbarrier, which the writers wait on before reusing the stage.  Three stages,
-// no block-wide barrier inside the loop.  At the end warps 0-3 read the
-// 128-lane accumulator with tcgen05.ld and store the block's partial counts;
-// a second kernel sums the slices (integer: order-free) and evaluates Ochiai
-// in fp64 exactly as the shared-memory histogram path does.
+// an exact integer contraction over tokens.  Each thread block owns one job
+// (C_l, M_l, or both from one tile of X_l) and one token slice.  Per stage of
+// 128 tokens eight builder warps write the stage's X tiles into shared
+// memory and arrive on its "full" mbarrier; a ninth warp waits on it, issues
+// tcgen05.mma kind::i8 (u8 x u8 -> s32, M = 128, K = 32 per instruction)
+// accumulating in tensor memory, and commits them to the stage's "empty"
+// mbarrier, which the builders wait on before rewriting the stage.  Three
+// stages, no block-wide barrier inside the loop.  At the end warps 0-3 read
+// the 128-lane accumulator with tcgen05.ld and store the block's partial
+// counts; a second kernel sums the slices (integer: order-free) and evaluates
+// Ochiai in fp64 exactly as the shared-memory histogram path does.
 //
-// Operand layout (K-major, 128-byte swizzle): an X tile of R rows (experts, R
-// a multiple of 128) and 128 tokens stores row r as 128 bytes, token u at
-//     r * 128 + (((u / 16) ^ (r % 8)) * 16) + (u % 16),
-// 8-row groups 1024 bytes apart; tiles start on 1024-byte boundaries.  The
-// MMA for tokens 32q..32q+31 starts its descriptors 32 q bytes into the rows.
+// Operand layout (MN-major, 128-byte swizzle).  A tile of X holds the stage's
+// 128 tokens as rows of expert bytes: token u's row is its one-hot vector,
+// one byte per expert, E padded to R = 128 or 256 ("rows").  Experts
+// 128a..128a+127 form the tile's a-th 16 KB block ("atom"); inside it token u
+// owns bytes [128 u, 128 u + 128), and its 16-byte chunk c (experts
+// 16c..16c+15 of the atom) sits at chunk position c ^ (u % 8), the 128-byte
+// swizzle.  A lane builds its token's whole row in registers -- the token's
+// picks as a bit mask, each 4 mask bits spread to 4 bytes by one multiply --
+// and writes it with 16-byte stores: eight lanes of a store cover all 32
+// banks, so the stores are conflict-free, and every byte of the row is
+// rewritten each stage (no clearing pass).  A repeated or out-of-range pick is
+// caught from the mask (popcount below k, or an id >= E) and leaves the row
+// empty.  For the MMA both operands are MN-major (the experts contiguous):
+// 32 tokens are 4 groups of 8 rows 1024 bytes apart (stride byte offset) and
+// the next 128 experts lie one atom, 16 KB, further on (leading byte offset).
+// The N = 256 operand [X_l; X_{l+1}] of a job that computes C_l and M_l in
+// one MMA is tile A followed by tile B, i.e. two atoms 16 KB apart.
 //
 // Every wait on an mbarrier is bounded (2 s of %globaltimer); a block that
 // gives up records MOE_DERR_TIMEOUT, waits (bounded again) for its last
@@ -44,21 +54,29 @@ constexpr int kMmaThreads = kBuildThreads + 32;
 constexpr int kTok = 128;                 // tokens per stage
 constexpr int kStages = 3;
 constexpr int kMmaReduceThreads = 256;
+constexpr int kAtom = kTok * 128;         // bytes of 128 experts x 128 tokens
 
-// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle
-// layout: rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte
-// offset 64 x 16 B), leading byte offset unused (1), descriptor version 1,
-// layout type 2 (128-byte swizzle).  addr may sit 32 k-bytes into a row: the
-// swizzle acts on the absolute address bits, as for the tile's own stores.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr)
+// Shared-memory matrix descriptor of an MN-major operand in the 128-byte
+// swizzle layout: start address, leading byte offset (the next 128 experts:
+// one atom, 16 KB), stride byte offset (the next 8 tokens: 1024 bytes),
+// descriptor version 1, layout type 2 (128-byte swizzle).  Start addresses
+// are multiples of 1024, so the base-offset field stays 0.
+__device__ __forceinline__ uint64_t smem_desc_mn(uint32_t addr)
 {
     uint64_t d = 0;
     d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-    d |= (uint64_t)1 << 16;
-    d |= (uint64_t)64 << 32;
+    d |= (uint64_t)(kAtom >> 4) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
     d |= (uint64_t)1 << 46;
     d |= (uint64_t)2 << 61;
     return d;
+}
+
+// Instruction descriptor of kind::i8: s32 accumulator, u8 A and B, both
+// MN-major, N columns, M = 128 rows.
+__host__ __device__ constexpr uint32_t idesc_u8_mn(int N)
+{
+    return (2u << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_u8(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc)
@@ -102,24 +120,48 @@ __device__ __forceinline__ void load_k(const int32_t *__restrict__ p, int (&v)[K
     }
 }
 
-// Byte of (expert row e, token slot u) in an X tile: rows of 128 bytes (the
-// stage's 128 tokens), the 16-byte chunk index XORed with e % 8 (the 128-byte
-// swizzle, which spreads a column's bytes over all banks).
-__device__ __forceinline__ int tile_byte(int e, int u)
+// 4 mask bits -> 4 bytes of value 0 or 1 (bit b to byte b): the multiplier
+// places copies of the nibble 7 bits apart, so bit b of copy b lands on bit
+// 8b, and no two copies' bits meet (no carries).
+__device__ __forceinline__ uint32_t nib_bytes(uint32_t x)
 {
-    return e * 128 + ((((u >> 4) ^ e) & 7) << 4) + (u & 15);
+    return ((x & 0xFu) * 0x00204081u) & 0x01010101u;
 }
 
-template <int K>
-__device__ __forceinline__ bool ids_in_range(const int (&v)[K], int E)
+// The one-hot row of one token as ROWS/32 mask words (bit e of word e/32 set
+// iff the token picks e); zero, with *bad set to the data-error code, when a
+// pick is out of [0, E) or repeats another (fewer than K distinct bits).
+template <int K, int ROWS>
+__device__ __forceinline__ void token_mask(const int (&v)[K], int E, uint32_t (&m)[ROWS / 32], int &bad)
 {
-    bool ok = true;
+    bool in_range = true;
 #pragma unroll
-    for (int a = 0; a < K; ++a) ok &= (unsigned)v[a] < (unsigned)E;
-    return ok;
+    for (int j = 0; j < K; ++j) in_range &= (unsigned)v[j] < (unsigned)E;
+#pragma unroll
+    for (int x = 0; x < ROWS / 32; ++x) m[x] = 0u;
+    bad = 0;
+    if (!in_range) {
+        bad = MOE_DERR_ID_RANGE;
+        return;
+    }
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        const uint32_t bit = 1u << (v[j] & 31);
+        const int w = v[j] >> 5;
+#pragma unroll
+        for (int x = 0; x < ROWS / 32; ++x) m[x] |= (w == x) ? bit : 0u;
+    }
+    int n = 0;
+#pragma unroll
+    for (int x = 0; x < ROWS / 32; ++x) n += __popc(m[x]);
+    if (n != K) {
+#pragma unroll
+        for (int x = 0; x < ROWS / 32; ++x) m[x] = 0u;
+        bad = MOE_DERR_ID_REPEAT;
+    }
 }
 
-template <int K>
+template <int K, int ROWS>
 __global__ void __launch_bounds__(kMmaThreads, 1)
 coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restrict__ part, int32_t *err)
 {
@@ -129,6 +171,7 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
     __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], done_bar;
     __shared__ uint32_t tmem_base_s;
 
+    constexpr int kMt = ROWS / 128;           // 128-row M tiles (= atoms per tile)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int job = blockIdx.x / G.S, slice = blockIdx.x % G.S;
     // a job: C of layer la (has_c) and/or M of layer la (has_m, tile B = layer lb)
@@ -148,21 +191,20 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
         has_m = true;
     }
     const int lb = has_m ? la + 1 : la;
-    const int T = G.T, E = G.E, rows = G.rows;
+    const int T = G.T, E = G.E;
     const int t0 = (int)((long long)T * slice / G.S), t1 = (int)((long long)T * (slice + 1) / G.S);
     const int nchunks = (t1 - t0 + kTok - 1) / kTok;
-    const int tile = rows * kTok;                      // bytes per X tile
+    constexpr int tile = ROWS * kTok;                  // bytes per X tile
     // stage s: tile A at s * per_stage, tile B right after it (M products)
     const int per_stage = has_m ? 2 * tile : tile;
-    // C_l and M_l in one MMA: tile B (X_{l+1}) follows tile A (X_l), so the
-    // 2*rows rows from tile A on are one N = 2*rows operand [X_l; X_{l+1}]
-    // (single 128-row tile, rows <= 128); D's columns [0, rows) are C_l's,
-    // [rows, 2 rows) M_l's
-    const bool stacked = has_c && has_m && G.mt == 1;
-    // TMEM column of the M accumulator
-    const uint32_t m_off = stacked ? (uint32_t)rows : (has_c ? (uint32_t)(G.mt * E) : 0u);
+    // C_l and M_l in one MMA (paired jobs have one 128-row tile): tile B
+    // (X_{l+1}) follows tile A (X_l), so the two form one N = 256 MN-major
+    // operand [X_l; X_{l+1}]; D's columns [0, 128) are C_l's, [128, 256) M_l's
+    const bool stacked = ROWS == 128 && has_c && has_m;
+    const uint32_t m_off = stacked ? (uint32_t)ROWS : 0u;   // TMEM column of the M accumulator
 
-    // zero the tiles once; later stages only set and clear their own ones
+    // zero the tiles once: the chunks past E stay zero, the others are
+    // rewritten whole every stage
     for (int i = tid * 16; i < kStages * per_stage; i += kMmaThreads * 16)
         *reinterpret_cast<uint4 *>(sm + i) = make_uint4(0, 0, 0, 0);
     if (tid == 0) {
@@ -185,67 +227,51 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
     bool ok = true;
 
     if (warp < kMmaWarp) {
-        // ---- builders: token slot u = tid % 128; threads < 128 write tile A
-        // (layer la), threads >= 128 tile B (layer lb, M only).  A token with
-        // an invalid pick leaves its column of that tile empty: it then adds
-        // nothing to the products that tile enters.  Repeats are checked for
-        // the layers whose C this launch computes (all layers when C is not
-        // wanted).
-        const int u = tid & (kTok - 1);
-        const bool writer = tid < kTok || has_m;
-        const int my_layer = (tid < kTok) ? la : lb;
-        const int my_tile = (tid < kTok) ? 0 : tile;
-        const bool check_repeat = (tid < kTok) ? (has_c || G.nc == 0) : (G.nc == 0);
-        // ids whose ones are in the tiles of chunks c-3, c-2, c-1 (registers, rotated)
-        int prevA[K], prevB[K], prevC[K];
-        bool setA = false, setB = false, setC = false;
+        // ---- builders.  With tile B (has_m): warps 0-3 write tile A (layer
+        // la), warps 4-7 tile B (layer lb), warp w the tokens 32 (w % 4) + lane
+        // of the stage.  Without it, warps w and w + 4 share tile A's rows:
+        // the first writes the low half of the used chunks, the second the
+        // high half.
+        const int u = (warp & 3) * 32 + lane;
+        const int nch = (E + 15) >> 4;                 // chunks holding experts < E
+        int c_lo = 0, c_hi = nch, my_layer = la, my_tile = 0;
+        if (has_m) {
+            if (warp >= 4) { my_layer = lb; my_tile = tile; }
+        } else {
+            c_lo = warp >= 4 ? nch / 2 : 0;
+            c_hi = warp >= 4 ? nch : nch / 2;
+        }
+        const int32_t *lay = ids + (size_t)my_layer * T * K;
         // ids of the stage being built (cur) and of the next two (n1, n2): the
         // loads for stage c+2 are issued before stage c waits and builds
         int cur_v[K], n1_v[K], n2_v[K];
         auto fetch = [&](int c, int (&v)[K]) {
             const int t = t0 + c * kTok + u;
-            if (writer && c < nchunks && t < t1) load_k<K>(ids + ((size_t)my_layer * T + t) * K, v);
+            if (c < nchunks && t < t1) load_k<K>(lay + (size_t)t * K, v);
         };
         fetch(0, cur_v);
         fetch(1, n1_v);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages, n = c / kStages;
             fetch(c + 2, n2_v);
+            uint32_t m[ROWS / 32];
+            int bad = 0;
+            const int t = t0 + c * kTok + u;
+            if (t < t1) {
+                token_mask<K, ROWS>(cur_v, E, m, bad);
+                if (bad) record_error(err, bad);
+            } else {
+#pragma unroll
+                for (int x = 0; x < ROWS / 32; ++x) m[x] = 0u;
+            }
             if (c >= kStages && !mbar_wait(&empty_bar[s], (n - 1) & 1)) { ok = false; break; }
-            uint8_t *t_s = sm + s * per_stage + my_tile;
-            if (writer) {
-                if (setA) {                            // chunk c-3 used this stage
+            uint8_t *row = sm + s * per_stage + my_tile + u * 128;
 #pragma unroll
-                    for (int j = 0; j < K; ++j) t_s[tile_byte(prevA[j], u)] = 0;
-                }
-#pragma unroll
-                for (int j = 0; j < K; ++j) { prevA[j] = prevB[j]; prevB[j] = prevC[j]; }
-                setA = setB;
-                setB = setC;
-                setC = false;
-                const int t = t0 + c * kTok + u;
-                if (t < t1) {
-                    if (!ids_in_range<K>(cur_v, E)) {
-                        record_error(err, MOE_DERR_ID_RANGE);
-                    } else {
-                        // a pick whose byte is already set repeats an earlier pick
-                        uint32_t seen = 0;
-#pragma unroll
-                        for (int j = 0; j < K; ++j) {
-                            uint8_t *b = t_s + tile_byte(cur_v[j], u);
-                            if (check_repeat) seen |= *b;
-                            *b = 1;
-                        }
-                        if (seen) {
-#pragma unroll
-                            for (int j = 0; j < K; ++j) t_s[tile_byte(cur_v[j], u)] = 0;
-                            record_error(err, MOE_DERR_ID_REPEAT);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < K; ++j) prevC[j] = cur_v[j];
-                            setC = true;
-                        }
-                    }
+            for (int ch = 0; ch < ROWS / 16; ++ch) {
+                if (ch >= c_lo && ch < c_hi) {
+                    const uint32_t h = m[ch >> 1] >> ((ch & 1) * 16);
+                    const uint4 o = make_uint4(nib_bytes(h), nib_bytes(h >> 4), nib_bytes(h >> 8), nib_bytes(h >> 12));
+                    *reinterpret_cast<uint4 *>(row + (ch >> 3) * kAtom + (((ch ^ u) & 7) << 4)) = o;
                 }
             }
             // the stores become visible to the tensor cores; one arrival per warp
@@ -256,10 +282,11 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
             for (int j = 0; j < K; ++j) { cur_v[j] = n1_v[j]; n1_v[j] = n2_v[j]; }
         }
     } else {
-        // ---- MMA warp: per full stage, one lane issues K / 32 x M tiles MMAs
-        // into each accumulator and commits them to the stage's empty barrier
-        const uint32_t idesc = (2u << 4) | ((uint32_t)(E >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-        const uint32_t idesc2 = (2u << 4) | ((uint32_t)((2 * rows) >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+        // ---- MMA warp: per full stage, one lane issues 4 k-steps of 32 tokens
+        // (x the M tiles) into each accumulator and commits them to the
+        // stage's empty barrier
+        constexpr uint32_t idesc = idesc_u8_mn(ROWS);
+        constexpr uint32_t idesc2 = ROWS == 128 ? idesc_u8_mn(256) : 0u;   // stacked jobs have ROWS = 128
         const uint32_t base = smem_addr(sm);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages, n = c / kStages;
@@ -270,17 +297,19 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
                 const uint32_t b0 = a0 + tile;
 #pragma unroll
                 for (int ks = 0; ks < kTok / 32; ++ks) {
-                    const uint32_t koff = (uint32_t)(32 * ks);              // 32 tokens = 32 bytes of each row
+                    const uint32_t koff = (uint32_t)(ks * 32 * 128);     // 32 token rows
                     const uint32_t acc = (c > 0 || ks > 0) ? 1u : 0u;
-                    const uint64_t dA = smem_desc_sw128(a0 + koff);         // all E rows of A as the N operand
-                    const uint64_t dB = smem_desc_sw128(b0 + koff);
-                    for (int mi = 0; mi < G.mt; ++mi) {
-                        const uint64_t da = smem_desc_sw128(a0 + koff + (uint32_t)(mi * 128 * 128));
+                    const uint64_t dA = smem_desc_mn(a0 + koff);          // all rows of tile A as the N operand
+                    const uint64_t dB = smem_desc_mn(b0 + koff);
+#pragma unroll
+                    for (int mi = 0; mi < kMt; ++mi) {
+                        const uint64_t da = smem_desc_mn(a0 + koff + (uint32_t)(mi * kAtom));
                         if (stacked) {
                             mma_u8(tmem, da, dA, idesc2, acc);
+                        } else if (has_c) {
+                            mma_u8(tmem + (uint32_t)(mi * ROWS), da, dA, idesc, acc);
                         } else {
-                            if (has_c) mma_u8(tmem + (uint32_t)(mi * E), da, dA, idesc, acc);
-                            if (has_m) mma_u8(tmem + m_off + (uint32_t)(mi * E), da, dB, idesc, acc);
+                            mma_u8(tmem + (uint32_t)(mi * ROWS), da, dB, idesc, acc);
                         }
                     }
                 }
@@ -304,12 +333,12 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
             const int prod = q == 0 ? la : G.nc + la;
             const uint32_t col0 = q == 0 ? 0u : m_off;
             uint32_t *dst = part + ((size_t)prod * G.S + slice) * E * E;
-            for (int mi = 0; mi < G.mt; ++mi) {
+            for (int mi = 0; mi < kMt; ++mi) {
                 const int row = mi * 128 + warp * 32 + lane;
                 for (int c0 = 0; c0 < E; c0 += 16) {
                     uint32_t r[16];
                     if (nchunks > 0) {
-                        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + col0 + (uint32_t)(mi * E + c0);
+                        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + col0 + (uint32_t)(mi * ROWS + c0);
                         asm volatile(
                             "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
                             "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
@@ -385,13 +414,19 @@ coact_mma_reduce_kernel(MmaGeom G, const uint32_t *__restrict__ part, uint32_t *
     }
 }
 
-template <int K>
+template <int K, int ROWS>
 moe_status launch_mma(const int32_t *ids, const MmaGeom &g, uint32_t *part, int32_t *err, cudaStream_t s)
 {
     const size_t smem = mma_smem_bytes(g);
-    if (allow_smem(coact_mma_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
-    coact_mma_kernel<K><<<g.J * g.S, kMmaThreads, smem, s>>>(ids, g, part, err);
+    if (allow_smem(coact_mma_kernel<K, ROWS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    coact_mma_kernel<K, ROWS><<<g.J * g.S, kMmaThreads, smem, s>>>(ids, g, part, err);
     return launch_status();
+}
+
+template <int K>
+moe_status launch_mma_rows(const int32_t *ids, const MmaGeom &g, uint32_t *part, int32_t *err, cudaStream_t s)
+{
+    return g.rows == 128 ? launch_mma<K, 128>(ids, g, part, err, s) : launch_mma<K, 256>(ids, g, part, err, s);
 }
 
 }  // namespace
@@ -408,11 +443,11 @@ bool make_mma_geom(int L, int T, int k, int E, bool want_c, bool want_t, MmaGeom
     g.P = g.nc + nm;
     if (g.P == 0) return false;
     // C_l and M_l share layer l's tile when both accumulators fit tensor memory
-    g.paired = g.nc > 0 && nm > 0 && 2 * g.mt * E <= 512;
+    g.paired = g.nc > 0 && nm > 0 && g.mt == 1 && 2 * g.rows <= 512;
     g.J = g.paired ? L : g.P;
     // paired implies one 128-row tile (2 * mt * E <= 512); its C and M share one
-    // N = 2 * rows accumulator
-    const int acc_cols = g.paired ? 2 * g.rows : g.mt * E;
+    // N = 2 * rows accumulator; otherwise one product of mt tiles of N = rows
+    const int acc_cols = g.paired ? 2 * g.rows : g.mt * g.rows;
     int cols = 32;
     while (cols < acc_cols) cols <<= 1;
     g.cols = cols;
@@ -444,14 +479,14 @@ moe_status coact_mma(const int32_t *ids, const MmaGeom &g, uint32_t *part, uint3
 {
     moe_status st = MOE_ERR_ARG;
     switch (g.k) {
-    case 1: st = launch_mma<1>(ids, g, part, err, stream); break;
-    case 2: st = launch_mma<2>(ids, g, part, err, stream); break;
-    case 3: st = launch_mma<3>(ids, g, part, err, stream); break;
-    case 4: st = launch_mma<4>(ids, g, part, err, stream); break;
-    case 5: st = launch_mma<5>(ids, g, part, err, stream); break;
-    case 6: st = launch_mma<6>(ids, g, part, err, stream); break;
-    case 7: st = launch_mma<7>(ids, g, part, err, stream); break;
-    case 8: st = launch_mma<8>(ids, g, part, err, stream); break;
+    case 1: st = launch_mma_rows<1>(ids, g, part, err, stream); break;
+    case 2: st = launch_mma_rows<2>(ids, g, part, err, stream); break;
+    case 3: st = launch_mma_rows<3>(ids, g, part, err, stream); break;
+    case 4: st = launch_mma_rows<4>(ids, g, part, err, stream); break;
+    case 5: st = launch_mma_rows<5>(ids, g, part, err, stream); break;
+    case 6: st = launch_mma_rows<6>(ids, g, part, err, stream); break;
+    case 7: st = launch_mma_rows<7>(ids, g, part, err, stream); break;
+    case 8: st = launch_mma_rows<8>(ids, g, part, err, stream); break;
     }
     if (st != MOE_OK) return st;
     note_launches(1);

@@ -31,8 +31,9 @@ moe_coact_stats does from its own).
 EPGroup is the multi-process form: torch.distributed (NCCL) for the counts,
 the statistics and the meetings; torch's symmetric memory for buffers that
 every device of the group can address.  EPEmulation runs the same phases for
-W virtual devices on one GPU, each with buffers of its own, one after another
-on one stream.
+W virtual devices on one GPU, each with buffers and a CUDA stream of its own:
+within a phase the devices' launches run side by side, as separate GPUs
+would, and each meeting is a join of the W streams.
 """
 from __future__ import annotations
 
@@ -122,6 +123,7 @@ class EPEmulation:
         counts_all = self.shards[0].counts_all
         for s in self.shards:
             s.counts_all = counts_all
+        self.streams = None
         self.recv = [torch.empty((recv_cap, d), dtype=dtype, device=device) for _ in range(W)]
         self.recv_base = _bases(self.recv, device)
         self.prereduce = prereduce
@@ -138,27 +140,43 @@ class EPEmulation:
     def _part(self, a: torch.Tensor, h: int) -> torch.Tensor:
         return a[h * self.Tl:(h + 1) * self.Tl]
 
+    def _phase(self, fn):
+        """fn(shard) for every device on the device's own stream, all of them
+        after the work enqueued so far on the current stream and before any
+        work enqueued on it afterwards (a meeting of the W devices)."""
+        main = torch.cuda.current_stream()
+        if self.streams is None:
+            self.streams = [torch.cuda.Stream(device=main.device) for _ in range(self.W)]
+        start = torch.cuda.Event()
+        start.record(main)
+        for s, st in zip(self.shards, self.streams):
+            st.wait_event(start)
+            with torch.cuda.stream(st):
+                fn(s)
+            done = torch.cuda.Event()
+            done.record(st)
+            main.wait_event(done)
+
     def step(self, ids: torch.Tensor, x: torch.Tensor, gates: torch.Tensor, expert_to_rank: torch.Tensor):
         """One layer for all T tokens (device h owns tokens [h*T/W, (h+1)*T/W)); returns the W outputs."""
         sh = self.shards
-        for s in sh:
-            s.plan_layer(self._part(ids, s.me), expert_to_rank)
+        self._phase(lambda s: s.plan_layer(self._part(ids, s.me), expert_to_rank))
         sh[0].counts_all.copy_(torch.cat([s.my_counts() for s in sh]))
-        for s in sh:
+
+        def send(s):
             s.routes()
-        for s in sh:
             s.dispatch(self._part(x, s.me), self.recv_base, self.recv_cap)
-        if self.prereduce:
-            for s in sh:
+            if self.prereduce:
                 s.dispatch_gates(self._part(ids, s.me), self._part(gates, s.me), self.e_base, self.w_base,
                                  self.recv_cap)
-            for s in sh:
-                s.experts(self.recv[s.me], self.recv_e[s.me], self.recv_w[s.me], self.scale, self.y[s.me])
+        self._phase(send)
+        if self.prereduce:
+            self._phase(lambda s: s.experts(self.recv[s.me], self.recv_e[s.me], self.recv_w[s.me], self.scale,
+                                            self.y[s.me]))
             y_base = self.y_base
         else:
             y_base = self.recv_base
-        for s in sh:
-            s.combine(y_base, self.dtype, self.recv_cap, self._part(gates, s.me))
+        self._phase(lambda s: s.combine(y_base, self.dtype, self.recv_cap, self._part(gates, s.me)))
         return [s.out for s in sh]
 
     def errors(self) -> List[int]:

@@ -39,13 +39,15 @@
  *    caller zeroes `err` and reads it after synchronising.  When it is
  *    non-zero the outputs of that call are unspecified.  Kernels never trap.
  *  - Calls keep no state between invocations except the global launch
- *    counter, the statistics method setting (moe_coact_stats_method) and the
- *    static scratch of moe_plan_dispatch_static.  Workspace ("ws") is
+ *    counter, the method settings (moe_coact_stats_method,
+ *    moe_plan_dispatch_method) and the static scratch of
+ *    moe_plan_dispatch_static.  Workspace ("ws") is
  *    caller-provided device memory of at least the size the matching
  *    *_workspace query returns, 256-byte aligned.
  *  - The only kernels that wait on other blocks or on the tensor cores
- *    (moe_shuffle_balanced, the tensor-core method of moe_coact_stats) give
- *    every wait a 2 s limit and then report MOE_DERR_TIMEOUT in `err`.
+ *    (moe_shuffle_balanced, moe_assign_replicas_capped, the single-launch
+ *    method of the dispatch plan, the tensor-core method of moe_coact_stats)
+ *    give every wait a 2 s limit and then report MOE_DERR_TIMEOUT in `err`.
  */
 #ifndef MOE_COACT_H
 #define MOE_COACT_H
@@ -159,6 +161,17 @@ typedef struct {
  * T*k < 2^31.  Data errors: MOE_DERR_ID_RANGE, MOE_DERR_ID_REPEAT,
  * MOE_DERR_RANK_RANGE. */
 size_t moe_plan_dispatch_workspace(int T, int k, int G, int with_src_rank);
+/* How the plan is launched (process-wide; returns the previous setting, or -1
+ * for an invalid argument): 0 = default: separate kernels (counting sort by
+ * source, counts, scatter), each of which runs beside other work on the GPU
+ * without waiting on it; 1 = one cooperative launch whose phases are
+ * separated by grid barriers, when the plan has at most 512 chunks of 1024
+ * tokens (else the separate kernels run).  A cooperative launch needs all its
+ * blocks resident at once, so use 1 where the plan runs in line on its stream
+ * rather than beside long kernels on another.  Results are identical; the
+ * setting also applies to moe_plan_dispatch_ranks and
+ * moe_plan_dispatch_static and affects calls issued after it returns. */
+int moe_plan_dispatch_method(int method);
 moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E, int G, int rpn,
                              const int32_t *expert_to_rank, const int32_t *src_rank,
                              const moe_plan *plan, int32_t *err,

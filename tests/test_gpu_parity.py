@@ -140,15 +140,38 @@ def check_plan(p, o, T, k):
     assert (host(p.row_of)[:T] == o["row_of"]).all()
 
 
+@pytest.mark.parametrize("method", [0, 1])
 @pytest.mark.parametrize("shape", PLAN_SHAPES)
-def test_plan_small(cap, shape):
+def test_plan_small(cap, shape, method):
+    """Both launch methods: separate kernels (0) and one cooperative launch (1)."""
     T, k, E, G, rpn, mode = shape
     rng = np.random.default_rng(T + k + E + G)
     ids = clustered_ids(rng, 1, T, E, k)[0]
     e2r = rng.permutation(orc.place_uniform(E, G)).astype(np.int32)
     src = make_src(rng, mode, T, G)
-    p = cap.plan_dispatch(dev(ids), E, G, rpn, dev(e2r), src_rank=None if src is None else dev(src))
+    prev = cap.plan_dispatch_method(method)
+    try:
+        p = cap.plan_dispatch(dev(ids), E, G, rpn, dev(e2r), src_rank=None if src is None else dev(src))
+    finally:
+        cap.plan_dispatch_method(prev)
     check_plan(p, orc.plan(ids, E, G, rpn, e2r, src_rank=src), T, k)
+
+
+@pytest.mark.parametrize("T,G,mode", [(131072, 64, "rand"), (524288, 64, None), (16384, 8, "skew"), (262144, 32, "rand")])
+def test_plan_single_launch_large(cap, T, G, mode):
+    """The single-launch plan where blocks loop over several chunks (more
+    chunks than resident blocks) and at its chunk limit, against the oracle."""
+    k, E = 8, 64
+    rng = np.random.default_rng(T + G)
+    ids = clustered_ids(rng, 1, T, E, k)[0]
+    e2r = rng.permutation(orc.place_uniform(E, G)).astype(np.int32)
+    src = make_src(rng, mode, T, G)
+    prev = cap.plan_dispatch_method(1)
+    try:
+        p = cap.plan_dispatch(dev(ids), E, G, 8, dev(e2r), src_rank=None if src is None else dev(src))
+    finally:
+        cap.plan_dispatch_method(prev)
+    check_plan(p, orc.plan(ids, E, G, 8, e2r, src_rank=src), T, k)
 
 
 def test_plan_reuses_workspace_and_buffers(cap):
