@@ -191,6 +191,7 @@ plan_src_count_kernel(const int32_t *__restrict__ src_rank, int T, int G, PlanWs
     __shared__ int32_t tot[64];
     __shared__ int32_t seg[kChunk];
     __shared__ bool last;
+    pdl_release();                        // the scatter's prologue reads only src_rank
     if (threadIdx.x < G) hist[threadIdx.x] = 0;
     __syncthreads();
     const int t = blockIdx.x * kChunk + threadIdx.x;
@@ -246,6 +247,8 @@ plan_src_scatter_kernel(const int32_t *__restrict__ src_rank, int T, int G, Plan
         }
     }
     __syncthreads();
+    pdl_wait();                           // the counts and their scan
+    pdl_release();
     if (act) {
         const int pos = __ldcg(w.soff + s) + __ldcg(w.sblk_pref + (size_t)blockIdx.x * G + s) + wbase[wid][s] + rank;
         w.perm[pos] = t;
@@ -342,8 +345,10 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
     if (!PICKS)
         for (int e = threadIdx.x; e < E; e += kChunk) e2r[e] = clamp_rank(__ldg(e2r_g + e), G, err);
     if (threadIdx.x < 64) cnt[threadIdx.x] = 0;
-    load_shards(sh, G, with_src, w);
+    load_shards(sh, G, with_src, w);      // from the source count, two launches back: complete
     __syncthreads();
+    pdl_wait();                           // the source permutation
+    pdl_release();
 
     const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, sh);
     unsigned long long my[4] = {0, 0, 0, 0};
@@ -439,23 +444,28 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
     __shared__ uint32_t colw[kWarps][64];      // lanes of the warp with a row for the rank
     __shared__ ShardTable sh;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    // prologue, before the counts are complete: the shard table and the
+    // source permutation (written two and more launches back), the tokens'
+    // destination sets and their per-warp ranks
     load_shards(sh, G, with_src, w);
     __syncthreads();
     const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, sh);
-    if (!c.active) return;
+    if (!c.active) {
+        pdl_wait();
+        return;
+    }
     if (!PICKS)
         for (int e = threadIdx.x; e < E; e += kChunk) {
             const int r = __ldg(e2r_g + e);
             e2r[e] = (unsigned)r >= (unsigned)G ? 0 : r;
         }
-    if (threadIdx.x < G)
-        base[threadIdx.x] = __ldcg(P.offsets + threadIdx.x * G) + __ldcg(w.blk_pref + (size_t)blockIdx.x * G + threadIdx.x);
     __syncthreads();
 
     const int p = c.p0 + threadIdx.x;
     const bool act = p < c.p1;
     int t = 0, v[K], r[K];
     unsigned long long m = 0;
+    bool bad = false;
     if (act) {
         t = with_src ? __ldcg(w.perm + p) : p;
         load_token<K>(ids + (size_t)t * K, v);
@@ -463,8 +473,7 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
 #pragma unroll
             for (int j = 0; j < K; ++j) m |= 1ull << r[j];
         } else {
-#pragma unroll
-            for (int j = 0; j < K; ++j) P.row_of[(size_t)t * K + j] = -1;
+            bad = true;
         }
     }
     // column d of the warp's 32 x G destination bit matrix: which lanes send to rank d
@@ -486,6 +495,13 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
             wcnt[q][threadIdx.x] = run;
             run += x;
         }
+    }
+    pdl_wait();                           // the counts, offsets and chunk prefixes
+    if (threadIdx.x < G)
+        base[threadIdx.x] = __ldcg(P.offsets + threadIdx.x * G) + __ldcg(w.blk_pref + (size_t)blockIdx.x * G + threadIdx.x);
+    if (bad) {
+#pragma unroll
+        for (int j = 0; j < K; ++j) P.row_of[(size_t)t * K + j] = -1;
     }
     __syncthreads();
     // each lane writes its own rows: rank within the warp = earlier lanes with that rank
@@ -811,17 +827,29 @@ moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const i
     const bool with_src = src_rank != nullptr;
     const size_t smem = PICKS ? 0 : sizeof(int32_t) * (size_t)E;
     int launched = 0;
+    // the first kernel starts after everything before the call; each later
+    // one may start early (programmatic dependent launch) and waits inside
+    // for its predecessor before reading what that one writes
     if (with_src) {
         const int Bs = src_blocks(T);
         plan_src_count_kernel<<<Bs, kChunk, 0, s>>>(src_rank, T, G, w, err);
-        plan_src_scatter_kernel<<<Bs, kChunk, 0, s>>>(src_rank, T, G, w);
+        if (launch_pdl(plan_src_scatter_kernel, dim3(Bs), dim3(kChunk), 0, s, src_rank, T, G, w) != cudaSuccess)
+            return MOE_ERR_CUDA;
         launched += 2;
     }
     const int Bc = chunk_blocks(T, G, with_src);
     if (allow_smem(plan_count_kernel<K, PICKS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
     if (allow_smem(plan_scatter_kernel<K, PICKS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
-    plan_count_kernel<K, PICKS><<<Bc, kChunk, smem, s>>>(ids, T, E, G, rpn, e2r, picks, with_src, w, P, err);
-    plan_scatter_kernel<K, PICKS><<<Bc, kChunk, smem, s>>>(ids, T, E, G, e2r, picks, with_src, w, P);
+    if (with_src) {
+        if (launch_pdl(plan_count_kernel<K, PICKS>, dim3(Bc), dim3(kChunk), smem, s, ids, T, E, G, rpn, e2r, picks,
+                       with_src, w, P, err) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    } else {
+        plan_count_kernel<K, PICKS><<<Bc, kChunk, smem, s>>>(ids, T, E, G, rpn, e2r, picks, with_src, w, P, err);
+    }
+    if (launch_pdl(plan_scatter_kernel<K, PICKS>, dim3(Bc), dim3(kChunk), smem, s, ids, T, E, G, e2r, picks, with_src,
+                   w, P) != cudaSuccess)
+        return MOE_ERR_CUDA;
     launched += 2;
     moe_status st = launch_status();
     if (st == MOE_OK) note_launches(launched);

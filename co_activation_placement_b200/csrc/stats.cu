@@ -389,11 +389,14 @@ moe_status launch_hist(const int32_t *ids, const StatsGeom &g, uint32_t *part, i
 using namespace moe;
 
 namespace {
-// 0: default (the histograms: on B200 they measured as fast as or faster than
-// the tensor-core contraction for E <= 256, k = 8, where building the one-hot
-// operand tiles costs about what the counter increments do); 1: histograms;
-// 2: tensor cores where the shape allows
+// 0: default -- the tensor cores for E >= 128 where the shape allows (on B200
+// they measured faster than the histograms at E = 128 and 256 with k = 8),
+// the histograms below (at E = 64 the operand tiles, padded to 128 experts,
+// cost more than the counter increments); 1: histograms; 2: tensor cores
+// where the shape allows
 std::atomic<int> g_coact_method{0};
+
+bool tensor_method(int method, int E) { return method == 2 || (method == 0 && E >= 128); }
 }  // namespace
 
 extern "C" int moe_coact_stats_method(int method)
@@ -407,7 +410,7 @@ extern "C" int moe_coact_stats_path(int L, int T, int k, int E, int with_trans)
     if (L < 1 || T < 1 || k < 1 || k > 8 || E < k || E > 1024) return 0;
     const int method = g_coact_method.load();
     MmaGeom mg;
-    if (method == 2 && make_mma_geom(L, T, k, E, true, with_trans != 0, mg)) return 2;
+    if (tensor_method(method, E) && make_mma_geom(L, T, k, E, true, with_trans != 0, mg)) return 2;
     return 1;
 }
 
@@ -447,7 +450,7 @@ extern "C" moe_status moe_coact_stats(const int32_t *ids, int L, int T, int k, i
     }
     const int method = g_coact_method.load();
     MmaGeom mg;
-    if (method == 2 && aligned16(ids) && make_mma_geom(L, T, k, E, want_c, want_t, mg)) {
+    if (tensor_method(method, E) && aligned16(ids) && make_mma_geom(L, T, k, E, want_c, want_t, mg)) {
         const size_t need = mma_partial_words(mg) * sizeof(uint32_t);
         if (!ws || !aligned256(ws) || ws_bytes < need) return MOE_ERR_WORKSPACE;
         return coact_mma(ids, mg, static_cast<uint32_t *>(ws), coact, ochiai, trans, err, stream);

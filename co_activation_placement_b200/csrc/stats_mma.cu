@@ -14,9 +14,11 @@
 // accumulating in tensor memory, and commits them to the stage's "empty"
 // mbarrier, which the builders wait on before rewriting the stage.  Three
 // stages, no block-wide barrier inside the loop.  At the end warps 0-3 read
-// the 128-lane accumulator with tcgen05.ld and store the block's partial
-// counts; a second kernel sums the slices (integer: order-free) and evaluates
-// Ochiai in fp64 exactly as the shared-memory histogram path does.
+// the 128-lane accumulator with tcgen05.ld, stage it in shared memory row by
+// row and add it into the job's count matrices with bulk asynchronous
+// reductions (cp.reduce.async.bulk .add.u32, integer: order-free); a second
+// kernel copies the counts out and evaluates Ochiai in fp64 exactly as the
+// shared-memory histogram path does.
 //
 // Operand layout (MN-major, 128-byte swizzle).  A tile of X holds the stage's
 // 128 tokens as rows of expert bytes: token u's row is its one-hot vector,
@@ -24,17 +26,15 @@
 // 128a..128a+127 form the tile's a-th 16 KB block ("atom"); inside it token u
 // owns bytes [128 u, 128 u + 128), and its 16-byte chunk c (experts
 // 16c..16c+15 of the atom) sits at chunk position c ^ (u % 8), the 128-byte
-// swizzle.  A lane builds its token's whole row in registers -- the token's
-// picks as a bit mask, each 4 mask bits spread to 4 bytes by one multiply --
-// and writes it with 16-byte stores: eight lanes of a store cover all 32
-// banks, so the stores are conflict-free, and every byte of the row is
-// rewritten each stage (no clearing pass).  A repeated or out-of-range pick is
-// caught from the mask (popcount below k, or an id >= E) and leaves the row
-// empty.  For the MMA both operands are MN-major (the experts contiguous):
-// 32 tokens are 4 groups of 8 rows 1024 bytes apart (stride byte offset) and
-// the next 128 experts lie one atom, 16 KB, further on (leading byte offset).
-// The N = 256 operand [X_l; X_{l+1}] of a job that computes C_l and M_l in
-// one MMA is tile A followed by tile B, i.e. two atoms 16 KB apart.
+// swizzle.  A lane writes its own token's row: zeros with 16-byte stores
+// (eight lanes of a store cover all 32 banks, so these are conflict-free),
+// then one byte store per pick.  A token with a repeated or out-of-range pick
+// keeps an empty row and reports the data error.  For the MMA both operands
+// are MN-major (the experts contiguous): 32 tokens are 4 groups of 8 rows
+// 1024 bytes apart (stride byte offset) and the next 128 experts lie one
+// atom, 16 KB, further on (leading byte offset).  The N = 256 operand
+// [X_l; X_{l+1}] of a job that computes C_l and M_l in one MMA is tile A
+// followed by tile B, i.e. two atoms 16 KB apart.
 //
 // Every wait on an mbarrier is bounded (2 s of %globaltimer); a block that
 // gives up records MOE_DERR_TIMEOUT, waits (bounded again) for its last
@@ -120,50 +120,25 @@ __device__ __forceinline__ void load_k(const int32_t *__restrict__ p, int (&v)[K
     }
 }
 
-// 4 mask bits -> 4 bytes of value 0 or 1 (bit b to byte b): the multiplier
-// places copies of the nibble 7 bits apart, so bit b of copy b lands on bit
-// 8b, and no two copies' bits meet (no carries).
-__device__ __forceinline__ uint32_t nib_bytes(uint32_t x)
+// 0 when the token's K picks are distinct and in [0, E), else the device
+// error code: the range check, then the pairs compared (a sorting network
+// costs about as much for K <= 8).
+template <int K>
+__device__ __forceinline__ int token_check(const int (&v)[K], int E)
 {
-    return ((x & 0xFu) * 0x00204081u) & 0x01010101u;
-}
-
-// The one-hot row of one token as ROWS/32 mask words (bit e of word e/32 set
-// iff the token picks e); zero, with *bad set to the data-error code, when a
-// pick is out of [0, E) or repeats another (fewer than K distinct bits).
-template <int K, int ROWS>
-__device__ __forceinline__ void token_mask(const int (&v)[K], int E, uint32_t (&m)[ROWS / 32], int &bad)
-{
-    bool in_range = true;
+    bool in_range = true, rep = false;
 #pragma unroll
-    for (int j = 0; j < K; ++j) in_range &= (unsigned)v[j] < (unsigned)E;
+    for (int a = 0; a < K; ++a) {
+        in_range &= (unsigned)v[a] < (unsigned)E;
 #pragma unroll
-    for (int x = 0; x < ROWS / 32; ++x) m[x] = 0u;
-    bad = 0;
-    if (!in_range) {
-        bad = MOE_DERR_ID_RANGE;
-        return;
+        for (int b = 0; b < a; ++b) rep |= v[a] == v[b];
     }
-#pragma unroll
-    for (int j = 0; j < K; ++j) {
-        const uint32_t bit = 1u << (v[j] & 31);
-        const int w = v[j] >> 5;
-#pragma unroll
-        for (int x = 0; x < ROWS / 32; ++x) m[x] |= (w == x) ? bit : 0u;
-    }
-    int n = 0;
-#pragma unroll
-    for (int x = 0; x < ROWS / 32; ++x) n += __popc(m[x]);
-    if (n != K) {
-#pragma unroll
-        for (int x = 0; x < ROWS / 32; ++x) m[x] = 0u;
-        bad = MOE_DERR_ID_REPEAT;
-    }
+    return !in_range ? MOE_DERR_ID_RANGE : (rep ? MOE_DERR_ID_REPEAT : 0);
 }
 
 template <int K, int ROWS>
 __global__ void __launch_bounds__(kMmaThreads, 1)
-coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restrict__ part, int32_t *err)
+coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *cnt_c, uint32_t *cnt_m, int32_t *err)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     // full[s]: the builders wrote stage s; empty[s]: the MMAs that read it are
@@ -254,24 +229,26 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages, n = c / kStages;
             fetch(c + 2, n2_v);
-            uint32_t m[ROWS / 32];
-            int bad = 0;
             const int t = t0 + c * kTok + u;
+            int bad = 0;
             if (t < t1) {
-                token_mask<K, ROWS>(cur_v, E, m, bad);
+                bad = token_check<K>(cur_v, E);
                 if (bad) record_error(err, bad);
-            } else {
-#pragma unroll
-                for (int x = 0; x < ROWS / 32; ++x) m[x] = 0u;
             }
+            const bool set = t < t1 && !bad;
             if (c >= kStages && !mbar_wait(&empty_bar[s], (n - 1) & 1)) { ok = false; break; }
             uint8_t *row = sm + s * per_stage + my_tile + u * 128;
+            // clear the row's chunks, then set the token's bytes (same thread:
+            // the stores land in program order)
 #pragma unroll
-            for (int ch = 0; ch < ROWS / 16; ++ch) {
-                if (ch >= c_lo && ch < c_hi) {
-                    const uint32_t h = m[ch >> 1] >> ((ch & 1) * 16);
-                    const uint4 o = make_uint4(nib_bytes(h), nib_bytes(h >> 4), nib_bytes(h >> 8), nib_bytes(h >> 12));
-                    *reinterpret_cast<uint4 *>(row + (ch >> 3) * kAtom + (((ch ^ u) & 7) << 4)) = o;
+            for (int ch = 0; ch < ROWS / 16; ++ch)
+                if (ch >= c_lo && ch < c_hi)
+                    *reinterpret_cast<uint4 *>(row + (ch >> 3) * kAtom + (((ch ^ u) & 7) << 4)) = make_uint4(0, 0, 0, 0);
+            if (set) {
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    const int e = cur_v[j], ch = e >> 4;
+                    if (ch >= c_lo && ch < c_hi) row[(ch >> 3) * kAtom + (((ch ^ u) & 7) << 4) + (e & 15)] = 1;
                 }
             }
             // the stores become visible to the tensor cores; one arrival per warp
@@ -321,46 +298,58 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
     }
     if (!ok) record_error(err, MOE_DERR_TIMEOUT);
 
-    // epilogue: warp w (< 4) reads TMEM lanes 32w..32w+31 = rows of each M tile
+    // epilogue: warp w (< 4) reads TMEM lanes 32w..32w+31 = rows of each M
+    // tile.  The block's counts are added into the job's count matrices in
+    // global memory by bulk asynchronous reductions: a thread stages its row
+    // in shared memory (rows 16 bytes longer than E words, so that the 16-byte
+    // stores of a warp fall in distinct banks) and adds it with one
+    // cp.reduce.async.bulk (element-wise adds performed in L2, atomic with
+    // respect to the other blocks' adds).
     if (warp < 4) {
         bool ready = ok;
         if (nchunks > 0) ready = mbar_wait(&done_bar, 0) && ready;
         ready = __all_sync(0xffffffffu, ready);
         if (!ready && lane == 0) record_error(err, MOE_DERR_TIMEOUT);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        for (int q = 0; ready && q < 2; ++q) {
+        const int pitch = E + 4;                          // staged row, in words
+        uint32_t *srow = reinterpret_cast<uint32_t *>(sm) + (size_t)(warp * 32 + lane) * pitch;
+        for (int q = 0; ready && nchunks > 0 && q < 2; ++q) {
             if (q == 0 ? !has_c : !has_m) continue;
-            const int prod = q == 0 ? la : G.nc + la;
             const uint32_t col0 = q == 0 ? 0u : m_off;
-            uint32_t *dst = part + ((size_t)prod * G.S + slice) * E * E;
+            uint32_t *dst = (q == 0 ? cnt_c : cnt_m) + (size_t)la * E * E;
             for (int mi = 0; mi < kMt; ++mi) {
                 const int row = mi * 128 + warp * 32 + lane;
                 for (int c0 = 0; c0 < E; c0 += 16) {
                     uint32_t r[16];
-                    if (nchunks > 0) {
-                        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + col0 + (uint32_t)(mi * ROWS + c0);
-                        asm volatile(
-                            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-                            "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-                            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                              "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-                              "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-                            : "r"(ta));
-                        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                    } else {
-#pragma unroll
-                        for (int x = 0; x < 16; ++x) r[x] = 0;
-                    }
+                    const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + col0 + (uint32_t)(mi * ROWS + c0);
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                          "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                          "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                        : "r"(ta));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                     if (row < E) {
-                        uint4 *o = reinterpret_cast<uint4 *>(dst + (size_t)row * E + c0);
+                        uint4 *o = reinterpret_cast<uint4 *>(srow + c0);
                         o[0] = make_uint4(r[0], r[1], r[2], r[3]);
                         o[1] = make_uint4(r[4], r[5], r[6], r[7]);
                         o[2] = make_uint4(r[8], r[9], r[10], r[11]);
                         o[3] = make_uint4(r[12], r[13], r[14], r[15]);
                     }
                 }
+                if (row < E) {
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.u32 [%0], [%1], %2;"
+                                 ::"l"(dst + (size_t)row * E), "r"(smem_addr(srow)), "r"((uint32_t)(E * 4))
+                                 : "memory");
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    // the staged row is rewritten next: wait until the add has read it
+                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                }
             }
         }
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -369,39 +358,26 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *__restric
                      : "memory");
 }
 
-// Sum of n partial words at base, base + stride, ... (8 loads in flight).
-__device__ __forceinline__ uint32_t mma_sum(const uint32_t *__restrict__ part, size_t base, size_t stride, int n)
-{
-    uint32_t s = 0;
-    int q = 0;
-    for (; q + 8 <= n; q += 8) {
-        uint32_t v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = __ldg(part + base + (size_t)(q + i) * stride);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) s += v[i];
-    }
-    for (; q < n; ++q) s += __ldg(part + base + (size_t)q * stride);
-    return s;
-}
-
 // blockIdx.y = product: C of layer y (y < nc), M of layer y - nc otherwise.
+// The counts were summed over the blocks by the bulk reductions; this copies
+// them out and evaluates Ochiai in fp64 (IEEE multiply, square root and
+// divide, one rounding to fp32), exactly as the histogram path does.
 __global__ void __launch_bounds__(kMmaReduceThreads)
-coact_mma_reduce_kernel(MmaGeom G, const uint32_t *__restrict__ part, uint32_t *coact, float *ochiai, uint32_t *trans)
+coact_mma_finish_kernel(MmaGeom G, const uint32_t *__restrict__ cnt, uint32_t *coact, float *ochiai, uint32_t *trans)
 {
     extern __shared__ uint32_t mdiag[];
     const int E = G.E, p = blockIdx.y;
     const size_t EE = (size_t)E * E;
     const size_t c = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const size_t pbase = (size_t)p * G.S * EE;
+    const uint32_t *m = cnt + (size_t)p * EE;
     if (p < G.nc) {
         if (ochiai) {
-            for (int e = threadIdx.x; e < E; e += blockDim.x) mdiag[e] = mma_sum(part, pbase + (size_t)e * E + e, EE, G.S);
+            for (int e = threadIdx.x; e < E; e += blockDim.x) mdiag[e] = __ldg(m + (size_t)e * E + e);
             __syncthreads();
         }
         if (c < EE) {
             const int i = (int)(c / E), j = (int)(c % E);
-            const uint32_t v = mma_sum(part, pbase + c, EE, G.S);
+            const uint32_t v = __ldg(m + c);
             if (coact) coact[(size_t)p * EE + c] = v;
             if (ochiai) {
                 const double den = __dmul_rn((double)mdiag[i], (double)mdiag[j]);
@@ -410,7 +386,7 @@ coact_mma_reduce_kernel(MmaGeom G, const uint32_t *__restrict__ part, uint32_t *
             }
         }
     } else if (c < EE && trans) {
-        trans[(size_t)(p - G.nc) * EE + c] = mma_sum(part, pbase + c, EE, G.S);
+        trans[(size_t)(p - G.nc) * EE + c] = __ldg(m + c);
     }
 }
 
@@ -419,7 +395,8 @@ moe_status launch_mma(const int32_t *ids, const MmaGeom &g, uint32_t *part, int3
 {
     const size_t smem = mma_smem_bytes(g);
     if (allow_smem(coact_mma_kernel<K, ROWS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
-    coact_mma_kernel<K, ROWS><<<g.J * g.S, kMmaThreads, smem, s>>>(ids, g, part, err);
+    coact_mma_kernel<K, ROWS><<<g.J * g.S, kMmaThreads, smem, s>>>(ids, g, part, part + (size_t)g.nc * g.E * g.E,
+                                                                   err);
     return launch_status();
 }
 
@@ -466,17 +443,21 @@ bool make_mma_geom(int L, int T, int k, int E, bool want_c, bool want_t, MmaGeom
 size_t mma_smem_bytes(const MmaGeom &g)
 {
     const bool any_m = g.P > g.nc;
-    return (size_t)kStages * (any_m ? 2 : 1) * g.rows * kTok;
+    const size_t stages = (size_t)kStages * (any_m ? 2 : 1) * g.rows * kTok;
+    const size_t staged_rows = (size_t)128 * (g.E + 4) * sizeof(uint32_t);   // the epilogue's rows
+    return std::max(stages, staged_rows);
 }
 
 size_t mma_partial_words(const MmaGeom &g)
 {
-    return (size_t)g.P * g.S * g.E * g.E;
+    return (size_t)g.P * g.E * g.E;          // every product's counts, summed in place
 }
 
 moe_status coact_mma(const int32_t *ids, const MmaGeom &g, uint32_t *part, uint32_t *coact, float *ochiai,
                      uint32_t *trans, int32_t *err, cudaStream_t stream)
 {
+    // the count matrices start at zero: every block adds its tokens' counts
+    if (cudaMemsetAsync(part, 0, mma_partial_words(g) * sizeof(uint32_t), stream) != cudaSuccess) return MOE_ERR_CUDA;
     moe_status st = MOE_ERR_ARG;
     switch (g.k) {
     case 1: st = launch_mma_rows<1>(ids, g, part, err, stream); break;
@@ -492,7 +473,7 @@ moe_status coact_mma(const int32_t *ids, const MmaGeom &g, uint32_t *part, uint3
     note_launches(1);
     const size_t EE = (size_t)g.E * g.E;
     dim3 grid((unsigned)((EE + kMmaReduceThreads - 1) / kMmaReduceThreads), (unsigned)g.P);
-    coact_mma_reduce_kernel<<<grid, kMmaReduceThreads, sizeof(uint32_t) * g.E, stream>>>(g, part, coact, ochiai,
+    coact_mma_finish_kernel<<<grid, kMmaReduceThreads, sizeof(uint32_t) * g.E, stream>>>(g, part, coact, ochiai,
                                                                                           trans);
     st = launch_status();
     if (st == MOE_OK) note_launches(1);

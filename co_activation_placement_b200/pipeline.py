@@ -153,16 +153,6 @@ class HotPath:
                                                      err=self.err, ws=self.stats_ws))
 
     def _plan(self, l):
-        # a plan with nothing beside it (every plan in line; with the overlap,
-        # the first layer's, which opens the step) runs as one cooperative
-        # launch; beside the row traffic, as separate kernels
-        prev = cap.plan_dispatch_method(1 if (not self.overlap or l == 0) else 0)
-        try:
-            self._plan_calls(l)
-        finally:
-            cap.plan_dispatch_method(prev)
-
-    def _plan_calls(self, l):
         src = self.targets[l - 1] if (self.shuffle and l > 0) else None
         if self.replicas:
             # each task to a replica of its expert: fewest remote nodes per token

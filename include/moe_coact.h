@@ -105,13 +105,14 @@ uint64_t moe_launch_count(void);
  * ---------------------------------------------------------------------- */
 size_t moe_coact_stats_workspace(int L, int T, int k, int E, int with_trans);
 /* How moe_coact_stats counts (process-wide; returns the previous setting, or
- * -1 for an invalid argument): 0 = default = 1 (measured on B200 as fast as or
- * faster than 2 for E <= 256, k = 8); 1 = shared-memory histograms (per-token
- * counter increments); 2 = tensor cores where the shape allows (E % 16 == 0,
- * 32 <= E <= 256, ids 16-byte aligned): C_l = X_l X_l^T and M_l = X_l
- * X_{l+1}^T for the one-hot X_l[e][t], tcgen05.mma kind::i8 with exact int32
- * accumulation.  Both give identical results.  The setting affects calls
- * issued after it returns. */
+ * -1 for an invalid argument): 0 = default: 2 for E >= 128 where the shape
+ * allows, else 1 (measured on B200 with k = 8: the tensor cores are faster at
+ * E = 128 and 256, the histograms at E = 64); 1 = shared-memory histograms
+ * (per-token counter increments); 2 = tensor cores where the shape allows
+ * (E % 16 == 0, 32 <= E <= 256, ids 16-byte aligned): C_l = X_l X_l^T and
+ * M_l = X_l X_{l+1}^T for the one-hot X_l[e][t], tcgen05.mma kind::i8 with
+ * exact int32 accumulation.  Both give identical results.  The setting affects
+ * calls issued after it returns. */
 int moe_coact_stats_method(int method);
 /* Which method a moe_coact_stats call with these sizes (and C wanted) would use
  * under the current setting: 1 = histograms, 2 = tensor cores; 0 for sizes
