@@ -806,12 +806,14 @@ def run_ep(a, w, rank, world, device, seed):
 NVLINK_GBS = 770.0   # measured peer copy per direction per GPU on this machine (the profiling recipe's figure)
 
 
-def exchange_record(cap, counts_layers, G, W, rowB, ms_step):
+def exchange_record(cap, counts_layers, G, W, rowB, ms_step, crossed=True):
     """Rows and bytes that cross devices in the exchange with the G ranks on W
     devices (moe_ep_exchange_rows on each layer's gathered counts), and the
     NVLink floor they set: per layer the busiest device sends or receives
     max(sent_h, received_h) rows in the dispatch and again in the combine, at
-    NVLINK_GBS per direction."""
+    NVLINK_GBS per direction.  crossed: the rows did cross NVLink in the timed
+    steps (several GPUs); else (virtual devices on one GPU) only the floor is
+    reported, beside the measured step."""
     rows, busiest = [], []
     for c in counts_layers:
         sent, recv = cap.ep_exchange_rows(c, G, W)
@@ -819,13 +821,16 @@ def exchange_record(cap, counts_layers, G, W, rowB, ms_step):
         busiest.append(int(max(sent.max(), recv.max())))
     floor_ms = sum(2.0 * b * rowB / (NVLINK_GBS * 1e9) * 1e3 for b in busiest)
     busiest_bytes = sum(2 * b * rowB for b in busiest)
+    nv = {"bound": "nvlink", "peak": NVLINK_GBS, "unit": "GB/s",
+          "peak_kind": "measured peer copy per direction (pool figure)",
+          "busiest_device_bytes_per_step": busiest_bytes, "floor_ms_per_step": floor_ms}
+    if crossed and ms_step > 0 and W > 1:
+        nv["achieved"] = busiest_bytes / (ms_step * 1e-3) / 1e9
+        nv["frac"] = nv["achieved"] / NVLINK_GBS
+    else:
+        nv["floor_over_measured_step"] = floor_ms / ms_step if ms_step > 0 else None
     return {"devices": W, "rows_crossing_per_layer": rows, "bytes_each_way_per_step": sum(rows) * rowB,
-            "busiest_device_rows_per_layer": busiest,
-            "nvlink": {"bound": "nvlink", "peak": NVLINK_GBS, "unit": "GB/s",
-                       "peak_kind": "measured peer copy per direction (pool figure)",
-                       "busiest_device_bytes_per_step": busiest_bytes, "floor_ms_per_step": floor_ms,
-                       "achieved": busiest_bytes / (ms_step * 1e-3) / 1e9 if ms_step > 0 else None,
-                       "frac": floor_ms / ms_step if ms_step > 0 else None}}
+            "busiest_device_rows_per_layer": busiest, "nvlink": nv}
 
 
 def run_ep_emulated(hp, w, W, steps, warmup, hbm, sb, pg):
@@ -877,9 +882,10 @@ def run_ep_emulated(hp, w, W, steps, warmup, hbm, sb, pg):
         counts.append(emu.shards[0].counts_all.cpu().numpy())
     nbytes = sb.permute + sb.combine
     return {"devices": W, "ranks_per_device": Gl, "tokens_per_device": w.T // W, "recv_rows_max": rows,
-            "exchange": exchange_record(cap, counts, w.G, W, w.d * hp.x.element_size(), ms),
+            "exchange": exchange_record(cap, counts, w.G, W, w.d * hp.x.element_size(), ms, crossed=False),
             "exchange_note": "the rows that would cross NVLink with the W devices on W GPUs; here they move "
-                             "within one GPU's memory, so the nvlink frac is the floor over the measured step",
+                             "within one GPU's memory: floor_over_measured_step > 1 means W GPUs would be "
+                             "NVLink-bound at the measured peer bandwidth",
             "ms_per_step": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
             "errors": emu.errors(),
             "note": "W virtual devices on this GPU, each with its own receive buffer and stream (a phase of the W devices runs side by side, each meeting joins the streams); "

@@ -90,7 +90,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 }
 
 // true once the mbarrier phase with the given parity has completed; false
-// when that took longer than kWaitLimitNs
+// when that took longer than kWaitLimitNs.  Each try_wait may suspend the
+// thread in hardware until the phase completes, for at most kSuspendHintNs,
+// so a waiting warp takes no issue slots from the warps doing the work.
+constexpr uint32_t kSuspendHintNs = 1000000;   // 1 ms
+
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
     const uint32_t a = smem_addr(bar);
@@ -99,10 +103,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(done)
-            : "r"(a), "r"(parity)
+            : "r"(a), "r"(parity), "r"(kSuspendHintNs)
             : "memory");
         if (done) return true;
         if (gtimer_ns() - t0 > kWaitLimitNs) return false;
