@@ -82,7 +82,12 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of one CUDA graph")
     ap.add_argument("--no-overlap", action="store_true",
-                    help="run plans, shuffle targets and statistics in line instead of on a second stream")
+                    help="run plans, shuffle targets and statistics in line instead of on a second stream "
+                         "(the same as --schedule inline)")
+    ap.add_argument("--schedule", default=None, choices=["overlap", "forward", "inline"],
+                    help="overlap (default): all control work ahead on a second stream; forward: the order of a "
+                         "forward pass, each layer's plan in line before its rows, shuffle targets and statistics "
+                         "beside them; inline: everything in line")
     ap.add_argument("--replicas", type=int, default=0, metavar="EXTRA",
                     help="replicate experts (EXTRA more per rank) and assign tasks to the fewest remote nodes")
     ap.add_argument("--replica-eps", type=float, default=None, metavar="EPS",
@@ -378,7 +383,8 @@ def main():
                           shuffle=shuffle, out_dtype=out_dtype, device=device, timers=True,
                           scales=make_expert_scales(w, seed=seed) if a.prereduce else None,
                           replica_extra=a.replicas, shuffle_capacity=w.T // w.G if balanced else 0,
-                          overlap=not a.no_overlap, replica_eps=a.replica_eps)
+                          overlap=not a.no_overlap, replica_eps=a.replica_eps,
+                          schedule="inline" if a.no_overlap else a.schedule)
     place = time_placement(cap, ids_cal, w, a.placement, device)
 
     def barrier():
@@ -498,7 +504,7 @@ def main():
     # with the overlap the control calls' event times include waiting for SM
     # slots beside the row traffic: the dominant kernel is taken among the
     # calls on the main stream, whose chain is the step
-    side_calls = ("stats", "plan", "shuffle") if hp.overlap else ()
+    side_calls = hp.side_calls
     dom = max((n for n in kern if n not in side_calls), key=lambda n: kern[n]["ms_per_step"])
     nl = launches_of[dom]
     per_launch_ms = kern[dom]["ms_per_step"] / nl
@@ -512,7 +518,7 @@ def main():
     stats_ms = kern["stats"]["ms_per_step"]
     # in line only: with the overlap the statistics share the SMs with the
     # row kernels and their event time is not their own (the sweep times them alone)
-    coact_tps = None if hp.overlap else world * w.L * w.T / (stats_ms * 1e-3)
+    coact_tps = None if "stats" in hp.side_calls else world * w.L * w.T / (stats_ms * 1e-3)
     sweep = None
     if not a.no_sweep:
         sweep = run_sweep(cap, pipeline, device, seed, a.steps, a.warmup, hbm, pg)
@@ -542,7 +548,12 @@ def main():
                                   else "source-side weighted (identity experts)",
                        "replicas_per_rank": a.replicas,
                        "replica_eps": a.replica_eps if a.replicas else None,
-                       "overlap": "plans, shuffle targets and statistics on a second stream"
+                       "schedule": hp.schedule,
+                       "overlap": (", ".join({"stats": "statistics", "plan": "plans", "shuffle": "shuffle targets"}[c]
+                                             for c in hp.side_calls) + " on a second stream" +
+                                   ("; its cooperative launches with one block per rank"
+                                    if (balanced and "shuffle" in hp.side_calls) or
+                                    (a.replicas and a.replica_eps is not None and "plan" in hp.side_calls) else ""))
                                   if hp.overlap else "none",
                        "shuffle": ("balanced (T/G tokens per rank)" if balanced else True) if shuffle else False,
                        "parallelism": "replicas (weak scaling, one batch per GPU)",
@@ -660,12 +671,30 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
 
 def replica_load(hp, w):
     """Per-rank task loads the capped replica assignment returned (one row
-    per layer): busiest rank over the mean, next to V in "rows"."""
+    per layer): busiest rank over the mean, next to V in "rows"; beside them
+    the same assignment without a cap (eps = inf) on the same inputs, and
+    the ranks whose tasks reach the cap."""
     if not hp.replicas or hp.replica_eps is None:
         return None
+    import torch
+    import co_activation_placement_b200 as cap
     ld = hp.rank_load.cpu().double()
-    return {"eps": hp.replica_eps, "max_over_mean": [float(r.max() / r.mean()) for r in ld],
-            "max": [int(r.max()) for r in ld], "mean": [float(r.mean()) for r in ld]}
+    free = torch.zeros_like(hp.rank_load)
+    pick = torch.empty_like(hp.pick_rank)
+    for l in range(hp.L):
+        src = hp.targets[l - 1] if (hp.shuffle and l > 0) else None
+        rr, nr = hp.replicas[l]
+        cap.assign_replicas_capped(hp.ids[l], hp.E, hp.G, hp.rpn, rr, nr, float("inf"), src_rank=src,
+                                   pick_rank=pick, rank_load=free[l], err=hp.err, ws=hp.capped_ws)
+    torch.cuda.synchronize()
+    fr = free.cpu().double()
+    limit = int(((1.0 + hp.replica_eps) * hp.T * hp.k) // hp.G)
+    return {"eps": hp.replica_eps, "cap": limit,
+            "max_over_mean": [float(r.max() / r.mean()) for r in ld],
+            "max": [int(r.max()) for r in ld], "mean": [float(r.mean()) for r in ld],
+            "ranks_at_cap": [int((r >= limit).sum()) for r in ld],
+            "uncapped_max_over_mean": [float(r.max() / r.mean()) for r in fr],
+            "uncapped_ranks_over_cap": [int((r > limit).sum()) for r in fr]}
 
 
 def time_placement(cap, ids_cal, w, placement, device):

@@ -13,7 +13,7 @@ Entry points (names follow the C ABI without the ``moe_`` prefix):
   place_replicas, assign_replicas, assign_replicas_capped, plan_dispatch_ranks,
   ep_routes, ep_permute, ep_combine, ep_scatter_rows, ep_exchange_rows (ranks over several devices),
   place_uniform, place_capacity, place_correlated, place_correlated_capped, rank_loads,
-  selftest_wait_timeout, launch_count.
+  cooperative_blocks, selftest_wait_timeout, launch_count.
 """
 from __future__ import annotations
 
@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "moe_coact_stats": ([P, i, i, i, i, P, P, P, P, P, sz, P], i),
             "moe_plan_dispatch_workspace": ([i, i, i, i], sz),
             "moe_plan_dispatch_method": ([i], i),
+            "moe_cooperative_blocks": ([i], i),
             "moe_plan_dispatch": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
             "moe_permute": ([P, i, i, i, i, P, i64, P, P, P], i),
             "moe_combine": ([P, i, i64, i, P, P, i, i, P, i, P, P], i),
@@ -278,6 +279,16 @@ def plan_dispatch_method(method: int) -> int:
     prev = int(lib().moe_plan_dispatch_method(int(method)))
     if prev < 0:
         raise ValueError("method must be 0 or 1")
+    return prev
+
+
+def cooperative_blocks(blocks: int) -> int:
+    """Blocks of the cooperative launches (shuffle_balanced,
+    assign_replicas_capped): 0 = one per SM (default), n > 0 = n blocks;
+    returns the previous setting (process-wide)."""
+    prev = int(lib().moe_cooperative_blocks(int(blocks)))
+    if prev < 0:
+        raise ValueError("blocks must be >= 0")
     return prev
 
 

@@ -1,4 +1,5 @@
-// Library-wide entry points: status strings and launch accounting.
+// Library-wide entry points: status strings, launch accounting and the
+// cooperative kernels' grid size.
 #include <atomic>
 
 #include "common.cuh"
@@ -6,6 +7,7 @@
 namespace moe {
 
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<int> g_coop_blocks{0};
 
 void note_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
@@ -23,7 +25,19 @@ int sm_count()
     return cached[dev];
 }
 
+int coop_grid()
+{
+    const int n = g_coop_blocks.load(std::memory_order_relaxed), sms = sm_count();
+    return n > 0 && n < sms ? n : sms;
+}
+
 }  // namespace moe
+
+extern "C" int moe_cooperative_blocks(int blocks)
+{
+    if (blocks < 0) return -1;
+    return moe::g_coop_blocks.exchange(blocks);
+}
 
 extern "C" const char *moe_status_string(moe_status s)
 {

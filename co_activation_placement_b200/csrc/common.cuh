@@ -44,6 +44,10 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Number of SMs of the current device (cached per device ordinal).
 int sm_count();
 
+// Blocks of a cooperative launch (moe_cooperative_blocks): one per SM unless
+// a smaller count is set.
+int coop_grid();
+
 // Programmatic dependent launch.  A kernel launched with launch_pdl may start
 // while the previous kernel on its stream is still running: it does the part
 // of its work that reads only the call's own inputs, then pdl_wait() -- which

@@ -7,11 +7,11 @@
 //
 // Exact per token: with at most 8 nodes, the smallest set S of remote nodes
 // covering the token's experts (those without a replica on the source node) is
-// found by enumerating the submasks of the candidate nodes (ties: smallest S
-// as a bit pattern).  Then, pick by pick in j order, among the ranks hosting
-// the expert on the source node (or, if none, on the nodes of S): rank s if
-// it is one of them, else the lowest one an earlier pick already uses (no new
-// row), else the lowest one.
+// found by trying the sets of candidate nodes by size, each size in
+// increasing order (ties: smallest S as a bit pattern).  Then, pick by pick in
+// j order, among the ranks hosting the expert on the source node (or, if
+// none, on the nodes of S): rank s if it is one of them, else the lowest one
+// an earlier pick already uses (no new row), else the lowest one.
 // One thread per token; the replica table sits in shared memory.
 //
 // Under a load tolerance ("Cobalt", "Problem Formulation": the tasks of rank
@@ -21,13 +21,14 @@
 // its experts' open replicas (all of them when none is open).  Token t's
 // choice depends on every earlier token only through the set of closed
 // ranks, which changes at most G times, so one cooperative launch computes
-// it in rounds: every remaining token's choice under the current closed set,
-// in parallel; per-block task counts per rank and their running sum over
-// blocks locate the first token tau at which an open rank reaches the cap
-// (a block-wide scan inside the block where that happens); the choices of
-// tokens before tau are final, their tasks join the loads, the ranks at the
-// cap close, and the next round starts at tau.  At most G + 1 rounds, each
-// ending in a grid barrier with a bounded wait.
+// it in rounds: the remaining tokens' choices under the current closed set,
+// in parallel, one warp per token (after the first round only the tokens
+// with an expert whose usable replicas changed); per-block task counts per rank and their
+// running sum over blocks locate the first token tau at which an open rank
+// reaches the cap (a block-wide scan inside the block where that happens);
+// the choices of tokens before tau are final, their tasks join the loads,
+// the ranks at the cap close, and the next round starts at tau.  At most
+// G + 1 rounds of two grid barriers with bounded waits.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -41,6 +42,72 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxNodes = 8;
 
+// The fewest remote nodes covering the needed picks: the smallest set S of
+// the candidate nodes `cand` such that every pick j in `need` has a node of
+// nm[j] in S; among sets of that size the smallest as a bit pattern.  A pick
+// with one candidate node forces that node into every cover (F); the picks F
+// leaves uncovered are covered by the fewest of their own candidate nodes,
+// tried by size and within a size in increasing order (Gosper's successor on
+// the candidates' positions, deposited back onto them), so the first cover
+// found is the answer and S = F | that cover (F's bits are common to every
+// minimum S, so the order of the covers is that of the S).  With one or two
+// replicas per expert nearly every pick is forced and little is left to try.
+// Returns |S| (best = S), or -1 when a needed pick has no candidate node.
+template <int K>
+__device__ __forceinline__ int fewest_nodes(uint32_t need, const uint32_t (&nm)[K], uint32_t cand, uint32_t &best)
+{
+    best = 0;
+    if (need == 0) return 0;
+    uint32_t forced = 0;
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+        if ((need >> j) & 1u) {
+            const uint32_t c = nm[j] & cand;
+            if (c == 0) return -1;
+            if ((c & (c - 1u)) == 0) forced |= c;
+        }
+    uint32_t rest = 0, rc = 0, all = ~0u;
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+        if (((need >> j) & 1u) && (nm[j] & forced) == 0) {
+            rest |= 1u << j;
+            rc |= nm[j] & cand;
+            all &= nm[j];
+        }
+    const int nf = __popc(forced);
+    if (rest == 0) {
+        best = forced;
+        return nf;
+    }
+    all &= rc;
+    if (all) {                                   // one node covers the rest: the lowest such
+        best = forced | (all & (0u - all));
+        return nf + 1;
+    }
+    const int m = __popc(rc);
+    for (int p = 2; p <= m; ++p) {
+        for (uint32_t x = (1u << p) - 1; x < (1u << m);) {
+            uint32_t sub = 0, c = rc;
+            for (uint32_t y = x; y; y >>= 1) {
+                const uint32_t low = c & (0u - c);
+                if (y & 1u) sub |= low;
+                c ^= low;
+            }
+            bool ok = true;
+#pragma unroll
+            for (int j = 0; j < K; ++j)
+                if ((rest >> j) & 1u) ok &= (nm[j] & sub) != 0;
+            if (ok) {
+                best = forced | sub;
+                return nf + p;
+            }
+            const uint32_t lo = x & (0u - x), r = x + lo;
+            x = (((r ^ x) >> 2) >> (__ffs(lo) - 1)) | r;
+        }
+    }
+    return -1;
+}
+
 template <int K>
 __global__ void __launch_bounds__(kThreads)
 assign_replicas_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
@@ -49,8 +116,10 @@ assign_replicas_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int
                        int32_t *__restrict__ n_remote, int32_t *err)
 {
     extern __shared__ int32_t sm[];
+    __shared__ int node_of[64];                 // rank -> node
     const int nodes = G / rpn, max_rep = 1 + nodes;
     int32_t *rep = sm;                          // [E][max_rep]
+    for (int r = threadIdx.x; r < G; r += blockDim.x) node_of[r] = r / rpn;
     uint32_t *nmask = reinterpret_cast<uint32_t *>(sm + E * max_rep);   // [E] nodes hosting e
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         uint32_t m = 0;
@@ -93,22 +162,11 @@ assign_replicas_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int
             }
         }
         cand &= ~(1u << ns);
-        int best_pop = 99;
         uint32_t best = 0;
+        int best_pop = 0;
         if (!bad) {
-            for (uint32_t sub = cand;; sub = (sub - 1) & cand) {
-                bool ok = true;
-#pragma unroll
-                for (int j = 0; j < K; ++j)
-                    if ((need >> j) & 1u) ok &= (nm[j] & sub) != 0;
-                const int pop = __popc(sub);
-                if (ok && (pop < best_pop || (pop == best_pop && sub < best))) {
-                    best_pop = pop;
-                    best = sub;
-                }
-                if (sub == 0) break;
-            }
-            if (best_pop == 99) bad = true;    // an expert with no replica at all
+            best_pop = fewest_nodes<K>(need, nm, cand, best);
+            if (best_pop < 0) bad = true;      // an expert with no replica at all
         }
         if (bad) {
             record_error(err, MOE_DERR_ID_RANGE);
@@ -126,7 +184,8 @@ assign_replicas_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int
             for (int q = 0; q < max_rep; ++q) {
                 const int r = rl[q];
                 if (r < 0) continue;
-                const bool allowed = any_ns ? (r / rpn == ns) : ((best >> (r / rpn)) & 1u);
+                const int nr = node_of[r];
+                const bool allowed = any_ns ? (nr == ns) : ((best >> nr) & 1u);
                 if (!allowed) continue;
                 if (r == s) pick = r;
                 if (((used >> r) & 1ull) && (used_pick < 0 || r < used_pick)) used_pick = r;
@@ -142,14 +201,13 @@ assign_replicas_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int
 
 // ---- load-capped assignment ---------------------------------------------
 
-constexpr int kCapThreads = 512;
+constexpr int kCapThreads = 1024;
 constexpr int kCapMaxBlocks = 1024;
 
 struct CapHeader {
     GridBarrier bar;
-    int tau[2];           // first token seeing a newly closed rank (by round parity)
+    int tau[3];           // first token seeing a newly closed rank (round % 3)
     int rounds;           // rounds run
-    int pad;
 };
 
 struct CapArgs {
@@ -160,75 +218,147 @@ struct CapArgs {
     int32_t *pick, *nrem;
     long long *rank_load;     // [G] out or null
     CapHeader *h;
-    unsigned long long *load; // [G] tasks committed per rank
-    int *blk;                 // [gridDim.x][G] tasks per rank of each block's tokens this round
+    int *blk;                 // [2][gridDim.x][G] tasks per rank of each block's tokens (round parity)
     int32_t *err;
 };
 
-// Token t's choice over the usable replicas (uok[e]: usable ranks of e,
-// unm[e]: their nodes): the fewest remote nodes, then the pick rule.
-// Returns |S| or -1 for an invalid token (ids, source, an expert without
-// replicas); the picks are written to pk.
-template <int K>
-__device__ __forceinline__ int choose_capped(const int (&v)[K], int s, int E, int G, int rpn, int max_rep,
-                                             const int32_t *rep, const uint32_t *unm,
-                                             const unsigned long long *uok, int (&pk)[K])
+// x's bits deposited, lowest first, onto the set bits of mask (<= 8 of them).
+__device__ __forceinline__ uint32_t deposit8(uint32_t x, uint32_t mask)
 {
-    bool bad = (unsigned)s >= (unsigned)G;
+    uint32_t r = 0;
 #pragma unroll
-    for (int a = 0; a < K; ++a) {
-        bad |= (unsigned)v[a] >= (unsigned)E;
-#pragma unroll
-        for (int b = 0; b < a; ++b) bad |= v[a] == v[b];
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t low = mask & (0u - mask);
+        if (x & 1u) r |= low;
+        mask ^= low;
+        x >>= 1;
     }
-    if (bad) return -1;
-    const int ns = s / rpn;
-    uint32_t need = 0, cand = 0, nm[K];
+    return r;
+}
+
+// A listed token's inputs, loaded by its warp ahead of its turn: lane j < K
+// its pick j's expert and, after the first round, the rank it had.
+struct TokenIn {
+    int t, v, s, old;
+};
+
+template <int K>
+__device__ __forceinline__ TokenIn load_token(int t, const CapArgs &a, int rd)
+{
+    const int lane = threadIdx.x & 31;
+    TokenIn x{t, -1, 0, -1};
+    if (t < 0) return x;
+    if (lane < K) x.v = __ldg(a.ids + (size_t)t * K + lane);
+    x.s = a.src ? __ldg(a.src + t) : t / (a.T / a.G);
+    if (rd > 0 && lane < K) x.old = __ldcg(a.pick + (size_t)t * K + lane);
+    return x;
+}
+
+// Token x.t assigned by one warp over the usable replicas (uok[e]: usable
+// ranks of e, unm[e]: their nodes), the same rule as the uncapped kernel:
+// lane j < K holds pick j.  The fewest remote nodes come from warp
+// reductions: the forced nodes, then one node covering the rest, else every
+// set of the remaining candidate nodes at once (lanes over sets, the minimum
+// of (size, set)).  Then every lane finds its pick's candidate ranks; a pick
+// with one candidate, or with rank s among them, is settled at once, and the
+// others take, in j order, the lowest candidate an earlier pick uses, else
+// the lowest.  Every step is warp-uniform.  Writes pick_rank[t][*] and
+// n_remote[t] (-1 for an invalid token) and moves the token's tasks in
+// `hist` from its previous choice (rd > 0) to the new one.
+template <int K>
+__device__ __forceinline__ void assign_token_warp(const TokenIn &x, const CapArgs &a, int rd, int max_rep,
+                                                  const int32_t *rep, const int *node_of, const uint32_t *unm,
+                                                  const unsigned long long *uok, int *hist)
+{
+    const int lane = threadIdx.x & 31;
+    constexpr unsigned kAll = 0xffffffffu, kPicks = (1u << K) - 1u;
+    const int t = x.t, v = x.v, s = x.s;
+    const unsigned same = __match_any_sync(kAll, v);
+    bool bad = __any_sync(kAll, lane < K && ((unsigned)v >= (unsigned)a.E || __popc(same & kPicks) > 1)) ||
+               (unsigned)s >= (unsigned)a.G;
+    int pick = -1, pop = -1;
+    if (!bad) {
+        const int ns = node_of[s];
+        const uint32_t nm = lane < K ? unm[v] : 0u;
+        const bool need = lane < K && !((nm >> ns) & 1u);
+        const uint32_t cand = __reduce_or_sync(kAll, need ? nm : 0u) & ~(1u << ns);
+        const uint32_t c = nm & cand;
+        uint32_t best = 0;
+        pop = 0;
+        if (__any_sync(kAll, need)) {
+            if (__any_sync(kAll, need && c == 0)) {
+                pop = -1;                        // an expert without replicas
+            } else {
+                const uint32_t forced = __reduce_or_sync(kAll, (need && (c & (c - 1u)) == 0) ? c : 0u);
+                const bool rest = need && (nm & forced) == 0;
+                best = forced;
+                pop = __popc(forced);
+                if (__any_sync(kAll, rest)) {
+                    const uint32_t rc = __reduce_or_sync(kAll, rest ? c : 0u);
+                    const uint32_t one = __reduce_and_sync(kAll, rest ? nm : ~0u) & rc;
+                    if (one) {
+                        best |= one & (0u - one);
+                        pop += 1;
+                    } else {
+                        uint32_t nmv[K];
+                        const unsigned restm = __ballot_sync(kAll, rest);
 #pragma unroll
-    for (int j = 0; j < K; ++j) {
-        nm[j] = unm[v[j]];
-        if (!((nm[j] >> ns) & 1u)) {
-            need |= 1u << j;
-            cand |= nm[j];
+                        for (int j = 0; j < K; ++j) nmv[j] = __shfl_sync(kAll, nm, j);
+                        const uint32_t nsets = 1u << __popc(rc);
+                        unsigned key = kAll;
+                        for (uint32_t q = (uint32_t)lane + 1u; q < nsets; q += 32u) {
+                            const uint32_t sub = deposit8(q, rc);
+                            bool ok = true;
+#pragma unroll
+                            for (int j = 0; j < K; ++j)
+                                if ((restm >> j) & 1u) ok &= (nmv[j] & sub) != 0;
+                            if (ok) key = min(key, ((unsigned)__popc(q) << 8) | q);
+                        }
+                        key = __reduce_min_sync(kAll, key);
+                        best |= deposit8(key & 0xffu, rc);
+                        pop += (int)(key >> 8);
+                    }
+                }
+            }
+        }
+        if (pop < 0) {
+            bad = true;
+        } else {
+            // candidate ranks of pick j: usable replicas on the source node,
+            // or (none there) on the nodes of S
+            unsigned long long cm = 0;
+            if (lane < K) {
+                const unsigned long long ok = uok[v];
+                const bool any_ns = (nm >> ns) & 1u;
+                for (int q = 0; q < max_rep; ++q) {
+                    const int r = rep[v * max_rep + q];
+                    if (r >= 0 && ((ok >> r) & 1ull)) {
+                        const int nr = node_of[r];
+                        if (any_ns ? nr == ns : ((best >> nr) & 1u)) cm |= 1ull << r;
+                    }
+                }
+                if ((cm >> s) & 1ull) pick = s;
+                else if ((cm & (cm - 1ull)) == 0) pick = __ffsll((long long)cm) - 1;
+            }
+            for (unsigned open = __ballot_sync(kAll, lane < K && pick < 0); open; open &= open - 1u) {
+                const int j = __ffs(open) - 1;   // picks before j are settled
+                const unsigned long long mine = (lane < j) ? (1ull << pick) : 0ull;
+                const unsigned long long used = ((unsigned long long)__reduce_or_sync(kAll, (unsigned)(mine >> 32)) << 32) |
+                                                __reduce_or_sync(kAll, (unsigned)mine);
+                if (lane == j) {
+                    const unsigned long long u = cm & used;
+                    pick = __ffsll((long long)(u ? u : cm)) - 1;
+                }
+            }
         }
     }
-    cand &= ~(1u << ns);
-    int best_pop = 99;
-    uint32_t best = 0;
-    for (uint32_t sub = cand;; sub = (sub - 1) & cand) {
-        bool ok = true;
-#pragma unroll
-        for (int j = 0; j < K; ++j)
-            if ((need >> j) & 1u) ok &= (nm[j] & sub) != 0;
-        const int pop = __popc(sub);
-        if (ok && (pop < best_pop || (pop == best_pop && sub < best))) {
-            best_pop = pop;
-            best = sub;
-        }
-        if (sub == 0) break;
+    if (bad && rd == 0 && lane == 0) record_error(a.err, MOE_DERR_ID_RANGE);
+    if (lane < K) {
+        if (x.old >= 0) atomicSub(&hist[x.old], 1);
+        a.pick[(size_t)t * K + lane] = bad ? -1 : pick;
+        if (!bad) atomicAdd(&hist[pick], 1);
     }
-    if (best_pop == 99) return -1;
-    unsigned long long used = 0;
-#pragma unroll
-    for (int j = 0; j < K; ++j) {
-        const int32_t *rl = rep + v[j] * max_rep;
-        const unsigned long long ok = uok[v[j]];
-        const bool any_ns = (nm[j] >> ns) & 1u;
-        int pick = -1, used_pick = -1, low = -1;
-        for (int q = 0; q < max_rep; ++q) {
-            const int r = rl[q];
-            if (r < 0 || !((ok >> r) & 1ull)) continue;
-            const bool allowed = any_ns ? (r / rpn == ns) : ((best >> (r / rpn)) & 1u);
-            if (!allowed) continue;
-            if (r == s) pick = r;
-            if (((used >> r) & 1ull) && (used_pick < 0 || r < used_pick)) used_pick = r;
-            if (low < 0 || r < low) low = r;
-        }
-        if (pick < 0) pick = used_pick >= 0 ? used_pick : low;
-        used |= 1ull << pick;
-        pk[j] = pick;
-    }
-    return best_pop;
+    if (lane == 0 && a.nrem) a.nrem[t] = bad ? -1 : pop;
 }
 
 // Inclusive block-wide sum scan of one value per thread (kCapThreads).
@@ -257,6 +387,52 @@ __device__ __forceinline__ int block_scan_incl(int x, int *warp_tot)
     return x + before;
 }
 
+// The block holding token t under the fixed partition [T q / nb, T (q + 1) / nb).
+__device__ __forceinline__ int block_of(int t, int T, int nb)
+{
+    int q = (int)((long long)t * nb / T);
+    while (q + 1 < nb && (int)((long long)T * (q + 1) / nb) <= t) ++q;
+    while (q > 0 && (int)((long long)T * q / nb) > t) --q;
+    return q;
+}
+
+// out[r] += sum over blocks q in [q_lo, q_hi) of blk[q][r], r < G (<= 64):
+// the kCapThreads threads split into kCapThreads / 64 parts over q, eight
+// independent loads in flight per thread, then the parts are added.
+__device__ __forceinline__ void add_block_rows(const int *blk, int G, int q_lo, int q_hi,
+                                               unsigned long long (*red)[64], unsigned long long *out)
+{
+    constexpr int kParts = kCapThreads / 64, kInFlight = 8;
+    const int r = threadIdx.x & 63, part = threadIdx.x / 64;
+    unsigned long long x = 0;
+    if (r < G) {
+        for (int q0 = q_lo + part; q0 < q_hi; q0 += kInFlight * kParts) {
+            unsigned v[kInFlight];
+#pragma unroll
+            for (int u = 0; u < kInFlight; ++u) {
+                const int q = q0 + u * kParts;
+                v[u] = q < q_hi ? (unsigned)__ldcg(blk + (size_t)q * G + r) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kInFlight; ++u) x += v[u];
+        }
+    }
+    red[part][r] = x;
+    __syncthreads();
+    if ((int)threadIdx.x < G) {
+        unsigned long long s = 0;
+#pragma unroll
+        for (int p = 0; p < kParts; ++p) s += red[p][threadIdx.x];
+        out[threadIdx.x] += s;
+    }
+    __syncthreads();
+}
+
+// Block b owns the tokens [T b / nb, T (b + 1) / nb) for the whole launch and
+// keeps, in shared memory, the tasks per rank of its tokens not yet committed
+// (those at or after tc).  A round re-evaluates only the tokens with an
+// expert whose usable replicas changed with the ranks closed last round: for
+// any other token the options, and so the choice, are the same as before.
 template <int K>
 __global__ void __launch_bounds__(kCapThreads)
 assign_capped_kernel(CapArgs a)
@@ -264,14 +440,21 @@ assign_capped_kernel(CapArgs a)
     extern __shared__ __align__(16) unsigned char csm[];
     const int E = a.E, G = a.G, rpn = a.rpn, T = a.T;
     const int nodes = G / rpn, max_rep = 1 + nodes;
-    const int nb = gridDim.x, b = blockIdx.x, tid = threadIdx.x;
+    const int nb = gridDim.x, b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     unsigned long long *uok = reinterpret_cast<unsigned long long *>(csm);             // [E]
-    unsigned long long *base = uok + E;                                                   // [G]
-    int32_t *rep = reinterpret_cast<int32_t *>(base + G);                                 // [E][max_rep]
+    int32_t *rep = reinterpret_cast<int32_t *>(uok + E);                                  // [E][max_rep]
     uint32_t *unm = reinterpret_cast<uint32_t *>(rep + E * max_rep);                      // [E]
-    int *hist = reinterpret_cast<int *>(unm + E);                                         // [G]
+    int *chg = reinterpret_cast<int *>(unm + E);                                          // [E]
     __shared__ int warp_tot[32];
     __shared__ unsigned long long closed_s;
+    __shared__ unsigned long long lds[64];    // tasks committed per rank (the same in every block)
+    __shared__ unsigned long long base[64];   // tasks per rank before this block's first open token
+    __shared__ unsigned long long rc[64];     // tasks per rank of the partly committed block
+    __shared__ unsigned long long red[kCapThreads / 64][64];
+    __shared__ int hist[64];                  // this block's uncommitted tasks per rank
+    __shared__ int node_of[64];               // rank -> node
+    __shared__ int list_s[kCapThreads];       // tokens of a tile to assign
+    __shared__ int nlist_s;
     __shared__ int tau_s, cross_s, tile_tot_s;
 
     for (int e = tid; e < E; e += blockDim.x) {
@@ -284,23 +467,33 @@ assign_capped_kernel(CapArgs a)
             }
             rep[e * max_rep + q] = r;
         }
+        uok[e] = 0;
     }
     if (b == 0 && tid == 0) {
         a.h->tau[0] = T;
         a.h->tau[1] = T;
     }
+    if (tid == 0) nlist_s = 0;
+    for (int r = tid; r < 64; r += blockDim.x) {
+        lds[r] = 0;
+        hist[r] = 0;
+        node_of[r] = r / rpn;
+    }
+    const int lo = (int)((long long)T * b / nb), hi = (int)((long long)T * (b + 1) / nb);
     if (!grid_barrier(&a.h->bar, a.err)) return;
 
     int tc = 0;
     for (int rd = 0; rd <= G + 1; ++rd) {
-        // (a) the closed ranks and each expert's usable replicas
+        int *blk = a.blk + (size_t)(rd & 1) * kCapMaxBlocks * G;
+        const int q0 = block_of(tc, T, nb);             // the block holding tc
+        // (a) the closed ranks, each expert's usable replicas, and whether
+        // they changed since the last round
         if (tid == 0) {
             unsigned long long c = 0;
             for (int r = 0; r < G; ++r)
-                if ((long long)__ldcg(a.load + r) >= a.cap) c |= 1ull << r;
+                if ((long long)lds[r] >= a.cap) c |= 1ull << r;
             closed_s = c;
         }
-        for (int r = tid; r < G; r += blockDim.x) hist[r] = 0;
         __syncthreads();
         const unsigned long long closed = closed_s;
         for (int e = tid; e < E; e += blockDim.x) {
@@ -317,98 +510,117 @@ assign_capped_kernel(CapArgs a)
                 const int r = rep[e * max_rep + q];
                 if (r >= 0 && ((u >> r) & 1ull)) m |= 1u << (r / rpn);
             }
+            chg[e] = rd == 0 || u != uok[e];
             uok[e] = u;
             unm[e] = m;
         }
         __syncthreads();
-        // (b) every remaining token's choice; this block's tokens [lo, hi)
-        const int lo = tc + (int)((long long)(T - tc) * b / nb);
-        const int hi = tc + (int)((long long)(T - tc) * (b + 1) / nb);
-        for (int t = lo + tid; t < hi; t += blockDim.x) {
-            int v[K], pk[K];
+        // (b) the choices of this block's open tokens whose options changed:
+        // a tile of tokens (one per thread) is checked, the changed ones are
+        // listed in shared memory, and the warps assign the listed tokens one
+        // token per warp at a time
+        for (int t0 = max(lo, tc); t0 < hi; t0 += kCapThreads) {
+            const int t = t0 + tid;
+            bool dirty = t < hi && rd == 0;
+            if (t < hi && rd > 0) {
 #pragma unroll
-            for (int j = 0; j < K; ++j) v[j] = __ldg(a.ids + (size_t)t * K + j);
-            const int s = a.src ? __ldg(a.src + t) : t / (T / G);
-            const int n = choose_capped<K>(v, s, E, G, rpn, max_rep, rep, unm, uok, pk);
-            if (n < 0) {
-                if (rd == 0) record_error(a.err, MOE_DERR_ID_RANGE);
-#pragma unroll
-                for (int j = 0; j < K; ++j) a.pick[(size_t)t * K + j] = -1;
-                if (a.nrem) a.nrem[t] = -1;
-                continue;
-            }
-#pragma unroll
-            for (int j = 0; j < K; ++j) {
-                a.pick[(size_t)t * K + j] = pk[j];
-                atomicAdd(&hist[pk[j]], 1);
-            }
-            if (a.nrem) a.nrem[t] = n;
-        }
-        __syncthreads();
-        for (int r = tid; r < G; r += blockDim.x) a.blk[(size_t)b * G + r] = hist[r];
-        if (b == 0 && tid == 0) a.h->tau[(rd + 1) & 1] = T;
-        if (!grid_barrier(&a.h->bar, a.err)) return;
-        // (c) the loads at this block's first token; a rank that reaches the
-        // cap inside the block's tokens gives the first token that sees it
-        // closed
-        for (int r = tid; r < G; r += blockDim.x) {
-            unsigned long long x = __ldcg(a.load + r);
-            for (int q = 0; q < b; ++q) x += (unsigned)__ldcg(a.blk + (size_t)q * G + r);
-            base[r] = x;
-        }
-        __syncthreads();
-        for (int r = 0; r < G; ++r) {
-            if ((closed >> r) & 1ull) continue;
-            const long long b0 = (long long)base[r];
-            if (b0 >= a.cap || b0 + hist[r] < a.cap) continue;
-            // the crossing lies in [lo, hi): scan the block's tokens in order
-            const long long need = a.cap - b0;          // tasks on r that reach the cap
-            long long run = 0;
-            if (tid == 0) cross_s = -1;
-            __syncthreads();
-            for (int t0 = lo; t0 < hi; t0 += blockDim.x) {
-                const int t = t0 + tid;
-                int c = 0;
-                if (t < hi) {
-#pragma unroll
-                    for (int j = 0; j < K; ++j) c += __ldcg(a.pick + (size_t)t * K + j) == r;
+                for (int j = 0; j < K; ++j) {
+                    const int e = __ldg(a.ids + (size_t)t * K + j);
+                    if ((unsigned)e < (unsigned)E) dirty |= chg[e] != 0;
                 }
-                const int incl = block_scan_incl(c, warp_tot);
-                // the one token whose tasks on r take the running count to need
-                if (t < hi && run + incl >= need && run + incl - c < need) cross_s = t;
-                if (tid == (int)blockDim.x - 1) tile_tot_s = incl;
-                __syncthreads();
-                const bool found = cross_s >= 0;
-                run += tile_tot_s;
-                __syncthreads();
-                if (found) break;
             }
-            if (tid == 0 && cross_s >= 0) atomicMin(&a.h->tau[rd & 1], cross_s + 1);
+            const unsigned bal = __ballot_sync(0xffffffffu, dirty);
+            int at = 0;
+            if (lane == 0 && bal) at = atomicAdd(&nlist_s, __popc(bal));
+            at = __shfl_sync(0xffffffffu, at, 0);
+            if (dirty) list_s[at + __popc(bal & ((1u << lane) - 1u))] = t;
+            __syncthreads();
+            const int n = nlist_s;
+            // each warp's next token is loaded while it assigns the current one
+            TokenIn cur = load_token<K>(warp < n ? list_s[warp] : -1, a, rd);
+            for (int i = warp; i < n; i += kCapThreads / 32) {
+                const int i2 = i + kCapThreads / 32;
+                const TokenIn nxt = load_token<K>(i2 < n ? list_s[i2] : -1, a, rd);
+                assign_token_warp<K>(cur, a, rd, max_rep, rep, node_of, unm, uok, hist);
+                cur = nxt;
+            }
+            __syncthreads();
+            if (tid == 0) nlist_s = 0;
             __syncthreads();
         }
+        __syncthreads();
+        for (int r = tid; r < G; r += blockDim.x) blk[(size_t)b * G + r] = hist[r];
+        // the slot of the next round, last read three rounds ago
+        if (b == 0 && tid == 0) a.h->tau[(rd + 1) % 3] = T;
         if (!grid_barrier(&a.h->bar, a.err)) return;
-        // (d) commit the tokens before tau
-        if (tid == 0) tau_s = __ldcg(&a.h->tau[rd & 1]);
+        // (c) the loads at this block's first open token; a rank that
+        // reaches the cap inside the block's open tokens gives the first
+        // token that sees it closed
+        if (hi > tc) {
+            for (int r = tid; r < G; r += blockDim.x) base[r] = lds[r];
+            __syncthreads();
+            add_block_rows(blk, G, q0, b, red, base);
+            const int first = max(lo, tc);
+            for (int r = 0; r < G; ++r) {
+                if ((closed >> r) & 1ull) continue;
+                const long long b0 = (long long)base[r];
+                if (b0 >= a.cap || b0 + hist[r] < a.cap) continue;
+                // the crossing lies in [first, hi): scan the block's tokens in order
+                const long long need = a.cap - b0;          // tasks on r that reach the cap
+                long long run = 0;
+                if (tid == 0) cross_s = -1;
+                __syncthreads();
+                for (int t0 = first; t0 < hi; t0 += blockDim.x) {
+                    const int t = t0 + tid;
+                    int c = 0;
+                    if (t < hi) {
+#pragma unroll
+                        for (int j = 0; j < K; ++j) c += __ldcg(a.pick + (size_t)t * K + j) == r;
+                    }
+                    const int incl = block_scan_incl(c, warp_tot);
+                    // the one token whose tasks on r take the running count to need
+                    if (t < hi && run + incl >= need && run + incl - c < need) cross_s = t;
+                    if (tid == (int)blockDim.x - 1) tile_tot_s = incl;
+                    __syncthreads();
+                    const bool found = cross_s >= 0;
+                    run += tile_tot_s;
+                    __syncthreads();
+                    if (found) break;
+                }
+                if (tid == 0 && cross_s >= 0) atomicMin(&a.h->tau[rd % 3], cross_s + 1);
+                __syncthreads();
+            }
+        }
+        if (!grid_barrier(&a.h->bar, a.err)) return;
+        // (d) commit the tokens before tau: every block adds, in its own copy
+        // of the loads, the counts of the blocks whose open tokens all
+        // precede tau and recounts the one block that holds tau (no third
+        // barrier: the counts are double-buffered by round, tau kept in three
+        // slots)
+        if (tid == 0) tau_s = __ldcg(&a.h->tau[rd % 3]);
         __syncthreads();
         const int tau = tau_s;
-        if (hi <= tau) {
-            for (int r = tid; r < G; r += blockDim.x)
-                if (hist[r]) atomicAdd(a.load + r, (unsigned long long)hist[r]);
-        } else if (lo < tau) {
+        const int qs = tau < T ? block_of(tau, T, nb) : nb;   // blocks [q0, qs) commit whole
+        add_block_rows(blk, G, q0, qs, red, lds);
+        const int ls = qs < nb ? max((int)((long long)T * qs / nb), tc) : T;
+        if (ls < tau) {
+            for (int r = tid; r < G; r += blockDim.x) rc[r] = 0;
             __syncthreads();
-            for (int r = tid; r < G; r += blockDim.x) hist[r] = 0;
-            __syncthreads();
-            for (int t = lo + tid; t < tau; t += blockDim.x)
+            for (int t = ls + tid; t < tau; t += blockDim.x)
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
                     const int r = __ldcg(a.pick + (size_t)t * K + j);
-                    if (r >= 0) atomicAdd(&hist[r], 1);
+                    if (r >= 0) atomicAdd(&rc[r], 1ull);
                 }
             __syncthreads();
-            for (int r = tid; r < G; r += blockDim.x)
-                if (hist[r]) atomicAdd(a.load + r, (unsigned long long)hist[r]);
+            for (int r = tid; r < G; r += blockDim.x) {
+                lds[r] += rc[r];
+                if (b == qs) hist[r] -= (int)rc[r];
+            }
         }
-        if (!grid_barrier(&a.h->bar, a.err)) return;
+        if (hi <= tau)
+            for (int r = tid; r < G; r += blockDim.x) hist[r] = 0;
+        __syncthreads();
         tc = tau;
         if (tc >= T) {
             if (b == 0 && tid == 0) a.h->rounds = rd + 1;
@@ -417,7 +629,7 @@ assign_capped_kernel(CapArgs a)
         if (rd == G + 1) record_error(a.err, MOE_DERR_TIMEOUT);   // more rounds than ranks: not reachable
     }
     if (b == 0 && a.rank_load)
-        for (int r = tid; r < G; r += blockDim.x) a.rank_load[r] = (long long)__ldcg(a.load + r);
+        for (int r = tid; r < G; r += blockDim.x) a.rank_load[r] = (long long)lds[r];
 }
 
 template <int K>
@@ -425,15 +637,15 @@ moe_status launch_capped(CapArgs args, cudaStream_t s)
 {
     auto kern = assign_capped_kernel<K>;
     const int max_rep = 1 + args.G / args.rpn;
-    const size_t smem = sizeof(unsigned long long) * ((size_t)args.E + args.G) +
-                        sizeof(int32_t) * ((size_t)args.E * max_rep + args.E + args.G);
+    const size_t smem = sizeof(unsigned long long) * (size_t)args.E +
+                        sizeof(int32_t) * ((size_t)args.E * max_rep + 2 * (size_t)args.E);
     if (allow_smem(kern, smem) != cudaSuccess) return MOE_ERR_CUDA;
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCapThreads, smem) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (per_sm < 1) return MOE_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)std::min(sm_count(), kCapMaxBlocks));   // one block per SM: co-resident
+    cfg.gridDim = dim3((unsigned)std::min(coop_grid(), kCapMaxBlocks));   // at most one block per SM: co-resident
     cfg.blockDim = dim3(kCapThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
@@ -492,7 +704,7 @@ extern "C" moe_status moe_assign_replicas(const int32_t *ids, int T, int k, int 
 extern "C" size_t moe_assign_replicas_capped_workspace(int G)
 {
     if (G < 1 || G > 64) return 0;
-    return 256 + 512 + round_up(sizeof(int) * (size_t)kCapMaxBlocks * G, 256);
+    return 256 + round_up(sizeof(int) * 2 * (size_t)kCapMaxBlocks * G, 256);
 }
 
 extern "C" moe_status moe_assign_replicas_capped(const int32_t *ids, int T, int k, int E, int G, int rpn,
@@ -504,7 +716,7 @@ extern "C" moe_status moe_assign_replicas_capped(const int32_t *ids, int T, int 
     if (T < 0 || k < 1 || k > 8 || E < k || G < 1 || G > 64 || rpn < 1 || G % rpn != 0 || !err) return MOE_ERR_ARG;
     if (!(eps >= 0.0)) return MOE_ERR_ARG;
     if (G / rpn > kMaxNodes) return MOE_ERR_UNSUPPORTED;
-    if ((size_t)E * (G / rpn + 2) * sizeof(int32_t) + (size_t)(E + G) * 8 > 200 * 1024) return MOE_ERR_UNSUPPORTED;
+    if ((size_t)E * (G / rpn + 3) * sizeof(int32_t) + (size_t)E * 8 > 200 * 1024) return MOE_ERR_UNSUPPORTED;
     if (!src_rank && T % G != 0) return MOE_ERR_ARG;
     if (T == 0) {
         if (rank_load && cudaMemsetAsync(rank_load, 0, sizeof(long long) * G, stream) != cudaSuccess)
@@ -523,10 +735,9 @@ extern "C" moe_status moe_assign_replicas_capped(const int32_t *ids, int T, int 
     a.cap = c >= 9.0e18 ? (long long)INT64_MAX : (long long)c;
     a.pick = pick_rank; a.nrem = n_remote; a.rank_load = rank_load;
     a.h = reinterpret_cast<CapHeader *>(w);
-    a.load = reinterpret_cast<unsigned long long *>(w + 256);
-    a.blk = reinterpret_cast<int *>(w + 256 + 512);
+    a.blk = reinterpret_cast<int *>(w + 256);
     a.err = err;
-    if (cudaMemsetAsync(w, 0, 256 + 512, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(w, 0, 256, stream) != cudaSuccess) return MOE_ERR_CUDA;
     moe_status st = MOE_ERR_ARG;
     switch (k) {
     case 1: st = launch_capped<1>(a, stream); break;

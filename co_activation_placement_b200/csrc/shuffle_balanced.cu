@@ -530,7 +530,7 @@ moe_status launch_balanced(BalArgs args, cudaStream_t s)
         return MOE_ERR_CUDA;
     if (per_sm < 1) return MOE_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)sm_count());     // one block per SM: co-resident by construction
+    cfg.gridDim = dim3((unsigned)coop_grid());    // at most one block per SM: co-resident by construction
     cfg.blockDim = dim3(kBalThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;

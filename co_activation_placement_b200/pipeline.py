@@ -68,6 +68,19 @@ class HotPath:
     shuffle_capacity: int = 0          # > 0: at most this many tokens per rank (moe_shuffle_balanced)
     replica_eps: Optional[float] = None   # load tolerance of the replica assignment (None: no cap)
     overlap: bool = True               # control work on a second stream beside the row traffic
+    # "overlap": every layer's plan, shuffle and the statistics ahead on a
+    # second stream (all routing known up front); "forward": the order of a
+    # forward pass -- layer l's plan in line before its rows, its shuffle
+    # targets and the statistics beside them; "inline": everything in line.
+    # None: "overlap" if overlap else "inline".
+    schedule: Optional[str] = None
+    # blocks of the cooperative launches (balanced shuffle, capped assignment)
+    # when they run beside the row traffic.  None: the balanced shuffle takes
+    # min(G, 32) blocks (the rest of the SMs stream rows; on large_ep64 32
+    # blocks gave the shortest step, 64 and 24 longer ones), the capped
+    # assignment one block per SM (its rounds' work per block grows as T / blocks)
+    side_coop_blocks: Optional[int] = None
+    side_priority: int = 0             # priority of the second stream (lower = higher priority)
     # buffers
     stats: dict = field(default_factory=dict)
     plans: List[cap.Plan] = field(default_factory=list)
@@ -101,21 +114,21 @@ class HotPath:
                                           dtype=torch.uint8, device=dev)
             # rounds and proposals of each balanced shuffle
             self.shuffle_info = torch.zeros((max(L - 1, 1), 6), dtype=torch.int64, device=dev)
-        if self.shuffle and self.shuffle_capacity > 0:
-            # the balanced shuffle is one cooperative launch over every SM:
-            # beside the row kernels it would slow them and itself
-            self.overlap = False
+        if self.schedule is None:
+            self.schedule = "overlap" if self.overlap else "inline"
+        if self.schedule not in ("overlap", "forward", "inline"):
+            raise ValueError("schedule must be overlap, forward or inline")
+        self.overlap = self.schedule != "inline"
         if self.overlap:
-            self.side = torch.cuda.Stream(device=dev)
+            self.side = torch.cuda.Stream(device=dev, priority=self.side_priority)
             self.fork_ev = torch.cuda.Event()
             self.join_ev = torch.cuda.Event()
             self.plan_ev = [torch.cuda.Event() for _ in range(L)]
+            self.shuffle_ev = [torch.cuda.Event() for _ in range(L)]
         if self.replicas:
             self.pick_rank = torch.empty((T, k), dtype=torch.int32, device=dev)
             self.n_remote = torch.empty(T, dtype=torch.int32, device=dev)
             if self.replica_eps is not None:
-                # the capped assignment is one cooperative launch over every SM
-                self.overlap = False
                 self.rank_load = torch.zeros((L, self.G), dtype=torch.int64, device=dev)
                 self.capped_ws = torch.empty(cap.assign_replicas_capped_workspace(self.G), dtype=torch.uint8,
                                              device=dev)
@@ -143,6 +156,26 @@ class HotPath:
                 self.events.append((name, a, b))
         return out
 
+    @property
+    def side_calls(self):
+        """The calls that run on the second stream, beside the row traffic."""
+        return {"overlap": ("stats", "plan", "shuffle"), "forward": ("stats", "shuffle"), "inline": ()}[self.schedule]
+
+    def _coop(self, fn, name):
+        """Run a call that makes a cooperative launch; beside the row traffic
+        the balanced shuffle takes fewer blocks than SMs, leaving the other
+        SMs to the rows."""
+        if name not in self.side_calls:
+            return fn()
+        n = self.side_coop_blocks
+        if n is None:
+            n = min(self.G, 32) if name == "shuffle" else 0
+        prev = cap.cooperative_blocks(n)
+        try:
+            return fn()
+        finally:
+            cap.cooperative_blocks(prev)
+
     def reset_events(self):
         self.events = []
 
@@ -160,9 +193,10 @@ class HotPath:
 
             def go():
                 if self.replica_eps is not None:
-                    cap.assign_replicas_capped(self.ids[l], self.E, self.G, self.rpn, rr, nr, self.replica_eps,
-                                               src_rank=src, pick_rank=self.pick_rank, n_remote=self.n_remote,
-                                               rank_load=self.rank_load[l], err=self.err, ws=self.capped_ws)
+                    self._coop(lambda: cap.assign_replicas_capped(
+                        self.ids[l], self.E, self.G, self.rpn, rr, nr, self.replica_eps, src_rank=src,
+                        pick_rank=self.pick_rank, n_remote=self.n_remote, rank_load=self.rank_load[l], err=self.err,
+                        ws=self.capped_ws), "plan")
                 else:
                     cap.assign_replicas(self.ids[l], self.E, self.G, self.rpn, rr, nr, src_rank=src,
                                         pick_rank=self.pick_rank, n_remote=self.n_remote, err=self.err)
@@ -192,24 +226,24 @@ class HotPath:
         if not (self.shuffle and l + 1 < self.L):
             return
         if self.shuffle_capacity > 0:
-            self._call("shuffle", lambda: cap.shuffle_balanced(self.ids[l], self.E, self.G, self.rank_scores[l],
-                                                               self.shuffle_capacity, target=self.targets[l],
-                                                               info=self.shuffle_info[l], err=self.err,
-                                                               ws=self.shuffle_ws))
+            self._call("shuffle", lambda: self._coop(lambda: cap.shuffle_balanced(
+                self.ids[l], self.E, self.G, self.rank_scores[l], self.shuffle_capacity, target=self.targets[l],
+                info=self.shuffle_info[l], err=self.err, ws=self.shuffle_ws), "shuffle"))
         else:
             self._call("shuffle", lambda: cap.shuffle_targets(self.ids[l], self.E, self.G, self.rank_scores[l],
                                                               target=self.targets[l], err=self.err))
 
     def step(self):
-        """One step.  With overlap, the control work -- plans, shuffle targets
-        and statistics, which read only routing ids and tables -- runs on a
-        second stream that starts when everything before the step is done and
-        keeps ahead of the row traffic; the permute and combine of layer l wait
-        only for layer l's plan."""
+        """One step.  With the overlap schedule, the control work -- plans,
+        shuffle targets and statistics, which read only routing ids and tables
+        -- runs on a second stream that starts when everything before the
+        step is done and keeps ahead of the row traffic; the permute and
+        combine of layer l wait only for layer l's plan.  The forward schedule
+        keeps each plan on the critical path (see the field's comment)."""
         if not self.rows:
             self._stats()
             return
-        if not self.overlap:
+        if self.schedule == "inline":
             self._stats()
             for l in range(self.L):
                 self._plan(l)
@@ -217,6 +251,31 @@ class HotPath:
                 self._shuffle(l)
             return
         main = torch.cuda.current_stream(self.ids.device)
+        if self.schedule == "forward":
+            # layer l's routing exists once layer l - 1's rows are done: its
+            # plan runs in line before its rows; its shuffle targets (needed
+            # by the next layer's plan) and, after the last layer, the
+            # statistics run beside the rows on the second stream
+            for l in range(self.L):
+                if l > 0 and self.shuffle:
+                    main.wait_event(self.shuffle_ev[l - 1])
+                self._plan(l)
+                # layer l's routing is known from its plan on; the side work
+                # starts after the plan so that it does not delay it
+                self.plan_ev[l].record(main)
+                if self.shuffle and l + 1 < self.L:
+                    self.side.wait_event(self.plan_ev[l])
+                    with torch.cuda.stream(self.side):
+                        self._shuffle(l)
+                        self.shuffle_ev[l].record(self.side)
+                if l == self.L - 1:
+                    self.side.wait_event(self.plan_ev[l])
+                    with torch.cuda.stream(self.side):
+                        self._stats()
+                        self.join_ev.record(self.side)
+                self._rows(l)
+            main.wait_event(self.join_ev)
+            return
         self.fork_ev.record(main)
         self.side.wait_event(self.fork_ev)
         with torch.cuda.stream(self.side):
@@ -329,7 +388,7 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
             x_dtype: str, ids_cal: np.ndarray, placement: str = "correlated", shuffle: bool = True,
             out_dtype=torch.bfloat16, device="cuda", rows: bool = True, timers: bool = False,
             scales: Optional[np.ndarray] = None, replica_extra: int = 0, shuffle_capacity: int = 0,
-            overlap: bool = True, replica_eps: Optional[float] = None) -> HotPath:
+            overlap: bool = True, replica_eps: Optional[float] = None, schedule: Optional[str] = None) -> HotPath:
     """Upload a batch (host numpy arrays; x as float32 or bf16 bit patterns)
     and its calibration batch, calibrate, and return the step's HotPath."""
     dev = torch.device(device)
@@ -346,7 +405,7 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
         if scales is not None else []
     return HotPath(E=E, G=G, rpn=rpn, ids=ids_d, gates=gates_d, x=x_d, e2r=e2r, rank_scores=rs,
                    out_dtype=out_dtype, rows=rows, timers=timers, prereduce=scales is not None, scales=scales_d,
-                   replicas=reps, shuffle_capacity=shuffle_capacity, overlap=overlap,
+                   replicas=reps, shuffle_capacity=shuffle_capacity, overlap=overlap, schedule=schedule,
                    replica_eps=replica_eps if replica_extra > 0 else None)
 
 

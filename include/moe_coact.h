@@ -39,8 +39,8 @@
  *    caller zeroes `err` and reads it after synchronising.  When it is
  *    non-zero the outputs of that call are unspecified.  Kernels never trap.
  *  - Calls keep no state between invocations except the global launch
- *    counter, the method settings (moe_coact_stats_method,
- *    moe_plan_dispatch_method) and the static scratch of
+ *    counter, the settings (moe_coact_stats_method,
+ *    moe_plan_dispatch_method, moe_cooperative_blocks) and the static scratch of
  *    moe_plan_dispatch_static.  Workspace ("ws") is
  *    caller-provided device memory of at least the size the matching
  *    *_workspace query returns, 256-byte aligned.
@@ -173,6 +173,15 @@ size_t moe_plan_dispatch_workspace(int T, int k, int G, int with_src_rank);
  * setting also applies to moe_plan_dispatch_ranks and
  * moe_plan_dispatch_static and affects calls issued after it returns. */
 int moe_plan_dispatch_method(int method);
+
+/* Blocks of the cooperative kernels' launches (moe_shuffle_balanced,
+ * moe_assign_replicas_capped; process-wide; returns the previous setting, or
+ * -1 for a negative argument): 0 = default, one block per SM; n > 0 = n
+ * blocks (at most one per SM).  Results are identical for every setting.  A
+ * smaller grid leaves the other SMs to kernels running beside the call on
+ * other streams -- the row traffic, when these run on a second stream -- at
+ * the cost of a longer call.  Affects calls issued after it returns. */
+int moe_cooperative_blocks(int blocks);
 moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E, int G, int rpn,
                              const int32_t *expert_to_rank, const int32_t *src_rank,
                              const moe_plan *plan, int32_t *err,
@@ -230,8 +239,9 @@ moe_status moe_assign_replicas(const int32_t *ids, int T, int k, int E, int G, i
  * rank_load device int64 [G] out or NULL (tasks per rank after the batch);
  * ws device, moe_assign_replicas_capped_workspace(G) bytes, 256-byte aligned,
  * caller-owned, overwritten by each call (calls on one workspace must not
- * overlap).  Data errors as moe_assign_replicas; an invalid token counts for
- * no rank.
+ * overlap).  Limits: G <= 64, G/rpn <= 8 nodes, E * (4 (G/rpn + 3) + 8)
+ * bytes <= 200 KB (else MOE_ERR_UNSUPPORTED).  Data errors as
+ * moe_assign_replicas; an invalid token counts for no rank.
  * ---------------------------------------------------------------------- */
 size_t moe_assign_replicas_capped_workspace(int G);
 moe_status moe_assign_replicas_capped(const int32_t *ids, int T, int k, int E, int G, int rpn,

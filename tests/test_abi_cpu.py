@@ -44,6 +44,19 @@ def test_every_declared_symbol_is_exported(cap):
     assert not missing, missing
 
 
+def test_process_wide_settings(cap):
+    """The method and grid settings return the previous value and reject bad
+    arguments without touching a device."""
+    prev = cap.cooperative_blocks(7)
+    assert cap.cooperative_blocks(prev) == 7
+    with pytest.raises(ValueError):
+        cap.cooperative_blocks(-1)
+    prev = cap.plan_dispatch_method(1)
+    assert cap.plan_dispatch_method(prev) == 1
+    with pytest.raises(ValueError):
+        cap.plan_dispatch_method(2)
+
+
 def test_status_strings(cap):
     assert cap.lib().moe_status_string(0) == b"ok"
     assert cap.lib().moe_status_string(3).startswith(b"workspace")

@@ -448,18 +448,19 @@ def test_pipeline_capacity_placement(cap, name, placement):
 
 @pytest.mark.parametrize("name", ["ep32", "large_ep64"])
 def test_overlapped_step_equals_serial_step(cap, name):
-    """The step with the control work on a second stream produces every
-    output bit for bit as the step run in line, also when replayed from a
-    CUDA graph."""
+    """The step with the control work on a second stream -- all of it ahead
+    (overlap), or the forward-pass order with only the shuffle targets and
+    statistics beside the rows (forward) -- produces every output bit for bit
+    as the step run in line, also when replayed from a CUDA graph."""
     from co_activation_placement_b200 import pipeline
     w = WORKLOADS[name]
     ids = make_routing(w)
     ids_cal = make_routing(w, seed=w.seed + 1)
     gates, x = make_gates(w), make_hidden(w)
     outs = {}
-    for overlap in (False, True):
+    for overlap in ("inline", "overlap", "forward"):
         hp = pipeline.prepare(w.E, w.G, w.rpn, ids, gates, x, w.dtype, ids_cal, out_dtype=torch.float32,
-                              overlap=overlap)
+                              schedule=overlap)
         hp.step()
         g = hp.capture(2)
         g.replay()
@@ -470,5 +471,6 @@ def test_overlapped_step_equals_serial_step(cap, name):
                          + [host(o).copy() for o in hp.outs])
         del g, hp
         torch.cuda.empty_cache()
-    for a, b in zip(outs[False], outs[True]):
-        assert (a.view(np.uint8) == b.view(np.uint8)).all()
+    for sched in ("overlap", "forward"):
+        for a, b in zip(outs["inline"], outs[sched]):
+            assert (a.view(np.uint8) == b.view(np.uint8)).all()

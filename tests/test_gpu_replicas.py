@@ -165,3 +165,87 @@ def test_capped_assignment_errors(cap):
     # the context stays usable
     pr, _, _ = cap.assign_replicas_capped(dev(ids), E, G, rpn, dev(rr), dev(nr), 0.1)
     assert (host(pr)[:T] == orc.assign_replicas_capped(ids, E, G, rpn, rr, nr, 0.1)[0]).all()
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_capped_assignment_random(cap, seed):
+    """Random shapes, replica budgets and tolerances, with skewed expert
+    popularity so that many ranks reach the cap at scattered tokens: every
+    round re-evaluates only the tokens whose options changed."""
+    rng = np.random.default_rng(900 + seed)
+    rpn = int(rng.choice([1, 2, 4, 8]))
+    G = rpn * int(rng.integers(1, min(8, 64 // rpn) + 1))
+    E = G * int(rng.integers(1, 9))
+    k = int(rng.integers(1, min(8, E) + 1))
+    T = int(rng.integers(1, 20000))
+    if rng.random() < 0.5:
+        T = T // G * G or G
+    eps = float(rng.choice([0.0, 0.01, 0.05, 0.3]))
+    extra = int(rng.integers(1, 4))
+    pop = rng.zipf(1.3, E).astype(np.float64)
+    pop /= pop.sum()
+    ids = np.stack([rng.choice(E, k, replace=False, p=pop) for _ in range(T)]).astype(np.int32)
+    C = orc.coact(ids[None], E, want=("coact",))["coact"][0]
+    e2r = orc.place_correlated(C, G, rpn)
+    rr, nr = orc.place_replicas(C, G, rpn, e2r, extra)
+    src = rng.integers(0, G, T).astype(np.int32) if (T % G or rng.random() < 0.5) else None
+    err = cap.new_err("cuda")
+    pr, nrem, load = cap.assign_replicas_capped(dev(ids), E, G, rpn, dev(rr), dev(nr), eps,
+                                                src_rank=None if src is None else dev(src), err=err)
+    pr_o, nrem_o, load_o = orc.assign_replicas_capped(ids, E, G, rpn, rr, nr, eps, src_rank=src)
+    assert int(host(err)[0]) == 0
+    assert (host(pr)[:T] == pr_o).all() and (host(nrem)[:T] == nrem_o).all()
+    assert host(load).tolist() == load_o.tolist()
+
+
+@pytest.mark.parametrize("blocks", [1, 3, 64, 0])
+def test_capped_assignment_grid_sizes(cap, blocks):
+    """The result does not depend on the cooperative grid (moe_cooperative_blocks):
+    one block, a few, one per rank, one per SM."""
+    w = WORKLOADS["large_ep64"]
+    ids = make_routing(w)[0]
+    cal = make_routing(w, seed=1)[0]
+    C = orc.coact(cal[None], w.E, want=("coact",))["coact"][0]
+    rr, nr = orc.place_replicas(C, w.G, w.rpn, orc.place_correlated(C, w.G, w.rpn), 1)
+    prev = cap.cooperative_blocks(blocks)
+    try:
+        err = cap.new_err("cuda")
+        pr, nrem, load = cap.assign_replicas_capped(dev(ids), w.E, w.G, w.rpn, dev(rr), dev(nr), 0.1, err=err)
+        torch.cuda.synchronize()
+    finally:
+        cap.cooperative_blocks(prev)
+    pr_o, nrem_o, load_o = orc.assign_replicas_capped(ids, w.E, w.G, w.rpn, rr, nr, 0.1)
+    assert int(host(err)[0]) == 0
+    assert (host(pr)[: w.T] == pr_o).all() and (host(nrem)[: w.T] == nrem_o).all()
+    assert host(load).tolist() == load_o.tolist()
+
+
+@pytest.mark.parametrize("name,overlap", [("ep32", True), ("ep32", False), ("large_ep64", True)])
+def test_pipeline_with_capped_replicas(cap, name, overlap):
+    """A whole step with the load-capped assignment (eps = 0.1): every layer's
+    plan over the picks the oracle's token-order greedy makes, with the
+    previous layer's shuffle targets as source ranks; beside the row traffic
+    (one block per rank) or in line."""
+    from co_activation_placement_b200 import pipeline
+    from synth import make_gates, make_hidden
+    w = WORKLOADS[name]
+    ids = make_routing(w)
+    ids_cal = make_routing(w, seed=w.seed + 1)
+    hp = pipeline.prepare(w.E, w.G, w.rpn, ids, make_gates(w), make_hidden(w), w.dtype, ids_cal,
+                          shuffle=True, out_dtype=torch.float32, replica_extra=1, replica_eps=0.1,
+                          overlap=overlap)
+    hp.step()
+    torch.cuda.synchronize()
+    assert int(host(hp.err)[0]) == 0
+    oc = orc.coact(ids_cal, w.E, want=("coact", "trans"))
+    e2r = [orc.place_correlated(oc["coact"][l], w.G, w.rpn) for l in range(w.L)]
+    src = None
+    for l in range(w.L):
+        rr, nr = orc.place_replicas(oc["coact"][l], w.G, w.rpn, e2r[l], 1)
+        pr, _, load = orc.assign_replicas_capped(ids[l], w.E, w.G, w.rpn, rr, nr, 0.1, src_rank=src)
+        assert host(hp.rank_load[l]).tolist() == load.tolist()
+        op = orc.plan(ids[l], w.E, w.G, w.rpn, None, src_rank=src, pick_rank=pr)
+        assert host(hp.plans[l].summary).tolist() == op["summary"].tolist()
+        assert (host(hp.plans[l].row_of)[: w.T] == op["row_of"]).all()
+        if l + 1 < w.L:
+            src = orc.shuffle_targets(ids[l], w.E, w.G, orc.rank_score(oc["trans"][l], e2r[l + 1], w.G))

@@ -131,17 +131,38 @@ def test_empty_and_argument_errors(cap):
     assert ei.value.status == cap.MOE_ERR_ARG
 
 
-@pytest.mark.parametrize("name", ["one_node", "large_ep64"])
-def test_pipeline_with_balanced_shuffle(cap, name):
+@pytest.mark.parametrize("blocks", [1, 5, 64])
+def test_grid_sizes(cap, blocks):
+    """The result does not depend on the cooperative grid (moe_cooperative_blocks):
+    blocks that own several ranks, or none."""
+    w = WORKLOADS["large_ep64"]
+    ids = make_routing(w)[0]
+    cal = make_routing(w, seed=w.seed + 1)
+    oc = orc.coact(cal[:2], w.E, want=("coact", "trans"))
+    rs = orc.rank_score(oc["trans"][0], orc.place_correlated(oc["coact"][1], w.G, w.rpn), w.G)
+    prev = cap.cooperative_blocks(blocks)
+    try:
+        got, info, err = run(cap, ids, w.E, w.G, rs, w.T // w.G)
+    finally:
+        cap.cooperative_blocks(prev)
+    assert err == 0
+    assert (got == orc.shuffle_balanced(ids, w.E, w.G, rs, w.T // w.G)).all()
+
+
+@pytest.mark.parametrize("name,overlap", [("one_node", True), ("one_node", False), ("large_ep64", True),
+                                          ("large_ep64", False)])
+def test_pipeline_with_balanced_shuffle(cap, name, overlap):
     """A whole step with capped shards: every layer's plan uses the previous
-    layer's balanced targets as source ranks, as the oracle does."""
+    layer's balanced targets as source ranks, as the oracle does; the shuffle
+    beside the row traffic (one block per rank) or in line."""
     from co_activation_placement_b200 import pipeline
     from synth import make_gates, make_hidden
     w = WORKLOADS[name]
     ids = make_routing(w)
     ids_cal = make_routing(w, seed=w.seed + 1)
     hp = pipeline.prepare(w.E, w.G, w.rpn, ids, make_gates(w), make_hidden(w), w.dtype, ids_cal,
-                          shuffle=True, out_dtype=torch.float32, shuffle_capacity=w.T // w.G)
+                          shuffle=True, out_dtype=torch.float32, shuffle_capacity=w.T // w.G,
+                          overlap=overlap)
     hp.step()
     torch.cuda.synchronize()
     assert int(host(hp.err)[0]) == 0
