@@ -23,7 +23,7 @@
 // ranks, which changes at most G times, so one cooperative launch computes
 // it in rounds: the remaining tokens' choices under the current closed set,
 // in parallel, one warp per token (after the first round only the tokens
-// with an expert whose usable replicas changed); per-block task counts per rank and their
+// with a pick on a rank that just closed); per-block task counts per rank and their
 // running sum over blocks locate the first token tau at which an open rank
 // reaches the cap (a block-wide scan inside the block where that happens);
 // the choices of tokens before tau are final, their tasks join the loads,
@@ -456,6 +456,7 @@ assign_capped_kernel(CapArgs a)
     __shared__ int list_s[kCapThreads];       // tokens of a tile to assign
     __shared__ int nlist_s;
     __shared__ int tau_s, cross_s, tile_tot_s;
+    __shared__ unsigned cross_s2[2];
 
     for (int e = tid; e < E; e += blockDim.x) {
         const int n = min(max(__ldg(a.nr + e), 0), max_rep);
@@ -482,7 +483,8 @@ assign_capped_kernel(CapArgs a)
     const int lo = (int)((long long)T * b / nb), hi = (int)((long long)T * (b + 1) / nb);
     if (!grid_barrier(&a.h->bar, a.err)) return;
 
-    int tc = 0;
+    int tc = 0, any_chg = 0;
+    unsigned long long closed_before = 0;
     for (int rd = 0; rd <= G + 1; ++rd) {
         int *blk = a.blk + (size_t)(rd & 1) * kCapMaxBlocks * G;
         const int q0 = block_of(tc, T, nb);             // the block holding tc
@@ -496,6 +498,8 @@ assign_capped_kernel(CapArgs a)
         }
         __syncthreads();
         const unsigned long long closed = closed_s;
+        const unsigned long long closing = closed & ~closed_before;   // ranks closed since the last round
+        closed_before = closed;
         for (int e = tid; e < E; e += blockDim.x) {
             unsigned long long all = 0, open = 0;
             for (int q = 0; q < max_rep; ++q) {
@@ -511,22 +515,43 @@ assign_capped_kernel(CapArgs a)
                 if (r >= 0 && ((u >> r) & 1ull)) m |= 1u << (r / rpn);
             }
             chg[e] = rd == 0 || u != uok[e];
+            any_chg |= chg[e];
             uok[e] = u;
             unm[e] = m;
         }
-        __syncthreads();
-        // (b) the choices of this block's open tokens whose options changed:
-        // a tile of tokens (one per thread) is checked, the changed ones are
-        // listed in shared memory, and the warps assign the listed tokens one
-        // token per warp at a time
-        for (int t0 = max(lo, tc); t0 < hi; t0 += kCapThreads) {
+        // no expert's usable replicas changed: no choice changes this round
+        const bool some_chg = __syncthreads_or(any_chg) != 0;
+        any_chg = 0;
+        // (b) round 0: the choices are those of the uncapped assignment
+        // (no rank is open-and-closed yet: every replica is usable), which
+        // the launch before this one wrote; count them
+        if (rd == 0)
+            for (int t = lo + tid; t < hi; t += kCapThreads)
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    const int r = __ldcg(a.pick + (size_t)t * K + j);
+                    if (r >= 0) atomicAdd(&hist[r], 1);
+                }
+        // later rounds: the choices of this block's open tokens whose options
+        // changed: a tile of tokens (one per thread) is checked, the changed
+        // ones are listed in shared memory, and the warps assign the listed
+        // tokens one token per warp at a time
+        for (int t0 = max(lo, tc); rd > 0 && some_chg && t0 < hi; t0 += kCapThreads) {
             const int t = t0 + tid;
-            bool dirty = t < hi && rd == 0;
-            if (t < hi && rd > 0) {
+            // a token's choice can change only through a pick on a rank that
+            // just closed, of an expert whose usable replicas changed: while
+            // every pick stays usable the old node set stays feasible, and
+            // with fewer options it stays the smallest (and so do the picks);
+            // options grow only when an expert's last open replica closes,
+            // and that replica was then its pick
+            bool dirty = false;
+            if (t < hi) {
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
                     const int e = __ldg(a.ids + (size_t)t * K + j);
-                    if ((unsigned)e < (unsigned)E) dirty |= chg[e] != 0;
+                    const int r = __ldcg(a.pick + (size_t)t * K + j);
+                    if ((unsigned)e < (unsigned)E && r >= 0)
+                        dirty |= chg[e] != 0 && ((closing >> r) & 1ull);
                 }
             }
             const unsigned bal = __ballot_sync(0xffffffffu, dirty);
@@ -561,10 +586,20 @@ assign_capped_kernel(CapArgs a)
             __syncthreads();
             add_block_rows(blk, G, q0, b, red, base);
             const int first = max(lo, tc);
-            for (int r = 0; r < G; ++r) {
-                if ((closed >> r) & 1ull) continue;
+            if (tid < 64) {                      // the open ranks whose cap falls in this block
+                bool x = false;
+                if (tid < G && !((closed >> tid) & 1ull)) {
+                    const long long b0 = (long long)base[tid];
+                    x = b0 < a.cap && b0 + hist[tid] >= a.cap;
+                }
+                const unsigned bl = __ballot_sync(0xffffffffu, x);
+                if (lane == 0) cross_s2[warp] = bl;
+            }
+            __syncthreads();
+            const unsigned long long xm = ((unsigned long long)cross_s2[1] << 32) | cross_s2[0];
+            for (unsigned long long mr = xm; mr; mr &= mr - 1ull) {
+                const int r = __ffsll((long long)mr) - 1;
                 const long long b0 = (long long)base[r];
-                if (b0 >= a.cap || b0 + hist[r] < a.cap) continue;
                 // the crossing lies in [first, hi): scan the block's tokens in order
                 const long long need = a.cap - b0;          // tasks on r that reach the cap
                 long long run = 0;
@@ -738,17 +773,20 @@ extern "C" moe_status moe_assign_replicas_capped(const int32_t *ids, int T, int 
     a.blk = reinterpret_cast<int *>(w + 256);
     a.err = err;
     if (cudaMemsetAsync(w, 0, 256, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    // the first round's choices -- every replica usable -- are the uncapped
+    // assignment: one thread per token over the whole GPU, then the rounds
     moe_status st = MOE_ERR_ARG;
     switch (k) {
-    case 1: st = launch_capped<1>(a, stream); break;
-    case 2: st = launch_capped<2>(a, stream); break;
-    case 3: st = launch_capped<3>(a, stream); break;
-    case 4: st = launch_capped<4>(a, stream); break;
-    case 5: st = launch_capped<5>(a, stream); break;
-    case 6: st = launch_capped<6>(a, stream); break;
-    case 7: st = launch_capped<7>(a, stream); break;
-    case 8: st = launch_capped<8>(a, stream); break;
+#define MOE_CAPPED_CASE(KK)                                                                                  \
+    case KK:                                                                                                 \
+        st = launch_assign<KK>(ids, T, E, G, rpn, replica_rank, n_rep, src_rank, pick_rank, n_remote, err,   \
+                               stream);                                                                      \
+        if (st == MOE_OK) st = launch_capped<KK>(a, stream);                                                 \
+        break;
+    MOE_CAPPED_CASE(1) MOE_CAPPED_CASE(2) MOE_CAPPED_CASE(3) MOE_CAPPED_CASE(4)
+    MOE_CAPPED_CASE(5) MOE_CAPPED_CASE(6) MOE_CAPPED_CASE(7) MOE_CAPPED_CASE(8)
+#undef MOE_CAPPED_CASE
     }
-    if (st == MOE_OK) note_launches(1);
+    if (st == MOE_OK) note_launches(2);
     return st;
 }
