@@ -601,30 +601,73 @@ def main():
 
 def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
     """Co-activation statistics on the 1M-token, 8-layer sweep: tokens/s and
-    the fraction of HBM the statistics kernels reach on their input bytes."""
+    the fraction of HBM the statistics kernels reach on their input bytes,
+    for the default counting method and, beside it, for each method alone
+    (shared-memory histograms; the one-hot contraction on the tensor cores),
+    each against its own ceiling."""
     import torch
     from synth import WORKLOADS, make_routing
     w = WORKLOADS["stats_sweep"]
     ids = make_routing(w, seed=seed)
-    hp = pipeline.HotPath(E=w.E, G=1, rpn=1, ids=torch.from_numpy(ids).to(device), gates=None, x=None,
-                          e2r=[], rank_scores=[], rows=False)
+    ids_d = torch.from_numpy(ids).to(device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-    for _ in range(warmup):
-        hp.step()
-    torch.cuda.synchronize()
-    tot = 0.0
+    world = pg.get_world_size() if pg is not None else 1
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
     n = max(steps, 10)
-    for _ in range(n):
-        flush.zero_()                                 # ids (268 MB) exceed L2; flush anyway
-        s = torch.cuda.Event(enable_timing=True)
-        e = torch.cuda.Event(enable_timing=True)
-        s.record()
-        hp.step()
-        e.record()
-        torch.cuda.synchronize()
-        tot += s.elapsed_time(e)
-    ms = reduce_max(tot / n, pg, device)
+
+    def timed(method):
+        prev = cap.coact_stats_method(method)
+        try:
+            hp = pipeline.HotPath(E=w.E, G=1, rpn=1, ids=ids_d, gates=None, x=None, e2r=[], rank_scores=[],
+                                  rows=False)
+            path = cap.coact_stats_path(w.L, w.T, w.k, w.E, True)
+            for _ in range(warmup):
+                hp.step()
+            torch.cuda.synchronize()
+            tot = 0.0
+            for _ in range(n):
+                flush.zero_()                         # ids (268 MB) exceed L2; flush anyway
+                s_ = torch.cuda.Event(enable_timing=True)
+                e_ = torch.cuda.Event(enable_timing=True)
+                s_.record()
+                hp.step()
+                e_.record()
+                torch.cuda.synchronize()
+                tot += s_.elapsed_time(e_)
+            err = int(hp.err.item())
+        finally:
+            cap.coact_stats_method(prev)
+        return reduce_max(tot / n, pg, device), path, hp, err
+
+    def record(ms, path, nbytes):
+        incs = (w.L * w.T * w.k * (w.k + 1) // 2 + (w.L - 1) * w.T * w.k * w.k) / (ms * 1e-3)
+        r = {"ms": ms, "method": path, "tokens_per_s": world * w.L * w.T / (ms * 1e-3),
+             "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm}
+        if path == "tensor":
+            # C_l = X_l X_l^T and M_l = X_l X_{l+1}^T: 2 E^2 T int8 operations each
+            ops = 2.0 * w.E * w.E * w.T * (2 * w.L - 1) / (ms * 1e-3)
+            bf16, kind = tensor_peak()
+            r["tensor_roofline"] = {
+                "bound": "tensor", "achieved": ops / 1e12, "unit": "TOP/s (int8)", "peak": 2 * bf16,
+                "frac": ops / 1e12 / (2 * bf16),
+                "peak_note": "%s bf16 dense %.1f TFLOP/s x 2 (nominal int8 / bf16 ratio 4.5 / 2.25)" % (kind, bf16)}
+        else:
+            # shared memory serves 32 4-byte accesses per clock per SM, so at
+            # most 32 counter increments per clock per SM
+            peak_inc = 32.0 * sms * SM_MAX_MHZ * 1e6
+            r["increments_per_s"] = world * incs
+            r["atomic_roofline"] = {"bound": "shared-memory atomics", "achieved": incs, "unit": "increments/s",
+                                    "peak": peak_inc, "frac": incs / peak_inc,
+                                    "peak_note": "32 per clock per SM x %d SMs x %.0f MHz" % (sms, SM_MAX_MHZ)}
+        return r
+
+    ms, path, hp, err = timed(0)
     nbytes = hp.step_bytes(None).stats
+    methods = {}
+    for name, m in (("histogram", 1), ("tensor", 2)):
+        ms_m, path_m, _, err_m = timed(m)
+        methods[name] = record(ms_m, path_m, nbytes)
+        methods[name]["err"] = err_m
     # what the placements do on this batch: local share, V per token and rank
     # load balance at each rank count (8 ranks per node), placements from a
     # calibration batch
@@ -642,31 +685,10 @@ def run_sweep(cap, pipeline, device, seed, steps, warmup, hbm, pg):
                               "load_cv": [round(float(x.std() / x.mean()), 4) for x in rl]}
         effect["G=%d" % G] = row
     del ids_cal
-    world = pg.get_world_size() if pg is not None else 1
-    incs = (w.L * w.T * w.k * (w.k + 1) // 2 + (w.L - 1) * w.T * w.k * w.k) / (ms * 1e-3)
-    # the unit that bounds this kernel: shared memory serves 32 4-byte accesses
-    # per clock per SM, so at most 32 counter increments per clock per SM
-    sms = torch.cuda.get_device_properties(device).multi_processor_count
-    peak_inc = 32.0 * sms * SM_MAX_MHZ * 1e6
-    path = cap.coact_stats_path(w.L, w.T, w.k, w.E, True)
-    tensor = None
-    if path == "tensor":
-        # C_l = X_l X_l^T and M_l = X_l X_{l+1}^T: 2 E^2 T int8 operations each
-        ops = 2.0 * w.E * w.E * w.T * (2 * w.L - 1) / (ms * 1e-3)
-        bf16, kind = tensor_peak()
-        tensor = {"bound": "tensor", "achieved": ops / 1e12, "unit": "TOP/s (int8)", "peak": 2 * bf16,
-                  "frac": ops / 1e12 / (2 * bf16),
-                  "peak_note": "%s bf16 dense %.1f TFLOP/s x 2 (nominal int8 / bf16 ratio 4.5 / 2.25)" % (kind, bf16)}
-    return {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "L": w.L, "ms": ms, "method": path,
-            "tensor_roofline": tensor,
-            "tokens_per_s": world * w.L * w.T / (ms * 1e-3),
-            "increments_per_s": world * incs,
-            "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
-            "atomic_roofline": {"bound": "shared-memory atomics", "achieved": incs, "unit": "increments/s",
-                                "peak": peak_inc, "frac": incs / peak_inc,
-                                "peak_note": "32 per clock per SM x %d SMs x %.0f MHz" % (sms, SM_MAX_MHZ)},
-            "algorithmic_bytes": nbytes, "err": int(hp.err.item()),
-            "placement_effect": effect}
+    out = {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "L": w.L}
+    out.update(record(ms, path, nbytes))
+    out.update({"methods": methods, "algorithmic_bytes": nbytes, "err": err, "placement_effect": effect})
+    return out
 
 
 def replica_load(hp, w):
