@@ -492,10 +492,13 @@ def main():
     hbm, hbm_kind = peaks()
     value = weak_value(world, sb.dispatch_combine, ms_step)
     kern = {}
+    # the source order computed ahead (forward schedule): src_rank read, perm written
+    presort = bool(getattr(hp, "presort", False))
     bytes_of = {"stats": sb.stats, "plan": sb.plan, "permute": sb.permute, "combine": sb.combine,
-                "shuffle": sb.shuffle, "gates": sb.gates, "reduce": sb.reduce}
+                "shuffle": sb.shuffle, "gates": sb.gates, "reduce": sb.reduce,
+                "sources": (w.L - 1) * 8 * w.T if presort else 0}
     launches_of = {"stats": 1, "plan": w.L, "permute": w.L, "combine": w.L, "shuffle": (w.L - 1) if shuffle else 0,
-                   "gates": w.L, "reduce": w.L}
+                   "gates": w.L, "reduce": w.L, "sources": (w.L - 1) if presort else 0}
     for name, tot_ms in per_kernel.items():
         ms = tot_ms / ev_steps                        # per step
         gbs = bytes_of[name] / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
@@ -549,9 +552,10 @@ def main():
                        "replicas_per_rank": a.replicas,
                        "replica_eps": a.replica_eps if a.replicas else None,
                        "schedule": hp.schedule,
-                       "overlap": (", ".join({"stats": "statistics", "plan": "plans", "shuffle": "shuffle targets"}[c]
+                       "overlap": (", ".join({"stats": "statistics", "plan": "plans", "shuffle": "shuffle targets",
+                                              "sources": "the next layer's source order"}[c]
                                              for c in hp.side_calls) + " on a second stream" +
-                                   ("; its cooperative launches with one block per rank"
+                                   ("; its cooperative launches on fewer blocks than SMs"
                                     if (balanced and "shuffle" in hp.side_calls) or
                                     (a.replicas and a.replica_eps is not None and "plan" in hp.side_calls) else ""))
                                   if hp.overlap else "none",

@@ -8,7 +8,7 @@ import of any entry point raises: there is no fallback.
 
 Entry points (names follow the C ABI without the ``moe_`` prefix):
   coact_stats, coact_stats_method, coact_stats_path, coact_ema,
-  plan_dispatch, plan_dispatch_method, permute, combine, rank_score, shuffle_targets, shuffle_balanced,
+  plan_dispatch, plan_sources, plan_dispatch_method, permute, combine, rank_score, shuffle_targets, shuffle_balanced,
   dispatch_gates, expert_reduce, combine_rows,
   place_replicas, assign_replicas, assign_replicas_capped, plan_dispatch_ranks,
   ep_routes, ep_permute, ep_combine, ep_scatter_rows, ep_exchange_rows (ranks over several devices),
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
             "moe_plan_dispatch_method": ([i], i),
             "moe_cooperative_blocks": ([i], i),
             "moe_plan_dispatch": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
+            "moe_plan_sources": ([P, i, i, P, P, sz, P], i),
+            "moe_plan_dispatch_presorted": ([P, i, i, i, i, i, P, P, ctypes.POINTER(_Plan), P, P, sz, P], i),
             "moe_permute": ([P, i, i, i, i, P, i64, P, P, P], i),
             "moe_combine": ([P, i, i64, i, P, P, i, i, P, i, P, P], i),
             "moe_dispatch_gates": ([P, P, i, i, P, P, P, i64, P, P, P, P], i),
@@ -296,10 +298,22 @@ def plan_dispatch_workspace(T: int, k: int, G: int, with_src_rank: bool) -> int:
     return int(lib().moe_plan_dispatch_workspace(T, k, G, int(bool(with_src_rank))))
 
 
+def plan_sources(src_rank: torch.Tensor, G: int, ws: torch.Tensor, err: torch.Tensor) -> None:
+    """The first step of a plan with source ranks (the tokens' order by source
+    rank) into ws, ahead of plan_dispatch(..., presorted=True) with the same
+    src_rank and ws; err: the plan's device error word."""
+    _dev(src_rank, torch.int32, "src_rank", 1)
+    _dev(ws, torch.uint8, "ws", 1)
+    T = src_rank.shape[0]
+    st = lib().moe_plan_sources(_ptr(src_rank), T, G, _ptr(err), _ptr(ws), ws.numel(), _stream(src_rank))
+    _check("moe_plan_sources", st)
+
+
 def plan_dispatch(ids: torch.Tensor, E: int, G: int, rpn: int, expert_to_rank: torch.Tensor,
                   src_rank: Optional[torch.Tensor] = None, plan: Optional[Plan] = None,
-                  ws: Optional[torch.Tensor] = None) -> Plan:
-    """ids int32 [T][k] (one layer) -> Plan (device tensors; row arrays sized T*k)."""
+                  ws: Optional[torch.Tensor] = None, presorted: bool = False) -> Plan:
+    """ids int32 [T][k] (one layer) -> Plan (device tensors; row arrays sized T*k).
+    presorted: plan_sources already put src_rank's order into ws."""
     _dev(ids, torch.int32, "ids", 2)
     _dev(expert_to_rank, torch.int32, "expert_to_rank", 1)
     if src_rank is not None:
@@ -311,10 +325,13 @@ def plan_dispatch(ids: torch.Tensor, E: int, G: int, rpn: int, expert_to_rank: t
     need = plan_dispatch_workspace(T, k, G, src_rank is not None)
     if ws is None:
         ws = _workspace(dev, "plan").get(need)
+    if presorted and ws is None:
+        raise ValueError("a presorted plan needs the workspace plan_sources filled")
     cs = plan.c_struct()
-    st = lib().moe_plan_dispatch(_ptr(ids), T, k, E, G, rpn, _ptr(expert_to_rank), _ptr(src_rank),
-                                 ctypes.byref(cs), _ptr(plan.err), _ptr(ws), ws.numel(), _stream(ids))
-    _check("moe_plan_dispatch", st)
+    fn = lib().moe_plan_dispatch_presorted if presorted else lib().moe_plan_dispatch
+    st = fn(_ptr(ids), T, k, E, G, rpn, _ptr(expert_to_rank), _ptr(src_rank),
+            ctypes.byref(cs), _ptr(plan.err), _ptr(ws), ws.numel(), _stream(ids))
+    _check("moe_plan_dispatch_presorted" if presorted else "moe_plan_dispatch", st)
     return plan
 
 

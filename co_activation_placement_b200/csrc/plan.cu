@@ -815,12 +815,24 @@ moe_status launch_plan_fused(const int32_t *ids, int T, int E, int G, int rpn, c
 // another); 1: one cooperative launch when the chunk count allows
 std::atomic<int> g_plan_method{0};
 
+// Step 1 alone: the tokens' stable order by source rank, into the workspace.
+// The first kernel starts after everything before it on the stream; the
+// second may start early and waits inside for the first's counts.
+moe_status launch_sources(const int32_t *src_rank, int T, int G, int32_t *err, const PlanWs &w, cudaStream_t s)
+{
+    const int Bs = src_blocks(T);
+    plan_src_count_kernel<<<Bs, kChunk, 0, s>>>(src_rank, T, G, w, err);
+    if (launch_pdl(plan_src_scatter_kernel, dim3(Bs), dim3(kChunk), 0, s, src_rank, T, G, w) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return launch_status();
+}
+
 template <int K, bool PICKS>
 moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const int32_t *e2r, const int32_t *picks,
-                       const int32_t *src_rank, const moe_plan &P, int32_t *err, const PlanWs &w,
+                       const int32_t *src_rank, bool presorted, const moe_plan &P, int32_t *err, const PlanWs &w,
                        cudaStream_t s)
 {
-    if (g_plan_method.load() == 1) {
+    if (g_plan_method.load() == 1 && !presorted) {
         const moe_status fs = launch_plan_fused<K, PICKS>(ids, T, E, G, rpn, e2r, picks, src_rank, P, err, w, s);
         if (fs != MOE_ERR_UNSUPPORTED) return fs;
     }
@@ -830,17 +842,14 @@ moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const i
     // the first kernel starts after everything before the call; each later
     // one may start early (programmatic dependent launch) and waits inside
     // for its predecessor before reading what that one writes
-    if (with_src) {
-        const int Bs = src_blocks(T);
-        plan_src_count_kernel<<<Bs, kChunk, 0, s>>>(src_rank, T, G, w, err);
-        if (launch_pdl(plan_src_scatter_kernel, dim3(Bs), dim3(kChunk), 0, s, src_rank, T, G, w) != cudaSuccess)
-            return MOE_ERR_CUDA;
+    if (with_src && !presorted) {
+        if (launch_sources(src_rank, T, G, err, w, s) != MOE_OK) return MOE_ERR_CUDA;
         launched += 2;
     }
     const int Bc = chunk_blocks(T, G, with_src);
     if (allow_smem(plan_count_kernel<K, PICKS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
     if (allow_smem(plan_scatter_kernel<K, PICKS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
-    if (with_src) {
+    if (with_src && !presorted) {
         if (launch_pdl(plan_count_kernel<K, PICKS>, dim3(Bc), dim3(kChunk), smem, s, ids, T, E, G, rpn, e2r, picks,
                        with_src, w, P, err) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -877,9 +886,10 @@ extern "C" size_t moe_plan_dispatch_workspace(int T, int k, int G, int with_src_
 namespace {
 
 moe_status plan_entry(const int32_t *ids, int T, int k, int E, int G, int rpn, const int32_t *expert_to_rank,
-                      const int32_t *pick_rank, const int32_t *src_rank, const moe_plan *plan, int32_t *err,
-                      void *ws, size_t ws_bytes, cudaStream_t stream)
+                      const int32_t *pick_rank, const int32_t *src_rank, bool presorted, const moe_plan *plan,
+                      int32_t *err, void *ws, size_t ws_bytes, cudaStream_t stream)
 {
+    if (presorted && !src_rank) return MOE_ERR_ARG;
     if (T < 0 || k < 1 || k > 8 || E < k || G < 1 || G > 64 || rpn < 1 || G % rpn != 0) return MOE_ERR_ARG;
     if ((long long)T * k >= (1ll << 31)) return MOE_ERR_ARG;
     if (E > 12 * 1024) return MOE_ERR_UNSUPPORTED;
@@ -898,13 +908,17 @@ moe_status plan_entry(const int32_t *ids, int T, int k, int E, int G, int rpn, c
     PlanWs w;
     const size_t need = carve(ws, T, G, src_rank != nullptr, &w);
     if (!ws || !aligned256(ws) || ws_bytes < need) return MOE_ERR_WORKSPACE;
+    // (a presorted plan keeps the source order moe_plan_sources left in the
+    // workspace; only the header's counters are reset)
     if (cudaMemsetAsync(w.hdr, 0, sizeof(PlanWsHeader), stream) != cudaSuccess) return MOE_ERR_CUDA;
     const int32_t *e2r = expert_to_rank;
     const int32_t *pk = pick_rank;
 #define MOE_PLAN_CASE(KK)                                                                                  \
     case KK:                                                                                               \
-        return pk ? launch_plan<KK, true>(ids, T, E, G, rpn, e2r, pk, src_rank, *plan, err, w, stream)   \
-                  : launch_plan<KK, false>(ids, T, E, G, rpn, e2r, pk, src_rank, *plan, err, w, stream);
+        return pk ? launch_plan<KK, true>(ids, T, E, G, rpn, e2r, pk, src_rank, presorted, *plan, err, w,   \
+                                          stream)                                                          \
+                  : launch_plan<KK, false>(ids, T, E, G, rpn, e2r, pk, src_rank, presorted, *plan, err, w,  \
+                                           stream);
     switch (k) {
         MOE_PLAN_CASE(1)
         MOE_PLAN_CASE(2)
@@ -927,7 +941,33 @@ extern "C" moe_status moe_plan_dispatch(const int32_t *ids, int T, int k, int E,
                                         void *ws, size_t ws_bytes, cudaStream_t stream)
 {
     if (!expert_to_rank) return MOE_ERR_ARG;
-    return plan_entry(ids, T, k, E, G, rpn, expert_to_rank, nullptr, src_rank, plan, err, ws, ws_bytes, stream);
+    return plan_entry(ids, T, k, E, G, rpn, expert_to_rank, nullptr, src_rank, false, plan, err, ws, ws_bytes,
+                      stream);
+}
+
+extern "C" moe_status moe_plan_sources(const int32_t *src_rank, int T, int G, int32_t *err, void *ws,
+                                       size_t ws_bytes, cudaStream_t stream)
+{
+    if (T < 0 || G < 1 || G > 64 || !err) return MOE_ERR_ARG;
+    if (T == 0) return MOE_OK;
+    if (!src_rank) return MOE_ERR_ARG;
+    PlanWs w;
+    const size_t need = carve(ws, T, G, true, &w);
+    if (!ws || !aligned256(ws) || ws_bytes < need) return MOE_ERR_WORKSPACE;
+    if (cudaMemsetAsync(w.hdr, 0, sizeof(PlanWsHeader), stream) != cudaSuccess) return MOE_ERR_CUDA;
+    const moe_status st = launch_sources(src_rank, T, G, err, w, stream);
+    if (st == MOE_OK) note_launches(2);
+    return st;
+}
+
+extern "C" moe_status moe_plan_dispatch_presorted(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                                                  const int32_t *expert_to_rank, const int32_t *src_rank,
+                                                  const moe_plan *plan, int32_t *err,
+                                                  void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!expert_to_rank) return MOE_ERR_ARG;
+    return plan_entry(ids, T, k, E, G, rpn, expert_to_rank, nullptr, src_rank, true, plan, err, ws, ws_bytes,
+                      stream);
 }
 
 extern "C" moe_status moe_plan_dispatch_ranks(const int32_t *ids, int T, int k, int E, int G, int rpn,
@@ -936,5 +976,5 @@ extern "C" moe_status moe_plan_dispatch_ranks(const int32_t *ids, int T, int k, 
                                               void *ws, size_t ws_bytes, cudaStream_t stream)
 {
     if (!pick_rank) return MOE_ERR_ARG;
-    return plan_entry(ids, T, k, E, G, rpn, nullptr, pick_rank, src_rank, plan, err, ws, ws_bytes, stream);
+    return plan_entry(ids, T, k, E, G, rpn, nullptr, pick_rank, src_rank, false, plan, err, ws, ws_bytes, stream);
 }

@@ -105,6 +105,11 @@ class HotPath:
         self.shuffle = len(self.rank_scores) > 0
         self.plans = [cap.Plan.empty(T, k, self.G, dev) for _ in range(L)]
         self.plan_ws = torch.empty(max(cap.plan_dispatch_workspace(T, k, self.G, True), 1), dtype=torch.uint8, device=dev)
+        # forward schedule: the next layer's source order (a counting sort of
+        # the shuffle targets) is computed beside the rows, into that layer's
+        # own plan workspace, so its plan on the critical path skips it
+        self.presort = (self.schedule == "forward" and self.shuffle and not self.replicas and L > 1)
+        self.plan_ws_l = [torch.empty_like(self.plan_ws) for _ in range(L)] if self.presort else []
         d = self.x.shape[1]
         self.send = torch.empty((T * k, d), dtype=self.x.dtype, device=dev)
         self.outs = [torch.empty((T, d), dtype=self.out_dtype, device=dev) for _ in range(L)]
@@ -159,7 +164,8 @@ class HotPath:
     @property
     def side_calls(self):
         """The calls that run on the second stream, beside the row traffic."""
-        return {"overlap": ("stats", "plan", "shuffle"), "forward": ("stats", "shuffle"), "inline": ()}[self.schedule]
+        return {"overlap": ("stats", "plan", "shuffle"), "forward": ("stats", "shuffle", "sources"),
+                "inline": ()}[self.schedule]
 
     def _coop(self, fn, name):
         """Run a call that makes a cooperative launch; beside the row traffic
@@ -203,9 +209,18 @@ class HotPath:
                 cap.plan_dispatch_ranks(self.ids[l], self.E, self.G, self.rpn, self.pick_rank, src_rank=src,
                                         plan=self.plans[l], ws=self.plan_ws)
             self._call("plan", go)
+        elif self.presort and src is not None:
+            self._call("plan", lambda: cap.plan_dispatch(self.ids[l], self.E, self.G, self.rpn, self.e2r[l],
+                                                         src_rank=src, plan=self.plans[l], ws=self.plan_ws_l[l],
+                                                         presorted=True))
         else:
             self._call("plan", lambda: cap.plan_dispatch(self.ids[l], self.E, self.G, self.rpn, self.e2r[l],
                                                          src_rank=src, plan=self.plans[l], ws=self.plan_ws))
+
+    def _sources(self, l):
+        """Layer l's source order from layer l - 1's shuffle targets."""
+        self._call("sources", lambda: cap.plan_sources(self.targets[l - 1], self.G, self.plan_ws_l[l],
+                                                        self.plans[l].err))
 
     def _rows(self, l):
         p = self.plans[l]
@@ -267,6 +282,8 @@ class HotPath:
                     self.side.wait_event(self.plan_ev[l])
                     with torch.cuda.stream(self.side):
                         self._shuffle(l)
+                        if self.presort:
+                            self._sources(l + 1)
                         self.shuffle_ev[l].record(self.side)
                 if l == self.L - 1:
                     self.side.wait_event(self.plan_ev[l])

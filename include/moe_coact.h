@@ -162,6 +162,27 @@ typedef struct {
  * T*k < 2^31.  Data errors: MOE_DERR_ID_RANGE, MOE_DERR_ID_REPEAT,
  * MOE_DERR_RANK_RANGE. */
 size_t moe_plan_dispatch_workspace(int T, int k, int G, int with_src_rank);
+/* The plan with source ranks in two calls.  moe_plan_sources computes its
+ * first step alone -- the tokens' stable order by source rank, a counting
+ * sort of src_rank -- into ws (moe_plan_dispatch_workspace(T, k, G, 1)
+ * bytes); moe_plan_dispatch_presorted then takes the same arguments as
+ * moe_plan_dispatch (src_rank not NULL) and the same workspace, and runs the
+ * rest.  The result is moe_plan_dispatch's.  The source order depends only on
+ * src_rank, so it can be computed as soon as the source ranks exist (the
+ * previous layer's shuffle targets), on another stream, ahead of the layer's
+ * routing; the caller orders the two calls (same stream, or an event) and
+ * keeps the workspace for this plan in between.  moe_plan_sources: T >= 0,
+ * 1 <= G <= 64, src_rank device int32 [T] (values outside [0, G) are
+ * reported as MOE_DERR_RANK_RANGE in err and counted as rank 0, as by
+ * moe_plan_dispatch).  moe_plan_dispatch_presorted does not re-read src_rank
+ * and always launches separate kernels (moe_plan_dispatch_method does not
+ * apply). */
+moe_status moe_plan_sources(const int32_t *src_rank, int T, int G, int32_t *err, void *ws, size_t ws_bytes,
+                            cudaStream_t stream);
+moe_status moe_plan_dispatch_presorted(const int32_t *ids, int T, int k, int E, int G, int rpn,
+                                       const int32_t *expert_to_rank, const int32_t *src_rank,
+                                       const moe_plan *plan, int32_t *err,
+                                       void *ws, size_t ws_bytes, cudaStream_t stream);
 /* How the plan is launched (process-wide; returns the previous setting, or -1
  * for an invalid argument): 0 = default: separate kernels (counting sort by
  * source, counts, scatter), each of which runs beside other work on the GPU

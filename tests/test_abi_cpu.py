@@ -126,6 +126,12 @@ def test_argument_errors_return_before_device_work(cap):
     assert L.moe_plan_dispatch(fake, 64, 2, 8, 65, 1, fake, None, ctypes.byref(pl), fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
     assert L.moe_plan_dispatch(fake, 64, 2, 8, 8, 3, fake, None, ctypes.byref(pl), fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
     assert L.moe_plan_dispatch(fake, 63, 2, 8, 8, 8, fake, None, ctypes.byref(pl), fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
+    # the plan in two calls: no source ranks, G out of range, a short workspace
+    assert L.moe_plan_dispatch_presorted(fake, 64, 2, 8, 8, 8, fake, None, ctypes.byref(pl), fake, fake, 1 << 20,
+                                         None) == cap.MOE_ERR_ARG
+    assert L.moe_plan_sources(None, 64, 8, fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
+    assert L.moe_plan_sources(fake, 64, 65, fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
+    assert L.moe_plan_sources(fake, 4096, 8, fake, fake, 64, None) == cap.MOE_ERR_WORKSPACE
     # misaligned rows / unsupported row size / bad dtype
     assert L.moe_permute(P(264), cap.MOE_BF16, 4, 8, 2, fake, 8, fake, fake, None) == cap.MOE_ERR_ARG
     assert L.moe_permute(fake, cap.MOE_BF16, 4, 7, 2, fake, 8, fake, fake, None) == cap.MOE_ERR_UNSUPPORTED

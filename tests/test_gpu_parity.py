@@ -157,6 +157,34 @@ def test_plan_small(cap, shape, method):
     check_plan(p, orc.plan(ids, E, G, rpn, e2r, src_rank=src), T, k)
 
 
+@pytest.mark.parametrize("shape", [s_ for s_ in PLAN_SHAPES if s_[5] is not None] +
+                         [(131072, 8, 256, 64, 8, "rand"), (65536, 6, 64, 32, 8, "skew")])
+def test_plan_presorted(cap, shape):
+    """The plan in two calls -- the source order first (moe_plan_sources, on a
+    second stream ordered by an event), then moe_plan_dispatch_presorted --
+    equals the one-call plan and the oracle bit for bit."""
+    T, k, E, G, rpn, mode = shape
+    rng = np.random.default_rng(T + 3 * k + E + G)
+    ids = clustered_ids(rng, 1, T, E, k)[0]
+    e2r = rng.permutation(orc.place_uniform(E, G)).astype(np.int32)
+    src = make_src(rng, mode, T, G)
+    ids_d, e2r_d, src_d = dev(ids), dev(e2r), dev(src)
+    ws = torch.empty(cap.plan_dispatch_workspace(T, k, G, True), dtype=torch.uint8, device="cuda")
+    p = cap.Plan.empty(T, k, G, ids_d.device)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        cap.plan_sources(src_d, G, ws, p.err)
+        ev = torch.cuda.Event()
+        ev.record(side)
+    torch.cuda.current_stream().wait_event(ev)
+    cap.plan_dispatch(ids_d, E, G, rpn, e2r_d, src_rank=src_d, plan=p, ws=ws, presorted=True)
+    check_plan(p, orc.plan(ids, E, G, rpn, e2r, src_rank=src), T, k)
+    q = cap.plan_dispatch(ids_d, E, G, rpn, e2r_d, src_rank=src_d)
+    for a, b in ((p.row_of, q.row_of), (p.offsets, q.offsets), (p.summary, q.summary)):
+        assert (host(a) == host(b)).all()
+
+
 @pytest.mark.parametrize("T,G,mode", [(131072, 64, "rand"), (524288, 64, None), (16384, 8, "skew"), (262144, 32, "rand")])
 def test_plan_single_launch_large(cap, T, G, mode):
     """The single-launch plan where blocks loop over several chunks (more
