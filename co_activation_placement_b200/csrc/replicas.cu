@@ -526,12 +526,15 @@ assign_capped_kernel(CapArgs a)
         // (no rank is open-and-closed yet: every replica is usable), which
         // the launch before this one wrote; count them
         if (rd == 0)
-            for (int t = lo + tid; t < hi; t += kCapThreads)
+            for (int t0 = lo; t0 < hi; t0 += kCapThreads) {
+                const int t = t0 + tid;
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
-                    const int r = __ldcg(a.pick + (size_t)t * K + j);
-                    if (r >= 0) atomicAdd(&hist[r], 1);
+                    const int r = t < hi ? __ldcg(a.pick + (size_t)t * K + j) : -1;
+                    const unsigned same = __match_any_sync(0xffffffffu, r);
+                    if (r >= 0 && lane == __ffs(same) - 1) atomicAdd(&hist[r], __popc(same));
                 }
+            }
         // later rounds: the choices of this block's open tokens whose options
         // changed: a tile of tokens (one per thread) is checked, the changed
         // ones are listed in shared memory, and the warps assign the listed
@@ -641,12 +644,17 @@ assign_capped_kernel(CapArgs a)
         if (ls < tau) {
             for (int r = tid; r < G; r += blockDim.x) rc[r] = 0;
             __syncthreads();
-            for (int t = ls + tid; t < tau; t += blockDim.x)
+            // a warp's lanes on one rank add once (the picks crowd onto the
+            // hot ranks, whose counters would otherwise take them one by one)
+            for (int t0 = ls; t0 < tau; t0 += kCapThreads) {
+                const int t = t0 + tid;
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
-                    const int r = __ldcg(a.pick + (size_t)t * K + j);
-                    if (r >= 0) atomicAdd(&rc[r], 1ull);
+                    const int r = t < tau ? __ldcg(a.pick + (size_t)t * K + j) : -1;
+                    const unsigned same = __match_any_sync(0xffffffffu, r);
+                    if (r >= 0 && lane == __ffs(same) - 1) atomicAdd(&rc[r], (unsigned long long)__popc(same));
                 }
+            }
             __syncthreads();
             for (int r = tid; r < G; r += blockDim.x) {
                 lds[r] += rc[r];
