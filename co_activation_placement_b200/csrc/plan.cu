@@ -195,10 +195,10 @@ plan_src_count_kernel(const int32_t *__restrict__ src_rank, int T, int G, PlanWs
     if (threadIdx.x < G) hist[threadIdx.x] = 0;
     __syncthreads();
     const int t = blockIdx.x * kChunk + threadIdx.x;
-    if (t < T) {
-        const int s = clamp_rank(__ldg(src_rank + t), G, err);
-        atomicAdd(&hist[s], 1);
-    }
+    const int s = t < T ? clamp_rank(__ldg(src_rank + t), G, err) : -1;
+    // one add per rank and warp (shuffle targets crowd onto a few ranks)
+    const unsigned same = __match_any_sync(0xffffffffu, s);
+    if (s >= 0 && (int)(threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[s], __popc(same));
     __syncthreads();
     if (threadIdx.x < G) w.sblk[(size_t)blockIdx.x * G + threadIdx.x] = hist[threadIdx.x];
     __threadfence();

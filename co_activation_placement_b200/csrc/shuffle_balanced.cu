@@ -237,8 +237,11 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
                 }
                 __stcg(a.prop_r + i, my_r);
                 __stcg(a.prop_key + i, my_key);
-                atomicAdd(&cnt_s[my_r], 1);
             }
+            // one add per rank and warp: proposals crowd onto the hot ranks
+            const int cr = mine ? my_r : -1;
+            const unsigned same = __match_any_sync(0xffffffffu, cr);
+            if (cr >= 0 && lane == __ffs(same) - 1) atomicAdd(&cnt_s[cr], __popc(same));
         }
         __syncthreads();
         if (tid < G && cnt_s[tid]) atomicAdd(&h->cnt[p][tid], cnt_s[tid]);
@@ -372,6 +375,7 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
                     for (int u = 0; u < 8; ++u)
                         if (x0 + u * kBalThreads < len && (v[u] & pmask) == prefix)
                             atomicAdd(&hist_s[(v[u] >> shift) & 255u], 1u);
+                }
                 }
                 __syncthreads();
                 if (warp == 0) {
