@@ -376,7 +376,6 @@ __global__ void __launch_bounds__(kBalThreads, 1) shuffle_balanced_kernel(BalArg
                         if (x0 + u * kBalThreads < len && (v[u] & pmask) == prefix)
                             atomicAdd(&hist_s[(v[u] >> shift) & 255u], 1u);
                 }
-                }
                 __syncthreads();
                 if (warp == 0) {
                     // lane l owns digits 255-8l down to 248-8l (descending)
