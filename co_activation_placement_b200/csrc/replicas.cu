@@ -27,8 +27,9 @@
 // running sum over blocks locate the first token tau at which an open rank
 // reaches the cap (a block-wide scan inside the block where that happens);
 // the choices of tokens before tau are final, their tasks join the loads,
-// the ranks at the cap close, and the next round starts at tau.  At most
-// G + 1 rounds of two grid barriers with bounded waits.
+// the ranks at the cap close, and the next round starts at tau.  Every
+// block finds tau and commits by itself from all blocks' counts, so a round
+// takes one grid barrier (bounded wait); at most G + 1 rounds.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -202,11 +203,10 @@ assign_replicas_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int
 // ---- load-capped assignment ---------------------------------------------
 
 constexpr int kCapThreads = 1024;
-constexpr int kCapMaxBlocks = 1024;
+constexpr int kCapMaxBlocks = 256;      // grid limit: every block keeps a [G][blocks] table
 
 struct CapHeader {
     GridBarrier bar;
-    int tau[3];           // first token seeing a newly closed rank (round % 3)
     int rounds;           // rounds run
 };
 
@@ -396,38 +396,6 @@ __device__ __forceinline__ int block_of(int t, int T, int nb)
     return q;
 }
 
-// out[r] += sum over blocks q in [q_lo, q_hi) of blk[q][r], r < G (<= 64):
-// the kCapThreads threads split into kCapThreads / 64 parts over q, eight
-// independent loads in flight per thread, then the parts are added.
-__device__ __forceinline__ void add_block_rows(const int *blk, int G, int q_lo, int q_hi,
-                                               unsigned long long (*red)[64], unsigned long long *out)
-{
-    constexpr int kParts = kCapThreads / 64, kInFlight = 8;
-    const int r = threadIdx.x & 63, part = threadIdx.x / 64;
-    unsigned long long x = 0;
-    if (r < G) {
-        for (int q0 = q_lo + part; q0 < q_hi; q0 += kInFlight * kParts) {
-            unsigned v[kInFlight];
-#pragma unroll
-            for (int u = 0; u < kInFlight; ++u) {
-                const int q = q0 + u * kParts;
-                v[u] = q < q_hi ? (unsigned)__ldcg(blk + (size_t)q * G + r) : 0u;
-            }
-#pragma unroll
-            for (int u = 0; u < kInFlight; ++u) x += v[u];
-        }
-    }
-    red[part][r] = x;
-    __syncthreads();
-    if ((int)threadIdx.x < G) {
-        unsigned long long s = 0;
-#pragma unroll
-        for (int p = 0; p < kParts; ++p) s += red[p][threadIdx.x];
-        out[threadIdx.x] += s;
-    }
-    __syncthreads();
-}
-
 // Block b owns the tokens [T b / nb, T (b + 1) / nb) for the whole launch and
 // keeps, in shared memory, the tasks per rank of its tokens not yet committed
 // (those at or after tc).  A round re-evaluates only the tokens with an
@@ -445,18 +413,19 @@ assign_capped_kernel(CapArgs a)
     int32_t *rep = reinterpret_cast<int32_t *>(uok + E);                                  // [E][max_rep]
     uint32_t *unm = reinterpret_cast<uint32_t *>(rep + E * max_rep);                      // [E]
     int *chg = reinterpret_cast<int *>(unm + E);                                          // [E]
+    int *pre = chg + E;                                                                   // [G][stride]
+    const int stride = nb | 1;                // odd: the transposed writes spread over the banks
     __shared__ int warp_tot[32];
-    __shared__ unsigned long long closed_s;
+    __shared__ unsigned closed_w[2];
     __shared__ unsigned long long lds[64];    // tasks committed per rank (the same in every block)
-    __shared__ unsigned long long base[64];   // tasks per rank before this block's first open token
+    __shared__ unsigned long long tot_s[64];  // open tokens' tasks per rank, all blocks
     __shared__ unsigned long long rc[64];     // tasks per rank of the partly committed block
-    __shared__ unsigned long long red[kCapThreads / 64][64];
     __shared__ int hist[64];                  // this block's uncommitted tasks per rank
     __shared__ int node_of[64];               // rank -> node
+    __shared__ int qx_s[64];                  // first block (from q0) where the rank reaches the cap
     __shared__ int list_s[kCapThreads];       // tokens of a tile to assign
     __shared__ int nlist_s;
-    __shared__ int tau_s, cross_s, tile_tot_s;
-    __shared__ unsigned cross_s2[2];
+    __shared__ int cross_s, tile_tot_s, qmin_s;
 
     for (int e = tid; e < E; e += blockDim.x) {
         const int n = min(max(__ldg(a.nr + e), 0), max_rep);
@@ -469,10 +438,6 @@ assign_capped_kernel(CapArgs a)
             rep[e * max_rep + q] = r;
         }
         uok[e] = 0;
-    }
-    if (b == 0 && tid == 0) {
-        a.h->tau[0] = T;
-        a.h->tau[1] = T;
     }
     if (tid == 0) nlist_s = 0;
     for (int r = tid; r < 64; r += blockDim.x) {
@@ -490,14 +455,12 @@ assign_capped_kernel(CapArgs a)
         const int q0 = block_of(tc, T, nb);             // the block holding tc
         // (a) the closed ranks, each expert's usable replicas, and whether
         // they changed since the last round
-        if (tid == 0) {
-            unsigned long long c = 0;
-            for (int r = 0; r < G; ++r)
-                if ((long long)lds[r] >= a.cap) c |= 1ull << r;
-            closed_s = c;
+        if (tid < 64) {
+            const unsigned bl = __ballot_sync(0xffffffffu, tid < G && (long long)lds[tid] >= a.cap);
+            if (lane == 0) closed_w[warp] = bl;
         }
         __syncthreads();
-        const unsigned long long closed = closed_s;
+        const unsigned long long closed = ((unsigned long long)closed_w[1] << 32) | closed_w[0];
         const unsigned long long closing = closed & ~closed_before;   // ranks closed since the last round
         closed_before = closed;
         for (int e = tid; e < E; e += blockDim.x) {
@@ -578,75 +541,95 @@ assign_capped_kernel(CapArgs a)
         }
         __syncthreads();
         for (int r = tid; r < G; r += blockDim.x) blk[(size_t)b * G + r] = hist[r];
-        // the slot of the next round, last read three rounds ago
-        if (b == 0 && tid == 0) a.h->tau[(rd + 1) % 3] = T;
         if (!grid_barrier(&a.h->bar, a.err)) return;
-        // (c) the loads at this block's first open token; a rank that
-        // reaches the cap inside the block's open tokens gives the first
-        // token that sees it closed
-        if (hi > tc) {
-            for (int r = tid; r < G; r += blockDim.x) base[r] = lds[r];
-            __syncthreads();
-            add_block_rows(blk, G, q0, b, red, base);
-            const int first = max(lo, tc);
-            if (tid < 64) {                      // the open ranks whose cap falls in this block
-                bool x = false;
-                if (tid < G && !((closed >> tid) & 1ull)) {
-                    const long long b0 = (long long)base[tid];
-                    x = b0 < a.cap && b0 + hist[tid] >= a.cap;
+        // (c) every block alike, from all blocks' counts: per rank the running
+        // sum over the blocks with open tokens (q0 on, in token order), the
+        // first block in which an open rank reaches the cap, the token inside
+        // it at which that happens (tau - 1), and the commit of the tokens
+        // before tau in this block's copy of the loads.  One grid barrier a
+        // round: the counts are double-buffered by round, and the picks read
+        // here (tokens before tau) are final.
+        const int nq = nb - q0;                       // blocks with open tokens
+        for (int i = tid; i < nq * G; i += blockDim.x) {
+            const int q = i / G, r = i - q * G;
+            pre[r * stride + q] = __ldcg(blk + (size_t)(q0 + q) * G + r);
+        }
+        __syncthreads();
+        for (int r = warp; r < G; r += kCapThreads / 32) {
+            // exclusive running sums in place; the first block where the
+            // committed tasks plus the running sum reach the cap
+            const bool open = (long long)lds[r] < a.cap;
+            const long long need = a.cap - (long long)lds[r];
+            long long run = 0;
+            int qx = nq;
+            for (int c0 = 0; c0 < nq; c0 += 32) {
+                const int q = c0 + lane;
+                const int v = q < nq ? pre[r * stride + q] : 0;
+                long long incl = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
                 }
-                const unsigned bl = __ballot_sync(0xffffffffu, x);
-                if (lane == 0) cross_s2[warp] = bl;
+                if (q < nq) pre[r * stride + q] = (int)(run + incl - v);
+                const unsigned hit = __ballot_sync(0xffffffffu, open && q < nq && run + incl >= need);
+                if (qx == nq && hit) qx = c0 + __ffs(hit) - 1;
+                run += __shfl_sync(0xffffffffu, incl, 31);
             }
+            if (lane == 0) {
+                qx_s[r] = qx;
+                tot_s[r] = (unsigned long long)run;
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int m = nq;
+            if (lane < G) m = min(m, qx_s[lane]);
+            if (lane + 32 < G) m = min(m, qx_s[lane + 32]);
+            m = (int)__reduce_min_sync(0xffffffffu, (unsigned)m);
+            if (lane == 0) qmin_s = m;
+        }
+        __syncthreads();
+        const int qm = qmin_s;
+        int tau = T;
+        if (qm < nq) {
+            const int qb = q0 + qm;                   // the block holding the first crossing
+            const int first = max((int)((long long)T * qb / nb), tc);
+            const int last = (int)((long long)T * (qb + 1) / nb);
+            if (tid == 0) cross_s = last;
             __syncthreads();
-            const unsigned long long xm = ((unsigned long long)cross_s2[1] << 32) | cross_s2[0];
-            for (unsigned long long mr = xm; mr; mr &= mr - 1ull) {
-                const int r = __ffsll((long long)mr) - 1;
-                const long long b0 = (long long)base[r];
-                // the crossing lies in [first, hi): scan the block's tokens in order
-                const long long need = a.cap - b0;          // tasks on r that reach the cap
+            for (int r = 0; r < G; ++r) {
+                if (qx_s[r] != qm) continue;
+                // tasks on r that reach the cap inside block qb
+                const long long need = a.cap - (long long)lds[r] - pre[r * stride + qm];
+                const int upto = cross_s;             // no later crossing can matter
                 long long run = 0;
-                if (tid == 0) cross_s = -1;
-                __syncthreads();
-                for (int t0 = first; t0 < hi; t0 += blockDim.x) {
+                for (int t0 = first; t0 < upto; t0 += blockDim.x) {
                     const int t = t0 + tid;
                     int c = 0;
-                    if (t < hi) {
+                    if (t < upto) {
 #pragma unroll
                         for (int j = 0; j < K; ++j) c += __ldcg(a.pick + (size_t)t * K + j) == r;
                     }
                     const int incl = block_scan_incl(c, warp_tot);
                     // the one token whose tasks on r take the running count to need
-                    if (t < hi && run + incl >= need && run + incl - c < need) cross_s = t;
+                    const bool at = t < upto && run + incl >= need && run + incl - c < need;
+                    if (at) atomicMin(&cross_s, t);
                     if (tid == (int)blockDim.x - 1) tile_tot_s = incl;
                     __syncthreads();
-                    const bool found = cross_s >= 0;
+                    const bool found = __syncthreads_or(at) != 0;
                     run += tile_tot_s;
-                    __syncthreads();
                     if (found) break;
                 }
-                if (tid == 0 && cross_s >= 0) atomicMin(&a.h->tau[rd % 3], cross_s + 1);
                 __syncthreads();
             }
-        }
-        if (!grid_barrier(&a.h->bar, a.err)) return;
-        // (d) commit the tokens before tau: every block adds, in its own copy
-        // of the loads, the counts of the blocks whose open tokens all
-        // precede tau and recounts the one block that holds tau (no third
-        // barrier: the counts are double-buffered by round, tau kept in three
-        // slots)
-        if (tid == 0) tau_s = __ldcg(&a.h->tau[rd % 3]);
-        __syncthreads();
-        const int tau = tau_s;
-        const int qs = tau < T ? block_of(tau, T, nb) : nb;   // blocks [q0, qs) commit whole
-        add_block_rows(blk, G, q0, qs, red, lds);
-        const int ls = qs < nb ? max((int)((long long)T * qs / nb), tc) : T;
-        if (ls < tau) {
+            tau = cross_s + 1;
+            // commit: the whole blocks before qb, and qb's tokens before tau
+            // (a warp's lanes on one rank add once: the picks crowd onto the
+            // hot ranks)
             for (int r = tid; r < G; r += blockDim.x) rc[r] = 0;
             __syncthreads();
-            // a warp's lanes on one rank add once (the picks crowd onto the
-            // hot ranks, whose counters would otherwise take them one by one)
-            for (int t0 = ls; t0 < tau; t0 += kCapThreads) {
+            for (int t0 = first; t0 < tau; t0 += kCapThreads) {
                 const int t = t0 + tid;
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
@@ -657,9 +640,11 @@ assign_capped_kernel(CapArgs a)
             }
             __syncthreads();
             for (int r = tid; r < G; r += blockDim.x) {
-                lds[r] += rc[r];
-                if (b == qs) hist[r] -= (int)rc[r];
+                lds[r] += (unsigned long long)pre[r * stride + qm] + rc[r];
+                if (b == qb) hist[r] -= (int)rc[r];
             }
+        } else {
+            for (int r = tid; r < G; r += blockDim.x) lds[r] += tot_s[r];   // no rank closes: all final
         }
         if (hi <= tau)
             for (int r = tid; r < G; r += blockDim.x) hist[r] = 0;
@@ -680,15 +665,16 @@ moe_status launch_capped(CapArgs args, cudaStream_t s)
 {
     auto kern = assign_capped_kernel<K>;
     const int max_rep = 1 + args.G / args.rpn;
+    const int nb = std::min(coop_grid(), kCapMaxBlocks);
     const size_t smem = sizeof(unsigned long long) * (size_t)args.E +
-                        sizeof(int32_t) * ((size_t)args.E * max_rep + 2 * (size_t)args.E);
+                        sizeof(int32_t) * ((size_t)args.E * max_rep + 2 * (size_t)args.E + (size_t)args.G * (nb | 1));
     if (allow_smem(kern, smem) != cudaSuccess) return MOE_ERR_CUDA;
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCapThreads, smem) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (per_sm < 1) return MOE_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)std::min(coop_grid(), kCapMaxBlocks));   // at most one block per SM: co-resident
+    cfg.gridDim = dim3((unsigned)nb);        // at most one block per SM: co-resident
     cfg.blockDim = dim3(kCapThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
@@ -759,7 +745,9 @@ extern "C" moe_status moe_assign_replicas_capped(const int32_t *ids, int T, int 
     if (T < 0 || k < 1 || k > 8 || E < k || G < 1 || G > 64 || rpn < 1 || G % rpn != 0 || !err) return MOE_ERR_ARG;
     if (!(eps >= 0.0)) return MOE_ERR_ARG;
     if (G / rpn > kMaxNodes) return MOE_ERR_UNSUPPORTED;
-    if ((size_t)E * (G / rpn + 3) * sizeof(int32_t) + (size_t)E * 8 > 200 * 1024) return MOE_ERR_UNSUPPORTED;
+    if ((size_t)E * (G / rpn + 3) * sizeof(int32_t) + (size_t)E * 8 +
+            (size_t)G * (std::min(coop_grid(), kCapMaxBlocks) | 1) * sizeof(int32_t) > 200 * 1024)
+        return MOE_ERR_UNSUPPORTED;
     if (!src_rank && T % G != 0) return MOE_ERR_ARG;
     if (T == 0) {
         if (rank_load && cudaMemsetAsync(rank_load, 0, sizeof(long long) * G, stream) != cudaSuccess)
