@@ -84,6 +84,9 @@ def parse():
     ap.add_argument("--no-overlap", action="store_true",
                     help="run plans, shuffle targets and statistics in line instead of on a second stream "
                          "(the same as --schedule inline)")
+    ap.add_argument("--row-chunks", type=int, default=1, metavar="C",
+                    help="pipeline each layer's permute and combine over C token chunks (the combine of a chunk "
+                         "beside the permute of the next); the per-kernel times then overlap")
     ap.add_argument("--schedule", default=None, choices=["overlap", "forward", "inline"],
                     help="overlap (default): all control work ahead on a second stream; forward: the order of a "
                          "forward pass, each layer's plan in line before its rows, shuffle targets and statistics "
@@ -384,7 +387,7 @@ def main():
                           scales=make_expert_scales(w, seed=seed) if a.prereduce else None,
                           replica_extra=a.replicas, shuffle_capacity=w.T // w.G if balanced else 0,
                           overlap=not a.no_overlap, replica_eps=a.replica_eps,
-                          schedule="inline" if a.no_overlap else a.schedule)
+                          schedule="inline" if a.no_overlap else a.schedule, row_chunks=a.row_chunks)
     place = time_placement(cap, ids_cal, w, a.placement, device)
 
     def barrier():
@@ -497,7 +500,9 @@ def main():
     bytes_of = {"stats": sb.stats, "plan": sb.plan, "permute": sb.permute, "combine": sb.combine,
                 "shuffle": sb.shuffle, "gates": sb.gates, "reduce": sb.reduce,
                 "sources": (w.L - 1) * 8 * w.T if presort else 0}
-    launches_of = {"stats": 1, "plan": w.L, "permute": w.L, "combine": w.L, "shuffle": (w.L - 1) if shuffle else 0,
+    rc = getattr(hp, "row_chunks", 1)
+    launches_of = {"stats": 1, "plan": w.L, "permute": w.L * rc, "combine": w.L * rc,
+                   "shuffle": (w.L - 1) if shuffle else 0,
                    "gates": w.L, "reduce": w.L, "sources": (w.L - 1) if presort else 0}
     for name, tot_ms in per_kernel.items():
         ms = tot_ms / ev_steps                        # per step
@@ -552,6 +557,7 @@ def main():
                        "replicas_per_rank": a.replicas,
                        "replica_eps": a.replica_eps if a.replicas else None,
                        "schedule": hp.schedule,
+                       "row_chunks": hp.row_chunks,
                        "overlap": (", ".join({"stats": "statistics", "plan": "plans", "shuffle": "shuffle targets",
                                               "sources": "the next layer's source order"}[c]
                                              for c in hp.side_calls) + " on a second stream" +

@@ -81,6 +81,11 @@ class HotPath:
     # blocks for the shuffle, 32, 96 and 148 for the assignment were slower)
     side_coop_blocks: Optional[int] = None
     side_priority: int = 0             # priority of the second stream (lower = higher priority)
+    # > 1: a layer's permute and combine pipelined over this many token
+    # chunks (the combine of chunk c beside the permute of chunk c + 1: a
+    # token's combine reads only that token's rows), mixing the permute's
+    # writes with the combine's reads in HBM; not with the pre-reduced combine
+    row_chunks: int = 1
     # buffers
     stats: dict = field(default_factory=dict)
     plans: List[cap.Plan] = field(default_factory=list)
@@ -124,6 +129,11 @@ class HotPath:
         if self.schedule not in ("overlap", "forward", "inline"):
             raise ValueError("schedule must be overlap, forward or inline")
         self.overlap = self.schedule != "inline"
+        if self.prereduce or self.row_chunks < 1:
+            self.row_chunks = 1
+        if self.row_chunks > 1:
+            self.comb_stream = torch.cuda.Stream(device=dev)
+            self.chunk_ev = [torch.cuda.Event() for _ in range(self.row_chunks)]
         if self.overlap:
             self.side = torch.cuda.Stream(device=dev, priority=self.side_priority)
             self.fork_ev = torch.cuda.Event()
@@ -224,6 +234,25 @@ class HotPath:
 
     def _rows(self, l):
         p = self.plans[l]
+        if self.row_chunks > 1 and not self.prereduce:
+            # chunk c's combine waits only for chunk c's permute; the next
+            # layer's permute (which rewrites the send buffer) waits for all
+            main = torch.cuda.current_stream(self.ids.device)
+            C, T = self.row_chunks, self.T
+            b = [T * c // C for c in range(C + 1)]
+            for c in range(C):
+                t0, t1 = b[c], b[c + 1]
+                self._call("permute", lambda: cap.permute(self.x[t0:t1], p.row_of[t0:t1], p.R_max, send=self.send,
+                                                          err=self.err))
+                self.chunk_ev[c].record(main)
+            for c in range(C):
+                t0, t1 = b[c], b[c + 1]
+                self.comb_stream.wait_event(self.chunk_ev[c])
+                with torch.cuda.stream(self.comb_stream):
+                    self._call("combine", lambda: cap.combine(self.send, p.row_of[t0:t1], self.gates[l][t0:t1],
+                                                              out=self.outs[l][t0:t1], err=self.err))
+            main.wait_stream(self.comb_stream)
+            return
         self._call("permute", lambda: cap.permute(self.x, p.row_of, p.R_max, send=self.send, err=self.err))
         if self.prereduce:
             # gates travel with the rows; the receiving rank applies its
@@ -405,7 +434,8 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
             x_dtype: str, ids_cal: np.ndarray, placement: str = "correlated", shuffle: bool = True,
             out_dtype=torch.bfloat16, device="cuda", rows: bool = True, timers: bool = False,
             scales: Optional[np.ndarray] = None, replica_extra: int = 0, shuffle_capacity: int = 0,
-            overlap: bool = True, replica_eps: Optional[float] = None, schedule: Optional[str] = None) -> HotPath:
+            overlap: bool = True, replica_eps: Optional[float] = None, schedule: Optional[str] = None,
+            row_chunks: int = 1) -> HotPath:
     """Upload a batch (host numpy arrays; x as float32 or bf16 bit patterns)
     and its calibration batch, calibrate, and return the step's HotPath."""
     dev = torch.device(device)
@@ -423,6 +453,7 @@ def prepare(E: int, G: int, rpn: int, ids: np.ndarray, gates: Optional[np.ndarra
     return HotPath(E=E, G=G, rpn=rpn, ids=ids_d, gates=gates_d, x=x_d, e2r=e2r, rank_scores=rs,
                    out_dtype=out_dtype, rows=rows, timers=timers, prereduce=scales is not None, scales=scales_d,
                    replicas=reps, shuffle_capacity=shuffle_capacity, overlap=overlap, schedule=schedule,
+                   row_chunks=row_chunks,
                    replica_eps=replica_eps if replica_extra > 0 else None)
 
 

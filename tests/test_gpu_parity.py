@@ -478,17 +478,19 @@ def test_pipeline_capacity_placement(cap, name, placement):
 def test_overlapped_step_equals_serial_step(cap, name):
     """The step with the control work on a second stream -- all of it ahead
     (overlap), or the forward-pass order with only the shuffle targets and
-    statistics beside the rows (forward) -- produces every output bit for bit
-    as the step run in line, also when replayed from a CUDA graph."""
+    statistics beside the rows (forward) -- and with each layer's permute and
+    combine pipelined over token chunks produces every output bit for bit as
+    the step run in line, also when replayed from a CUDA graph."""
     from co_activation_placement_b200 import pipeline
     w = WORKLOADS[name]
     ids = make_routing(w)
     ids_cal = make_routing(w, seed=w.seed + 1)
     gates, x = make_gates(w), make_hidden(w)
     outs = {}
-    for overlap in ("inline", "overlap", "forward"):
+    for overlap in ("inline", "overlap", "forward", "overlap/4", "forward/3"):
+        sched, _, chunks = overlap.partition("/")
         hp = pipeline.prepare(w.E, w.G, w.rpn, ids, gates, x, w.dtype, ids_cal, out_dtype=torch.float32,
-                              schedule=overlap)
+                              schedule=sched, row_chunks=int(chunks or 1))
         hp.step()
         g = hp.capture(2)
         g.replay()
@@ -499,6 +501,6 @@ def test_overlapped_step_equals_serial_step(cap, name):
                          + [host(o).copy() for o in hp.outs])
         del g, hp
         torch.cuda.empty_cache()
-    for sched in ("overlap", "forward"):
+    for sched in ("overlap", "forward", "overlap/4", "forward/3"):
         for a, b in zip(outs["inline"], outs[sched]):
             assert (a.view(np.uint8) == b.view(np.uint8)).all()
