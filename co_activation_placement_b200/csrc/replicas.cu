@@ -3,7 +3,7 @@
 // "Cobalt", "Problem Formulation": a task (t, e) runs on a rank r_t^e holding
 // a replica of e, and the cross-node cost V counts, per token, the distinct
 // nodes other than the source's that its tasks reach; the communication-aware
-// assignment "routes tokens to the fewest remote nodes possible".
+// assignment sends each token to as few remote nodes as it can.
 //
 // Exact per token: with at most 8 nodes, the smallest set S of remote nodes
 // covering the token's experts (those without a replica on the source node) is

@@ -123,7 +123,7 @@ moe_status moe_coact_stats(const int32_t *ids, int L, int T, int k, int E,
                            int32_t *err, void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
- * Deduplicated dispatch plan  ([EC]: "sends each token to each GPU once";
+ * Deduplicated dispatch plan  ([EC]: each token travels to each GPU at most once;
  * [CB] "Problem Formulation": V with node-level deduplication, r_t^e = p(e))
  *
  * Rows are the pairs (t, r) with r in m_t = {p(e) : e in D_t}, i.e. one row
@@ -222,7 +222,7 @@ moe_status moe_plan_dispatch_ranks(const int32_t *ids, int T, int k, int E, int 
 /* ------------------------------------------------------------------------
  * Communication-aware task assignment over replicas  ([CB] "Problem
  * Formulation": V counts the remote nodes a token's tasks reach; the
- * assignment "routes tokens to the fewest remote nodes possible")
+ * assignment sends each token to as few remote nodes as it can)
  *
  * For every token t (source rank s = src_rank[t], or t/(T/G) when NULL; node
  * ns = s / rpn): the smallest set S of nodes other than ns such that every

@@ -36,8 +36,8 @@
 #define ORC_ERR_ARG 1
 #define ORC_ERR_DATA 2
 
-/* A token's D_t is a set of k distinct expert ids in [0, E) ([EC]: "each
- * token is routed to k of these experts").  Returns 1 when valid. */
+/* A token's D_t is a set of k distinct expert ids in [0, E) ([EC], abstract: each
+ * token goes to k of the experts, so its picks are distinct).  Returns 1 when valid. */
 static int token_valid(const int32_t *d, int k, int E)
 {
     for (int a = 0; a < k; ++a) {
@@ -51,7 +51,7 @@ static int token_valid(const int32_t *d, int k, int E)
 /* Co-activation counts, Ochiai similarity and cross-layer transitions.
  *
  * C_l[i][j] = |{t : i in D_t^l and j in D_t^l}|  ([EC]: pairs of experts
- *   "selected together" by a token; [CB] Problem/Stage 1: the number of tokens
+ *   a token picks at once; [CB] Problem/Stage 1: the number of tokens
  *   selecting both experts i and j).  C_l[i][i] = n_i, the expert's load.
  * S_l[i][j] = |A_i & A_j| / sqrt(|A_i| |A_j|) = C_ij / sqrt(C_ii C_jj)
  *   ([CB] "Key Observation": Ochiai over the token sets of two experts);
@@ -412,8 +412,8 @@ static double load_elem(const void *Y, int y_is_bf16, size_t i)
     return (double)((const float *)Y)[i];
 }
 
-/* Weighted combine, the inverse of dispatch ([EC]: dispatch tokens to their
- * experts "and then combine the results"; [CE] footnote 3: the hidden-state
+/* Weighted combine, the inverse of dispatch ([EC]: tokens are dispatched to
+ * their experts and the results combined; [CE] footnote 3: the hidden-state
  * combine): out[t][c] = sum_j w[t][j] * Y[idx[t][j]][c], summed in fp64 in j
  * order. */
 int orc_combine(const void *Y, int y_is_bf16, int64_t R_max, int d, const int32_t *idx,
@@ -687,8 +687,8 @@ int orc_place_replicas(const uint32_t *coact, int E, int G, int rpn, const int32
     return ORC_OK;
 }
 
-/* Communication-aware task assignment of one token ([CB]: tokens are routed
- * "to the fewest remote nodes possible"; V counts, per token, the remote
+/* Communication-aware task assignment of one token ([CB]: each token goes to as
+ * few remote nodes as it can; V counts, per token, the remote
  * nodes its tasks reach).  Token with picks d[0..k) and source rank s (node
  * ns = s / rpn).  A replica of a pick's expert may serve it when its rank is
  * open (bit r of open_ranks), or when none of that expert's replicas is open.
@@ -765,7 +765,7 @@ static int check_replica_table(int E, int G, int max_rep, const int32_t *replica
     return ORC_OK;
 }
 
-/* Every rank open: the assignment of [CB]'s "fewest remote nodes possible"
+/* Every rank open: the assignment of [CB]'s fewest-remote-nodes rule
  * alone.  Requires G/rpn <= 8.  pick_rank [T][k] out; n_remote [T] out (|S|,
  * may be NULL). */
 int orc_assign_replicas(const int32_t *ids, int T, int k, int E, int G, int rpn, const int32_t *replica_rank,

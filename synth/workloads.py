@@ -1,15 +1,15 @@
 """Synthetic routing, gate weights and hidden states for the five workloads.
 
 The pages measure on real routing of trained MoE models (Megatron-LM
-pretraining runs on page 1, "Expert Coupling in MoE Pretraining", abstract;
-GLM-4.5-Air on page 3, Cobalt summary, "Key Observation").  Neither the
-weights nor the data exist here, so these generators stand in for them with
-the structure the pages describe: experts that are "often selected together"
-(clusters of experts chosen jointly by a token) and next-layer experts that
-are predictable from this layer's (cluster persistence across layers), with a
-skewed (Zipf) popularity of clusters.  Page 5 (DODOCO abstract) warns that
-Zipf mock tokens overstate routing imbalance; these are stand-ins, not a
-model of real routing.
+pretraining runs in "Expert Coupling in MoE Pretraining", abstract;
+GLM-4.5-Air in "Cobalt", "Key Observation").  Neither the weights nor the
+data exist here, so these generators stand in for them with the structure
+the pages describe: experts that tokens tend to pick jointly (clusters of
+experts chosen together by a token) and next-layer experts that are
+predictable from this layer's (cluster persistence across layers), with a
+skewed (Zipf) popularity of clusters.  The DODOCO abstract warns that Zipf
+mock tokens overstate routing imbalance; these are stand-ins, not a model of
+real routing.
 
 Recipe (draw order is part of the definition, so both sides of a test see the
 same bits):
