@@ -101,6 +101,12 @@ class HotPath:
         E = self.E
         self.L, self.T, self.k = L, T, k
         self.err = cap.new_err(dev)
+        if self.schedule is None:
+            self.schedule = "overlap" if self.overlap else "inline"
+        if self.schedule not in ("overlap", "forward", "inline"):
+            raise ValueError("schedule must be overlap, forward or inline")
+        self.overlap = self.schedule != "inline"
+        self.presort = False
         self.stats = dict(coact=torch.empty((L, E, E), dtype=torch.uint32, device=dev),
                           ochiai=torch.empty((L, E, E), dtype=torch.float32, device=dev),
                           trans=torch.empty((max(L - 1, 1), E, E), dtype=torch.uint32, device=dev) if L > 1 else None)
@@ -124,11 +130,6 @@ class HotPath:
                                           dtype=torch.uint8, device=dev)
             # rounds and proposals of each balanced shuffle
             self.shuffle_info = torch.zeros((max(L - 1, 1), 6), dtype=torch.int64, device=dev)
-        if self.schedule is None:
-            self.schedule = "overlap" if self.overlap else "inline"
-        if self.schedule not in ("overlap", "forward", "inline"):
-            raise ValueError("schedule must be overlap, forward or inline")
-        self.overlap = self.schedule != "inline"
         if self.prereduce or self.row_chunks < 1:
             self.row_chunks = 1
         if self.row_chunks > 1:
