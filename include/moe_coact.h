@@ -253,9 +253,10 @@ moe_status moe_assign_replicas(const int32_t *ids, int T, int k, int E, int G, i
  * moe_assign_replicas over the open replicas of its experts -- a pick whose
  * expert has no open replica may use all of them (the cap gives way, never
  * the task).  A token can take a rank past the cap by at most k - 1 tasks;
- * eps = inf gives moe_assign_replicas's result.  The kernel reaches the same
- * result with every token in flight at once, in at most G + 1 rounds of one
- * cooperative launch (grid barriers with the library's 2 s bounded wait).
+ * eps = inf gives moe_assign_replicas's result.  The call reaches the same
+ * result with every token in flight at once: the uncapped assignment (the
+ * first round's choices), then at most G + 1 rounds of one cooperative
+ * launch (one grid barrier a round, with the library's 2 s bounded wait).
  * Arguments as moe_assign_replicas, plus: eps >= 0 (else MOE_ERR_ARG);
  * rank_load device int64 [G] out or NULL (tasks per rank after the batch);
  * ws device, moe_assign_replicas_capped_workspace(G) bytes, 256-byte aligned,
@@ -503,7 +504,8 @@ moe_status moe_shuffle_targets(const int32_t *ids, int T, int k, int E, int G,
  *   pair when t has no rank yet and r holds fewer than `capacity` tokens --
  *   the unique stable assignment of tokens to ranks under these orders.  With
  *   capacity >= T it equals moe_shuffle_targets.  Computed by deferred
- *   acceptance in one cooperative kernel (one block per SM).
+ *   acceptance in one cooperative kernel (one block per SM, or as many as
+ *   moe_cooperative_blocks sets; blocks own ranks in turn).
  *   ids device int32 [T][k]; rank_score device uint32 [E][G], E*G <= 16384,
  *   G <= 64, T < 2^27; requires G*capacity >= T (MOE_ERR_ARG otherwise);
  *   target device int32 [T] (out); info device int64 [6] (out, may be NULL):
