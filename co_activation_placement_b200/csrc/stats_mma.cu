@@ -7,7 +7,8 @@
 // layer l) these are the products
 //     C_l = X_l X_l^T,     M_l = X_l X_{l+1}^T,
 // an exact integer contraction over tokens.  Each thread block owns one job
-// (C_l, M_l, or both from one tile of X_l) and one token slice.  Per stage of
+// (C_l, M_l, or both from one tile of X_l; with E <= 128 both products of two
+// consecutive layers, see coact_quad_kernel) and one token slice.  Per stage of
 // 128 tokens eight builder warps write the stage's X tiles into shared
 // memory and arrive on its "full" mbarrier; a ninth warp waits on it, issues
 // tcgen05.mma kind::i8 (u8 x u8 -> s32, M = 128, K = 32 per instruction)
@@ -358,6 +359,189 @@ coact_mma_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *cnt_c, ui
                      : "memory");
 }
 
+// Two consecutive layers per block.  When C_l and M_l fit one N = 256
+// accumulator (E <= 128), a block owning layers la and la + 1 fills all 512
+// tensor-memory columns with the products of both: [C_la | M_la] at columns
+// 0-255 from A = X_la and B = [X_la; X_la+1], [C_la+1 | M_la+1] at 256-511
+// from A = X_la+1 and B = [X_la+1; X_la+2].  A stage then holds the three
+// tiles X_la, X_la+1, X_la+2 one atom apart, each written once, so that the
+// eight layers of a sweep are built 11 times per token instead of 15 (one
+// block a job: X_l for job l and again as the stacked half of job l - 1).
+// Four builder warps per tile (a lane per token of the stage, its row written
+// as in the one-layer kernel) and one MMA warp; one block per SM.
+constexpr int kQuadTiles = 3;
+constexpr int kQuadWarpsPerTile = 4;
+constexpr int kQuadBuildThreads = kQuadTiles * kQuadWarpsPerTile * 32;
+constexpr int kQuadMmaWarp = kQuadBuildThreads / 32;
+constexpr int kQuadThreads = kQuadBuildThreads + 32;
+constexpr int kQuadStages = 4;
+constexpr int kQuadStage = kQuadTiles * kAtom;     // bytes per stage
+
+template <int K>
+__global__ void __launch_bounds__(kQuadThreads, 1)
+coact_quad_kernel(const int32_t *__restrict__ ids, MmaGeom G, uint32_t *cnt_c, uint32_t *cnt_m, int32_t *err)
+{
+    extern __shared__ __align__(1024) uint8_t sm[];
+    __shared__ __align__(8) uint64_t full_bar[kQuadStages], empty_bar[kQuadStages], done_bar;
+    __shared__ uint32_t tmem_base_s;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int job = blockIdx.x / G.S, slice = blockIdx.x % G.S;
+    const int la = 2 * job;
+    const int nt = min(kQuadTiles, G.L - la);          // tiles: layers la .. la + nt - 1
+    const int nj = min(2, G.L - la);                   // C products: layers la .. la + nj - 1
+    const int T = G.T, E = G.E;
+    const int t0 = (int)((long long)T * slice / G.S), t1 = (int)((long long)T * (slice + 1) / G.S);
+    const int nchunks = (t1 - t0 + kTok - 1) / kTok;
+
+    for (int i = tid * 16; i < kQuadStages * kQuadStage; i += kQuadThreads * 16)
+        *reinterpret_cast<uint4 *>(sm + i) = make_uint4(0, 0, 0, 0);
+    if (tid == 0) {
+        for (int q = 0; q < kQuadStages; ++q) {
+            mbar_init(&full_bar[q], kQuadWarpsPerTile * nt);   // one arrival per active builder warp
+            mbar_init(&empty_bar[q], 1);
+        }
+        mbar_init(&done_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kQuadMmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_addr(&tmem_base_s)), "r"((uint32_t)G.cols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = tmem_base_s;
+    bool ok = true;
+
+    if (warp < kQuadMmaWarp) {
+        // ---- builders: warp w writes tile w / 4 (layer la + w / 4), tokens
+        // 32 (w % 4) + lane of the stage; warps of a missing tile sit out
+        const int tt = warp / kQuadWarpsPerTile;
+        if (tt < nt) {
+            const int u = (warp % kQuadWarpsPerTile) * 32 + lane;
+            const int nch = (E + 15) >> 4;
+            const int32_t *lay = ids + (size_t)(la + tt) * T * K;
+            int cur_v[K], n1_v[K], n2_v[K];
+            auto fetch = [&](int c, int (&v)[K]) {
+                const int t = t0 + c * kTok + u;
+                if (c < nchunks && t < t1) load_k<K>(lay + (size_t)t * K, v);
+            };
+            fetch(0, cur_v);
+            fetch(1, n1_v);
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % kQuadStages, n = c / kQuadStages;
+                fetch(c + 2, n2_v);
+                const int t = t0 + c * kTok + u;
+                int bad = 0;
+                if (t < t1) {
+                    bad = token_check<K>(cur_v, E);
+                    if (bad) record_error(err, bad);
+                }
+                const bool set = t < t1 && !bad;
+                if (c >= kQuadStages && !mbar_wait(&empty_bar[s], (n - 1) & 1)) { ok = false; break; }
+                uint8_t *row = sm + s * kQuadStage + tt * kAtom + u * 128;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    if (ch < nch) *reinterpret_cast<uint4 *>(row + (((ch ^ u) & 7) << 4)) = make_uint4(0, 0, 0, 0);
+                if (set) {
+#pragma unroll
+                    for (int j = 0; j < K; ++j) {
+                        const int e = cur_v[j];
+                        row[((((e >> 4) ^ u) & 7) << 4) + (e & 15)] = 1;
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_bar[s]);
+#pragma unroll
+                for (int j = 0; j < K; ++j) { cur_v[j] = n1_v[j]; n1_v[j] = n2_v[j]; }
+            }
+        }
+    } else {
+        // ---- MMA warp: per full stage and k-step of 32 tokens, product j
+        // reads tile j as A and tiles j, j + 1 as the N = 256 operand (N = 128
+        // without layer la + j + 1)
+        constexpr uint32_t idesc1 = idesc_u8_mn(128), idesc2 = idesc_u8_mn(256);
+        const uint32_t base = smem_addr(sm);
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kQuadStages, n = c / kQuadStages;
+            if (!mbar_wait(&full_bar[s], n & 1)) { ok = false; break; }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            if (lane == 0) {
+                const uint32_t a0 = base + s * kQuadStage;
+#pragma unroll
+                for (int ks = 0; ks < kTok / 32; ++ks) {
+                    const uint32_t acc = (c > 0 || ks > 0) ? 1u : 0u;
+                    for (int j = 0; j < nj; ++j) {
+                        const uint64_t d = smem_desc_mn(a0 + (uint32_t)(j * kAtom + ks * 32 * 128));
+                        mma_u8(tmem + (uint32_t)(256 * j), d, d, j + 1 < nt ? idesc2 : idesc1, acc);
+                    }
+                }
+                mma_commit(&empty_bar[s]);
+            }
+            __syncwarp();
+        }
+        if (ok && lane == 0 && nchunks > 0) mma_commit(&done_bar);
+    }
+    if (!ok) record_error(err, MOE_DERR_TIMEOUT);
+
+    // epilogue: warps 0-3 read TMEM lanes 32 w .. 32 w + 31 (rows of every
+    // product) and add each row into its count matrix by a bulk asynchronous
+    // reduction, as in the one-layer kernel
+    if (warp < 4) {
+        bool ready = ok;
+        if (nchunks > 0) ready = mbar_wait(&done_bar, 0) && ready;
+        ready = __all_sync(0xffffffffu, ready);
+        if (!ready && lane == 0) record_error(err, MOE_DERR_TIMEOUT);
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const int pitch = E + 4;
+        const int row = warp * 32 + lane;
+        uint32_t *srow = reinterpret_cast<uint32_t *>(sm) + (size_t)row * pitch;
+        for (int q = 0; ready && nchunks > 0 && q < 2 * nj; ++q) {
+            const int j = q >> 1;
+            const bool is_m = q & 1;
+            if (is_m && j + 1 >= nt) continue;           // no layer la + j + 1
+            const uint32_t col0 = (uint32_t)(256 * j + (is_m ? 128 : 0));
+            uint32_t *dst = (is_m ? cnt_m : cnt_c) + (size_t)(la + j) * E * E;
+            for (int c0 = 0; c0 < E; c0 += 16) {
+                uint32_t r[16];
+                const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + col0 + (uint32_t)c0;
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                    "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                    : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                      "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                      "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                    : "r"(ta));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (row < E) {
+                    uint4 *o = reinterpret_cast<uint4 *>(srow + c0);
+                    o[0] = make_uint4(r[0], r[1], r[2], r[3]);
+                    o[1] = make_uint4(r[4], r[5], r[6], r[7]);
+                    o[2] = make_uint4(r[8], r[9], r[10], r[11]);
+                    o[3] = make_uint4(r[12], r[13], r[14], r[15]);
+                }
+            }
+            if (row < E) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.u32 [%0], [%1], %2;"
+                             ::"l"(dst + (size_t)row * E), "r"(smem_addr(srow)), "r"((uint32_t)(E * 4))
+                             : "memory");
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            }
+        }
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == kQuadMmaWarp)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)G.cols)
+                     : "memory");
+}
+
 // blockIdx.y = product: C of layer y (y < nc), M of layer y - nc otherwise.
 // The counts were summed over the blocks by the bulk reductions; this copies
 // them out and evaluates Ochiai in fp64 (IEEE multiply, square root and
@@ -401,8 +585,18 @@ moe_status launch_mma(const int32_t *ids, const MmaGeom &g, uint32_t *part, int3
 }
 
 template <int K>
+moe_status launch_quad(const int32_t *ids, const MmaGeom &g, uint32_t *part, int32_t *err, cudaStream_t s)
+{
+    const size_t smem = mma_smem_bytes(g);
+    if (allow_smem(coact_quad_kernel<K>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    coact_quad_kernel<K><<<g.J * g.S, kQuadThreads, smem, s>>>(ids, g, part, part + (size_t)g.nc * g.E * g.E, err);
+    return launch_status();
+}
+
+template <int K>
 moe_status launch_mma_rows(const int32_t *ids, const MmaGeom &g, uint32_t *part, int32_t *err, cudaStream_t s)
 {
+    if (g.quad) return launch_quad<K>(ids, g, part, err, s);
     return g.rows == 128 ? launch_mma<K, 128>(ids, g, part, err, s) : launch_mma<K, 256>(ids, g, part, err, s);
 }
 
@@ -421,10 +615,12 @@ bool make_mma_geom(int L, int T, int k, int E, bool want_c, bool want_t, MmaGeom
     if (g.P == 0) return false;
     // C_l and M_l share layer l's tile when both accumulators fit tensor memory
     g.paired = g.nc > 0 && nm > 0 && g.mt == 1 && 2 * g.rows <= 512;
-    g.J = g.paired ? L : g.P;
+    // two consecutive layers' C and M per block (all 512 columns)
+    g.quad = g.paired && g.rows == 128;
+    g.J = g.quad ? (L + 1) / 2 : (g.paired ? L : g.P);
     // paired implies one 128-row tile (2 * mt * E <= 512); its C and M share one
     // N = 2 * rows accumulator; otherwise one product of mt tiles of N = rows
-    const int acc_cols = g.paired ? 2 * g.rows : g.mt * g.rows;
+    const int acc_cols = g.quad ? 4 * g.rows : (g.paired ? 2 * g.rows : g.mt * g.rows);
     int cols = 32;
     while (cols < acc_cols) cols <<= 1;
     g.cols = cols;
@@ -443,7 +639,8 @@ bool make_mma_geom(int L, int T, int k, int E, bool want_c, bool want_t, MmaGeom
 size_t mma_smem_bytes(const MmaGeom &g)
 {
     const bool any_m = g.P > g.nc;
-    const size_t stages = (size_t)kStages * (any_m ? 2 : 1) * g.rows * kTok;
+    const size_t stages = g.quad ? (size_t)kQuadStages * kQuadStage
+                                 : (size_t)kStages * (any_m ? 2 : 1) * g.rows * kTok;
     const size_t staged_rows = (size_t)128 * (g.E + 4) * sizeof(uint32_t);   // the epilogue's rows
     return std::max(stages, staged_rows);
 }

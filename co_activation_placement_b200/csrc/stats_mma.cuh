@@ -17,7 +17,8 @@ struct MmaGeom {
     int nc;      // C products (L, or 0 when only transitions are wanted)
     int P;       // products: C_0..C_{nc-1}, then M_0..M_{L-2} when wanted
     bool paired; // a block computes C_l and M_l together (both accumulators fit)
-    int J;       // jobs per token slice: L when paired, else P (one product each)
+    bool quad;   // a block computes C and M of layers 2j and 2j + 1 (E <= 128)
+    int J;       // jobs per token slice: (L + 1) / 2 when quad, L when paired, else P
     int S;       // token slices per job
     int cols;    // tensor-memory columns per block (a power of two >= mt*E)
 };

@@ -55,7 +55,11 @@ def test_one_block_first(cap):
 
 
 @pytest.mark.parametrize("L,T,k,E", [(2, 300, 3, 32), (3, 1000, 2, 48), (2, 129, 8, 160), (1, 5000, 4, 64),
-                                     (4, 4097, 8, 256), (2, 128, 1, 128), (3, 20000, 6, 96), (2, 1, 2, 32)])
+                                     (4, 4097, 8, 256), (2, 128, 1, 128), (3, 20000, 6, 96), (2, 1, 2, 32),
+                                     # two layers per block: odd L (a last block with one tile), E < 128,
+                                     # slices of one ragged stage and empty slices
+                                     (5, 3001, 8, 128), (8, 2000, 4, 64), (4, 777, 5, 112), (7, 40000, 8, 128),
+                                     (6, 90, 3, 80)])
 def test_shapes(cap, L, T, k, E):
     rng = np.random.default_rng(L * 1000 + T + E)
     ids = np.stack([np.argsort(rng.random((T, E)), axis=1)[:, :k] for _ in range(L)]).astype(np.int32)
