@@ -329,7 +329,7 @@ __device__ __forceinline__ int serving_ranks(const int (&v)[K], const int32_t *e
 }
 
 template <int K, bool PICKS>
-__global__ void __launch_bounds__(kChunk)
+__global__ void __launch_bounds__(kChunk, 2)
 plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
                   const int32_t *__restrict__ e2r_g, const int32_t *__restrict__ picks, bool with_src, PlanWs w,
                   moe_plan P, int32_t *err)
@@ -340,18 +340,22 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
     __shared__ int32_t seg[kChunk];
     __shared__ unsigned long long red[4][kWarps];
     __shared__ ShardTable sh;
+    __shared__ int32_t node_s[64];              // node of each rank (no division per pick)
     __shared__ bool last;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     if (!PICKS)
         for (int e = threadIdx.x; e < E; e += kChunk) e2r[e] = clamp_rank(__ldg(e2r_g + e), G, err);
-    if (threadIdx.x < 64) cnt[threadIdx.x] = 0;
+    if (threadIdx.x < 64) {
+        cnt[threadIdx.x] = 0;
+        node_s[threadIdx.x] = threadIdx.x / rpn;
+    }
     load_shards(sh, G, with_src, w);      // from the source count, two launches back: complete
     __syncthreads();
     pdl_wait();                           // the source permutation
     pdl_release();
 
     const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, sh);
-    unsigned long long my[4] = {0, 0, 0, 0};
+    uint32_t my[4] = {0, 0, 0, 0};             // per token at most 64: warp sums fit 32 bits
     const int p = c.p0 + threadIdx.x;
     unsigned long long m = 0;
     if (c.active && p < c.p1) {
@@ -369,13 +373,13 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
             for (int j = 0; j < K; ++j) {
                 const int r = rk[j];
                 m |= 1ull << r;
-                nodes |= 1ull << (r / rpn);
+                nodes |= 1ull << node_s[r];
                 local += r == c.s;
             }
             my[0] = __popcll(m);
             my[1] = __popcll(m & ~(1ull << c.s));
             my[2] = local;
-            my[3] = __popcll(nodes & ~(1ull << (c.s / rpn)));
+            my[3] = __popcll(nodes & ~(1ull << node_s[c.s]));
         }
         P.dest_mask[t] = m;
     }
@@ -387,8 +391,7 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        unsigned long long x = my[i];
-        for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        const uint32_t x = __reduce_add_sync(0xffffffffu, my[i]);
         if (lane == 0) red[i][wid] = x;
     }
     __syncthreads();
@@ -432,14 +435,106 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
 
 // ---- step 3: stable per-destination ranks and row writes -----------------
 
+// A token's row_of entries (K ints) as whole vectors where the alignment
+// allows: one 16-byte store per 4 picks, else 8-byte, else 4-byte.
+template <int K>
+__device__ __forceinline__ void store_row_of(int32_t *dst, const int (&x)[K], bool vec_ok)
+{
+    if constexpr (K % 4 == 0) {
+        if (vec_ok) {
+#pragma unroll
+            for (int q = 0; q < K / 4; ++q)
+                reinterpret_cast<int4 *>(dst)[q] = make_int4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+            return;
+        }
+    } else if constexpr (K % 2 == 0) {
+        if (vec_ok) {
+#pragma unroll
+            for (int q = 0; q < K / 2; ++q) reinterpret_cast<int2 *>(dst)[q] = make_int2(x[2 * q], x[2 * q + 1]);
+            return;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < K; ++j) dst[j] = x[j];
+}
+
+// The rows of one chunk.  On entry (after a block barrier): thread i holds
+// its token t (act: a position of the chunk), destination set m (0 for an
+// invalid token, whose row_of becomes -1) and serving ranks r; wcnt[w][d] is
+// the exclusive prefix over the block's warps of the rows for rank d,
+// colw[w][d] the lanes of warp w with a row for d, bcnt[d] the chunk's rows
+// for d and base[d] the chunk's first row of rank d.  A row's place in its
+// rank's run is its warp's prefix plus the earlier lanes of the warp that
+// have that rank (stable in token order).  The chunk's rows of rank d fill
+// one run [base[d], base[d] + bcnt[d]) of the output, so they are staged in
+// shared memory in (d, token order) -- thread, pick mask and rank packed in
+// one word -- and copied out with consecutive threads on consecutive rows;
+// row_of goes out per token in whole vectors.
+template <int K>
+__device__ __forceinline__ void write_chunk_rows(int t, bool act, unsigned long long m, const int (&r)[K], int G,
+                                                 const int32_t *base, const int32_t *bcnt, int32_t (*wcnt)[64],
+                                                 uint32_t (*colw)[64], int32_t *boff, int32_t *tok_s,
+                                                 uint32_t *rows_s, const moe_plan &P)
+{
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid < 32) {   // boff[d]: the chunk's rows of ranks below d
+        const int c0 = lane < G ? bcnt[lane] : 0, c1 = lane + 32 < G ? bcnt[lane + 32] : 0;
+        int s0 = c0, s1 = c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v0 = __shfl_up_sync(0xffffffffu, s0, o);
+            const int v1 = __shfl_up_sync(0xffffffffu, s1, o);
+            if (lane >= o) { s0 += v0; s1 += v1; }
+        }
+        const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+        boff[lane] = s0 - c0;
+        boff[lane + 32] = tot0 + s1 - c1;
+        if (lane == 31) boff[64] = tot0 + s1;
+    }
+    tok_s[tid] = t;
+    __syncthreads();
+    int rowj[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) rowj[j] = -1;
+    const unsigned lt = (1u << lane) - 1u;
+    for (unsigned long long q = m; q; q &= q - 1) {
+        const int d = __ffsll((long long)q) - 1;
+        const int within = wcnt[wid][d] + __popc(colw[wid][d] & lt);
+        unsigned jm = 0;
+#pragma unroll
+        for (int j = 0; j < K; ++j)
+            if (r[j] == d) {
+                jm |= 1u << j;
+                rowj[j] = base[d] + within;
+            }
+        rows_s[boff[d] + within] = ((uint32_t)tid << 14) | (jm << 6) | (uint32_t)d;
+    }
+    if (act) {
+        const bool vec_ok = (reinterpret_cast<uintptr_t>(P.row_of) & (K % 4 == 0 ? 15 : 7)) == 0;
+        store_row_of<K>(P.row_of + (size_t)t * K, rowj, vec_ok);
+    }
+    __syncthreads();
+    const int n = boff[64];
+    for (int i = tid; i < n; i += blockDim.x) {
+        const uint32_t v = rows_s[i];
+        const int d = (int)(v & 63u);
+        const int pos = base[d] + (i - boff[d]);
+        P.row_token[pos] = tok_s[v >> 14];
+        P.row_jmask[pos] = (uint8_t)((v >> 6) & 255u);
+    }
+}
+
 template <int K, bool PICKS>
-__global__ void __launch_bounds__(kChunk)
+__global__ void __launch_bounds__(kChunk, 2)
 plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
                     const int32_t *__restrict__ e2r_g, const int32_t *__restrict__ picks, bool with_src, PlanWs w,
                     moe_plan P)
 {
-    extern __shared__ int32_t e2r[];           // [E]
+    extern __shared__ int32_t e2r[];           // [E] (unused with PICKS), then the staged rows
+    uint32_t *rows_s = reinterpret_cast<uint32_t *>(e2r + (PICKS ? 0 : E));   // [kChunk * K]
     __shared__ int32_t base[64];               // first row of this chunk per rank
+    __shared__ int32_t bcnt[64], boff[65];     // the chunk's rows per rank and their exclusive prefix
+    __shared__ int32_t tok_s[kChunk];
     __shared__ int32_t wcnt[kWarps][64];       // rows per (warp, rank), then their exclusive prefix
     __shared__ uint32_t colw[kWarps][64];      // lanes of the warp with a row for the rank
     __shared__ ShardTable sh;
@@ -464,16 +559,13 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
     const int p = c.p0 + threadIdx.x;
     const bool act = p < c.p1;
     int t = 0, v[K], r[K];
-    unsigned long long m = 0;
-    bool bad = false;
+    unsigned long long m = 0;             // stays 0 for an invalid token: its row_of is all -1
     if (act) {
         t = with_src ? __ldcg(w.perm + p) : p;
         load_token<K>(ids + (size_t)t * K, v);
         if (token_error<K>(v, E) == 0 && serving_ranks<K, PICKS>(v, e2r, picks, t, G, r) == 0) {
 #pragma unroll
             for (int j = 0; j < K; ++j) m |= 1ull << r[j];
-        } else {
-            bad = true;
         }
     }
     // column d of the warp's 32 x G destination bit matrix: which lanes send to rank d
@@ -495,30 +587,13 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
             wcnt[q][threadIdx.x] = run;
             run += x;
         }
+        bcnt[threadIdx.x] = run;
     }
     pdl_wait();                           // the counts, offsets and chunk prefixes
     if (threadIdx.x < G)
         base[threadIdx.x] = __ldcg(P.offsets + threadIdx.x * G) + __ldcg(w.blk_pref + (size_t)blockIdx.x * G + threadIdx.x);
-    if (bad) {
-#pragma unroll
-        for (int j = 0; j < K; ++j) P.row_of[(size_t)t * K + j] = -1;
-    }
     __syncthreads();
-    // each lane writes its own rows: rank within the warp = earlier lanes with that rank
-    const unsigned lt = (1u << lane) - 1u;
-    for (unsigned long long q = m; q; q &= q - 1) {
-        const int d = __ffsll((long long)q) - 1;
-        const int pos = base[d] + wcnt[wid][d] + __popc(colw[wid][d] & lt);
-        unsigned jm = 0;
-#pragma unroll
-        for (int j = 0; j < K; ++j)
-            if (r[j] == d) {
-                jm |= 1u << j;
-                P.row_of[(size_t)t * K + j] = pos;
-            }
-        P.row_token[pos] = t;
-        P.row_jmask[pos] = (uint8_t)jm;
-    }
+    write_chunk_rows<K>(t, act, m, r, G, base, bcnt, wcnt, colw, boff, tok_s, rows_s, P);
 }
 
 // ---- the whole plan in one cooperative launch ------------------------------
@@ -566,8 +641,12 @@ template <int K, bool PICKS>
 __global__ void __launch_bounds__(kChunk, 1)
 plan_fused_kernel(FusedArgs a)
 {
-    extern __shared__ int32_t e2r[];           // [E] (unused with PICKS)
+    extern __shared__ int32_t e2r[];           // [E] (unused with PICKS), then the staged rows
+    uint32_t *rows_s = reinterpret_cast<uint32_t *>(e2r + (PICKS ? 0 : a.E));   // [kChunk * K]
     __shared__ int32_t cnt[64], base[64], tot[64], seg[64];
+    __shared__ int32_t bcnt[64], boff[65];
+    __shared__ int32_t tok_s[kChunk];
+    __shared__ int32_t node_s[64];             // node of each rank (no division per pick)
     __shared__ int32_t part[kChunk];
     __shared__ int32_t wcnt[kWarps][64];       // rows per (warp, rank), then their exclusive prefix
     __shared__ uint32_t colw[kWarps][64];      // lanes of the warp with a row for the rank
@@ -579,6 +658,7 @@ plan_fused_kernel(FusedArgs a)
     GridBarrier *bar = &a.w.hdr->bar;
     if (!PICKS)
         for (int e = tid; e < E; e += kChunk) e2r[e] = clamp_rank(__ldg(a.e2r_g + e), G, a.err);
+    if (tid < 64) node_s[tid] = tid / a.rpn;
 
     // ---- step 1 (source ranks given): counting sort of the tokens by s_t
     if (with_src) {
@@ -659,13 +739,13 @@ plan_fused_kernel(FusedArgs a)
                 for (int j = 0; j < K; ++j) {
                     const int r = rk[j];
                     m |= 1ull << r;
-                    nodes |= 1ull << (r / a.rpn);
+                    nodes |= 1ull << node_s[r];
                     local += r == c.s;
                 }
                 my[0] += __popcll(m);
                 my[1] += __popcll(m & ~(1ull << c.s));
                 my[2] += local;
-                my[3] += __popcll(nodes & ~(1ull << (c.s / a.rpn)));
+                my[3] += __popcll(nodes & ~(1ull << node_s[c.s]));
             }
             a.P.dest_mask[t] = m;
         }
@@ -730,9 +810,6 @@ plan_fused_kernel(FusedArgs a)
             if (token_error<K>(v, E) == 0 && serving_ranks<K, PICKS>(v, e2r, a.picks, t, G, r) == 0) {
 #pragma unroll
                 for (int j = 0; j < K; ++j) m |= 1ull << r[j];
-            } else {
-#pragma unroll
-                for (int j = 0; j < K; ++j) a.P.row_of[(size_t)t * K + j] = -1;
             }
         }
         const uint32_t clo = warp_transpose32((uint32_t)m, lane);
@@ -753,22 +830,10 @@ plan_fused_kernel(FusedArgs a)
                 wcnt[q][tid] = run;
                 run += x;
             }
+            bcnt[tid] = run;
         }
         __syncthreads();
-        const unsigned lt = (1u << lane) - 1u;
-        for (unsigned long long q = m; q; q &= q - 1) {
-            const int d = __ffsll((long long)q) - 1;
-            const int pos = base[d] + wcnt[wid][d] + __popc(colw[wid][d] & lt);
-            unsigned jm = 0;
-#pragma unroll
-            for (int j = 0; j < K; ++j)
-                if (r[j] == d) {
-                    jm |= 1u << j;
-                    a.P.row_of[(size_t)t * K + j] = pos;
-                }
-            a.P.row_token[pos] = t;
-            a.P.row_jmask[pos] = (uint8_t)jm;
-        }
+        write_chunk_rows<K>(t, act, m, r, G, base, bcnt, wcnt, colw, boff, tok_s, rows_s, a.P);
         __syncthreads();
     }
 }
@@ -785,7 +850,7 @@ moe_status launch_plan_fused(const int32_t *ids, int T, int E, int G, int rpn, c
     const int Bc = chunk_blocks(T, G, with_src);
     if (Bc > kFusedMaxChunks || Bs > kFusedMaxChunks) return MOE_ERR_UNSUPPORTED;
     auto kern = plan_fused_kernel<K, PICKS>;
-    const size_t smem = PICKS ? 0 : sizeof(int32_t) * (size_t)E;
+    const size_t smem = sizeof(int32_t) * ((PICKS ? 0 : (size_t)E) + (size_t)kChunk * K);
     if (allow_smem(kern, smem) != cudaSuccess) return MOE_ERR_CUDA;
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kChunk, smem) != cudaSuccess) return MOE_ERR_CUDA;
@@ -847,8 +912,9 @@ moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const i
         launched += 2;
     }
     const int Bc = chunk_blocks(T, G, with_src);
+    const size_t smem_sc = smem + sizeof(int32_t) * (size_t)kChunk * K;     // plus the staged rows
     if (allow_smem(plan_count_kernel<K, PICKS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
-    if (allow_smem(plan_scatter_kernel<K, PICKS>, smem) != cudaSuccess) return MOE_ERR_CUDA;
+    if (allow_smem(plan_scatter_kernel<K, PICKS>, smem_sc) != cudaSuccess) return MOE_ERR_CUDA;
     if (with_src && !presorted) {
         if (launch_pdl(plan_count_kernel<K, PICKS>, dim3(Bc), dim3(kChunk), smem, s, ids, T, E, G, rpn, e2r, picks,
                        with_src, w, P, err) != cudaSuccess)
@@ -856,8 +922,8 @@ moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const i
     } else {
         plan_count_kernel<K, PICKS><<<Bc, kChunk, smem, s>>>(ids, T, E, G, rpn, e2r, picks, with_src, w, P, err);
     }
-    if (launch_pdl(plan_scatter_kernel<K, PICKS>, dim3(Bc), dim3(kChunk), smem, s, ids, T, E, G, e2r, picks, with_src,
-                   w, P) != cudaSuccess)
+    if (launch_pdl(plan_scatter_kernel<K, PICKS>, dim3(Bc), dim3(kChunk), smem_sc, s, ids, T, E, G, e2r, picks,
+                   with_src, w, P) != cudaSuccess)
         return MOE_ERR_CUDA;
     launched += 2;
     moe_status st = launch_status();
