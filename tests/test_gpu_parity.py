@@ -202,6 +202,32 @@ def test_plan_single_launch_large(cap, T, G, mode):
     check_plan(p, orc.plan(ids, E, G, 8, e2r, src_rank=src), T, k)
 
 
+@pytest.mark.parametrize("method", [0, 1])
+@pytest.mark.parametrize("T,k,G,shift", [(3000, 8, 64, 1), (3000, 8, 64, 2), (2048, 6, 32, 1), (2048, 6, 32, 2),
+                                         (999, 5, 8, 1)])
+def test_plan_row_of_alignment(cap, T, k, G, shift, method):
+    """row_of in a caller's buffer that is not 16-byte (shift 1: not 8-byte)
+    aligned: the plan writes a token's entries with narrower stores, same
+    values as the oracle."""
+    E = 4 * G
+    rng = np.random.default_rng(T + 7 * k + shift)
+    ids = clustered_ids(rng, 1, T, E, k)[0]
+    e2r = rng.permutation(orc.place_uniform(E, G)).astype(np.int32)
+    src = make_src(rng, "rand", T, G)
+    p = cap.Plan.empty(T, k, G, "cuda")
+    buf = torch.full((T * k + 4,), -7, dtype=torch.int32, device="cuda")
+    p.row_of = buf[shift:shift + T * k].view(T, k)
+    assert p.row_of.data_ptr() % 16 != 0
+    prev = cap.plan_dispatch_method(method)
+    try:
+        cap.plan_dispatch(dev(ids), E, G, 8 if G % 8 == 0 else 1, dev(e2r), src_rank=dev(src), plan=p)
+    finally:
+        cap.plan_dispatch_method(prev)
+    check_plan(p, orc.plan(ids, E, G, 8 if G % 8 == 0 else 1, e2r, src_rank=src), T, k)
+    b = host(buf)
+    assert (b[:shift] == -7).all() and (b[shift + T * k:] == -7).all()
+
+
 def test_plan_reuses_workspace_and_buffers(cap):
     # the same Plan and workspace reused across calls of different sizes
     rng = np.random.default_rng(5)
