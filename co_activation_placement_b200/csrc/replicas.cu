@@ -203,6 +203,7 @@ assign_replicas_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int
 // ---- load-capped assignment ---------------------------------------------
 
 constexpr int kCapThreads = 1024;
+constexpr size_t kCapSetSmem = 160 * 1024;   // dynamic shared memory allowed with the pick-rank sets
 constexpr int kCapMaxBlocks = 256;      // grid limit: every block keeps a [G][blocks] table
 
 struct CapHeader {
@@ -220,6 +221,7 @@ struct CapArgs {
     CapHeader *h;
     int *blk;                 // [2][gridDim.x][G] tasks per rank of each block's tokens (round parity)
     int32_t *err;
+    int cache_tok;            // tokens per block whose pick-rank sets live in shared memory (0: none)
 };
 
 // x's bits deposited, lowest first, onto the set bits of mask (<= 8 of them).
@@ -268,7 +270,8 @@ __device__ __forceinline__ TokenIn load_token(int t, const CapArgs &a, int rd)
 template <int K>
 __device__ __forceinline__ void assign_token_warp(const TokenIn &x, const CapArgs &a, int rd, int max_rep,
                                                   const int32_t *rep, const int *node_of, const uint32_t *unm,
-                                                  const unsigned long long *uok, int *hist)
+                                                  const unsigned long long *uok, int *hist,
+                                                  unsigned long long *pm_s, int lo)
 {
     const int lane = threadIdx.x & 31;
     constexpr unsigned kAll = 0xffffffffu, kPicks = (1u << K) - 1u;
@@ -359,6 +362,12 @@ __device__ __forceinline__ void assign_token_warp(const TokenIn &x, const CapArg
         if (!bad) atomicAdd(&hist[pick], 1);
     }
     if (lane == 0 && a.nrem) a.nrem[t] = bad ? -1 : pop;
+    if (pm_s) {   // the block's copy of the token's pick-rank set
+        const unsigned long long bit = (lane < K && !bad) ? 1ull << pick : 0ull;
+        const unsigned lo32 = __reduce_or_sync(kAll, (unsigned)bit);
+        const unsigned hi32 = __reduce_or_sync(kAll, (unsigned)(bit >> 32));
+        if (lane == 0) pm_s[t - lo] = ((unsigned long long)hi32 << 32) | lo32;
+    }
 }
 
 // Inclusive block-wide sum scan of one value per thread (kCapThreads).
@@ -415,17 +424,25 @@ assign_capped_kernel(CapArgs a)
     int *chg = reinterpret_cast<int *>(unm + E);                                          // [E]
     int *pre = chg + E;                                                                   // [G][stride]
     const int stride = nb | 1;                // odd: the transposed writes spread over the banks
+    // the ranks of each of this block's tokens' picks as one 64-bit set
+    // (when they fit): a token none of whose picks sits on a rank that just
+    // closed keeps its choice, and the set tells that without global loads
+    const size_t pm_off = ((size_t)E * 8 + 4 * ((size_t)E * max_rep + 2 * (size_t)E + (size_t)G * stride) + 7) &
+                          ~(size_t)7;
+    unsigned long long *pm_s = a.cache_tok ? reinterpret_cast<unsigned long long *>(csm + pm_off) : nullptr;
     __shared__ int warp_tot[32];
     __shared__ unsigned closed_w[2];
     __shared__ unsigned long long lds[64];    // tasks committed per rank (the same in every block)
     __shared__ unsigned long long tot_s[64];  // open tokens' tasks per rank, all blocks
     __shared__ unsigned long long rc[64];     // tasks per rank of the partly committed block
+    __shared__ long long run_s[64];           // a candidate rank's tasks in qb's tokens scanned so far
     __shared__ int hist[64];                  // this block's uncommitted tasks per rank
     __shared__ int node_of[64];               // rank -> node
     __shared__ int qx_s[64];                  // first block (from q0) where the rank reaches the cap
     __shared__ int list_s[kCapThreads];       // tokens of a tile to assign
     __shared__ int nlist_s;
-    __shared__ int cross_s, tile_tot_s, qmin_s;
+    __shared__ int cross_s, qmin_s;
+    __shared__ unsigned long long cand_s;     // the ranks that reach the cap in block q0 + qmin_s
 
     for (int e = tid; e < E; e += blockDim.x) {
         const int n = min(max(__ldg(a.nr + e), 0), max_rep);
@@ -475,7 +492,7 @@ assign_capped_kernel(CapArgs a)
             uint32_t m = 0;
             for (int q = 0; q < max_rep; ++q) {
                 const int r = rep[e * max_rep + q];
-                if (r >= 0 && ((u >> r) & 1ull)) m |= 1u << (r / rpn);
+                if (r >= 0 && ((u >> r) & 1ull)) m |= 1u << node_of[r];
             }
             chg[e] = rd == 0 || u != uok[e];
             any_chg |= chg[e];
@@ -491,12 +508,15 @@ assign_capped_kernel(CapArgs a)
         if (rd == 0)
             for (int t0 = lo; t0 < hi; t0 += kCapThreads) {
                 const int t = t0 + tid;
+                unsigned long long pm = 0;
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
                     const int r = t < hi ? __ldcg(a.pick + (size_t)t * K + j) : -1;
                     const unsigned same = __match_any_sync(0xffffffffu, r);
                     if (r >= 0 && lane == __ffs(same) - 1) atomicAdd(&hist[r], __popc(same));
+                    if (r >= 0) pm |= 1ull << r;
                 }
+                if (pm_s && t < hi) pm_s[t - lo] = pm;
             }
         // later rounds: the choices of this block's open tokens whose options
         // changed: a tile of tokens (one per thread) is checked, the changed
@@ -511,7 +531,7 @@ assign_capped_kernel(CapArgs a)
             // options grow only when an expert's last open replica closes,
             // and that replica was then its pick
             bool dirty = false;
-            if (t < hi) {
+            if (t < hi && (!pm_s || (pm_s[t - lo] & closing) != 0)) {
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
                     const int e = __ldg(a.ids + (size_t)t * K + j);
@@ -532,7 +552,7 @@ assign_capped_kernel(CapArgs a)
             for (int i = warp; i < n; i += kCapThreads / 32) {
                 const int i2 = i + kCapThreads / 32;
                 const TokenIn nxt = load_token<K>(i2 < n ? list_s[i2] : -1, a, rd);
-                assign_token_warp<K>(cur, a, rd, max_rep, rep, node_of, unm, uok, hist);
+                assign_token_warp<K>(cur, a, rd, max_rep, rep, node_of, unm, uok, hist, pm_s, lo);
                 cur = nxt;
             }
             __syncthreads();
@@ -550,9 +570,12 @@ assign_capped_kernel(CapArgs a)
         // round: the counts are double-buffered by round, and the picks read
         // here (tokens before tau) are final.
         const int nq = nb - q0;                       // blocks with open tokens
-        for (int i = tid; i < nq * G; i += blockDim.x) {
-            const int q = i / G, r = i - q * G;
-            pre[r * stride + q] = __ldcg(blk + (size_t)(q0 + q) * G + r);
+        {
+            // thread (qq, r) copies rows qq, qq + P, ... of column r (one
+            // division per thread, not per element)
+            const int P = kCapThreads / G, qq = tid / G, r = tid - qq * G;
+            if (qq < P)
+                for (int q = qq; q < nq; q += P) pre[r * stride + q] = __ldcg(blk + (size_t)(q0 + q) * G + r);
         }
         __syncthreads();
         for (int r = warp; r < G; r += kCapThreads / 32) {
@@ -587,7 +610,13 @@ assign_capped_kernel(CapArgs a)
             if (lane < G) m = min(m, qx_s[lane]);
             if (lane + 32 < G) m = min(m, qx_s[lane + 32]);
             m = (int)__reduce_min_sync(0xffffffffu, (unsigned)m);
-            if (lane == 0) qmin_s = m;
+            // the ranks that reach the cap inside that block
+            const unsigned c0 = __ballot_sync(0xffffffffu, lane < G && qx_s[lane] == m);
+            const unsigned c1 = __ballot_sync(0xffffffffu, lane + 32 < G && qx_s[lane + 32] == m);
+            if (lane == 0) {
+                qmin_s = m;
+                cand_s = ((unsigned long long)c1 << 32) | c0;
+            }
         }
         __syncthreads();
         const int qm = qmin_s;
@@ -596,49 +625,49 @@ assign_capped_kernel(CapArgs a)
             const int qb = q0 + qm;                   // the block holding the first crossing
             const int first = max((int)((long long)T * qb / nb), tc);
             const int last = (int)((long long)T * (qb + 1) / nb);
+            const unsigned long long cand = cand_s;
             if (tid == 0) cross_s = last;
+            for (int r = tid; r < G; r += blockDim.x) {
+                rc[r] = 0;
+                run_s[r] = 0;
+            }
             __syncthreads();
-            for (int r = 0; r < G; ++r) {
-                if (qx_s[r] != qm) continue;
-                // tasks on r that reach the cap inside block qb
-                const long long need = a.cap - (long long)lds[r] - pre[r * stride + qm];
-                const int upto = cross_s;             // no later crossing can matter
-                long long run = 0;
-                for (int t0 = first; t0 < upto; t0 += blockDim.x) {
-                    const int t = t0 + tid;
-                    int c = 0;
-                    if (t < upto) {
+            // one pass over qb's tokens, a tile at a time, the picks loaded
+            // once: per candidate rank the token whose tasks take the rank's
+            // running count to its remaining room (the earliest over the
+            // ranks is the crossing, tau - 1), then the commit of the tile's
+            // tokens before tau (a warp's lanes on one rank add once: the
+            // picks crowd onto the hot ranks)
+            for (int t0 = first; t0 < last; t0 += kCapThreads) {
+                const int t = t0 + tid;
+                int pk[K];
 #pragma unroll
-                        for (int j = 0; j < K; ++j) c += __ldcg(a.pick + (size_t)t * K + j) == r;
-                    }
+                for (int j = 0; j < K; ++j) pk[j] = t < last ? __ldcg(a.pick + (size_t)t * K + j) : -1;
+                for (unsigned long long cm = cand; cm; cm &= cm - 1ull) {
+                    const int r = __ffsll((long long)cm) - 1;
+                    const long long need = a.cap - (long long)lds[r] - pre[r * stride + qm];
+                    int c = 0;
+#pragma unroll
+                    for (int j = 0; j < K; ++j) c += pk[j] == r;
                     const int incl = block_scan_incl(c, warp_tot);
-                    // the one token whose tasks on r take the running count to need
-                    const bool at = t < upto && run + incl >= need && run + incl - c < need;
-                    if (at) atomicMin(&cross_s, t);
-                    if (tid == (int)blockDim.x - 1) tile_tot_s = incl;
+                    const long long run = run_s[r];
+                    if (t < last && run + incl >= need && run + incl - c < need) atomicMin(&cross_s, t);
                     __syncthreads();
-                    const bool found = __syncthreads_or(at) != 0;
-                    run += tile_tot_s;
-                    if (found) break;
+                    if (tid == kCapThreads - 1) run_s[r] = run + incl;
                 }
                 __syncthreads();
-            }
-            tau = cross_s + 1;
-            // commit: the whole blocks before qb, and qb's tokens before tau
-            // (a warp's lanes on one rank add once: the picks crowd onto the
-            // hot ranks)
-            for (int r = tid; r < G; r += blockDim.x) rc[r] = 0;
-            __syncthreads();
-            for (int t0 = first; t0 < tau; t0 += kCapThreads) {
-                const int t = t0 + tid;
+                const int cross = cross_s;
+                const int upto = min(cross + 1, last);
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
-                    const int r = t < tau ? __ldcg(a.pick + (size_t)t * K + j) : -1;
+                    const int r = t < upto ? pk[j] : -1;
                     const unsigned same = __match_any_sync(0xffffffffu, r);
                     if (r >= 0 && lane == __ffs(same) - 1) atomicAdd(&rc[r], (unsigned long long)__popc(same));
                 }
+                if (cross < last) break;              // the same in every thread
             }
             __syncthreads();
+            tau = cross_s + 1;
             for (int r = tid; r < G; r += blockDim.x) {
                 lds[r] += (unsigned long long)pre[r * stride + qm] + rc[r];
                 if (b == qb) hist[r] -= (int)rc[r];
@@ -666,8 +695,16 @@ moe_status launch_capped(CapArgs args, cudaStream_t s)
     auto kern = assign_capped_kernel<K>;
     const int max_rep = 1 + args.G / args.rpn;
     const int nb = std::min(coop_grid(), kCapMaxBlocks);
-    const size_t smem = sizeof(unsigned long long) * (size_t)args.E +
-                        sizeof(int32_t) * ((size_t)args.E * max_rep + 2 * (size_t)args.E + (size_t)args.G * (nb | 1));
+    size_t smem = sizeof(unsigned long long) * (size_t)args.E +
+                  sizeof(int32_t) * ((size_t)args.E * max_rep + 2 * (size_t)args.E + (size_t)args.G * (nb | 1));
+    // the per-token pick-rank sets of a block's tokens, when they fit
+    const size_t tpb = ((size_t)args.T + nb - 1) / nb;
+    const size_t with_sets = round_up(smem, 8) + sizeof(unsigned long long) * tpb;
+    args.cache_tok = 0;
+    if (with_sets <= kCapSetSmem) {
+        args.cache_tok = (int)tpb;
+        smem = with_sets;
+    }
     if (allow_smem(kern, smem) != cudaSuccess) return MOE_ERR_CUDA;
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCapThreads, smem) != cudaSuccess)
