@@ -588,10 +588,10 @@ assign_capped_kernel(CapArgs a)
             for (int c0 = 0; c0 < nq; c0 += 32) {
                 const int q = c0 + lane;
                 const int v = q < nq ? pre[r * stride + q] : 0;
-                long long incl = v;
+                int incl = v;                         // 32 blocks' tasks: at most T k < 2^31
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
-                    const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
                     if (lane >= o) incl += y;
                 }
                 if (q < nq) pre[r * stride + q] = (int)(run + incl - v);
@@ -780,7 +780,7 @@ extern "C" moe_status moe_assign_replicas_capped(const int32_t *ids, int T, int 
                                                  void *ws, size_t ws_bytes, cudaStream_t stream)
 {
     if (T < 0 || k < 1 || k > 8 || E < k || G < 1 || G > 64 || rpn < 1 || G % rpn != 0 || !err) return MOE_ERR_ARG;
-    if (!(eps >= 0.0)) return MOE_ERR_ARG;
+    if (!(eps >= 0.0) || (long long)T * k >= (1ll << 31)) return MOE_ERR_ARG;   // task counts are int32
     if (G / rpn > kMaxNodes) return MOE_ERR_UNSUPPORTED;
     if ((size_t)E * (G / rpn + 3) * sizeof(int32_t) + (size_t)E * 8 +
             (size_t)G * (std::min(coop_grid(), kCapMaxBlocks) | 1) * sizeof(int32_t) > 200 * 1024)

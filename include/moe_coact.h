@@ -261,10 +261,12 @@ moe_status moe_assign_replicas(const int32_t *ids, int T, int k, int E, int G, i
  * rank_load device int64 [G] out or NULL (tasks per rank after the batch);
  * ws device, moe_assign_replicas_capped_workspace(G) bytes, 256-byte aligned,
  * caller-owned, overwritten by each call (calls on one workspace must not
- * overlap).  Limits: G <= 64, G/rpn <= 8 nodes, E * (4 (G/rpn + 3) + 8) +
- * 4 G (B | 1) bytes <= 200 KB for a grid of B blocks (one per SM, or
- * moe_cooperative_blocks; else MOE_ERR_UNSUPPORTED).  Data errors as
- * moe_assign_replicas; an invalid token counts for no rank.
+ * overlap).  Limits: T k < 2^31 (else MOE_ERR_ARG), G <= 64, G/rpn <= 8
+ * nodes, E * (4 (G/rpn + 3) + 8) + 4 G (B | 1) bytes <= 200 KB for a grid of
+ * B blocks (one per SM, or moe_cooperative_blocks; else
+ * MOE_ERR_UNSUPPORTED).  When a block's share of the tokens fits, their
+ * pick-rank sets (8 bytes a token) also live in its shared memory.  Data
+ * errors as moe_assign_replicas; an invalid token counts for no rank.
  * ---------------------------------------------------------------------- */
 size_t moe_assign_replicas_capped_workspace(int G);
 moe_status moe_assign_replicas_capped(const int32_t *ids, int T, int k, int E, int G, int rpn,

@@ -161,6 +161,11 @@ def test_argument_errors_return_before_device_work(cap):
     assert L.moe_ep_scatter_rows(fake, 6, 8, fake, 8, 2, fake, 8, fake, None) == cap.MOE_ERR_ARG
     assert L.moe_ep_scatter_rows(P(258), 8, 8, fake, 8, 2, fake, 8, fake, None) == cap.MOE_ERR_ARG
     assert cap.ep_route_len(64, 8) == 2 * 64 * 8 + 2
+    # capped task assignment: eps < 0, T k past int32 task counts
+    assert L.moe_assign_replicas_capped(fake, 64, 2, 8, 8, 8, fake, fake, None, ctypes.c_double(-0.5), fake, None,
+                                        None, fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
+    assert L.moe_assign_replicas_capped(fake, 1 << 28, 8, 64, 8, 8, fake, fake, fake, ctypes.c_double(0.1), fake,
+                                        None, None, fake, fake, 1 << 20, None) == cap.MOE_ERR_ARG
 
 
 @pytest.mark.parametrize("E,G,rpn,extra", [(16, 8, 2, 1), (64, 8, 8, 2), (64, 32, 8, 1), (256, 64, 8, 1), (24, 6, 1, 3)])
