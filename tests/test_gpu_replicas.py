@@ -201,7 +201,9 @@ def test_capped_assignment_random(cap, seed):
 @pytest.mark.parametrize("blocks", [1, 3, 64, 0])
 def test_capped_assignment_grid_sizes(cap, blocks):
     """The result does not depend on the cooperative grid (moe_cooperative_blocks):
-    one block, a few, one per rank, one per SM."""
+    one block, a few, one per rank, one per SM.  With 1 and 3 blocks a block's
+    131,072 / B tokens are too many for their pick-rank sets to sit in shared
+    memory, so those grids also cover the kernel without them."""
     w = WORKLOADS["large_ep64"]
     ids = make_routing(w)[0]
     cal = make_routing(w, seed=1)[0]
