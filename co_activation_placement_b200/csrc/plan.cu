@@ -36,9 +36,8 @@ constexpr int kChunk = 1024;  // tokens per block, one per thread
 constexpr int kWarps = kChunk / 32;
 
 struct PlanWsHeader {
-    unsigned int done_count;      // blocks finished in plan_count
     unsigned int done_src;        // blocks finished in plan_src_count
-    unsigned int pad[2];
+    unsigned int pad[3];
     unsigned long long acc[4];    // R, R_remote, local, V
     GridBarrier bar;              // the single-launch plan's grid barrier
 };
@@ -336,12 +335,9 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
 {
     extern __shared__ int32_t e2r[];           // [E] (unused with PICKS)
     __shared__ int32_t cnt[64];
-    __shared__ int32_t tot[64];
-    __shared__ int32_t seg[kChunk];
     __shared__ unsigned long long red[4][kWarps];
     __shared__ ShardTable sh;
     __shared__ int32_t node_s[64];              // node of each rank (no division per pick)
-    __shared__ bool last;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     if (!PICKS)
         for (int e = threadIdx.x; e < E; e += kChunk) e2r[e] = clamp_rank(__ldg(e2r_g + e), G, err);
@@ -401,15 +397,69 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
         if (x) atomicAdd(&w.hdr->acc[threadIdx.x], x);
     }
     if (threadIdx.x < G) w.blk[(size_t)blockIdx.x * G + threadIdx.x] = cnt[threadIdx.x];
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) last = atomicAdd(&w.hdr->done_count, 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
+}
 
-    // the last block: scan chunk counts, then offsets, counts and summary
-    const int B = with_src ? sh.cpre[G] : gridDim.x;
+// ---- step 3: stable per-destination ranks and row writes -----------------
+
+// The first row of chunk b for every rank, base[d] (shared): the rows of
+// ranks below d, then those of rank d in chunks before b -- both column sums
+// of the [B][G] per-chunk counts, taken in one pass by the whole block
+// (thread (q, d) sums rows q, q + nseg, ... of column d).  Ends with a
+// barrier.
+__device__ __forceinline__ void chunk_bases(const int32_t *blk, int B, int b, int G, int32_t *base, int32_t *ptot,
+                                            int32_t *pbef)
+{
+    const int nseg = blockDim.x / G, d = threadIdx.x % G, q = threadIdx.x / G;
+    if (q < nseg) {
+        int tot = 0, bef = 0;
+        constexpr int kBatch = 8;             // independent L2 loads in flight per thread
+        for (int r0 = q; r0 < B; r0 += kBatch * nseg) {
+            int v[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                const int row = r0 + i * nseg;
+                v[i] = row < B ? __ldcg(blk + (size_t)row * G + d) : 0;
+            }
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                tot += v[i];
+                if (r0 + i * nseg < b) bef += v[i];
+            }
+        }
+        ptot[q * G + d] = tot;
+        pbef[q * G + d] = bef;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        // exclusive prefix over ranks of the totals, plus the rows before b
+        const int lane = threadIdx.x;
+        int t0 = 0, t1 = 0, b0 = 0, b1 = 0;
+        for (int qq = 0; qq < nseg; ++qq) {
+            if (lane < G) { t0 += ptot[qq * G + lane]; b0 += pbef[qq * G + lane]; }
+            if (lane + 32 < G) { t1 += ptot[qq * G + lane + 32]; b1 += pbef[qq * G + lane + 32]; }
+        }
+        int s0 = t0, s1 = t1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y0 = __shfl_up_sync(0xffffffffu, s0, o);
+            const int y1 = __shfl_up_sync(0xffffffffu, s1, o);
+            if (lane >= o) { s0 += y0; s1 += y1; }
+        }
+        const int all0 = __shfl_sync(0xffffffffu, s0, 31);
+        if (lane < G) base[lane] = s0 - t0 + b0;
+        if (lane + 32 < G) base[lane + 32] = all0 + s1 - t1 + b1;
+    }
+    __syncthreads();
+}
+
+// The plan's tables from the per-chunk counts (one block, beside the row
+// writes of the others): the exclusive scan of the counts over chunks per
+// rank, the rank segments, offsets[d][s] (first row of shard s in rank d's
+// segment), counts[s][d], offsets[G*G] = R and the summary.
+template <int K>
+__device__ void write_tables(int B, int G, bool with_src, const ShardTable &sh, const PlanWs &w, const moe_plan &P,
+                             int T, int32_t *tot, int32_t *seg)
+{
     scan_columns(w.blk, w.blk_pref, B, G, tot, seg);
     if (threadIdx.x == 0) {
         int run = 0;
@@ -417,23 +467,19 @@ plan_count_kernel(const int32_t *__restrict__ ids, int T, int E, int G, int rpn,
         P.offsets[G * G] = run;
     }
     __syncthreads();
-    const int nshard = G;
-    for (int i = threadIdx.x; i < G * G; i += kChunk) {
+    for (int i = threadIdx.x; i < G * G; i += blockDim.x) {
         const int d = i / G, s = i % G;   // offsets in (d, s) order
         int b0, b1;
         if (with_src) { b0 = sh.cpre[s]; b1 = sh.cpre[s + 1]; }
-        else { const int nch = B / nshard; b0 = s * nch; b1 = b0 + nch; }
+        else { const int nch = B / G; b0 = s * nch; b1 = b0 + nch; }
         const int a0 = __ldcg(w.blk_pref + (size_t)b0 * G + d);
         const int a1 = __ldcg(w.blk_pref + (size_t)b1 * G + d);
         P.offsets[d * G + s] = seg[d] + a0;
         P.counts[s * G + d] = a1 - a0;
     }
-    if (threadIdx.x < 4) P.summary[threadIdx.x] = (int64_t)atomicAdd(&w.hdr->acc[threadIdx.x], 0ull);
+    if (threadIdx.x < 4) P.summary[threadIdx.x] = (int64_t)__ldcg(&w.hdr->acc[threadIdx.x]);
     if (threadIdx.x == 4) P.summary[4] = (int64_t)T * K;
-    if (threadIdx.x == 0) w.hdr->done_count = 0;
 }
-
-// ---- step 3: stable per-destination ranks and row writes -----------------
 
 // A token's row_of entries (K ints) as whole vectors where the alignment
 // allows: one 16-byte store per 4 picks, else 8-byte, else 4-byte.
@@ -537,6 +583,7 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
     __shared__ int32_t tok_s[kChunk];
     __shared__ int32_t wcnt[kWarps][64];       // rows per (warp, rank), then their exclusive prefix
     __shared__ uint32_t colw[kWarps][64];      // lanes of the warp with a row for the rank
+    __shared__ int32_t part[2][kChunk];        // column sums: per (segment, rank) partials
     __shared__ ShardTable sh;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     // prologue, before the counts are complete: the shard table and the
@@ -544,6 +591,12 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
     // destination sets and their per-warp ranks
     load_shards(sh, G, with_src, w);
     __syncthreads();
+    const int B = gridDim.x - 1;               // chunks; the last block writes the tables
+    if (blockIdx.x == B) {
+        pdl_wait();
+        write_tables<K>(B, G, with_src, sh, w, P, T, &part[0][0], &part[1][0]);
+        return;
+    }
     const ChunkRange c = chunk_range(blockIdx.x, T, G, with_src, sh);
     if (!c.active) {
         pdl_wait();
@@ -589,10 +642,17 @@ plan_scatter_kernel(const int32_t *__restrict__ ids, int T, int E, int G,
         }
         bcnt[threadIdx.x] = run;
     }
-    pdl_wait();                           // the counts, offsets and chunk prefixes
-    if (threadIdx.x < G)
-        base[threadIdx.x] = __ldcg(P.offsets + threadIdx.x * G) + __ldcg(w.blk_pref + (size_t)blockIdx.x * G + threadIdx.x);
-    __syncthreads();
+    // the picks' ranks (< 64) as bytes while the bases are summed: fewer
+    // registers live across that pass
+    uint32_t rpk[(K + 3) / 4];
+#pragma unroll
+    for (int q = 0; q < (K + 3) / 4; ++q) rpk[q] = 0;
+#pragma unroll
+    for (int j = 0; j < K; ++j) rpk[j / 4] |= (m ? (uint32_t)r[j] & 255u : 0u) << (8 * (j % 4));
+    pdl_wait();                           // the per-chunk counts
+    chunk_bases(w.blk, B, blockIdx.x, G, base, &part[0][0], &part[1][0]);
+#pragma unroll
+    for (int j = 0; j < K; ++j) r[j] = (int)((rpk[j / 4] >> (8 * (j % 4))) & 255u);
     write_chunk_rows<K>(t, act, m, r, G, base, bcnt, wcnt, colw, boff, tok_s, rows_s, P);
 }
 
@@ -922,7 +982,7 @@ moe_status launch_plan(const int32_t *ids, int T, int E, int G, int rpn, const i
     } else {
         plan_count_kernel<K, PICKS><<<Bc, kChunk, smem, s>>>(ids, T, E, G, rpn, e2r, picks, with_src, w, P, err);
     }
-    if (launch_pdl(plan_scatter_kernel<K, PICKS>, dim3(Bc), dim3(kChunk), smem_sc, s, ids, T, E, G, e2r, picks,
+    if (launch_pdl(plan_scatter_kernel<K, PICKS>, dim3(Bc + 1), dim3(kChunk), smem_sc, s, ids, T, E, G, e2r, picks,
                    with_src, w, P) != cudaSuccess)
         return MOE_ERR_CUDA;
     launched += 2;
