@@ -12,15 +12,16 @@
 //   2. the token sequence in perm order is cut into chunks of kChunk tokens
 //      that never straddle a source shard.  Each chunk's block computes m_t
 //      (bitmask of destination ranks), the summary terms and its per-rank row
-//      counts; the last block to finish scans the counts over chunks (column
-//      per rank), which yields every chunk's first row per rank, the rank
-//      segment offsets and counts[s][r] (chunks of one shard are adjacent);
-//   3. each chunk's block ranks its rows per destination, stable in perm
-//      order: a warp transposes its 32 x G destination bit matrix with five
-//      shuffle stages, so lane d holds the ballot of rank d; a row's rank in
-//      the warp is a popcount of that word below the lane, and warps are
-//      ordered by a prefix over the block.  It writes row_token, row_jmask and
-//      row_of.
+//      counts;
+//   3. each chunk's block sums the counts of the chunks before it and of all
+//      chunks per rank (its first row per rank), then ranks its rows per
+//      destination, stable in perm order: a warp transposes its 32 x G
+//      destination bit matrix with five shuffle stages, so lane d holds the
+//      ballot of rank d; a row's rank in the warp is a popcount of that word
+//      below the lane, and warps are ordered by a prefix over the block.  It
+//      writes row_token, row_jmask and row_of.  One more block of the same
+//      launch scans the counts over chunks for the rank segment offsets and
+//      counts[s][r] (chunks of one shard are adjacent) and the summary.
 // All arithmetic is integer; the result is unique and does not depend on
 // scheduling.  No kernel waits on another block.
 #include <algorithm>
