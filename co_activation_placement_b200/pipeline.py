@@ -76,9 +76,10 @@ class HotPath:
     schedule: Optional[str] = None
     # blocks of the cooperative launches (balanced shuffle, capped assignment)
     # when they run beside the row traffic.  None: the balanced shuffle takes
-    # min(G, 32) blocks and the capped assignment 64 (the rest of the SMs
+    # min(G, 32) blocks and the capped assignment 48 (the rest of the SMs
     # stream rows; on large_ep64 these gave the shortest steps: 24, 48 and 64
-    # blocks for the shuffle, 32, 96 and 148 for the assignment were slower)
+    # blocks for the shuffle, 64, 96 and 148 for the assignment were slower,
+    # 32 as fast)
     side_coop_blocks: Optional[int] = None
     side_priority: int = 0             # priority of the second stream (lower = higher priority)
     # > 1: a layer's permute and combine pipelined over this many token
@@ -186,7 +187,7 @@ class HotPath:
             return fn()
         n = self.side_coop_blocks
         if n is None:
-            n = min(self.G, 32) if name == "shuffle" else 64
+            n = min(self.G, 32) if name == "shuffle" else 48
         prev = cap.cooperative_blocks(n)
         try:
             return fn()
