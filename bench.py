@@ -47,22 +47,33 @@ FALLBACK_HBM_GBS = 6650.0
 SM_MAX_MHZ = 1965.0            # B200 clocks.max.sm
 
 
-def peaks():
+def measured_peak(key):
+    """A positive number under `key` in MEASURED_PEAKS.json (written per pool:
+    hbm_gbs, bf16_tflops, bf16_tflops_sustained; a value may also sit in a
+    {"value": ...} object), else None: no file, unreadable, or no such key."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
+    if not os.path.exists(p):
+        return None
+    try:
         with open(p) as f:
-            d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return FALLBACK_HBM_GBS, "fallback"
+            v = json.load(f).get(key)
+        if isinstance(v, dict):
+            v = v.get("value")
+        v = float(v)
+    except (OSError, ValueError, TypeError, AttributeError):
+        return None
+    return v if v > 0 else None
+
+
+def peaks():
+    v = measured_peak("hbm_gbs")
+    return (v, "measured") if v is not None else (FALLBACK_HBM_GBS, "fallback")
 
 
 def tensor_peak():
     """Dense bf16 TFLOP/s for a kernel timed alone: the measured burst figure."""
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            return float(json.load(f)["bf16_tflops"]), "measured"
-    return 1590.0, "fallback"
+    v = measured_peak("bf16_tflops")
+    return (v, "measured") if v is not None else (1590.0, "fallback")
 
 
 def parse():

@@ -97,3 +97,19 @@ def test_reference_arm_prints_contract_line(monkeypatch):
     assert line["impl"] == "reference" and line["value"] > 0 and line["higher_is_better"] is True
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["config"]["workload"] == "tiny"
+
+
+def test_measured_peaks_file(monkeypatch, tmp_path):
+    """The roofline denominators come from MEASURED_PEAKS.json when it holds
+    them (plain numbers or {"value": ...}), else the fallbacks."""
+    import json
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.peaks() == (bench.FALLBACK_HBM_GBS, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6559.4, "bf16_tflops": {"value": 1585.0}}))
+    assert bench.peaks() == (6559.4, "measured")
+    assert bench.tensor_peak() == (1585.0, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").write_text("{not json")
+    assert bench.peaks() == (bench.FALLBACK_HBM_GBS, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": None}))
+    assert bench.tensor_peak() == (1590.0, "fallback") and bench.peaks()[1] == "fallback"
