@@ -159,8 +159,10 @@ typedef struct {
  * src_rank       device int32 [T] or NULL; NULL means contiguous shards
  *                s_t = t / (T/G) and then requires G | T
  * Limits: 1 <= k <= 8, k <= E, 1 <= G <= 64, rpn >= 1, G % rpn == 0, T >= 0,
- * T*k < 2^31.  Data errors: MOE_DERR_ID_RANGE, MOE_DERR_ID_REPEAT,
- * MOE_DERR_RANK_RANGE. */
+ * T*k < 2^31 (else MOE_ERR_ARG); E <= 12288 (else MOE_ERR_UNSUPPORTED).  The
+ * plan's arrays need only their element alignment (row_of is written with
+ * wider stores where it is 16- or 8-byte aligned).  Data errors:
+ * MOE_DERR_ID_RANGE, MOE_DERR_ID_REPEAT, MOE_DERR_RANK_RANGE. */
 size_t moe_plan_dispatch_workspace(int T, int k, int G, int with_src_rank);
 /* The plan with source ranks in two calls.  moe_plan_sources computes its
  * first step alone -- the tokens' stable order by source rank, a counting
